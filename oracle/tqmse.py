@@ -1,0 +1,95 @@
+"""TurboQuant-MSE encode of one row per bit-width group, and the record format.
+
+Pages: Block-GTQ abstract / blockgtq README -- the widths chosen by the
+allocator go to the TQ-MSE encoder, and the serving path keeps a packed
+cache of the codes.  TQ-MSE (TurboQuant, arXiv 2504.19874, cited by the
+pages): rotate, normalise, scalar-quantise each rotated coordinate with the
+Lloyd-Max codebook.  Readings used here (the pages give neither):
+
+encode, group g of width b over dims D_g (d = |D_g|):
+    x_g = x[D_g]                       (fp16 input as float64)
+    n   = ||x_g||                      (float64, exact input)
+    y   = Pi_g x_g                     (Pi_g the fp32 table, as float64)
+    u   = sqrt(d) * y / n              (u = 0 when n = 0)
+    code_i = #{fp32 thresholds <= u_i} (ties go up)
+    stored norm = fp16(n), round-to-nearest-even; codes use the unrounded n.
+
+record: the codes of all groups (width-descending, rotated-coordinate order
+inside a group) as one LSB-first bitstream in little-endian 32-bit words;
+code k of width b occupies bits [o_k, o_k + b) with o_k the sum of the
+widths before it.  A record is A * D / 8 bytes for an average of A bits per
+dim -- 48 bytes for D = 128 at 3 bits.
+"""
+import numpy as np
+
+from .lloyd_max import quantise
+
+
+def encode_group(x_rows, dims, rotation, bits):
+    """Codes [n, d] (int64) and norms [n] (float64, unrounded) of one group.
+
+    x_rows: [n, D] float64 (exact fp16 values); rotation: fp32 [d, d].
+    """
+    xg = np.asarray(x_rows, dtype=np.float64)[:, dims]
+    d = len(dims)
+    norms = np.sqrt(np.sum(xg * xg, axis=1))
+    y = xg @ rotation.astype(np.float64).T                 # y = Pi x per row
+    safe = np.where(norms > 0, norms, 1.0)
+    u = np.sqrt(float(d)) * y / safe[:, None]
+    u[norms == 0] = 0.0
+    return quantise(u, bits), norms
+
+
+def fp16_round(values):
+    """Round float64 values to fp16 (numpy rounds to nearest even)."""
+    return np.asarray(values, dtype=np.float64).astype(np.float16)
+
+
+def record_widths(groups):
+    """Per-position widths of a record, in record order."""
+    return np.concatenate([np.full(len(dims), b, dtype=np.int64) for b, dims in groups])
+
+
+def pack_records(codes, widths, record_bytes):
+    """Pack codes [n, P] (record order) with per-position widths [P] into uint8 [n, record_bytes]."""
+    codes = np.asarray(codes, dtype=np.uint64)
+    widths = np.asarray(widths, dtype=np.int64)
+    n, p = codes.shape
+    assert p == len(widths)
+    total_bits = int(np.sum(widths))
+    assert total_bits <= 8 * record_bytes and record_bytes % 4 == 0
+    nwords = record_bytes // 4
+    acc = np.zeros((n, nwords + 1), dtype=np.uint64)
+    offset = 0
+    for k in range(p):
+        b = int(widths[k])
+        if b == 0:
+            continue
+        assert np.all(codes[:, k] < (1 << b))
+        w, sh = offset >> 5, offset & 31
+        val = codes[:, k] << np.uint64(sh)
+        acc[:, w] |= val & np.uint64(0xFFFFFFFF)
+        acc[:, w + 1] |= val >> np.uint64(32)
+        offset += b
+    assert np.all(acc[:, nwords] == 0)
+    words = acc[:, :nwords].astype(np.uint32)
+    return words.astype("<u4").view(np.uint8).reshape(n, record_bytes)
+
+
+def unpack_records(records, widths):
+    """Inverse of pack_records: uint8 [n, record_bytes] -> codes [n, P] int64."""
+    records = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
+    n, nbytes = records.shape
+    words = records.view("<u4").reshape(n, nbytes // 4).astype(np.uint64)
+    words = np.concatenate([words, np.zeros((n, 1), dtype=np.uint64)], axis=1)
+    out = np.zeros((n, len(widths)), dtype=np.int64)
+    offset = 0
+    for k, b in enumerate(widths):
+        b = int(b)
+        if b == 0:
+            continue
+        w, sh = offset >> 5, offset & 31
+        both = words[:, w] | (words[:, w + 1] << np.uint64(32))
+        out[:, k] = ((both >> np.uint64(sh)) & np.uint64((1 << b) - 1)).astype(np.int64)
+        offset += b
+    return out

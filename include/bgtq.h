@@ -1,0 +1,211 @@
+/*
+ * bgtq.h -- C ABI of the Block-GTQ packed KV-cache library for B200 (sm_100a).
+ *
+ * Block-GTQ ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Liang,
+ * Zhang, Jia; arXiv 2606.24033 abstract and the blockgtq README) quantises
+ * the key cache per RoPE 2-D frequency block: a label-free Q/K energy score
+ * per block, greedy integer bit widths by marginal gain under a fixed
+ * average, then the TurboQuant-MSE (TQ-MSE) encoder; a packed-cache serving
+ * path decodes attention straight from the codes.  This library implements
+ * that hot path:
+ *
+ *   bgtq_allocate       energy score per block + greedy allocation + tables
+ *   bgtq_encode_append  rotate, normalise, Lloyd-Max quantise, bit-pack K/V
+ *   bgtq_rotate_query   the query in each width group's rotated basis
+ *   bgtq_decode_attn    one GQA decode step over the packed cache
+ *
+ * Conventions
+ *  - Every function returns 0 (BGTQ_OK) or a negative BGTQ_ERR_* code and
+ *    never throws or aborts.  Argument checks happen before any launch; a
+ *    call that fails its checks launches nothing.
+ *  - Device buffers are owned by the caller (allocated e.g. with torch); the
+ *    library never allocates or frees device memory.  Host memory for the
+ *    tables is owned by the state and freed by bgtq_destroy.
+ *  - "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls marked ASYNC only enqueue work on that stream; calls
+ *    marked SYNC wait for their own work before returning.
+ *  - K and Q arrive after RoPE; the library never applies RoPE.  head_dim
+ *    must be 128 (64 RoPE blocks).  Softmax scale is 1/sqrt(head_dim).
+ *    Query head h reads KV head h / G, G = n_q_heads / n_kv_heads.
+ *  - fp16 tensors are IEEE binary16, row-major, densely packed, 16-byte
+ *    aligned.
+ *
+ * Cache layout inside d_cache (offsets from bgtq_cache_offsets, each
+ * 256-byte aligned; L layers, B = max_batch, H = n_kv_heads, C = capacity):
+ *   K records  uint8 [L][B][H][C][16*k_avg_bits]   LSB-first bitstream of
+ *              the codes in little-endian 32-bit words; width groups in
+ *              descending width, rotated-coordinate order inside a group
+ *   K norms    fp16  [L][B][H][C][4]   slot i = norm of group i (width
+ *              descending); unused slots 0
+ *   V records  uint8 [L][B][H][C][16*v_avg_bits]  same bitstream, one group
+ *   V norms    fp16  [L][B][H][C]
+ */
+#ifndef BGTQ_H
+#define BGTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  BGTQ_OK = 0,
+  BGTQ_ERR_INVALID_ARG = -1,   /* a size, index or config field out of range */
+  BGTQ_ERR_NULL = -2,          /* a required pointer is NULL */
+  BGTQ_ERR_CUDA = -3,          /* a CUDA runtime call failed (launch or copy) */
+  BGTQ_ERR_BUFFER_SIZE = -4,   /* a caller buffer is smaller than required */
+  BGTQ_ERR_NOT_READY = -5,     /* no allocation set yet (allocate/set_allocation first) */
+  BGTQ_ERR_DEVICE = -6,        /* a kernel raised its error flag (see bgtq_get_device_error) */
+  BGTQ_ERR_HOST_ALLOC = -7,    /* host malloc failed */
+  BGTQ_ERR_ALIGNMENT = -8      /* a device pointer is not 16-byte aligned */
+};
+
+/* Device error flag bits, reported by bgtq_get_device_error. */
+enum {
+  BGTQ_DEVERR_CAPACITY = 1,    /* encode_append: start + count > capacity (rows skipped) */
+  BGTQ_DEVERR_SEQ_LEN = 2,     /* decode_attn: a seq_len < 0 or > capacity (sequence skipped, output 0) */
+  BGTQ_DEVERR_ARG = 4          /* encode_append: start < 0 or count < 0 or count > n */
+};
+
+typedef struct {
+  int32_t n_layers;          /* >= 1 */
+  int32_t n_kv_heads;        /* >= 1 */
+  int32_t n_q_heads;         /* multiple of n_kv_heads; G = n_q_heads / n_kv_heads <= 16 */
+  int32_t head_dim;          /* must be 128 */
+  int32_t max_batch;         /* >= 1 */
+  int32_t k_avg_bits;        /* average K bits per dim, 1..4 (record = 16*k bytes) */
+  int32_t v_avg_bits;        /* V bits per dim, 1..4 */
+  int32_t b_min;             /* smallest K width, 0..4 (0: a block may store nothing) */
+  int32_t b_max;             /* largest K width, b_min..4, b_min <= k_avg_bits <= b_max */
+  int32_t rope_pairing;      /* 0: block j = dims (j, j+64) (rotate_half); 1: (2j, 2j+1) */
+  int32_t max_splits;        /* split-K slots per (layer, seq, KV head); 0 = 256 */
+  int32_t reserved;          /* must be 0 */
+  int64_t capacity_tokens;   /* cached tokens per sequence, >= 1 */
+  uint64_t seed;             /* seeds the Haar rotations */
+} bgtq_config;
+
+typedef struct bgtq_state bgtq_state;
+
+/* Bytes of the two caller-owned device buffers for a config.
+ * cache_bytes: the packed K/V cache (layout above).  workspace_bytes: the
+ * device tables plus scratch (energy partial sums, rotated queries, split-K
+ * partials, error flag).  SYNC (host only). */
+int bgtq_required_bytes(const bgtq_config* cfg, size_t* cache_bytes, size_t* workspace_bytes);
+
+/* Creates a state over caller buffers of at least the required sizes (both
+ * 256-byte aligned).  The state keeps the pointers; the buffers must outlive
+ * it.  Uploads the Lloyd-Max codebooks and clears the error flag on
+ * "stream".  No allocation is set: call bgtq_allocate or
+ * bgtq_set_allocation before encoding.  SYNC. */
+int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes,
+                void* d_workspace, size_t workspace_bytes, void* stream, bgtq_state** out);
+
+/* Frees the host-side state (never the caller's device buffers). NULL is a no-op. */
+void bgtq_destroy(bgtq_state* st);
+
+/* Block-GTQ allocation ("for each layer and KV head, computes a label-free
+ * energy score for each RoPE block and greedily allocates integer bit widths
+ * by marginal gain", abstract).  Score of block j: s_j = EQ_j * EK_j with
+ * EQ_j = sum over rows and the G query heads of the group of ||q_j||^2 and
+ * EK_j = sum over rows of ||k_j||^2, accumulated exactly on the GPU (fp16 x
+ * 2^24 is an integer; 128-bit sums).  Greedy: every block starts at b_min;
+ * each step gives one bit to the block with the largest s_j*(Dist(b_j) -
+ * Dist(b_j+1)) below b_max (ties: lowest block), until sum_j b_j =
+ * k_avg_bits * 64.  Dist(b) = N(0,1) Lloyd-Max MSE {1, .363380, .117482,
+ * .034548, .009497}.  Then builds the per-(layer, KV head) group layout and
+ * Haar rotations and uploads them.
+ *   d_calib_q  fp16 [n_layers][nq][n_q_heads][128]
+ *   d_calib_k  fp16 [n_layers][nk][n_kv_heads][128]
+ * nq, nk >= 1.  SYNC (copies the exact sums back, runs the greedy on the host). */
+int bgtq_allocate(bgtq_state* st, const void* d_calib_q, int32_t nq,
+                  const void* d_calib_k, int32_t nk, void* stream);
+
+/* Sets the widths directly (e.g. uniform TQ-MSE: every block = k_avg_bits)
+ * and builds/uploads the tables as bgtq_allocate does.
+ *   h_widths int8 [n_layers][n_kv_heads][64], each in [b_min, b_max],
+ *            each (layer, head) summing to 64 * k_avg_bits.  SYNC. */
+int bgtq_set_allocation(bgtq_state* st, const int8_t* h_widths, void* stream);
+
+/* Copies the current widths out (int8 [n_layers][n_kv_heads][64]). SYNC. */
+int bgtq_get_allocation(const bgtq_state* st, int8_t* h_widths);
+
+/* The exact energies of the last bgtq_allocate as 128-bit integers in units
+ * of 2^-48, little-endian (lo, hi) uint64 pairs:
+ *   h_eq, h_ek  uint64 [n_layers][n_kv_heads][64][2].  SYNC. */
+int bgtq_get_energy(const bgtq_state* st, uint64_t* h_eq, uint64_t* h_ek);
+
+/* The fp32 Lloyd-Max codebook for bits in 1..4 (TurboQuant's scalar
+ * quantiser on N(0,1)): h_centroids[2^bits], h_thresholds[2^bits - 1]. */
+int bgtq_get_codebook(int32_t bits, float* h_centroids, float* h_thresholds);
+
+/* Group layout of (layer, kv_head): *n_groups, per group its width and size
+ * (h_width[4], h_size[4]; unused 0) and h_perm[128] = the original dim at
+ * each record position.  SYNC (host tables). */
+int bgtq_get_layout(const bgtq_state* st, int32_t layer, int32_t kv_head, int32_t* n_groups,
+                    int32_t* h_width, int32_t* h_size, int32_t* h_perm);
+
+/* The fp32 Haar rotation of one group (kind 0 = K, group index 0..n_groups-1)
+ * or of V (kind 1, group ignored), row-major d x d, y = R x.  *d receives
+ * the size; h_out must hold 128*128 floats.  SYNC (host tables). */
+int bgtq_get_rotation(const bgtq_state* st, int32_t layer, int32_t kv_head, int32_t kind,
+                      int32_t group, float* h_out, int32_t* d);
+
+/* Byte offsets of the four cache arrays inside d_cache:
+ * out[0] K records, out[1] K norms, out[2] V records, out[3] V norms. */
+int bgtq_cache_offsets(const bgtq_state* st, size_t* out);
+
+/* TQ-MSE encode + bit-pack of new rows into the cache.  For each layer
+ * l in [layer, layer + layer_count), sequence b < batch, row r < count[b]:
+ * the K and V rows at d_k/d_v[l - layer][b][r][h][:] go to cache position
+ * start[b] + r of (l, b, h).  Per K width group g (dims D_g, d = |D_g|):
+ * n = ||x[D_g]|| (float64), y = R_g x[D_g] (fp32), u = sqrt(d) y / n,
+ * code = #{thresholds <= u}; stored norm = fp16(n).  V: one group of 128.
+ *   d_k, d_v   fp16 [layer_count][batch][n][n_kv_heads][128]
+ *   d_start    int32 [batch]  first cache position written
+ *   d_count    int32 [batch]  rows of this sequence, 0..n
+ * Rows with start + r >= capacity are skipped and set BGTQ_DEVERR_CAPACITY.
+ * ASYNC. */
+int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count,
+                       const void* d_k, const void* d_v, const int32_t* d_start,
+                       const int32_t* d_count, int32_t batch, int32_t n, void* stream);
+
+/* q~ in record order: per K group g, (1/sqrt(128)) (1/sqrt(d_g)) R_g q[D_g].
+ *   d_q     fp16 [layer_count][batch][n_q_heads][128]
+ *   d_qrot  fp32 [layer_count][batch][n_q_heads][128].  ASYNC. */
+int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                      int32_t batch, float* d_qrot, void* stream);
+
+/* One decode step: for each layer in [layer, layer + layer_count), sequence
+ * b < batch and query head h,
+ *   out = sum_t softmax_t(q . k_hat_t / sqrt(128)) v_hat_t over cache
+ *   positions t < seq_lens[b],
+ * taken in the rotated domain (logits from q~ and the codes; V accumulated
+ * in V's rotated basis and rotated back once).  seq_lens[b] = 0 gives 0.
+ *   d_q        fp16 [layer_count][batch][n_q_heads][128]
+ *   d_seq_lens int32 [batch], 0..capacity
+ *   d_out      fp16 [layer_count][batch][n_q_heads][128]
+ * Uses the workspace for q~ and split-K partials, so calls on one state
+ * must not overlap on the GPU.  ASYNC. */
+int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
+
+/* Tokens per split-K chunk for bgtq_decode_attn: 0 = automatic (from
+ * capacity, max_splits and the SM count), else a multiple of 64 with
+ * ceil(capacity / tokens) <= max_splits.  Results do not depend on it beyond
+ * floating-point reassociation. */
+int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens);
+
+/* Synchronises "stream", reads the device error flag into *h_flags
+ * (BGTQ_DEVERR_* bits) and clears it.  SYNC. */
+int bgtq_get_device_error(bgtq_state* st, void* stream, int32_t* h_flags);
+
+/* Static description of a status code. */
+const char* bgtq_error_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BGTQ_H */

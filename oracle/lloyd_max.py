@@ -18,6 +18,7 @@ The codebook is symmetric, so only the positive half is iterated and the
 negative half is its mirror image (which makes the middle threshold 0
 exactly).
 """
+import functools
 import math
 
 import numpy as np
@@ -48,6 +49,7 @@ def _cond_mean(a, b):
     return (_phi(a) - _phi(b)) / (_Phi(b) - _Phi(a))
 
 
+@functools.lru_cache(maxsize=None)
 def positive_centroids(bits, tol=1e-15, max_iter=100000):
     """Positive half of the 2**bits-level Lloyd-Max codebook, ascending, float64.
 
@@ -60,7 +62,7 @@ def positive_centroids(bits, tol=1e-15, max_iter=100000):
         raise ValueError("bits must be in 1..4")
     half = 1 << (bits - 1)
     if half == 1:
-        return [_cond_mean(0.0, math.inf)]          # sqrt(2/pi)
+        return (_cond_mean(0.0, math.inf),)         # sqrt(2/pi)
     c = [(k + 0.5) * 4.0 / half for k in range(half)]
     for _ in range(max_iter):
         t = [0.0] + [0.5 * (c[k] + c[k + 1]) for k in range(half - 1)] + [math.inf]
@@ -69,7 +71,7 @@ def positive_centroids(bits, tol=1e-15, max_iter=100000):
         c = new
         if moved <= tol:
             break
-    return c
+    return tuple(c)
 
 
 def centroids(bits):

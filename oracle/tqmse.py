@@ -25,11 +25,8 @@ import numpy as np
 from .lloyd_max import quantise
 
 
-def encode_group(x_rows, dims, rotation, bits):
-    """Codes [n, d] (int64) and norms [n] (float64, unrounded) of one group.
-
-    x_rows: [n, D] float64 (exact fp16 values); rotation: fp32 [d, d].
-    """
+def rotated_normalised(x_rows, dims, rotation):
+    """(u [n, d], norms [n]) of one group: u = sqrt(d) Pi x / ||x|| (0 for a zero x)."""
     xg = np.asarray(x_rows, dtype=np.float64)[:, dims]
     d = len(dims)
     norms = np.sqrt(np.sum(xg * xg, axis=1))
@@ -37,6 +34,15 @@ def encode_group(x_rows, dims, rotation, bits):
     safe = np.where(norms > 0, norms, 1.0)
     u = np.sqrt(float(d)) * y / safe[:, None]
     u[norms == 0] = 0.0
+    return u, norms
+
+
+def encode_group(x_rows, dims, rotation, bits):
+    """Codes [n, d] (int64) and norms [n] (float64, unrounded) of one group.
+
+    x_rows: [n, D] float64 (exact fp16 values); rotation: fp32 [d, d].
+    """
+    u, norms = rotated_normalised(x_rows, dims, rotation)
     return quantise(u, bits), norms
 
 

@@ -1,0 +1,323 @@
+"""Python binding of the C ABI in include/bgtq.h (ctypes, argument marshalling only).
+
+Every ``bgtq_*`` function here calls the function of the same name in the
+in-tree ``libbgtq.so``; nothing is computed in Python.  ``PackedKVCache``
+owns the two device buffers (torch tensors) and one library state.
+
+The library must be built (``python -m packed_decode_attention_b200.build``
+or ``__graft_entry__.build()``); importing the binding without it raises.
+"""
+import ctypes
+import os
+from dataclasses import dataclass, fields
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbgtq.so")
+
+HEAD_DIM = 128
+N_BLOCKS = HEAD_DIM // 2
+
+DEVERR_CAPACITY = 1
+DEVERR_SEQ_LEN = 2
+DEVERR_ARG = 4
+DEVERR_NONFINITE = 8
+
+
+class BgtqError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"bgtq status {status}: {message}")
+        self.status = status
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [
+        ("n_layers", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("max_batch", ctypes.c_int32),
+        ("k_avg_bits", ctypes.c_int32),
+        ("v_avg_bits", ctypes.c_int32),
+        ("b_min", ctypes.c_int32),
+        ("b_max", ctypes.c_int32),
+        ("rope_pairing", ctypes.c_int32),
+        ("max_splits", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("capacity_tokens", ctypes.c_int64),
+        ("seed", ctypes.c_uint64),
+    ]
+
+
+@dataclass
+class Config:
+    """Mirror of bgtq_config."""
+    n_layers: int
+    n_kv_heads: int
+    n_q_heads: int
+    max_batch: int
+    capacity_tokens: int
+    k_avg_bits: int = 3
+    v_avg_bits: int = 3
+    b_min: int = 1
+    b_max: int = 4
+    rope_pairing: int = 0
+    max_splits: int = 0
+    seed: int = 0
+    head_dim: int = HEAD_DIM
+
+    def to_c(self):
+        c = _Config()
+        for f in fields(self):
+            setattr(c, f.name, getattr(self, f.name))
+        c.reserved = 0
+        return c
+
+    @property
+    def group_size(self):
+        return self.n_q_heads // self.n_kv_heads
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_SIGS = {
+    "bgtq_required_bytes": (ctypes.c_int, [ctypes.POINTER(_Config), ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "bgtq_create": (ctypes.c_int, [ctypes.POINTER(_Config), _VP, ctypes.c_size_t, _VP, ctypes.c_size_t, _VP, ctypes.POINTER(_VP)]),
+    "bgtq_destroy": (None, [_VP]),
+    "bgtq_allocate": (ctypes.c_int, [_VP, _VP, _I32, _VP, _I32, _VP]),
+    "bgtq_set_allocation": (ctypes.c_int, [_VP, _VP, _VP]),
+    "bgtq_get_allocation": (ctypes.c_int, [_VP, _VP]),
+    "bgtq_get_energy": (ctypes.c_int, [_VP, _VP, _VP]),
+    "bgtq_get_codebook": (ctypes.c_int, [_I32, _VP, _VP]),
+    "bgtq_get_layout": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP]),
+    "bgtq_get_rotation": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _VP, _VP]),
+    "bgtq_cache_offsets": (ctypes.c_int, [_VP, _VP]),
+    "bgtq_encode_append": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
+    "bgtq_rotate_query": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
+    "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "bgtq_set_split_tokens": (ctypes.c_int, [_VP, _I32]),
+    "bgtq_get_device_error": (ctypes.c_int, [_VP, _VP, _VP]),
+    "bgtq_error_string": (ctypes.c_char_p, [_I32]),
+}
+
+
+def lib():
+    """The loaded libbgtq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m packed_decode_attention_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def declared_symbols():
+    return list(_SIGS)
+
+
+def _check(status):
+    if status != 0:
+        raise BgtqError(status, lib().bgtq_error_string(status).decode())
+
+
+def _ptr(x):
+    """Device or host address of a torch tensor / numpy array / int."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+# ---- same-name wrappers -------------------------------------------------
+
+def bgtq_required_bytes(cfg):
+    c = cfg.to_c()
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().bgtq_required_bytes(ctypes.byref(c), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def bgtq_create(cfg, d_cache, cache_bytes, d_workspace, workspace_bytes, stream=None):
+    c = cfg.to_c()
+    out = _VP()
+    _check(lib().bgtq_create(ctypes.byref(c), _ptr(d_cache), cache_bytes, _ptr(d_workspace), workspace_bytes,
+                             _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def bgtq_destroy(state):
+    lib().bgtq_destroy(state)
+
+
+def bgtq_allocate(state, d_calib_q, nq, d_calib_k, nk, stream=None):
+    _check(lib().bgtq_allocate(state, _ptr(d_calib_q), nq, _ptr(d_calib_k), nk, _stream(stream)))
+
+
+def bgtq_set_allocation(state, h_widths, stream=None):
+    w = np.ascontiguousarray(h_widths, dtype=np.int8)
+    _check(lib().bgtq_set_allocation(state, w.ctypes.data, _stream(stream)))
+
+
+def bgtq_get_allocation(state, n_layers, n_kv_heads):
+    w = np.zeros((n_layers, n_kv_heads, N_BLOCKS), dtype=np.int8)
+    _check(lib().bgtq_get_allocation(state, w.ctypes.data))
+    return w
+
+
+def bgtq_get_energy(state, n_layers, n_kv_heads):
+    """Exact energies as nested lists of Python ints [L][Hkv][64] (units 2**-48)."""
+    eq = np.zeros((n_layers, n_kv_heads, N_BLOCKS, 2), dtype=np.uint64)
+    ek = np.zeros_like(eq)
+    _check(lib().bgtq_get_energy(state, eq.ctypes.data, ek.ctypes.data))
+    to_int = lambda a: [[[int(a[l, h, j, 0]) + (int(a[l, h, j, 1]) << 64) for j in range(N_BLOCKS)]
+                         for h in range(n_kv_heads)] for l in range(n_layers)]
+    return to_int(eq), to_int(ek)
+
+
+def bgtq_get_codebook(bits):
+    c = np.zeros(1 << bits, dtype=np.float32)
+    t = np.zeros((1 << bits) - 1, dtype=np.float32)
+    _check(lib().bgtq_get_codebook(bits, c.ctypes.data, t.ctypes.data))
+    return c, t
+
+
+def bgtq_get_layout(state, layer, kv_head):
+    ng = ctypes.c_int32()
+    w = np.zeros(4, dtype=np.int32)
+    s = np.zeros(4, dtype=np.int32)
+    perm = np.zeros(HEAD_DIM, dtype=np.int32)
+    _check(lib().bgtq_get_layout(state, layer, kv_head, ctypes.byref(ng), w.ctypes.data, s.ctypes.data, perm.ctypes.data))
+    return ng.value, w, s, perm
+
+
+def bgtq_get_rotation(state, layer, kv_head, kind, group=0):
+    buf = np.zeros(HEAD_DIM * HEAD_DIM, dtype=np.float32)
+    d = ctypes.c_int32()
+    _check(lib().bgtq_get_rotation(state, layer, kv_head, kind, group, buf.ctypes.data, ctypes.byref(d)))
+    return buf[: d.value * d.value].reshape(d.value, d.value).copy()
+
+
+def bgtq_cache_offsets(state):
+    out = np.zeros(4, dtype=np.uint64)
+    _check(lib().bgtq_cache_offsets(state, out.ctypes.data))
+    return [int(x) for x in out]
+
+
+def bgtq_encode_append(state, layer, layer_count, d_k, d_v, d_start, d_count, batch, n, stream=None):
+    _check(lib().bgtq_encode_append(state, layer, layer_count, _ptr(d_k), _ptr(d_v), _ptr(d_start), _ptr(d_count),
+                                    batch, n, _stream(stream)))
+
+
+def bgtq_rotate_query(state, layer, layer_count, d_q, batch, d_qrot, stream=None):
+    _check(lib().bgtq_rotate_query(state, layer, layer_count, _ptr(d_q), batch, _ptr(d_qrot), _stream(stream)))
+
+
+def bgtq_decode_attn(state, layer, layer_count, d_q, d_seq_lens, batch, d_out, stream=None):
+    _check(lib().bgtq_decode_attn(state, layer, layer_count, _ptr(d_q), _ptr(d_seq_lens), batch, _ptr(d_out),
+                                  _stream(stream)))
+
+
+def bgtq_set_split_tokens(state, tokens):
+    _check(lib().bgtq_set_split_tokens(state, tokens))
+
+
+def bgtq_get_device_error(state, stream=None):
+    f = ctypes.c_int32()
+    _check(lib().bgtq_get_device_error(state, _stream(stream), ctypes.byref(f)))
+    return f.value
+
+
+def bgtq_error_string(status):
+    return lib().bgtq_error_string(status).decode()
+
+
+class PackedKVCache:
+    """One library state over torch-owned device buffers."""
+
+    def __init__(self, cfg, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.cache_bytes, self.workspace_bytes = bgtq_required_bytes(cfg)
+        self.cache = torch.zeros(self.cache_bytes, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.zeros(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        self.state = bgtq_create(cfg, self.cache, self.cache_bytes, self.workspace, self.workspace_bytes)
+        self.offsets = bgtq_cache_offsets(self.state)
+
+    def close(self):
+        if getattr(self, "state", None):
+            bgtq_destroy(self.state)
+            self.state = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- views of the cache arrays (no copies) --
+    def _tokens(self):
+        c = self.cfg
+        return (c.n_layers, c.max_batch, c.n_kv_heads, c.capacity_tokens)
+
+    def k_records(self):
+        n = int(np.prod(self._tokens())) * 16 * self.cfg.k_avg_bits
+        return self.cache[self.offsets[0]:self.offsets[0] + n].view(*self._tokens(), 16 * self.cfg.k_avg_bits)
+
+    def k_norms(self):
+        import torch
+        n = int(np.prod(self._tokens())) * 8
+        return self.cache[self.offsets[1]:self.offsets[1] + n].view(torch.float16).view(*self._tokens(), 4)
+
+    def v_records(self):
+        n = int(np.prod(self._tokens())) * 16 * self.cfg.v_avg_bits
+        return self.cache[self.offsets[2]:self.offsets[2] + n].view(*self._tokens(), 16 * self.cfg.v_avg_bits)
+
+    def v_norms(self):
+        import torch
+        n = int(np.prod(self._tokens())) * 2
+        return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*self._tokens())
+
+    # -- calls --
+    def allocate(self, calib_q, calib_k):
+        bgtq_allocate(self.state, calib_q, calib_q.shape[1], calib_k, calib_k.shape[1])
+
+    def set_allocation(self, widths):
+        bgtq_set_allocation(self.state, widths)
+
+    def get_allocation(self):
+        return bgtq_get_allocation(self.state, self.cfg.n_layers, self.cfg.n_kv_heads)
+
+    def encode_append(self, layer, k, v, start, count, layer_count=1):
+        """k, v fp16 [layer_count, batch, n, Hkv, 128]; start, count int32 [batch] on the device."""
+        bgtq_encode_append(self.state, layer, layer_count, k, v, start, count, k.shape[1], k.shape[2])
+
+    def rotate_query(self, layer, q, out, layer_count=1):
+        bgtq_rotate_query(self.state, layer, layer_count, q, q.shape[1], out)
+
+    def decode_attn(self, layer, q, seq_lens, out, layer_count=1):
+        """q, out fp16 [layer_count, batch, Hq, 128]; seq_lens int32 [batch] on the device."""
+        bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, q.shape[1], out)
+
+    def set_split_tokens(self, tokens):
+        bgtq_set_split_tokens(self.state, tokens)
+
+    def device_error(self):
+        return bgtq_get_device_error(self.state)

@@ -1,0 +1,464 @@
+// The C ABI declared in include/bgtq.h.  Host logic only: argument checks,
+// buffer carving, table construction and upload, kernel launches.  Every
+// step of the path itself runs in kernels.cu.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/bgtq.h"
+#include "device_tables.h"
+#include "host_tables.h"
+
+using bgtq::kD;
+
+struct bgtq_state {
+  bgtq_config cfg;
+  bgtq::Shape shape;
+  bgtq::Workspace ws;
+  bgtq::CacheDev cache;
+  size_t cache_off[4];
+  size_t cache_bytes, ws_bytes;
+  int split_tokens = 0;  // 0 = automatic
+  int num_sms = 148;
+  bool ready = false;
+  bool have_energy = false;
+  std::vector<int8_t> widths;                    // [L][Hkv][64]
+  std::vector<bgtq::GroupLayout> layouts;        // [L][Hkv]
+  std::vector<float> krot;                       // [L][Hkv][4][128*128] per group, row-major d x d
+  std::vector<float> vrot;                       // [L][Hkv][128*128]
+  std::vector<uint64_t> energy_q, energy_k;      // [L][Hkv][64][2]
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int validate_config(const bgtq_config* c) {
+  if (!c) return BGTQ_ERR_NULL;
+  if (c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->max_batch < 1) return BGTQ_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0 || c->n_q_heads / c->n_kv_heads > 16) return BGTQ_ERR_INVALID_ARG;
+  if (c->head_dim != kD) return BGTQ_ERR_INVALID_ARG;
+  if (c->k_avg_bits < 1 || c->k_avg_bits > 4 || c->v_avg_bits < 1 || c->v_avg_bits > 4) return BGTQ_ERR_INVALID_ARG;
+  if (c->b_min < 0 || c->b_max > 4 || c->b_min > c->b_max) return BGTQ_ERR_INVALID_ARG;
+  if (c->k_avg_bits < c->b_min || c->k_avg_bits > c->b_max) return BGTQ_ERR_INVALID_ARG;
+  if (c->rope_pairing != 0 && c->rope_pairing != 1) return BGTQ_ERR_INVALID_ARG;
+  if (c->max_splits < 0 || c->max_splits > 1024 || c->reserved != 0) return BGTQ_ERR_INVALID_ARG;
+  if (c->capacity_tokens < 1 || c->capacity_tokens > (int64_t(1) << 30)) return BGTQ_ERR_INVALID_ARG;
+  return BGTQ_OK;
+}
+
+int max_splits_of(const bgtq_config* c) { return c->max_splits == 0 ? 256 : c->max_splits; }
+
+struct Layout {
+  size_t krec, knorm, vrec, vnorm, cache_total;
+  size_t err, codebook, layouts, mkt, mvt, mv, energy_q, energy_k, qrot, partials, ws_total;
+};
+
+Layout plan(const bgtq_config* c) {
+  Layout p{};
+  const size_t toks = size_t(c->n_layers) * c->max_batch * c->n_kv_heads * size_t(c->capacity_tokens);
+  p.krec = 0;
+  p.knorm = align_up(p.krec + toks * 16 * c->k_avg_bits);
+  p.vrec = align_up(p.knorm + toks * 4 * sizeof(uint16_t));
+  p.vnorm = align_up(p.vrec + toks * 16 * c->v_avg_bits);
+  p.cache_total = align_up(p.vnorm + toks * sizeof(uint16_t));
+  const size_t lh = size_t(c->n_layers) * c->n_kv_heads;
+  p.err = 0;
+  p.codebook = align_up(p.err + sizeof(uint32_t));
+  p.layouts = align_up(p.codebook + sizeof(bgtq::CodebookDev));
+  p.mkt = align_up(p.layouts + lh * sizeof(bgtq::LayoutDev));
+  p.mvt = align_up(p.mkt + lh * kD * kD * sizeof(float));
+  p.mv = align_up(p.mvt + lh * kD * kD * sizeof(float));
+  p.energy_q = align_up(p.mv + lh * kD * kD * sizeof(float));
+  p.energy_k = align_up(p.energy_q + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
+  p.qrot = align_up(p.energy_k + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
+  const size_t qrows = size_t(c->n_layers) * c->max_batch * c->n_q_heads;
+  p.partials = align_up(p.qrot + qrows * kD * sizeof(float));
+  p.ws_total = align_up(p.partials + qrows * max_splits_of(c) * bgtq::kPartialStride * sizeof(float));
+  return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Builds the host tables for the current widths and uploads them.
+int build_and_upload(bgtq_state* st, cudaStream_t stream) {
+  const bgtq_config& c = st->cfg;
+  const int L = c.n_layers, H = c.n_kv_heads;
+  st->layouts.assign(size_t(L) * H, bgtq::GroupLayout());
+  st->krot.assign(size_t(L) * H * 4 * kD * kD, 0.f);
+  st->vrot.assign(size_t(L) * H * kD * kD, 0.f);
+  std::vector<bgtq::LayoutDev> ldev(size_t(L) * H);
+  std::vector<float> mkt(size_t(L) * H * kD * kD, 0.f), mvt(size_t(L) * H * kD * kD), mv(size_t(L) * H * kD * kD);
+  for (int l = 0; l < L; ++l) {
+    for (int h = 0; h < H; ++h) {
+      const size_t lh = size_t(l) * H + h;
+      int bw[bgtq::kBlocks];
+      for (int j = 0; j < bgtq::kBlocks; ++j) bw[j] = st->widths[lh * bgtq::kBlocks + j];
+      const bgtq::GroupLayout lay = bgtq::build_layout(bw, c.rope_pairing);
+      st->layouts[lh] = lay;
+      bgtq::LayoutDev& d = ldev[lh];
+      std::memset(&d, 0, sizeof(d));
+      d.n_groups = lay.n_groups;
+      d.n_positions = lay.n_positions;
+      for (int g = 0; g < bgtq::kNumGroupsMax; ++g) {
+        d.width[g] = lay.width[g];
+        d.size[g] = lay.size[g];
+        d.start[g] = g < lay.n_groups ? lay.start[g] : lay.n_positions;
+        d.bitoff[g] = lay.bitoff[g];
+        d.inv_sqrt_d[g] = lay.size[g] > 0 ? static_cast<float>(1.0 / std::sqrt(double(lay.size[g]))) : 0.f;
+      }
+      for (int i = 0; i < kD; ++i) d.perm[i] = lay.perm[i];
+      float* mk = mkt.data() + lh * kD * kD;
+      for (int g = 0; g < lay.n_groups; ++g) {
+        const int dg = lay.size[g], s0 = lay.start[g];
+        const std::vector<double> R =
+            bgtq::haar_rotation(dg, bgtq::rotation_key(c.seed, l, h, 0, uint64_t(lay.width[g])));
+        float* hr = st->krot.data() + (lh * 4 + g) * kD * kD;
+        for (int i = 0; i < dg; ++i)
+          for (int j = 0; j < dg; ++j) {
+            const float v = static_cast<float>(R[size_t(i) * dg + j]);
+            hr[i * dg + j] = v;
+            mk[size_t(s0 + j) * kD + (s0 + i)] = v;  // transposed: [in][out]
+          }
+      }
+      const std::vector<double> RV = bgtq::haar_rotation(kD, bgtq::rotation_key(c.seed, l, h, 1, uint64_t(c.v_avg_bits)));
+      float* hv = st->vrot.data() + lh * kD * kD;
+      float* vt = mvt.data() + lh * kD * kD;
+      float* vv = mv.data() + lh * kD * kD;
+      for (int i = 0; i < kD; ++i)
+        for (int j = 0; j < kD; ++j) {
+          const float v = static_cast<float>(RV[size_t(i) * kD + j]);
+          hv[i * kD + j] = v;
+          vv[i * kD + j] = v;
+          vt[j * kD + i] = v;
+        }
+    }
+  }
+  cudaError_t e = cudaMemcpyAsync(st->ws.layouts, ldev.data(), ldev.size() * sizeof(bgtq::LayoutDev),
+                                  cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mkt, mkt.data(), mkt.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mvt, mvt.data(), mvt.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mv, mv.data(), mv.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return BGTQ_ERR_CUDA;
+  st->ready = true;
+  return BGTQ_OK;
+}
+
+int auto_split_tokens(const bgtq_state* st, int units) {
+  const int64_t cap = st->cfg.capacity_tokens;
+  const int maxs = max_splits_of(&st->cfg);
+  const int target = 8 * st->num_sms;
+  int nspl = std::max(1, std::min(maxs, (target + units - 1) / std::max(units, 1)));
+  int64_t t = (cap + nspl - 1) / nspl;
+  t = std::max<int64_t>(256, (t + 255) / 256 * 256);
+  while ((cap + t - 1) / t > maxs) t += 256;
+  return static_cast<int>(t);
+}
+
+}  // namespace
+
+extern "C" {
+
+int bgtq_required_bytes(const bgtq_config* cfg, size_t* cache_bytes, size_t* workspace_bytes) {
+  const int v = validate_config(cfg);
+  if (v != BGTQ_OK) return v;
+  if (!cache_bytes || !workspace_bytes) return BGTQ_ERR_NULL;
+  const Layout p = plan(cfg);
+  *cache_bytes = p.cache_total;
+  *workspace_bytes = p.ws_total;
+  return BGTQ_OK;
+}
+
+int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void* d_workspace,
+                size_t workspace_bytes, void* stream, bgtq_state** out) {
+  const int v = validate_config(cfg);
+  if (v != BGTQ_OK) return v;
+  if (!d_cache || !d_workspace || !out) return BGTQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(d_cache) | reinterpret_cast<uintptr_t>(d_workspace)) % kAlign) return BGTQ_ERR_ALIGNMENT;
+  const Layout p = plan(cfg);
+  if (cache_bytes < p.cache_total || workspace_bytes < p.ws_total) return BGTQ_ERR_BUFFER_SIZE;
+  bgtq_state* st = new (std::nothrow) bgtq_state();
+  if (!st) return BGTQ_ERR_HOST_ALLOC;
+  st->cfg = *cfg;
+  st->shape.n_layers = cfg->n_layers;
+  st->shape.n_kv_heads = cfg->n_kv_heads;
+  st->shape.n_q_heads = cfg->n_q_heads;
+  st->shape.group = cfg->n_q_heads / cfg->n_kv_heads;
+  st->shape.max_batch = cfg->max_batch;
+  st->shape.kbits = cfg->k_avg_bits;
+  st->shape.vbits = cfg->v_avg_bits;
+  st->shape.max_splits = max_splits_of(cfg);
+  st->shape.capacity = cfg->capacity_tokens;
+  uint8_t* c8 = static_cast<uint8_t*>(d_cache);
+  st->cache.krec = c8 + p.krec;
+  st->cache.knorm = reinterpret_cast<__half*>(c8 + p.knorm);
+  st->cache.vrec = c8 + p.vrec;
+  st->cache.vnorm = reinterpret_cast<__half*>(c8 + p.vnorm);
+  st->cache_off[0] = p.krec;
+  st->cache_off[1] = p.knorm;
+  st->cache_off[2] = p.vrec;
+  st->cache_off[3] = p.vnorm;
+  st->cache_bytes = p.cache_total;
+  st->ws_bytes = p.ws_total;
+  uint8_t* w8 = static_cast<uint8_t*>(d_workspace);
+  st->ws.err = reinterpret_cast<uint32_t*>(w8 + p.err);
+  st->ws.codebook = reinterpret_cast<bgtq::CodebookDev*>(w8 + p.codebook);
+  st->ws.layouts = reinterpret_cast<bgtq::LayoutDev*>(w8 + p.layouts);
+  st->ws.mkt = reinterpret_cast<float*>(w8 + p.mkt);
+  st->ws.mvt = reinterpret_cast<float*>(w8 + p.mvt);
+  st->ws.mv = reinterpret_cast<float*>(w8 + p.mv);
+  st->ws.energy_q = reinterpret_cast<unsigned __int128*>(w8 + p.energy_q);
+  st->ws.energy_k = reinterpret_cast<unsigned __int128*>(w8 + p.energy_k);
+  st->ws.qrot = reinterpret_cast<float*>(w8 + p.qrot);
+  st->ws.partials = reinterpret_cast<float*>(w8 + p.partials);
+  st->widths.assign(size_t(cfg->n_layers) * cfg->n_kv_heads * bgtq::kBlocks, 0);
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) st->num_sms = sms;
+  }
+  bgtq::CodebookDev cb;
+  std::memset(&cb, 0, sizeof(cb));
+  for (int b = 1; b <= 4; ++b) {
+    std::vector<float> cen, thr;
+    bgtq::lloyd_max_codebook(b, &cen, &thr);
+    for (size_t i = 0; i < cen.size(); ++i) cb.centroid[b][i] = cen[i];
+    for (size_t i = 0; i < thr.size(); ++i) cb.threshold[b][i] = thr[i];
+  }
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaMemcpyAsync(st->ws.codebook, &cb, sizeof(cb), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->ws.err, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    delete st;
+    return BGTQ_ERR_CUDA;
+  }
+  *out = st;
+  return BGTQ_OK;
+}
+
+void bgtq_destroy(bgtq_state* st) { delete st; }
+
+int bgtq_allocate(bgtq_state* st, const void* d_calib_q, int32_t nq, const void* d_calib_k, int32_t nk, void* stream) {
+  if (!st || !d_calib_q || !d_calib_k) return BGTQ_ERR_NULL;
+  if (nq < 1 || nk < 1) return BGTQ_ERR_INVALID_ARG;
+  const bgtq_config& c = st->cfg;
+  cudaStream_t s = as_stream(stream);
+  if (bgtq::launch_energy(st->shape, st->ws, static_cast<const __half*>(d_calib_q), nq,
+                          static_cast<const __half*>(d_calib_k), nk, c.rope_pairing, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  const size_t lh = size_t(c.n_layers) * c.n_kv_heads;
+  const size_t n128 = size_t(bgtq::kEnergyChunks) * lh * 64;
+  std::vector<uint64_t> pq(2 * n128), pk(2 * n128);
+  uint32_t flag = 0;
+  cudaError_t e = cudaMemcpyAsync(pq.data(), st->ws.energy_q, n128 * 16, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(pk.data(), st->ws.energy_k, n128 * 16, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, st->ws.err, sizeof(flag), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return BGTQ_ERR_CUDA;
+  if (flag & bgtq::kErrNonFinite) return BGTQ_ERR_DEVICE;
+  st->energy_q.assign(lh * 64 * 2, 0);
+  st->energy_k.assign(lh * 64 * 2, 0);
+  std::vector<double> scores(64);
+  for (size_t i = 0; i < lh; ++i) {
+    for (int j = 0; j < 64; ++j) {
+      unsigned __int128 sq = 0, sk = 0;
+      for (int ch = 0; ch < bgtq::kEnergyChunks; ++ch) {
+        const size_t o = (size_t(ch) * lh + i) * 64 + j;
+        sq += (static_cast<unsigned __int128>(pq[2 * o + 1]) << 64) | pq[2 * o];
+        sk += (static_cast<unsigned __int128>(pk[2 * o + 1]) << 64) | pk[2 * o];
+      }
+      const size_t o = (i * 64 + j) * 2;
+      st->energy_q[o] = static_cast<uint64_t>(sq);
+      st->energy_q[o + 1] = static_cast<uint64_t>(sq >> 64);
+      st->energy_k[o] = static_cast<uint64_t>(sk);
+      st->energy_k[o + 1] = static_cast<uint64_t>(sk >> 64);
+      scores[j] = bgtq::u128_to_double(st->energy_q[o], st->energy_q[o + 1]) *
+                  bgtq::u128_to_double(st->energy_k[o], st->energy_k[o + 1]);
+    }
+    const std::vector<int> w = bgtq::greedy_allocate(scores.data(), c.k_avg_bits, c.b_min, c.b_max);
+    for (int j = 0; j < 64; ++j) st->widths[i * 64 + j] = static_cast<int8_t>(w[j]);
+  }
+  st->have_energy = true;
+  return build_and_upload(st, s);
+}
+
+int bgtq_set_allocation(bgtq_state* st, const int8_t* h_widths, void* stream) {
+  if (!st || !h_widths) return BGTQ_ERR_NULL;
+  const bgtq_config& c = st->cfg;
+  const size_t lh = size_t(c.n_layers) * c.n_kv_heads;
+  for (size_t i = 0; i < lh; ++i) {
+    int sum = 0;
+    for (int j = 0; j < 64; ++j) {
+      const int w = h_widths[i * 64 + j];
+      if (w < c.b_min || w > c.b_max) return BGTQ_ERR_INVALID_ARG;
+      sum += w;
+    }
+    if (sum != 64 * c.k_avg_bits) return BGTQ_ERR_INVALID_ARG;
+  }
+  std::memcpy(st->widths.data(), h_widths, lh * 64);
+  return build_and_upload(st, as_stream(stream));
+}
+
+int bgtq_get_allocation(const bgtq_state* st, int8_t* h_widths) {
+  if (!st || !h_widths) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  std::memcpy(h_widths, st->widths.data(), st->widths.size());
+  return BGTQ_OK;
+}
+
+int bgtq_get_energy(const bgtq_state* st, uint64_t* h_eq, uint64_t* h_ek) {
+  if (!st || !h_eq || !h_ek) return BGTQ_ERR_NULL;
+  if (!st->have_energy) return BGTQ_ERR_NOT_READY;
+  std::memcpy(h_eq, st->energy_q.data(), st->energy_q.size() * 8);
+  std::memcpy(h_ek, st->energy_k.data(), st->energy_k.size() * 8);
+  return BGTQ_OK;
+}
+
+int bgtq_get_codebook(int32_t bits, float* h_centroids, float* h_thresholds) {
+  if (!h_centroids || !h_thresholds) return BGTQ_ERR_NULL;
+  if (bits < 1 || bits > 4) return BGTQ_ERR_INVALID_ARG;
+  std::vector<float> cen, thr;
+  bgtq::lloyd_max_codebook(bits, &cen, &thr);
+  std::memcpy(h_centroids, cen.data(), cen.size() * 4);
+  std::memcpy(h_thresholds, thr.data(), thr.size() * 4);
+  return BGTQ_OK;
+}
+
+int bgtq_get_layout(const bgtq_state* st, int32_t layer, int32_t kv_head, int32_t* n_groups, int32_t* h_width,
+                    int32_t* h_size, int32_t* h_perm) {
+  if (!st || !n_groups || !h_width || !h_size || !h_perm) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  if (layer < 0 || layer >= st->cfg.n_layers || kv_head < 0 || kv_head >= st->cfg.n_kv_heads) return BGTQ_ERR_INVALID_ARG;
+  const bgtq::GroupLayout& L = st->layouts[size_t(layer) * st->cfg.n_kv_heads + kv_head];
+  *n_groups = L.n_groups;
+  for (int g = 0; g < 4; ++g) {
+    h_width[g] = L.width[g];
+    h_size[g] = L.size[g];
+  }
+  for (int i = 0; i < kD; ++i) h_perm[i] = L.perm[i];
+  return BGTQ_OK;
+}
+
+int bgtq_get_rotation(const bgtq_state* st, int32_t layer, int32_t kv_head, int32_t kind, int32_t group, float* h_out,
+                      int32_t* d) {
+  if (!st || !h_out || !d) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  if (layer < 0 || layer >= st->cfg.n_layers || kv_head < 0 || kv_head >= st->cfg.n_kv_heads) return BGTQ_ERR_INVALID_ARG;
+  const size_t lh = size_t(layer) * st->cfg.n_kv_heads + kv_head;
+  if (kind == 1) {
+    std::memcpy(h_out, st->vrot.data() + lh * kD * kD, kD * kD * 4);
+    *d = kD;
+    return BGTQ_OK;
+  }
+  if (kind != 0) return BGTQ_ERR_INVALID_ARG;
+  const bgtq::GroupLayout& L = st->layouts[lh];
+  if (group < 0 || group >= L.n_groups) return BGTQ_ERR_INVALID_ARG;
+  const int dg = L.size[group];
+  std::memcpy(h_out, st->krot.data() + (lh * 4 + group) * kD * kD, size_t(dg) * dg * 4);
+  *d = dg;
+  return BGTQ_OK;
+}
+
+int bgtq_cache_offsets(const bgtq_state* st, size_t* out) {
+  if (!st || !out) return BGTQ_ERR_NULL;
+  for (int i = 0; i < 4; ++i) out[i] = st->cache_off[i];
+  return BGTQ_OK;
+}
+
+int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                       const int32_t* d_start, const int32_t* d_count, int32_t batch, int32_t n, void* stream) {
+  if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  const bgtq_config& c = st->cfg;
+  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)) return BGTQ_ERR_ALIGNMENT;
+  if (n == 0) return BGTQ_OK;
+  return bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, static_cast<const __half*>(d_k),
+                             static_cast<const __half*>(d_v), d_start, d_count, batch, n, as_stream(stream)) ==
+                 cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
+int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q, int32_t batch, float* d_qrot,
+                      void* stream) {
+  if (!st || !d_q || !d_qrot) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  const bgtq_config& c = st->cfg;
+  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_qrot)) return BGTQ_ERR_ALIGNMENT;
+  return bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
+                                   d_qrot, as_stream(stream)) == cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
+int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q, const int32_t* d_seq_lens,
+                     int32_t batch, void* d_out, void* stream) {
+  if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  const bgtq_config& c = st->cfg;
+  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
+  const int split = st->split_tokens > 0 ? st->split_tokens : auto_split_tokens(st, batch * c.n_kv_heads * layer_count);
+  cudaStream_t s = as_stream(stream);
+  if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
+                                st->ws.qrot, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_decode(st->shape, st->ws, st->cache, layer, layer_count, d_seq_lens, batch, split,
+                          static_cast<__half*>(d_out), s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  return BGTQ_OK;
+}
+
+int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens) {
+  if (!st) return BGTQ_ERR_NULL;
+  if (tokens < 0 || tokens % bgtq::kSplitGranule != 0) return BGTQ_ERR_INVALID_ARG;
+  if (tokens > 0 && (st->cfg.capacity_tokens + tokens - 1) / tokens > max_splits_of(&st->cfg)) return BGTQ_ERR_INVALID_ARG;
+  st->split_tokens = tokens;
+  return BGTQ_OK;
+}
+
+int bgtq_get_device_error(bgtq_state* st, void* stream, int32_t* h_flags) {
+  if (!st || !h_flags) return BGTQ_ERR_NULL;
+  cudaStream_t s = as_stream(stream);
+  uint32_t flag = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, st->ws.err, sizeof(flag), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->ws.err, 0, sizeof(flag), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return BGTQ_ERR_CUDA;
+  *h_flags = static_cast<int32_t>(flag);
+  return BGTQ_OK;
+}
+
+const char* bgtq_error_string(int32_t status) {
+  switch (status) {
+    case BGTQ_OK: return "ok";
+    case BGTQ_ERR_INVALID_ARG: return "invalid argument";
+    case BGTQ_ERR_NULL: return "null pointer";
+    case BGTQ_ERR_CUDA: return "CUDA runtime error";
+    case BGTQ_ERR_BUFFER_SIZE: return "buffer too small";
+    case BGTQ_ERR_NOT_READY: return "no allocation set";
+    case BGTQ_ERR_DEVICE: return "device error flag raised";
+    case BGTQ_ERR_HOST_ALLOC: return "host allocation failed";
+    case BGTQ_ERR_ALIGNMENT: return "misaligned pointer";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,83 @@
+// Device-side table formats and kernel launch parameters shared by the
+// kernels (kernels.cu) and the C ABI (api.cu).
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bgtq {
+
+constexpr int kD = 128;               // head_dim
+constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
+constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
+constexpr int kPartialStride = 132;   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kSplitGranule = 64;     // split sizes are multiples of this many tokens
+
+// Per-(layer, KV head) K layout.  Positions are record order: group 0
+// (widest) first; perm maps a position to the original dim.
+struct alignas(16) LayoutDev {
+  int32_t n_groups;
+  int32_t n_positions;
+  int32_t pad0, pad1;
+  int32_t width[kNumGroupsMax];
+  int32_t size[kNumGroupsMax];
+  int32_t start[kNumGroupsMax];
+  int32_t bitoff[kNumGroupsMax];
+  float inv_sqrt_d[kNumGroupsMax];    // 1 / sqrt(d_g)
+  int32_t perm[kD];
+  int32_t pad2[8];
+};
+static_assert(sizeof(LayoutDev) == 640, "layout record size");
+
+// fp32 Lloyd-Max codebooks indexed by width (row 0 unused).
+struct CodebookDev {
+  float centroid[5][16];
+  float threshold[5][16];
+};
+
+// Pointers into the caller's workspace buffer.
+struct Workspace {
+  uint32_t* err;                 // device error flag bits
+  CodebookDev* codebook;
+  LayoutDev* layouts;            // [L][Hkv]
+  float* mkt;                    // [L][Hkv][128 in][128 out]: K rotation, block diagonal in record order, transposed
+  float* mvt;                    // [L][Hkv][128 in][128 out]: V rotation transposed
+  float* mv;                     // [L][Hkv][128 out][128 in]: V rotation (for the inverse rotation)
+  unsigned __int128* energy_q;   // [kEnergyChunks][L][Hkv][64]
+  unsigned __int128* energy_k;   // [kEnergyChunks][L][Hkv][64]
+  float* qrot;                   // [L][B][Hq][128]
+  float* partials;               // [L][B][Hq][max_splits][kPartialStride]
+};
+
+struct CacheDev {
+  uint8_t* krec;                 // [L][B][Hkv][C][16*kbits]
+  __half* knorm;                 // [L][B][Hkv][C][4]
+  uint8_t* vrec;                 // [L][B][Hkv][C][16*vbits]
+  __half* vnorm;                 // [L][B][Hkv][C]
+};
+
+struct Shape {
+  int32_t n_layers, n_kv_heads, n_q_heads, group, max_batch;
+  int32_t kbits, vbits, max_splits;
+  int64_t capacity;
+};
+
+// Error flag bits (same values as BGTQ_DEVERR_* in bgtq.h).
+constexpr uint32_t kErrCapacity = 1;
+constexpr uint32_t kErrSeqLen = 2;
+constexpr uint32_t kErrArg = 4;
+constexpr uint32_t kErrNonFinite = 8;
+
+// Launchers (kernels.cu).  Each returns the cudaError_t of its launch.
+cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,
+                          const __half* calib_k, int nk, int pairing, cudaStream_t stream);
+cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                          int layer_count, const __half* k, const __half* v, const int32_t* start,
+                          const int32_t* count, int batch, int n, cudaStream_t stream);
+cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
+                                const __half* q, int batch, float* qrot, cudaStream_t stream);
+cudaError_t launch_decode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                          int layer_count, const int32_t* seq_lens, int batch, int split_tokens,
+                          __half* out, cudaStream_t stream);
+
+}  // namespace bgtq

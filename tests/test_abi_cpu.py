@@ -1,0 +1,59 @@
+"""CPU checks of the C-ABI library: it loads and exports every declared symbol."""
+import os
+import re
+
+import pytest
+
+from packed_decode_attention_b200 import bgtq
+from packed_decode_attention_b200 import build as pkg_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bgtq.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bgtq_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkg_build.build()
+    return bgtq.lib()
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    names = header_functions()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(bgtq.declared_symbols()) == names
+
+
+def test_error_strings(lib):
+    assert bgtq.bgtq_error_string(0) == "ok"
+    assert bgtq.bgtq_error_string(-1) == "invalid argument"
+    assert bgtq.bgtq_error_string(-999) == "unknown status"
+
+
+def test_required_bytes_is_host_only_and_validates(lib):
+    cfg = bgtq.Config(n_layers=36, n_kv_heads=2, n_q_heads=16, max_batch=1, capacity_tokens=131072)
+    cache, ws = bgtq.bgtq_required_bytes(cfg)
+    toks = 36 * 2 * 131072
+    assert cache >= toks * (48 + 8 + 48 + 2)
+    assert cache < toks * (48 + 8 + 48 + 2) + 4 * 256
+    assert cache % 256 == 0 and ws % 256 == 0
+    bad = [dict(head_dim=64), dict(n_q_heads=15), dict(k_avg_bits=5), dict(b_min=4, b_max=3),
+           dict(k_avg_bits=1, b_min=2), dict(rope_pairing=2), dict(capacity_tokens=0), dict(max_splits=2000)]
+    for change in bad:
+        c = bgtq.Config(**{**cfg.__dict__, **change})
+        with pytest.raises(bgtq.BgtqError) as e:
+            bgtq.bgtq_required_bytes(c)
+        assert e.value.status == -1
+
+
+def test_library_fails_loudly_when_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(bgtq, "_lib", None)
+    monkeypatch.setattr(bgtq, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError):
+        bgtq.lib()

@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Decode-attention throughput of the packed Block-GTQ cache on B200.
+
+One step = one decode step of the whole model: for every layer, append the
+step's new token to the packed cache (TQ-MSE encode of its K and V rows at
+position len-1, so lengths stay fixed) and run GQA decode attention over the
+packed cache (rotate the query, split-K pass, combine).  Steps run as one
+CUDA graph.  value = sequences * steps / time  (decode tokens/s).
+
+Printed as one JSON line on rank 0.  Also measured in the same run:
+  roofline      the split-K decode kernel alone, CUDA events around each launch
+  e2e           same step through the C ABI from pinned host buffers (H2D of
+                the queries and new K/V, D2H of the outputs inside the timing)
+  multi_layer   all layers in one launch per kernel
+  fp16_baseline dense fp16 FlashAttention-2 decode over the unquantised K/V
+  cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU)
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen3b]
+  python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp16-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid):
+        self.uuid = device_uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mhz, mx, reasons = [], [], set()
+        rows = [l for t, l in self.lines if t0 - 0.25 <= t <= t1 + 0.25] or [l for _, l in self.lines]
+        for l in rows:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def token_bytes(kv, cfg):
+    """Algorithmic packed bytes per cached token for each (layer, KV head)."""
+    from packed_decode_attention_b200 import bgtq
+    out = {}
+    for l in range(cfg.n_layers):
+        for h in range(cfg.n_kv_heads):
+            ng = bgtq.bgtq_get_layout(kv.state, l, h)[0]
+            out[l, h] = 16 * cfg.k_avg_bits + 16 * cfg.v_avg_bits + 2 * ng + 2
+    return out
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        n = 1
+    return max(n, 1)
+
+
+class OracleSample:
+    """A bounded sample of the workload for the CPU oracle: a few (layer, KV
+    head) pairs of sequence 0 at its full length, each with its own oracle
+    allocation, tables and packed cache (built once, untimed).  One timed unit
+    is the oracle's decode of the G query heads of a pair over its cache plus
+    the encode of one new K/V row; a full step is every (layer, KV head) of
+    every sequence, so the step time is the unit time scaled by
+    layers * KV heads * (total cached tokens / sample length)."""
+
+    def __init__(self, w, lens, max_pairs=4):
+        import numpy as np
+
+        from oracle import model
+        from packed_decode_attention_b200 import workloads as wl
+
+        self.w, self.lens = w, lens
+        pairs = [(l, h) for l in range(w.n_layers) for h in range(w.n_kv_heads)]
+        self.n_pairs = len(pairs)
+        pick = [pairs[i] for i in np.linspace(0, len(pairs) - 1, num=min(max_pairs, len(pairs))).astype(int)]
+        self.t_len = lens[0]
+        cfg = model.Config(w.n_layers, w.n_kv_heads, w.n_q_heads, 128, w.k_bits, w.v_bits, 1, 4, 0, w.seed)
+        self.units = []
+        for (l, h) in pick:
+            cq = wl.queries(w, l, 0, np.arange(w.n_calib), tag=1)[None]
+            ck = wl.keys(w, l, 0, 0, w.n_calib)[None]
+            c1 = model.Config(1, w.n_kv_heads, w.n_q_heads, 128, w.k_bits, w.v_bits, 1, 4, 0, w.seed)
+            full = np.zeros((w.n_layers, w.n_kv_heads, 64), dtype=np.int64)
+            full[l] = model.allocate(c1, cq.numpy(), ck.numpy())[0]
+            tb = model.Tables(cfg, full, layers=[l])
+            k = wl.keys(w, l, 0, 0, self.t_len)[:, h].numpy()
+            v = wl.values(w, l, 0, 0, self.t_len)[:, h].numpy()
+            enc = model.encode_rows(tb, l, h, k, v)
+            q = wl.queries(w, l, 0, [self.t_len], tag=2)[0, h * w.group:(h + 1) * w.group].numpy()
+            self.units.append((tb, l, h, k[-1:], v[-1:], q, enc))
+
+    def time_unit(self, i):
+        from oracle import model
+        tb, l, h, k1, v1, q, enc = self.units[i % len(self.units)]
+        t0 = time.perf_counter()
+        model.encode_rows(tb, l, h, k1, v1)
+        model.decode(tb, l, h, q, enc["k_rec"], enc["k_norms"], enc["v_rec"], enc["v_norm"])
+        return time.perf_counter() - t0
+
+    def step_seconds(self, unit_s):
+        return unit_s * self.w.n_layers * self.w.n_kv_heads * (sum(self.lens) / float(self.t_len))
+
+    def describe(self, n_timed):
+        w = self.w
+        return (f"oracle decode of the {w.group} query heads of one (layer, KV head) over {self.t_len} tokens "
+                f"+ encode of one K/V row; {n_timed} units over {len(self.units)} of {self.n_pairs} pairs "
+                f"(sequence 0 of {w.batch}); step time = unit time x {w.n_layers * w.n_kv_heads} pairs "
+                f"x total/sample tokens")
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return 0
+    from packed_decode_attention_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    lens = wl.seq_lens(w)
+    sample = OracleSample(w, lens, max_pairs=2)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = sample.time_unit(i)
+        if i >= args.warmup:
+            times.append(sample.step_seconds(dt))
+    step_s = statistics.mean(times)
+    value = w.batch / step_s
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": "decode_tokens_per_s", "value": value, "unit": "tokens/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, lens),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample.describe(args.steps)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, lens):
+    return {"workload": f"{w.name}: {w.n_layers} layers x {w.n_kv_heads} KV heads, {w.n_q_heads} q heads, "
+                        f"head_dim 128, batch {w.batch} x {max(lens)} cached tokens, K{w.k_bits}V{w.v_bits}",
+            "layers": w.n_layers, "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads, "batch": w.batch,
+            "context": max(lens), "total_cached_tokens": int(sum(lens)), "k_bits": w.k_bits, "v_bits": w.v_bits,
+            "l2": "inputs larger than L2: every step streams the whole packed cache of all layers",
+            "parallelism": "replicas"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+
+    from packed_decode_attention_b200 import bgtq
+    from packed_decode_attention_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = wl.WORKLOADS[args.workload]
+    lens = wl.seq_lens(w)
+    L, H, HQ, B = w.n_layers, w.n_kv_heads, w.n_q_heads, w.batch
+    cap = w.seq_len
+    cfg = bgtq.Config(n_layers=L, n_kv_heads=H, n_q_heads=HQ, max_batch=B, capacity_tokens=cap,
+                      k_avg_bits=w.k_bits, v_avg_bits=w.v_bits, seed=w.seed,
+                      max_splits=64 if B > 4 else 0)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- calibration + allocation (one-time) ----
+    cq, ck = wl.calibration(w, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    kv.allocate(cq, ck)
+    e1.record()
+    torch.cuda.synchronize()
+    alloc_ms = e0.elapsed_time(e1)
+    del cq, ck
+
+    # ---- prefill: encode the whole cache (and keep fp16 K/V for the dense baseline) ----
+    want_fp16 = not args.no_fp16_baseline
+    kf = [torch.empty((B, cap, H, 128), dtype=torch.float16, device=dev) for _ in range(L)] if want_fp16 else None
+    vf = [torch.empty((B, cap, H, 128), dtype=torch.float16, device=dev) for _ in range(L)] if want_fp16 else None
+    chunk = 32768
+    enc_ms = 0.0
+    enc_rows = 0
+    for l in range(L):
+        for b in range(B):
+            for s0 in range(0, lens[b], chunk):
+                n = min(chunk, lens[b] - s0)
+                kk = torch.zeros((1, B, n, H, 128), dtype=torch.float16, device=dev)
+                vv = torch.zeros_like(kk)
+                kk[0, b] = wl.keys(w, l, b, s0, n, device=dev)
+                vv[0, b] = wl.values(w, l, b, s0, n, device=dev)
+                if want_fp16:
+                    kf[l][b, s0:s0 + n] = kk[0, b]
+                    vf[l][b, s0:s0 + n] = vv[0, b]
+                start = torch.zeros(B, dtype=torch.int32, device=dev)
+                count = torch.zeros(B, dtype=torch.int32, device=dev)
+                start[b] = s0
+                count[b] = n
+                e0.record()
+                kv.encode_append(l, kk, vv, start, count)
+                e1.record()
+                torch.cuda.synchronize()
+                enc_ms += e0.elapsed_time(e1)
+                enc_rows += n * H
+    assert kv.device_error() == 0, "device error after prefill"
+
+    # ---- step inputs ----
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    start1 = seq - 1
+    count1 = torch.ones(B, dtype=torch.int32, device=dev)
+    q_all = torch.stack([wl.decode_query(w, l, lens, device=dev) for l in range(L)])          # [L, B, HQ, 128]
+    knew = torch.zeros((L, B, 1, H, 128), dtype=torch.float16, device=dev)
+    vnew = torch.zeros_like(knew)
+    for l in range(L):
+        for b in range(B):
+            knew[l, b, 0] = wl.keys(w, l, b, lens[b] - 1, 1, device=dev)[0]
+            vnew[l, b, 0] = wl.values(w, l, b, lens[b] - 1, 1, device=dev)[0]
+    out = torch.empty((L, B, HQ, 128), dtype=torch.float16, device=dev)
+
+    def step():
+        for l in range(L):
+            kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
+            kv.decode_attn(l, q_all[l:l + 1], seq, out[l:l + 1])
+
+    def step_multi():
+        kv.encode_append(0, knew, vnew, start1, count1, layer_count=L)
+        kv.decode_attn(0, q_all, seq, out, layer_count=L)
+
+    def time_graph(fn, steps, warmup, sampler=None):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_wall0 = time.time()
+        a.record()
+        for _ in range(steps):
+            g.replay()
+        z.record()
+        torch.cuda.synchronize()
+        t_wall1 = time.time()
+        barrier()
+        return a.elapsed_time(z) / steps, g, (t_wall0, t_wall1)
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    ms_step, graph, (tw0, tw1) = time_graph(step, args.steps, args.warmup)
+    sampler.stop()
+    clocks = sampler.summary(tw0, tw1)
+    ms_step = max_over_ranks(ms_step)
+    assert kv.device_error() == 0, "device error during the timed steps"
+    out_check = out.float()
+    assert torch.isfinite(out_check).all(), "non-finite decode output"
+
+    ms_multi, g_multi, _ = time_graph(step_multi, args.steps, args.warmup)
+    ms_multi = max_over_ranks(ms_multi)
+    del g_multi
+
+    # ---- the split-K kernel alone: events around each launch ----
+    tb = token_bytes(kv, cfg)
+    qrot = torch.empty((1, B, HQ, 128), dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    split_ms = []
+    for it in range(args.warmup + args.steps):
+        for l in range(L):
+            kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
+            kv.rotate_query(l, q_all[l:l + 1], qrot)
+            ev[l][0].record()
+            kv.decode_split(l, qrot, seq)
+            ev[l][1].record()
+            kv.decode_combine(l, seq, out[l:l + 1])
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            split_ms.extend(a.elapsed_time(z) for a, z in ev)
+    split_avg_ms = statistics.mean(split_ms)
+    bytes_per_layer = [sum(lens[b] * tb[l, h] for b in range(B) for h in range(H)) for l in range(L)]
+    alg_bytes = statistics.mean(bytes_per_layer)
+    achieved = alg_bytes / (split_avg_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+
+    # ---- end to end from pinned host memory ----
+    q_h = q_all.cpu().pin_memory()
+    k_h = knew.cpu().pin_memory()
+    v_h = vnew.cpu().pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
+    d2h = o_h.numel() * 2
+    for _ in range(args.warmup):
+        q_all.copy_(q_h, non_blocking=True)
+        knew.copy_(k_h, non_blocking=True)
+        vnew.copy_(v_h, non_blocking=True)
+        graph.replay()
+        o_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        q_all.copy_(q_h, non_blocking=True)
+        knew.copy_(k_h, non_blocking=True)
+        vnew.copy_(v_h, non_blocking=True)
+        graph.replay()
+        o_h.copy_(out, non_blocking=True)
+    z.record()
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(a.elapsed_time(z) / args.steps)
+    del graph
+
+    # ---- dense fp16 baseline (FlashAttention-2 decode) ----
+    fp16 = None
+    if want_fp16:
+        import torch.nn.functional as F
+        qf = q_all.view(L, B, 1, HQ, 128)
+
+        def fp16_step_sdpa():
+            for l in range(L):
+                for b in range(B):
+                    qq = q_all[l, b][None, :, None, :]
+                    kk = kf[l][b, :lens[b]].transpose(0, 1)[None]
+                    vv = vf[l][b, :lens[b]].transpose(0, 1)[None]
+                    F.scaled_dot_product_attention(qq, kk, vv, enable_gqa=True)
+
+        try:
+            from flash_attn import flash_attn_with_kvcache
+
+            def fp16_step():
+                for l in range(L):
+                    flash_attn_with_kvcache(qf[l], kf[l], vf[l], cache_seqlens=seq)
+
+            fp16_step()
+            torch.cuda.synchronize()
+            name = "flash_attn_with_kvcache (FlashAttention-2 decode)"
+        except Exception:
+            fp16_step = fp16_step_sdpa
+            name = "torch scaled_dot_product_attention"
+        try:
+            ms_fp16, g16, _ = time_graph(fp16_step, args.steps, args.warmup)
+            ms_fp16 = max_over_ranks(ms_fp16)
+            del g16
+            fp16 = {"impl": name, "ms_per_step": ms_fp16, "tokens_per_s": world * B / (ms_fp16 * 1e-3),
+                    "bytes_per_step": int(sum(lens) * H * L * 512), "speedup_of_packed": ms_fp16 / ms_step}
+        except Exception as e:  # report, do not fail the bench
+            fp16 = {"impl": name, "error": str(e)[:200]}
+        del kf, vf
+
+    # ---- CPU oracle on a bounded sample ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(w, lens, max_pairs=3)
+        units = [sample.time_unit(i) for i in range(len(sample.units) * 2)]
+        st = sample.step_seconds(statistics.mean(units))
+        cpu = {"value": B / st, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample.describe(len(units))}
+
+    value = world * B / (ms_step * 1e-3)
+    step_bytes = sum(bytes_per_layer) + L * B * HQ * 512
+    line = {
+        "metric": "decode_tokens_per_s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, lens),
+        "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "decode_split_kernel",
+                     "launch_ms": split_avg_ms, "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind},
+        "e2e": {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * L * args.steps,
+        "clocks": clocks,
+        "multi_layer": {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
+                        "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},
+        "fp16_baseline": fp16,
+        "cpu_baseline": cpu,
+        "allocate_ms": alloc_ms,
+        "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),
+        "compression_vs_fp16": 512.0 / (sum(lens[b] * tb[l, h] for l in range(L) for b in range(B) for h in range(H))
+                                        / (sum(lens) * L * H)),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    kv.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -191,6 +191,18 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
 int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                      const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
 
+/* The two stages of bgtq_decode_attn after bgtq_rotate_query, for callers
+ * that time or schedule them separately (same arguments and results):
+ * bgtq_decode_split runs the split-K pass over the packed cache from the
+ * rotated queries d_qrot (fp32 [layer_count][batch][n_q_heads][128], as
+ * written by bgtq_rotate_query) into the workspace's partials, and
+ * bgtq_decode_combine merges them into d_out.  Both must see the same
+ * layer, layer_count, batch and split setting.  ASYNC. */
+int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const float* d_qrot,
+                      const int32_t* d_seq_lens, int32_t batch, void* stream);
+int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, const int32_t* d_seq_lens,
+                        int32_t batch, void* d_out, void* stream);
+
 /* Tokens per split-K chunk for bgtq_decode_attn: 0 = automatic (from
  * capacity, max_splits and the SM count), else a multiple of 64 with
  * ceil(capacity / tokens) <= max_splits.  Results do not depend on it beyond

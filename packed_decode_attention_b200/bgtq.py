@@ -97,6 +97,8 @@ _SIGS = {
     "bgtq_encode_append": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
     "bgtq_rotate_query": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
+    "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_set_split_tokens": (ctypes.c_int, [_VP, _I32]),
     "bgtq_get_device_error": (ctypes.c_int, [_VP, _VP, _VP]),
     "bgtq_error_string": (ctypes.c_char_p, [_I32]),
@@ -234,6 +236,14 @@ def bgtq_decode_attn(state, layer, layer_count, d_q, d_seq_lens, batch, d_out, s
                                   _stream(stream)))
 
 
+def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
+    _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
+
+
+def bgtq_decode_combine(state, layer, layer_count, d_seq_lens, batch, d_out, stream=None):
+    _check(lib().bgtq_decode_combine(state, layer, layer_count, _ptr(d_seq_lens), batch, _ptr(d_out), _stream(stream)))
+
+
 def bgtq_set_split_tokens(state, tokens):
     _check(lib().bgtq_set_split_tokens(state, tokens))
 
@@ -315,6 +325,13 @@ class PackedKVCache:
     def decode_attn(self, layer, q, seq_lens, out, layer_count=1):
         """q, out fp16 [layer_count, batch, Hq, 128]; seq_lens int32 [batch] on the device."""
         bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, q.shape[1], out)
+
+    def decode_split(self, layer, qrot, seq_lens, layer_count=1):
+        """The split-K stage alone from rotated queries (fp32 [layer_count, batch, Hq, 128])."""
+        bgtq_decode_split(self.state, layer, layer_count, qrot, seq_lens, qrot.shape[1])
+
+    def decode_combine(self, layer, seq_lens, out, layer_count=1):
+        bgtq_decode_combine(self.state, layer, layer_count, seq_lens, out.shape[1], out)
 
     def set_split_tokens(self, tokens):
         bgtq_set_split_tokens(self.state, tokens)

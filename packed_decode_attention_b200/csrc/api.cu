@@ -406,21 +406,63 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
              : BGTQ_ERR_CUDA;
 }
 
-int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q, const int32_t* d_seq_lens,
-                     int32_t batch, void* d_out, void* stream) {
-  if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+namespace {
+
+int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, int32_t batch) {
   if (!st->ready) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
   if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
+  return BGTQ_OK;
+}
+
+int split_for(const bgtq_state* st, int32_t layer_count, int32_t batch) {
+  return st->split_tokens > 0 ? st->split_tokens : auto_split_tokens(st, batch * st->cfg.n_kv_heads * layer_count);
+}
+
+}  // namespace
+
+int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const float* d_qrot,
+                      const int32_t* d_seq_lens, int32_t batch, void* stream) {
+  if (!st || !d_qrot || !d_seq_lens) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
+  if (!aligned16(d_qrot) || !aligned16(d_seq_lens)) return BGTQ_ERR_ALIGNMENT;
+  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, batch,
+                                   split_for(st, layer_count, batch), as_stream(stream)) == cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
+int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, const int32_t* d_seq_lens, int32_t batch,
+                        void* d_out, void* stream) {
+  if (!st || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
+  if (!aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
+  return bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch,
+                              split_for(st, layer_count, batch), static_cast<__half*>(d_out),
+                              as_stream(stream)) == cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
+int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q, const int32_t* d_seq_lens,
+                     int32_t batch, void* d_out, void* stream) {
+  if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  const int split = st->split_tokens > 0 ? st->split_tokens : auto_split_tokens(st, batch * c.n_kv_heads * layer_count);
+  const int split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode(st->shape, st->ws, st->cache, layer, layer_count, d_seq_lens, batch, split,
-                          static_cast<__half*>(d_out), s) != cudaSuccess)
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, st->ws.qrot, d_seq_lens, batch,
+                                split, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split,
+                           static_cast<__half*>(d_out), s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   return BGTQ_OK;
 }

@@ -76,8 +76,11 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           const int32_t* count, int batch, int n, cudaStream_t stream);
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
-cudaError_t launch_decode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                          int layer_count, const int32_t* seq_lens, int batch, int split_tokens,
-                          __half* out, cudaStream_t stream);
+cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
+                                int split_tokens, cudaStream_t stream);
+cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
+                           const int32_t* seq_lens, int batch, int split_tokens, __half* out,
+                           cudaStream_t stream);
 
 }  // namespace bgtq

@@ -358,7 +358,7 @@ struct DecodeSmem {
 
 template <int KB, int GP, int TPL>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(Shape sh, Workspace ws, CacheDev cache,
-                                                                   int layer0,
+                                                                   int layer0, const float* __restrict__ qrot,
                                                                    const int32_t* __restrict__ seq_lens,
                                                                    int batch, int split_tokens) {
   constexpr int NW = 4 * KB;  // 32-bit words per K record
@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(Shape sh, Wor
     reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
   for (int i = tid; i < 5 * 16; i += kDecThreads) (&S.cent[0][0])[i] = (&ws.codebook->centroid[0][0])[i];
   {
-    const float* qsrc = ws.qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G) * kD;
+    const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G) * kD;
     for (int e = tid; e < kD * GP; e += kDecThreads) {
       const int hh = e / kD, i = e % kD;
       S.qs[i][hh] = hh < G ? qsrc[hh * kD + i] * kLog2e : 0.f;
@@ -658,34 +658,43 @@ __global__ void __launch_bounds__(128) combine_kernel(Shape sh, Workspace ws, in
   out[row * kD + i] = __float2half(o);
 }
 
+// Raises a kernel's dynamic shared-memory limit.  Callers keep the result
+// in a function-local static of a function that is unique per kernel, so
+// the attribute is set once per process and never inside a graph capture.
 template <typename F>
 cudaError_t set_smem(F* fn, size_t bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
+template <int KIND>
+cudaError_t encode_smem_once() {
+  static const cudaError_t status = set_smem(encode_kernel<KIND>, sizeof(EncodeSmem));
+  return status;
+}
+
 template <int KB, int GP, int TPL>
 cudaError_t launch_decode_t(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                            int layer_count, const int32_t* seq_lens, int batch, int split_tokens,
-                            cudaStream_t stream) {
+                            int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
+                            int split_tokens, cudaStream_t stream) {
   const size_t smem = sizeof(DecodeSmem<GP, TPL>);
   auto* fn = decode_split_kernel<KB, GP, TPL>;
-  cudaError_t e = set_smem(fn, smem);
-  if (e != cudaSuccess) return e;
+  static const cudaError_t attr = set_smem(fn, smem);  // one static per instantiation
+  if (attr != cudaSuccess) return attr;
   const int nspl = static_cast<int>((s.capacity + split_tokens - 1) / split_tokens);
   dim3 grid(nspl, batch * s.n_kv_heads, layer_count);
-  fn<<<grid, kDecThreads, smem, stream>>>(s, ws, cache, layer0, seq_lens, batch, split_tokens);
+  fn<<<grid, kDecThreads, smem, stream>>>(s, ws, cache, layer0, qrot, seq_lens, batch, split_tokens);
   return cudaGetLastError();
 }
 
 template <int GP, int TPL>
 cudaError_t launch_decode_g(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                            int layer_count, const int32_t* seq_lens, int batch, int split_tokens,
-                            cudaStream_t stream) {
+                            int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
+                            int split_tokens, cudaStream_t stream) {
   switch (s.kbits) {
-    case 1: return launch_decode_t<1, GP, TPL>(s, ws, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-    case 2: return launch_decode_t<2, GP, TPL>(s, ws, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-    case 3: return launch_decode_t<3, GP, TPL>(s, ws, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-    default: return launch_decode_t<4, GP, TPL>(s, ws, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
+    case 1: return launch_decode_t<1, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    case 2: return launch_decode_t<2, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    case 3: return launch_decode_t<3, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    default: return launch_decode_t<4, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
   }
 }
 
@@ -704,9 +713,9 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           const int32_t* count, int batch, int n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
   const size_t smem = sizeof(EncodeSmem);
-  cudaError_t e = set_smem(encode_kernel<0>, smem);
+  cudaError_t e = encode_smem_once<0>();
   if (e != cudaSuccess) return e;
-  e = set_smem(encode_kernel<1>, smem);
+  e = encode_smem_once<1>();
   if (e != cudaSuccess) return e;
   dim3 grid(layer_count * batch * s.n_kv_heads, (n + kEncRows - 1) / kEncRows);
   encode_kernel<0><<<grid, kEncThreads, smem, stream>>>(s, ws, cache, layer0, k, start, count, batch, n);
@@ -722,18 +731,19 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                          int layer_count, const int32_t* seq_lens, int batch, int split_tokens,
-                          __half* out, cudaStream_t stream) {
-  Workspace w2 = ws;
-  cudaError_t e;
+cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
+                                int split_tokens, cudaStream_t stream) {
   if (s.group <= 4)
-    e = launch_decode_g<4, 4>(s, w2, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-  else if (s.group <= 8)
-    e = launch_decode_g<8, 2>(s, w2, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-  else
-    e = launch_decode_g<16, 1>(s, w2, cache, layer0, layer_count, seq_lens, batch, split_tokens, stream);
-  if (e != cudaSuccess) return e;
+    return launch_decode_g<4, 4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+  if (s.group <= 8)
+    return launch_decode_g<8, 2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+  return launch_decode_g<16, 1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+}
+
+cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
+                           const int32_t* seq_lens, int batch, int split_tokens, __half* out,
+                           cudaStream_t stream) {
   combine_kernel<<<layer_count * batch * s.n_q_heads, kD, 0, stream>>>(s, ws, layer0, seq_lens, batch, split_tokens,
                                                                        out);
   return cudaGetLastError();

@@ -328,3 +328,34 @@ def test_uniform_allocation_is_tq_mse(dev):
     ref = haar.rotation_fp32(128, cfg.seed, 0, 0, 0, 3)
     assert np.all(np.abs(rot.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64)) <= 1)
     kv.close()
+
+
+def test_stage_calls_equal_decode_attn(dev):
+    """rotate_query + decode_split + decode_combine is the same computation as decode_attn."""
+    w = wl.scaled(wl.WORKLOADS["llama"], n_calib=128, seq_len=5000, batch=2)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    kv.allocate(cq.to(dev), ck.to(dev))
+    lens = [5000, 3333]
+    for b, ln in enumerate(lens):
+        k = torch.zeros((1, 2, ln, cfg.n_kv_heads, 128), dtype=torch.float16)
+        v = torch.zeros_like(k)
+        k[0, b] = wl.keys(w, 0, b, 0, ln)
+        v[0, b] = wl.values(w, 0, b, 0, ln)
+        start = torch.zeros(2, dtype=torch.int32, device=dev)
+        count = torch.zeros(2, dtype=torch.int32, device=dev)
+        count[b] = ln
+        kv.encode_append(0, k.to(dev), v.to(dev), start, count)
+    q = wl.decode_query(w, 0, lens)[None].to(dev)
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    a = torch.empty((1, 2, cfg.n_q_heads, 128), dtype=torch.float16, device=dev)
+    kv.decode_attn(0, q, seq, a)
+    qrot = torch.empty((1, 2, cfg.n_q_heads, 128), dtype=torch.float32, device=dev)
+    kv.rotate_query(0, q, qrot)
+    kv.decode_split(0, qrot, seq)
+    bb = torch.empty_like(a)
+    kv.decode_combine(0, seq, bb)
+    assert torch.equal(a, bb)
+    assert kv.device_error() == 0
+    kv.close()

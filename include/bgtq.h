@@ -203,6 +203,32 @@ int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const 
 int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, const int32_t* d_seq_lens,
                         int32_t batch, void* d_out, void* stream);
 
+/* No Block-GTQ counterpart on the pages: a library convenience.
+ *
+ * Same computation, arguments and results as bgtq_decode_attn, for callers
+ * that cannot allocate device memory themselves: code that issues work from
+ * inside a CUDA stream capture (allocation is not a capturable operation),
+ * or a runtime whose device memory is fully reserved up front by its own
+ * pool.  This call needs no caller-provided scratch: the rotated queries
+ * and split-K partials live in one static device array inside the library
+ * of BGTQ_STATIC_SCRATCH_BYTES (16 MiB), which every GPU that loads the
+ * library holds until the process exits.  The call allocates nothing.
+ *
+ * The scratch needed is layer_count * max_batch * n_q_heads * (512 +
+ * n_splits * 528) bytes, n_splits = ceil(capacity_tokens / split tokens)
+ * with the split chosen as for bgtq_decode_attn; a call needing more returns
+ * BGTQ_ERR_BUFFER_SIZE before launching anything.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any
+ * stream capture.  Every call on a device shares the one array and reads
+ * only what the same call wrote: calls that overlap on the GPU (different
+ * streams, or different states at once) race on it.  ASYNC after the first
+ * call. */
+#define BGTQ_STATIC_SCRATCH_BYTES (16u << 20)
+int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                                    const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
+
 /* Tokens per split-K chunk for bgtq_decode_attn: 0 = automatic (from
  * capacity, max_splits and the SM count), else a multiple of 64 with
  * ceil(capacity / tokens) <= max_splits.  Results do not depend on it beyond

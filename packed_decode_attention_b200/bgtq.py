@@ -99,6 +99,7 @@ _SIGS = {
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
+    "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_set_split_tokens": (ctypes.c_int, [_VP, _I32]),
     "bgtq_get_device_error": (ctypes.c_int, [_VP, _VP, _VP]),
     "bgtq_error_string": (ctypes.c_char_p, [_I32]),
@@ -242,6 +243,13 @@ def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stre
 
 def bgtq_decode_combine(state, layer, layer_count, d_seq_lens, batch, d_out, stream=None):
     _check(lib().bgtq_decode_combine(state, layer, layer_count, _ptr(d_seq_lens), batch, _ptr(d_out), _stream(stream)))
+
+
+def bgtq_decode_attn_static_scratch(state, layer, layer_count, d_q, d_seq_lens, batch, d_out, stream=None):
+    """bgtq_decode_attn with the split-K scratch in the library's static device
+    array (for callers that cannot allocate device memory)."""
+    _check(lib().bgtq_decode_attn_static_scratch(state, layer, layer_count, _ptr(d_q), _ptr(d_seq_lens), batch,
+                                                 _ptr(d_out), _stream(stream)))
 
 
 def bgtq_set_split_tokens(state, tokens):

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -463,6 +464,71 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split,
                            static_cast<__half*>(d_out), s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  return BGTQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Static-scratch decode: the split-K scratch lives in this library's own
+// device array instead of the caller's workspace.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_scratch[BGTQ_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_static_scratch for the current device (looked up once
+// per device, with that device current).
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BGTQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BGTQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return BGTQ_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return BGTQ_OK;
+}
+
+}  // namespace
+
+int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                                    const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream) {
+  if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
+  if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
+  const int split = split_for(st, layer_count, batch);
+  const int64_t nspl = (st->cfg.capacity_tokens + split - 1) / split;
+  const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
+  const size_t qrot_bytes = rows * kD * sizeof(float);
+  const size_t part_bytes = rows * size_t(nspl) * bgtq::kPartialStride * sizeof(float);
+  if (qrot_bytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES) return BGTQ_ERR_BUFFER_SIZE;
+  void* base = nullptr;
+  const int a = static_scratch_address(&base);
+  if (a != BGTQ_OK) return a;
+  // the same kernels as bgtq_decode_attn, with q~ and the partials redirected
+  // to the static array (partials packed with n_splits as their stride)
+  bgtq::Workspace ws = st->ws;
+  ws.qrot = static_cast<float*>(base);
+  ws.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + qrot_bytes);
+  bgtq::Shape shape = st->shape;
+  shape.max_splits = static_cast<int32_t>(nspl);
+  cudaStream_t s = as_stream(stream);
+  if (bgtq::launch_rotate_query(shape, ws, layer, layer_count, static_cast<const __half*>(d_q), batch, ws.qrot, s) !=
+      cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, ws.qrot, d_seq_lens, batch, split, s) !=
+      cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, static_cast<__half*>(d_out), s) !=
+      cudaSuccess)
     return BGTQ_ERR_CUDA;
   return BGTQ_OK;
 }

@@ -41,6 +41,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3b")
+    ap.add_argument("--layers", type=int, default=0, help="use only the first N layers (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp16-baseline", action="store_true")
     return ap.parse_args()
@@ -269,6 +270,8 @@ def main():
         return float(t.item())
 
     w = wl.WORKLOADS[args.workload]
+    if args.layers:
+        w = wl.scaled(w, n_layers=args.layers)
     lens = wl.seq_lens(w)
     L, H, HQ, B = w.n_layers, w.n_kv_heads, w.n_q_heads, w.batch
     cap = w.seq_len

@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   // Y tile
   const int rg = tid >> 4, og = tid & 15;
   const int i0 = og * 8;
-  if (i0 < npos) {
+  if (i0 < npos && rg * 4 < rows) {
     int gi[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -602,60 +602,83 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(Shape sh, Wor
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq), 128 threads.
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq), 256
+// threads: the 8 warps share the splits (lane = 4 rotated coordinates),
+// then o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), w_s = 2^(m_s - M).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) combine_kernel(Shape sh, Workspace ws, int layer0,
-                                                      const int32_t* __restrict__ seq_lens, int batch,
-                                                      int split_tokens, __half* __restrict__ out) {
+constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
+
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
+                                                               const int32_t* __restrict__ seq_lens, int batch,
+                                                               int split_tokens, __half* __restrict__ out) {
   const int hq = blockIdx.x % sh.n_q_heads;
   const int b = (blockIdx.x / sh.n_q_heads) % batch;
   const int li = blockIdx.x / (sh.n_q_heads * batch);
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
-  const int i = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int len = seq_lens[b];
   if (len < 0 || len > sh.capacity) {
-    if (i == 0 && hq == 0) atomicOr(ws.err, kErrSeqLen);
+    if (tid == 0 && hq == 0) atomicOr(ws.err, kErrSeqLen);
     len = 0;
   }
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
   const int nspl = (len + split_tokens - 1) / split_tokens;
   if (nspl == 0) {
-    out[row * kD + i] = __float2half(0.f);
+    if (tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
   }
   const float* part =
       ws.partials + ((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq) * sh.max_splits * kPartialStride;
-  __shared__ float wgt[1024];
-  __shared__ float red[4];
+  __shared__ float red[kCombWarps];
+  __shared__ float accs[kCombWarps][kD];
+  __shared__ float lsw[kCombWarps];
   __shared__ float a_s[kD];
   float M = -CUDART_INF_F;
-  for (int s = i; s < nspl; s += 128) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
+  for (int s = tid; s < nspl; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if ((i & 31) == 0) red[i >> 5] = M;
+  if (lane == 0) red[warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  float lsum = 0.f;
-  for (int s = i; s < nspl; s += 128) {
-    const float w = exp2f(part[static_cast<size_t>(s) * kPartialStride] - M);
-    wgt[s] = w;
-    lsum = fmaf(w, part[static_cast<size_t>(s) * kPartialStride + 1], lsum);
-  }
+  M = red[0];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if ((i & 31) == 0) red[i >> 5] = lsum;
+  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < nspl; s += kCombWarps) {
+    const float* p = part + static_cast<size_t>(s) * kPartialStride;
+    const float wgt = exp2f(p[0] - M);
+    lsum = fmaf(wgt, p[1], lsum);
+    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+    acc.x = fmaf(wgt, a.x, acc.x);
+    acc.y = fmaf(wgt, a.y, acc.y);
+    acc.z = fmaf(wgt, a.z, acc.z);
+    acc.w = fmaf(wgt, a.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
+  if (lane == 0) lsw[warp] = lsum;
   __syncthreads();
-  lsum = red[0] + red[1] + red[2] + red[3];
-  float a = 0.f;
-  for (int s = 0; s < nspl; ++s) a = fmaf(wgt[s], part[static_cast<size_t>(s) * kPartialStride + 4 + i], a);
-  a_s[i] = a / lsum;
+  if (tid < kD) {
+    float a = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      a += accs[w][tid];
+      l += lsw[w];
+    }
+    a_s[tid] = a / l;
+  }
   __syncthreads();
+  // inverse V rotation: thread pair (d, half) sums half of the 128 inputs
   const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  const int d = tid & (kD - 1), half = tid >> 7;
   float o = 0.f;
-  for (int r = 0; r < kD; ++r) o = fmaf(mv[r * kD + i], a_s[r], o);
-  out[row * kD + i] = __float2half(o);
+#pragma unroll 8
+  for (int r = half * 64; r < half * 64 + 64; ++r) o = fmaf(mv[r * kD + d], a_s[r], o);
+  if (half == 1) accs[0][d] = o;
+  __syncthreads();
+  if (half == 0) out[row * kD + d] = __float2half(o + accs[0][d]);
 }
 
 // Raises a kernel's dynamic shared-memory limit.  Callers keep the result
@@ -744,8 +767,8 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int split_tokens, __half* out,
                            cudaStream_t stream) {
-  combine_kernel<<<layer_count * batch * s.n_q_heads, kD, 0, stream>>>(s, ws, layer0, seq_lens, batch, split_tokens,
-                                                                       out);
+  combine_kernel<<<layer_count * batch * s.n_q_heads, kCombThreads, 0, stream>>>(s, ws, layer0, seq_lens, batch,
+                                                                                 split_tokens, out);
   return cudaGetLastError();
 }
 

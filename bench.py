@@ -184,7 +184,7 @@ class OracleSample:
         tb, l, h, k1, v1, q, enc = self.units[i % len(self.units)]
         t0 = time.perf_counter()
         model.encode_rows(tb, l, h, k1, v1)
-        model.decode(tb, l, h, q, enc["k_rec"], enc["k_norms"], enc["v_rec"], enc["v_norm"])
+        model.decode(tb, l, h, q, enc["k_tiles"], enc["k_norms"], enc["v_tiles"], enc["v_norm"], enc["n"])
         return time.perf_counter() - t0
 
     def step_seconds(self, unit_s):

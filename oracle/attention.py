@@ -9,19 +9,19 @@ over the dequantised cache:
     v_hat      = (n_V / sqrt(D))   * Pi_V^T C_bV[codes_V]
     out_h      = sum_t softmax_t(q_h . k_hat_t / sqrt(D)) v_hat_t
 
-with n the stored fp16 norms and C, Pi the fp32 tables, all in float64.
+with n the stored fp16 norms, C the fp16 codebook and Pi the fp32 rotations,
+all in float64.
 Query head h of the KV group reads the same cache.  Nothing here uses the
 rotated-domain shortcut of the GPU path; tests check that the two agree.
 """
 import numpy as np
 
-from .tqmse import unpack_records
+def dequantise_keys(codes, k_norms, groups, rotations, codebooks, head_dim):
+    """k_hat [T, D] float64 from record-order codes [T, P].
 
-
-def dequantise_keys(k_records, k_norms, groups, rotations, codebooks, head_dim):
-    """k_hat [T, D] float64.  groups: [(width, dims)]; rotations/codebooks keyed by width."""
-    widths = np.concatenate([np.full(len(dims), b, dtype=np.int64) for b, dims in groups])
-    codes = unpack_records(k_records, widths)
+    groups: [(width, dims)]; rotations/codebooks keyed by width.
+    """
+    codes = np.asarray(codes, dtype=np.int64)
     t = codes.shape[0]
     k_hat = np.zeros((t, head_dim), dtype=np.float64)
     pos = 0
@@ -35,10 +35,9 @@ def dequantise_keys(k_records, k_norms, groups, rotations, codebooks, head_dim):
     return k_hat
 
 
-def dequantise_values(v_records, v_norms, rotation, codebook, bits, head_dim):
-    """v_hat [T, D] float64 for the single uniform V group."""
-    codes = unpack_records(v_records, np.full(head_dim, bits, dtype=np.int64))
-    c = codebook.astype(np.float64)[codes]
+def dequantise_values(codes, v_norms, rotation, codebook, head_dim):
+    """v_hat [T, D] float64 for the single uniform V group from codes [T, D]."""
+    c = codebook.astype(np.float64)[np.asarray(codes, dtype=np.int64)]
     n = np.asarray(v_norms, dtype=np.float16).astype(np.float64)
     return (n / np.sqrt(float(head_dim)))[:, None] * (c @ rotation.astype(np.float64))
 

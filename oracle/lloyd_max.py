@@ -100,21 +100,29 @@ def mse(bits):
     return 1.0 - total
 
 
-def codebook_fp32(bits):
-    """The stored tables: centroids and thresholds rounded to fp32.
+def codebook_fp16(bits):
+    """The stored tables: centroids rounded once to binary16 (kept as exact
+    float32 values) and the cell boundaries at the exact midpoints of those
+    rounded centroids.
 
-    Thresholds are the float64 midpoints rounded once to fp32 (not midpoints
-    of the rounded centroids).
+    Reading: the pages leave the codebook's storage precision open; the
+    decode multiplies codes' centroids with fp16 operands, so the table is
+    the binary16 rounding of the float64 Lloyd-Max levels (a relative shift of
+    at most 2**-12 per level).  Thresholds are the nearest-neighbour cell
+    boundaries of that table: (C[k] + C[k+1]) / 2, exact in float32.
     """
-    return centroids(bits).astype(np.float32), thresholds(bits).astype(np.float32)
+    c16 = centroids(bits).astype(np.float16).astype(np.float32)
+    th = ((c16[:-1].astype(np.float64) + c16[1:].astype(np.float64)) / 2.0).astype(np.float32)
+    assert np.array_equal(th.astype(np.float64), (c16[:-1].astype(np.float64) + c16[1:].astype(np.float64)) / 2.0)
+    return c16, th
 
 
 def quantise(u, bits):
-    """Code of each element of ``u``: the number of fp32 thresholds <= u.
+    """Code of each element of ``u``: the number of thresholds <= u.
 
     A value equal to a threshold goes to the upper cell; u = 0 gives code
     2**(bits-1), the first positive centroid.  ``u`` may be float64 (the
     oracle) -- the thresholds are compared as their exact fp32 values.
     """
-    _, th = codebook_fp32(bits)
+    _, th = codebook_fp16(bits)
     return np.searchsorted(th.astype(np.float64), np.asarray(u, dtype=np.float64), side="right").astype(np.int64)

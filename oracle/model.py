@@ -5,20 +5,20 @@ attention) on plain arrays for one layer at a time.  The per-(layer, KV head)
 tables are the group layout from the allocation, one fp32 Haar rotation per
 K width group and one for V, and the fp32 Lloyd-Max codebooks.
 
-Cache record formats (the bytes the library writes, compared bit for bit):
-  K record  uint8[16 * k_avg_bits]  -- the bitstream of ``tqmse``
-  K norms   fp16[4]                 -- slot i = group i in width-descending
-                                       order; unused slots are +0
-  V record  uint8[16 * v_avg_bits]  -- V is one group of all D dims at the
-                                       uniform width v_avg_bits
-  V norm    fp16
+Cache contents (the bytes the library writes, compared bit for bit):
+  K tiles   uint8[1024 * k_avg_bits] per 64 positions -- ``tiles`` format
+  K norms   fp16[4] per position -- slot i = group i in width-descending
+            order; unused slots are +0
+  V tiles   uint8[1024 * v_avg_bits] per 64 positions -- V is one group of
+            all D dims at the uniform width v_avg_bits
+  V norm    fp16 per position
 """
 from dataclasses import dataclass
 
 import numpy as np
 
 from . import allocate as alloc
-from . import energy, haar, lloyd_max, tqmse
+from . import energy, haar, lloyd_max, tiles, tqmse
 from .attention import attend, dequantise_keys, dequantise_values
 
 KIND_K = 0
@@ -43,13 +43,6 @@ class Config:
     def group_size(self):
         return self.n_q_heads // self.n_kv_heads
 
-    @property
-    def k_record_bytes(self):
-        return self.k_avg_bits * self.head_dim // 8
-
-    @property
-    def v_record_bytes(self):
-        return self.v_avg_bits * self.head_dim // 8
 
 
 def allocate(cfg, calib_q, calib_k):
@@ -74,7 +67,7 @@ class Tables:
         self.block_widths = np.asarray(block_widths, dtype=np.int64)
         self.codebooks = {}
         for b in range(1, lloyd_max.MAX_BITS + 1):
-            self.codebooks[b] = lloyd_max.codebook_fp32(b)[0]
+            self.codebooks[b] = lloyd_max.codebook_fp16(b)[0]
         self.groups = {}
         self.k_rot = {}
         self.v_rot = {}
@@ -90,10 +83,10 @@ class Tables:
 
 
 def encode_rows(tables, layer, head, k_rows, v_rows):
-    """Encode rows of one (layer, KV head): fp16 [n, D] each.
+    """Encode rows of one (layer, KV head): fp16 [n, D] each, as cache positions 0..n-1.
 
-    Returns a dict with the cache bytes (k_rec, k_norms, v_rec, v_norm) and,
-    for diagnostics, the codes and the unrounded u values.
+    Returns a dict with the cache bytes (k_tiles, k_norms, v_tiles, v_norm;
+    the tiles padded with code 0 past row n) and the codes in record order.
     """
     cfg = tables.cfg
     k = np.asarray(k_rows, dtype=np.float16).astype(np.float64)
@@ -107,13 +100,11 @@ def encode_rows(tables, layer, head, k_rows, v_rows):
         k_codes.append(codes)
         k_norms[:, gi] = tqmse.fp16_round(norms)
     k_codes = np.concatenate(k_codes, axis=1) if k_codes else np.zeros((n, 0), dtype=np.int64)
-    k_rec = tqmse.pack_records(k_codes, tqmse.record_widths(groups), cfg.k_record_bytes)
     all_dims = np.arange(cfg.head_dim)
     v_codes, v_norm = tqmse.encode_group(v, all_dims, tables.v_rot[layer, head], cfg.v_avg_bits)
-    v_rec = tqmse.pack_records(v_codes, np.full(cfg.head_dim, cfg.v_avg_bits, dtype=np.int64),
-                               cfg.v_record_bytes)
-    return {"k_rec": k_rec, "k_norms": k_norms, "v_rec": v_rec,
-            "v_norm": tqmse.fp16_round(v_norm), "k_codes": k_codes, "v_codes": v_codes}
+    return {"k_tiles": tiles.pack_k_tiles(k_codes, groups, cfg.k_avg_bits), "k_norms": k_norms,
+            "v_tiles": tiles.pack_v_tiles(v_codes, cfg.v_avg_bits), "v_norm": tqmse.fp16_round(v_norm),
+            "k_codes": k_codes, "v_codes": v_codes, "n": n}
 
 
 def rotated_query(tables, layer, head, q):
@@ -127,12 +118,16 @@ def rotated_query(tables, layer, head, q):
     return np.concatenate(parts, axis=1)
 
 
-def decode(tables, layer, head, q, k_rec, k_norms, v_rec, v_norm):
-    """Decode attention of the G query heads of one KV head: out float64 [G, D]."""
+def decode(tables, layer, head, q, k_tiles, k_norms, v_tiles, v_norm, n):
+    """Decode attention of the G query heads of one KV head over positions
+    0..n-1 of the given tiles: out float64 [G, D]."""
     cfg = tables.cfg
-    k_hat = dequantise_keys(k_rec, k_norms, tables.groups[layer, head], tables.k_rot[layer, head],
-                            tables.codebooks, cfg.head_dim)
-    v_hat = dequantise_values(v_rec, v_norm, tables.v_rot[layer, head],
-                              tables.codebooks[cfg.v_avg_bits], cfg.v_avg_bits, cfg.head_dim)
+    groups = tables.groups[layer, head]
+    kc = tiles.unpack_k_tiles(k_tiles, groups, n) if n else np.zeros((0, 128), dtype=np.int64)
+    vc = tiles.unpack_v_tiles(v_tiles, cfg.v_avg_bits, n) if n else np.zeros((0, 128), dtype=np.int64)
+    k_hat = dequantise_keys(kc, np.asarray(k_norms)[:n], groups, tables.k_rot[layer, head], tables.codebooks,
+                            cfg.head_dim)
+    v_hat = dequantise_values(vc, np.asarray(v_norm)[:n], tables.v_rot[layer, head],
+                              tables.codebooks[cfg.v_avg_bits], cfg.head_dim)
     q64 = np.asarray(q, dtype=np.float16).astype(np.float64)
     return attend(q64, k_hat, v_hat)

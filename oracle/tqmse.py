@@ -54,48 +54,3 @@ def fp16_round(values):
 def record_widths(groups):
     """Per-position widths of a record, in record order."""
     return np.concatenate([np.full(len(dims), b, dtype=np.int64) for b, dims in groups])
-
-
-def pack_records(codes, widths, record_bytes):
-    """Pack codes [n, P] (record order) with per-position widths [P] into uint8 [n, record_bytes]."""
-    codes = np.asarray(codes, dtype=np.uint64)
-    widths = np.asarray(widths, dtype=np.int64)
-    n, p = codes.shape
-    assert p == len(widths)
-    total_bits = int(np.sum(widths))
-    assert total_bits <= 8 * record_bytes and record_bytes % 4 == 0
-    nwords = record_bytes // 4
-    acc = np.zeros((n, nwords + 1), dtype=np.uint64)
-    offset = 0
-    for k in range(p):
-        b = int(widths[k])
-        if b == 0:
-            continue
-        assert np.all(codes[:, k] < (1 << b))
-        w, sh = offset >> 5, offset & 31
-        val = codes[:, k] << np.uint64(sh)
-        acc[:, w] |= val & np.uint64(0xFFFFFFFF)
-        acc[:, w + 1] |= val >> np.uint64(32)
-        offset += b
-    assert np.all(acc[:, nwords] == 0)
-    words = acc[:, :nwords].astype(np.uint32)
-    return words.astype("<u4").view(np.uint8).reshape(n, record_bytes)
-
-
-def unpack_records(records, widths):
-    """Inverse of pack_records: uint8 [n, record_bytes] -> codes [n, P] int64."""
-    records = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
-    n, nbytes = records.shape
-    words = records.view("<u4").reshape(n, nbytes // 4).astype(np.uint64)
-    words = np.concatenate([words, np.zeros((n, 1), dtype=np.uint64)], axis=1)
-    out = np.zeros((n, len(widths)), dtype=np.int64)
-    offset = 0
-    for k, b in enumerate(widths):
-        b = int(b)
-        if b == 0:
-            continue
-        w, sh = offset >> 5, offset & 31
-        both = words[:, w] | (words[:, w + 1] << np.uint64(32))
-        out[:, k] = ((both >> np.uint64(sh)) & np.uint64((1 << b) - 1)).astype(np.int64)
-        offset += b
-    return out

@@ -42,7 +42,7 @@ def compare_codes(gpu_codes, ora_codes, ora_u, widths_per_pos):
     bad = np.argwhere(~eq)
     for r, p in bad:
         b = int(widths_per_pos[p])
-        th = lloyd_max.codebook_fp32(b)[1].astype(np.float64)
+        th = lloyd_max.codebook_fp16(b)[1].astype(np.float64)
         if np.min(np.abs(th - ora_u[r, p])) > THRESHOLD_SLACK or abs(int(gpu_codes[r, p]) - int(ora_codes[r, p])) != 1:
             ok = False
     return frac, ok, len(bad)

@@ -43,7 +43,7 @@ def _setup(w, dev, **over):
 def test_codebooks_bit_exact(dev):
     for b in range(1, 5):
         c, t = bgtq.bgtq_get_codebook(b)
-        oc, ot = lloyd_max.codebook_fp32(b)
+        oc, ot = lloyd_max.codebook_fp16(b)
         assert np.array_equal(c, oc) and np.array_equal(t, ot), b
 
 

@@ -50,9 +50,14 @@ def test_symmetry_and_midpoints(bits):
     assert np.array_equal(c, -c[::-1])
     assert t[len(t) // 2] == 0.0
     assert np.allclose(t, 0.5 * (c[:-1] + c[1:]), rtol=0, atol=0)
-    cf, tf = lm.codebook_fp32(bits)
+    cf, tf = lm.codebook_fp16(bits)
     assert cf.dtype == np.float32 and tf.dtype == np.float32
-    assert np.all(np.abs(cf.astype(np.float64) - c) <= np.abs(c) * 2.0 ** -24)
+    # the table is the binary16 rounding of the float64 levels (half an fp16 ulp)
+    assert np.array_equal(cf, c.astype(np.float16).astype(np.float32))
+    assert np.all(np.abs(cf.astype(np.float64) - c) <= np.abs(c) * 2.0 ** -11)
+    # thresholds: exact midpoints of the stored levels, symmetric, middle one 0
+    assert np.array_equal(tf.astype(np.float64), (cf[:-1].astype(np.float64) + cf[1:].astype(np.float64)) / 2)
+    assert np.array_equal(tf, -tf[::-1]) and tf[len(tf) // 2] == 0.0
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
@@ -74,7 +79,7 @@ def test_optimality_by_sampling(bits):
 def test_quantiser_is_nearest_centroid(bits):
     rng = np.random.default_rng(7)
     u = rng.standard_normal(100_000) * 1.5
-    cf, tf = lm.codebook_fp32(bits)
+    cf, tf = lm.codebook_fp16(bits)
     code = lm.quantise(u, bits)
     nearest = np.argmin(np.abs(u[:, None] - cf.astype(np.float64)[None, :]), axis=1)
     near_tie = np.min(np.abs(u[:, None] - tf.astype(np.float64)[None, :]), axis=1) < 1e-6

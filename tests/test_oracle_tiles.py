@@ -1,0 +1,109 @@
+"""Pins for oracle/tiles.py: the tile format's two renderings agree, it is a
+bijection on codes, and a hand-worked quartet."""
+import numpy as np
+import pytest
+
+from oracle import allocate as oalloc
+from oracle import tiles
+
+
+def test_quartet_golden(golden):
+    for row in golden("quartet_example.txt"):
+        b = int(row[0])
+        sel = [int(x, 16) for x in row[1:5]]
+        assert [f"{w:08X}" for w in tiles.quartet_pack(sel, b)] == row[5:]
+
+
+def _selectors_k(codes_tile, start, d, j, lane):
+    """Lane's four selector words for chunk j from the plain definition."""
+    out = []
+    for mu in range(4):
+        w = 0
+        for n in range(8):
+            token, coord = tiles._k_selector_member(mu, j, lane, n)
+            w |= int(codes_tile[token, start + coord]) << (4 * n)
+        out.append(w)
+    return out
+
+
+@pytest.mark.parametrize("widths_seed", range(6))
+def test_k_tile_quartets_match_the_plane_formulas(widths_seed):
+    rng = np.random.default_rng(widths_seed)
+    kavg = 2 + widths_seed % 2
+    bw = np.full(64, kavg)
+    idx = rng.permutation(64)
+    for a, c in zip(idx[:25], idx[25:50]):            # move bits, keeping the budget
+        if bw[a] < 4 and bw[c] > 1:
+            bw[a] += 1
+            bw[c] -= 1
+    groups = oalloc.group_layout(bw, 128, 0)
+    assert any(len(d) % 16 for _, d in groups) or widths_seed > 3
+    codes = np.concatenate([rng.integers(0, 1 << b, size=(64, len(d))) for b, d in groups], axis=1)
+    packed = tiles.pack_k_tiles(codes, groups, kavg)[0]
+    words = packed.view("<u4")
+    assert len(words) == 256 * kavg
+    off = 0
+    start = 0
+    for b, d in groups:
+        d = len(d)
+        for j in range(d // 16):
+            for lane in range(32):
+                expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, lane), b)
+                got = [int(words[off + 32 * k + lane]) for k in range(b)]
+                assert got == expect, (b, d, j, lane)
+            off += 32 * b
+        r = d % 16
+        if r:
+            off += 2 * r * b
+        start += d
+    assert off == len(words)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_round_trips(seed):
+    rng = np.random.default_rng(seed)
+    for _ in range(3):
+        bw = np.full(64, 3)
+        idx = rng.permutation(64)
+        # move bits between blocks keeping the sum (widths 1..4)
+        for a, c in zip(idx[:20], idx[20:40]):
+            if bw[a] < 4 and bw[c] > 1:
+                bw[a] += 1
+                bw[c] -= 1
+        groups = oalloc.group_layout(bw, 128, 0)
+        n = int(rng.integers(1, 300))
+        codes = np.concatenate([rng.integers(0, 1 << b, size=(n, len(d))) for b, d in groups], axis=1)
+        t = tiles.pack_k_tiles(codes, groups, 3)
+        assert t.shape == ((n + 63) // 64, 3072)
+        assert np.array_equal(tiles.unpack_k_tiles(t, groups, n), codes)
+        for vb in (1, 2, 3, 4):
+            vc = rng.integers(0, 1 << vb, size=(n, 128))
+            vt = tiles.pack_v_tiles(vc, vb)
+            assert vt.shape == ((n + 63) // 64, 1024 * vb)
+            assert np.array_equal(tiles.unpack_v_tiles(vt, vb, n), vc)
+
+
+def test_v_tile_layout_matches_fragment_order():
+    """Word (m, k, lane) holds plane k of the lane's quartet for dim-tile m."""
+    rng = np.random.default_rng(9)
+    vc = rng.integers(0, 8, size=(64, 128))
+    words = tiles.pack_v_tiles(vc, 3)[0].view("<u4")
+    for m in (0, 5, 7):
+        for lane in (0, 13, 31):
+            sel = []
+            for kappa in range(4):
+                w = 0
+                for n in range(8):
+                    token, coord = tiles._v_selector_member(m, kappa, lane, n)
+                    w |= int(vc[token, coord]) << (4 * n)
+                sel.append(w)
+            assert [int(words[m * 96 + 32 * k + lane]) for k in range(3)] == tiles.quartet_pack(sel, 3)
+
+
+def test_every_code_bit_stored_once():
+    groups = oalloc.group_layout(np.array([4] * 10 + [3] * 30 + [2] * 14 + [1] * 10), 128, 0)
+    tok, pos, cb = tiles.k_tile_bitmap(tiles.group_spec(groups))
+    widths = np.concatenate([np.full(len(d), b) for b, d in groups])
+    keys = set(zip(tok.tolist(), pos.tolist(), cb.tolist()))
+    assert len(keys) == len(tok) == 64 * int(widths.sum())
+    assert all(c < widths[p] for _, p, c in keys)

@@ -34,11 +34,17 @@ index 32 k + L).  K quartets: one per full chunk, s_mu for mu = 0..3.  V
 quartets: one per dim-tile m, s_kappa for kappa = 0..3.
 
 K tile (1024 * k_avg_bits bytes): group regions widest group first; in each,
-the full chunks' quartets in chunk order, then the partial chunk as a dense
-LSB-first bitstream in little-endian 32-bit words holding every lane's real
-codes, lanes in order, inside a lane M-tile major then nibble order, b bits
-each (a nibble is real when its coordinate is < d).  V tile (1024 *
-v_avg_bits bytes): the 8 dim-tiles' quartets in order.
+the full chunks' quartets in chunk order (b x 32 words each), then the
+partial chunk (r = d - 16j coordinates, r even):
+  * lanes with a full quad (t < nf = r // 4) store their quartet as above,
+    word k of lane (g, t) at index 8 nf k + (g nf + t);
+  * if r % 4 == 2, the eight lanes with t = nf hold two real members per
+    token (nibbles 0, 1, 4, 5).  Their half selectors -- those nibbles moved
+    to nibbles 0..3 -- are paired into four virtual lanes V = g // 2 (lane
+    2V in bits 0..15, lane 2V+1 in bits 16..31) stored as quartets, word k
+    of V at index 8 nf b + 4 k + V.
+  The partial chunk takes 2 r b words, so the tile is dense.
+V tile (1024 * v_avg_bits bytes): the 8 dim-tiles' quartets in order.
 """
 import functools
 
@@ -46,6 +52,7 @@ import numpy as np
 
 TILE = 64
 V_MEMBERS = (0, 1, 8, 9)          # token offsets 2t + V_MEMBERS[n % 4]
+HALF_NIBBLES = (0, 1, 4, 5)       # the real nibbles of a half quad
 
 
 def _quartet_source(b, k, p):
@@ -76,8 +83,7 @@ def k_tile_bitmap(group_spec):
 
     group_spec: tuple of (width, size) per group in record order.  Returns
     int arrays (token, position, code_bit), one entry per tile bit (bit q of
-    32-bit word w is entry 32 w + q); position -1 marks an unused bit (none
-    in a well-formed layout).
+    32-bit word w is entry 32 w + q); every bit of the tile holds a code bit.
     """
     tok, pos, cb = [], [], []
     start = 0
@@ -94,19 +100,28 @@ def k_tile_bitmap(group_spec):
                         cb.append(bit)
         r = d - 16 * n_full
         if r:
-            stream = []
-            for lane in range(32):
-                for mu in range(4):
-                    for n in range(8):
-                        token, coord = _k_selector_member(mu, n_full, lane, n)
-                        if coord < d:
-                            stream.append((token, start + coord))
-            for token, position in stream:
-                for bit in range(b):
-                    tok.append(token)
-                    pos.append(position)
-                    cb.append(bit)
-            assert len(stream) * b % 32 == 0
+            nf = r // 4
+            for k in range(b):
+                for g in range(8):
+                    for t in range(nf):
+                        for p in range(32):
+                            s, n, bit = _quartet_source(b, k, p)
+                            token, coord = _k_selector_member(s, n_full, 4 * g + t, n)
+                            tok.append(token)
+                            pos.append(start + coord)
+                            cb.append(bit)
+            if r % 4:
+                for k in range(b):
+                    for v in range(4):
+                        for p in range(32):
+                            s, nv, bit = _quartet_source(b, k, p)
+                            g = 2 * v + nv // 4
+                            n = HALF_NIBBLES[nv % 4]
+                            token, coord = _k_selector_member(s, n_full, 4 * g + nf, n)
+                            assert coord < d
+                            tok.append(token)
+                            pos.append(start + coord)
+                            cb.append(bit)
         start += d
     return np.array(tok), np.array(pos), np.array(cb)
 

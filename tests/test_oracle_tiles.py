@@ -15,13 +15,15 @@ def test_quartet_golden(golden):
 
 
 def _selectors_k(codes_tile, start, d, j, lane):
-    """Lane's four selector words for chunk j from the plain definition."""
+    """Lane's four selector words for chunk j from the plain definition
+    (nibbles whose coordinate is past the group are 0)."""
     out = []
     for mu in range(4):
         w = 0
         for n in range(8):
             token, coord = tiles._k_selector_member(mu, j, lane, n)
-            w |= int(codes_tile[token, start + coord]) << (4 * n)
+            if coord < d:
+                w |= int(codes_tile[token, start + coord]) << (4 * n)
         out.append(w)
     return out
 
@@ -54,6 +56,22 @@ def test_k_tile_quartets_match_the_plane_formulas(widths_seed):
             off += 32 * b
         r = d % 16
         if r:
+            j = d // 16
+            nf = r // 4
+            for g in range(8):
+                for t in range(nf):
+                    expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, 4 * g + t), b)
+                    got = [int(words[off + 8 * nf * k + g * nf + t]) for k in range(b)]
+                    assert got == expect, ("partial full lane", b, d, g, t)
+            if r % 4:
+                for v in range(4):
+                    halves = []
+                    for g in (2 * v, 2 * v + 1):
+                        sel = _selectors_k(codes, start, d, j, 4 * g + nf)       # padding nibbles are 0
+                        halves.append([(w & 0xFF) | ((w >> 8) & 0xFF00) for w in sel])
+                    virt = [halves[0][mu] | (halves[1][mu] << 16) for mu in range(4)]
+                    got = [int(words[off + 8 * nf * b + 4 * k + v]) for k in range(b)]
+                    assert got == tiles.quartet_pack(virt, b), ("partial half lanes", b, d, v)
             off += 2 * r * b
         start += d
     assert off == len(words)

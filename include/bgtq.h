@@ -31,14 +31,19 @@
  *    aligned.
  *
  * Cache layout inside d_cache (offsets from bgtq_cache_offsets, each
- * 256-byte aligned; L layers, B = max_batch, H = n_kv_heads, C = capacity):
- *   K records  uint8 [L][B][H][C][16*k_avg_bits]   LSB-first bitstream of
- *              the codes in little-endian 32-bit words; width groups in
- *              descending width, rotated-coordinate order inside a group
- *   K norms    fp16  [L][B][H][C][4]   slot i = norm of group i (width
+ * 256-byte aligned; L layers, B = max_batch, H = n_kv_heads, T =
+ * ceil(capacity / 64) tiles of 64 positions per (layer, sequence, head)):
+ *   K tiles    uint8 [L][B][H][T][1024*k_avg_bits]  codes of 64 positions,
+ *              laid out for the tensor-core decode (per lane, the nibble
+ *              selectors of its mma A-fragments as bit planes; width groups
+ *              widest first; see the tile-format definition shipped with
+ *              the tests' CPU oracle)
+ *   K norms    fp16  [L][B][H][T*64][4]   slot i = norm of group i (width
  *              descending); unused slots 0
- *   V records  uint8 [L][B][H][C][16*v_avg_bits]  same bitstream, one group
- *   V norms    fp16  [L][B][H][C]
+ *   V tiles    uint8 [L][B][H][T][1024*v_avg_bits]  same scheme, one group
+ *   V norms    fp16  [L][B][H][T*64]
+ * Codebook: the N(0,1) Lloyd-Max levels for 1..4 bits rounded once to
+ * binary16; thresholds are the exact midpoints of those levels.
  */
 #ifndef BGTQ_H
 #define BGTQ_H
@@ -66,7 +71,9 @@ enum {
 enum {
   BGTQ_DEVERR_CAPACITY = 1,    /* encode_append: start + count > capacity (rows skipped) */
   BGTQ_DEVERR_SEQ_LEN = 2,     /* decode_attn: a seq_len < 0 or > capacity (sequence skipped, output 0) */
-  BGTQ_DEVERR_ARG = 4          /* encode_append: start < 0 or count < 0 or count > n */
+  BGTQ_DEVERR_ARG = 4,         /* encode_append: start < 0 or count < 0 or count > n */
+  BGTQ_DEVERR_NONFINITE = 8,   /* allocate: a calibration value is Inf or NaN */
+  BGTQ_DEVERR_TIMEOUT = 16     /* decode: a wait for a tile copy gave up (bounded spin) */
 };
 
 typedef struct {
@@ -136,8 +143,9 @@ int bgtq_get_allocation(const bgtq_state* st, int8_t* h_widths);
  *   h_eq, h_ek  uint64 [n_layers][n_kv_heads][64][2].  SYNC. */
 int bgtq_get_energy(const bgtq_state* st, uint64_t* h_eq, uint64_t* h_ek);
 
-/* The fp32 Lloyd-Max codebook for bits in 1..4 (TurboQuant's scalar
- * quantiser on N(0,1)): h_centroids[2^bits], h_thresholds[2^bits - 1]. */
+/* The Lloyd-Max codebook for bits in 1..4 (TurboQuant's scalar quantiser on
+ * N(0,1)) as stored: h_centroids[2^bits] (binary16 values as floats),
+ * h_thresholds[2^bits - 1] (their midpoints). */
 int bgtq_get_codebook(int32_t bits, float* h_centroids, float* h_thresholds);
 
 /* Group layout of (layer, kv_head): *n_groups, per group its width and size
@@ -153,7 +161,7 @@ int bgtq_get_rotation(const bgtq_state* st, int32_t layer, int32_t kv_head, int3
                       int32_t group, float* h_out, int32_t* d);
 
 /* Byte offsets of the four cache arrays inside d_cache:
- * out[0] K records, out[1] K norms, out[2] V records, out[3] V norms. */
+ * out[0] K tiles, out[1] K norms, out[2] V tiles, out[3] V norms. */
 int bgtq_cache_offsets(const bgtq_state* st, size_t* out);
 
 /* TQ-MSE encode + bit-pack of new rows into the cache.  For each layer
@@ -230,9 +238,9 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
                                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
 
 /* Tokens per split-K chunk for bgtq_decode_attn: 0 = automatic (from
- * capacity, max_splits and the SM count), else a multiple of 64 with
- * ceil(capacity / tokens) <= max_splits.  Results do not depend on it beyond
- * floating-point reassociation. */
+ * capacity, max_splits and the SM count), else a multiple of 64 (one tile)
+ * with ceil(capacity / tokens) <= max_splits.  Results do not depend on it
+ * beyond floating-point reassociation. */
 int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens);
 
 /* Synchronises "stream", reads the device error flag into *h_flags

@@ -18,11 +18,13 @@ LIB_PATH = os.path.join(_PKG, "libbgtq.so")
 
 HEAD_DIM = 128
 N_BLOCKS = HEAD_DIM // 2
+TILE = 64
 
 DEVERR_CAPACITY = 1
 DEVERR_SEQ_LEN = 2
 DEVERR_ARG = 4
 DEVERR_NONFINITE = 8
+DEVERR_TIMEOUT = 16
 
 
 class BgtqError(RuntimeError):
@@ -291,27 +293,31 @@ class PackedKVCache:
             pass
 
     # -- views of the cache arrays (no copies) --
-    def _tokens(self):
+    def _tiles(self):
         c = self.cfg
-        return (c.n_layers, c.max_batch, c.n_kv_heads, c.capacity_tokens)
+        return (c.n_layers, c.max_batch, c.n_kv_heads, (c.capacity_tokens + TILE - 1) // TILE)
 
-    def k_records(self):
-        n = int(np.prod(self._tokens())) * 16 * self.cfg.k_avg_bits
-        return self.cache[self.offsets[0]:self.offsets[0] + n].view(*self._tokens(), 16 * self.cfg.k_avg_bits)
+    def k_tiles(self):
+        t = self._tiles()
+        n = int(np.prod(t)) * 1024 * self.cfg.k_avg_bits
+        return self.cache[self.offsets[0]:self.offsets[0] + n].view(*t, 1024 * self.cfg.k_avg_bits)
 
     def k_norms(self):
         import torch
-        n = int(np.prod(self._tokens())) * 8
-        return self.cache[self.offsets[1]:self.offsets[1] + n].view(torch.float16).view(*self._tokens(), 4)
+        t = self._tiles()
+        n = int(np.prod(t)) * TILE * 8
+        return self.cache[self.offsets[1]:self.offsets[1] + n].view(torch.float16).view(*t[:3], t[3] * TILE, 4)
 
-    def v_records(self):
-        n = int(np.prod(self._tokens())) * 16 * self.cfg.v_avg_bits
-        return self.cache[self.offsets[2]:self.offsets[2] + n].view(*self._tokens(), 16 * self.cfg.v_avg_bits)
+    def v_tiles(self):
+        t = self._tiles()
+        n = int(np.prod(t)) * 1024 * self.cfg.v_avg_bits
+        return self.cache[self.offsets[2]:self.offsets[2] + n].view(*t, 1024 * self.cfg.v_avg_bits)
 
     def v_norms(self):
         import torch
-        n = int(np.prod(self._tokens())) * 2
-        return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*self._tokens())
+        t = self._tiles()
+        n = int(np.prod(t)) * TILE * 2
+        return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*t[:3], t[3] * TILE)
 
     # -- calls --
     def allocate(self, calib_q, calib_k):

@@ -62,13 +62,17 @@ struct Layout {
   size_t err, codebook, layouts, mkt, mvt, mv, energy_q, energy_k, qrot, partials, ws_total;
 };
 
+int64_t tiles_of(const bgtq_config* c) { return (c->capacity_tokens + bgtq::kTile - 1) / bgtq::kTile; }
+
 Layout plan(const bgtq_config* c) {
   Layout p{};
-  const size_t toks = size_t(c->n_layers) * c->max_batch * c->n_kv_heads * size_t(c->capacity_tokens);
+  const size_t seqs = size_t(c->n_layers) * c->max_batch * c->n_kv_heads;
+  const size_t tiles = seqs * size_t(tiles_of(c));
+  const size_t toks = tiles * bgtq::kTile;
   p.krec = 0;
-  p.knorm = align_up(p.krec + toks * 16 * c->k_avg_bits);
+  p.knorm = align_up(p.krec + tiles * 1024 * c->k_avg_bits);
   p.vrec = align_up(p.knorm + toks * 4 * sizeof(uint16_t));
-  p.vnorm = align_up(p.vrec + toks * 16 * c->v_avg_bits);
+  p.vnorm = align_up(p.vrec + tiles * 1024 * c->v_avg_bits);
   p.cache_total = align_up(p.vnorm + toks * sizeof(uint16_t));
   const size_t lh = size_t(c->n_layers) * c->n_kv_heads;
   p.err = 0;
@@ -118,6 +122,15 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
         d.inv_sqrt_d[g] = lay.size[g] > 0 ? static_cast<float>(1.0 / std::sqrt(double(lay.size[g]))) : 0.f;
       }
       for (int i = 0; i < kD; ++i) d.perm[i] = lay.perm[i];
+      int word = 0, chunk = 0;
+      for (int g = 0; g < bgtq::kNumGroupsMax; ++g) {
+        d.tile_word[g] = word;
+        d.chunk_base[g] = chunk;
+        if (g < lay.n_groups) {
+          word += 2 * lay.size[g] * lay.width[g];  // 64 positions x d x b bits
+          chunk += (lay.size[g] + 15) / 16;
+        }
+      }
       float* mk = mkt.data() + lh * kD * kD;
       for (int g = 0; g < lay.n_groups; ++g) {
         const int dg = lay.size[g], s0 = lay.start[g];
@@ -155,14 +168,16 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   return BGTQ_OK;
 }
 
+// Tokens per split-K chunk: about two CTAs per SM over the launch (the decode
+// kernel fits two per SM), in whole tiles, within max_splits.
 int auto_split_tokens(const bgtq_state* st, int units) {
   const int64_t cap = st->cfg.capacity_tokens;
   const int maxs = max_splits_of(&st->cfg);
-  const int target = 8 * st->num_sms;
-  int nspl = std::max(1, std::min(maxs, (target + units - 1) / std::max(units, 1)));
+  const int target = 2 * st->num_sms;
+  const int nspl = std::max(1, std::min(maxs, (target + units - 1) / std::max(units, 1)));
   int64_t t = (cap + nspl - 1) / nspl;
-  t = std::max<int64_t>(256, (t + 255) / 256 * 256);
-  while ((cap + t - 1) / t > maxs) t += 256;
+  t = (t + bgtq::kTile - 1) / bgtq::kTile * bgtq::kTile;
+  while ((cap + t - 1) / t > maxs) t += bgtq::kTile;
   return static_cast<int>(t);
 }
 
@@ -200,10 +215,11 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->shape.vbits = cfg->v_avg_bits;
   st->shape.max_splits = max_splits_of(cfg);
   st->shape.capacity = cfg->capacity_tokens;
+  st->shape.ntiles = tiles_of(cfg);
   uint8_t* c8 = static_cast<uint8_t*>(d_cache);
-  st->cache.krec = c8 + p.krec;
+  st->cache.ktile = reinterpret_cast<uint32_t*>(c8 + p.krec);
   st->cache.knorm = reinterpret_cast<__half*>(c8 + p.knorm);
-  st->cache.vrec = c8 + p.vrec;
+  st->cache.vtile = reinterpret_cast<uint32_t*>(c8 + p.vrec);
   st->cache.vnorm = reinterpret_cast<__half*>(c8 + p.vnorm);
   st->cache_off[0] = p.krec;
   st->cache_off[1] = p.knorm;
@@ -418,7 +434,9 @@ int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, 
 }
 
 int split_for(const bgtq_state* st, int32_t layer_count, int32_t batch) {
-  return st->split_tokens > 0 ? st->split_tokens : auto_split_tokens(st, batch * st->cfg.n_kv_heads * layer_count);
+  const int head_blocks = (st->shape.group + 7) / 8;
+  return st->split_tokens > 0 ? st->split_tokens
+                              : auto_split_tokens(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count);
 }
 
 }  // namespace

@@ -11,7 +11,9 @@ constexpr int kD = 128;               // head_dim
 constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
 constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
 constexpr int kPartialStride = 132;   // floats per split-K partial: m, l, pad, pad, acc[128]
-constexpr int kSplitGranule = 64;     // split sizes are multiples of this many tokens
+constexpr int kTile = 64;             // cache positions per packed tile
+constexpr int kSplitGranule = kTile;  // split sizes are multiples of the tile
+constexpr int kMaxChunks = 12;        // 16-coordinate K chunks per head (8 + one partial per group)
 
 // Per-(layer, KV head) K layout.  Positions are record order: group 0
 // (widest) first; perm maps a position to the original dim.
@@ -25,7 +27,8 @@ struct alignas(16) LayoutDev {
   int32_t bitoff[kNumGroupsMax];
   float inv_sqrt_d[kNumGroupsMax];    // 1 / sqrt(d_g)
   int32_t perm[kD];
-  int32_t pad2[8];
+  int32_t tile_word[kNumGroupsMax];   // first 32-bit word of the group's region in a K tile
+  int32_t chunk_base[kNumGroupsMax];  // index of the group's first 16-coordinate chunk
 };
 static_assert(sizeof(LayoutDev) == 640, "layout record size");
 
@@ -49,17 +52,19 @@ struct Workspace {
   float* partials;               // [L][B][Hq][max_splits][kPartialStride]
 };
 
+// Cache arrays; T = ceil(capacity / 64) tiles per (layer, sequence, KV head).
 struct CacheDev {
-  uint8_t* krec;                 // [L][B][Hkv][C][16*kbits]
-  __half* knorm;                 // [L][B][Hkv][C][4]
-  uint8_t* vrec;                 // [L][B][Hkv][C][16*vbits]
-  __half* vnorm;                 // [L][B][Hkv][C]
+  uint32_t* ktile;               // [L][B][Hkv][T][256*kbits] words (tile format)
+  __half* knorm;                 // [L][B][Hkv][T*64][4]
+  uint32_t* vtile;               // [L][B][Hkv][T][256*vbits] words
+  __half* vnorm;                 // [L][B][Hkv][T*64]
 };
 
 struct Shape {
   int32_t n_layers, n_kv_heads, n_q_heads, group, max_batch;
   int32_t kbits, vbits, max_splits;
   int64_t capacity;
+  int64_t ntiles;                // tiles per (layer, sequence, KV head)
 };
 
 // Error flag bits (same values as BGTQ_DEVERR_* in bgtq.h).
@@ -67,6 +72,7 @@ constexpr uint32_t kErrCapacity = 1;
 constexpr uint32_t kErrSeqLen = 2;
 constexpr uint32_t kErrArg = 4;
 constexpr uint32_t kErrNonFinite = 8;
+constexpr uint32_t kErrTimeout = 16;
 
 // Launchers (kernels.cu).  Each returns the cudaError_t of its launch.
 cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,

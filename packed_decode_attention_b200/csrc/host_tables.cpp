@@ -70,17 +70,28 @@ uint64_t mix64(uint64_t z) {
 
 }  // namespace
 
+// Round a double to the nearest binary16 value (ties to even), returned as a
+// double; normal range only (the codebook levels lie in [0.12, 2.8]).
+double round_to_fp16(double x) {
+  if (x == 0.0) return 0.0;
+  int e = 0;
+  const double m = std::frexp(x, &e);            // x = m * 2^e, 0.5 <= |m| < 1
+  const double q = std::nearbyint(std::ldexp(m, 11));  // 11 significant bits, to nearest even
+  return std::ldexp(q, e - 11);
+}
+
 void lloyd_max_codebook(int bits, std::vector<float>* centroids, std::vector<float>* thresholds) {
   const std::vector<double> pos = positive_levels(bits);
   const int half = static_cast<int>(pos.size());
   std::vector<double> all(2 * half);
   for (int k = 0; k < half; ++k) {
-    all[half + k] = pos[k];
-    all[half - 1 - k] = -pos[k];
+    all[half + k] = round_to_fp16(pos[k]);
+    all[half - 1 - k] = -round_to_fp16(pos[k]);
   }
   centroids->resize(2 * half);
   thresholds->resize(2 * half - 1);
   for (int k = 0; k < 2 * half; ++k) (*centroids)[k] = static_cast<float>(all[k]);
+  // midpoints of binary16 values are exact in float32
   for (int k = 0; k + 1 < 2 * half; ++k) (*thresholds)[k] = static_cast<float>(0.5 * (all[k] + all[k + 1]));
 }
 

@@ -15,8 +15,8 @@ constexpr int kMaxGroups = 4;
 // model (six-digit constants, index = width).
 extern const double kDistortion[kMaxBits + 1];
 
-// Codebook of 2^bits levels: ascending centroids and the 2^bits-1 midpoints,
-// both computed in double and rounded once to fp32.
+// Codebook of 2^bits levels: the double Lloyd-Max levels rounded once to
+// binary16 (held as exact floats) and the 2^bits-1 exact midpoints.
 void lloyd_max_codebook(int bits, std::vector<float>* centroids, std::vector<float>* thresholds);
 
 // SplitMix64 (Steele, Lea, Flood 2014).

@@ -1,9 +1,9 @@
 // CUDA kernels of the Block-GTQ packed-cache path for B200 (sm_100a).
 //
 //   energy_kernel        label-free per-RoPE-block Q/K energy, exact 128-bit sums
-//   encode_kernel<KIND>  TQ-MSE: rotate (fp32), normalise (fp64), quantise, bit-pack
+//   encode_kernel        TQ-MSE: rotate (fp32), normalise (fp64), quantise, pack tiles
 //   rotate_query_kernel  q~ per width group (rotated basis, 1/sqrt(d_g), 1/sqrt(D))
-//   decode_split_kernel  split-K flash decoding straight from the packed codes
+//   decode_mma_kernel    split-K flash decoding from the packed tiles (mma.sync)
 //   combine_kernel       log-sum-exp merge of the splits + inverse V rotation
 //
 // Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (Block-GTQ;
@@ -84,36 +84,310 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
   if (bad) atomicOr(err, kErrNonFinite);
 }
 
+
 // ---------------------------------------------------------------------------
-// a3: encode.  Grid (layer_count * batch * Hkv, ceil(n / 64)), 256 threads.
-// Each CTA: 64 rows of one (layer, sequence, KV head).  Y = X R^T as a
-// 64 x 128 x 128 fp32 register-tiled product (4 rows x 8 outputs per
-// thread); the K rotation is block diagonal in record order, so each thread
-// only runs over the groups its outputs fall in.
+// Tile format helpers.  A 64-position tile stores each lane's mma A-fragment
+// selectors (8 nibble codes per 32-bit word) as bit-plane "quartets":
+//   b = 1: P = s0&M1 | (s1&M1)<<1 | (s2&M1)<<2 | (s3&M1)<<3
+//   b = 2: A = s0&M3 | (s1&M3)<<2,  B = s2&M3 | (s3&M3)<<2
+//   b = 3: A, B and H = (s0&M4)>>2 | (s1&M4)>>1 | s2&M4 | (s3&M4)<<1
+//   b = 4: s0..s3
+// K selector (chunk j, M-tile mu, lane 4g+t) nibble n: token 16mu+g+8(n>=4),
+// group coordinate 16j+4t+n%4.  V selector (dim tile m, token step kappa):
+// coordinate 16m+g+8(n>=4), token 16kappa+(2t,2t+1,2t+8,2t+9)[n%4].
 // ---------------------------------------------------------------------------
-constexpr int kEncRows = 64;
+constexpr uint32_t M1 = 0x11111111u, M3 = 0x33333333u, M4 = 0x44444444u;
+
+template <int B>
+__device__ __forceinline__ void quartet_decode(const uint32_t* w, uint32_t* s) {
+  if constexpr (B == 4) {
+    s[0] = w[0]; s[1] = w[1]; s[2] = w[2]; s[3] = w[3];
+  } else if constexpr (B == 3) {
+    s[0] = (w[0] & M3) | ((w[2] << 2) & M4);
+    s[1] = ((w[0] >> 2) & M3) | ((w[2] << 1) & M4);
+    s[2] = (w[1] & M3) | (w[2] & M4);
+    s[3] = ((w[1] >> 2) & M3) | ((w[2] >> 1) & M4);
+  } else if constexpr (B == 2) {
+    s[0] = w[0] & M3; s[1] = (w[0] >> 2) & M3; s[2] = w[1] & M3; s[3] = (w[1] >> 2) & M3;
+  } else {
+    s[0] = w[0] & M1; s[1] = (w[0] >> 1) & M1; s[2] = (w[0] >> 2) & M1; s[3] = (w[0] >> 3) & M1;
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void quartet_encode(const uint32_t* s, uint32_t* w) {
+  if constexpr (B == 4) {
+    w[0] = s[0]; w[1] = s[1]; w[2] = s[2]; w[3] = s[3];
+  } else if constexpr (B == 1) {
+    w[0] = (s[0] & M1) | ((s[1] & M1) << 1) | ((s[2] & M1) << 2) | ((s[3] & M1) << 3);
+  } else {
+    w[0] = (s[0] & M3) | ((s[1] & M3) << 2);
+    w[1] = (s[2] & M3) | ((s[3] & M3) << 2);
+    if constexpr (B == 3) w[2] = ((s[0] & M4) >> 2) | ((s[1] & M4) >> 1) | (s[2] & M4) | ((s[3] & M4) << 1);
+  }
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Byte tables of the fp16 codebook: lo[i] / hi[i] hold the low / high bytes
+// of entries 4i .. 4i+3.
+struct ByteTab {
+  uint32_t lo[4], hi[4];
+};
+
+// Four codes (selector nibbles 0..3) -> two fp16x2 registers: codes (0, 1)
+// and codes (2, 3).  PRMT picks bytes 0..7 of its two table words by the
+// nibble's low three bits; width-4 codes look up both halves of the table
+// and pick by their top bit.
+template <int B>
+__device__ __forceinline__ void lookup4(const ByteTab& t, uint32_t sel, uint32_t& r01, uint32_t& r23) {
+  uint32_t lo, hi;
+  if constexpr (B <= 3) {
+    lo = prmt(t.lo[0], t.lo[1], sel);
+    hi = prmt(t.hi[0], t.hi[1], sel);
+  } else {
+    const uint32_t s7 = sel & 0x7777u;
+    const uint32_t pick = 0x3210u | ((sel >> 1) & 0x4444u);
+    lo = prmt(prmt(t.lo[0], t.lo[1], s7), prmt(t.lo[2], t.lo[3], s7), pick);
+    hi = prmt(prmt(t.hi[0], t.hi[1], s7), prmt(t.hi[2], t.hi[3], s7), pick);
+  }
+  r01 = prmt(lo, hi, 0x5140u);
+  r23 = prmt(lo, hi, 0x7362u);
+}
+
+// D += A * B for one m16n8k16 tile, fp16 operands, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// A-fragment from one selector word (rows g and g+8) times a B-fragment.
+template <int B>
+__device__ __forceinline__ void mma_selector(float* c, const ByteTab& t, uint32_t s, uint32_t b0, uint32_t b1) {
+  uint32_t r0, r1, r2, r3;
+  lookup4<B>(t, s, r0, r2);
+  lookup4<B>(t, s >> 16, r1, r3);
+  mma16816(c, r0, r1, r2, r3, b0, b1);
+}
+
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(x));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void fill_bytetab(ByteTab& t, const float* centroids, int bits) {
+  uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+  const int n = 1 << bits;
+  for (int e = 0; e < n; ++e) {
+    const uint32_t h = __half_as_ushort(__float2half_rn(centroids[e]));
+    lo[e >> 2] |= (h & 0xFFu) << (8 * (e & 3));
+    hi[e >> 2] |= (h >> 8) << (8 * (e & 3));
+  }
+  for (int i = 0; i < 4; ++i) {
+    t.lo[i] = lo[i];
+    t.hi[i] = hi[i];
+  }
+}
+
+// Group geometry of a K layout (record order, widest group first).
+struct GroupGeo {
+  int width, d, nfull, r, word, chunk, start;
+};
+
+__device__ __forceinline__ GroupGeo group_geo(const LayoutDev& lay, int g) {
+  GroupGeo q;
+  q.width = lay.width[g];
+  q.d = lay.size[g];
+  q.nfull = q.d >> 4;
+  q.r = q.d & 15;
+  q.word = lay.tile_word[g];
+  q.chunk = lay.chunk_base[g];
+  q.start = lay.start[g];
+  return q;
+}
+
+// ---- tile unpack / pack over a CTA (codes[64][128] in shared memory) ----
+
+// The lane's selector for chunk j, M-tile mu: token and group coordinate of nibble n.
+__device__ __forceinline__ int k_token(int mu, int lane, int n) { return 16 * mu + (lane >> 2) + 8 * (n >= 4); }
+__device__ __forceinline__ int k_coord(int j, int lane, int n) { return 16 * j + 4 * (lane & 3) + (n & 3); }
+
+template <int B>
+__device__ void unpack_k_group(const uint32_t* tw, const GroupGeo& q, uint8_t (*codes)[kD], int tid, int nthreads) {
+  const uint32_t* gw = tw + q.word;
+  for (int u = tid; u < q.nfull * 32; u += nthreads) {
+    const int j = u >> 5, lane = u & 31;
+    uint32_t w[B], s[4];
+    for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
+    quartet_decode<B>(w, s);
+    for (int mu = 0; mu < 4; ++mu)
+      for (int n = 0; n < 8; ++n)
+        codes[k_token(mu, lane, n)][q.start + k_coord(j, lane, n)] = (s[mu] >> (4 * n)) & 15u;
+  }
+  if (q.r) {
+    const uint32_t* pc = gw + q.nfull * 32 * B;
+    const int nf = q.r >> 2;
+    for (int u = tid; u < 8 * nf; u += nthreads) {
+      const int g = u / nf, t = u % nf, lane = 4 * g + t;
+      uint32_t w[B], s[4];
+      for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * k + u];
+      quartet_decode<B>(w, s);
+      for (int mu = 0; mu < 4; ++mu)
+        for (int n = 0; n < 8; ++n)
+          codes[k_token(mu, lane, n)][q.start + k_coord(q.nfull, lane, n)] = (s[mu] >> (4 * n)) & 15u;
+    }
+    if (q.r & 3) {
+      for (int v = tid; v < 4; v += nthreads) {
+        uint32_t w[B], s[4];
+        for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * B + 4 * k + v];
+        quartet_decode<B>(w, s);
+        for (int mu = 0; mu < 4; ++mu)
+          for (int nv = 0; nv < 8; ++nv) {
+            const int lane = 4 * (2 * v + (nv >> 2)) + nf;
+            const int n = (nv & 1) + 4 * ((nv >> 1) & 1);  // half nibbles 0, 1, 4, 5
+            codes[k_token(mu, lane, n)][q.start + k_coord(q.nfull, lane, n)] = (s[mu] >> (4 * nv)) & 15u;
+          }
+      }
+    }
+  }
+}
+
+template <int B>
+__device__ void pack_k_group(uint32_t* tw, const GroupGeo& q, const uint8_t (*codes)[kD], int tid, int nthreads) {
+  uint32_t* gw = tw + q.word;
+  for (int u = tid; u < q.nfull * 32; u += nthreads) {
+    const int j = u >> 5, lane = u & 31;
+    uint32_t s[4], w[B];
+    for (int mu = 0; mu < 4; ++mu) {
+      uint32_t x = 0;
+      for (int n = 0; n < 8; ++n) x |= uint32_t(codes[k_token(mu, lane, n)][q.start + k_coord(j, lane, n)]) << (4 * n);
+      s[mu] = x;
+    }
+    quartet_encode<B>(s, w);
+    for (int k = 0; k < B; ++k) gw[j * 32 * B + 32 * k + lane] = w[k];
+  }
+  if (q.r) {
+    uint32_t* pc = gw + q.nfull * 32 * B;
+    const int nf = q.r >> 2;
+    for (int u = tid; u < 8 * nf; u += nthreads) {
+      const int g = u / nf, t = u % nf, lane = 4 * g + t;
+      uint32_t s[4], w[B];
+      for (int mu = 0; mu < 4; ++mu) {
+        uint32_t x = 0;
+        for (int n = 0; n < 8; ++n)
+          x |= uint32_t(codes[k_token(mu, lane, n)][q.start + k_coord(q.nfull, lane, n)]) << (4 * n);
+        s[mu] = x;
+      }
+      quartet_encode<B>(s, w);
+      for (int k = 0; k < B; ++k) pc[8 * nf * k + u] = w[k];
+    }
+    if (q.r & 3) {
+      for (int v = tid; v < 4; v += nthreads) {
+        uint32_t s[4], w[B];
+        for (int mu = 0; mu < 4; ++mu) {
+          uint32_t x = 0;
+          for (int nv = 0; nv < 8; ++nv) {
+            const int lane = 4 * (2 * v + (nv >> 2)) + nf;
+            const int n = (nv & 1) + 4 * ((nv >> 1) & 1);
+            x |= uint32_t(codes[k_token(mu, lane, n)][q.start + k_coord(q.nfull, lane, n)]) << (4 * nv);
+          }
+          s[mu] = x;
+        }
+        quartet_encode<B>(s, w);
+        for (int k = 0; k < B; ++k) pc[8 * nf * B + 4 * k + v] = w[k];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int v_token(int kappa, int lane, int n) {
+  const int t = lane & 3;
+  const int member = n & 3;
+  return 16 * kappa + 2 * t + (member & 1) + 8 * (member >> 1);
+}
+__device__ __forceinline__ int v_coord(int m, int lane, int n) { return 16 * m + (lane >> 2) + 8 * (n >= 4); }
+
+template <int B>
+__device__ void unpack_v_tile(const uint32_t* tw, uint8_t (*codes)[kD], int tid, int nthreads) {
+  for (int u = tid; u < 8 * 32; u += nthreads) {
+    const int m = u >> 5, lane = u & 31;
+    uint32_t w[B], s[4];
+    for (int k = 0; k < B; ++k) w[k] = tw[m * 32 * B + 32 * k + lane];
+    quartet_decode<B>(w, s);
+    for (int kappa = 0; kappa < 4; ++kappa)
+      for (int n = 0; n < 8; ++n) codes[v_token(kappa, lane, n)][v_coord(m, lane, n)] = (s[kappa] >> (4 * n)) & 15u;
+  }
+}
+
+template <int B>
+__device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kD], int tid, int nthreads) {
+  for (int u = tid; u < 8 * 32; u += nthreads) {
+    const int m = u >> 5, lane = u & 31;
+    uint32_t s[4], w[B];
+    for (int kappa = 0; kappa < 4; ++kappa) {
+      uint32_t x = 0;
+      for (int n = 0; n < 8; ++n) x |= uint32_t(codes[v_token(kappa, lane, n)][v_coord(m, lane, n)]) << (4 * n);
+      s[kappa] = x;
+    }
+    quartet_encode<B>(s, w);
+    for (int k = 0; k < B; ++k) tw[m * 32 * B + 32 * k + lane] = w[k];
+  }
+}
+
+#define BGTQ_WIDTH_SWITCH(b, F, ...) \
+  switch (b) {                       \
+    case 1: F<1>(__VA_ARGS__); break; \
+    case 2: F<2>(__VA_ARGS__); break; \
+    case 3: F<3>(__VA_ARGS__); break; \
+    default: F<4>(__VA_ARGS__); break; \
+  }
+
+// ---------------------------------------------------------------------------
+// a3: encode.  Grid (layer_count * batch * Hkv, ceil(n / 64) + 1, 2 kinds),
+// 256 threads.  A CTA owns one 64-position tile of one (layer, sequence, KV
+// head) and kind (K or V): it unpacks the tile's codes when the call writes
+// only part of it, encodes its new rows (y = R x in fp32, norms in fp64,
+// u = sqrt(d) y / n, code = #{thresholds <= u}) into the codes, and packs
+// the tile again.
+// ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
 
 struct EncodeSmem {
-  float xt[kD][kEncRows];        // xt[j][r] = x[r][perm[j]]
-  float mt[kD][kD];              // mt[j][i] = R[i][j]
-  float fac[kEncRows][kNumGroupsMax];
-  __half nrm[kEncRows][kNumGroupsMax];
-  uint32_t rec[kEncRows][17];
+  float xt[kD][kTile];           // new rows, transposed, record order (zero elsewhere)
+  float mt[kD][kD];              // mt[j][i] = R[i][j] (record order)
+  float fac[kTile][kNumGroupsMax];
+  __half nrm[kTile][kNumGroupsMax];
+  uint8_t codes[kTile][kD];
+  uint32_t words[1024];
   float thr[5][16];
-  int32_t inv[kD];               // dim -> record position
+  int32_t inv[kD];
+  int32_t gof[kD];               // group of each record position (-1: width 0)
   LayoutDev lay;
 };
 
-template <int KIND>
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace ws, CacheDev cache,
-                                                             int layer0, const __half* __restrict__ x,
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                             const __half* __restrict__ kx,
+                                                             const __half* __restrict__ vx,
                                                              const int32_t* __restrict__ start_v,
-                                                             const int32_t* __restrict__ count_v,
-                                                             int batch, int n) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   EncodeSmem& S = *reinterpret_cast<EncodeSmem*>(smem_raw);
   const int tid = threadIdx.x;
+  const int kind = blockIdx.z;
   const int h = blockIdx.x % sh.n_kv_heads;
   const int b = (blockIdx.x / sh.n_kv_heads) % batch;
   const int li = blockIdx.x / (sh.n_kv_heads * batch);
@@ -121,18 +395,28 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   const int start = start_v[b];
   const int count = count_v[b];
   if (start < 0 || count < 0 || count > n) {
-    if (tid == 0 && blockIdx.y == 0) atomicOr(ws.err, kErrArg);
+    if (tid == 0 && blockIdx.y == 0 && kind == 0) atomicOr(ws.err, kErrArg);
     return;
   }
-  const int r0 = blockIdx.y * kEncRows;
-  if (r0 >= count) return;
-  const int rows = min(kEncRows, count - r0);
-  const int bits_avg = KIND == 0 ? sh.kbits : sh.vbits;
-  const int nwords = 4 * bits_avg;
+  if (count == 0) return;
+  const int64_t tile = start / kTile + blockIdx.y;
+  const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
+  int64_t p1 = min(tile * kTile + kTile, static_cast<int64_t>(start) + count);
+  if (p0 >= p1) return;
+  if (p1 > sh.capacity) {
+    if (tid == 0) atomicOr(ws.err, kErrCapacity);
+    p1 = sh.capacity;
+    if (p0 >= p1) return;
+  }
+  const int tr0 = static_cast<int>(p0 - tile * kTile), tr1 = static_cast<int>(p1 - tile * kTile);
+  const bool whole = (tr0 == 0 && tr1 == kTile);
+  const int bits_avg = kind == 0 ? sh.kbits : sh.vbits;
+  const int nwords = 256 * bits_avg;
   const int lh = layer * sh.n_kv_heads + h;
+  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
+  uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + (seq_tiles + tile) * nwords;
 
-  // layout (K) or the trivial single group (V)
-  if (KIND == 0) {
+  if (kind == 0) {
     if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
       reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
   } else if (tid == 0) {
@@ -143,37 +427,58 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
       S.lay.size[g] = g == 0 ? kD : 0;
       S.lay.start[g] = g == 0 ? 0 : kD;
       S.lay.bitoff[g] = 0;
+      S.lay.tile_word[g] = 0;
+      S.lay.chunk_base[g] = 0;
     }
   }
   for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
-  for (int i = tid; i < kEncRows * 17; i += kEncThreads) (&S.rec[0][0])[i] = 0u;
-  const float* mglob = (KIND == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
+  const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
   for (int i = tid; i < kD * kD / 4; i += kEncThreads)
     reinterpret_cast<float4*>(&S.mt[0][0])[i] = reinterpret_cast<const float4*>(mglob)[i];
   __syncthreads();
-  if (tid < kD) {
-    if (KIND == 0) S.inv[S.lay.perm[tid]] = tid;
-    else S.inv[tid] = tid;
-  }
-  __syncthreads();
-  // rows -> xt (transposed, record order); rows past `rows` are zero
-  const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
-  const __half* xbase =
-      x + ((static_cast<size_t>(li) * batch + b) * n + r0) * row_stride + static_cast<size_t>(h) * kD;
-  for (int e = tid; e < kEncRows * kD; e += kEncThreads) {
-    const int r = e / kD, dm = e % kD;
-    const float v = r < rows ? __half2float(xbase[r * row_stride + dm]) : 0.f;
-    S.xt[S.inv[dm]][r] = v;
-  }
-  __syncthreads();
   const int ng = S.lay.n_groups;
   const int npos = S.lay.n_positions;
-  // per (row, group): norm in fp64, the fp16 stored norm and the factor sqrt(d)/n
+  if (tid < kD) {
+    S.inv[kind == 0 ? S.lay.perm[tid] : tid] = tid;
+    int g = -1;
+    if (tid < npos) {
+      g = 0;
+      for (int t = 1; t < ng; ++t)
+        if (tid >= S.lay.start[t]) g = t;
+    }
+    S.gof[tid] = g;
+  }
+  // existing codes of a partly written tile
+  if (!whole) {
+    if (kind == 0) {
+      for (int g = 0; g < ng; ++g) {
+        const GroupGeo q = group_geo(S.lay, g);
+        BGTQ_WIDTH_SWITCH(q.width, unpack_k_group, gtile, q, S.codes, tid, kEncThreads)
+      }
+    } else {
+      BGTQ_WIDTH_SWITCH(sh.vbits, unpack_v_tile, gtile, S.codes, tid, kEncThreads)
+    }
+  }
+  __syncthreads();
+  // new rows -> xt (record order)
+  const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
+  const __half* x = kind == 0 ? kx : vx;
+  const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
+                        static_cast<size_t>(h) * kD;
+  for (int e = tid; e < kTile * kD; e += kEncThreads) {
+    const int r = e / kD, dm = e % kD;
+    const int tr = r;
+    const bool valid = tr >= tr0 && tr < tr1;
+    const float v = valid ? __half2float(xbase[static_cast<size_t>(tr - tr0) * row_stride + dm]) : 0.f;
+    S.xt[S.inv[dm]][tr] = v;
+  }
+  __syncthreads();
+  // norms: fp64 sum of squares of the exact fp16 inputs
   {
     const int r = tid >> 2, g = tid & 3;
     float f = 0.f;
     __half nh = __float2half(0.f);
-    if (g < ng) {
+    if (g < ng && r >= tr0 && r < tr1) {
       const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
       double s2 = 0.0;
       for (int j = j0; j < j1; ++j) {
@@ -188,108 +493,96 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     S.nrm[r][g] = nh;
   }
   __syncthreads();
-  // Y tile
-  const int rg = tid >> 4, og = tid & 15;
-  const int i0 = og * 8;
-  if (i0 < npos && rg * 4 < rows) {
-    int gi[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int i = i0 + q;
-      int g = 0;
-      for (int t = 1; t < ng; ++t)
-        if (i >= S.lay.start[t]) g = t;
-      gi[q] = i < npos ? g : -1;
+  // y = R x per new row, then the codes
+  const int nrows = tr1 - tr0;
+  if (nrows <= 16) {
+    // few rows (decode-time appends): one output per thread
+    const int i = tid & (kD - 1);
+    const int g = S.gof[i];
+    if (g >= 0) {
+      const int w = S.lay.width[g];
+      const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
+      const int nt = (1 << w) - 1;
+      for (int r = tr0 + (tid >> 7); r < tr1; r += 2) {
+        float y = 0.f;
+        for (int j = j0; j < j1; ++j) y = fmaf(S.mt[j][i], S.xt[j][r], y);
+        const float u = y * S.fac[r][g];
+        int code = 0;
+        for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
+        S.codes[r][i] = static_cast<uint8_t>(code);
+      }
     }
-    // groups are contiguous in record order: run over the groups of the
-    // first and last valid output (the rotation is zero elsewhere)
-    const int glo = gi[0];
-    int ghi = glo;
+  } else {
+    // register tile: 4 rows x 8 outputs per thread over all 64 rows
+    const int rg = tid >> 4, og = tid & 15;
+    const int i0 = og * 8;
+    if (i0 < npos && rg * 4 < tr1 && rg * 4 + 4 > tr0) {
+      int gi[8];
 #pragma unroll
-    for (int q = 1; q < 8; ++q)
-      if (gi[q] > ghi) ghi = gi[q];
-    const int jlo = S.lay.start[glo];
-    const int jhi = S.lay.start[ghi] + S.lay.size[ghi];
-    float acc[4][8];
+      for (int q = 0; q < 8; ++q) gi[q] = S.gof[i0 + q];
+      int ghi = gi[0];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
-    for (int j = jlo; j < jhi; ++j) {
-      const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][rg * 4]);
-      const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][i0]);
-      const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][i0 + 4]);
-      const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+      for (int q = 1; q < 8; ++q)
+        if (gi[q] > ghi) ghi = gi[q];
+      const int jlo = S.lay.start[gi[0]];
+      const int jhi = S.lay.start[ghi] + S.lay.size[ghi];
+      float acc[4][8];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[a][q] = fmaf(xs[a], ms[q], acc[a][q]);
-    }
-    // quantise + pack
-    int bo[8];
+        for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
+      for (int j = jlo; j < jhi; ++j) {
+        const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][rg * 4]);
+        const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][i0]);
+        const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][i0 + 4]);
+        const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int g = gi[q];
-      bo[q] = g >= 0 ? S.lay.bitoff[g] + (i0 + q - S.lay.start[g]) * S.lay.width[g] : 0;
-    }
-    const int base = bo[0] & ~31;
+        for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = rg * 4 + a;
-      uint64_t word = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int g = gi[q];
-        if (g < 0) continue;
-        const int w = S.lay.width[g];
-        const float u = acc[a][q] * S.fac[r][g];
-        int code = 0;
-        const int nt = (1 << w) - 1;
-        for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
-        word |= static_cast<uint64_t>(code) << (bo[q] - base);
+          for (int q = 0; q < 8; ++q) acc[a][q] = fmaf(xs[a], ms[q], acc[a][q]);
       }
-      if (r < rows) {
-        atomicOr(&S.rec[r][base >> 5], static_cast<uint32_t>(word));
-        const uint32_t hi = static_cast<uint32_t>(word >> 32);
-        if (hi) atomicOr(&S.rec[r][(base >> 5) + 1], hi);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int r = rg * 4 + a;
+        if (r < tr0 || r >= tr1) continue;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int g = gi[q];
+          if (g < 0) continue;
+          const int w = S.lay.width[g];
+          const float u = acc[a][q] * S.fac[r][g];
+          int code = 0;
+          const int nt = (1 << w) - 1;
+          for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
+          S.codes[r][i0 + q] = static_cast<uint8_t>(code);
+        }
       }
     }
   }
   __syncthreads();
-  // write records and norms; rows past capacity are skipped and flagged
-  const size_t tok0 = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.capacity;
-  const int chunks = nwords / 4;
-  uint8_t* recbase = (KIND == 0 ? cache.krec : cache.vrec);
-  bool over = false;
-  for (int e = tid; e < rows * chunks; e += kEncThreads) {
-    const int r = e / chunks, c = e % chunks;
-    const int64_t pos = static_cast<int64_t>(start) + r0 + r;
-    if (pos >= sh.capacity) {
-      over = true;
-      continue;
+  // repack the tile and write it back
+  if (kind == 0) {
+    for (int g = 0; g < ng; ++g) {
+      const GroupGeo q = group_geo(S.lay, g);
+      BGTQ_WIDTH_SWITCH(q.width, pack_k_group, S.words, q, S.codes, tid, kEncThreads)
     }
-    const uint4 v = make_uint4(S.rec[r][4 * c], S.rec[r][4 * c + 1], S.rec[r][4 * c + 2], S.rec[r][4 * c + 3]);
-    reinterpret_cast<uint4*>(recbase + (tok0 + pos) * (16 * bits_avg))[c] = v;
+  } else {
+    BGTQ_WIDTH_SWITCH(sh.vbits, pack_v_tile, S.words, S.codes, tid, kEncThreads)
   }
-  if (tid < rows) {
-    const int r = tid;
-    const int64_t pos = static_cast<int64_t>(start) + r0 + r;
-    if (pos < sh.capacity) {
-      if (KIND == 0) {
-        __half2 n01 = __halves2half2(S.nrm[r][0], S.nrm[r][1]);
-        __half2 n23 = __halves2half2(S.nrm[r][2], S.nrm[r][3]);
-        __half2* dst = reinterpret_cast<__half2*>(cache.knorm + (tok0 + pos) * 4);
-        dst[0] = n01;
-        dst[1] = n23;
-      } else {
-        cache.vnorm[tok0 + pos] = S.nrm[r][0];
-      }
+  __syncthreads();
+  for (int i = tid; i < nwords / 4; i += kEncThreads)
+    reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
+  if (tid >= tr0 && tid < tr1) {
+    const size_t pos = seq_tiles * kTile + tile * kTile + tid;
+    if (kind == 0) {
+      __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
+      dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
+      dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
     } else {
-      over = true;
+      cache.vnorm[pos] = S.nrm[tid][0];
     }
   }
-  if (over) atomicOr(ws.err, kErrCapacity);
 }
 
 // ---------------------------------------------------------------------------
@@ -324,51 +617,169 @@ __global__ void __launch_bounds__(128) rotate_query_kernel(Shape sh, Workspace w
 }
 
 // ---------------------------------------------------------------------------
-// a5: split-K decode from packed codes (SIMT fp32).
+// a5: split-K decode straight from the packed tiles on the tensor cores.
 //
-// Grid (n_splits, batch * Hkv, layer_count), 128 threads = 4 warps.  A CTA
-// owns tokens [s*T, min((s+1)*T, len)) of one (layer, sequence, KV head);
-// its warps take tiles of 32*TPL tokens round-robin and keep their own
-// online-softmax state for the GP (padded) query heads of the group.
+// Grid (n_splits, batch * Hkv * head_blocks, layer_count), 128 threads.  A
+// CTA owns the positions [s*T, min((s+1)*T, len)) of one (layer, sequence,
+// KV head) and up to 8 of its G query heads; its 4 warps take 64-position
+// tiles round-robin, each with its own 3-stage bulk-copy pipeline (K tile,
+// V tile, norms -> shared memory, completion on an mbarrier) and its own
+// online-softmax state.
 //
-// Phase A (logits), lane = token (TPL tokens per lane): the K records sit in
-// registers; the loop over record words is unrolled at compile time and the
-// codes starting in each word are walked at run time (widths and group
-// boundaries are uniform across the warp), so every code is one funnel
-// shift + mask + a shared-memory centroid lookup, shared by all GP heads.
-// Per group g the partial dot products q~_g . C[codes] are scaled by the
-// token's group norm.  Logits are kept in log2 units (q~ * log2 e).
-// Phase B (P V), lane = 4 rotated V coordinates: each token's weight
-// p * n_V / sqrt(D) times the centroids of the lane's 4 codes.
+// Logits (per warp per tile): S^T[64 tokens x 8 heads] = K_hat q~^T as
+// mma.sync m16n8k16 tiles -- A = centroids C[codes] (exact in fp16), looked
+// up in registers with PRMT byte tables from the lane's selector words;
+// B = q~ * log2(e) split into fp16 hi + lo (two MMAs).  Each width group
+// accumulates separately and is scaled by its per-token norm.
+// P V: O^T[128 dims x 8 heads] += V_hat^T P'^T with P' = 2^(logit - max) *
+// n_V / sqrt(D) in fp16, moved from the logit accumulator layout into a B
+// operand with movmatrix.  Everything stays in V's rotated basis; the
+// combine kernel rotates back.
 // ---------------------------------------------------------------------------
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kStages = 3;
+constexpr int kWaitLimit = 1 << 22;
 
-template <int GP, int TPL>
-struct DecodeSmem {
-  float qs[kD][GP];
-  float pw[kDecWarps][32 * TPL][GP];
-  float accs[kDecWarps][GP][kD];
-  uint32_t vr[kDecWarps][32 * TPL][17];
-  float cent[5][16];
-  float ms[kDecWarps][GP];
-  float ls[kDecWarps][GP];
-  LayoutDev lay;
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity; gives up after kWaitLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+struct DecodeLayout {  // byte offsets inside the dynamic shared memory
+  int bars, bq, tabk, geo, ms, ls, stage, stage_bytes, total;
 };
 
-template <int KB, int GP, int TPL>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(Shape sh, Workspace ws, CacheDev cache,
-                                                                   int layer0, const float* __restrict__ qrot,
-                                                                   const int32_t* __restrict__ seq_lens,
-                                                                   int batch, int split_tokens) {
-  constexpr int NW = 4 * KB;  // 32-bit words per K record
-  constexpr int TILE = 32 * TPL;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  DecodeSmem<GP, TPL>& S = *reinterpret_cast<DecodeSmem<GP, TPL>*>(smem_raw);
+__host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
+
+__host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
+  DecodeLayout L;
+  L.bars = 0;
+  L.bq = align128(kDecWarps * kStages * 8);
+  L.tabk = L.bq + kMaxChunks * 32 * 16;
+  L.geo = L.tabk + kNumGroupsMax * 8 * 4;
+  L.ms = L.geo + kNumGroupsMax * 8 * 4;
+  L.ls = L.ms + kDecWarps * 8 * 4;
+  L.stage = align128(L.ls + kDecWarps * 8 * 4);
+  L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
+  const int stages = kDecWarps * kStages * L.stage_bytes;
+  const int merge = kDecWarps * 8 * kD * 4;  // reuses the stage buffers after the loop
+  L.total = L.stage + (stages > merge ? stages : merge);
+  return L;
+}
+
+// Logits of one width group for the warp's tile: S[mu][4] (M-tile mu).
+template <int B>
+__device__ __forceinline__ void group_logits(const uint32_t* kt, const GroupGeo& q, const uint4* bq,
+                                             const uint32_t* tab8, int lane, float (*S)[4]) {
+  ByteTab t;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    t.lo[i] = tab8[i];
+    t.hi[i] = tab8[4 + i];
+  }
+  const uint32_t* gw = kt + q.word;
+  for (int j = 0; j < q.nfull; ++j) {
+    uint32_t w[B], s[4];
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
+    quartet_decode<B>(w, s);
+    const uint4 bf = bq[(q.chunk + j) * 32 + lane];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      uint32_t r0, r1, r2, r3;
+      lookup4<B>(t, s[mu], r0, r2);
+      lookup4<B>(t, s[mu] >> 16, r1, r3);
+      mma16816(S[mu], r0, r1, r2, r3, bf.x, bf.y);
+      mma16816(S[mu], r0, r1, r2, r3, bf.z, bf.w);
+    }
+  }
+  if (q.r) {
+    const uint32_t* pc = gw + q.nfull * 32 * B;
+    const int nf = q.r >> 2;
+    const int g = lane >> 2, tl = lane & 3;
+    uint32_t s[4] = {0u, 0u, 0u, 0u};
+    uint32_t w[B];
+    if (tl < nf) {
+#pragma unroll
+      for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * k + g * nf + tl];
+      quartet_decode<B>(w, s);
+    } else if ((q.r & 3) && tl == nf) {
+      uint32_t sv[4];
+#pragma unroll
+      for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * B + 4 * k + (g >> 1)];
+      quartet_decode<B>(w, sv);
+      const int sh = 16 * (g & 1);
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        const uint32_t x = (sv[mu] >> sh) & 0xFFFFu;
+        s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
+      }
+    }
+    const uint4 bf = bq[(q.chunk + q.nfull) * 32 + lane];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      uint32_t r0, r1, r2, r3;
+      lookup4<B>(t, s[mu], r0, r2);
+      lookup4<B>(t, s[mu] >> 16, r1, r3);
+      mma16816(S[mu], r0, r1, r2, r3, bf.x, bf.y);
+      mma16816(S[mu], r0, r1, r2, r3, bf.z, bf.w);
+    }
+  }
+}
+
+template <int VB>
+__global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                                 const float* __restrict__ qrot,
+                                                                 const int32_t* __restrict__ seq_lens, int batch,
+                                                                 int split_tokens, int head_blocks) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const DecodeLayout DL = decode_layout(sh.kbits, VB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
+  uint4* bq = reinterpret_cast<uint4*>(smem_raw + DL.bq);
+  uint32_t* tabk = reinterpret_cast<uint32_t*>(smem_raw + DL.tabk);
+  int32_t* geo = reinterpret_cast<int32_t*>(smem_raw + DL.geo);
+  float* ms = reinterpret_cast<float*>(smem_raw + DL.ms);
+  float* ls = reinterpret_cast<float*>(smem_raw + DL.ls);
+  unsigned char* stage_base = smem_raw + DL.stage;
+
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, t4 = lane & 3;
   const int s = blockIdx.x;
-  const int h = blockIdx.y % sh.n_kv_heads;
-  const int b = blockIdx.y / sh.n_kv_heads;
+  const int hb = blockIdx.y % head_blocks;
+  const int h = (blockIdx.y / head_blocks) % sh.n_kv_heads;
+  const int b = blockIdx.y / (head_blocks * sh.n_kv_heads);
   const int li = blockIdx.z;
   const int layer = layer0 + li;
   int len = seq_lens[b];
@@ -377,221 +788,259 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(Shape sh, Wor
   if (t0 >= len) return;
   const int t1 = min(t0 + split_tokens, len);
   const int G = sh.group;
+  const int h0 = 8 * hb;                       // first query head of this block within the group
+  const int nh = min(8, G - h0);
   const int lh = layer * sh.n_kv_heads + h;
+  const LayoutDev& lay = ws.layouts[lh];
 
-  if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
-    reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
-  for (int i = tid; i < 5 * 16; i += kDecThreads) (&S.cent[0][0])[i] = (&ws.codebook->centroid[0][0])[i];
+  // ---- per-CTA set-up: q~ B fragments, byte tables, group geometry ----
+  const int ng = lay.n_groups;
+  if (tid < kNumGroupsMax) {
+    int word = 0, chunk = 0;
+    for (int g = 0; g < tid && g < ng; ++g) {
+      word += 2 * lay.size[g] * lay.width[g];
+      chunk += (lay.size[g] + 15) >> 4;
+    }
+    geo[tid * 8 + 0] = tid < ng ? lay.width[tid] : 0;
+    geo[tid * 8 + 1] = tid < ng ? lay.size[tid] : 0;
+    geo[tid * 8 + 2] = tid < ng ? lay.start[tid] : 0;
+    geo[tid * 8 + 3] = word;
+    geo[tid * 8 + 4] = chunk;
+  }
+  if (tid < kNumGroupsMax * 8) {
+    const int g = tid >> 3, wd = tid & 7;
+    uint32_t v = 0;
+    if (g < ng) {
+      const int bits = lay.width[g];
+      const float* cen = ws.codebook->centroid[bits];
+      const int n = 1 << bits;
+      for (int c = 0; c < 4; ++c) {
+        const int e = 4 * (wd & 3) + c;
+        if (e < n) {
+          const uint32_t hb16 = __half_as_ushort(__float2half_rn(cen[e]));
+          v |= (wd < 4 ? (hb16 & 0xFFu) : (hb16 >> 8)) << (8 * c);
+        }
+      }
+    }
+    tabk[tid] = v;
+  }
+  if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
+  __syncthreads();
+  if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   {
-    const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G) * kD;
-    for (int e = tid; e < kD * GP; e += kDecThreads) {
-      const int hh = e / kD, i = e % kD;
-      S.qs[i][hh] = hh < G ? qsrc[hh * kD + i] * kLog2e : 0.f;
+    const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
+    int nchunk = 0;
+    for (int g = 0; g < ng; ++g) nchunk += (lay.size[g] + 15) >> 4;
+    for (int u = tid; u < nchunk * 32; u += kDecThreads) {
+      const int c = u >> 5, ln = u & 31;
+      int g = 0;
+      while (g + 1 < ng && c >= geo[(g + 1) * 8 + 4]) ++g;
+      const int j = c - geo[g * 8 + 4];
+      const int d = geo[g * 8 + 1], st = geo[g * 8 + 2];
+      const int head = ln >> 2;
+      float v[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int coord = 16 * j + 4 * (ln & 3) + m;
+        v[m] = (head < nh && coord < d) ? qsrc[head * kD + st + coord] * kLog2e : 0.f;
+      }
+      uint32_t hi01, hi23, lo01, lo23;
+      {
+        const __half2 a = __floats2half2_rn(v[0], v[1]);
+        const __half2 c2 = __floats2half2_rn(v[2], v[3]);
+        const float2 af = __half22float2(a), cf = __half22float2(c2);
+        const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
+        const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
+        hi01 = *reinterpret_cast<const uint32_t*>(&a);
+        hi23 = *reinterpret_cast<const uint32_t*>(&c2);
+        lo01 = *reinterpret_cast<const uint32_t*>(&al);
+        lo23 = *reinterpret_cast<const uint32_t*>(&cl);
+      }
+      bq[u] = make_uint4(hi01, hi23, lo01, lo23);
     }
   }
-  for (int e = tid; e < kDecWarps * GP * kD; e += kDecThreads) (&S.accs[0][0][0])[e] = 0.f;
+  ByteTab tv;
+  fill_bytetab(tv, ws.codebook->centroid[VB], VB);
   __syncthreads();
 
-  const size_t tok0 = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.capacity;
-  const uint8_t* krec = cache.krec + tok0 * (16 * KB);
-  const __half* knorm = cache.knorm + tok0 * 4;
-  const int vb = sh.vbits;
-  const int vw = 4 * vb;
-  const uint8_t* vrec = cache.vrec + tok0 * (16 * vb);
-  const __half* vnorm = cache.vnorm + tok0;
-  const float* cv = S.cent[vb];
-  const uint32_t vmask = (1u << vb) - 1u;
-  const int vbit0 = 4 * vb * lane;
-  const int vw0 = vbit0 >> 5, vsh = vbit0 & 31;
+  // ---- per-warp pipeline over this warp's tiles ----
+  const int tiles_cta = (t1 - t0 + kTile - 1) / kTile;
+  const int my_tiles = tiles_cta > warp ? (tiles_cta - warp + kDecWarps - 1) / kDecWarps : 0;
+  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
+  const int kwords = 256 * sh.kbits, vwords = 256 * VB;
+  const uint32_t kbytes = 4u * kwords, vbytes = 4u * vwords;
+  const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
+  unsigned char* my_stage = stage_base + static_cast<size_t>(warp) * kStages * DL.stage_bytes;
+  uint64_t* my_bars = bars + warp * kStages;
 
-  float m_run[GP], l_run[GP];
-#pragma unroll
-  for (int hh = 0; hh < GP; ++hh) {
-    m_run[hh] = -CUDART_INF_F;
-    l_run[hh] = 0.f;
-  }
+  auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
+    const int tile = t0 / kTile + warp + k * kDecWarps;
+    unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
+    uint64_t* bar = &my_bars[k % kStages];
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(bar, stage_tx);
+    bulk_copy_g2s(dst, cache.ktile + (seq_tiles + tile) * kwords, kbytes, bar);
+    bulk_copy_g2s(dst + kbytes, cache.vtile + (seq_tiles + tile) * vwords, vbytes, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes, cache.knorm + (seq_tiles * kTile + static_cast<size_t>(tile) * kTile) * 4,
+                  kTile * 8, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, cache.vnorm + seq_tiles * kTile + static_cast<size_t>(tile) * kTile,
+                  kTile * 2, bar);
+  };
+  if (lane == 0)
+    for (int k = 0; k < kStages && k < my_tiles; ++k) issue(k);
 
-  for (int tile = t0 + warp * TILE; tile < t1; tile += kDecWarps * TILE) {
-    // ---- phase A: logits, lane = token ----
-    float L[TPL][GP];
-    float vn[TPL];
-    {
-      uint32_t rec[TPL][NW + 1];
-      float kn[TPL][kNumGroupsMax];
+  float O[8][4];
 #pragma unroll
-      for (int k = 0; k < TPL; ++k) {
-        const int t = tile + lane + 32 * k;
-        const int tt = t < t1 ? t : t0;
-        const uint4* src = reinterpret_cast<const uint4*>(krec + static_cast<size_t>(tt) * (16 * KB));
+  for (int m = 0; m < 8; ++m)
 #pragma unroll
-        for (int c = 0; c < KB; ++c) {
-          const uint4 v = __ldg(src + c);
-          rec[k][4 * c] = v.x;
-          rec[k][4 * c + 1] = v.y;
-          rec[k][4 * c + 2] = v.z;
-          rec[k][4 * c + 3] = v.w;
-        }
-        rec[k][NW] = 0u;
-        const uint2 nv = __ldg(reinterpret_cast<const uint2*>(knorm + static_cast<size_t>(tt) * 4));
-        const __half2 n01 = *reinterpret_cast<const __half2*>(&nv.x);
-        const __half2 n23 = *reinterpret_cast<const __half2*>(&nv.y);
-        kn[k][0] = __low2float(n01);
-        kn[k][1] = __high2float(n01);
-        kn[k][2] = __low2float(n23);
-        kn[k][3] = __high2float(n23);
-        vn[k] = t < t1 ? __half2float(vnorm[tt]) * kInvSqrtD : 0.f;
-        // stage this token's V record for phase B
-        const uint4* vsrc = reinterpret_cast<const uint4*>(vrec + static_cast<size_t>(tt) * (16 * vb));
-        uint32_t* vdst = S.vr[warp][lane + 32 * k];
-        for (int c = 0; c < vb; ++c) {
-          const uint4 v = __ldg(vsrc + c);
-          vdst[4 * c] = v.x;
-          vdst[4 * c + 1] = v.y;
-          vdst[4 * c + 2] = v.z;
-          vdst[4 * c + 3] = v.w;
-        }
-        vdst[vw] = 0u;
-      }
-      float Sg[TPL][GP];
+    for (int r = 0; r < 4; ++r) O[m][r] = 0.f;
+  float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
+  int failed_at = -1;
+
+  for (int k = 0; k < my_tiles; ++k) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&my_bars[k % kStages], (k / kStages) & 1))) {
+      failed_at = k;
+      break;
+    }
+    const unsigned char* st = my_stage + (k % kStages) * DL.stage_bytes;
+    const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
+    const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
+    const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
+    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
+    const int tile_pos = t0 + (warp + k * kDecWarps) * kTile;
+    const int nvalid = min(kTile, t1 - tile_pos);
+
+    // logits
+    float L[4][4];
 #pragma unroll
-      for (int k = 0; k < TPL; ++k)
+    for (int mu = 0; mu < 4; ++mu)
 #pragma unroll
-        for (int hh = 0; hh < GP; ++hh) {
-          L[k][hh] = 0.f;
-          Sg[k][hh] = 0.f;
-        }
-      const int npos = S.lay.n_positions;
-      int p = 0, g = 0;
-      int gend = S.lay.size[0];
-      int bw = S.lay.width[0];
-      uint32_t msk = (1u << bw) - 1u;
-      const float* cb = S.cent[bw];
-      int bo = 0;
-      float curn[TPL];
+      for (int r = 0; r < 4; ++r) L[mu][r] = 0.f;
+    for (int g = 0; g < ng; ++g) {
+      GroupGeo q;
+      q.width = geo[g * 8 + 0];
+      q.d = geo[g * 8 + 1];
+      q.start = geo[g * 8 + 2];
+      q.word = geo[g * 8 + 3];
+      q.chunk = geo[g * 8 + 4];
+      q.nfull = q.d >> 4;
+      q.r = q.d & 15;
+      float S[4][4];
 #pragma unroll
-      for (int k = 0; k < TPL; ++k) curn[k] = kn[k][0];
+      for (int mu = 0; mu < 4; ++mu)
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        while (p < npos && bo < 32 * (w + 1)) {
-          if (p == gend) {
+        for (int r = 0; r < 4; ++r) S[mu][r] = 0.f;
+      BGTQ_WIDTH_SWITCH(q.width, group_logits, kt, q, bq, tabk + 8 * g, lane, S)
 #pragma unroll
-            for (int k = 0; k < TPL; ++k)
-#pragma unroll
-              for (int hh = 0; hh < GP; ++hh) {
-                L[k][hh] = fmaf(curn[k], Sg[k][hh], L[k][hh]);
-                Sg[k][hh] = 0.f;
-              }
-            ++g;
-#pragma unroll
-            for (int k = 0; k < TPL; ++k) curn[k] = g == 1 ? kn[k][1] : (g == 2 ? kn[k][2] : kn[k][3]);
-            gend += S.lay.size[g];
-            bw = S.lay.width[g];
-            msk = (1u << bw) - 1u;
-            cb = S.cent[bw];
-          }
-          const int shf = bo - 32 * w;
-          float c[TPL];
-#pragma unroll
-          for (int k = 0; k < TPL; ++k) c[k] = cb[__funnelshift_r(rec[k][w], rec[k][w + 1], shf) & msk];
-#pragma unroll
-          for (int hh = 0; hh < GP; ++hh) {
-            const float qv = S.qs[p][hh];
-#pragma unroll
-            for (int k = 0; k < TPL; ++k) Sg[k][hh] = fmaf(qv, c[k], Sg[k][hh]);
-          }
-          ++p;
-          bo += bw;
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < TPL; ++k) {
-        const bool valid = tile + lane + 32 * k < t1;
-#pragma unroll
-        for (int hh = 0; hh < GP; ++hh) {
-          const float v = fmaf(curn[k], Sg[k][hh], L[k][hh]);
-          L[k][hh] = valid ? v : -CUDART_INF_F;
-        }
+      for (int mu = 0; mu < 4; ++mu) {
+        const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
+        const float nb = __half2float(kn[(16 * mu + g8 + 8) * 4 + g]);
+        L[mu][0] = fmaf(na, S[mu][0], L[mu][0]);
+        L[mu][1] = fmaf(na, S[mu][1], L[mu][1]);
+        L[mu][2] = fmaf(nb, S[mu][2], L[mu][2]);
+        L[mu][3] = fmaf(nb, S[mu][3], L[mu][3]);
       }
     }
-    // ---- online softmax over the tile ----
-    float alpha[GP];
+    // online softmax over the tile for heads 2*t4 and 2*t4+1
+    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-    for (int hh = 0; hh < GP; ++hh) {
-      float mx = L[0][hh];
+    for (int mu = 0; mu < 4; ++mu) {
+      const bool va = 16 * mu + g8 < nvalid, vbv = 16 * mu + g8 + 8 < nvalid;
+      if (!va) L[mu][0] = L[mu][1] = -CUDART_INF_F;
+      if (!vbv) L[mu][2] = L[mu][3] = -CUDART_INF_F;
+      mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
+      mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
+    }
 #pragma unroll
-      for (int k = 1; k < TPL; ++k) mx = fmaxf(mx, L[k][hh]);
+    for (int o = 4; o < 32; o <<= 1) {
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+      mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
+    }
+    float alpha[2], sum[2] = {0.f, 0.f};
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float mnew = fmaxf(m_run[hh], mx);
-      alpha[hh] = exp2f(m_run[hh] - mnew);
-      float sum = 0.f;
+    for (int c = 0; c < 2; ++c) {
+      const float mnew = fmaxf(m_run[c], mx[c]);
+      alpha[c] = exp2f(m_run[c] - mnew);
+      m_run[c] = mnew;
+    }
+    uint32_t bp[4][2];
 #pragma unroll
-      for (int k = 0; k < TPL; ++k) {
-        const float pv = exp2f(L[k][hh] - mnew);
-        sum += pv;
-        S.pw[warp][lane + 32 * k][hh] = pv * vn[k];
-      }
+    for (int mu = 0; mu < 4; ++mu) {
+      // positions past the valid length carry no weight (their norms may be anything)
+      const float wa = 16 * mu + g8 < nvalid ? __half2float(vn[16 * mu + g8]) * kInvSqrtD : 0.f;
+      const float wb = 16 * mu + g8 + 8 < nvalid ? __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD : 0.f;
+      const float p0 = exp2f(L[mu][0] - m_run[0]), p1 = exp2f(L[mu][1] - m_run[1]);
+      const float p2 = exp2f(L[mu][2] - m_run[0]), p3 = exp2f(L[mu][3] - m_run[1]);
+      sum[0] += p0 + p2;
+      sum[1] += p1 + p3;
+      bp[mu][0] = transpose8x8(pack_half2(p0 * wa, p1 * wa));
+      bp[mu][1] = transpose8x8(pack_half2(p2 * wb, p3 * wb));
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      l_run[hh] = fmaf(l_run[hh], alpha[hh], sum);
-      m_run[hh] = mnew;
+    for (int o = 4; o < 32; o <<= 1) {
+      sum[0] += __shfl_xor_sync(0xffffffffu, sum[0], o);
+      sum[1] += __shfl_xor_sync(0xffffffffu, sum[1], o);
+    }
+    l_run[0] = fmaf(l_run[0], alpha[0], sum[0]);
+    l_run[1] = fmaf(l_run[1], alpha[1], sum[1]);
+    // P V in V's rotated basis
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      O[m][0] *= alpha[0];
+      O[m][1] *= alpha[1];
+      O[m][2] *= alpha[0];
+      O[m][3] *= alpha[1];
+      uint32_t w[VB], sv[4];
+#pragma unroll
+      for (int kk = 0; kk < VB; ++kk) w[kk] = vt[m * 32 * VB + 32 * kk + lane];
+      quartet_decode<VB>(w, sv);
+#pragma unroll
+      for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
     }
     __syncwarp();
-    // ---- phase B: P V in V's rotated basis, lane = 4 coordinates ----
-    {
-      float acc[GP][4];
-#pragma unroll
-      for (int hh = 0; hh < GP; ++hh) {
-        const float4 a = *reinterpret_cast<const float4*>(&S.accs[warp][hh][4 * lane]);
-        acc[hh][0] = a.x * alpha[hh];
-        acc[hh][1] = a.y * alpha[hh];
-        acc[hh][2] = a.z * alpha[hh];
-        acc[hh][3] = a.w * alpha[hh];
-      }
-      const int ntok = min(TILE, t1 - tile);
-      for (int tt = 0; tt < ntok; ++tt) {
-        const uint32_t* vrow = S.vr[warp][tt];
-        const uint32_t bits = __funnelshift_r(vrow[vw0], vrow[vw0 + 1], vsh);
-        float c[4];
-#pragma unroll
-        for (int dk = 0; dk < 4; ++dk) c[dk] = cv[(bits >> (vb * dk)) & vmask];
-#pragma unroll
-        for (int hh = 0; hh < GP; ++hh) {
-          const float pv = S.pw[warp][tt][hh];
-#pragma unroll
-          for (int dk = 0; dk < 4; ++dk) acc[hh][dk] = fmaf(pv, c[dk], acc[hh][dk]);
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < GP; ++hh)
-        *reinterpret_cast<float4*>(&S.accs[warp][hh][4 * lane]) =
-            make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
-    }
-    __syncwarp();
+    if (lane == 0 && k + kStages < my_tiles) issue(k + kStages);
   }
-  if (lane == 0) {
-#pragma unroll
-    for (int hh = 0; hh < GP; ++hh) {
-      S.ms[warp][hh] = m_run[hh];
-      S.ls[warp][hh] = l_run[hh];
-    }
+  const bool timed_out = failed_at >= 0;
+  if (timed_out) {
+    if (lane == 0) atomicOr(ws.err, kErrTimeout);
+    // copies issued but not yet consumed: let them land (bounded) before the
+    // stage buffers are reused or the CTA exits
+    const int issued = min(my_tiles, failed_at + kStages);
+    for (int k = failed_at; k < issued; ++k) mbar_wait(&my_bars[k % kStages], (k / kStages) & 1);
   }
   __syncthreads();
-  // merge the warps; thread = rotated coordinate
+  // ---- merge the warps (the stage buffers are reused) ----
+  float* accs = reinterpret_cast<float*>(stage_base);  // [warp][8 heads][128]
+  if (g8 == 0) {
+    ms[warp * 8 + 2 * t4] = m_run[0];
+    ms[warp * 8 + 2 * t4 + 1] = m_run[1];
+    ls[warp * 8 + 2 * t4] = l_run[0];
+    ls[warp * 8 + 2 * t4 + 1] = l_run[1];
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    float* a = accs + warp * 8 * kD;
+    a[(2 * t4) * kD + 16 * m + g8] = O[m][0];
+    a[(2 * t4 + 1) * kD + 16 * m + g8] = O[m][1];
+    a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
+    a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
+  }
+  __syncthreads();
+  if (__syncthreads_or(timed_out)) return;
   const int i = tid;
-  for (int hh = 0; hh < G; ++hh) {
+  for (int hh = 0; hh < nh; ++hh) {
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, S.ms[w][hh]);
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + hh]);
     float lsum = 0.f, a = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
-      const float sc = exp2f(S.ms[w][hh] - M);
-      lsum = fmaf(sc, S.ls[w][hh], lsum);
-      a = fmaf(sc, S.accs[w][hh][i], a);
+      const float sc = exp2f(ms[w * 8 + hh] - M);
+      lsum = fmaf(sc, ls[w * 8 + hh], lsum);
+      a = fmaf(sc, accs[(w * 8 + hh) * kD + i], a);
     }
     float* part = ws.partials +
-                  ((((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + hh) * sh.max_splits) + s) *
+                  ((((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0 + hh) * sh.max_splits) + s) *
                       kPartialStride;
     part[4 + i] = a;
     if (i == 0) {
@@ -681,44 +1130,32 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   if (half == 0) out[row * kD + d] = __float2half(o + accs[0][d]);
 }
 
-// Raises a kernel's dynamic shared-memory limit.  Callers keep the result
-// in a function-local static of a function that is unique per kernel, so
-// the attribute is set once per process and never inside a graph capture.
+// Raises a kernel's dynamic shared-memory limit; callers keep the result in
+// a function-local static of a function unique per kernel, so the attribute
+// is set once per process and never inside a graph capture.
 template <typename F>
 cudaError_t set_smem(F* fn, size_t bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
-template <int KIND>
 cudaError_t encode_smem_once() {
-  static const cudaError_t status = set_smem(encode_kernel<KIND>, sizeof(EncodeSmem));
+  static const cudaError_t status = set_smem(encode_kernel, sizeof(EncodeSmem));
   return status;
 }
 
-template <int KB, int GP, int TPL>
-cudaError_t launch_decode_t(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                            int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
-                            int split_tokens, cudaStream_t stream) {
-  const size_t smem = sizeof(DecodeSmem<GP, TPL>);
-  auto* fn = decode_split_kernel<KB, GP, TPL>;
-  static const cudaError_t attr = set_smem(fn, smem);  // one static per instantiation
+template <int VB>
+cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                             const float* qrot, const int32_t* seq_lens, int batch, int split_tokens,
+                             cudaStream_t stream) {
+  // the largest layout over K widths, so one attribute value serves every call
+  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
+  const int head_blocks = (s.group + 7) / 8;
   const int nspl = static_cast<int>((s.capacity + split_tokens - 1) / split_tokens);
-  dim3 grid(nspl, batch * s.n_kv_heads, layer_count);
-  fn<<<grid, kDecThreads, smem, stream>>>(s, ws, cache, layer0, qrot, seq_lens, batch, split_tokens);
+  dim3 grid(nspl, batch * s.n_kv_heads * head_blocks, layer_count);
+  decode_mma_kernel<VB><<<grid, kDecThreads, decode_layout(s.kbits, VB).total, stream>>>(
+      s, ws, cache, layer0, qrot, seq_lens, batch, split_tokens, head_blocks);
   return cudaGetLastError();
-}
-
-template <int GP, int TPL>
-cudaError_t launch_decode_g(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                            int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
-                            int split_tokens, cudaStream_t stream) {
-  switch (s.kbits) {
-    case 1: return launch_decode_t<1, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    case 2: return launch_decode_t<2, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    case 3: return launch_decode_t<3, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    default: return launch_decode_t<4, GP, TPL>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-  }
 }
 
 }  // namespace
@@ -735,16 +1172,10 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           int layer_count, const __half* k, const __half* v, const int32_t* start,
                           const int32_t* count, int batch, int n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
-  const size_t smem = sizeof(EncodeSmem);
-  cudaError_t e = encode_smem_once<0>();
+  const cudaError_t e = encode_smem_once();
   if (e != cudaSuccess) return e;
-  e = encode_smem_once<1>();
-  if (e != cudaSuccess) return e;
-  dim3 grid(layer_count * batch * s.n_kv_heads, (n + kEncRows - 1) / kEncRows);
-  encode_kernel<0><<<grid, kEncThreads, smem, stream>>>(s, ws, cache, layer0, k, start, count, batch, n);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  encode_kernel<1><<<grid, kEncThreads, smem, stream>>>(s, ws, cache, layer0, v, start, count, batch, n);
+  dim3 grid(layer_count * batch * s.n_kv_heads, (n + kTile - 1) / kTile + 1, 2);
+  encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
   return cudaGetLastError();
 }
 
@@ -757,11 +1188,12 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                                 int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
                                 int split_tokens, cudaStream_t stream) {
-  if (s.group <= 4)
-    return launch_decode_g<4, 4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-  if (s.group <= 8)
-    return launch_decode_g<8, 2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-  return launch_decode_g<16, 1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+  switch (s.vbits) {
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+  }
 }
 
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,

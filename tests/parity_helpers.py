@@ -4,7 +4,7 @@ tables from the same calibration rows; no oracle input comes from the GPU."""
 import numpy as np
 import torch
 
-from oracle import lloyd_max, model, tqmse
+from oracle import lloyd_max, model, tiles, tqmse
 from packed_decode_attention_b200 import bgtq
 from packed_decode_attention_b200 import workloads as wl
 
@@ -65,13 +65,22 @@ def fp16_ulp_apart(a, b):
     return np.abs(ai - bi)
 
 
-def upload_oracle_rows(kv, layer, seq, head, start, enc):
-    """Write the oracle's packed bytes into the library's cache (identical caches)."""
-    n = enc["k_rec"].shape[0]
-    kv.k_records()[layer, seq, head, start:start + n].copy_(torch.from_numpy(enc["k_rec"]))
-    kv.k_norms()[layer, seq, head, start:start + n].copy_(torch.from_numpy(enc["k_norms"]))
-    kv.v_records()[layer, seq, head, start:start + n].copy_(torch.from_numpy(enc["v_rec"]))
-    kv.v_norms()[layer, seq, head, start:start + n].copy_(torch.from_numpy(enc["v_norm"]))
+def upload_oracle_rows(kv, layer, seq, head, enc):
+    """Write the oracle's packed tiles and norms (positions 0..n-1) into the library's cache."""
+    n = enc["n"]
+    nt = enc["k_tiles"].shape[0]
+    kv.k_tiles()[layer, seq, head, :nt].copy_(torch.from_numpy(enc["k_tiles"]))
+    kv.v_tiles()[layer, seq, head, :nt].copy_(torch.from_numpy(enc["v_tiles"]))
+    kv.k_norms()[layer, seq, head, :n].copy_(torch.from_numpy(enc["k_norms"]))
+    kv.v_norms()[layer, seq, head, :n].copy_(torch.from_numpy(enc["v_norm"]))
+
+
+def gpu_codes(kv, tb, layer, seq, head, n, vbits):
+    """The library's K and V codes of positions 0..n-1, unpacked with the oracle's tile definition."""
+    nt = (n + 63) // 64
+    kt = kv.k_tiles()[layer, seq, head, :nt].cpu().numpy()
+    vt = kv.v_tiles()[layer, seq, head, :nt].cpu().numpy()
+    return (tiles.unpack_k_tiles(kt, tb.groups[layer, head], n), tiles.unpack_v_tiles(vt, vbits, n), kt, vt)
 
 
 def encode_on_gpu(kv, w, layers, lens, dev, chunk=1 << 16):

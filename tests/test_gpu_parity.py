@@ -16,7 +16,8 @@ from oracle import haar, lloyd_max, model, tqmse
 from packed_decode_attention_b200 import bgtq
 from packed_decode_attention_b200 import workloads as wl
 
-from parity_helpers import (CODE_AGREEMENT, REL_TOL, compare_codes, fp16_ulp_apart, library_config,
+from oracle import tiles as otiles
+from parity_helpers import (CODE_AGREEMENT, REL_TOL, compare_codes, fp16_ulp_apart, gpu_codes, library_config,
                             oracle_config, oracle_u, row_rel_err, upload_oracle_rows)
 
 pytestmark = pytest.mark.gpu
@@ -97,20 +98,22 @@ def _encode_and_compare(w, dev, layer_seq_rows, **over):
     for h in range(cfg.n_kv_heads):
         enc = model.encode_rows(tb, 0, h, k[:, h].numpy(), v[:, h].numpy())
         widths_pos = tqmse.record_widths(tb.groups[0, h])
-        g_krec = kv.k_records()[0, 0, h, :n].cpu().numpy()
-        g_vrec = kv.v_records()[0, 0, h, :n].cpu().numpy()
-        g_kc = tqmse.unpack_records(g_krec, widths_pos)
-        g_vc = tqmse.unpack_records(g_vrec, np.full(128, cfg.v_avg_bits))
+        g_kc, g_vc, g_kt, g_vt = gpu_codes(kv, tb, 0, 0, h, n, cfg.v_avg_bits)
         fk, okk, nbk = compare_codes(g_kc, enc["k_codes"], oracle_u(tb, 0, h, k[:, h].numpy(), 0), widths_pos)
         fv, okv, nbv = compare_codes(g_vc, enc["v_codes"], oracle_u(tb, 0, h, v[:, h].numpy(), 1),
                                      np.full(128, cfg.v_avg_bits))
         assert fk >= CODE_AGREEMENT and okk, (h, fk, nbk)
         assert fv >= CODE_AGREEMENT and okv, (h, fv, nbv)
-        # rows whose codes all agree pack to identical bytes
-        same_k = np.all(g_kc == enc["k_codes"], axis=1)
-        assert np.array_equal(g_krec[same_k], enc["k_rec"][same_k])
-        same_v = np.all(g_vc == enc["v_codes"], axis=1)
-        assert np.array_equal(g_vrec[same_v], enc["v_rec"][same_v])
+        # tiles whose codes all agree pack to identical bytes
+        ntile = (n + 63) // 64
+        for t in range(ntile):
+            rows = slice(64 * t, min(n, 64 * t + 64))
+            if n % 64 and t == ntile - 1:
+                continue            # the library's last tile holds zeros past n, like the oracle's
+            if np.array_equal(g_kc[rows], enc["k_codes"][rows]):
+                assert np.array_equal(g_kt[t], enc["k_tiles"][t]), (h, t)
+            if np.array_equal(g_vc[rows], enc["v_codes"][rows]):
+                assert np.array_equal(g_vt[t], enc["v_tiles"][t]), (h, t)
         g_kn = kv.k_norms()[0, 0, h, :n].cpu().numpy()
         g_vn = kv.v_norms()[0, 0, h, :n].cpu().numpy()
         assert np.all(fp16_ulp_apart(g_kn, enc["k_norms"]) <= 1)
@@ -168,7 +171,7 @@ def _decode_identical(w, dev, lens, heads=None, split=None, **over):
             enc = model.encode_rows(tb, 0, h, k[:, h].numpy(), v[:, h].numpy())
             encs[b, h] = enc
             if ln:
-                upload_oracle_rows(kv, 0, b, h, 0, enc)
+                upload_oracle_rows(kv, 0, b, h, enc)
     q = wl.decode_query(w, 0, lens, pairing=cfg.rope_pairing)        # [B, Hq, 128]
     out = torch.full((1, len(lens), cfg.n_q_heads, 128), float("nan"), dtype=torch.float16, device=dev)
     seq = torch.tensor(lens, dtype=torch.int32, device=dev)
@@ -181,8 +184,8 @@ def _decode_identical(w, dev, lens, heads=None, split=None, **over):
     for b in range(len(lens)):
         for h in heads:
             e = encs[b, h]
-            ref = model.decode(tb, 0, h, q[b, h * g:(h + 1) * g].numpy(), e["k_rec"], e["k_norms"], e["v_rec"],
-                               e["v_norm"])
+            ref = model.decode(tb, 0, h, q[b, h * g:(h + 1) * g].numpy(), e["k_tiles"], e["k_norms"], e["v_tiles"],
+                               e["v_norm"], e["n"])
             err = row_rel_err(got[b, h * g:(h + 1) * g], ref)
             if lens[b] == 0:
                 assert np.all(got[b, h * g:(h + 1) * g] == 0)
@@ -224,7 +227,7 @@ def test_decode_single_token_is_v_hat(dev):
     v = wl.values(w, 0, 0, 0, 1)[:, 0].numpy()
     enc = model.encode_rows(tb, 0, 0, wl.keys(w, 0, 0, 0, 1)[:, 0].numpy(), v)
     from oracle.attention import dequantise_values
-    vh = dequantise_values(enc["v_rec"], enc["v_norm"], tb.v_rot[0, 0], tb.codebooks[3], 3, 128)
+    vh = dequantise_values(enc["v_codes"], enc["v_norm"], tb.v_rot[0, 0], tb.codebooks[3], 128)
     assert np.all(row_rel_err(got[0], np.repeat(vh, 4, axis=0)) <= REL_TOL)
 
 
@@ -248,11 +251,11 @@ def test_multi_layer_launch_equals_per_layer(dev):
     start = torch.zeros(1, dtype=torch.int32, device=dev)
     count = torch.full((1,), n, dtype=torch.int32, device=dev)
     kv.encode_append(0, k, v, start, count, layer_count=3)
-    multi = kv.k_records()[:3, 0].clone()
+    multi = kv.k_tiles()[:3, 0].clone()
     kv.cache.zero_()
     for l in range(3):
         kv.encode_append(l, k[l:l + 1], v[l:l + 1], start, count)
-    assert torch.equal(multi, kv.k_records()[:3, 0])
+    assert torch.equal(multi, kv.k_tiles()[:3, 0])
     q = torch.stack([wl.decode_query(w, l, [n]) for l in range(3)]).to(dev)
     seq = torch.full((1,), n, dtype=torch.int32, device=dev)
     out_all = torch.empty((3, 1, cfg.n_q_heads, 128), dtype=torch.float16, device=dev)
@@ -280,8 +283,9 @@ def test_capacity_overflow_and_bad_lengths_raise_flags(dev):
     count = torch.full((1,), 20, dtype=torch.int32, device=dev)
     kv.encode_append(0, k, v, start, count)
     assert kv.device_error() == bgtq.DEVERR_CAPACITY
-    assert kv.k_records()[0, 0, 0, 90:100].any()          # in-range rows written
-    assert not kv.k_records()[0, 0, 0, :90].any()
+    assert kv.k_tiles()[0, 0, 0, 1].any()                 # positions 90..99 written (tile 1)
+    assert not kv.k_tiles()[0, 0, 0, 0].any()             # positions 0..63 untouched
+    assert kv.k_norms()[0, 0, 0, 90:100].any() and not kv.k_norms()[0, 0, 0, :90].any()
     bad = torch.full((1,), -1, dtype=torch.int32, device=dev)
     kv.encode_append(0, k, v, bad, count)
     assert kv.device_error() == bgtq.DEVERR_ARG
@@ -358,4 +362,28 @@ def test_stage_calls_equal_decode_attn(dev):
     kv.decode_combine(0, seq, bb)
     assert torch.equal(a, bb)
     assert kv.device_error() == 0
+    kv.close()
+
+
+def test_appends_in_pieces_equal_one_encode(dev):
+    """Appends at unaligned starts rewrite partly covered tiles; the result
+    is the same packed cache as one encode of all rows."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], seq_len=400, n_calib=64)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    kv.allocate(cq.to(dev), ck.to(dev))
+    n = 333
+    k = wl.keys(w, 0, 0, 0, n)[None, None].to(dev)
+    v = wl.values(w, 0, 0, 0, n)[None, None].to(dev)
+    one = torch.zeros(1, dtype=torch.int32, device=dev)
+    kv.encode_append(0, k, v, one * 0, one * n)
+    whole_k, whole_v = kv.k_tiles().clone(), kv.v_tiles().clone()
+    whole_kn, whole_vn = kv.k_norms().clone(), kv.v_norms().clone()
+    kv.cache.zero_()
+    for a, b2 in ((0, 37), (37, 38), (38, 64), (64, 200), (200, 333)):
+        kv.encode_append(0, k[:, :, a:b2].contiguous(), v[:, :, a:b2].contiguous(), one * a, one * (b2 - a))
+    assert kv.device_error() == 0
+    assert torch.equal(whole_k, kv.k_tiles()) and torch.equal(whole_v, kv.v_tiles())
+    assert torch.equal(whole_kn, kv.k_norms()) and torch.equal(whole_vn, kv.v_norms())
     kv.close()

@@ -168,17 +168,17 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   return BGTQ_OK;
 }
 
-// Tokens per split-K chunk: about two CTAs per SM over the launch (the decode
-// kernel fits two per SM), in whole tiles, within max_splits.
+// Tokens per split-K chunk: one wave of about three CTAs per SM (the decode
+// kernel fits three per SM) over all (layer, sequence, head block) units, in
+// whole 64-position tiles, within max_splits.
 int auto_split_tokens(const bgtq_state* st, int units) {
-  const int64_t cap = st->cfg.capacity_tokens;
+  const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
   const int maxs = max_splits_of(&st->cfg);
-  const int target = 2 * st->num_sms;
-  const int nspl = std::max(1, std::min(maxs, (target + units - 1) / std::max(units, 1)));
-  int64_t t = (cap + nspl - 1) / nspl;
-  t = (t + bgtq::kTile - 1) / bgtq::kTile * bgtq::kTile;
-  while ((cap + t - 1) / t > maxs) t += bgtq::kTile;
-  return static_cast<int>(t);
+  const int slots = 3 * st->num_sms;
+  const int per_unit = std::max(1, std::min(maxs, slots / std::max(units, 1)));
+  int64_t per_split = (tiles + per_unit - 1) / per_unit;
+  while ((tiles + per_split - 1) / per_split > maxs) ++per_split;
+  return static_cast<int>(per_split * bgtq::kTile);
 }
 
 }  // namespace

@@ -638,8 +638,9 @@ __global__ void __launch_bounds__(128) rotate_query_kernel(Shape sh, Workspace w
 // ---------------------------------------------------------------------------
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kWaitLimit = 1 << 22;
+constexpr float kRescaleSlack = 8.f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -699,63 +700,76 @@ __host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
   return L;
 }
 
-// Logits of one width group for the warp's tile: S[mu][4] (M-tile mu).
+// The lane's four selectors (M-tiles 0..3) of chunk j of a width-B group:
+// a quartet for full chunks; for the partial chunk, a quartet of the lanes
+// with a full quad, half selectors of a virtual lane for the half quad, 0
+// for lanes with no coordinates (their B rows are 0).
 template <int B>
-__device__ __forceinline__ void group_logits(const uint32_t* kt, const GroupGeo& q, const uint4* bq,
-                                             const uint32_t* tab8, int lane, float (*S)[4]) {
-  ByteTab t;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    t.lo[i] = tab8[i];
-    t.hi[i] = tab8[4 + i];
-  }
-  const uint32_t* gw = kt + q.word;
-  for (int j = 0; j < q.nfull; ++j) {
-    uint32_t w[B], s[4];
+__device__ __forceinline__ void chunk_selectors(const uint32_t* gw, int j, int nfull, int r, int lane, uint32_t* s) {
+  uint32_t w[B];
+  if (j < nfull) {
 #pragma unroll
     for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
     quartet_decode<B>(w, s);
-    const uint4 bf = bq[(q.chunk + j) * 32 + lane];
+    return;
+  }
+  const uint32_t* pc = gw + nfull * 32 * B;
+  const int nf = r >> 2, g = lane >> 2, tl = lane & 3;
+  s[0] = s[1] = s[2] = s[3] = 0u;
+  if (tl < nf) {
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * k + g * nf + tl];
+    quartet_decode<B>(w, s);
+  } else if ((r & 3) && tl == nf) {
+    uint32_t sv[4];
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * B + 4 * k + (g >> 1)];
+    quartet_decode<B>(w, sv);
+    const int sh = 16 * (g & 1);
 #pragma unroll
     for (int mu = 0; mu < 4; ++mu) {
-      uint32_t r0, r1, r2, r3;
-      lookup4<B>(t, s[mu], r0, r2);
-      lookup4<B>(t, s[mu] >> 16, r1, r3);
-      mma16816(S[mu], r0, r1, r2, r3, bf.x, bf.y);
-      mma16816(S[mu], r0, r1, r2, r3, bf.z, bf.w);
+      const uint32_t x = (sv[mu] >> sh) & 0xFFFFu;
+      s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
     }
   }
-  if (q.r) {
-    const uint32_t* pc = gw + q.nfull * 32 * B;
-    const int nf = q.r >> 2;
-    const int g = lane >> 2, tl = lane & 3;
-    uint32_t s[4] = {0u, 0u, 0u, 0u};
-    uint32_t w[B];
-    if (tl < nf) {
+}
+
+// S[mu] += A(selector s[mu]) * (q~ hi + q~ lo) for the four M-tiles of a chunk.
+template <bool WIDE>
+__device__ __forceinline__ void chunk_mma(const ByteTab& t, const uint32_t* s, uint4 bf, float (*S)[4]) {
+  uint32_t a[4][4];
 #pragma unroll
-      for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * k + g * nf + tl];
-      quartet_decode<B>(w, s);
-    } else if ((q.r & 3) && tl == nf) {
-      uint32_t sv[4];
+  for (int mu = 0; mu < 4; ++mu) {
+    lookup4<WIDE ? 4 : 3>(t, s[mu], a[mu][0], a[mu][2]);
+    lookup4<WIDE ? 4 : 3>(t, s[mu] >> 16, a[mu][1], a[mu][3]);
+  }
 #pragma unroll
-      for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * B + 4 * k + (g >> 1)];
-      quartet_decode<B>(w, sv);
-      const int sh = 16 * (g & 1);
+  for (int mu = 0; mu < 4; ++mu) mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.x, bf.y);
 #pragma unroll
-      for (int mu = 0; mu < 4; ++mu) {
-        const uint32_t x = (sv[mu] >> sh) & 0xFFFFu;
-        s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
-      }
+  for (int mu = 0; mu < 4; ++mu) mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.z, bf.w);
+}
+
+// Logits of one width group for the warp's tile: S[mu][4] (M-tile mu).
+__device__ __forceinline__ void group_logits(const uint32_t* kt, const GroupGeo& q, const uint4* bq,
+                                             const uint32_t* tab8, int lane, float (*S)[4]) {
+  ByteTab t;
+  const uint4 tl = *reinterpret_cast<const uint4*>(tab8);
+  const uint4 th = *reinterpret_cast<const uint4*>(tab8 + 4);
+  t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
+  t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+  const uint32_t* gw = kt + q.word;
+  const int nchunks = q.nfull + (q.r ? 1 : 0);
+  for (int j = 0; j < nchunks; ++j) {
+    uint32_t s[4];
+    switch (q.width) {
+      case 1: chunk_selectors<1>(gw, j, q.nfull, q.r, lane, s); break;
+      case 2: chunk_selectors<2>(gw, j, q.nfull, q.r, lane, s); break;
+      case 3: chunk_selectors<3>(gw, j, q.nfull, q.r, lane, s); break;
+      default: chunk_selectors<4>(gw, j, q.nfull, q.r, lane, s); break;
     }
-    const uint4 bf = bq[(q.chunk + q.nfull) * 32 + lane];
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      uint32_t r0, r1, r2, r3;
-      lookup4<B>(t, s[mu], r0, r2);
-      lookup4<B>(t, s[mu] >> 16, r1, r3);
-      mma16816(S[mu], r0, r1, r2, r3, bf.x, bf.y);
-      mma16816(S[mu], r0, r1, r2, r3, bf.z, bf.w);
-    }
+    const uint4 bf = bq[(q.chunk + j) * 32 + lane];
+    if (q.width == 4) chunk_mma<true>(t, s, bf, S);
+    else chunk_mma<false>(t, s, bf, S);
   }
 }
 
@@ -930,7 +944,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
       for (int mu = 0; mu < 4; ++mu)
 #pragma unroll
         for (int r = 0; r < 4; ++r) S[mu][r] = 0.f;
-      BGTQ_WIDTH_SWITCH(q.width, group_logits, kt, q, bq, tabk + 8 * g, lane, S)
+      group_logits(kt, q, bq, tabk + 8 * g, lane, S);
 #pragma unroll
       for (int mu = 0; mu < 4; ++mu) {
         const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
@@ -956,12 +970,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
       mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
       mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
     }
-    float alpha[2], sum[2] = {0.f, 0.f};
+    // The reference maximum moves only when the tile's maximum exceeds it by
+    // more than kRescaleSlack (log2 units), so O is rescaled rarely; weights
+    // stay <= 2^kRescaleSlack and l and O always share the same reference.
+    float alpha[2] = {1.f, 1.f}, sum[2] = {0.f, 0.f};
+    bool moved = false;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const float mnew = fmaxf(m_run[c], mx[c]);
-      alpha[c] = exp2f(m_run[c] - mnew);
-      m_run[c] = mnew;
+      if (mx[c] > m_run[c] + kRescaleSlack) {
+        alpha[c] = exp2f(m_run[c] - mx[c]);
+        m_run[c] = mx[c];
+        moved = true;
+      }
     }
     uint32_t bp[4][2];
 #pragma unroll
@@ -983,13 +1003,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
     }
     l_run[0] = fmaf(l_run[0], alpha[0], sum[0]);
     l_run[1] = fmaf(l_run[1], alpha[1], sum[1]);
+    if (moved) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        O[m][0] *= alpha[0];
+        O[m][1] *= alpha[1];
+        O[m][2] *= alpha[0];
+        O[m][3] *= alpha[1];
+      }
+    }
     // P V in V's rotated basis
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
-      O[m][0] *= alpha[0];
-      O[m][1] *= alpha[1];
-      O[m][2] *= alpha[0];
-      O[m][3] *= alpha[1];
       uint32_t w[VB], sv[4];
 #pragma unroll
       for (int kk = 0; kk < VB; ++kk) w[kk] = vt[m * 32 * VB + 32 * kk + lane];

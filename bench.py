@@ -275,9 +275,7 @@ def main():
     lens = wl.seq_lens(w)
     L, H, HQ, B = w.n_layers, w.n_kv_heads, w.n_q_heads, w.batch
     cap = w.seq_len
-    cfg = bgtq.Config(n_layers=L, n_kv_heads=H, n_q_heads=HQ, max_batch=B, capacity_tokens=cap,
-                      k_avg_bits=w.k_bits, v_avg_bits=w.v_bits, seed=w.seed,
-                      max_splits=64 if B > 4 else 0)
+    cfg = bgtq.Config(**wl.bench_config_fields(w))
     kv = bgtq.PackedKVCache(cfg, dev)
     stream = torch.cuda.current_stream()
 

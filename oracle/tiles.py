@@ -150,12 +150,24 @@ def _pack(codes, bitmap, nbytes):
     return np.packbits(bits, axis=1, bitorder="little")
 
 
-def _unpack(tiles, bitmap, npos):
+def _inverse(bitmap, npos):
+    """inv[token, position, code_bit] = the tile bit holding it (-1 if none)."""
     tok, pos, cb = bitmap
+    inv = np.full((TILE, npos, 4), -1, dtype=np.int64)
+    inv[tok, pos, cb] = np.arange(len(tok))
+    return inv
+
+
+def _unpack(tiles, bitmap, npos):
+    """uint8 [tiles, nbytes] -> codes [tiles, 64, npos]: gather each code's bits."""
+    inv = _inverse(bitmap, npos)
     tiles = np.asarray(tiles, dtype=np.uint8)
-    bits = np.unpackbits(tiles, axis=1, bitorder="little").astype(np.int64)
+    bits = np.unpackbits(tiles, axis=1, bitorder="little")
     out = np.zeros((tiles.shape[0], TILE, npos), dtype=np.int64)
-    np.add.at(out, (slice(None), tok, pos), bits << cb[None, :])
+    for k in range(4):
+        have = inv[:, :, k] >= 0
+        idx = np.where(have, inv[:, :, k], 0)
+        out += (bits[:, idx].astype(np.int64) * have[None]) << k
     return out
 
 

@@ -371,6 +371,7 @@ struct EncodeSmem {
   float mt[kD][kD];              // mt[j][i] = R[i][j] (record order)
   float fac[kTile][kNumGroupsMax];
   __half nrm[kTile][kNumGroupsMax];
+  float fac2[kD];                // partial rotation sums of the append path
   uint8_t codes[kTile][kD];
   uint32_t words[1024];
   float thr[5][16];
@@ -433,8 +434,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   }
   for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
   const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
-  for (int i = tid; i < kD * kD / 4; i += kEncThreads)
-    reinterpret_cast<float4*>(&S.mt[0][0])[i] = reinterpret_cast<const float4*>(mglob)[i];
+  const int nrows = tr1 - tr0;
+  if (nrows > 16)  // the register-tile path reads the rotation from shared memory
+    for (int i = tid; i < kD * kD / 4; i += kEncThreads)
+      reinterpret_cast<float4*>(&S.mt[0][0])[i] = reinterpret_cast<const float4*>(mglob)[i];
   __syncthreads();
   const int ng = S.lay.n_groups;
   const int npos = S.lay.n_positions;
@@ -494,23 +497,31 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   }
   __syncthreads();
   // y = R x per new row, then the codes
-  const int nrows = tr1 - tr0;
   if (nrows <= 16) {
-    // few rows (decode-time appends): one output per thread
-    const int i = tid & (kD - 1);
+    // few rows (decode-time appends): two threads per output, each holding
+    // half of the rotation's column in registers (read from global memory
+    // with all loads in flight at once; zero outside the output's group);
+    // the two partial sums meet in shared memory
+    const int i = tid & (kD - 1), half = tid >> 7;
+    float m[64];
+#pragma unroll
+    for (int u = 0; u < 64; ++u) m[u] = __ldg(mglob + (half * 64 + u) * kD + i);
     const int g = S.gof[i];
-    if (g >= 0) {
-      const int w = S.lay.width[g];
-      const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
-      const int nt = (1 << w) - 1;
-      for (int r = tr0 + (tid >> 7); r < tr1; r += 2) {
-        float y = 0.f;
-        for (int j = j0; j < j1; ++j) y = fmaf(S.mt[j][i], S.xt[j][r], y);
-        const float u = y * S.fac[r][g];
+    for (int r = tr0; r < tr1; ++r) {
+      float y = 0.f;
+#pragma unroll
+      for (int u = 0; u < 64; ++u) y = fmaf(m[u], S.xt[half * 64 + u][r], y);
+      if (half == 1) S.fac2[i] = y;
+      __syncthreads();
+      if (half == 0 && g >= 0) {
+        const int w = S.lay.width[g];
+        const float u = (y + S.fac2[i]) * S.fac[r][g];
         int code = 0;
+        const int nt = (1 << w) - 1;
         for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
         S.codes[r][i] = static_cast<uint8_t>(code);
       }
+      __syncthreads();
     }
   } else {
     // register tile: 4 rows x 8 outputs per thread over all 64 rows
@@ -588,32 +599,45 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
 // ---------------------------------------------------------------------------
 // a4: rotate the query.  Grid (layer_count * batch * Hq), 128 threads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
-                                                           const __half* __restrict__ q, int batch,
-                                                           float* __restrict__ qrot) {
+constexpr int kRotThreads = 256;
+
+__global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
+                                                                   const __half* __restrict__ q, int batch,
+                                                                   float* __restrict__ qrot) {
+  // the decode kernel that follows may start its own set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int hq = blockIdx.x % sh.n_q_heads;
   const int b = (blockIdx.x / sh.n_q_heads) % batch;
   const int li = blockIdx.x / (sh.n_q_heads * batch);
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const LayoutDev& lay = ws.layouts[layer * sh.n_kv_heads + kvh];
+  const int tid = threadIdx.x, i = tid & (kD - 1), half = tid >> 7;
+  // this thread's half column of the (block-diagonal) rotation, all loads in flight at once
+  const float* mt = ws.mkt + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  float m[64];
+#pragma unroll
+  for (int u = 0; u < 64; ++u) m[u] = __ldg(mt + (half * 64 + u) * kD + i);
   __shared__ float qp[kD];
+  __shared__ float part[kD];
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  const int i = threadIdx.x;
-  qp[i] = __half2float(q[row * kD + lay.perm[i]]);
+  if (tid < kD) qp[tid] = __half2float(q[row * kD + lay.perm[tid]]);
   __syncthreads();
-  float out = 0.f;
-  if (i < lay.n_positions) {
-    int g = 0;
-    for (int t = 1; t < lay.n_groups; ++t)
-      if (i >= lay.start[t]) g = t;
-    const float* mt = ws.mkt + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-    float s = 0.f;
-    const int j1 = lay.start[g] + lay.size[g];
-    for (int j = lay.start[g]; j < j1; ++j) s = fmaf(mt[j * kD + i], qp[j], s);
-    out = s * lay.inv_sqrt_d[g] * kInvSqrtD;
+  float sacc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 64; ++u) sacc = fmaf(m[u], qp[half * 64 + u], sacc);
+  if (half == 1) part[i] = sacc;
+  __syncthreads();
+  if (half == 0) {
+    float out = 0.f;
+    if (i < lay.n_positions) {
+      int g = 0;
+      for (int t = 1; t < lay.n_groups; ++t)
+        if (i >= lay.start[t]) g = t;
+      out = (sacc + part[i]) * lay.inv_sqrt_d[g] * kInvSqrtD;
+    }
+    qrot[row * kD + i] = out;
   }
-  qrot[row * kD + i] = out;
 }
 
 // ---------------------------------------------------------------------------
@@ -796,11 +820,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
   const int b = blockIdx.y / (head_blocks * sh.n_kv_heads);
   const int li = blockIdx.z;
   const int layer = layer0 + li;
-  int len = seq_lens[b];
-  if (len < 0 || len > sh.capacity) len = 0;  // flagged by the combine kernel
-  const int t0 = s * split_tokens;
-  if (t0 >= len) return;
-  const int t1 = min(t0 + split_tokens, len);
   const int G = sh.group;
   const int h0 = 8 * hb;                       // first query head of this block within the group
   const int nh = min(8, G - h0);
@@ -841,6 +860,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
   if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
   __syncthreads();
   if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  // Launched as a programmatic dependent of the previous kernel (the query
+  // rotation): everything above reads only the library's tables; the
+  // sequence lengths, rotated queries and cache are read after that kernel
+  // has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  int len = seq_lens[b];
+  if (len < 0 || len > sh.capacity) len = 0;  // flagged by the combine kernel
+  const int t0 = s * split_tokens;
+  if (t0 >= len) return;
+  const int t1 = min(t0 + split_tokens, len);
   {
     const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
     int nchunk = 0;
@@ -1025,6 +1054,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
     __syncwarp();
     if (lane == 0 && k + kStages < my_tiles) issue(k + kStages);
   }
+  // the combine kernel may be scheduled now; it waits for this grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const bool timed_out = failed_at >= 0;
   if (timed_out) {
     if (lane == 0) atomicOr(ws.err, kErrTimeout);
@@ -1092,6 +1123,16 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the inverse V rotation's column for this thread (a library table),
+  // loaded while the previous kernel finishes
+  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  const int d = tid & (kD - 1), half = tid >> 7;
+  float mvr[64];
+#pragma unroll
+  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + d);
+  // Launched as a programmatic dependent of the split pass: inputs, partials
+  // and the output are touched only after that kernel has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = seq_lens[b];
   if (len < 0 || len > sh.capacity) {
     if (tid == 0 && hq == 0) atomicOr(ws.err, kErrSeqLen);
@@ -1145,11 +1186,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   }
   __syncthreads();
   // inverse V rotation: thread pair (d, half) sums half of the 128 inputs
-  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-  const int d = tid & (kD - 1), half = tid >> 7;
   float o = 0.f;
-#pragma unroll 8
-  for (int r = half * 64; r < half * 64 + 64; ++r) o = fmaf(mv[r * kD + d], a_s[r], o);
+#pragma unroll
+  for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
   if (half == 1) accs[0][d] = o;
   __syncthreads();
   if (half == 0) out[row * kD + d] = __float2half(o + accs[0][d]);
@@ -1168,6 +1207,26 @@ cudaError_t encode_smem_once() {
   return status;
 }
 
+// Launches a kernel as a programmatic dependent of the previous kernel in
+// the stream: it may start while that kernel finishes and must execute
+// griddepcontrol.wait before reading that kernel's results.  Used only for
+// the second and third kernels of a decode call, never for the first.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
                              const float* qrot, const int32_t* seq_lens, int batch, int split_tokens,
@@ -1178,9 +1237,8 @@ cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev
   const int head_blocks = (s.group + 7) / 8;
   const int nspl = static_cast<int>((s.capacity + split_tokens - 1) / split_tokens);
   dim3 grid(nspl, batch * s.n_kv_heads * head_blocks, layer_count);
-  decode_mma_kernel<VB><<<grid, kDecThreads, decode_layout(s.kbits, VB).total, stream>>>(
-      s, ws, cache, layer0, qrot, seq_lens, batch, split_tokens, head_blocks);
-  return cudaGetLastError();
+  return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
+                          ws, cache, layer0, qrot, seq_lens, batch, split_tokens, head_blocks);
 }
 
 }  // namespace
@@ -1206,7 +1264,7 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
 
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream) {
-  rotate_query_kernel<<<layer_count * batch * s.n_q_heads, kD, 0, stream>>>(s, ws, layer0, q, batch, qrot);
+  rotate_query_kernel<<<layer_count * batch * s.n_q_heads, kRotThreads, 0, stream>>>(s, ws, layer0, q, batch, qrot);
   return cudaGetLastError();
 }
 
@@ -1224,9 +1282,8 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int split_tokens, __half* out,
                            cudaStream_t stream) {
-  combine_kernel<<<layer_count * batch * s.n_q_heads, kCombThreads, 0, stream>>>(s, ws, layer0, seq_lens, batch,
-                                                                                 split_tokens, out);
-  return cudaGetLastError();
+  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kCombThreads), 0, stream, s,
+                          ws, layer0, seq_lens, batch, split_tokens, out);
 }
 
 }  // namespace bgtq

@@ -152,3 +152,31 @@ def scaled(w, **changes):
     d = dict(w.__dict__)
     d.update(changes)
     return Workload(**d)
+
+
+def bench_config_fields(w):
+    """Library config fields the benchmark and its full-size tests use for a workload."""
+    return dict(n_layers=w.n_layers, n_kv_heads=w.n_kv_heads, n_q_heads=w.n_q_heads, max_batch=w.batch,
+                capacity_tokens=w.seq_len, k_avg_bits=w.k_bits, v_avg_bits=w.v_bits, seed=w.seed,
+                max_splits=64 if w.batch > 4 else 0)
+
+
+def prefill(kv, w, lens, device, chunk=32768, on_chunk=None):
+    """Append every sequence's keys/values [0, len) of every layer to a
+    library cache, in chunks generated on ``device``.  ``on_chunk(layer, seq,
+    start, k, v)`` sees each chunk (fp16 [n, Hkv, 128]) after it is queued."""
+    for layer in range(w.n_layers):
+        for b in range(w.batch):
+            for s0 in range(0, lens[b], chunk):
+                n = min(chunk, lens[b] - s0)
+                kk = torch.zeros((1, w.batch, n, w.n_kv_heads, 128), dtype=torch.float16, device=device)
+                vv = torch.zeros_like(kk)
+                kk[0, b] = keys(w, layer, b, s0, n, device=device)
+                vv[0, b] = values(w, layer, b, s0, n, device=device)
+                start = torch.zeros(w.batch, dtype=torch.int32, device=device)
+                count = torch.zeros(w.batch, dtype=torch.int32, device=device)
+                start[b] = s0
+                count[b] = n
+                kv.encode_append(layer, kk, vv, start, count)
+                if on_chunk is not None:
+                    on_chunk(layer, b, s0, kk[0, b], vv[0, b])

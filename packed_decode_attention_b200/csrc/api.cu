@@ -25,6 +25,7 @@ struct bgtq_state {
   size_t cache_off[4];
   size_t cache_bytes, ws_bytes;
   int split_tokens = 0;  // 0 = automatic
+  int ctas_per_sm = 0;   // resident decode CTAs per SM (looked up on first use)
   int num_sms = 148;
   bool ready = false;
   bool have_energy = false;
@@ -59,10 +60,16 @@ int max_splits_of(const bgtq_config* c) { return c->max_splits == 0 ? 256 : c->m
 
 struct Layout {
   size_t krec, knorm, vrec, vnorm, cache_total;
-  size_t err, codebook, layouts, mkt, mvt, mv, energy_q, energy_k, qrot, partials, ws_total;
+  size_t err, codebook, layouts, dectab, mkt, mvt, mv, energy_q, energy_k, qrot, qfrag, partials, ws_total;
 };
 
 int64_t tiles_of(const bgtq_config* c) { return (c->capacity_tokens + bgtq::kTile - 1) / bgtq::kTile; }
+
+// q~ fragment bytes for calls of up to layer_count layers.
+size_t frag_bytes(const bgtq_config* c, int layer_count) {
+  const int hbs = (c->n_q_heads / c->n_kv_heads + 7) / 8;
+  return size_t(layer_count) * c->max_batch * c->n_kv_heads * hbs * bgtq::kFragEntries * 16;
+}
 
 Layout plan(const bgtq_config* c) {
   Layout p{};
@@ -78,14 +85,16 @@ Layout plan(const bgtq_config* c) {
   p.err = 0;
   p.codebook = align_up(p.err + sizeof(uint32_t));
   p.layouts = align_up(p.codebook + sizeof(bgtq::CodebookDev));
-  p.mkt = align_up(p.layouts + lh * sizeof(bgtq::LayoutDev));
+  p.dectab = align_up(p.layouts + lh * sizeof(bgtq::LayoutDev));
+  p.mkt = align_up(p.dectab + lh * sizeof(bgtq::DecodeTableDev));
   p.mvt = align_up(p.mkt + lh * kD * kD * sizeof(float));
   p.mv = align_up(p.mvt + lh * kD * kD * sizeof(float));
   p.energy_q = align_up(p.mv + lh * kD * kD * sizeof(float));
   p.energy_k = align_up(p.energy_q + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
   p.qrot = align_up(p.energy_k + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
   const size_t qrows = size_t(c->n_layers) * c->max_batch * c->n_q_heads;
-  p.partials = align_up(p.qrot + qrows * kD * sizeof(float));
+  p.qfrag = align_up(p.qrot + qrows * kD * sizeof(float));
+  p.partials = align_up(p.qfrag + frag_bytes(c, c->n_layers));
   p.ws_total = align_up(p.partials + qrows * max_splits_of(c) * bgtq::kPartialStride * sizeof(float));
   return p;
 }
@@ -93,6 +102,58 @@ Layout plan(const bgtq_config* c) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+uint32_t half_bits(float x) {
+  const __half h = __float2half_rn(x);
+  uint16_t v;
+  std::memcpy(&v, &h, 2);
+  return v;
+}
+
+// PRMT byte tables of a width's fp16 codebook: words 0..3 hold the low
+// bytes of entries 4i..4i+3, words 4..7 the high bytes.
+void byte_table(int bits, uint32_t* out) {
+  std::vector<float> cen, thr;
+  bgtq::lloyd_max_codebook(bits, &cen, &thr);
+  for (int i = 0; i < 8; ++i) out[i] = 0;
+  for (int e = 0; e < (1 << bits); ++e) {
+    const uint32_t h = half_bits(cen[e]);
+    out[e >> 2] |= (h & 0xFFu) << (8 * (e & 3));
+    out[4 + (e >> 2)] |= (h >> 8) << (8 * (e & 3));
+  }
+}
+
+// The split decode kernel's table for one (layer, KV head) layout.
+bgtq::DecodeTableDev decode_table(const bgtq::LayoutDev& d, int vbits) {
+  bgtq::DecodeTableDev t;
+  std::memset(&t, 0, sizeof(t));
+  for (int g = 0; g < d.n_groups; ++g) {
+    const int size = d.size[g], bw = d.width[g];
+    t.grp[g][0] = bw;
+    t.grp[g][1] = size >> 4;
+    t.grp[g][2] = size & 15;
+    t.grp[g][3] = d.tile_word[g];
+    t.grp[g][4] = d.chunk_base[g];
+    t.grp[g][5] = size;
+    t.grp[g][6] = d.start[g];
+    byte_table(bw, t.tabk[g]);
+    // partial chunk: lanes with a full quad read their quartet (word k at
+    // 8 nf k + g nf + t); the half-quad lanes read virtual lane g / 2 (word k
+    // at 8 nf b + 4 k + g / 2, upper half for odd g); other lanes read word 0
+    const int r = size & 15, nf = r >> 2;
+    for (int ln = 0; ln < 32; ++ln) {
+      const int gg = ln >> 2, tl = ln & 3;
+      uint32_t pd = 0;
+      if (tl < nf)
+        pd = uint32_t(gg * nf + tl) | (uint32_t(8 * nf) << 12);
+      else if ((r & 3) && tl == nf)
+        pd = uint32_t(8 * nf * bw + (gg >> 1)) | (4u << 12) | (1u << 20) | (uint32_t(gg & 1) << 21);
+      t.pdesc[g][ln] = pd;
+    }
+  }
+  byte_table(vbits, t.tabv);
+  return t;
+}
 
 // Builds the host tables for the current widths and uploads them.
 int build_and_upload(bgtq_state* st, cudaStream_t stream) {
@@ -102,6 +163,7 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   st->krot.assign(size_t(L) * H * 4 * kD * kD, 0.f);
   st->vrot.assign(size_t(L) * H * kD * kD, 0.f);
   std::vector<bgtq::LayoutDev> ldev(size_t(L) * H);
+  std::vector<bgtq::DecodeTableDev> dtab(size_t(L) * H);
   std::vector<float> mkt(size_t(L) * H * kD * kD, 0.f), mvt(size_t(L) * H * kD * kD), mv(size_t(L) * H * kD * kD);
   for (int l = 0; l < L; ++l) {
     for (int h = 0; h < H; ++h) {
@@ -157,8 +219,12 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
         }
     }
   }
+  for (size_t i = 0; i < ldev.size(); ++i) dtab[i] = decode_table(ldev[i], c.v_avg_bits);
   cudaError_t e = cudaMemcpyAsync(st->ws.layouts, ldev.data(), ldev.size() * sizeof(bgtq::LayoutDev),
                                   cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->ws.dectab, dtab.data(), dtab.size() * sizeof(bgtq::DecodeTableDev),
+                        cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mkt, mkt.data(), mkt.size() * 4, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mvt, mvt.data(), mvt.size() * 4, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mv, mv.data(), mv.size() * 4, cudaMemcpyHostToDevice, stream);
@@ -168,17 +234,17 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   return BGTQ_OK;
 }
 
-// Tokens per split-K chunk: one wave of about three CTAs per SM (the decode
-// kernel fits three per SM) over all (layer, sequence, head block) units, in
-// whole 64-position tiles, within max_splits.
-int auto_split_tokens(const bgtq_state* st, int units) {
+// Split-K partials per (layer, sequence, KV head, head block): one wave of
+// resident decode CTAs over all such units (the CTAs of a unit share its
+// tiles round-robin), at most max_splits and one per 4 tiles of capacity.
+int auto_splits(bgtq_state* st, int units) {
+  if (st->ctas_per_sm <= 0) st->ctas_per_sm = std::max(1, bgtq::decode_ctas_per_sm(st->shape));
   const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
-  const int maxs = max_splits_of(&st->cfg);
-  const int slots = 3 * st->num_sms;
-  const int per_unit = std::max(1, std::min(maxs, slots / std::max(units, 1)));
-  int64_t per_split = (tiles + per_unit - 1) / per_unit;
-  while ((tiles + per_split - 1) / per_split > maxs) ++per_split;
-  return static_cast<int>(per_split * bgtq::kTile);
+  const int64_t slots = int64_t(st->ctas_per_sm) * st->num_sms;
+  int64_t n = slots / std::max(units, 1);
+  n = std::min<int64_t>(n, max_splits_of(&st->cfg));
+  n = std::min<int64_t>(n, (tiles + 3) / 4);
+  return static_cast<int>(std::max<int64_t>(n, 1));
 }
 
 }  // namespace
@@ -236,7 +302,9 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->ws.mv = reinterpret_cast<float*>(w8 + p.mv);
   st->ws.energy_q = reinterpret_cast<unsigned __int128*>(w8 + p.energy_q);
   st->ws.energy_k = reinterpret_cast<unsigned __int128*>(w8 + p.energy_k);
+  st->ws.dectab = reinterpret_cast<bgtq::DecodeTableDev*>(w8 + p.dectab);
   st->ws.qrot = reinterpret_cast<float*>(w8 + p.qrot);
+  st->ws.qfrag = reinterpret_cast<uint4*>(w8 + p.qfrag);
   st->ws.partials = reinterpret_cast<float*>(w8 + p.partials);
   st->widths.assign(size_t(cfg->n_layers) * cfg->n_kv_heads * bgtq::kBlocks, 0);
   int dev = 0;
@@ -433,10 +501,13 @@ int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, 
   return BGTQ_OK;
 }
 
-int split_for(const bgtq_state* st, int32_t layer_count, int32_t batch) {
+// Number of split-K partials per unit for a call (see auto_splits); a set
+// split size t gives ceil(capacity / t).
+int split_for(bgtq_state* st, int32_t layer_count, int32_t batch) {
   const int head_blocks = (st->shape.group + 7) / 8;
-  return st->split_tokens > 0 ? st->split_tokens
-                              : auto_split_tokens(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count);
+  if (st->split_tokens > 0)
+    return static_cast<int>((st->cfg.capacity_tokens + st->split_tokens - 1) / st->split_tokens);
+  return auto_splits(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count);
 }
 
 }  // namespace
@@ -447,7 +518,7 @@ int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const 
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_qrot) || !aligned16(d_seq_lens)) return BGTQ_ERR_ALIGNMENT;
-  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, batch,
+  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, true, d_seq_lens, batch,
                                    split_for(st, layer_count, batch), as_stream(stream)) == cudaSuccess
              ? BGTQ_OK
              : BGTQ_ERR_CUDA;
@@ -477,7 +548,7 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, st->ws.qrot, d_seq_lens, batch,
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, st->ws.qrot, false, d_seq_lens, batch,
                                 split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split,
@@ -523,11 +594,12 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
   const int split = split_for(st, layer_count, batch);
-  const int64_t nspl = (st->cfg.capacity_tokens + split - 1) / split;
+  const int64_t nspl = split;
   const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
   const size_t qrot_bytes = rows * kD * sizeof(float);
+  const size_t fbytes = frag_bytes(&st->cfg, layer_count);
   const size_t part_bytes = rows * size_t(nspl) * bgtq::kPartialStride * sizeof(float);
-  if (qrot_bytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES) return BGTQ_ERR_BUFFER_SIZE;
+  if (qrot_bytes + fbytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES) return BGTQ_ERR_BUFFER_SIZE;
   void* base = nullptr;
   const int a = static_scratch_address(&base);
   if (a != BGTQ_OK) return a;
@@ -535,14 +607,15 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   // to the static array (partials packed with n_splits as their stride)
   bgtq::Workspace ws = st->ws;
   ws.qrot = static_cast<float*>(base);
-  ws.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + qrot_bytes);
+  ws.qfrag = reinterpret_cast<uint4*>(static_cast<unsigned char*>(base) + qrot_bytes);
+  ws.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + qrot_bytes + fbytes);
   bgtq::Shape shape = st->shape;
   shape.max_splits = static_cast<int32_t>(nspl);
   cudaStream_t s = as_stream(stream);
   if (bgtq::launch_rotate_query(shape, ws, layer, layer_count, static_cast<const __half*>(d_q), batch, ws.qrot, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, ws.qrot, d_seq_lens, batch, split, s) !=
+  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, ws.qrot, false, d_seq_lens, batch, split, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, static_cast<__half*>(d_out), s) !=

@@ -32,6 +32,23 @@ struct alignas(16) LayoutDev {
 };
 static_assert(sizeof(LayoutDev) == 640, "layout record size");
 
+// Per-(layer, KV head) tables of the split decode kernel, built on the host
+// from the layout and the codebook (800 bytes, copied to shared memory by
+// every CTA).
+struct alignas(16) DecodeTableDev {
+  int32_t grp[kNumGroupsMax][8];      // width, full chunks, size % 16, first tile word, first chunk, size, start, 0
+  uint32_t tabk[kNumGroupsMax][8];    // byte tables of the group's codebook: low bytes [4], high bytes [4]
+  uint32_t pdesc[kNumGroupsMax][32];  // partial-chunk descriptor of each lane (see group_logits)
+  uint32_t tabv[8];                   // byte table of the V codebook
+};
+static_assert(sizeof(DecodeTableDev) == 800, "decode table size");
+
+// q~ of one (layer, sequence, KV head, block of 8 query heads) as mma.sync
+// B fragments: entry 32 c + 4 h + t holds, for chunk c and head h of the
+// block, coordinates 16 j + 4 t .. + 3 of the chunk's group scaled by
+// log2(e), split into fp16 hi and lo: (hi01, hi23, lo01, lo23).
+constexpr int kFragEntries = kMaxChunks * 32;
+
 // fp32 Lloyd-Max codebooks indexed by width (row 0 unused).
 struct CodebookDev {
   float centroid[5][16];
@@ -48,7 +65,9 @@ struct Workspace {
   float* mv;                     // [L][Hkv][128 out][128 in]: V rotation (for the inverse rotation)
   unsigned __int128* energy_q;   // [kEnergyChunks][L][Hkv][64]
   unsigned __int128* energy_k;   // [kEnergyChunks][L][Hkv][64]
+  DecodeTableDev* dectab;        // [L][Hkv]
   float* qrot;                   // [L][B][Hq][128]
+  uint4* qfrag;                  // [L][B][Hkv][head blocks][kFragEntries]
   float* partials;               // [L][B][Hq][max_splits][kPartialStride]
 };
 
@@ -82,11 +101,15 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           const int32_t* count, int batch, int n, cudaStream_t stream);
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
+// The split pass reads q~ from ws.qfrag; frag_from_qrot first rebuilds those
+// fragments from qrot (callers that rotated the query themselves).
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
-                                int split_tokens, cudaStream_t stream);
+                                int layer_count, const float* qrot, bool frag_from_qrot, const int32_t* seq_lens,
+                                int batch, int n_splits, cudaStream_t stream);
+// Resident split-decode CTAs per SM for a config (0 on error).
+int decode_ctas_per_sm(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int split_tokens, __half* out,
+                           const int32_t* seq_lens, int batch, int n_splits, __half* out,
                            cudaStream_t stream);
 
 }  // namespace bgtq

@@ -601,6 +601,48 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
 // ---------------------------------------------------------------------------
 constexpr int kRotThreads = 256;
 
+__device__ __forceinline__ uint4* frag_block(const Shape& sh, const Workspace& ws, int li, int b, int kvh, int hb) {
+  const int hbs = (sh.group + 7) >> 3;
+  return ws.qfrag + ((((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_kv_heads + kvh) * hbs) + hb) * kFragEntries;
+}
+
+// Writes the B-fragment entries of query head hg (index within its KV
+// group) from its q~ in record order (qs, shared memory): for chunk c of
+// group g and quad t, coordinates 16 j + 4 t + m (j = c - first chunk of g)
+// times log2(e), zero past the group's size, split into fp16 hi + lo.  The
+// last head of a block also zeroes the unused head slots of the block.
+__device__ void write_frags(const LayoutDev& lay, const float* qs, int hg, int G, uint4* fb, int tid, int nthreads) {
+  const int hh = hg & 7;
+  const int nh = min(8, G - (hg & ~7));
+  const int ng = lay.n_groups;
+  const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+  for (int u = tid; u < nchunk * 4; u += nthreads) {
+    const int c = u >> 2, t = u & 3;
+    int g = 0;
+    while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
+    const int j = c - lay.chunk_base[g];
+    const int d = lay.size[g], st = lay.start[g];
+    float v[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int coord = 16 * j + 4 * t + m;
+      v[m] = coord < d ? qs[st + coord] * kLog2e : 0.f;
+    }
+    const __half2 a = __floats2half2_rn(v[0], v[1]);
+    const __half2 c2 = __floats2half2_rn(v[2], v[3]);
+    const float2 af = __half22float2(a), cf = __half22float2(c2);
+    const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
+    const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
+    fb[c * 32 + 4 * hh + t] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&c2),
+                                         *reinterpret_cast<const uint32_t*>(&al), *reinterpret_cast<const uint32_t*>(&cl));
+  }
+  if (hh == nh - 1)
+    for (int u = tid; u < nchunk * 4 * (8 - nh); u += nthreads) {
+      const int c = u % nchunk, rest = u / nchunk;
+      fb[c * 32 + 4 * (nh + (rest >> 2)) + (rest & 3)] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
                                                                    const __half* __restrict__ q, int batch,
                                                                    float* __restrict__ qrot) {
@@ -637,7 +679,27 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
       out = (sacc + part[i]) * lay.inv_sqrt_d[g] * kInvSqrtD;
     }
     qrot[row * kD + i] = out;
+    qp[i] = out;
   }
+  __syncthreads();
+  write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), tid, kRotThreads);
+}
+
+// The B fragments of q~ from a rotated query given by the caller (the
+// split stage called on its own).  Grid (layer_count * batch * Hq), 128 threads.
+__global__ void __launch_bounds__(kD) fragment_kernel(Shape sh, Workspace ws, int layer0,
+                                                      const float* __restrict__ qrot, int batch) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int hq = blockIdx.x % sh.n_q_heads;
+  const int b = (blockIdx.x / sh.n_q_heads) % batch;
+  const int li = blockIdx.x / (sh.n_q_heads * batch);
+  const int kvh = hq / sh.group;
+  const LayoutDev& lay = ws.layouts[(layer0 + li) * sh.n_kv_heads + kvh];
+  __shared__ float qp[kD];
+  qp[threadIdx.x] = qrot[((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq) * kD + threadIdx.x];
+  __syncthreads();
+  write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), threadIdx.x,
+              kD);
 }
 
 // ---------------------------------------------------------------------------
@@ -663,6 +725,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kStages = 2;
+constexpr int kDecMinBlocks = 3;  // CTAs per SM the register budget is sized for
 constexpr int kWaitLimit = 1 << 22;
 constexpr float kRescaleSlack = 8.f;
 
@@ -703,7 +766,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 struct DecodeLayout {  // byte offsets inside the dynamic shared memory
-  int bars, bq, tabk, geo, ms, ls, stage, stage_bytes, total;
+  int bars, bq, tabk, grp, pdesc, ms, ls, stage, stage_bytes, total;
 };
 
 __host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
@@ -712,9 +775,10 @@ __host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
   DecodeLayout L;
   L.bars = 0;
   L.bq = align128(kDecWarps * kStages * 8);
-  L.tabk = L.bq + kMaxChunks * 32 * 16;
-  L.geo = L.tabk + kNumGroupsMax * 8 * 4;
-  L.ms = L.geo + kNumGroupsMax * 8 * 4;
+  L.grp = L.bq + kMaxChunks * 32 * 16;    // a copy of DecodeTableDev: grp, tabk, pdesc, tabv
+  L.tabk = L.grp + kNumGroupsMax * 8 * 4;
+  L.pdesc = L.tabk + kNumGroupsMax * 8 * 4;
+  L.ms = L.grp + static_cast<int>(sizeof(DecodeTableDev));
   L.ls = L.ms + kDecWarps * 8 * 4;
   L.stage = align128(L.ls + kDecWarps * 8 * 4);
   L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
@@ -724,38 +788,10 @@ __host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
   return L;
 }
 
-// The lane's four selectors (M-tiles 0..3) of chunk j of a width-B group:
-// a quartet for full chunks; for the partial chunk, a quartet of the lanes
-// with a full quad, half selectors of a virtual lane for the half quad, 0
-// for lanes with no coordinates (their B rows are 0).
-template <int B>
-__device__ __forceinline__ void chunk_selectors(const uint32_t* gw, int j, int nfull, int r, int lane, uint32_t* s) {
-  uint32_t w[B];
-  if (j < nfull) {
-#pragma unroll
-    for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
-    quartet_decode<B>(w, s);
-    return;
-  }
-  const uint32_t* pc = gw + nfull * 32 * B;
-  const int nf = r >> 2, g = lane >> 2, tl = lane & 3;
-  s[0] = s[1] = s[2] = s[3] = 0u;
-  if (tl < nf) {
-#pragma unroll
-    for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * k + g * nf + tl];
-    quartet_decode<B>(w, s);
-  } else if ((r & 3) && tl == nf) {
-    uint32_t sv[4];
-#pragma unroll
-    for (int k = 0; k < B; ++k) w[k] = pc[8 * nf * B + 4 * k + (g >> 1)];
-    quartet_decode<B>(w, sv);
-    const int sh = 16 * (g & 1);
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      const uint32_t x = (sv[mu] >> sh) & 0xFFFFu;
-      s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
-    }
-  }
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // S[mu] += A(selector s[mu]) * (q~ hi + q~ lo) for the four M-tiles of a chunk.
@@ -773,48 +809,67 @@ __device__ __forceinline__ void chunk_mma(const ByteTab& t, const uint32_t* s, u
   for (int mu = 0; mu < 4; ++mu) mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.z, bf.w);
 }
 
-// Logits of one width group for the warp's tile: S[mu][4] (M-tile mu).
-__device__ __forceinline__ void group_logits(const uint32_t* kt, const GroupGeo& q, const uint4* bq,
-                                             const uint32_t* tab8, int lane, float (*S)[4]) {
-  ByteTab t;
-  const uint4 tl = *reinterpret_cast<const uint4*>(tab8);
-  const uint4 th = *reinterpret_cast<const uint4*>(tab8 + 4);
-  t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
-  t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
-  const uint32_t* gw = kt + q.word;
-  const int nchunks = q.nfull + (q.r ? 1 : 0);
-  for (int j = 0; j < nchunks; ++j) {
-    uint32_t s[4];
-    switch (q.width) {
-      case 1: chunk_selectors<1>(gw, j, q.nfull, q.r, lane, s); break;
-      case 2: chunk_selectors<2>(gw, j, q.nfull, q.r, lane, s); break;
-      case 3: chunk_selectors<3>(gw, j, q.nfull, q.r, lane, s); break;
-      default: chunk_selectors<4>(gw, j, q.nfull, q.r, lane, s); break;
+// Logits of one width-B group for the warp's tile, S[mu][4] (M-tile mu):
+// the group's full 16-coordinate chunks as quartets, then its partial chunk
+// (if any) through the lane's descriptor pd: word offset (bits 0..11) and
+// stride per plane word (bits 12..19) inside the partial region, bit 20 set
+// for a half-quad lane, bit 21 for the upper half of its virtual lane.  Lanes
+// with no coordinates read any word of the region: their B rows are zero.
+template <int B>
+__device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool partial, uint32_t pd,
+                                             const uint4* bqg, const ByteTab& t, int lane, float (*S)[4]) {
+#pragma unroll 1
+  for (int j = 0; j < nfull; ++j) {
+    uint32_t w[B], s[4];
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
+    quartet_decode<B>(w, s);
+    chunk_mma<B == 4>(t, s, bqg[j * 32], S);
+  }
+  if (partial) {
+    const uint32_t* pc = gw + nfull * 32 * B;
+    const int base = pd & 0xFFF, stride = (pd >> 12) & 0xFF;
+    uint32_t w[B], s[4];
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = pc[base + stride * k];
+    quartet_decode<B>(w, s);
+    if (pd & (1u << 20)) {
+      const int sh = (pd >> 21) & 1 ? 16 : 0;
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        const uint32_t x = (s[mu] >> sh) & 0xFFFFu;
+        s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
+      }
     }
-    const uint4 bf = bq[(q.chunk + j) * 32 + lane];
-    if (q.width == 4) chunk_mma<true>(t, s, bf, S);
-    else chunk_mma<false>(t, s, bf, S);
+    chunk_mma<B == 4>(t, s, bqg[nfull * 32], S);
   }
 }
 
+// Grid (ctas_per_unit, batch * Hkv * head_blocks, layer_count), 128 threads.
+// A unit is one (layer, sequence, KV head, block of up to 8 query heads);
+// its tiles are dealt round-robin over the 4 * ctas_per_unit warps of its
+// CTAs (warp w of CTA c takes tiles 4c + w, 4c + w + W, ..., W = 4 *
+// ctas_per_unit), so every warp gets the same number of tiles to within one.
+// Each CTA writes one partial (m, l, acc) per query head -- an empty one
+// (m = -inf, l = 0) when it has no tile.
 template <int VB>
-__global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
-                                                                 const float* __restrict__ qrot,
-                                                                 const int32_t* __restrict__ seq_lens, int batch,
-                                                                 int split_tokens, int head_blocks) {
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+    decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const int32_t* __restrict__ seq_lens,
+                      int batch, int ctas_per_unit, int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const DecodeLayout DL = decode_layout(sh.kbits, VB);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
   uint4* bq = reinterpret_cast<uint4*>(smem_raw + DL.bq);
   uint32_t* tabk = reinterpret_cast<uint32_t*>(smem_raw + DL.tabk);
-  int32_t* geo = reinterpret_cast<int32_t*>(smem_raw + DL.geo);
+  int32_t* grp = reinterpret_cast<int32_t*>(smem_raw + DL.grp);
+  uint32_t* pdesc = reinterpret_cast<uint32_t*>(smem_raw + DL.pdesc);
   float* ms = reinterpret_cast<float*>(smem_raw + DL.ms);
   float* ls = reinterpret_cast<float*>(smem_raw + DL.ls);
   unsigned char* stage_base = smem_raw + DL.stage;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, t4 = lane & 3;
-  const int s = blockIdx.x;
+  const int cu = blockIdx.x;
   const int hb = blockIdx.y % head_blocks;
   const int h = (blockIdx.y / head_blocks) % sh.n_kv_heads;
   const int b = blockIdx.y / (head_blocks * sh.n_kv_heads);
@@ -826,36 +881,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
   const int lh = layer * sh.n_kv_heads + h;
   const LayoutDev& lay = ws.layouts[lh];
 
-  // ---- per-CTA set-up: q~ B fragments, byte tables, group geometry ----
+  // ---- per-CTA set-up: the (layer, KV head) decode table (a library table) ----
   const int ng = lay.n_groups;
-  if (tid < kNumGroupsMax) {
-    int word = 0, chunk = 0;
-    for (int g = 0; g < tid && g < ng; ++g) {
-      word += 2 * lay.size[g] * lay.width[g];
-      chunk += (lay.size[g] + 15) >> 4;
-    }
-    geo[tid * 8 + 0] = tid < ng ? lay.width[tid] : 0;
-    geo[tid * 8 + 1] = tid < ng ? lay.size[tid] : 0;
-    geo[tid * 8 + 2] = tid < ng ? lay.start[tid] : 0;
-    geo[tid * 8 + 3] = word;
-    geo[tid * 8 + 4] = chunk;
-  }
-  if (tid < kNumGroupsMax * 8) {
-    const int g = tid >> 3, wd = tid & 7;
-    uint32_t v = 0;
-    if (g < ng) {
-      const int bits = lay.width[g];
-      const float* cen = ws.codebook->centroid[bits];
-      const int n = 1 << bits;
-      for (int c = 0; c < 4; ++c) {
-        const int e = 4 * (wd & 3) + c;
-        if (e < n) {
-          const uint32_t hb16 = __half_as_ushort(__float2half_rn(cen[e]));
-          v |= (wd < 4 ? (hb16 & 0xFFu) : (hb16 >> 8)) << (8 * c);
-        }
-      }
-    }
-    tabk[tid] = v;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(ws.dectab + lh);
+    uint4* dst = reinterpret_cast<uint4*>(grp);  // grp, tabk, pdesc, tabv are contiguous
+    for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += kDecThreads) dst[u] = src[u];
   }
   if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
   __syncthreads();
@@ -867,48 +898,43 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = seq_lens[b];
   if (len < 0 || len > sh.capacity) len = 0;  // flagged by the combine kernel
-  const int t0 = s * split_tokens;
-  if (t0 >= len) return;
-  const int t1 = min(t0 + split_tokens, len);
-  {
-    const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
-    int nchunk = 0;
-    for (int g = 0; g < ng; ++g) nchunk += (lay.size[g] + 15) >> 4;
-    for (int u = tid; u < nchunk * 32; u += kDecThreads) {
-      const int c = u >> 5, ln = u & 31;
-      int g = 0;
-      while (g + 1 < ng && c >= geo[(g + 1) * 8 + 4]) ++g;
-      const int j = c - geo[g * 8 + 4];
-      const int d = geo[g * 8 + 1], st = geo[g * 8 + 2];
-      const int head = ln >> 2;
-      float v[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int coord = 16 * j + 4 * (ln & 3) + m;
-        v[m] = (head < nh && coord < d) ? qsrc[head * kD + st + coord] * kLog2e : 0.f;
+  const int ntl = (len + kTile - 1) / kTile;
+  const int W = ctas_per_unit * kDecWarps;
+  const int wu = cu * kDecWarps + warp;
+  const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
+  float* part_base = ws.partials +
+                     (((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0) * sh.max_splits + cu) *
+                         kPartialStride;
+  const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
+  if (cu * kDecWarps >= ntl) {
+    // no tile for this CTA: an empty partial per head
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int hh = 0; hh < nh; ++hh) {
+      float* part = part_base + hh * part_head_stride;
+      part[4 + tid] = 0.f;
+      if (tid == 0) {
+        part[0] = -CUDART_INF_F;
+        part[1] = 0.f;
       }
-      uint32_t hi01, hi23, lo01, lo23;
-      {
-        const __half2 a = __floats2half2_rn(v[0], v[1]);
-        const __half2 c2 = __floats2half2_rn(v[2], v[3]);
-        const float2 af = __half22float2(a), cf = __half22float2(c2);
-        const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
-        const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
-        hi01 = *reinterpret_cast<const uint32_t*>(&a);
-        hi23 = *reinterpret_cast<const uint32_t*>(&c2);
-        lo01 = *reinterpret_cast<const uint32_t*>(&al);
-        lo23 = *reinterpret_cast<const uint32_t*>(&cl);
-      }
-      bq[u] = make_uint4(hi01, hi23, lo01, lo23);
     }
+    return;
+  }
+  {
+    // q~ fragments of this unit, written by the query rotation
+    const uint4* src = frag_block(sh, ws, li, b, h, hb);
+    const int n = 32 * (lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4));
+    for (int u = tid; u < n; u += kDecThreads) bq[u] = src[u];
   }
   ByteTab tv;
-  fill_bytetab(tv, ws.codebook->centroid[VB], VB);
+  {
+    const uint4 a0 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32);
+    const uint4 a1 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32 + 4);
+    tv.lo[0] = a0.x; tv.lo[1] = a0.y; tv.lo[2] = a0.z; tv.lo[3] = a0.w;
+    tv.hi[0] = a1.x; tv.hi[1] = a1.y; tv.hi[2] = a1.z; tv.hi[3] = a1.w;
+  }
   __syncthreads();
 
   // ---- per-warp pipeline over this warp's tiles ----
-  const int tiles_cta = (t1 - t0 + kTile - 1) / kTile;
-  const int my_tiles = tiles_cta > warp ? (tiles_cta - warp + kDecWarps - 1) / kDecWarps : 0;
   const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
   const int kwords = 256 * sh.kbits, vwords = 256 * VB;
   const uint32_t kbytes = 4u * kwords, vbytes = 4u * vwords;
@@ -917,7 +943,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
   uint64_t* my_bars = bars + warp * kStages;
 
   auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
-    const int tile = t0 / kTile + warp + k * kDecWarps;
+    const int tile = wu + k * W;
     unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
     uint64_t* bar = &my_bars[k % kStages];
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -950,30 +976,36 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
     const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
     const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
     const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
-    const int tile_pos = t0 + (warp + k * kDecWarps) * kTile;
-    const int nvalid = min(kTile, t1 - tile_pos);
+    const int nvalid = min(kTile, len - (wu + k * W) * kTile);
 
-    // logits
+    // logits, one width group at a time, each scaled by its per-token norm
     float L[4][4];
 #pragma unroll
     for (int mu = 0; mu < 4; ++mu)
 #pragma unroll
       for (int r = 0; r < 4; ++r) L[mu][r] = 0.f;
     for (int g = 0; g < ng; ++g) {
-      GroupGeo q;
-      q.width = geo[g * 8 + 0];
-      q.d = geo[g * 8 + 1];
-      q.start = geo[g * 8 + 2];
-      q.word = geo[g * 8 + 3];
-      q.chunk = geo[g * 8 + 4];
-      q.nfull = q.d >> 4;
-      q.r = q.d & 15;
+      const int4 gp = *reinterpret_cast<const int4*>(grp + g * 8);  // width, nfull, r, word
+      const int chunk = grp[g * 8 + 4];
+      ByteTab t;
+      const uint4 tl = *reinterpret_cast<const uint4*>(tabk + 8 * g);
+      const uint4 th = *reinterpret_cast<const uint4*>(tabk + 8 * g + 4);
+      t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
+      t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+      const uint32_t pd = pdesc[g * 32 + lane];
+      const uint32_t* gw = kt + gp.w;
+      const uint4* bqg = bq + chunk * 32 + lane;
       float S[4][4];
 #pragma unroll
       for (int mu = 0; mu < 4; ++mu)
 #pragma unroll
         for (int r = 0; r < 4; ++r) S[mu][r] = 0.f;
-      group_logits(kt, q, bq, tabk + 8 * g, lane, S);
+      switch (gp.x) {
+        case 1: group_logits<1>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 2: group_logits<2>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 3: group_logits<3>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        default: group_logits<4>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+      }
 #pragma unroll
       for (int mu = 0; mu < 4; ++mu) {
         const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
@@ -984,13 +1016,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
         L[mu][3] = fmaf(nb, S[mu][3], L[mu][3]);
       }
     }
-    // online softmax over the tile for heads 2*t4 and 2*t4+1
+    // online softmax over the tile for heads 2*t4 and 2*t4+1; positions past
+    // the valid length carry no weight (their norms may be anything)
+    float wv[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      wv[mu][0] = __half2float(vn[16 * mu + g8]) * kInvSqrtD;
+      wv[mu][1] = __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD;
+    }
+    if (nvalid < kTile) {
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        if (16 * mu + g8 >= nvalid) {
+          L[mu][0] = L[mu][1] = -CUDART_INF_F;
+          wv[mu][0] = 0.f;
+        }
+        if (16 * mu + g8 + 8 >= nvalid) {
+          L[mu][2] = L[mu][3] = -CUDART_INF_F;
+          wv[mu][1] = 0.f;
+        }
+      }
+    }
     float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
     for (int mu = 0; mu < 4; ++mu) {
-      const bool va = 16 * mu + g8 < nvalid, vbv = 16 * mu + g8 + 8 < nvalid;
-      if (!va) L[mu][0] = L[mu][1] = -CUDART_INF_F;
-      if (!vbv) L[mu][2] = L[mu][3] = -CUDART_INF_F;
       mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
       mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
     }
@@ -1007,7 +1056,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       if (mx[c] > m_run[c] + kRescaleSlack) {
-        alpha[c] = exp2f(m_run[c] - mx[c]);
+        alpha[c] = fast_exp2(m_run[c] - mx[c]);
         m_run[c] = mx[c];
         moved = true;
       }
@@ -1015,15 +1064,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
     uint32_t bp[4][2];
 #pragma unroll
     for (int mu = 0; mu < 4; ++mu) {
-      // positions past the valid length carry no weight (their norms may be anything)
-      const float wa = 16 * mu + g8 < nvalid ? __half2float(vn[16 * mu + g8]) * kInvSqrtD : 0.f;
-      const float wb = 16 * mu + g8 + 8 < nvalid ? __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD : 0.f;
-      const float p0 = exp2f(L[mu][0] - m_run[0]), p1 = exp2f(L[mu][1] - m_run[1]);
-      const float p2 = exp2f(L[mu][2] - m_run[0]), p3 = exp2f(L[mu][3] - m_run[1]);
+      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
+      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
       sum[0] += p0 + p2;
       sum[1] += p1 + p3;
-      bp[mu][0] = transpose8x8(pack_half2(p0 * wa, p1 * wa));
-      bp[mu][1] = transpose8x8(pack_half2(p2 * wb, p3 * wb));
+      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
+      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -1091,13 +1137,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_mma_kernel(Shape sh, Works
     float lsum = 0.f, a = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
-      const float sc = exp2f(ms[w * 8 + hh] - M);
+      // warps without a tile hold m = -inf, l = 0, acc = 0
+      const float mw = ms[w * 8 + hh];
+      const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
       lsum = fmaf(sc, ls[w * 8 + hh], lsum);
       a = fmaf(sc, accs[(w * 8 + hh) * kD + i], a);
     }
-    float* part = ws.partials +
-                  ((((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0 + hh) * sh.max_splits) + s) *
-                      kPartialStride;
+    float* part = part_base + hh * part_head_stride;
     part[4 + i] = a;
     if (i == 0) {
       part[0] = M;
@@ -1116,7 +1162,7 @@ constexpr int kCombWarps = kCombThreads / 32;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
-                                                               int split_tokens, __half* __restrict__ out) {
+                                                               int n_splits, __half* __restrict__ out) {
   const int hq = blockIdx.x % sh.n_q_heads;
   const int b = (blockIdx.x / sh.n_q_heads) % batch;
   const int li = blockIdx.x / (sh.n_q_heads * batch);
@@ -1139,7 +1185,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
     len = 0;
   }
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  const int nspl = (len + split_tokens - 1) / split_tokens;
+  const int nspl = len > 0 ? n_splits : 0;
   if (nspl == 0) {
     if (tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
@@ -1229,19 +1275,37 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
-                             const float* qrot, const int32_t* seq_lens, int batch, int split_tokens,
-                             cudaStream_t stream) {
+                             const int32_t* seq_lens, int batch, int n_splits, cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
   static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
-  const int nspl = static_cast<int>((s.capacity + split_tokens - 1) / split_tokens);
-  dim3 grid(nspl, batch * s.n_kv_heads * head_blocks, layer_count);
+  dim3 grid(n_splits, batch * s.n_kv_heads * head_blocks, layer_count);
   return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, qrot, seq_lens, batch, split_tokens, head_blocks);
+                          ws, cache, layer0, seq_lens, batch, n_splits, head_blocks);
+}
+
+template <int VB>
+int ctas_per_sm_vb(const Shape& s) {
+  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
+  if (attr != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<VB>, kDecThreads,
+                                                    decode_layout(s.kbits, VB).total) != cudaSuccess)
+    return 0;
+  return n;
 }
 
 }  // namespace
+
+int decode_ctas_per_sm(const Shape& s) {
+  switch (s.vbits) {
+    case 1: return ctas_per_sm_vb<1>(s);
+    case 2: return ctas_per_sm_vb<2>(s);
+    case 3: return ctas_per_sm_vb<3>(s);
+    default: return ctas_per_sm_vb<4>(s);
+  }
+}
 
 cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,
                           const __half* calib_k, int nk, int pairing, cudaStream_t stream) {
@@ -1269,21 +1333,26 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 }
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
-                                int split_tokens, cudaStream_t stream) {
+                                int layer_count, const float* qrot, bool frag_from_qrot, const int32_t* seq_lens,
+                                int batch, int n_splits, cudaStream_t stream) {
+  if (frag_from_qrot) {
+    fragment_kernel<<<layer_count * batch * s.n_q_heads, kD, 0, stream>>>(s, ws, layer0, qrot, batch);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   switch (s.vbits) {
-    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
-    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, split_tokens, stream);
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
   }
 }
 
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int split_tokens, __half* out,
+                           const int32_t* seq_lens, int batch, int n_splits, __half* out,
                            cudaStream_t stream) {
   return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kCombThreads), 0, stream, s,
-                          ws, layer0, seq_lens, batch, split_tokens, out);
+                          ws, layer0, seq_lens, batch, n_splits, out);
 }
 
 }  // namespace bgtq

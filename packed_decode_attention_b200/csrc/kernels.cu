@@ -371,7 +371,6 @@ struct EncodeSmem {
   float mt[kD][kD];              // mt[j][i] = R[i][j] (record order)
   float fac[kTile][kNumGroupsMax];
   __half nrm[kTile][kNumGroupsMax];
-  float fac2[kD];                // partial rotation sums of the append path
   uint8_t codes[kTile][kD];
   uint32_t words[1024];
   float thr[5][16];
@@ -434,9 +433,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   }
   for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
   const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
-  const int nrows = tr1 - tr0;
-  if (nrows > 16)  // the register-tile path reads the rotation from shared memory
-    for (int i = tid; i < kD * kD / 4; i += kEncThreads)
+  for (int i = tid; i < kD * kD / 4; i += kEncThreads)
       reinterpret_cast<float4*>(&S.mt[0][0])[i] = reinterpret_cast<const float4*>(mglob)[i];
   __syncthreads();
   const int ng = S.lay.n_groups;
@@ -496,34 +493,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     S.nrm[r][g] = nh;
   }
   __syncthreads();
-  // y = R x per new row, then the codes
-  if (nrows <= 16) {
-    // few rows (decode-time appends): two threads per output, each holding
-    // half of the rotation's column in registers (read from global memory
-    // with all loads in flight at once; zero outside the output's group);
-    // the two partial sums meet in shared memory
-    const int i = tid & (kD - 1), half = tid >> 7;
-    float m[64];
-#pragma unroll
-    for (int u = 0; u < 64; ++u) m[u] = __ldg(mglob + (half * 64 + u) * kD + i);
-    const int g = S.gof[i];
-    for (int r = tr0; r < tr1; ++r) {
-      float y = 0.f;
-#pragma unroll
-      for (int u = 0; u < 64; ++u) y = fmaf(m[u], S.xt[half * 64 + u][r], y);
-      if (half == 1) S.fac2[i] = y;
-      __syncthreads();
-      if (half == 0 && g >= 0) {
-        const int w = S.lay.width[g];
-        const float u = (y + S.fac2[i]) * S.fac[r][g];
-        int code = 0;
-        const int nt = (1 << w) - 1;
-        for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
-        S.codes[r][i] = static_cast<uint8_t>(code);
-      }
-      __syncthreads();
-    }
-  } else {
+  // y = R x per new row (fp32, coordinate order), then the codes
+  {
     // register tile: 4 rows x 8 outputs per thread over all 64 rows
     const int rg = tid >> 4, og = tid & 15;
     const int i0 = og * 8;
@@ -592,6 +563,188 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
       dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
     } else {
       cache.vnorm[pos] = S.nrm[tid][0];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3 for a few rows (decode-time appends): grid (layer_count * batch * Hkv,
+// n, 2 kinds), 128 threads.  A CTA encodes one new row of one (layer,
+// sequence, KV head) and kind with the same arithmetic as encode_kernel
+// (norms summed in fp64 in coordinate order, y = sum_j R[i][j] x_j in fp32
+// in coordinate order from the group's first coordinate, u = y * sqrt(d) /
+// ||x||, code = #{thresholds <= u}) and rewrites only that row's code bits
+// in the packed tile, with global atomics: bits of other positions are never
+// touched, so rows appended by different CTAs to the same tile do not race.
+// ---------------------------------------------------------------------------
+constexpr int kAppThreads = 128;
+constexpr int kAppendMaxRows = 16;  // calls with at most this many rows per sequence use append_kernel
+
+// Plane word (0..b-1) and bit of code bit q of selector sel, nibble n, in a
+// quartet of width b (see the quartet formulas above).
+__device__ __forceinline__ void quartet_bit(int b, int sel, int n, int q, int& k, int& bit) {
+  if (b == 4) {
+    k = sel;
+    bit = 4 * n + q;
+  } else if (b == 1) {
+    k = 0;
+    bit = 4 * n + sel;
+  } else if (q < 2) {
+    k = sel >> 1;
+    bit = 4 * n + 2 * (sel & 1) + q;
+  } else {
+    k = 2;
+    bit = 4 * n + sel;
+  }
+}
+
+// Word (relative to the tile) of plane k for a K code, and the selector
+// and nibble it sits in: token p (0..63), coordinate c of group g.
+__device__ __forceinline__ int k_code_word(const LayoutDev& lay, int g, int c, int p, int k, int& sel, int& n) {
+  const int b = lay.width[g], d = lay.size[g];
+  const int nfull = d >> 4, r = d & 15, nf = r >> 2;
+  const int j = c >> 4, cc = c & 15, t = cc >> 2, m4 = cc & 3;
+  const int pr = p & 15, gg = pr & 7;
+  sel = p >> 4;
+  n = m4 + 4 * (pr >> 3);
+  const int base = lay.tile_word[g];
+  if (j < nfull) return base + j * 32 * b + 32 * k + 4 * gg + t;
+  const int pc = base + nfull * 32 * b;
+  if (t < nf) return pc + 8 * nf * k + gg * nf + t;
+  // half quad of the partial chunk: virtual lane gg / 2, upper half for odd gg
+  n = (n & 1) + 2 * (n >> 2) + 4 * (gg & 1);
+  return pc + 8 * nf * b + 4 * k + (gg >> 1);
+}
+
+// Same for a V code: token p, dimension i.
+__device__ __forceinline__ int v_code_word(int vb, int i, int p, int k, int& sel, int& n) {
+  const int m = i >> 4, cm = i & 15, gg = cm & 7;
+  const int pt = p & 15, t = (pt & 7) >> 1, member = (pt & 1) + 2 * (pt >> 3);
+  sel = p >> 4;
+  n = member + 4 * (cm >> 3);
+  return m * 32 * vb + 32 * k + 4 * gg + t;
+}
+
+__global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                             const __half* __restrict__ kx,
+                                                             const __half* __restrict__ vx,
+                                                             const int32_t* __restrict__ start_v,
+                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+  const int tid = threadIdx.x;
+  const int kind = blockIdx.z;
+  const int h = blockIdx.x % sh.n_kv_heads;
+  const int b = (blockIdx.x / sh.n_kv_heads) % batch;
+  const int li = blockIdx.x / (sh.n_kv_heads * batch);
+  const int layer = layer0 + li;
+  const int row = blockIdx.y;
+  const int start = start_v[b];
+  const int count = count_v[b];
+  if (start < 0 || count < 0 || count > n) {
+    if (tid == 0 && row == 0 && kind == 0) atomicOr(ws.err, kErrArg);
+    return;
+  }
+  if (row >= count) return;
+  const int64_t pos = static_cast<int64_t>(start) + row;
+  if (pos >= sh.capacity) {
+    if (tid == 0) atomicOr(ws.err, kErrCapacity);
+    return;
+  }
+  const int lh = layer * sh.n_kv_heads + h;
+  __shared__ LayoutDev lay;
+  __shared__ float xs[kD];
+  __shared__ float fac[kNumGroupsMax];
+  __shared__ __half nrm[kNumGroupsMax];
+  if (kind == 0) {
+    if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
+      reinterpret_cast<int32_t*>(&lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
+    for (int u = tid + kAppThreads; u < static_cast<int>(sizeof(LayoutDev) / 4); u += kAppThreads)
+      reinterpret_cast<int32_t*>(&lay)[u] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[u];
+  } else if (tid == 0) {
+    lay.n_groups = 1;
+    lay.n_positions = kD;
+    for (int g = 0; g < kNumGroupsMax; ++g) {
+      lay.width[g] = g == 0 ? sh.vbits : 0;
+      lay.size[g] = g == 0 ? kD : 0;
+      lay.start[g] = g == 0 ? 0 : kD;
+      lay.tile_word[g] = 0;
+    }
+  }
+  __syncthreads();
+  const __half* x = (kind == 0 ? kx : vx) +
+                    ((static_cast<size_t>(li) * batch + b) * n + row) * sh.n_kv_heads * kD + static_cast<size_t>(h) * kD;
+  // record order: position i holds dim perm[i] (K); V keeps the dims
+  if (kind == 0) {
+    if (tid < lay.n_positions) xs[tid] = __half2float(x[lay.perm[tid]]);
+  } else {
+    xs[tid] = __half2float(x[tid]);
+  }
+  __syncthreads();
+  const int ng = lay.n_groups;
+  if (tid < ng) {
+    const int j0 = lay.start[tid], j1 = j0 + lay.size[tid];
+    double s2 = 0.0;
+    for (int j = j0; j < j1; ++j) {
+      const double v = xs[j];
+      s2 += v * v;
+    }
+    const double nr = sqrt(s2);
+    nrm[tid] = __double2half(nr);
+    fac[tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[tid])) / nr) : 0.f;
+  }
+  __syncthreads();
+  const int i = tid;
+  const int tile = static_cast<int>(pos / kTile), p = static_cast<int>(pos % kTile);
+  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
+  if (i < lay.n_positions) {
+    int g = 0;
+    for (int t = 1; t < ng; ++t)
+      if (i >= lay.start[t]) g = t;
+    const float* mt = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
+    const int j0 = lay.start[g], j1 = j0 + lay.size[g];
+    float y = 0.f;
+    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], __ldg(mt + static_cast<size_t>(j) * kD + i), y);
+    const int w = lay.width[g];
+    const float u = y * fac[g];
+    int code = 0;
+    const int nt = (1 << w) - 1;
+    for (int t = 0; t < nt; ++t) code += (ws.codebook->threshold[w][t] <= u) ? 1 : 0;
+    // rewrite this code's bits, one atomic pair per touched word
+    const int nwords = 256 * (kind == 0 ? sh.kbits : sh.vbits);
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + (seq_tiles + tile) * nwords;
+    int cur = -1;
+    uint32_t mask = 0, val = 0;
+    for (int q = 0; q < w; ++q) {
+      int k, bit, sel, nib;
+      if (kind == 0) k_code_word(lay, g, i - lay.start[g], p, 0, sel, nib);
+      else v_code_word(w, i, p, 0, sel, nib);
+      quartet_bit(w, sel, nib, q, k, bit);
+      const int wk = kind == 0 ? k_code_word(lay, g, i - lay.start[g], p, k, sel, nib) : v_code_word(w, i, p, k, sel, nib);
+      if (wk != cur) {
+        if (cur >= 0) {
+          atomicAnd(gtile + cur, ~mask);
+          atomicOr(gtile + cur, val);
+        }
+        cur = wk;
+        mask = 0;
+        val = 0;
+      }
+      mask |= 1u << bit;
+      val |= static_cast<uint32_t>((code >> q) & 1) << bit;
+    }
+    if (cur >= 0) {
+      atomicAnd(gtile + cur, ~mask);
+      atomicOr(gtile + cur, val);
+    }
+  }
+  if (tid == 0) {
+    const size_t tp = seq_tiles * kTile + static_cast<size_t>(pos);
+    if (kind == 0) {
+      __half2* dst = reinterpret_cast<__half2*>(cache.knorm + tp * 4);
+      const __half z = __float2half(0.f);
+      dst[0] = __halves2half2(nrm[0], ng > 1 ? nrm[1] : z);
+      dst[1] = __halves2half2(ng > 2 ? nrm[2] : z, ng > 3 ? nrm[3] : z);
+    } else {
+      cache.vnorm[tp] = nrm[0];
     }
   }
 }
@@ -1153,12 +1306,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq), 256
-// threads: the 8 warps share the splits (lane = 4 rotated coordinates),
-// then o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), w_s = 2^(m_s - M).
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq), 512
+// threads.  w_s = 2^(m_s - M) per split (0 for empty splits); the 16 warps
+// share the splits (lane = 4 rotated coordinates), then
+// o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), four threads per output.
 // ---------------------------------------------------------------------------
-constexpr int kCombThreads = 256;
+constexpr int kCombThreads = 512;
 constexpr int kCombWarps = kCombThreads / 32;
+constexpr int kCombMaxSplits = 1024;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
@@ -1169,13 +1324,13 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // the inverse V rotation's column for this thread (a library table),
-  // loaded while the previous kernel finishes
+  // a quarter of the inverse V rotation's column for this thread (a library
+  // table), loaded while the previous kernel finishes
   const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-  const int d = tid & (kD - 1), half = tid >> 7;
-  float mvr[64];
+  const int d = tid & (kD - 1), quarter = tid >> 7;
+  float mvr[32];
 #pragma unroll
-  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + d);
+  for (int r = 0; r < 32; ++r) mvr[r] = __ldg(mv + (quarter * 32 + r) * kD + d);
   // Launched as a programmatic dependent of the split pass: inputs, partials
   // and the output are touched only after that kernel has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1185,7 +1340,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
     len = 0;
   }
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  const int nspl = len > 0 ? n_splits : 0;
+  const int nspl = len > 0 ? min(n_splits, kCombMaxSplits) : 0;
   if (nspl == 0) {
     if (tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
@@ -1193,9 +1348,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const float* part =
       ws.partials + ((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq) * sh.max_splits * kPartialStride;
   __shared__ float red[kCombWarps];
+  __shared__ float sc[kCombMaxSplits];
   __shared__ float accs[kCombWarps][kD];
-  __shared__ float lsw[kCombWarps];
   __shared__ float a_s[kD];
+  // the largest split maximum
   float M = -CUDART_INF_F;
   for (int s = tid; s < nspl; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
 #pragma unroll
@@ -1205,39 +1361,48 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   M = red[0];
 #pragma unroll
   for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  // split weights and the softmax denominator
   float lsum = 0.f;
+  for (int s = tid; s < nspl; s += kCombThreads) {
+    const float ms = part[static_cast<size_t>(s) * kPartialStride];
+    const float w = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+    sc[s] = w;
+    lsum = fmaf(w, part[static_cast<size_t>(s) * kPartialStride + 1], lsum);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();
+  lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombWarps; ++w) lsum += red[w];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int s = warp; s < nspl; s += kCombWarps) {
-    const float* p = part + static_cast<size_t>(s) * kPartialStride;
-    const float wgt = exp2f(p[0] - M);
-    lsum = fmaf(wgt, p[1], lsum);
-    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+    const float wgt = sc[s];
+    const float4 a = *reinterpret_cast<const float4*>(part + static_cast<size_t>(s) * kPartialStride + 4 + 4 * lane);
     acc.x = fmaf(wgt, a.x, acc.x);
     acc.y = fmaf(wgt, a.y, acc.y);
     acc.z = fmaf(wgt, a.z, acc.z);
     acc.w = fmaf(wgt, a.w, acc.w);
   }
   *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
-  if (lane == 0) lsw[warp] = lsum;
   __syncthreads();
   if (tid < kD) {
-    float a = 0.f, l = 0.f;
+    float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) {
-      a += accs[w][tid];
-      l += lsw[w];
-    }
-    a_s[tid] = a / l;
+    for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
+    a_s[tid] = a / lsum;
   }
   __syncthreads();
-  // inverse V rotation: thread pair (d, half) sums half of the 128 inputs
+  // inverse V rotation: four threads per output, a quarter of the inputs each
   float o = 0.f;
 #pragma unroll
-  for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
-  if (half == 1) accs[0][d] = o;
+  for (int r = 0; r < 32; ++r) o = fmaf(mvr[r], a_s[quarter * 32 + r], o);
+  accs[quarter][d] = o;
   __syncthreads();
-  if (half == 0) out[row * kD + d] = __float2half(o + accs[0][d]);
+  if (tid < kD) out[row * kD + d] = __float2half((accs[0][d] + accs[1][d]) + (accs[2][d] + accs[3][d]));
 }
 
 // Raises a kernel's dynamic shared-memory limit; callers keep the result in
@@ -1321,6 +1486,12 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
   if (n <= 0) return cudaSuccess;
   const cudaError_t e = encode_smem_once();
   if (e != cudaSuccess) return e;
+  if (n <= kAppendMaxRows) {
+    // a few rows per sequence: rewrite only their code bits
+    append_kernel<<<dim3(layer_count * batch * s.n_kv_heads, n, 2), kAppThreads, 0, stream>>>(s, ws, cache, layer0, k, v,
+                                                                                             start, count, batch, n);
+    return cudaGetLastError();
+  }
   dim3 grid(layer_count * batch * s.n_kv_heads, (n + kTile - 1) / kTile + 1, 2);
   encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
   return cudaGetLastError();

@@ -387,3 +387,41 @@ def test_appends_in_pieces_equal_one_encode(dev):
     assert torch.equal(whole_k, kv.k_tiles()) and torch.equal(whole_v, kv.v_tiles())
     assert torch.equal(whole_kn, kv.k_norms()) and torch.equal(whole_vn, kv.v_norms())
     kv.close()
+
+
+def test_small_appends_equal_one_encode(dev):
+    """Appends of 1..16 rows per sequence rewrite only their rows' code bits
+    (the decode-time path); with ragged starts across a batch the packed
+    cache is byte-identical to one encode of all rows."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], seq_len=300, n_calib=64, batch=2, n_kv_heads=2, n_q_heads=8)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    kv.allocate(cq.to(dev), ck.to(dev))
+    n = 200
+    k = torch.stack([wl.keys(w, 0, b, 0, n) for b in range(2)])[None].to(dev)     # [1, 2, n, H, 128]
+    v = torch.stack([wl.values(w, 0, b, 0, n) for b in range(2)])[None].to(dev)
+    zeros = torch.zeros(2, dtype=torch.int32, device=dev)
+    kv.encode_append(0, k, v, zeros, torch.full((2,), n, dtype=torch.int32, device=dev))
+    whole = kv.cache.clone()
+    kv.cache.zero_()
+    sizes = [1, 3, 16, 7, 2, 1, 9, 16, 5, 11, 1, 13]
+    pos = [0, 0]
+    step = 0
+    while min(pos) < n:
+        cnt = [min(sizes[(step + b) % len(sizes)], n - pos[b]) for b in range(2)]
+        m = max(cnt)
+        kk = torch.zeros((1, 2, m, cfg.n_kv_heads, 128), dtype=torch.float16, device=dev)
+        vv = torch.zeros_like(kk)
+        for b in range(2):
+            kk[0, b, :cnt[b]] = k[0, b, pos[b]:pos[b] + cnt[b]]
+            vv[0, b, :cnt[b]] = v[0, b, pos[b]:pos[b] + cnt[b]]
+        start = torch.tensor(pos, dtype=torch.int32, device=dev)
+        count = torch.tensor(cnt, dtype=torch.int32, device=dev)
+        kv.encode_append(0, kk, vv, start, count)
+        pos = [pos[b] + cnt[b] for b in range(2)]
+        step += 1
+    torch.cuda.synchronize()
+    assert kv.device_error() == 0
+    assert torch.equal(whole, kv.cache)
+    kv.close()

@@ -60,7 +60,8 @@ int max_splits_of(const bgtq_config* c) { return c->max_splits == 0 ? 256 : c->m
 
 struct Layout {
   size_t krec, knorm, vrec, vnorm, cache_total;
-  size_t err, codebook, layouts, dectab, mkt, mvt, mv, energy_q, energy_k, qrot, qfrag, partials, ws_total;
+  size_t err, codebook, layouts, dectab, mkt, mvt, mv, energy_q, energy_k, qrot, qfrag, partials, comb_mid, comb_count,
+      ws_total;
 };
 
 int64_t tiles_of(const bgtq_config* c) { return (c->capacity_tokens + bgtq::kTile - 1) / bgtq::kTile; }
@@ -95,7 +96,9 @@ Layout plan(const bgtq_config* c) {
   const size_t qrows = size_t(c->n_layers) * c->max_batch * c->n_q_heads;
   p.qfrag = align_up(p.qrot + qrows * kD * sizeof(float));
   p.partials = align_up(p.qfrag + frag_bytes(c, c->n_layers));
-  p.ws_total = align_up(p.partials + qrows * max_splits_of(c) * bgtq::kPartialStride * sizeof(float));
+  p.comb_mid = align_up(p.partials + qrows * max_splits_of(c) * bgtq::kPartialStride * sizeof(float));
+  p.comb_count = align_up(p.comb_mid + qrows * bgtq::kCombSlices * bgtq::kPartialStride * sizeof(float));
+  p.ws_total = align_up(p.comb_count + qrows * sizeof(uint32_t));
   return p;
 }
 
@@ -306,6 +309,9 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->ws.qrot = reinterpret_cast<float*>(w8 + p.qrot);
   st->ws.qfrag = reinterpret_cast<uint4*>(w8 + p.qfrag);
   st->ws.partials = reinterpret_cast<float*>(w8 + p.partials);
+  st->ws.comb_mid = reinterpret_cast<float*>(w8 + p.comb_mid);
+  st->ws.comb_count = reinterpret_cast<uint32_t*>(w8 + p.comb_count);
+  const size_t comb_count_bytes = p.ws_total - p.comb_count;
   st->widths.assign(size_t(cfg->n_layers) * cfg->n_kv_heads * bgtq::kBlocks, 0);
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -323,6 +329,7 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaMemcpyAsync(st->ws.codebook, &cb, sizeof(cb), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(st->ws.err, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->ws.comb_count, 0, comb_count_bytes, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     delete st;
@@ -563,6 +570,9 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_static_scratch[BGTQ_STATIC_SCRATCH_BYTES];
 
+// Bytes at the start of the static array for the combine's arrival counters.
+constexpr size_t kStaticCountBytes = 64 << 10;
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -596,19 +606,29 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   const int split = split_for(st, layer_count, batch);
   const int64_t nspl = split;
   const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
+  // the combine's arrival counters first, at a fixed place (they are 0
+  // between calls, whatever the call's layout), then q~, its fragments, the
+  // split partials and the combine's slice merges
+  const size_t count_bytes = kStaticCountBytes;
   const size_t qrot_bytes = rows * kD * sizeof(float);
   const size_t fbytes = frag_bytes(&st->cfg, layer_count);
   const size_t part_bytes = rows * size_t(nspl) * bgtq::kPartialStride * sizeof(float);
-  if (qrot_bytes + fbytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES) return BGTQ_ERR_BUFFER_SIZE;
+  const size_t mid_bytes = rows * bgtq::kCombSlices * bgtq::kPartialStride * sizeof(float);
+  if (rows * sizeof(uint32_t) > count_bytes ||
+      count_bytes + qrot_bytes + fbytes + part_bytes + mid_bytes > BGTQ_STATIC_SCRATCH_BYTES)
+    return BGTQ_ERR_BUFFER_SIZE;
   void* base = nullptr;
   const int a = static_scratch_address(&base);
   if (a != BGTQ_OK) return a;
   // the same kernels as bgtq_decode_attn, with q~ and the partials redirected
   // to the static array (partials packed with n_splits as their stride)
   bgtq::Workspace ws = st->ws;
-  ws.qrot = static_cast<float*>(base);
-  ws.qfrag = reinterpret_cast<uint4*>(static_cast<unsigned char*>(base) + qrot_bytes);
-  ws.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + qrot_bytes + fbytes);
+  unsigned char* b8 = static_cast<unsigned char*>(base);
+  ws.comb_count = reinterpret_cast<uint32_t*>(b8);
+  ws.qrot = reinterpret_cast<float*>(b8 + count_bytes);
+  ws.qfrag = reinterpret_cast<uint4*>(b8 + count_bytes + qrot_bytes);
+  ws.partials = reinterpret_cast<float*>(b8 + count_bytes + qrot_bytes + fbytes);
+  ws.comb_mid = reinterpret_cast<float*>(b8 + count_bytes + qrot_bytes + fbytes + part_bytes);
   bgtq::Shape shape = st->shape;
   shape.max_splits = static_cast<int32_t>(nspl);
   cudaStream_t s = as_stream(stream);

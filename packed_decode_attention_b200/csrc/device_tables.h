@@ -10,7 +10,8 @@ namespace bgtq {
 constexpr int kD = 128;               // head_dim
 constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
 constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
-constexpr int kPartialStride = 132;   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kPartialStride = 132;
+constexpr int kCombSlices = 8;       // CTAs merging one row's splits in the combine   // floats per split-K partial: m, l, pad, pad, acc[128]
 constexpr int kTile = 64;             // cache positions per packed tile
 constexpr int kSplitGranule = kTile;  // split sizes are multiples of the tile
 constexpr int kMaxChunks = 12;        // 16-coordinate K chunks per head (8 + one partial per group)
@@ -69,6 +70,8 @@ struct Workspace {
   float* qrot;                   // [L][B][Hq][128]
   uint4* qfrag;                  // [L][B][Hkv][head blocks][kFragEntries]
   float* partials;               // [L][B][Hq][max_splits][kPartialStride]
+  float* comb_mid;               // [L][B][Hq][kCombSlices][kPartialStride]: slice merges of the combine
+  uint32_t* comb_count;          // [L][B][Hq]: slices merged so far (0 between calls)
 };
 
 // Cache arrays; T = ceil(capacity / 64) tiles per (layer, sequence, KV head).

@@ -637,6 +637,20 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
   const int li = blockIdx.x / (sh.n_kv_heads * batch);
   const int layer = layer0 + li;
   const int row = blockIdx.y;
+  const int lh = layer * sh.n_kv_heads + h;
+  // the next kernel of the stream may start its own table-only set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the kind's rotation (transposed, [in][out]) in shared memory, all loads
+  // in flight; a library table, read before the inputs are ready
+  extern __shared__ __align__(16) float mts[];  // [kD][kD]
+  {
+    const uint4* src = reinterpret_cast<const uint4*>((kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD);
+#pragma unroll 8
+    for (int u = tid; u < kD * kD / 4; u += kAppThreads) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
+  }
+  // Launched as a programmatic dependent of the previous kernel of the
+  // stream: the call's inputs and the cache are read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int start = start_v[b];
   const int count = count_v[b];
   if (start < 0 || count < 0 || count > n) {
@@ -649,7 +663,6 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
     if (tid == 0) atomicOr(ws.err, kErrCapacity);
     return;
   }
-  const int lh = layer * sh.n_kv_heads + h;
   __shared__ LayoutDev lay;
   __shared__ float xs[kD];
   __shared__ float fac[kNumGroupsMax];
@@ -699,10 +712,9 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
     int g = 0;
     for (int t = 1; t < ng; ++t)
       if (i >= lay.start[t]) g = t;
-    const float* mt = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
     const int j0 = lay.start[g], j1 = j0 + lay.size[g];
     float y = 0.f;
-    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], __ldg(mt + static_cast<size_t>(j) * kD + i), y);
+    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
     const int w = lay.width[g];
     const float u = y * fac[g];
     int code = 0;
@@ -816,6 +828,9 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
   __shared__ float qp[kD];
   __shared__ float part[kD];
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
+  // Launched as a programmatic dependent of the previous kernel of the
+  // stream: the query is read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid < kD) qp[tid] = __half2float(q[row * kD + lay.perm[tid]]);
   __syncthreads();
   float sacc = 0.f;
@@ -879,7 +894,7 @@ constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kStages = 2;
 constexpr int kDecMinBlocks = 3;  // CTAs per SM the register budget is sized for
-constexpr int kWaitLimit = 1 << 22;
+constexpr int kWaitLimit = 1 << 20;  // polls of up to kPollSuspendNs each: about a second
 constexpr float kRescaleSlack = 8.f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -901,12 +916,15 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// One bounded poll: the thread may sleep up to kPollSuspendNs waiting for the phase.
+constexpr uint32_t kPollSuspendNs = 1000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kPollSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -919,7 +937,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 struct DecodeLayout {  // byte offsets inside the dynamic shared memory
-  int bars, bq, tabk, grp, pdesc, ms, ls, stage, stage_bytes, total;
+  int bars, bq, tabk, grp, pdesc, ms, ls, mres, wsc, stage, stage_bytes, total;
 };
 
 __host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
@@ -933,7 +951,9 @@ __host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
   L.pdesc = L.tabk + kNumGroupsMax * 8 * 4;
   L.ms = L.grp + static_cast<int>(sizeof(DecodeTableDev));
   L.ls = L.ms + kDecWarps * 8 * 4;
-  L.stage = align128(L.ls + kDecWarps * 8 * 4);
+  L.mres = L.ls + kDecWarps * 8 * 4;           // merged m, l per head [2][8]
+  L.wsc = L.mres + 2 * 8 * 4;                  // merge weights [warp][8]
+  L.stage = align128(L.wsc + kDecWarps * 8 * 4);
   L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
   const int stages = kDecWarps * kStages * L.stage_bytes;
   const int merge = kDecWarps * 8 * kD * 4;  // reuses the stage buffers after the loop
@@ -1196,42 +1216,25 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
       mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
     }
+    // The reference maximum moves only when some logit of the tile exceeds it
+    // by more than kRescaleSlack (log2 units), so O is rescaled rarely;
+    // weights stay <= 2^kRescaleSlack and l and O always share the same
+    // reference.  l is kept per lane and summed over the warp at the end.
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kRescaleSlack || mx[1] > m_run[1] + kRescaleSlack)) {
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
-      mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
-    }
-    // The reference maximum moves only when the tile's maximum exceeds it by
-    // more than kRescaleSlack (log2 units), so O is rescaled rarely; weights
-    // stay <= 2^kRescaleSlack and l and O always share the same reference.
-    float alpha[2] = {1.f, 1.f}, sum[2] = {0.f, 0.f};
-    bool moved = false;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      if (mx[c] > m_run[c] + kRescaleSlack) {
-        alpha[c] = fast_exp2(m_run[c] - mx[c]);
-        m_run[c] = mx[c];
-        moved = true;
+      for (int o = 4; o < 32; o <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
       }
-    }
-    uint32_t bp[4][2];
+      float alpha[2] = {1.f, 1.f};
 #pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
-      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
-      sum[0] += p0 + p2;
-      sum[1] += p1 + p3;
-      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
-      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      sum[0] += __shfl_xor_sync(0xffffffffu, sum[0], o);
-      sum[1] += __shfl_xor_sync(0xffffffffu, sum[1], o);
-    }
-    l_run[0] = fmaf(l_run[0], alpha[0], sum[0]);
-    l_run[1] = fmaf(l_run[1], alpha[1], sum[1]);
-    if (moved) {
+      for (int c = 0; c < 2; ++c) {
+        if (mx[c] > m_run[c] + kRescaleSlack) {
+          alpha[c] = fast_exp2(m_run[c] - mx[c]);
+          m_run[c] = mx[c];
+        }
+        l_run[c] *= alpha[c];
+      }
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         O[m][0] *= alpha[0];
@@ -1239,6 +1242,16 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
         O[m][2] *= alpha[0];
         O[m][3] *= alpha[1];
       }
+    }
+    uint32_t bp[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
+      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
+      l_run[0] += p0 + p2;
+      l_run[1] += p1 + p3;
+      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
+      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
     }
     // P V in V's rotated basis
 #pragma unroll
@@ -1265,6 +1278,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   }
   __syncthreads();
   // ---- merge the warps (the stage buffers are reused) ----
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
+  }
   float* accs = reinterpret_cast<float*>(stage_base);  // [warp][8 heads][128]
   if (g8 == 0) {
     ms[warp * 8 + 2 * t4] = m_run[0];
@@ -1280,80 +1298,90 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
     a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
   }
-  __syncthreads();
   if (__syncthreads_or(timed_out)) return;
-  const int i = tid;
-  for (int hh = 0; hh < nh; ++hh) {
+  // per head: the common maximum, the warps' weights (warps without a tile
+  // hold m = -inf, l = 0, acc = 0) and the weighted denominator
+  float* wsc = reinterpret_cast<float*>(smem_raw + DL.wsc);
+  float* mres = reinterpret_cast<float*>(smem_raw + DL.mres);
+  if (tid < 8) {
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + hh]);
-    float lsum = 0.f, a = 0.f;
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
+    float lsum = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
-      // warps without a tile hold m = -inf, l = 0, acc = 0
-      const float mw = ms[w * 8 + hh];
+      const float mw = ms[w * 8 + tid];
       const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
-      lsum = fmaf(sc, ls[w * 8 + hh], lsum);
-      a = fmaf(sc, accs[(w * 8 + hh) * kD + i], a);
+      wsc[w * 8 + tid] = sc;
+      lsum = fmaf(sc, ls[w * 8 + tid], lsum);
     }
+    mres[tid] = M;
+    mres[8 + tid] = lsum;
+  }
+  __syncthreads();
+  const int i = tid;
+  for (int hh = 0; hh < nh; ++hh) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) a = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a);
     float* part = part_base + hh * part_head_stride;
     part[4 + i] = a;
     if (i == 0) {
-      part[0] = M;
-      part[1] = lsum;
+      part[0] = mres[hh];
+      part[1] = mres[8 + hh];
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq), 512
-// threads.  w_s = 2^(m_s - M) per split (0 for empty splits); the 16 warps
-// share the splits (lane = 4 rotated coordinates), then
-// o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), four threads per output.
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq *
+// kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
+// (w_s = 2^(m_s - M) per split, 0 for empty splits; lane = 4 rotated
+// coordinates) into an intermediate (m, l, acc); the row's last CTA to finish
+// (an arrival counter, reset by that CTA) merges the slices and rotates
+// back: o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), two threads per output.
 // ---------------------------------------------------------------------------
-constexpr int kCombThreads = 512;
+constexpr int kCombThreads = 256;
 constexpr int kCombWarps = kCombThreads / 32;
-constexpr int kCombMaxSplits = 1024;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
                                                                int n_splits, __half* __restrict__ out) {
-  const int hq = blockIdx.x % sh.n_q_heads;
-  const int b = (blockIdx.x / sh.n_q_heads) % batch;
-  const int li = blockIdx.x / (sh.n_q_heads * batch);
+  const int slice = blockIdx.x % kCombSlices;
+  const int rowi = blockIdx.x / kCombSlices;
+  const int hq = rowi % sh.n_q_heads;
+  const int b = (rowi / sh.n_q_heads) % batch;
+  const int li = rowi / (sh.n_q_heads * batch);
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // a quarter of the inverse V rotation's column for this thread (a library
-  // table), loaded while the previous kernel finishes
-  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-  const int d = tid & (kD - 1), quarter = tid >> 7;
-  float mvr[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) mvr[r] = __ldg(mv + (quarter * 32 + r) * kD + d);
+  // the next kernel of the stream may start its own table-only set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Launched as a programmatic dependent of the split pass: inputs, partials
   // and the output are touched only after that kernel has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = seq_lens[b];
   if (len < 0 || len > sh.capacity) {
-    if (tid == 0 && hq == 0) atomicOr(ws.err, kErrSeqLen);
+    if (tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
     len = 0;
   }
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  const int nspl = len > 0 ? min(n_splits, kCombMaxSplits) : 0;
-  if (nspl == 0) {
-    if (tid < kD) out[row * kD + tid] = __float2half(0.f);
+  if (len == 0) {
+    if (slice == 0 && tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
   }
-  const float* part =
-      ws.partials + ((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq) * sh.max_splits * kPartialStride;
+  const size_t wrow = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq;  // workspace row
+  const float* part = ws.partials + wrow * sh.max_splits * kPartialStride;
   __shared__ float red[kCombWarps];
-  __shared__ float sc[kCombMaxSplits];
   __shared__ float accs[kCombWarps][kD];
+  __shared__ float lsw[kCombWarps];
   __shared__ float a_s[kD];
-  // the largest split maximum
+  __shared__ int last;
+  // ---- this slice's splits ----
+  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
+  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
   float M = -CUDART_INF_F;
-  for (int s = tid; s < nspl; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
+  for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) red[warp] = M;
@@ -1361,48 +1389,72 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   M = red[0];
 #pragma unroll
   for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-  // split weights and the softmax denominator
-  float lsum = 0.f;
-  for (int s = tid; s < nspl; s += kCombThreads) {
-    const float ms = part[static_cast<size_t>(s) * kPartialStride];
-    const float w = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-    sc[s] = w;
-    lsum = fmaf(w, part[static_cast<size_t>(s) * kPartialStride + 1], lsum);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if (lane == 0) red[warp] = lsum;
-  __syncthreads();
-  lsum = 0.f;
-#pragma unroll
-  for (int w = 0; w < kCombWarps; ++w) lsum += red[w];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
 #pragma unroll 4
-  for (int s = warp; s < nspl; s += kCombWarps) {
-    const float wgt = sc[s];
-    const float4 a = *reinterpret_cast<const float4*>(part + static_cast<size_t>(s) * kPartialStride + 4 + 4 * lane);
+  for (int s = s0 + warp; s < s1; s += kCombWarps) {
+    const float* p = part + static_cast<size_t>(s) * kPartialStride;
+    const float ms = p[0];
+    const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+    lsum = fmaf(wgt, p[1], lsum);
+    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
     acc.x = fmaf(wgt, a.x, acc.x);
     acc.y = fmaf(wgt, a.y, acc.y);
     acc.z = fmaf(wgt, a.z, acc.z);
     acc.w = fmaf(wgt, a.w, acc.w);
   }
   *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
+  if (lane == 0) lsw[warp] = lsum;
   __syncthreads();
+  float* mid = ws.comb_mid + (wrow * kCombSlices + slice) * kPartialStride;
   if (tid < kD) {
     float a = 0.f;
 #pragma unroll
     for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
-    a_s[tid] = a / lsum;
+    mid[4 + tid] = a;
   }
+  if (tid == 0) {
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
+    mid[0] = M;
+    mid[1] = l;
+  }
+  // ---- the row's last slice merges the slices ----
+  __threadfence();
   __syncthreads();
-  // inverse V rotation: four threads per output, a quarter of the inputs each
+  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == kCombSlices - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* mids = ws.comb_mid + wrow * kCombSlices * kPartialStride;
+  float Mt = -CUDART_INF_F;
+#pragma unroll
+  for (int k = 0; k < kCombSlices; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
+  float Lt = 0.f, at = 0.f;
+  const int dd = tid & (kD - 1);
+#pragma unroll
+  for (int k = 0; k < kCombSlices; ++k) {
+    const float mk = __ldcg(mids + k * kPartialStride);
+    const float w = mk == -CUDART_INF_F ? 0.f : exp2f(mk - Mt);
+    Lt = fmaf(w, __ldcg(mids + k * kPartialStride + 1), Lt);
+    at = fmaf(w, __ldcg(mids + k * kPartialStride + 4 + dd), at);
+  }
+  if (tid < kD) a_s[tid] = at / Lt;
+  if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
+  // inverse V rotation: two threads per output, half of the inputs each
+  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  const int half = tid >> 7;
+  float mvr[64];
+#pragma unroll
+  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+  __syncthreads();
   float o = 0.f;
 #pragma unroll
-  for (int r = 0; r < 32; ++r) o = fmaf(mvr[r], a_s[quarter * 32 + r], o);
-  accs[quarter][d] = o;
+  for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
+  if (half == 1) accs[0][dd] = o;
   __syncthreads();
-  if (tid < kD) out[row * kD + d] = __float2half((accs[0][d] + accs[1][d]) + (accs[2][d] + accs[3][d]));
+  if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd]);
 }
 
 // Raises a kernel's dynamic shared-memory limit; callers keep the result in
@@ -1419,9 +1471,11 @@ cudaError_t encode_smem_once() {
 }
 
 // Launches a kernel as a programmatic dependent of the previous kernel in
-// the stream: it may start while that kernel finishes and must execute
-// griddepcontrol.wait before reading that kernel's results.  Used only for
-// the second and third kernels of a decode call, never for the first.
+// the stream: it may start while that kernel finishes.  Every kernel
+// launched this way reads only library tables before griddepcontrol.wait and
+// everything produced by earlier work in the stream after it, so the chain
+// append -> rotate -> split -> combine (and the next call's kernels) keeps
+// stream order for all data while the table-only prologues overlap.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                              Args... args) {
@@ -1488,9 +1542,10 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
   if (e != cudaSuccess) return e;
   if (n <= kAppendMaxRows) {
     // a few rows per sequence: rewrite only their code bits
-    append_kernel<<<dim3(layer_count * batch * s.n_kv_heads, n, 2), kAppThreads, 0, stream>>>(s, ws, cache, layer0, k, v,
-                                                                                             start, count, batch, n);
-    return cudaGetLastError();
+    static const cudaError_t attr = set_smem(append_kernel, kD * kD * sizeof(float));
+    if (attr != cudaSuccess) return attr;
+    return launch_dependent(append_kernel, dim3(layer_count * batch * s.n_kv_heads, n, 2), dim3(kAppThreads),
+                            kD * kD * sizeof(float), stream, s, ws, cache, layer0, k, v, start, count, batch, n);
   }
   dim3 grid(layer_count * batch * s.n_kv_heads, (n + kTile - 1) / kTile + 1, 2);
   encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
@@ -1499,8 +1554,8 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
 
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream) {
-  rotate_query_kernel<<<layer_count * batch * s.n_q_heads, kRotThreads, 0, stream>>>(s, ws, layer0, q, batch, qrot);
-  return cudaGetLastError();
+  return launch_dependent(rotate_query_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kRotThreads), 0, stream, s,
+                          ws, layer0, q, batch, qrot);
 }
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
@@ -1522,7 +1577,8 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int n_splits, __half* out,
                            cudaStream_t stream) {
-  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kCombThreads), 0, stream, s,
+  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads * kCombSlices), dim3(kCombThreads), 0,
+                          stream, s,
                           ws, layer0, seq_lens, batch, n_splits, out);
 }
 

@@ -33,6 +33,12 @@ if ROOT not in sys.path:
 
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes (read + write) per split-kernel launch from the ncu capture
+# summarised in profiles/decode_split_mma_qwen3b.md, for the workload it was
+# taken on (an 8-layer copy of it: the same per-layer launch).  Reported as
+# the roofline's "traffic"; None for other workloads.
+NCU_TRAFFIC_PER_LAUNCH = {"qwen3b": 27.851e6 + 0.001e6}
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -65,19 +71,46 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while running."""
+    """SM clock and clock-event reasons sampled while running: NVML polled
+    every millisecond from a thread (read-only queries), else nvidia-smi
+    at its 200 ms minimum."""
 
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_uuid):
+    def __init__(self, device_uuid, device_index):
         self.uuid = device_uuid
+        self.index = device_index
+        self.samples = []          # (time, sm_mhz, max_mhz, reasons set)
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop_flag = threading.Event()
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            masks = [(n, getattr(pynvml, m)) for n, m in self.REASONS]
+            max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    mhz = pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    self.samples.append((time.time(), float(mhz), float(max_mhz), {n for n, m in masks if r & m}))
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -85,14 +118,23 @@ class ClockSampler:
         except Exception:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]),
+                                     {n for n, v in zip(names, parts[3:7]) if v.lower() == "active"}))
+            except ValueError:
+                continue
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -103,25 +145,15 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self, t0, t1):
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        mhz, mx, reasons = [], [], set()
-        rows = [l for t, l in self.lines if t0 - 0.25 <= t <= t1 + 0.25] or [l for _, l in self.lines]
-        for l in rows:
-            parts = [p.strip() for p in l.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                mhz.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not mhz:
+        rows = [x for x in self.samples if t0 <= x[0] <= t1] or \
+            [x for x in self.samples if t0 - 0.25 <= x[0] <= t1 + 0.25]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        reasons = set()
+        for x in rows:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in rows), "sm_max_mhz": max(x[2] for x in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
 
 
 def token_bytes(kv, cfg):
@@ -365,7 +397,7 @@ def main():
         return a.elapsed_time(z) / steps, g, (t_wall0, t_wall1)
 
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(uuid)
+    sampler = ClockSampler(uuid, local)
     sampler.start()
     time.sleep(0.5)
     ms_step, graph, (tw0, tw1) = time_graph(step, args.steps, args.warmup)
@@ -380,12 +412,15 @@ def main():
     ms_multi = max_over_ranks(ms_multi)
     del g_multi
 
-    # ---- the split-K kernel alone: events around each launch ----
+    # ---- the split-K kernel alone: events around each per-layer launch, in a
+    # captured step (the event nodes keep the split kernel from overlapping
+    # its neighbours, so each interval is that kernel's whole duration) ----
     tb = token_bytes(kv, cfg)
     qrot = torch.empty((1, B, HQ, 128), dtype=torch.float32, device=dev)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-    split_ms = []
-    for it in range(args.warmup + args.steps):
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in range(L)]
+
+    def step_timed_split():
         for l in range(L):
             kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
             kv.rotate_query(l, q_all[l:l + 1], qrot)
@@ -393,9 +428,19 @@ def main():
             kv.decode_split(l, qrot, seq)
             ev[l][1].record()
             kv.decode_combine(l, seq, out[l:l + 1])
+
+    step_timed_split()
+    torch.cuda.synchronize()
+    g_split = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_split):
+        step_timed_split()
+    split_ms = []
+    for it in range(args.warmup + args.steps):
+        g_split.replay()
         torch.cuda.synchronize()
         if it >= args.warmup:
             split_ms.extend(a.elapsed_time(z) for a, z in ev)
+    del g_split
     split_avg_ms = statistics.mean(split_ms)
     bytes_per_layer = [sum(lens[b] * tb[l, h] for b in range(B) for h in range(H)) for l in range(L)]
     alg_bytes = statistics.mean(bytes_per_layer)
@@ -485,11 +530,11 @@ def main():
         "config": workload_config(w, lens),
         "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "decode_split_kernel",
+                     "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload), "kernel": "decode_mma_kernel",
                      "launch_ms": split_avg_ms, "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind},
         "e2e": {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * L * args.steps,
+        "gpu_launches": 4 * L * args.steps,
         "clocks": clocks,
         "multi_layer": {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
                         "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},

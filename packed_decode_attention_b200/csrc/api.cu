@@ -525,7 +525,7 @@ int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const 
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_qrot) || !aligned16(d_seq_lens)) return BGTQ_ERR_ALIGNMENT;
-  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, true, d_seq_lens, batch,
+  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, batch,
                                    split_for(st, layer_count, batch), as_stream(stream)) == cudaSuccess
              ? BGTQ_OK
              : BGTQ_ERR_CUDA;
@@ -555,7 +555,7 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, st->ws.qrot, false, d_seq_lens, batch,
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, batch,
                                 split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split,
@@ -635,7 +635,7 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   if (bgtq::launch_rotate_query(shape, ws, layer, layer_count, static_cast<const __half*>(d_q), batch, ws.qrot, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, ws.qrot, false, d_seq_lens, batch, split, s) !=
+  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, nullptr, d_seq_lens, batch, split, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, static_cast<__half*>(d_out), s) !=

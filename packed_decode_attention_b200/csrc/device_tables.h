@@ -104,11 +104,11 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           const int32_t* count, int batch, int n, cudaStream_t stream);
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
-// The split pass reads q~ from ws.qfrag; frag_from_qrot first rebuilds those
-// fragments from qrot (callers that rotated the query themselves).
+// The split pass reads q~ as fragments from ws.qfrag (written by the query
+// rotation), or, when qrot is not null, builds them from qrot itself.
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, bool frag_from_qrot, const int32_t* seq_lens,
-                                int batch, int n_splits, cudaStream_t stream);
+                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
+                                int n_splits, cudaStream_t stream);
 // Resident split-decode CTAs per SM for a config (0 on error).
 int decode_ctas_per_sm(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,

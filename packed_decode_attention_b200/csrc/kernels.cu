@@ -853,23 +853,6 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
   write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), tid, kRotThreads);
 }
 
-// The B fragments of q~ from a rotated query given by the caller (the
-// split stage called on its own).  Grid (layer_count * batch * Hq), 128 threads.
-__global__ void __launch_bounds__(kD) fragment_kernel(Shape sh, Workspace ws, int layer0,
-                                                      const float* __restrict__ qrot, int batch) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int hq = blockIdx.x % sh.n_q_heads;
-  const int b = (blockIdx.x / sh.n_q_heads) % batch;
-  const int li = blockIdx.x / (sh.n_q_heads * batch);
-  const int kvh = hq / sh.group;
-  const LayoutDev& lay = ws.layouts[(layer0 + li) * sh.n_kv_heads + kvh];
-  __shared__ float qp[kD];
-  qp[threadIdx.x] = qrot[((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq) * kD + threadIdx.x];
-  __syncthreads();
-  write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), threadIdx.x,
-              kD);
-}
-
 // ---------------------------------------------------------------------------
 // a5: split-K decode straight from the packed tiles on the tensor cores.
 //
@@ -1027,8 +1010,8 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
 // (m = -inf, l = 0) when it has no tile.
 template <int VB>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
-    decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const int32_t* __restrict__ seq_lens,
-                      int batch, int ctas_per_unit, int head_blocks) {
+    decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
+                      const int32_t* __restrict__ seq_lens, int batch, int ctas_per_unit, int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const DecodeLayout DL = decode_layout(sh.kbits, VB);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
@@ -1093,10 +1076,38 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     return;
   }
   {
-    // q~ fragments of this unit, written by the query rotation
-    const uint4* src = frag_block(sh, ws, li, b, h, hb);
-    const int n = 32 * (lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4));
-    for (int u = tid; u < n; u += kDecThreads) bq[u] = src[u];
+    const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+    if (qrot == nullptr) {
+      // q~ fragments of this unit, written by the query rotation
+      const uint4* src = frag_block(sh, ws, li, b, h, hb);
+      for (int u = tid; u < 32 * nchunk; u += kDecThreads) bq[u] = src[u];
+    } else {
+      // the split pass on its own: the fragments from the caller's q~
+      // (fp32, record order): coordinates 16 j + 4 t .. + 3 of chunk c's
+      // group for head t / 4 ... see write_frags for the layout
+      const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
+      for (int u = tid; u < 32 * nchunk; u += kDecThreads) {
+        const int c = u >> 5, ln = u & 31;
+        int g = 0;
+        while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
+        const int j = c - lay.chunk_base[g];
+        const int d = lay.size[g], st = lay.start[g];
+        const int head = ln >> 2;
+        float v[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int coord = 16 * j + 4 * (ln & 3) + m;
+          v[m] = (head < nh && coord < d) ? qsrc[head * kD + st + coord] * kLog2e : 0.f;
+        }
+        const __half2 a = __floats2half2_rn(v[0], v[1]);
+        const __half2 c2 = __floats2half2_rn(v[2], v[3]);
+        const float2 af = __half22float2(a), cf = __half22float2(c2);
+        const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
+        const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
+        bq[u] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&c2),
+                           *reinterpret_cast<const uint32_t*>(&al), *reinterpret_cast<const uint32_t*>(&cl));
+      }
+    }
   }
   ByteTab tv;
   {
@@ -1494,14 +1505,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
-                             const int32_t* seq_lens, int batch, int n_splits, cudaStream_t stream) {
+                             const float* qrot, const int32_t* seq_lens, int batch, int n_splits,
+                             cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
   static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
   dim3 grid(n_splits, batch * s.n_kv_heads * head_blocks, layer_count);
   return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, seq_lens, batch, n_splits, head_blocks);
+                          ws, cache, layer0, qrot, seq_lens, batch, n_splits, head_blocks);
 }
 
 template <int VB>
@@ -1559,18 +1571,13 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 }
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, bool frag_from_qrot, const int32_t* seq_lens,
-                                int batch, int n_splits, cudaStream_t stream) {
-  if (frag_from_qrot) {
-    fragment_kernel<<<layer_count * batch * s.n_q_heads, kD, 0, stream>>>(s, ws, layer0, qrot, batch);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch, int n_splits,
+                                cudaStream_t stream) {
   switch (s.vbits) {
-    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
-    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
-    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
-    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, seq_lens, batch, n_splits, stream);
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
   }
 }
 

@@ -181,7 +181,8 @@ int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count,
 
 /* q~ in record order: per K group g, (1/sqrt(128)) (1/sqrt(d_g)) R_g q[D_g].
  *   d_q     fp16 [layer_count][batch][n_q_heads][128]
- *   d_qrot  fp32 [layer_count][batch][n_q_heads][128].  ASYNC. */
+ *   d_qrot  fp32 [layer_count][batch][n_q_heads][128]
+ * Also writes the tensor-core operand form of q~ into the workspace.  ASYNC. */
 int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                       int32_t batch, float* d_qrot, void* stream);
 
@@ -222,10 +223,11 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
  * of BGTQ_STATIC_SCRATCH_BYTES (16 MiB), which every GPU that loads the
  * library holds until the process exits.  The call allocates nothing.
  *
- * The scratch needed is layer_count * max_batch * n_q_heads * (512 +
- * n_splits * 528) bytes, n_splits = ceil(capacity_tokens / split tokens)
- * with the split chosen as for bgtq_decode_attn; a call needing more returns
- * BGTQ_ERR_BUFFER_SIZE before launching anything.
+ * The scratch needed is 64 KiB of arrival counters plus rows * (512 +
+ * n_splits * 528 + 8 * 528) bytes, rows = layer_count * max_batch *
+ * n_q_heads, plus 6 KiB per (layer, sequence, KV head, block of 8 query
+ * heads), with n_splits chosen as for bgtq_decode_attn; a call needing more
+ * returns BGTQ_ERR_BUFFER_SIZE before launching anything.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any
@@ -237,10 +239,11 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
 int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
 
-/* Tokens per split-K chunk for bgtq_decode_attn: 0 = automatic (from
- * capacity, max_splits and the SM count), else a multiple of 64 (one tile)
- * with ceil(capacity / tokens) <= max_splits.  Results do not depend on it
- * beyond floating-point reassociation. */
+/* Split-K width for bgtq_decode_attn: 0 = automatic (one wave of resident
+ * CTAs over all (layer, sequence, KV head) units, within max_splits), else a
+ * multiple of 64 (one tile): each unit's 64-position tiles are then dealt
+ * round-robin over ceil(capacity / tokens) <= max_splits split CTAs.  Results
+ * do not depend on it beyond floating-point reassociation. */
 int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens);
 
 /* Synchronises "stream", reads the device error flag into *h_flags

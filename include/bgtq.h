@@ -70,7 +70,8 @@ enum {
 /* Device error flag bits, reported by bgtq_get_device_error. */
 enum {
   BGTQ_DEVERR_CAPACITY = 1,    /* encode_append: start + count > capacity (rows skipped) */
-  BGTQ_DEVERR_SEQ_LEN = 2,     /* decode_attn: a seq_len < 0 or > capacity (sequence skipped, output 0) */
+  BGTQ_DEVERR_SEQ_LEN = 2,     /* decode: a seq_len < 0 or > capacity (sequence skipped, output 0), or a pos_lo /
+                                  buf_count out of range (clamped) */
   BGTQ_DEVERR_ARG = 4,         /* encode_append: start < 0 or count < 0 or count > n */
   BGTQ_DEVERR_NONFINITE = 8,   /* allocate: a calibration value is Inf or NaN */
   BGTQ_DEVERR_TIMEOUT = 16     /* decode: a wait for a tile copy gave up (bounded spin) */
@@ -199,6 +200,30 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
  * must not overlap on the GPU.  ASYNC. */
 int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                      const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
+
+/* Decode with an fp16 buffer: the Block-GTQ README's "withbuffer" setting
+ * (AIME commands: a few sink positions and a recent window kept
+ * unquantised).  For each layer, sequence b and query head h, attention runs
+ * over the packed positions [pos_lo[b], seq_lens[b]) and the sequence's
+ * first buf_count[b] buffered rows, with one softmax:
+ *   out = sum_t softmax_t(q . k_t / sqrt(128)) v_t
+ * over both sets (the packed rows dequantised as for bgtq_decode_attn, the
+ * buffered rows as given).  Which positions the buffered rows stand for is
+ * the caller's business (typically [0, n_sink) and [len - n_window, len),
+ * with pos_lo = n_sink and seq_lens = len - n_window).
+ *   d_q, d_out   fp16 [layer_count][batch][n_q_heads][128]
+ *   d_seq_lens   int32 [batch]  end of the packed range, 0..capacity
+ *   d_pos_lo     int32 [batch]  start of the packed range, 0..seq_lens[b]
+ *   d_buf_k/v    fp16 [layer_count][batch][n_buf][n_kv_heads][128]
+ *   d_buf_count  int32 [batch]  buffered rows used, 0..n_buf
+ *   n_buf        1..2048
+ * An empty packed range and no buffered row give 0.  Out-of-range
+ * lengths set BGTQ_DEVERR_SEQ_LEN and are clamped.  Uses the workspace like
+ * bgtq_decode_attn.  ASYNC. */
+int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
+                              const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,
+                              void* stream);
 
 /* The two stages of bgtq_decode_attn after bgtq_rotate_query, for callers
  * that time or schedule them separately (same arguments and results):

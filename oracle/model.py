@@ -131,3 +131,23 @@ def decode(tables, layer, head, q, k_tiles, k_norms, v_tiles, v_norm, n):
                               tables.codebooks[cfg.v_avg_bits], cfg.head_dim)
     q64 = np.asarray(q, dtype=np.float16).astype(np.float64)
     return attend(q64, k_hat, v_hat)
+
+
+def decode_buffered(tables, layer, head, q, k_tiles, k_norms, v_tiles, v_norm, lo, hi, buf_k, buf_v):
+    """Decode attention with an fp16 buffer (blockgtq README, AIME commands:
+    the "withbuffer" setting keeps a few sink positions and a recent window
+    unquantised): one softmax over the dequantised packed positions lo..hi-1
+    of the given tiles and the buffered rows buf_k / buf_v (fp16 [n_buf, D],
+    taken as they are).  out float64 [G, D]."""
+    cfg = tables.cfg
+    groups = tables.groups[layer, head]
+    kc = tiles.unpack_k_tiles(k_tiles, groups, hi)[lo:hi] if hi > lo else np.zeros((0, 128), dtype=np.int64)
+    vc = tiles.unpack_v_tiles(v_tiles, cfg.v_avg_bits, hi)[lo:hi] if hi > lo else np.zeros((0, 128), dtype=np.int64)
+    k_hat = dequantise_keys(kc, np.asarray(k_norms)[lo:hi], groups, tables.k_rot[layer, head], tables.codebooks,
+                            cfg.head_dim)
+    v_hat = dequantise_values(vc, np.asarray(v_norm)[lo:hi], tables.v_rot[layer, head],
+                              tables.codebooks[cfg.v_avg_bits], cfg.head_dim)
+    bk = np.asarray(buf_k, dtype=np.float16).astype(np.float64).reshape(-1, cfg.head_dim)
+    bv = np.asarray(buf_v, dtype=np.float16).astype(np.float64).reshape(-1, cfg.head_dim)
+    q64 = np.asarray(q, dtype=np.float16).astype(np.float64)
+    return attend(q64, np.concatenate([k_hat, bk]), np.concatenate([v_hat, bv]))

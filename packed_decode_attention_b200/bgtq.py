@@ -99,6 +99,7 @@ _SIGS = {
     "bgtq_encode_append": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
     "bgtq_rotate_query": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
@@ -239,6 +240,13 @@ def bgtq_decode_attn(state, layer, layer_count, d_q, d_seq_lens, batch, d_out, s
                                   _stream(stream)))
 
 
+def bgtq_decode_attn_buffered(state, layer, layer_count, d_q, d_seq_lens, d_pos_lo, batch, d_buf_k, d_buf_v,
+                              d_buf_count, n_buf, d_out, stream=None):
+    _check(lib().bgtq_decode_attn_buffered(state, layer, layer_count, _ptr(d_q), _ptr(d_seq_lens), _ptr(d_pos_lo),
+                                           batch, _ptr(d_buf_k), _ptr(d_buf_v), _ptr(d_buf_count), n_buf,
+                                           _ptr(d_out), _stream(stream)))
+
+
 def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
     _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
 
@@ -339,6 +347,13 @@ class PackedKVCache:
     def decode_attn(self, layer, q, seq_lens, out, layer_count=1):
         """q, out fp16 [layer_count, batch, Hq, 128]; seq_lens int32 [batch] on the device."""
         bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, q.shape[1], out)
+
+    def decode_attn_buffered(self, layer, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out, layer_count=1):
+        """Attention over the packed positions [pos_lo, seq_lens) and the first
+        buf_count fp16 buffered rows (buf_k, buf_v fp16 [layer_count, batch,
+        n_buf, Hkv, 128])."""
+        bgtq_decode_attn_buffered(self.state, layer, layer_count, q, seq_lens, pos_lo, q.shape[1], buf_k, buf_v,
+                                  buf_count, buf_k.shape[2], out)
 
     def decode_split(self, layer, qrot, seq_lens, layer_count=1):
         """The split-K stage alone from rotated queries (fp32 [layer_count, batch, Hq, 128])."""

@@ -97,7 +97,7 @@ Layout plan(const bgtq_config* c) {
   p.qfrag = align_up(p.qrot + qrows * kD * sizeof(float));
   p.partials = align_up(p.qfrag + frag_bytes(c, c->n_layers));
   p.comb_mid = align_up(p.partials + qrows * max_splits_of(c) * bgtq::kPartialStride * sizeof(float));
-  p.comb_count = align_up(p.comb_mid + qrows * bgtq::kCombSlices * bgtq::kPartialStride * sizeof(float));
+  p.comb_count = align_up(p.comb_mid + qrows * (bgtq::kCombSlices + 1) * bgtq::kPartialStride * sizeof(float));
   p.ws_total = align_up(p.comb_count + qrows * sizeof(uint32_t));
   return p;
 }
@@ -525,7 +525,7 @@ int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const 
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_qrot) || !aligned16(d_seq_lens)) return BGTQ_ERR_ALIGNMENT;
-  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, batch,
+  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, nullptr, batch,
                                    split_for(st, layer_count, batch), as_stream(stream)) == cudaSuccess
              ? BGTQ_OK
              : BGTQ_ERR_CUDA;
@@ -538,7 +538,7 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
   return bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch,
-                              split_for(st, layer_count, batch), static_cast<__half*>(d_out),
+                              split_for(st, layer_count, batch), bgtq::BufferArgs{}, static_cast<__half*>(d_out),
                               as_stream(stream)) == cudaSuccess
              ? BGTQ_OK
              : BGTQ_ERR_CUDA;
@@ -555,10 +555,42 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, batch,
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, nullptr, batch,
                                 split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split,
+  if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split, bgtq::BufferArgs{},
+                           static_cast<__half*>(d_out), s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  return BGTQ_OK;
+}
+
+int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
+                              const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,
+                              void* stream) {
+  if (!st || !d_q || !d_seq_lens || !d_pos_lo || !d_buf_k || !d_buf_v || !d_buf_count || !d_out) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
+  if (n_buf < 1 || n_buf > bgtq::kMaxBufferRows) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_pos_lo) || !aligned16(d_buf_k) ||
+      !aligned16(d_buf_v) || !aligned16(d_buf_count) || !aligned16(d_out))
+    return BGTQ_ERR_ALIGNMENT;
+  const int split = split_for(st, layer_count, batch);
+  cudaStream_t s = as_stream(stream);
+  bgtq::BufferArgs buf;
+  buf.q = static_cast<const __half*>(d_q);
+  buf.k = static_cast<const __half*>(d_buf_k);
+  buf.v = static_cast<const __half*>(d_buf_v);
+  buf.count = d_buf_count;
+  buf.pos_lo = d_pos_lo;
+  buf.n_buf = n_buf;
+  if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
+                                st->ws.qrot, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, d_pos_lo, batch,
+                                split, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split, buf,
                            static_cast<__half*>(d_out), s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   return BGTQ_OK;
@@ -613,7 +645,7 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   const size_t qrot_bytes = rows * kD * sizeof(float);
   const size_t fbytes = frag_bytes(&st->cfg, layer_count);
   const size_t part_bytes = rows * size_t(nspl) * bgtq::kPartialStride * sizeof(float);
-  const size_t mid_bytes = rows * bgtq::kCombSlices * bgtq::kPartialStride * sizeof(float);
+  const size_t mid_bytes = rows * (bgtq::kCombSlices + 1) * bgtq::kPartialStride * sizeof(float);
   if (rows * sizeof(uint32_t) > count_bytes ||
       count_bytes + qrot_bytes + fbytes + part_bytes + mid_bytes > BGTQ_STATIC_SCRATCH_BYTES)
     return BGTQ_ERR_BUFFER_SIZE;
@@ -635,10 +667,11 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   if (bgtq::launch_rotate_query(shape, ws, layer, layer_count, static_cast<const __half*>(d_q), batch, ws.qrot, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, nullptr, d_seq_lens, batch, split, s) !=
+  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, nullptr, d_seq_lens, nullptr, batch, split, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, static_cast<__half*>(d_out), s) !=
+  if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, bgtq::BufferArgs{},
+                           static_cast<__half*>(d_out), s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
   return BGTQ_OK;

@@ -11,7 +11,8 @@ constexpr int kD = 128;               // head_dim
 constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
 constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
 constexpr int kPartialStride = 132;
-constexpr int kCombSlices = 8;       // CTAs merging one row's splits in the combine   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kCombSlices = 8;       // CTAs merging one row's splits in the combine
+constexpr int kMaxBufferRows = 2048; // fp16 buffered rows per sequence a decode call may attend   // floats per split-K partial: m, l, pad, pad, acc[128]
 constexpr int kTile = 64;             // cache positions per packed tile
 constexpr int kSplitGranule = kTile;  // split sizes are multiples of the tile
 constexpr int kMaxChunks = 12;        // 16-coordinate K chunks per head (8 + one partial per group)
@@ -70,7 +71,7 @@ struct Workspace {
   float* qrot;                   // [L][B][Hq][128]
   uint4* qfrag;                  // [L][B][Hkv][head blocks][kFragEntries]
   float* partials;               // [L][B][Hq][max_splits][kPartialStride]
-  float* comb_mid;               // [L][B][Hq][kCombSlices][kPartialStride]: slice merges of the combine
+  float* comb_mid;               // [L][B][Hq][kCombSlices + 1][kPartialStride]: slice merges of the combine
   uint32_t* comb_count;          // [L][B][Hq]: slices merged so far (0 between calls)
 };
 
@@ -106,13 +107,27 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
 // The split pass reads q~ as fragments from ws.qfrag (written by the query
 // rotation), or, when qrot is not null, builds them from qrot itself.
+// pos_lo (int32 [batch], may be null = 0): the first packed position attended.
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch,
-                                int n_splits, cudaStream_t stream);
+                                int layer_count, const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo,
+                                int batch, int n_splits, cudaStream_t stream);
 // Resident split-decode CTAs per SM for a config (0 on error).
 int decode_ctas_per_sm(const Shape& s);
+// The fp16 buffered rows a decode call attends besides the packed cache
+// (k == nullptr: none).  q: the decode query fp16 [layer_count][batch][Hq][128];
+// k, v: fp16 [layer_count][batch][n_buf][Hkv][128]; count: int32 [batch]
+// rows used per sequence; pos_lo: int32 [batch] first packed position
+// attended (null = 0).
+struct BufferArgs {
+  const __half* q;
+  const __half* k;
+  const __half* v;
+  const int32_t* count;
+  const int32_t* pos_lo;
+  int n_buf;
+};
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int n_splits, __half* out,
+                           const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream);
 
 }  // namespace bgtq

@@ -1011,7 +1011,8 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
 template <int VB>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
-                      const int32_t* __restrict__ seq_lens, int batch, int ctas_per_unit, int head_blocks) {
+                      const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ pos_lo, int batch,
+                      int ctas_per_unit, int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const DecodeLayout DL = decode_layout(sh.kbits, VB);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
@@ -1054,7 +1055,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = seq_lens[b];
   if (len < 0 || len > sh.capacity) len = 0;  // flagged by the combine kernel
-  const int ntl = (len + kTile - 1) / kTile;
+  // the packed positions attended: [lo, len); lo > 0 when the caller keeps the
+  // first positions unquantised (their rows come through the combine)
+  int lo = pos_lo != nullptr ? pos_lo[b] : 0;
+  if (lo < 0 || lo > len) lo = len;            // flagged by the combine kernel
+  const int tlo = lo / kTile;
+  const int ntl = lo < len ? (len + kTile - 1) / kTile - tlo : 0;
   const int W = ctas_per_unit * kDecWarps;
   const int wu = cu * kDecWarps + warp;
   const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
@@ -1127,7 +1133,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   uint64_t* my_bars = bars + warp * kStages;
 
   auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
-    const int tile = wu + k * W;
+    const int tile = tlo + wu + k * W;
     unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
     uint64_t* bar = &my_bars[k % kStages];
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1160,7 +1166,9 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
     const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
     const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
-    const int nvalid = min(kTile, len - (wu + k * W) * kTile);
+    const int tpos = (tlo + wu + k * W) * kTile;
+    const int nvalid = min(kTile, len - tpos);       // positions [nlow, nvalid) of the tile are attended
+    const int nlow = max(0, lo - tpos);
 
     // logits, one width group at a time, each scaled by its per-token norm
     float L[4][4];
@@ -1208,14 +1216,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       wv[mu][0] = __half2float(vn[16 * mu + g8]) * kInvSqrtD;
       wv[mu][1] = __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD;
     }
-    if (nvalid < kTile) {
+    if (nvalid < kTile || nlow > 0) {
 #pragma unroll
       for (int mu = 0; mu < 4; ++mu) {
-        if (16 * mu + g8 >= nvalid) {
+        if (16 * mu + g8 >= nvalid || 16 * mu + g8 < nlow) {
           L[mu][0] = L[mu][1] = -CUDART_INF_F;
           wv[mu][0] = 0.f;
         }
-        if (16 * mu + g8 + 8 >= nvalid) {
+        if (16 * mu + g8 + 8 >= nvalid || 16 * mu + g8 + 8 < nlow) {
           L[mu][2] = L[mu][3] = -CUDART_INF_F;
           wv[mu][1] = 0.f;
         }
@@ -1345,21 +1353,25 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq *
-// kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
-// (w_s = 2^(m_s - M) per split, 0 for empty splits; lane = 4 rotated
-// coordinates) into an intermediate (m, l, acc); the row's last CTA to finish
-// (an arrival counter, reset by that CTA) merges the slices and rotates
-// back: o = R_V^T (sum_s w_s acc_s) / (sum_s w_s l_s), two threads per output.
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq * nsl),
+// 256 threads, nsl = kCombSlices, plus one when an fp16 buffer is attended.
+// Each of the first kCombSlices CTAs of a row merges one slice of the row's
+// splits (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated
+// coordinates) into an intermediate (m, l, acc) in V's rotated basis; the
+// buffer CTA attends the row's fp16 buffered rows directly (logits q . k /
+// sqrt(D) in log2 units, acc = sum p v unrotated).  The row's last CTA to
+// finish (an arrival counter, reset by that CTA) merges them:
+// o = (R_V^T sum_s w_s acc_s + w_buf acc_buf) / (sum_s w_s l_s + w_buf l_buf).
 // ---------------------------------------------------------------------------
 constexpr int kCombThreads = 256;
 constexpr int kCombWarps = kCombThreads / 32;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
-                                                               int n_splits, __half* __restrict__ out) {
-  const int slice = blockIdx.x % kCombSlices;
-  const int rowi = blockIdx.x / kCombSlices;
+                                                               int n_splits, BufferArgs buf, __half* __restrict__ out) {
+  const int nsl = kCombSlices + (buf.k != nullptr ? 1 : 0);
+  const int slice = blockIdx.x % nsl;
+  const int rowi = blockIdx.x / nsl;
   const int hq = rowi % sh.n_q_heads;
   const int b = (rowi / sh.n_q_heads) % batch;
   const int li = rowi / (sh.n_q_heads * batch);
@@ -1372,12 +1384,16 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   // and the output are touched only after that kernel has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int len = seq_lens[b];
-  if (len < 0 || len > sh.capacity) {
+  int lo = buf.pos_lo != nullptr ? buf.pos_lo[b] : 0;
+  int cnt = buf.k != nullptr ? buf.count[b] : 0;
+  if (len < 0 || len > sh.capacity || lo < 0 || lo > len || cnt < 0 || cnt > buf.n_buf) {
     if (tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
-    len = 0;
+    if (len < 0 || len > sh.capacity) len = 0;
+    if (lo < 0 || lo > len) lo = len;
+    cnt = cnt < 0 ? 0 : (cnt > buf.n_buf ? buf.n_buf : cnt);
   }
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  if (len == 0) {
+  if (lo >= len && cnt == 0) {
     if (slice == 0 && tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
   }
@@ -1387,69 +1403,122 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   __shared__ float accs[kCombWarps][kD];
   __shared__ float lsw[kCombWarps];
   __shared__ float a_s[kD];
+  __shared__ float lgb[kMaxBufferRows];
   __shared__ int last;
-  // ---- this slice's splits ----
-  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
-  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
-  float M = -CUDART_INF_F;
-  for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
+  float* mid = ws.comb_mid + (wrow * (kCombSlices + 1) + slice) * kPartialStride;
+  if (slice < kCombSlices) {
+    // ---- one slice of the row's splits ----
+    const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
+    const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
+    float M = -CUDART_INF_F;
+    for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
 #pragma unroll
-  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lsum = 0.f;
+    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f;
 #pragma unroll 4
-  for (int s = s0 + warp; s < s1; s += kCombWarps) {
-    const float* p = part + static_cast<size_t>(s) * kPartialStride;
-    const float ms = p[0];
-    const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-    lsum = fmaf(wgt, p[1], lsum);
-    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
-    acc.x = fmaf(wgt, a.x, acc.x);
-    acc.y = fmaf(wgt, a.y, acc.y);
-    acc.z = fmaf(wgt, a.z, acc.z);
-    acc.w = fmaf(wgt, a.w, acc.w);
-  }
-  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
-  if (lane == 0) lsw[warp] = lsum;
-  __syncthreads();
-  float* mid = ws.comb_mid + (wrow * kCombSlices + slice) * kPartialStride;
-  if (tid < kD) {
-    float a = 0.f;
+    for (int s = s0 + warp; s < s1; s += kCombWarps) {
+      const float* p = part + static_cast<size_t>(s) * kPartialStride;
+      const float ms = p[0];
+      const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+      lsum = fmaf(wgt, p[1], lsum);
+      const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+      acc.x = fmaf(wgt, a.x, acc.x);
+      acc.y = fmaf(wgt, a.y, acc.y);
+      acc.z = fmaf(wgt, a.z, acc.z);
+      acc.w = fmaf(wgt, a.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
+    if (lane == 0) lsw[warp] = lsum;
+    __syncthreads();
+    if (tid < kD) {
+      float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
-    mid[4 + tid] = a;
-  }
-  if (tid == 0) {
-    float l = 0.f;
+      for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
+      mid[4 + tid] = a;
+    }
+    if (tid == 0) {
+      float l = 0.f;
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
-    mid[0] = M;
-    mid[1] = l;
+      for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
+      mid[0] = M;
+      mid[1] = l;
+    }
+  } else {
+    // ---- the fp16 buffered rows of the row's KV head ----
+    const __half* qv = buf.q + row * kD;
+    const float qs = kInvSqrtD * kLog2e;
+    const float4 q4 = make_float4(__half2float(qv[4 * lane]) * qs, __half2float(qv[4 * lane + 1]) * qs,
+                                  __half2float(qv[4 * lane + 2]) * qs, __half2float(qv[4 * lane + 3]) * qs);
+    const size_t rstride = static_cast<size_t>(sh.n_kv_heads) * kD;
+    const size_t base = (static_cast<size_t>(li) * batch + b) * buf.n_buf * rstride + static_cast<size_t>(kvh) * kD;
+    for (int r = warp; r < cnt; r += kCombWarps) {
+      const uint2 kw = *reinterpret_cast<const uint2*>(buf.k + base + r * rstride + 4 * lane);
+      const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
+      const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
+      float d = q4.x * k01.x;
+      d = fmaf(q4.y, k01.y, d);
+      d = fmaf(q4.z, k23.x, d);
+      d = fmaf(q4.w, k23.y, d);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (lane == 0) lgb[r] = d;
+    }
+    __syncthreads();
+    float M = -CUDART_INF_F;
+    for (int r = tid; r < cnt; r += kCombThreads) M = fmaxf(M, lgb[r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
+    // P v over the rows: thread (dimension d, half of the rows)
+    const int d = tid & (kD - 1), hr = tid >> 7;
+    float acc = 0.f, lsum = 0.f;
+    for (int r = hr; r < cnt; r += 2) {
+      const float p = exp2f(lgb[r] - M);
+      lsum += p;
+      acc = fmaf(p, __half2float(buf.v[base + r * rstride + d]), acc);
+    }
+    if (hr == 1) {
+      accs[0][d] = acc;
+      if (d == 0) lsw[0] = lsum;
+    }
+    __syncthreads();
+    if (hr == 0) {
+      mid[4 + d] = cnt > 0 ? acc + accs[0][d] : 0.f;
+      if (d == 0) {
+        mid[0] = cnt > 0 ? M : -CUDART_INF_F;
+        mid[1] = cnt > 0 ? lsum + lsw[0] : 0.f;
+      }
+    }
   }
-  // ---- the row's last slice merges the slices ----
+  // ---- the row's last CTA merges the intermediates ----
   __threadfence();
   __syncthreads();
-  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == kCombSlices - 1;
+  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == static_cast<unsigned>(nsl - 1);
   __syncthreads();
   if (!last) return;
   __threadfence();
-  const float* mids = ws.comb_mid + wrow * kCombSlices * kPartialStride;
+  const float* mids = ws.comb_mid + wrow * (kCombSlices + 1) * kPartialStride;
   float Mt = -CUDART_INF_F;
-#pragma unroll
-  for (int k = 0; k < kCombSlices; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
-  float Lt = 0.f, at = 0.f;
+  for (int k = 0; k < nsl; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
+  float Lt = 0.f, at = 0.f, ab = 0.f;
   const int dd = tid & (kD - 1);
-#pragma unroll
-  for (int k = 0; k < kCombSlices; ++k) {
+  for (int k = 0; k < nsl; ++k) {
     const float mk = __ldcg(mids + k * kPartialStride);
     const float w = mk == -CUDART_INF_F ? 0.f : exp2f(mk - Mt);
     Lt = fmaf(w, __ldcg(mids + k * kPartialStride + 1), Lt);
-    at = fmaf(w, __ldcg(mids + k * kPartialStride + 4 + dd), at);
+    const float a = __ldcg(mids + k * kPartialStride + 4 + dd);
+    if (k < kCombSlices) at = fmaf(w, a, at);  // rotated basis
+    else ab = w * a;                             // the buffer's rows, unrotated
   }
   if (tid < kD) a_s[tid] = at / Lt;
   if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
@@ -1465,7 +1534,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
   if (half == 1) accs[0][dd] = o;
   __syncthreads();
-  if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd]);
+  if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
 }
 
 // Raises a kernel's dynamic shared-memory limit; callers keep the result in
@@ -1505,15 +1574,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
-                             const float* qrot, const int32_t* seq_lens, int batch, int n_splits,
-                             cudaStream_t stream) {
+                             const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo, int batch,
+                             int n_splits, cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
   static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
   dim3 grid(n_splits, batch * s.n_kv_heads * head_blocks, layer_count);
   return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, qrot, seq_lens, batch, n_splits, head_blocks);
+                          ws, cache, layer0, qrot, seq_lens, pos_lo, batch, n_splits, head_blocks);
 }
 
 template <int VB>
@@ -1571,22 +1640,26 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 }
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, int batch, int n_splits,
-                                cudaStream_t stream) {
+                                int layer_count, const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo,
+                                int batch, int n_splits, cudaStream_t stream) {
   switch (s.vbits) {
-    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
-    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
-    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
-    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, batch, n_splits, stream);
+    case 1:
+      return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
+    case 2:
+      return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
+    case 3:
+      return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
+    default:
+      return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
   }
 }
 
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int n_splits, __half* out,
+                           const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream) {
-  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads * kCombSlices), dim3(kCombThreads), 0,
-                          stream, s,
-                          ws, layer0, seq_lens, batch, n_splits, out);
+  const int nsl = kCombSlices + (buf.k != nullptr ? 1 : 0);
+  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads * nsl), dim3(kCombThreads), 0, stream,
+                          s, ws, layer0, seq_lens, batch, n_splits, buf, out);
 }
 
 }  // namespace bgtq

@@ -425,3 +425,88 @@ def test_small_appends_equal_one_encode(dev):
     assert kv.device_error() == 0
     assert torch.equal(whole, kv.cache)
     kv.close()
+
+
+@pytest.mark.parametrize("lens,n_sink,n_window", [
+    ([3000], 4, 128),
+    ([100, 3000, 132, 500], 4, 128),     # short sequences: the packed range empties
+    ([2000], 0, 64),
+    ([700], 16, 0),
+])
+def test_decode_buffered_sink_and_window(dev, lens, n_sink, n_window):
+    """fp16 sink + recent window next to the packed cache (the README's
+    "withbuffer" setting): the packed positions [n_sink, len - n_window) and
+    the buffered rows under one softmax, against the oracle on identical
+    caches."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], batch=len(lens), seq_len=max(lens), n_kv_heads=2, n_q_heads=8, n_calib=64)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    ocfg = oracle_config(cfg)
+    widths = model.allocate(ocfg, cq.numpy(), ck.numpy())
+    kv.set_allocation(widths.astype(np.int8))
+    tb = model.Tables(ocfg, widths)
+    n_buf = n_sink + n_window
+    B, H, g = len(lens), cfg.n_kv_heads, cfg.group_size
+    buf_k = torch.zeros((1, B, n_buf, H, 128), dtype=torch.float16)
+    buf_v = torch.zeros_like(buf_k)
+    lo, hi, cnt, encs = [], [], [], {}
+    for b, ln in enumerate(lens):
+        k = wl.keys(w, 0, b, 0, ln)
+        v = wl.values(w, 0, b, 0, ln)
+        l0 = min(n_sink, ln)
+        h1 = max(l0, ln - n_window)
+        rows = np.r_[0:l0, h1:ln]
+        lo.append(l0)
+        hi.append(h1)
+        cnt.append(len(rows))
+        buf_k[0, b, :len(rows)] = k[rows]
+        buf_v[0, b, :len(rows)] = v[rows]
+        for h in range(H):
+            enc = model.encode_rows(tb, 0, h, k[:, h].numpy(), v[:, h].numpy())
+            encs[b, h] = (enc, k[rows, h].numpy(), v[rows, h].numpy())
+            upload_oracle_rows(kv, 0, b, h, enc)
+    q = wl.decode_query(w, 0, lens)
+    out = torch.full((1, B, cfg.n_q_heads, 128), float("nan"), dtype=torch.float16, device=dev)
+    kv.decode_attn_buffered(0, q[None].to(dev), torch.tensor(hi, dtype=torch.int32, device=dev),
+                            torch.tensor(lo, dtype=torch.int32, device=dev), buf_k.to(dev), buf_v.to(dev),
+                            torch.tensor(cnt, dtype=torch.int32, device=dev), out)
+    torch.cuda.synchronize()
+    assert kv.device_error() == 0
+    got = out[0].float().cpu().numpy()
+    for (b, h), (enc, bk, bv) in encs.items():
+        ref = model.decode_buffered(tb, 0, h, q[b, h * g:(h + 1) * g].numpy(), enc["k_tiles"], enc["k_norms"],
+                                    enc["v_tiles"], enc["v_norm"], lo[b], hi[b], bk, bv)
+        err = row_rel_err(got[b, h * g:(h + 1) * g], ref)
+        assert np.all(err <= REL_TOL), (b, h, lens[b], err)
+    kv.close()
+
+
+def test_decode_buffered_without_buffer_rows_equals_decode(dev):
+    w = wl.scaled(wl.WORKLOADS["tiny"], batch=2, seq_len=2000, n_calib=64)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    kv.allocate(cq.to(dev), ck.to(dev))
+    lens = [2000, 1500]
+    for b, ln in enumerate(lens):
+        k = torch.zeros((1, 2, ln, 1, 128), dtype=torch.float16)
+        v = torch.zeros_like(k)
+        k[0, b] = wl.keys(w, 0, b, 0, ln)
+        v[0, b] = wl.values(w, 0, b, 0, ln)
+        start = torch.zeros(2, dtype=torch.int32, device=dev)
+        count = torch.zeros(2, dtype=torch.int32, device=dev)
+        count[b] = ln
+        kv.encode_append(0, k.to(dev), v.to(dev), start, count)
+    q = wl.decode_query(w, 0, lens)[None].to(dev)
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    a = torch.empty((1, 2, 4, 128), dtype=torch.float16, device=dev)
+    kv.decode_attn(0, q, seq, a)
+    bb = torch.empty_like(a)
+    z = torch.zeros(2, dtype=torch.int32, device=dev)
+    buf = torch.zeros((1, 2, 8, 1, 128), dtype=torch.float16, device=dev)
+    kv.decode_attn_buffered(0, q, seq, z, buf, buf, z, bb)
+    torch.cuda.synchronize()
+    assert kv.device_error() == 0
+    assert np.all(row_rel_err(bb[0].float().cpu().numpy(), a[0].float().cpu().numpy()) <= 1e-3)
+    kv.close()

@@ -412,6 +412,36 @@ def main():
     ms_multi = max_over_ranks(ms_multi)
     del g_multi
 
+    # ---- the same step with an fp16 sink + recent window (the README's
+    # "withbuffer" setting): packed positions [sink, len - window) plus the
+    # buffered rows ----
+    SINK, WINDOW = 4, 128
+    lo_b = [min(SINK, n) for n in lens]
+    hi_b = [max(lo_b[b], lens[b] - WINDOW) for b in range(B)]
+    n_buf = SINK + WINDOW
+    buf_k = torch.zeros((L, B, n_buf, H, 128), dtype=torch.float16, device=dev)
+    buf_v = torch.zeros_like(buf_k)
+    for l in range(L):
+        for b in range(B):
+            rows = list(range(lo_b[b])) + list(range(hi_b[b], lens[b]))
+            for j, r in enumerate(rows):
+                buf_k[l, b, j] = wl.keys(w, l, b, r, 1, device=dev)[0]
+                buf_v[l, b, j] = wl.values(w, l, b, r, 1, device=dev)[0]
+    buf_cnt = torch.tensor([lo_b[b] + lens[b] - hi_b[b] for b in range(B)], dtype=torch.int32, device=dev)
+    seq_hi = torch.tensor(hi_b, dtype=torch.int32, device=dev)
+    seq_lo = torch.tensor(lo_b, dtype=torch.int32, device=dev)
+
+    def step_buffered():
+        for l in range(L):
+            kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
+            kv.decode_attn_buffered(l, q_all[l:l + 1], seq_hi, seq_lo, buf_k[l:l + 1], buf_v[l:l + 1], buf_cnt,
+                                    out[l:l + 1])
+
+    ms_buf, g_buf, _ = time_graph(step_buffered, args.steps, args.warmup)
+    ms_buf = max_over_ranks(ms_buf)
+    del g_buf, buf_k, buf_v
+    assert kv.device_error() == 0, "device error in the buffered step"
+
     # ---- the split-K kernel alone: events around each per-layer launch, in a
     # captured step (the event nodes keep the split kernel from overlapping
     # its neighbours, so each interval is that kernel's whole duration) ----
@@ -536,6 +566,8 @@ def main():
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * L * args.steps,
         "clocks": clocks,
+        "buffered": {"ms_per_step": ms_buf, "tokens_per_s": world * B / (ms_buf * 1e-3), "sink": SINK,
+                     "window": WINDOW, "note": "fp16 sink + recent window next to the packed cache"},
         "multi_layer": {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
                         "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},
         "fp16_baseline": fp16,

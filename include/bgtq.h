@@ -216,10 +216,12 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
  *   d_pos_lo     int32 [batch]  start of the packed range, 0..seq_lens[b]
  *   d_buf_k/v    fp16 [layer_count][batch][n_buf][n_kv_heads][128]
  *   d_buf_count  int32 [batch]  buffered rows used, 0..n_buf
- *   n_buf        1..2048
+ *   n_buf        1..1024 (BGTQ_ERR_INVALID_ARG outside)
  * An empty packed range and no buffered row give 0.  Out-of-range
- * lengths set BGTQ_DEVERR_SEQ_LEN and are clamped.  Uses the workspace like
- * bgtq_decode_attn.  ASYNC. */
+ * lengths set BGTQ_DEVERR_SEQ_LEN and are clamped.  The buffered rows of a
+ * (sequence, KV head) are attended by one more CTA of the split pass,
+ * beside the packed ones.  Uses the workspace like bgtq_decode_attn.
+ * ASYNC. */
 int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                               const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
                               const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,

@@ -240,11 +240,11 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
 // Split-K partials per (layer, sequence, KV head, head block): one wave of
 // resident decode CTAs over all such units (the CTAs of a unit share its
 // tiles round-robin), at most max_splits and one per 4 tiles of capacity.
-int auto_splits(bgtq_state* st, int units) {
+int auto_splits(bgtq_state* st, int units, int extra) {
   if (st->ctas_per_sm <= 0) st->ctas_per_sm = std::max(1, bgtq::decode_ctas_per_sm(st->shape));
   const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
   const int64_t slots = int64_t(st->ctas_per_sm) * st->num_sms;
-  int64_t n = slots / std::max(units, 1);
+  int64_t n = slots / std::max(units, 1) - extra;  // extra CTAs per unit share the wave
   n = std::min<int64_t>(n, max_splits_of(&st->cfg));
   n = std::min<int64_t>(n, (tiles + 3) / 4);
   return static_cast<int>(std::max<int64_t>(n, 1));
@@ -509,12 +509,13 @@ int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, 
 }
 
 // Number of split-K partials per unit for a call (see auto_splits); a set
-// split size t gives ceil(capacity / t).
-int split_for(bgtq_state* st, int32_t layer_count, int32_t batch) {
+// split size t gives ceil(capacity / t).  `extra` = CTAs per unit the split
+// pass launches beside the splits (the buffer CTA of a buffered call).
+int split_for(bgtq_state* st, int32_t layer_count, int32_t batch, int extra = 0) {
   const int head_blocks = (st->shape.group + 7) / 8;
   if (st->split_tokens > 0)
     return static_cast<int>((st->cfg.capacity_tokens + st->split_tokens - 1) / st->split_tokens);
-  return auto_splits(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count);
+  return auto_splits(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count, extra);
 }
 
 }  // namespace
@@ -525,7 +526,7 @@ int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const 
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_qrot) || !aligned16(d_seq_lens)) return BGTQ_ERR_ALIGNMENT;
-  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, nullptr, batch,
+  return bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, d_qrot, d_seq_lens, bgtq::BufferArgs{}, batch,
                                    split_for(st, layer_count, batch), as_stream(stream)) == cudaSuccess
              ? BGTQ_OK
              : BGTQ_ERR_CUDA;
@@ -555,7 +556,7 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, nullptr, batch,
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, bgtq::BufferArgs{}, batch,
                                 split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split, bgtq::BufferArgs{},
@@ -575,7 +576,7 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_pos_lo) || !aligned16(d_buf_k) ||
       !aligned16(d_buf_v) || !aligned16(d_buf_count) || !aligned16(d_out))
     return BGTQ_ERR_ALIGNMENT;
-  const int split = split_for(st, layer_count, batch);
+  const int split = split_for(st, layer_count, batch, 1);
   cudaStream_t s = as_stream(stream);
   bgtq::BufferArgs buf;
   buf.q = static_cast<const __half*>(d_q);
@@ -587,7 +588,7 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, d_pos_lo, batch,
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, buf, batch,
                                 split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split, buf,
@@ -667,7 +668,7 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   if (bgtq::launch_rotate_query(shape, ws, layer, layer_count, static_cast<const __half*>(d_q), batch, ws.qrot, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
-  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, nullptr, d_seq_lens, nullptr, batch, split, s) !=
+  if (bgtq::launch_decode_split(shape, ws, st->cache, layer, layer_count, nullptr, d_seq_lens, bgtq::BufferArgs{}, batch, split, s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_combine(shape, ws, layer, layer_count, d_seq_lens, batch, split, bgtq::BufferArgs{},

@@ -12,7 +12,7 @@ constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
 constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
 constexpr int kPartialStride = 132;
 constexpr int kCombSlices = 8;       // CTAs merging one row's splits in the combine
-constexpr int kMaxBufferRows = 2048; // fp16 buffered rows per sequence a decode call may attend   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kMaxBufferRows = 1024; // fp16 buffered rows per sequence a decode call may attend   // floats per split-K partial: m, l, pad, pad, acc[128]
 constexpr int kTile = 64;             // cache positions per packed tile
 constexpr int kSplitGranule = kTile;  // split sizes are multiples of the tile
 constexpr int kMaxChunks = 12;        // 16-coordinate K chunks per head (8 + one partial per group)
@@ -107,12 +107,6 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
 // The split pass reads q~ as fragments from ws.qfrag (written by the query
 // rotation), or, when qrot is not null, builds them from qrot itself.
-// pos_lo (int32 [batch], may be null = 0): the first packed position attended.
-cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo,
-                                int batch, int n_splits, cudaStream_t stream);
-// Resident split-decode CTAs per SM for a config (0 on error).
-int decode_ctas_per_sm(const Shape& s);
 // The fp16 buffered rows a decode call attends besides the packed cache
 // (k == nullptr: none).  q: the decode query fp16 [layer_count][batch][Hq][128];
 // k, v: fp16 [layer_count][batch][n_buf][Hkv][128]; count: int32 [batch]
@@ -126,6 +120,14 @@ struct BufferArgs {
   const int32_t* pos_lo;
   int n_buf;
 };
+// The split pass over the packed positions [pos_lo, seq_lens) (buf.pos_lo;
+// null = 0); with buf.k set, one more CTA per unit attends the buffered rows
+// and posts them as the row's extra combine intermediate.
+cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const float* qrot, const int32_t* seq_lens, const BufferArgs& buf,
+                                int batch, int n_splits, cudaStream_t stream);
+// Resident split-decode CTAs per SM for a config (0 on error).
+int decode_ctas_per_sm(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream);

@@ -919,6 +919,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// Shared memory of the buffer CTA: q of 8 heads, logits / weights [8][rows], (M, L) per head.
+constexpr int kBufSmemBytes = (8 * kD + 8 * kMaxBufferRows + 16) * 4;
+
 struct DecodeLayout {  // byte offsets inside the dynamic shared memory
   int bars, bq, tabk, grp, pdesc, ms, ls, mres, wsc, stage, stage_bytes, total;
 };
@@ -940,7 +943,9 @@ __host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
   L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
   const int stages = kDecWarps * kStages * L.stage_bytes;
   const int merge = kDecWarps * 8 * kD * 4;  // reuses the stage buffers after the loop
-  L.total = L.stage + (stages > merge ? stages : merge);
+  int need = stages > merge ? stages : merge;
+  if (need < kBufSmemBytes) need = kBufSmemBytes;  // the buffer CTA of a buffered call
+  L.total = L.stage + need;
   return L;
 }
 
@@ -1008,11 +1013,161 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
 // ctas_per_unit), so every warp gets the same number of tiles to within one.
 // Each CTA writes one partial (m, l, acc) per query head -- an empty one
 // (m = -inf, l = 0) when it has no tile.
+// The range of a decode call's sequence: the packed positions [lo, len) and
+// the buffered row count, clamped the same way by every kernel that reads
+// them (the combine raises the flag).
+struct SeqRange {
+  int len, lo, cnt;
+  bool bad;
+};
+
+__device__ __forceinline__ SeqRange seq_range(const Shape& sh, const int32_t* seq_lens, const BufferArgs& buf, int b) {
+  SeqRange r;
+  r.len = seq_lens[b];
+  r.lo = buf.pos_lo != nullptr ? buf.pos_lo[b] : 0;
+  r.cnt = buf.k != nullptr ? buf.count[b] : 0;
+  r.bad = r.len < 0 || r.len > sh.capacity || r.lo < 0 || r.lo > r.len || r.cnt < 0 || r.cnt > buf.n_buf;
+  if (r.len < 0 || r.len > sh.capacity) r.len = 0;
+  if (r.lo < 0 || r.lo > r.len) r.lo = r.len;
+  r.cnt = r.cnt < 0 ? 0 : (r.cnt > buf.n_buf ? buf.n_buf : r.cnt);
+  return r;
+}
+
+// The fp16 buffered rows of one (layer, sequence, KV head, block of 8 query
+// heads), attended by one extra CTA of the split pass (128 threads): logits
+// q . k / sqrt(D) in log2 units (a thread per row), softmax per head, P v (a
+// thread per dimension, unrotated).  Each head's (m, l, acc) goes to the
+// row's extra combine intermediate, which then counts as arrived.
+__device__ void buffer_attend(const Shape& sh, const Workspace& ws, const BufferArgs& buf, const SeqRange& sr, int li,
+                              int b, int h, int h0, int nh, int batch, unsigned char* smem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = sh.group;
+  float* qs = reinterpret_cast<float*>(smem);   // [128 dims][8 heads]
+  float* lg = qs + 8 * kD;                      // [8][kMaxBufferRows]
+  float* ml = lg + 8 * kMaxBufferRows;          // [8][2]
+  const int cnt = sr.cnt;
+  const size_t qrow = ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
+  for (int i = tid; i < 8 * kD; i += kDecThreads) {
+    const int hh = i / kD, dim = i % kD;
+    qs[dim * 8 + hh] = hh < nh ? __half2float(buf.q[qrow + i]) * (kInvSqrtD * kLog2e) : 0.f;
+  }
+  __syncthreads();
+  const size_t rstride = static_cast<size_t>(sh.n_kv_heads) * kD;
+  const size_t base = (static_cast<size_t>(li) * batch + b) * buf.n_buf * rstride + static_cast<size_t>(h) * kD;
+  for (int r = tid; r < cnt; r += kDecThreads) {
+    const uint4* kr = reinterpret_cast<const uint4*>(buf.k + base + r * rstride);
+    float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // half of the row's dimensions per pass: 8 loads of 8 values in flight
+#pragma unroll 1
+    for (int c8 = 0; c8 < 2; ++c8) {
+      uint4 kw[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) kw[c] = kr[8 * c8 + c];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const __half2* h2 = reinterpret_cast<const __half2*>(&kw[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float kv = e & 1 ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
+          const float4* qa = reinterpret_cast<const float4*>(qs + (8 * (8 * c8 + c) + e) * 8);
+          const float4 a0 = qa[0], a1 = qa[1];
+          d[0] = fmaf(a0.x, kv, d[0]);
+          d[1] = fmaf(a0.y, kv, d[1]);
+          d[2] = fmaf(a0.z, kv, d[2]);
+          d[3] = fmaf(a0.w, kv, d[3]);
+          d[4] = fmaf(a1.x, kv, d[4]);
+          d[5] = fmaf(a1.y, kv, d[5]);
+          d[6] = fmaf(a1.z, kv, d[6]);
+          d[7] = fmaf(a1.w, kv, d[7]);
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) lg[hh * kMaxBufferRows + r] = d[hh];
+  }
+  __syncthreads();
+  // per head: maximum, weights 2^(logit - M) in place, denominator
+  for (int hh = warp; hh < 8; hh += kDecWarps) {
+    float M = -CUDART_INF_F;
+    for (int r = lane; r < cnt; r += 32) M = fmaxf(M, lg[hh * kMaxBufferRows + r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int r = lane; r < cnt; r += 32) {
+      const float p = exp2f(lg[hh * kMaxBufferRows + r] - M);
+      lg[hh * kMaxBufferRows + r] = p;
+      L += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      ml[2 * hh] = M;
+      ml[2 * hh + 1] = L;
+    }
+  }
+  __syncthreads();
+  // P v: thread (8 dimensions dg, row phase rp of 8), 8 values per load; the
+  // phases are then summed through shared memory (over the weights)
+  const int dg = tid & 15, rp = tid >> 4;
+  float acc[8][8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+#pragma unroll 4
+  for (int r = rp; r < cnt; r += 8) {
+    const uint4 vw = *reinterpret_cast<const uint4*>(buf.v + base + r * rstride + 8 * dg);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&vw);
+    float vv[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      vv[2 * e] = f.x;
+      vv[2 * e + 1] = f.y;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      const float p = lg[hh * kMaxBufferRows + r];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vv[e], acc[hh][e]);
+    }
+  }
+  __syncthreads();
+  float* red = lg;  // [8 phases][8 heads][128 dims]
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    float4* dst = reinterpret_cast<float4*>(red + (rp * 8 + hh) * kD + 8 * dg);
+    dst[0] = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+    dst[1] = make_float4(acc[hh][4], acc[hh][5], acc[hh][6], acc[hh][7]);
+  }
+  __syncthreads();
+  const int d = tid;  // kDecThreads == kD: a thread per output dimension
+  const size_t wrow0 = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0;
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    if (hh >= nh) break;
+    float* mid = ws.comb_mid + ((wrow0 + hh) * (kCombSlices + 1) + kCombSlices) * kPartialStride;
+    float a = 0.f;
+#pragma unroll
+    for (int ph = 0; ph < 8; ++ph) a += red[(ph * 8 + hh) * kD + d];
+    mid[4 + d] = cnt > 0 ? a : 0.f;
+    if (d == 0) {
+      mid[0] = cnt > 0 ? ml[2 * hh] : -CUDART_INF_F;
+      mid[1] = cnt > 0 ? ml[2 * hh + 1] : 0.f;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  // the combine of a row with no packed position and no buffered row writes
+  // zeros without counting arrivals: do not count this one either
+  if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
+}
+
 template <int VB>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
-                      const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ pos_lo, int batch,
-                      int ctas_per_unit, int head_blocks) {
+                      const int32_t* __restrict__ seq_lens, BufferArgs buf, int batch, int ctas_per_unit,
+                      int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const DecodeLayout DL = decode_layout(sh.kbits, VB);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
@@ -1053,12 +1208,17 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // sequence lengths, rotated queries and cache are read after that kernel
   // has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  int len = seq_lens[b];
-  if (len < 0 || len > sh.capacity) len = 0;  // flagged by the combine kernel
   // the packed positions attended: [lo, len); lo > 0 when the caller keeps the
-  // first positions unquantised (their rows come through the combine)
-  int lo = pos_lo != nullptr ? pos_lo[b] : 0;
-  if (lo < 0 || lo > len) lo = len;            // flagged by the combine kernel
+  // first positions unquantised (out-of-range values are flagged by the
+  // combine kernel)
+  const SeqRange sr = seq_range(sh, seq_lens, buf, b);
+  if (cu == ctas_per_unit) {
+    // the extra CTA of a buffered call: the unit's fp16 buffered rows
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    buffer_attend(sh, ws, buf, sr, li, b, h, h0, nh, batch, smem_raw + DL.stage);
+    return;
+  }
+  const int len = sr.len, lo = sr.lo;
   const int tlo = lo / kTile;
   const int ntl = lo < len ? (len + kTile - 1) / kTile - tlo : 0;
   const int W = ctas_per_unit * kDecWarps;
@@ -1353,14 +1513,13 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq * nsl),
-// 256 threads, nsl = kCombSlices, plus one when an fp16 buffer is attended.
-// Each of the first kCombSlices CTAs of a row merges one slice of the row's
-// splits (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated
-// coordinates) into an intermediate (m, l, acc) in V's rotated basis; the
-// buffer CTA attends the row's fp16 buffered rows directly (logits q . k /
-// sqrt(D) in log2 units, acc = sum p v unrotated).  The row's last CTA to
-// finish (an arrival counter, reset by that CTA) merges them:
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq *
+// kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
+// (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated coordinates) into
+// an intermediate (m, l, acc) in V's rotated basis.  In a buffered call the
+// split pass has already posted the row's fp16 buffered rows as one more
+// intermediate (acc unrotated).  The row's last CTA to finish (an arrival
+// counter, reset by that CTA) merges them:
 // o = (R_V^T sum_s w_s acc_s + w_buf acc_buf) / (sum_s w_s l_s + w_buf l_buf).
 // ---------------------------------------------------------------------------
 constexpr int kCombThreads = 256;
@@ -1369,9 +1528,9 @@ constexpr int kCombWarps = kCombThreads / 32;
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
                                                                int n_splits, BufferArgs buf, __half* __restrict__ out) {
-  const int nsl = kCombSlices + (buf.k != nullptr ? 1 : 0);
-  const int slice = blockIdx.x % nsl;
-  const int rowi = blockIdx.x / nsl;
+  const int has_buf = buf.k != nullptr ? 1 : 0;
+  const int slice = blockIdx.x % kCombSlices;
+  const int rowi = blockIdx.x / kCombSlices;
   const int hq = rowi % sh.n_q_heads;
   const int b = (rowi / sh.n_q_heads) % batch;
   const int li = rowi / (sh.n_q_heads * batch);
@@ -1383,17 +1542,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   // Launched as a programmatic dependent of the split pass: inputs, partials
   // and the output are touched only after that kernel has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  int len = seq_lens[b];
-  int lo = buf.pos_lo != nullptr ? buf.pos_lo[b] : 0;
-  int cnt = buf.k != nullptr ? buf.count[b] : 0;
-  if (len < 0 || len > sh.capacity || lo < 0 || lo > len || cnt < 0 || cnt > buf.n_buf) {
-    if (tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
-    if (len < 0 || len > sh.capacity) len = 0;
-    if (lo < 0 || lo > len) lo = len;
-    cnt = cnt < 0 ? 0 : (cnt > buf.n_buf ? buf.n_buf : cnt);
-  }
+  const SeqRange sr = seq_range(sh, seq_lens, buf, b);
+  if (sr.bad && tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  if (lo >= len && cnt == 0) {
+  if (sr.lo >= sr.len && sr.cnt == 0) {
     if (slice == 0 && tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
   }
@@ -1403,116 +1555,64 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   __shared__ float accs[kCombWarps][kD];
   __shared__ float lsw[kCombWarps];
   __shared__ float a_s[kD];
-  __shared__ float lgb[kMaxBufferRows];
   __shared__ int last;
   float* mid = ws.comb_mid + (wrow * (kCombSlices + 1) + slice) * kPartialStride;
-  if (slice < kCombSlices) {
-    // ---- one slice of the row's splits ----
-    const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
-    const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
-    float M = -CUDART_INF_F;
-    for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
+  // ---- one slice of the row's splits ----
+  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
+  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
+  float M = -CUDART_INF_F;
+  for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = red[0];
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
 #pragma unroll
-    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.f;
+  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
 #pragma unroll 4
-    for (int s = s0 + warp; s < s1; s += kCombWarps) {
-      const float* p = part + static_cast<size_t>(s) * kPartialStride;
-      const float ms = p[0];
-      const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-      lsum = fmaf(wgt, p[1], lsum);
-      const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
-      acc.x = fmaf(wgt, a.x, acc.x);
-      acc.y = fmaf(wgt, a.y, acc.y);
-      acc.z = fmaf(wgt, a.z, acc.z);
-      acc.w = fmaf(wgt, a.w, acc.w);
-    }
-    *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
-    if (lane == 0) lsw[warp] = lsum;
-    __syncthreads();
-    if (tid < kD) {
-      float a = 0.f;
+  for (int s = s0 + warp; s < s1; s += kCombWarps) {
+    const float* p = part + static_cast<size_t>(s) * kPartialStride;
+    const float ms = p[0];
+    const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+    lsum = fmaf(wgt, p[1], lsum);
+    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+    acc.x = fmaf(wgt, a.x, acc.x);
+    acc.y = fmaf(wgt, a.y, acc.y);
+    acc.z = fmaf(wgt, a.z, acc.z);
+    acc.w = fmaf(wgt, a.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
+  if (lane == 0) lsw[warp] = lsum;
+  __syncthreads();
+  if (tid < kD) {
+    float a = 0.f;
 #pragma unroll
-      for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
-      mid[4 + tid] = a;
-    }
-    if (tid == 0) {
-      float l = 0.f;
+    for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
+    mid[4 + tid] = a;
+  }
+  if (tid == 0) {
+    float l = 0.f;
 #pragma unroll
-      for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
-      mid[0] = M;
-      mid[1] = l;
-    }
-  } else {
-    // ---- the fp16 buffered rows of the row's KV head ----
-    const __half* qv = buf.q + row * kD;
-    const float qs = kInvSqrtD * kLog2e;
-    const float4 q4 = make_float4(__half2float(qv[4 * lane]) * qs, __half2float(qv[4 * lane + 1]) * qs,
-                                  __half2float(qv[4 * lane + 2]) * qs, __half2float(qv[4 * lane + 3]) * qs);
-    const size_t rstride = static_cast<size_t>(sh.n_kv_heads) * kD;
-    const size_t base = (static_cast<size_t>(li) * batch + b) * buf.n_buf * rstride + static_cast<size_t>(kvh) * kD;
-    for (int r = warp; r < cnt; r += kCombWarps) {
-      const uint2 kw = *reinterpret_cast<const uint2*>(buf.k + base + r * rstride + 4 * lane);
-      const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
-      const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
-      float d = q4.x * k01.x;
-      d = fmaf(q4.y, k01.y, d);
-      d = fmaf(q4.z, k23.x, d);
-      d = fmaf(q4.w, k23.y, d);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      if (lane == 0) lgb[r] = d;
-    }
-    __syncthreads();
-    float M = -CUDART_INF_F;
-    for (int r = tid; r < cnt; r += kCombThreads) M = fmaxf(M, lgb[r]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = red[0];
-#pragma unroll
-    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-    // P v over the rows: thread (dimension d, half of the rows)
-    const int d = tid & (kD - 1), hr = tid >> 7;
-    float acc = 0.f, lsum = 0.f;
-    for (int r = hr; r < cnt; r += 2) {
-      const float p = exp2f(lgb[r] - M);
-      lsum += p;
-      acc = fmaf(p, __half2float(buf.v[base + r * rstride + d]), acc);
-    }
-    if (hr == 1) {
-      accs[0][d] = acc;
-      if (d == 0) lsw[0] = lsum;
-    }
-    __syncthreads();
-    if (hr == 0) {
-      mid[4 + d] = cnt > 0 ? acc + accs[0][d] : 0.f;
-      if (d == 0) {
-        mid[0] = cnt > 0 ? M : -CUDART_INF_F;
-        mid[1] = cnt > 0 ? lsum + lsw[0] : 0.f;
-      }
-    }
+    for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
+    mid[0] = M;
+    mid[1] = l;
   }
   // ---- the row's last CTA merges the intermediates ----
+  const int nmid = kCombSlices + has_buf;
   __threadfence();
   __syncthreads();
-  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == static_cast<unsigned>(nsl - 1);
+  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == static_cast<unsigned>(nmid - 1);
   __syncthreads();
   if (!last) return;
   __threadfence();
   const float* mids = ws.comb_mid + wrow * (kCombSlices + 1) * kPartialStride;
   float Mt = -CUDART_INF_F;
-  for (int k = 0; k < nsl; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
+  for (int k = 0; k < nmid; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
   float Lt = 0.f, at = 0.f, ab = 0.f;
   const int dd = tid & (kD - 1);
-  for (int k = 0; k < nsl; ++k) {
+  for (int k = 0; k < nmid; ++k) {
     const float mk = __ldcg(mids + k * kPartialStride);
     const float w = mk == -CUDART_INF_F ? 0.f : exp2f(mk - Mt);
     Lt = fmaf(w, __ldcg(mids + k * kPartialStride + 1), Lt);
@@ -1574,15 +1674,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
-                             const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo, int batch,
+                             const float* qrot, const int32_t* seq_lens, const BufferArgs& buf, int batch,
                              int n_splits, cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
   static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
-  dim3 grid(n_splits, batch * s.n_kv_heads * head_blocks, layer_count);
+  dim3 grid(n_splits + (buf.k != nullptr ? 1 : 0), batch * s.n_kv_heads * head_blocks, layer_count);
   return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, qrot, seq_lens, pos_lo, batch, n_splits, head_blocks);
+                          ws, cache, layer0, qrot, seq_lens, buf, batch, n_splits, head_blocks);
 }
 
 template <int VB>
@@ -1640,24 +1740,20 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 }
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
-                                int layer_count, const float* qrot, const int32_t* seq_lens, const int32_t* pos_lo,
+                                int layer_count, const float* qrot, const int32_t* seq_lens, const BufferArgs& buf,
                                 int batch, int n_splits, cudaStream_t stream) {
   switch (s.vbits) {
-    case 1:
-      return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
-    case 2:
-      return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
-    case 3:
-      return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
-    default:
-      return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, pos_lo, batch, n_splits, stream);
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
   }
 }
 
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream) {
-  const int nsl = kCombSlices + (buf.k != nullptr ? 1 : 0);
+  const int nsl = kCombSlices;  // the buffered rows, if any, come from the split pass
   return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads * nsl), dim3(kCombThreads), 0, stream,
                           s, ws, layer0, seq_lens, batch, n_splits, buf, out);
 }

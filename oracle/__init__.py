@@ -22,4 +22,5 @@ allocate    greedy integer bit allocation by marginal gain; group layout.
 tqmse       rotate / normalise / quantise one row; bit-pack a record.
 attention   dense decode attention from packed records.
 model       the per-(layer, KV head) tables and the cache-level calls.
+diag        the per-layer logit MAE of a packed key cache (K only).
 """

@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=0, help="use only the first N layers (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp16-baseline", action="store_true")
+    ap.add_argument("--no-diag", action="store_true", help="skip the per-layer logit-MAE diagnostic")
     return ap.parse_args()
 
 
@@ -542,6 +543,42 @@ def main():
             fp16 = {"impl": name, "error": str(e)[:200]}
         del kf, vf
 
+    # ---- per-layer logit MAE (K only): Block-GTQ against uniform TQ-MSE at
+    # the same average width, over a 1024-position window of sequence 0 ----
+    diag = None
+    if not args.no_diag:
+        M = min(1024, lens[0])
+        qd = torch.stack([wl.queries(w, l, 0, torch.arange(M), tag=3, device=dev) for l in range(L)])
+        kd = torch.stack([wl.keys(w, l, 0, 0, M, device=dev) for l in range(L)])
+        mae_g = torch.zeros((L, HQ), dtype=torch.float64, device=dev)
+        kv.logit_mae(0, 0, 0, qd, kd, mae_g, layer_count=L)
+        torch.cuda.synchronize()
+        e0.record()
+        kv.logit_mae(0, 0, 0, qd, kd, mae_g, layer_count=L)
+        e1.record()
+        torch.cuda.synchronize()
+        diag_ms = e0.elapsed_time(e1)
+        ucfg = bgtq.Config(**dict(wl.bench_config_fields(w), capacity_tokens=M, max_batch=1))
+        kvu = bgtq.PackedKVCache(ucfg, dev)
+        kvu.set_allocation(np.full((L, H, 64), w.k_bits, dtype=np.int8))
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        cnt = torch.full((1,), M, dtype=torch.int32, device=dev)
+        kvu.encode_append(0, kd[:, None], kd[:, None], zero, cnt, layer_count=L)
+        mae_u = torch.zeros((L, HQ), dtype=torch.float64, device=dev)
+        kvu.logit_mae(0, 0, 0, qd, kd, mae_u, layer_count=L)
+        torch.cuda.synchronize()
+        assert kv.device_error() == 0 and kvu.device_error() == 0, "device error in the logit-MAE diagnostic"
+        kvu.close()
+        g_l = mae_g.mean(dim=1).cpu().numpy()
+        u_l = mae_u.mean(dim=1).cpu().numpy()
+        diag = {"window": M, "pairs_per_head": M * (M + 1) // 2, "block_gtq_mean": float(g_l.mean()),
+                "tq_mse_mean": float(u_l.mean()), "reduction": float(1 - g_l.mean() / u_l.mean()),
+                "wins": f"{int((g_l < u_l).sum())}/{L}", "ms_all_layers": diag_ms,
+                "per_layer_block_gtq": [round(float(x), 5) for x in g_l],
+                "per_layer_tq_mse": [round(float(x), 5) for x in u_l],
+                "note": "K-only logit MAE (q.k / sqrt(128)) over causal pairs, synthetic Q/K"}
+        del qd, kd
+
     # ---- CPU oracle on a bounded sample ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -571,6 +608,7 @@ def main():
         "multi_layer": {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
                         "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},
         "fp16_baseline": fp16,
+        "logit_mae": diag,
         "cpu_baseline": cpu,
         "allocate_ms": alloc_ms,
         "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),

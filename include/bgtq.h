@@ -227,6 +227,29 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
                               const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,
                               void* stream);
 
+/* Per-layer logit MAE of the packed keys: the Block-GTQ abstract's logit
+ * fidelity diagnostic and the blockgtq README's per-layer kernel MAE
+ * (bit allocation section, `--window-M 1024`), comparing Block-GTQ with
+ * uniform TQ-MSE at the same average width (two states, one allocated and
+ * one with bgtq_set_allocation, holding the same keys).  Only K is
+ * involved.  Over a window of m cached positions w0 .. w0+m-1 of sequence
+ * seq, with the queries at the same positions, for every causal pair
+ * (query i, key j), 0 <= j <= i < m, and each query head h:
+ *   d_mae[l][h] = mean |q_{i,h} . k_hat_j - q_{i,h} . k_j| / sqrt(128)
+ * where q . k_hat is the logit exactly as the decode computes it from the
+ * packed cache and k the exact key.  A layer's MAE is the mean over its
+ * heads.
+ *   d_q    fp16 [layer_count][m][n_q_heads][128]   queries (post-RoPE)
+ *   d_k    fp16 [layer_count][m][n_kv_heads][128]  the exact keys the cache
+ *          holds (encoded) at positions w0 .. w0+m-1 of sequence seq
+ *   d_mae  double [layer_count][n_q_heads], written by the call
+ * 0 <= seq < max_batch, m >= 1, w0 >= 0, w0 + m <= capacity_tokens,
+ * else BGTQ_ERR_INVALID_ARG.  The per-head sums use fp64 atomics, so the
+ * last bits can vary between runs.  Does not touch the workspace's decode
+ * scratch.  ASYNC. */
+int bgtq_logit_mae(bgtq_state* st, int32_t layer, int32_t layer_count, int32_t seq, int32_t w0, int32_t m,
+                   const void* d_q, const void* d_k, double* d_mae, void* stream);
+
 /* The two stages of bgtq_decode_attn after bgtq_rotate_query, for callers
  * that time or schedule them separately (same arguments and results):
  * bgtq_decode_split runs the split-K pass over the packed cache from the

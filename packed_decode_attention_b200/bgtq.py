@@ -100,6 +100,7 @@ _SIGS = {
     "bgtq_rotate_query": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
+    "bgtq_logit_mae": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
@@ -247,6 +248,11 @@ def bgtq_decode_attn_buffered(state, layer, layer_count, d_q, d_seq_lens, d_pos_
                                            _ptr(d_out), _stream(stream)))
 
 
+def bgtq_logit_mae(state, layer, layer_count, seq, w0, m, d_q, d_k, d_mae, stream=None):
+    _check(lib().bgtq_logit_mae(state, layer, layer_count, seq, w0, m, _ptr(d_q), _ptr(d_k), _ptr(d_mae),
+                                _stream(stream)))
+
+
 def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
     _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
 
@@ -354,6 +360,12 @@ class PackedKVCache:
         n_buf, Hkv, 128])."""
         bgtq_decode_attn_buffered(self.state, layer, layer_count, q, seq_lens, pos_lo, q.shape[1], buf_k, buf_v,
                                   buf_count, buf_k.shape[2], out)
+
+    def logit_mae(self, layer, seq, w0, q, k, out, layer_count=1):
+        """Per-head logit MAE of the packed keys at positions [w0, w0 + m) of
+        sequence seq: q fp16 [layer_count, m, Hq, 128], k (exact keys) fp16
+        [layer_count, m, Hkv, 128], out float64 [layer_count, Hq]."""
+        bgtq_logit_mae(self.state, layer, layer_count, seq, w0, q.shape[1], q, k, out)
 
     def decode_split(self, layer, qrot, seq_lens, layer_count=1):
         """The split-K stage alone from rotated queries (fp32 [layer_count, batch, Hq, 128])."""

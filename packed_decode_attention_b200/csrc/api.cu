@@ -597,6 +597,21 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
   return BGTQ_OK;
 }
 
+int bgtq_logit_mae(bgtq_state* st, int32_t layer, int32_t layer_count, int32_t seq, int32_t w0, int32_t m,
+                   const void* d_q, const void* d_k, double* d_mae, void* stream) {
+  if (!st || !d_q || !d_k || !d_mae) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, 1);
+  if (v != BGTQ_OK) return v;
+  if (seq < 0 || seq >= st->cfg.max_batch || m < 1 || w0 < 0 || int64_t(w0) + m > st->cfg.capacity_tokens)
+    return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_mae)) return BGTQ_ERR_ALIGNMENT;
+  return bgtq::launch_logit_mae(st->shape, st->ws, st->cache, layer, layer_count, seq, w0, m,
+                                static_cast<const __half*>(d_q), static_cast<const __half*>(d_k), d_mae,
+                                as_stream(stream)) == cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Static-scratch decode: the split-K scratch lives in this library's own
 // device array instead of the caller's workspace.

@@ -10,9 +10,9 @@ namespace bgtq {
 constexpr int kD = 128;               // head_dim
 constexpr int kNumGroupsMax = 4;      // widths 4, 3, 2, 1
 constexpr int kEnergyChunks = 32;     // calibration rows split into this many CTAs
-constexpr int kPartialStride = 132;
-constexpr int kCombSlices = 8;       // CTAs merging one row's splits in the combine
-constexpr int kMaxBufferRows = 1024; // fp16 buffered rows per sequence a decode call may attend   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kPartialStride = 132;   // floats per split-K partial: m, l, pad, pad, acc[128]
+constexpr int kCombSlices = 8;        // CTAs merging one row's splits in the combine
+constexpr int kMaxBufferRows = 1024;  // fp16 buffered rows per sequence a decode call may attend
 constexpr int kTile = 64;             // cache positions per packed tile
 constexpr int kSplitGranule = kTile;  // split sizes are multiples of the tile
 constexpr int kMaxChunks = 12;        // 16-coordinate K chunks per head (8 + one partial per group)
@@ -131,5 +131,13 @@ int decode_ctas_per_sm(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream);
+// Per-layer logit MAE of the packed keys of sequence seq at cache positions
+// [w0, w0 + m) against the exact keys k (fp16 [layer_count][m][Hkv][128]),
+// for the queries q (fp16 [layer_count][m][Hq][128]) at the same positions
+// and every causal pair; mae: double [layer_count][Hq] (zeroed, summed and
+// scaled by the launches).
+cudaError_t launch_logit_mae(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                             int layer_count, int seq, int w0, int m, const __half* q, const __half* k, double* mae,
+                             cudaStream_t stream);
 
 }  // namespace bgtq

@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp16-baseline", action="store_true")
     ap.add_argument("--no-diag", action="store_true", help="skip the per-layer logit-MAE diagnostic")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache step")
     return ap.parse_args()
 
 
@@ -443,6 +444,52 @@ def main():
     del g_buf, buf_k, buf_v
     assert kv.device_error() == 0, "device error in the buffered step"
 
+    # ---- the same step over a paged copy of the cache: a tight pool of
+    # 64-position pages, shuffled over the sequences' tiles ----
+    paged = None
+    if not args.no_paged:
+        T = (cap + 63) // 64
+        need = [(n + 63) // 64 for n in lens]
+        pool = sum(need)
+        ids = torch.randperm(pool, generator=torch.Generator().manual_seed(7)).to(torch.int32)
+        table = torch.full((B, T), -1, dtype=torch.int32)
+        k0 = 0
+        for b in range(B):
+            table[b, :need[b]] = ids[k0:k0 + need[b]]
+            k0 += need[b]
+        bt = table.to(dev)
+        kvp = bgtq.PackedKVCache(bgtq.Config(**dict(wl.bench_config_fields(w), page_pool_tiles=pool)), dev)
+        kvp.set_block_table(bt)
+        kvp.set_allocation(kv.get_allocation())
+        for l in range(L):
+            for b in range(B):
+                pg = bt[b, :need[b]].long()
+                for h in range(H):
+                    kvp.k_tiles()[l, h][pg] = kv.k_tiles()[l, b, h, :need[b]]
+                    kvp.v_tiles()[l, h][pg] = kv.v_tiles()[l, b, h, :need[b]]
+                    kvp.k_norms()[l, h].view(pool, 64, 4)[pg] = kv.k_norms()[l, b, h, :need[b] * 64].view(-1, 64, 4)
+                    kvp.v_norms()[l, h].view(pool, 64)[pg] = kv.v_norms()[l, b, h, :need[b] * 64].view(-1, 64)
+        out_p = torch.empty_like(out)
+
+        def step_paged():
+            for l in range(L):
+                kvp.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
+                kvp.decode_attn(l, q_all[l:l + 1], seq, out_p[l:l + 1])
+
+        ms_paged, g_p, _ = time_graph(step_paged, args.steps, args.warmup)
+        ms_paged = max_over_ranks(ms_paged)
+        del g_p
+        step()
+        step_paged()
+        torch.cuda.synchronize()
+        assert kvp.device_error() == 0, "device error in the paged step"
+        paged = {"ms_per_step": ms_paged, "tokens_per_s": world * B / (ms_paged * 1e-3), "pages": pool,
+                 "cache_bytes": kvp.cache_bytes, "contiguous_cache_bytes": kv.cache_bytes,
+                 "output_equal_to_contiguous": bool(torch.equal(out, out_p)),
+                 "note": "block-table indirection, pages shuffled over the sequences"}
+        kvp.close()
+        del kvp, out_p
+
     # ---- the split-K kernel alone: events around each per-layer launch, in a
     # captured step (the event nodes keep the split kernel from overlapping
     # its neighbours, so each interval is that kernel's whole duration) ----
@@ -609,6 +656,7 @@ def main():
                         "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},
         "fp16_baseline": fp16,
         "logit_mae": diag,
+        "paged": paged,
         "cpu_baseline": cpu,
         "allocate_ms": alloc_ms,
         "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),

@@ -42,6 +42,11 @@
  *              descending); unused slots 0
  *   V tiles    uint8 [L][B][H][T][1024*v_avg_bits]  same scheme, one group
  *   V norms    fp16  [L][B][H][T*64]
+ * Paged cache (page_pool_tiles = P > 0; PagedAttention's block table,
+ * cited by the blockgtq pages): the same four arrays with [L][H][P] in place
+ * of [L][B][H][T], and the caller's block table (bgtq_set_block_table)
+ * mapping tile t of sequence b to a page id, the same for every layer and
+ * KV head.  Sequences of a ragged batch then hold only the pages they use.
  * Codebook: the N(0,1) Lloyd-Max levels for 1..4 bits rounded once to
  * binary16; thresholds are the exact midpoints of those levels.
  */
@@ -74,7 +79,9 @@ enum {
                                   buf_count out of range (clamped) */
   BGTQ_DEVERR_ARG = 4,         /* encode_append: start < 0 or count < 0 or count > n */
   BGTQ_DEVERR_NONFINITE = 8,   /* allocate: a calibration value is Inf or NaN */
-  BGTQ_DEVERR_TIMEOUT = 16     /* decode: a wait for a tile copy gave up (bounded spin) */
+  BGTQ_DEVERR_TIMEOUT = 16,    /* decode: a wait for a tile copy gave up (bounded spin) */
+  BGTQ_DEVERR_PAGE = 32        /* paged cache: a block-table entry outside [0, page_pool_tiles) (encode skips the
+                                  tile, decode reads page 0 instead, logit MAE skips the tile) */
 };
 
 typedef struct {
@@ -89,7 +96,9 @@ typedef struct {
   int32_t b_max;             /* largest K width, b_min..4, b_min <= k_avg_bits <= b_max */
   int32_t rope_pairing;      /* 0: block j = dims (j, j+64) (rotate_half); 1: (2j, 2j+1) */
   int32_t max_splits;        /* split-K slots per (layer, seq, KV head); 0 = 256 */
-  int32_t reserved;          /* must be 0 */
+  int32_t page_pool_tiles;   /* 0: contiguous cache; > 0: paged cache with this many
+                                64-position pages per (layer, KV head), addressed
+                                through bgtq_set_block_table */
   int64_t capacity_tokens;   /* cached tokens per sequence, >= 1 */
   uint64_t seed;             /* seeds the Haar rotations */
 } bgtq_config;
@@ -288,6 +297,18 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
 #define BGTQ_STATIC_SCRATCH_BYTES (16u << 20)
 int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
+
+/* Paged cache only (page_pool_tiles > 0): the block table, int32
+ * [max_batch][ceil(capacity / 64)] in device memory, caller-owned: entry
+ * [b][t] = the page holding positions 64 t .. 64 t + 63 of sequence b, in
+ * 0 .. page_pool_tiles - 1.  Entries are read by the kernels when they run
+ * (so the caller may fill in new pages between calls, also under graph
+ * replay); only the tiles a call reads or writes need valid entries.  Two
+ * sequences must not share a page they write.  Until a table is set, calls
+ * that touch the cache return BGTQ_ERR_NOT_READY; on a contiguous cache
+ * this call returns BGTQ_ERR_INVALID_ARG.  NULL clears the table.  SYNC
+ * (host only). */
+int bgtq_set_block_table(bgtq_state* st, const int32_t* d_block_table);
 
 /* Split-K width for bgtq_decode_attn: 0 = automatic (one wave of resident
  * CTAs over all (layer, sequence, KV head) units, within max_splits), else a

@@ -46,7 +46,7 @@ class _Config(ctypes.Structure):
         ("b_max", ctypes.c_int32),
         ("rope_pairing", ctypes.c_int32),
         ("max_splits", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("page_pool_tiles", ctypes.c_int32),
         ("capacity_tokens", ctypes.c_int64),
         ("seed", ctypes.c_uint64),
     ]
@@ -68,12 +68,12 @@ class Config:
     max_splits: int = 0
     seed: int = 0
     head_dim: int = HEAD_DIM
+    page_pool_tiles: int = 0   # > 0: paged cache (pages per layer and KV head)
 
     def to_c(self):
         c = _Config()
         for f in fields(self):
             setattr(c, f.name, getattr(self, f.name))
-        c.reserved = 0
         return c
 
     @property
@@ -101,6 +101,7 @@ _SIGS = {
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_logit_mae": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
+    "bgtq_set_block_table": (ctypes.c_int, [_VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
@@ -253,6 +254,10 @@ def bgtq_logit_mae(state, layer, layer_count, seq, w0, m, d_q, d_k, d_mae, strea
                                 _stream(stream)))
 
 
+def bgtq_set_block_table(state, d_block_table):
+    _check(lib().bgtq_set_block_table(state, _ptr(d_block_table)))
+
+
 def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
     _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
 
@@ -308,7 +313,10 @@ class PackedKVCache:
 
     # -- views of the cache arrays (no copies) --
     def _tiles(self):
+        """Leading dims of the cache arrays: (L, B, Hkv, T) contiguous, (L, Hkv, pages) paged."""
         c = self.cfg
+        if c.page_pool_tiles > 0:
+            return (c.n_layers, c.n_kv_heads, c.page_pool_tiles)
         return (c.n_layers, c.max_batch, c.n_kv_heads, (c.capacity_tokens + TILE - 1) // TILE)
 
     def k_tiles(self):
@@ -320,7 +328,7 @@ class PackedKVCache:
         import torch
         t = self._tiles()
         n = int(np.prod(t)) * TILE * 8
-        return self.cache[self.offsets[1]:self.offsets[1] + n].view(torch.float16).view(*t[:3], t[3] * TILE, 4)
+        return self.cache[self.offsets[1]:self.offsets[1] + n].view(torch.float16).view(*t[:-1], t[-1] * TILE, 4)
 
     def v_tiles(self):
         t = self._tiles()
@@ -331,7 +339,7 @@ class PackedKVCache:
         import torch
         t = self._tiles()
         n = int(np.prod(t)) * TILE * 2
-        return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*t[:3], t[3] * TILE)
+        return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*t[:-1], t[-1] * TILE)
 
     # -- calls --
     def allocate(self, calib_q, calib_k):
@@ -373,6 +381,12 @@ class PackedKVCache:
 
     def decode_combine(self, layer, seq_lens, out, layer_count=1):
         bgtq_decode_combine(self.state, layer, layer_count, seq_lens, out.shape[1], out)
+
+    def set_block_table(self, table):
+        """Paged cache: int32 [max_batch, ceil(capacity / 64)] page ids on the
+        device (kept referenced here; its contents are read at kernel time)."""
+        bgtq_set_block_table(self.state, table)
+        self._block_table = table
 
     def set_split_tokens(self, tokens):
         bgtq_set_split_tokens(self.state, tokens)

@@ -42,6 +42,9 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Allocation set, and for a paged cache a block table given.
+bool cache_ready(const bgtq_state* st) { return st->ready && (st->cache.n_pages == 0 || st->cache.block_table); }
+
 int validate_config(const bgtq_config* c) {
   if (!c) return BGTQ_ERR_NULL;
   if (c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->max_batch < 1) return BGTQ_ERR_INVALID_ARG;
@@ -51,7 +54,7 @@ int validate_config(const bgtq_config* c) {
   if (c->b_min < 0 || c->b_max > 4 || c->b_min > c->b_max) return BGTQ_ERR_INVALID_ARG;
   if (c->k_avg_bits < c->b_min || c->k_avg_bits > c->b_max) return BGTQ_ERR_INVALID_ARG;
   if (c->rope_pairing != 0 && c->rope_pairing != 1) return BGTQ_ERR_INVALID_ARG;
-  if (c->max_splits < 0 || c->max_splits > 1024 || c->reserved != 0) return BGTQ_ERR_INVALID_ARG;
+  if (c->max_splits < 0 || c->max_splits > 1024 || c->page_pool_tiles < 0) return BGTQ_ERR_INVALID_ARG;
   if (c->capacity_tokens < 1 || c->capacity_tokens > (int64_t(1) << 30)) return BGTQ_ERR_INVALID_ARG;
   return BGTQ_OK;
 }
@@ -74,8 +77,11 @@ size_t frag_bytes(const bgtq_config* c, int layer_count) {
 
 Layout plan(const bgtq_config* c) {
   Layout p{};
-  const size_t seqs = size_t(c->n_layers) * c->max_batch * c->n_kv_heads;
-  const size_t tiles = seqs * size_t(tiles_of(c));
+  // one slot per tile: every (layer, sequence, KV head) its own T tiles, or
+  // a pool of page_pool_tiles pages per (layer, KV head)
+  const size_t tiles = c->page_pool_tiles > 0
+                           ? size_t(c->n_layers) * c->n_kv_heads * size_t(c->page_pool_tiles)
+                           : size_t(c->n_layers) * c->max_batch * c->n_kv_heads * size_t(tiles_of(c));
   const size_t toks = tiles * bgtq::kTile;
   p.krec = 0;
   p.knorm = align_up(p.krec + tiles * 1024 * c->k_avg_bits);
@@ -290,6 +296,8 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->cache.knorm = reinterpret_cast<__half*>(c8 + p.knorm);
   st->cache.vtile = reinterpret_cast<uint32_t*>(c8 + p.vrec);
   st->cache.vnorm = reinterpret_cast<__half*>(c8 + p.vnorm);
+  st->cache.block_table = nullptr;
+  st->cache.n_pages = cfg->page_pool_tiles;
   st->cache_off[0] = p.krec;
   st->cache_off[1] = p.knorm;
   st->cache_off[2] = p.vrec;
@@ -471,7 +479,7 @@ int bgtq_cache_offsets(const bgtq_state* st, size_t* out) {
 int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
                        const int32_t* d_start, const int32_t* d_count, int32_t batch, int32_t n, void* stream) {
   if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
-  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
   if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
@@ -501,7 +509,7 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
 namespace {
 
 int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, int32_t batch) {
-  if (!st->ready) return BGTQ_ERR_NOT_READY;
+  if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
   if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
@@ -690,6 +698,14 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
                            static_cast<__half*>(d_out), s) !=
       cudaSuccess)
     return BGTQ_ERR_CUDA;
+  return BGTQ_OK;
+}
+
+int bgtq_set_block_table(bgtq_state* st, const int32_t* d_block_table) {
+  if (!st) return BGTQ_ERR_NULL;
+  if (st->cache.n_pages == 0) return BGTQ_ERR_INVALID_ARG;
+  if (d_block_table && !aligned16(d_block_table)) return BGTQ_ERR_ALIGNMENT;
+  st->cache.block_table = d_block_table;
   return BGTQ_OK;
 }
 

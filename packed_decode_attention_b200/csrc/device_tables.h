@@ -76,11 +76,20 @@ struct Workspace {
 };
 
 // Cache arrays; T = ceil(capacity / 64) tiles per (layer, sequence, KV head).
+// The cache arrays hold one slot per 64-position tile.  Contiguous layout
+// (n_pages == 0): slot ((layer * B + b) * Hkv + h) * T + t.  Paged layout
+// (n_pages > 0): a pool of n_pages slots per (layer, KV head), slot
+// (layer * Hkv + h) * n_pages + block_table[b * T + t]; the caller's block
+// table maps a sequence's tile t to a page id, the same for every layer and
+// KV head.
 struct CacheDev {
-  uint32_t* ktile;               // [L][B][Hkv][T][256*kbits] words (tile format)
-  __half* knorm;                 // [L][B][Hkv][T*64][4]
-  uint32_t* vtile;               // [L][B][Hkv][T][256*vbits] words
-  __half* vnorm;                 // [L][B][Hkv][T*64]
+  uint32_t* ktile;               // [slots][256*kbits] words (tile format)
+  __half* knorm;                 // [slots][64][4]
+  uint32_t* vtile;               // [slots][256*vbits] words
+  __half* vnorm;                 // [slots][64]
+  const int32_t* block_table;    // paged: int32 [B][T] page ids (caller-owned device memory)
+  int32_t n_pages;               // pages per (layer, KV head); 0 = contiguous
+  int32_t pad;
 };
 
 struct Shape {
@@ -96,6 +105,7 @@ constexpr uint32_t kErrSeqLen = 2;
 constexpr uint32_t kErrArg = 4;
 constexpr uint32_t kErrNonFinite = 8;
 constexpr uint32_t kErrTimeout = 16;
+constexpr uint32_t kErrPage = 32;
 
 // Launchers (kernels.cu).  Each returns the cudaError_t of its launch.
 cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,

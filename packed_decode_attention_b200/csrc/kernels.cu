@@ -27,6 +27,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 
+// Cache slot of tile t of (layer, sequence b, KV head h): contiguous, or
+// through the block table of a paged cache.  -1 for a page id outside the
+// pool (the caller raises kErrPage).
+__device__ __forceinline__ int64_t tile_slot(const Shape& sh, const CacheDev& c, int layer, int b, int h, int64_t t) {
+  if (c.n_pages == 0) return ((static_cast<int64_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles + t;
+  const int32_t page = c.block_table[static_cast<int64_t>(b) * sh.ntiles + t];
+  if (page < 0 || page >= c.n_pages) return -1;
+  return (static_cast<int64_t>(layer) * sh.n_kv_heads + h) * c.n_pages + page;
+}
+
 __device__ __forceinline__ uint64_t fp16_fixed(uint16_t bits, uint32_t* nonfinite) {
   // |x| * 2^24 for a binary16 x: subnormals are m * 2^-24, normals
   // (1024 + m) * 2^(e - 25).
@@ -416,8 +426,12 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   const int bits_avg = kind == 0 ? sh.kbits : sh.vbits;
   const int nwords = 256 * bits_avg;
   const int lh = layer * sh.n_kv_heads + h;
-  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
-  uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + (seq_tiles + tile) * nwords;
+  const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+  if (slot < 0) {
+    if (tid == 0) atomicOr(ws.err, kErrPage);
+    return;
+  }
+  uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
 
   if (kind == 0) {
     if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
@@ -559,7 +573,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   for (int i = tid; i < nwords / 4; i += kEncThreads)
     reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
   if (tid >= tr0 && tid < tr1) {
-    const size_t pos = seq_tiles * kTile + tile * kTile + tid;
+    const size_t pos = static_cast<size_t>(slot) * kTile + tid;
     if (kind == 0) {
       __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
       dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
@@ -710,7 +724,11 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
   __syncthreads();
   const int i = tid;
   const int tile = static_cast<int>(pos / kTile), p = static_cast<int>(pos % kTile);
-  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
+  const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+  if (slot < 0) {  // uniform over the CTA; no barrier follows
+    if (tid == 0) atomicOr(ws.err, kErrPage);
+    return;
+  }
   if (i < lay.n_positions) {
     int g = 0;
     for (int t = 1; t < ng; ++t)
@@ -725,7 +743,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
     for (int t = 0; t < nt; ++t) code += (ws.codebook->threshold[w][t] <= u) ? 1 : 0;
     // rewrite this code's bits, one atomic pair per touched word
     const int nwords = 256 * (kind == 0 ? sh.kbits : sh.vbits);
-    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + (seq_tiles + tile) * nwords;
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
     int cur = -1;
     uint32_t mask = 0, val = 0;
     for (int q = 0; q < w; ++q) {
@@ -752,7 +770,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
     }
   }
   if (tid == 0) {
-    const size_t tp = seq_tiles * kTile + static_cast<size_t>(pos);
+    const size_t tp = static_cast<size_t>(slot) * kTile + p;
     if (kind == 0) {
       __half2* dst = reinterpret_cast<__half2*>(cache.knorm + tp * 4);
       const __half z = __float2half(0.f);
@@ -1288,7 +1306,6 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   __syncthreads();
 
   // ---- per-warp pipeline over this warp's tiles ----
-  const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles;
   const int kwords = 256 * sh.kbits, vwords = 256 * VB;
   const uint32_t kbytes = 4u * kwords, vbytes = 4u * vwords;
   const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
@@ -1297,16 +1314,19 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 
   auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
     const int tile = tlo + wu + k * W;
+    int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+    if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
+      atomicOr(ws.err, kErrPage);
+      slot = static_cast<int64_t>(layer * sh.n_kv_heads + h) * cache.n_pages;
+    }
     unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
     uint64_t* bar = &my_bars[k % kStages];
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_expect_tx(bar, stage_tx);
-    bulk_copy_g2s(dst, cache.ktile + (seq_tiles + tile) * kwords, kbytes, bar);
-    bulk_copy_g2s(dst + kbytes, cache.vtile + (seq_tiles + tile) * vwords, vbytes, bar);
-    bulk_copy_g2s(dst + kbytes + vbytes, cache.knorm + (seq_tiles * kTile + static_cast<size_t>(tile) * kTile) * 4,
-                  kTile * 8, bar);
-    bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, cache.vnorm + seq_tiles * kTile + static_cast<size_t>(tile) * kTile,
-                  kTile * 2, bar);
+    bulk_copy_g2s(dst, cache.ktile + slot * kwords, kbytes, bar);
+    bulk_copy_g2s(dst + kbytes, cache.vtile + slot * vwords, vbytes, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes, cache.knorm + slot * kTile * 4, kTile * 8, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, cache.vnorm + slot * kTile, kTile * 2, bar);
   };
   if (lane == 0)
     for (int k = 0; k < kStages && k < my_tiles; ++k) issue(k);
@@ -1755,13 +1775,17 @@ __global__ void __launch_bounds__(kDecThreads) logit_mae_kernel(Shape sh, Worksp
     }
     ByteTab t;
     const int ng = lay.n_groups;
-    const size_t seq_tiles = ((static_cast<size_t>(layer) * sh.max_batch + seq) * sh.n_kv_heads + h) * sh.ntiles;
     const int kwords = 256 * sh.kbits;
     const uint4* bq = frag + warp * kFragEntries;
     const size_t krow0 = static_cast<size_t>(li) * m;
     for (int tile = w0 / kTile; tile <= (w0 + i) / kTile; ++tile) {
-      const uint32_t* kt = cache.ktile + (seq_tiles + tile) * kwords;
-      const __half* kn = cache.knorm + (seq_tiles + tile) * kTile * 4;
+      const int64_t slot = tile_slot(sh, cache, layer, seq, h, tile);
+      if (slot < 0) {  // warp-uniform: skip the tile, flagged
+        if (lane == 0) atomicOr(ws.err, kErrPage);
+        continue;
+      }
+      const uint32_t* kt = cache.ktile + slot * kwords;
+      const __half* kn = cache.knorm + slot * kTile * 4;
       float L[4][4];
 #pragma unroll
       for (int mu = 0; mu < 4; ++mu)

@@ -44,12 +44,27 @@ def test_required_bytes_is_host_only_and_validates(lib):
     assert cache < toks * (48 + 8 + 48 + 2) + 4 * 256
     assert cache % 256 == 0 and ws % 256 == 0
     bad = [dict(head_dim=64), dict(n_q_heads=15), dict(k_avg_bits=5), dict(b_min=4, b_max=3),
-           dict(k_avg_bits=1, b_min=2), dict(rope_pairing=2), dict(capacity_tokens=0), dict(max_splits=2000)]
+           dict(k_avg_bits=1, b_min=2), dict(rope_pairing=2), dict(capacity_tokens=0), dict(max_splits=2000),
+           dict(page_pool_tiles=-1)]
     for change in bad:
         c = bgtq.Config(**{**cfg.__dict__, **change})
         with pytest.raises(bgtq.BgtqError) as e:
             bgtq.bgtq_required_bytes(c)
         assert e.value.status == -1
+
+
+def test_paged_cache_is_sized_by_its_pool(lib):
+    """A paged cache holds page_pool_tiles 64-position pages per (layer, KV
+    head), whatever max_batch and capacity are; the workspace is unchanged."""
+    base = dict(n_layers=28, n_kv_heads=4, n_q_heads=28, max_batch=16, capacity_tokens=32768, k_avg_bits=3,
+                v_avg_bits=2)
+    cont, ws = bgtq.bgtq_required_bytes(bgtq.Config(**base))
+    pool = 6000   # about 16 sequences of U[16K, 32K] tokens
+    paged, ws_p = bgtq.bgtq_required_bytes(bgtq.Config(**base, page_pool_tiles=pool))
+    per_page = 64 * (48 + 8 + 32 + 2)
+    assert 28 * 4 * pool * per_page <= paged < 28 * 4 * pool * per_page + 4 * 256
+    assert cont >= 28 * 4 * 16 * 512 * per_page
+    assert ws_p == ws
 
 
 def test_library_fails_loudly_when_missing(monkeypatch, tmp_path):

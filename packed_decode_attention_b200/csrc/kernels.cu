@@ -877,12 +877,11 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
 // ---------------------------------------------------------------------------
 // a5: split-K decode straight from the packed tiles on the tensor cores.
 //
-// Grid (n_splits, batch * Hkv * head_blocks, layer_count), 128 threads.  A
-// CTA owns the positions [s*T, min((s+1)*T, len)) of one (layer, sequence,
-// KV head) and up to 8 of its G query heads; its 4 warps take 64-position
-// tiles round-robin, each with its own 3-stage bulk-copy pipeline (K tile,
-// V tile, norms -> shared memory, completion on an mbarrier) and its own
-// online-softmax state.
+// Grid (n_splits, batch * Hkv * head_blocks, layer_count), 128 threads.  The
+// CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
+// its 64-position tiles; each warp has its own 2-stage bulk-copy pipeline
+// (K tile, V tile, norms -> shared memory, completion on an mbarrier) and its
+// own online-softmax state.
 //
 // Logits (per warp per tile): S^T[64 tokens x 8 heads] = K_hat q~^T as
 // mma.sync m16n8k16 tiles -- A = centroids C[codes] (exact in fp16), looked
@@ -1027,13 +1026,6 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
   }
 }
 
-// Grid (ctas_per_unit, batch * Hkv * head_blocks, layer_count), 128 threads.
-// A unit is one (layer, sequence, KV head, block of up to 8 query heads);
-// its tiles are dealt round-robin over the 4 * ctas_per_unit warps of its
-// CTAs (warp w of CTA c takes tiles 4c + w, 4c + w + W, ..., W = 4 *
-// ctas_per_unit), so every warp gets the same number of tiles to within one.
-// Each CTA writes one partial (m, l, acc) per query head -- an empty one
-// (m = -inf, l = 0) when it has no tile.
 // The range of a decode call's sequence: the packed positions [lo, len) and
 // the buffered row count, clamped the same way by every kernel that reads
 // them (the combine raises the flag).
@@ -1184,6 +1176,15 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
 }
 
+// Grid (ctas_per_unit [+ 1 buffer CTA], batch * Hkv * head_blocks,
+// layer_count), 128 threads.  A unit is one (layer, sequence, KV head, block
+// of up to 8 query heads); its tiles are dealt round-robin over the
+// W = 4 * ctas_per_unit warps of its CTAs, CTA-major within a round (warp w
+// of CTA c takes tiles w C + c, w C + c + W, ..., C = ctas_per_unit), so
+// every warp gets the same number of tiles to within one and the last,
+// partial round lands on as many CTAs as it can.  Each CTA writes one
+// partial (m, l, acc) per query head -- an empty one (m = -inf, l = 0) when
+// it has no tile.
 template <int VB>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
@@ -1242,14 +1243,17 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   const int len = sr.len, lo = sr.lo;
   const int tlo = lo / kTile;
   const int ntl = lo < len ? (len + kTile - 1) / kTile - tlo : 0;
+  // Tile t of the unit goes to warp (t mod W) / C of CTA (t mod W) mod C,
+  // C = ctas_per_unit: a partial last round of tiles is spread over all CTAs
+  // (and so over all SMs) before any CTA gets a second one.
   const int W = ctas_per_unit * kDecWarps;
-  const int wu = cu * kDecWarps + warp;
+  const int wu = warp * ctas_per_unit + cu;
   const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
   float* part_base = ws.partials +
                      (((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0) * sh.max_splits + cu) *
                          kPartialStride;
   const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
-  if (cu * kDecWarps >= ntl) {
+  if (cu >= ntl) {
     // no tile for this CTA: an empty partial per head
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int hh = 0; hh < nh; ++hh) {
@@ -1547,6 +1551,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kCombThreads = 256;
 constexpr int kCombWarps = kCombThreads / 32;
+static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates four at a time");
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
@@ -1560,6 +1565,13 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dd = tid & (kD - 1), half = tid >> 7;
+  // A library table, read before the split pass has finished: this thread's
+  // half column of the inverse V rotation (used if this CTA merges the row).
+  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  float mvr[64];
+#pragma unroll
+  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
   // the next kernel of the stream may start its own table-only set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Launched as a programmatic dependent of the split pass: inputs, partials
@@ -1574,53 +1586,77 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   }
   const size_t wrow = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq;  // workspace row
   const float* part = ws.partials + wrow * sh.max_splits * kPartialStride;
-  __shared__ float red[kCombWarps];
   __shared__ float accs[kCombWarps][kD];
-  __shared__ float lsw[kCombWarps];
+  __shared__ float msw[kCombWarps], lsw[kCombWarps];
   __shared__ float a_s[kD];
   __shared__ int last;
   float* mid = ws.comb_mid + (wrow * (kCombSlices + 1) + slice) * kPartialStride;
-  // ---- one slice of the row's splits ----
+  // ---- one slice of the row's splits: warp w takes splits s0 + w + 8 j,
+  // four at a time with all their loads in flight, merged online per warp
+  // (lane = 4 rotated coordinates), then across the warps ----
   const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
   const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
-  float M = -CUDART_INF_F;
-  for (int s = s0 + tid; s < s1; s += kCombThreads) M = fmaxf(M, part[static_cast<size_t>(s) * kPartialStride]);
+  float m_w = -CUDART_INF_F, l_w = 0.f;
+  float4 a_w = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int base = s0 + warp; base < s1; base += 4 * kCombWarps) {
+    float mm[4], ll[4];
+    float4 aa[4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
+    for (int j = 0; j < 4; ++j) {
+      const int sj = base + j * kCombWarps;
+      if (sj < s1) {
+        const float* p = part + static_cast<size_t>(sj) * kPartialStride;
+        mm[j] = p[0];
+        ll[j] = p[1];
+        aa[j] = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+      } else {
+        mm[j] = -CUDART_INF_F;
+        ll[j] = 0.f;
+        aa[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const float mb = fmaxf(fmaxf(m_w, fmaxf(mm[0], mm[1])), fmaxf(mm[2], mm[3]));
+    if (mb == -CUDART_INF_F) continue;  // only empty splits so far
+    const float f = m_w == -CUDART_INF_F ? 0.f : exp2f(m_w - mb);
+    l_w *= f;
+    a_w.x *= f; a_w.y *= f; a_w.z *= f; a_w.w *= f;
 #pragma unroll
-  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, red[w]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lsum = 0.f;
-#pragma unroll 4
-  for (int s = s0 + warp; s < s1; s += kCombWarps) {
-    const float* p = part + static_cast<size_t>(s) * kPartialStride;
-    const float ms = p[0];
-    const float wgt = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-    lsum = fmaf(wgt, p[1], lsum);
-    const float4 a = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
-    acc.x = fmaf(wgt, a.x, acc.x);
-    acc.y = fmaf(wgt, a.y, acc.y);
-    acc.z = fmaf(wgt, a.z, acc.z);
-    acc.w = fmaf(wgt, a.w, acc.w);
+    for (int j = 0; j < 4; ++j) {
+      const float wgt = mm[j] == -CUDART_INF_F ? 0.f : exp2f(mm[j] - mb);
+      l_w = fmaf(wgt, ll[j], l_w);
+      a_w.x = fmaf(wgt, aa[j].x, a_w.x);
+      a_w.y = fmaf(wgt, aa[j].y, a_w.y);
+      a_w.z = fmaf(wgt, aa[j].z, a_w.z);
+      a_w.w = fmaf(wgt, aa[j].w, a_w.w);
+    }
+    m_w = mb;
   }
-  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = acc;
-  if (lane == 0) lsw[warp] = lsum;
-  __syncthreads();
-  if (tid < kD) {
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) a += accs[w][tid];
-    mid[4 + tid] = a;
+  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = a_w;
+  if (lane == 0) {
+    msw[warp] = m_w;
+    lsw[warp] = l_w;
   }
-  if (tid == 0) {
-    float l = 0.f;
+  __syncthreads();
+  {
+    float M = msw[0];
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) l += lsw[w];
-    mid[0] = M;
-    mid[1] = l;
+    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, msw[w]);
+    if (tid < kD) {
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) {
+        const float wgt = msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M);
+        a = fmaf(wgt, accs[w][tid], a);
+      }
+      mid[4 + tid] = a;
+    }
+    if (tid == 0) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) l = fmaf(msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M), lsw[w], l);
+      mid[0] = M;
+      mid[1] = l;
+    }
   }
   // ---- the row's last CTA merges the intermediates ----
   const int nmid = kCombSlices + has_buf;
@@ -1631,27 +1667,34 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   if (!last) return;
   __threadfence();
   const float* mids = ws.comb_mid + wrow * (kCombSlices + 1) * kPartialStride;
+  float mk[kCombSlices + 1], lk[kCombSlices + 1], ak[kCombSlices + 1];
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) {
+    if (k < nmid) {
+      mk[k] = __ldcg(mids + k * kPartialStride);
+      lk[k] = __ldcg(mids + k * kPartialStride + 1);
+      ak[k] = __ldcg(mids + k * kPartialStride + 4 + dd);
+    } else {
+      mk[k] = -CUDART_INF_F;
+      lk[k] = 0.f;
+      ak[k] = 0.f;
+    }
+  }
   float Mt = -CUDART_INF_F;
-  for (int k = 0; k < nmid; ++k) Mt = fmaxf(Mt, __ldcg(mids + k * kPartialStride));
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) Mt = fmaxf(Mt, mk[k]);
   float Lt = 0.f, at = 0.f, ab = 0.f;
-  const int dd = tid & (kD - 1);
-  for (int k = 0; k < nmid; ++k) {
-    const float mk = __ldcg(mids + k * kPartialStride);
-    const float w = mk == -CUDART_INF_F ? 0.f : exp2f(mk - Mt);
-    Lt = fmaf(w, __ldcg(mids + k * kPartialStride + 1), Lt);
-    const float a = __ldcg(mids + k * kPartialStride + 4 + dd);
-    if (k < kCombSlices) at = fmaf(w, a, at);  // rotated basis
-    else ab = w * a;                             // the buffer's rows, unrotated
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) {
+    const float w = mk[k] == -CUDART_INF_F ? 0.f : exp2f(mk[k] - Mt);
+    Lt = fmaf(w, lk[k], Lt);
+    if (k < kCombSlices) at = fmaf(w, ak[k], at);  // rotated basis
+    else ab = w * ak[k];                            // the buffer's rows, unrotated
   }
   if (tid < kD) a_s[tid] = at / Lt;
   if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
-  // inverse V rotation: two threads per output, half of the inputs each
-  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-  const int half = tid >> 7;
-  float mvr[64];
-#pragma unroll
-  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
   __syncthreads();
+  // inverse V rotation: two threads per output, half of the inputs each
   float o = 0.f;
 #pragma unroll
   for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);

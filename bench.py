@@ -367,9 +367,10 @@ def main():
     out = torch.empty((L, B, HQ, 128), dtype=torch.float16, device=dev)
 
     def step():
+        # per layer: append the new K/V row, then attend (appends and query
+        # rotation share one launch, then the split pass and the combine)
         for l in range(L):
-            kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
-            kv.decode_attn(l, q_all[l:l + 1], seq, out[l:l + 1])
+            kv.decode_step(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq, out[l:l + 1])
 
     def step_multi():
         kv.encode_append(0, knew, vnew, start1, count1, layer_count=L)
@@ -473,8 +474,8 @@ def main():
 
         def step_paged():
             for l in range(L):
-                kvp.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
-                kvp.decode_attn(l, q_all[l:l + 1], seq, out_p[l:l + 1])
+                kvp.decode_step(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq,
+                                out_p[l:l + 1])
 
         ms_paged, g_p, _ = time_graph(step_paged, args.steps, args.warmup)
         ms_paged = max_over_ranks(ms_paged)
@@ -648,7 +649,7 @@ def main():
                      "launch_ms": split_avg_ms, "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind},
         "e2e": {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * L * args.steps,
+        "gpu_launches": 3 * L * args.steps,
         "clocks": clocks,
         "buffered": {"ms_per_step": ms_buf, "tokens_per_s": world * B / (ms_buf * 1e-3), "sink": SINK,
                      "window": WINDOW, "note": "fp16 sink + recent window next to the packed cache"},

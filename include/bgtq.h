@@ -210,6 +210,17 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
 int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                      const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
 
+/* One decode step of a layer range: bgtq_encode_append of the step's new
+ * rows followed by bgtq_decode_attn, with the same arguments, results and
+ * errors as those two calls in that order (seq_lens should count the new
+ * rows).  With 1 <= n <= 16 rows per sequence the appends and the query
+ * rotation run in one launch (they are independent), so a step takes three
+ * launches instead of four.  n = 0 appends nothing (d_k, d_v, d_start and
+ * d_count may then be NULL).  ASYNC. */
+int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                     const int32_t* d_start, const int32_t* d_count, int32_t n, const void* d_q,
+                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
+
 /* Decode with an fp16 buffer: the Block-GTQ README's "withbuffer" setting
  * (AIME commands: a few sink positions and a recent window kept
  * unquantised).  For each layer, sequence b and query head h, attention runs

@@ -101,6 +101,7 @@ _SIGS = {
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_logit_mae": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
+    "bgtq_decode_step": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_set_block_table": (ctypes.c_int, [_VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
@@ -258,6 +259,12 @@ def bgtq_set_block_table(state, d_block_table):
     _check(lib().bgtq_set_block_table(state, _ptr(d_block_table)))
 
 
+def bgtq_decode_step(state, layer, layer_count, d_k, d_v, d_start, d_count, n, d_q, d_seq_lens, batch, d_out,
+                     stream=None):
+    _check(lib().bgtq_decode_step(state, layer, layer_count, _ptr(d_k), _ptr(d_v), _ptr(d_start), _ptr(d_count), n,
+                                  _ptr(d_q), _ptr(d_seq_lens), batch, _ptr(d_out), _stream(stream)))
+
+
 def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
     _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
 
@@ -361,6 +368,11 @@ class PackedKVCache:
     def decode_attn(self, layer, q, seq_lens, out, layer_count=1):
         """q, out fp16 [layer_count, batch, Hq, 128]; seq_lens int32 [batch] on the device."""
         bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, q.shape[1], out)
+
+    def decode_step(self, layer, k, v, start, count, q, seq_lens, out, layer_count=1):
+        """encode_append(k, v, start, count) then decode_attn(q, seq_lens, out), in one call (the appends
+        and the query rotation share a launch when k holds at most 16 rows per sequence)."""
+        bgtq_decode_step(self.state, layer, layer_count, k, v, start, count, k.shape[2], q, seq_lens, q.shape[1], out)
 
     def decode_attn_buffered(self, layer, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out, layer_count=1):
         """Attention over the packed positions [pos_lo, seq_lens) and the first

@@ -573,6 +573,43 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   return BGTQ_OK;
 }
 
+int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                     const int32_t* d_start, const int32_t* d_count, int32_t n, const void* d_q,
+                     const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream) {
+  if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
+  if (n > 0 && (!d_k || !d_v || !d_start || !d_count)) return BGTQ_ERR_NULL;
+  const int v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
+  if (n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
+  if (n > 0 && (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)))
+    return BGTQ_ERR_ALIGNMENT;
+  const int split = split_for(st, layer_count, batch);
+  cudaStream_t s = as_stream(stream);
+  const __half* q = static_cast<const __half*>(d_q);
+  const __half* k = static_cast<const __half*>(d_k);
+  const __half* vv = static_cast<const __half*>(d_v);
+  cudaError_t e;
+  if (n >= 1 && n <= bgtq::kAppendMaxRows) {
+    // the appends and the query rotation in one launch
+    e = bgtq::launch_prep(st->shape, st->ws, st->cache, layer, layer_count, q, batch, st->ws.qrot, k, vv, d_start,
+                          d_count, n, s);
+  } else {
+    e = n > 0 ? bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, k, vv, d_start, d_count, batch,
+                                    n, s)
+              : cudaSuccess;
+    if (e == cudaSuccess) e = bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, q, batch, st->ws.qrot, s);
+  }
+  if (e != cudaSuccess) return BGTQ_ERR_CUDA;
+  if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens,
+                                bgtq::BufferArgs{}, batch, split, s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  if (bgtq::launch_combine(st->shape, st->ws, layer, layer_count, d_seq_lens, batch, split, bgtq::BufferArgs{},
+                           static_cast<__half*>(d_out), s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
+  return BGTQ_OK;
+}
+
 int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                               const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
                               const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,

@@ -115,6 +115,14 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
                           const int32_t* count, int batch, int n, cudaStream_t stream);
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
+// Calls with at most this many rows per sequence append row by row (the
+// decode-time path); launch_prep takes 1 <= n <= kAppendMaxRows.
+constexpr int kAppendMaxRows = 16;
+// One launch that rotates the query rows (as launch_rotate_query) and appends
+// n rows per sequence (as launch_encode's row path).
+cudaError_t launch_prep(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                        const __half* q, int batch, float* qrot, const __half* k, const __half* v,
+                        const int32_t* start, const int32_t* count, int n, cudaStream_t stream);
 // The split pass reads q~ as fragments from ws.qfrag (written by the query
 // rotation), or, when qrot is not null, builds them from qrot itself.
 // The fp16 buffered rows a decode call attends besides the packed cache

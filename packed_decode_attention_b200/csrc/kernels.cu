@@ -595,7 +595,6 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
 // touched, so rows appended by different CTAs to the same tile do not race.
 // ---------------------------------------------------------------------------
 constexpr int kAppThreads = 128;
-constexpr int kAppendMaxRows = 16;  // calls with at most this many rows per sequence use append_kernel
 
 // Plane word (0..b-1) and bit of code bit q of selector sel, nibble n, in a
 // quartet of width b (see the quartet formulas above).
@@ -642,28 +641,28 @@ __device__ __forceinline__ int v_code_word(int vb, int i, int p, int k, int& sel
   return m * 32 * vb + 32 * k + 4 * gg + t;
 }
 
-__global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
-                                                             const __half* __restrict__ kx,
-                                                             const __half* __restrict__ vx,
-                                                             const int32_t* __restrict__ start_v,
-                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+// One appended row of one (layer, sequence, KV head) and kind, by a CTA of
+// NT >= 128 threads: bx = (layer, sequence, KV head) index, row < n, kind 0
+// = K, 1 = V; mts = 64 KB of shared memory for the rotation.
+template <int NT>
+__device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws, const CacheDev& cache, int layer0,
+                                            const __half* __restrict__ kx, const __half* __restrict__ vx,
+                                            const int32_t* __restrict__ start_v, const int32_t* __restrict__ count_v,
+                                            int batch, int n, int bx, int row, int kind, float* mts) {
   const int tid = threadIdx.x;
-  const int kind = blockIdx.z;
-  const int h = blockIdx.x % sh.n_kv_heads;
-  const int b = (blockIdx.x / sh.n_kv_heads) % batch;
-  const int li = blockIdx.x / (sh.n_kv_heads * batch);
+  const int h = bx % sh.n_kv_heads;
+  const int b = (bx / sh.n_kv_heads) % batch;
+  const int li = bx / (sh.n_kv_heads * batch);
   const int layer = layer0 + li;
-  const int row = blockIdx.y;
   const int lh = layer * sh.n_kv_heads + h;
   // the next kernel of the stream may start its own table-only set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the kind's rotation (transposed, [in][out]) in shared memory, all loads
   // in flight; a library table, read before the inputs are ready
-  extern __shared__ __align__(16) float mts[];  // [kD][kD]
   {
     const uint4* src = reinterpret_cast<const uint4*>((kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD);
 #pragma unroll 8
-    for (int u = tid; u < kD * kD / 4; u += kAppThreads) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
+    for (int u = tid; u < kD * kD / 4; u += NT) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
   }
   // Launched as a programmatic dependent of the previous kernel of the
   // stream: the call's inputs and the cache are read after it has completed.
@@ -687,7 +686,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
   if (kind == 0) {
     if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
       reinterpret_cast<int32_t*>(&lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
-    for (int u = tid + kAppThreads; u < static_cast<int>(sizeof(LayoutDev) / 4); u += kAppThreads)
+    for (int u = tid + NT; u < static_cast<int>(sizeof(LayoutDev) / 4); u += NT)
       reinterpret_cast<int32_t*>(&lay)[u] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[u];
   } else if (tid == 0) {
     lay.n_groups = 1;
@@ -705,7 +704,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
   // record order: position i holds dim perm[i] (K); V keeps the dims
   if (kind == 0) {
     if (tid < lay.n_positions) xs[tid] = __half2float(x[lay.perm[tid]]);
-  } else {
+  } else if (tid < kD) {
     xs[tid] = __half2float(x[tid]);
   }
   __syncthreads();
@@ -782,6 +781,16 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
   }
 }
 
+__global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                             const __half* __restrict__ kx,
+                                                             const __half* __restrict__ vx,
+                                                             const int32_t* __restrict__ start_v,
+                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+  extern __shared__ __align__(16) float mts[];  // [kD][kD]
+  append_body<kAppThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, blockIdx.x, blockIdx.y,
+                           blockIdx.z, mts);
+}
+
 // ---------------------------------------------------------------------------
 // a4: rotate the query.  Grid (layer_count * batch * Hq), 128 threads.
 // ---------------------------------------------------------------------------
@@ -829,14 +838,15 @@ __device__ void write_frags(const LayoutDev& lay, const float* qs, int hg, int G
     }
 }
 
-__global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
-                                                                   const __half* __restrict__ q, int batch,
-                                                                   float* __restrict__ qrot) {
+// One query row (layer, sequence, query head) = bx, by a CTA of kRotThreads.
+__device__ __forceinline__ void rotate_body(const Shape& sh, const Workspace& ws, int layer0,
+                                            const __half* __restrict__ q, int batch, float* __restrict__ qrot,
+                                            int bx) {
   // the decode kernel that follows may start its own set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int hq = blockIdx.x % sh.n_q_heads;
-  const int b = (blockIdx.x / sh.n_q_heads) % batch;
-  const int li = blockIdx.x / (sh.n_q_heads * batch);
+  const int hq = bx % sh.n_q_heads;
+  const int b = (bx / sh.n_q_heads) % batch;
+  const int li = bx / (sh.n_q_heads * batch);
   const int layer = layer0 + li;
   const int kvh = hq / sh.group;
   const LayoutDev& lay = ws.layouts[layer * sh.n_kv_heads + kvh];
@@ -872,6 +882,33 @@ __global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Wor
   }
   __syncthreads();
   write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), tid, kRotThreads);
+}
+
+__global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
+                                                                   const __half* __restrict__ q, int batch,
+                                                                   float* __restrict__ qrot) {
+  rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
+}
+
+// A decode step's preparation in one launch: the first n_rot CTAs rotate the
+// query rows (as rotate_query_kernel), the others append the step's new K/V
+// rows (as append_kernel, CTA a - n_rot = ((kind * n + row) * n_units + unit),
+// n_units = layer_count * batch * Hkv).  The two parts are independent.
+__global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                           const __half* __restrict__ q, int batch,
+                                                           float* __restrict__ qrot, const __half* __restrict__ kx,
+                                                           const __half* __restrict__ vx,
+                                                           const int32_t* __restrict__ start_v,
+                                                           const int32_t* __restrict__ count_v, int n, int n_rot,
+                                                           int n_units) {
+  extern __shared__ __align__(16) float mts[];  // [kD][kD], the append part
+  if (static_cast<int>(blockIdx.x) < n_rot) {
+    rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
+  } else {
+    const int a = blockIdx.x - n_rot;
+    append_body<kRotThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, a % n_units,
+                             (a / n_units) % n, a / (n_units * n), mts);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1551,11 +1588,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kCombThreads = 256;
 constexpr int kCombWarps = kCombThreads / 32;
+// Up to this many rows per launch, every combine CTA loads its rotation
+// column early (8 slices x 64 KB per row of L2 reads).
+constexpr int kEarlyRotationRows = 256;
 static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates four at a time");
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
-                                                               int n_splits, BufferArgs buf, __half* __restrict__ out) {
+                                                               int n_splits, BufferArgs buf, __half* __restrict__ out,
+                                                               bool early_rotation) {
   const int has_buf = buf.k != nullptr ? 1 : 0;
   const int slice = blockIdx.x % kCombSlices;
   const int rowi = blockIdx.x / kCombSlices;
@@ -1566,12 +1607,16 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const int kvh = hq / sh.group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int dd = tid & (kD - 1), half = tid >> 7;
-  // A library table, read before the split pass has finished: this thread's
-  // half column of the inverse V rotation (used if this CTA merges the row).
+  // A library table: this thread's half column of the inverse V rotation,
+  // used if this CTA merges the row.  For a small launch every CTA reads it
+  // before the split pass has finished, off the critical path; for a large
+  // one (many layers per call) only the merging CTAs do, later.
   const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
   float mvr[64];
+  if (early_rotation) {
 #pragma unroll
-  for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+  }
   // the next kernel of the stream may start its own table-only set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Launched as a programmatic dependent of the split pass: inputs, partials
@@ -1693,6 +1738,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   }
   if (tid < kD) a_s[tid] = at / Lt;
   if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
+  if (!early_rotation) {
+#pragma unroll
+    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+  }
   __syncthreads();
   // inverse V rotation: two threads per output, half of the inputs each
   float o = 0.f;
@@ -2008,6 +2057,17 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
   return cudaGetLastError();
 }
 
+cudaError_t launch_prep(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                        const __half* q, int batch, float* qrot, const __half* k, const __half* v,
+                        const int32_t* start, const int32_t* count, int n, cudaStream_t stream) {
+  static const cudaError_t attr = set_smem(prep_kernel, kD * kD * sizeof(float));
+  if (attr != cudaSuccess) return attr;
+  const int n_rot = layer_count * batch * s.n_q_heads;
+  const int n_units = layer_count * batch * s.n_kv_heads;
+  return launch_dependent(prep_kernel, dim3(n_rot + n_units * n * 2), dim3(kRotThreads), kD * kD * sizeof(float),
+                          stream, s, ws, cache, layer0, q, batch, qrot, k, v, start, count, n, n_rot, n_units);
+}
+
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream) {
   return launch_dependent(rotate_query_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kRotThreads), 0, stream, s,
@@ -2029,8 +2089,9 @@ cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int 
                            const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
                            cudaStream_t stream) {
   const int nsl = kCombSlices;  // the buffered rows, if any, come from the split pass
-  return launch_dependent(combine_kernel, dim3(layer_count * batch * s.n_q_heads * nsl), dim3(kCombThreads), 0, stream,
-                          s, ws, layer0, seq_lens, batch, n_splits, buf, out);
+  const int rows = layer_count * batch * s.n_q_heads;
+  return launch_dependent(combine_kernel, dim3(rows * nsl), dim3(kCombThreads), 0, stream, s, ws, layer0, seq_lens,
+                          batch, n_splits, buf, out, rows <= kEarlyRotationRows);
 }
 
 cudaError_t launch_logit_mae(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,

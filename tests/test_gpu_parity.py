@@ -510,3 +510,51 @@ def test_decode_buffered_without_buffer_rows_equals_decode(dev):
     assert kv.device_error() == 0
     assert np.all(row_rel_err(bb[0].float().cpu().numpy(), a[0].float().cpu().numpy()) <= 1e-3)
     kv.close()
+
+
+@pytest.mark.parametrize("n", [1, 3, 16, 20, 0])
+def test_decode_step_equals_append_then_decode(dev, n):
+    """bgtq_decode_step (appends and query rotation in one launch for n <= 16
+    rows per sequence) gives the same cache bytes and the same output, bit for
+    bit, as bgtq_encode_append followed by bgtq_decode_attn."""
+    lens = [900, 333]
+    w = wl.scaled(wl.WORKLOADS["tiny"], n_kv_heads=2, n_q_heads=8, batch=2, seq_len=1024, n_calib=64)
+    cfg = library_config(w)
+    cq, ck = wl.calibration(w)
+    kvs = []
+    for _ in range(2):
+        kv = bgtq.PackedKVCache(cfg, dev)
+        kv.allocate(cq.to(dev), ck.to(dev))
+        for b, ln in enumerate(lens):
+            k = torch.zeros((1, 2, ln, 2, 128), dtype=torch.float16)
+            v = torch.zeros_like(k)
+            k[0, b] = wl.keys(w, 0, b, 0, ln)
+            v[0, b] = wl.values(w, 0, b, 0, ln)
+            start = torch.zeros(2, dtype=torch.int32, device=dev)
+            count = torch.zeros(2, dtype=torch.int32, device=dev)
+            count[b] = ln
+            kv.encode_append(0, k.to(dev), v.to(dev), start, count)
+        kvs.append(kv)
+    nn = max(n, 1)
+    kn = torch.stack([wl.keys(w, 0, b, lens[b], nn) for b in range(2)])[None].to(dev)
+    vn = torch.stack([wl.values(w, 0, b, lens[b], nn) for b in range(2)])[None].to(dev)
+    kn, vn = kn[:, :, :n], vn[:, :, :n]
+    start = torch.tensor(lens, dtype=torch.int32, device=dev)
+    count = torch.tensor([n, max(n - 1, 0)], dtype=torch.int32, device=dev)
+    seq = torch.tensor([lens[0] + n, lens[1] + max(n - 1, 0)], dtype=torch.int32, device=dev)
+    q = wl.decode_query(w, 0, [int(x) for x in seq.cpu()])[None].to(dev)
+    outs = []
+    a, bkv = kvs
+    oa = torch.empty((1, 2, 8, 128), dtype=torch.float16, device=dev)
+    if n:
+        a.encode_append(0, kn, vn, start, count)
+    a.decode_attn(0, q, seq, oa)
+    ob = torch.empty_like(oa)
+    bkv.decode_step(0, kn, vn, start, count, q, seq, ob)
+    torch.cuda.synchronize()
+    assert a.device_error() == 0 and bkv.device_error() == 0
+    assert torch.equal(a.cache, bkv.cache)
+    assert torch.equal(oa, ob)
+    assert torch.isfinite(ob.float()).all()
+    for kv in kvs:
+        kv.close()

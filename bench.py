@@ -37,7 +37,7 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/decode_split_mma_qwen3b.md, for the workload it was
 # taken on (an 8-layer copy of it: the same per-layer launch).  Reported as
 # the roofline's "traffic"; None for other workloads.
-NCU_TRAFFIC_PER_LAUNCH = {"qwen3b": 27.851e6 + 0.001e6}
+NCU_TRAFFIC_PER_LAUNCH = {"qwen3b": 27.8806e6 + 0.0003e6}
 
 
 def parse_args():

@@ -62,6 +62,31 @@ def dist_env():
     return rank, world, local
 
 
+def barrier(world):
+    """All ranks meet (no-op for one process)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    """The largest x over all ranks (a step time: the job is as slow as its
+    slowest replica).  device: where the process group's tensors live (a
+    CUDA device under NCCL, the CPU under gloo)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, batch, ms_step):
+    """Whole-job throughput: every rank decodes its own batch (weak scaling)."""
+    return world * batch / (ms_step * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -290,19 +315,6 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     w = wl.WORKLOADS[args.workload]
     if args.layers:
         w = wl.scaled(w, n_layers=args.layers)
@@ -386,7 +398,7 @@ def main():
         for _ in range(warmup):
             g.replay()
         torch.cuda.synchronize()
-        barrier()
+        barrier(world)
         torch.cuda.synchronize()
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t_wall0 = time.time()
@@ -396,7 +408,7 @@ def main():
         z.record()
         torch.cuda.synchronize()
         t_wall1 = time.time()
-        barrier()
+        barrier(world)
         return a.elapsed_time(z) / steps, g, (t_wall0, t_wall1)
 
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -406,13 +418,13 @@ def main():
     ms_step, graph, (tw0, tw1) = time_graph(step, args.steps, args.warmup)
     sampler.stop()
     clocks = sampler.summary(tw0, tw1)
-    ms_step = max_over_ranks(ms_step)
+    ms_step = max_over_ranks(ms_step, world, dev)
     assert kv.device_error() == 0, "device error during the timed steps"
     out_check = out.float()
     assert torch.isfinite(out_check).all(), "non-finite decode output"
 
     ms_multi, g_multi, _ = time_graph(step_multi, args.steps, args.warmup)
-    ms_multi = max_over_ranks(ms_multi)
+    ms_multi = max_over_ranks(ms_multi, world, dev)
     del g_multi
 
     # ---- the same step with an fp16 sink + recent window (the README's
@@ -441,7 +453,7 @@ def main():
                                     out[l:l + 1])
 
     ms_buf, g_buf, _ = time_graph(step_buffered, args.steps, args.warmup)
-    ms_buf = max_over_ranks(ms_buf)
+    ms_buf = max_over_ranks(ms_buf, world, dev)
     del g_buf, buf_k, buf_v
     assert kv.device_error() == 0, "device error in the buffered step"
 
@@ -478,7 +490,7 @@ def main():
                                 out_p[l:l + 1])
 
         ms_paged, g_p, _ = time_graph(step_paged, args.steps, args.warmup)
-        ms_paged = max_over_ranks(ms_paged)
+        ms_paged = max_over_ranks(ms_paged, world, dev)
         del g_p
         step()
         step_paged()
@@ -540,7 +552,7 @@ def main():
         graph.replay()
         o_h.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(args.steps):
@@ -551,7 +563,7 @@ def main():
         o_h.copy_(out, non_blocking=True)
     z.record()
     torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(a.elapsed_time(z) / args.steps)
+    ms_e2e = max_over_ranks(a.elapsed_time(z) / args.steps, world, dev)
     del graph
 
     # ---- dense fp16 baseline (FlashAttention-2 decode) ----
@@ -583,7 +595,7 @@ def main():
             name = "torch scaled_dot_product_attention"
         try:
             ms_fp16, g16, _ = time_graph(fp16_step, args.steps, args.warmup)
-            ms_fp16 = max_over_ranks(ms_fp16)
+            ms_fp16 = max_over_ranks(ms_fp16, world, dev)
             del g16
             fp16 = {"impl": name, "ms_per_step": ms_fp16, "tokens_per_s": world * B / (ms_fp16 * 1e-3),
                     "bytes_per_step": int(sum(lens) * H * L * 512), "speedup_of_packed": ms_fp16 / ms_step}
@@ -636,7 +648,7 @@ def main():
         cpu = {"value": B / st, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": sample.describe(len(units))}
 
-    value = world * B / (ms_step * 1e-3)
+    value = job_value(world, B, ms_step)
     step_bytes = sum(bytes_per_layer) + L * B * HQ * 512
     line = {
         "metric": "decode_tokens_per_s", "value": value, "unit": "tokens/s", "n_gpus": world,

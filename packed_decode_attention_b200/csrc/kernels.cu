@@ -956,6 +956,11 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// A hint to bring [p, p + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // One bounded poll: the thread may sleep up to kPollSuspendNs waiting for the phase.
 constexpr uint32_t kPollSuspendNs = 1000;
 
@@ -1262,6 +1267,27 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
   __syncthreads();
   if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  // While the previous kernel may still run: an L2 prefetch hint for this
+  // warp's first tiles, taken as if the sequence were full (the length is an
+  // input, read only after the wait).  A prefetch reads nothing into the
+  // CTA and leaves memory as it is, so a stale or unused line costs only
+  // bandwidth; the copies below still read after the wait.
+  if (lane == 0 && cu < ctas_per_unit) {
+    const int Wp = ctas_per_unit * kDecWarps;
+    const int wp = warp * ctas_per_unit + cu;
+    const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
+#pragma unroll
+    for (int k = 0; k < kStages; ++k) {
+      const int64_t tile = wp + static_cast<int64_t>(k) * Wp;
+      if (tile >= sh.ntiles) break;
+      const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+      if (slot < 0) break;
+      prefetch_l2(cache.ktile + slot * (kb / 4), kb);
+      prefetch_l2(cache.vtile + slot * (vb / 4), vb);
+      prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
+      prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
+    }
+  }
   // Launched as a programmatic dependent of the previous kernel (the query
   // rotation): everything above reads only the library's tables; the
   // sequence lengths, rotated queries and cache are read after that kernel

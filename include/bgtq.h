@@ -296,7 +296,8 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
  * The scratch needed is 64 KiB of arrival counters plus rows * (512 +
  * n_splits * 528 + 8 * 528) bytes, rows = layer_count * max_batch *
  * n_q_heads, plus 6 KiB per (layer, sequence, KV head, block of 8 query
- * heads), with n_splits chosen as for bgtq_decode_attn; a call needing more
+ * heads), with n_splits the most split CTAs a unit can get as for
+ * bgtq_decode_attn (see bgtq_set_split_tokens); a call needing more
  * returns BGTQ_ERR_BUFFER_SIZE before launching anything.
  *
  * The first call on a device looks up the array's device address (once per
@@ -321,11 +322,14 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
  * (host only). */
 int bgtq_set_block_table(bgtq_state* st, const int32_t* d_block_table);
 
-/* Split-K width for bgtq_decode_attn: 0 = automatic (one wave of resident
- * CTAs over all (layer, sequence, KV head) units, within max_splits), else a
- * multiple of 64 (one tile): each unit's 64-position tiles are then dealt
- * round-robin over ceil(capacity / tokens) <= max_splits split CTAs.  Results
- * do not depend on it beyond floating-point reassociation. */
+/* Split-K width for the decode calls: 0 = automatic (one wave of resident
+ * CTAs spread over all (layer, sequence, KV head) units in proportion to
+ * their lengths, so that the sequences of a ragged batch finish together;
+ * at most twice a unit's even share and max_splits), else a multiple of 64
+ * (one tile): a sequence of len positions then gets ceil(len / tokens) <=
+ * max_splits split CTAs per unit.  The split counts are computed on the GPU
+ * from the lengths.  Results do not depend on the setting beyond
+ * floating-point reassociation. */
 int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens);
 
 /* Synchronises "stream", reads the device error flag into *h_flags

@@ -371,8 +371,10 @@ class PackedKVCache:
 
     def decode_step(self, layer, k, v, start, count, q, seq_lens, out, layer_count=1):
         """encode_append(k, v, start, count) then decode_attn(q, seq_lens, out), in one call (the appends
-        and the query rotation share a launch when k holds at most 16 rows per sequence)."""
-        bgtq_decode_step(self.state, layer, layer_count, k, v, start, count, k.shape[2], q, seq_lens, q.shape[1], out)
+        and the query rotation share a launch when k holds at most 16 rows per sequence); k = None
+        appends nothing."""
+        n = 0 if k is None else k.shape[2]
+        bgtq_decode_step(self.state, layer, layer_count, k, v, start, count, n, q, seq_lens, q.shape[1], out)
 
     def decode_attn_buffered(self, layer, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out, layer_count=1):
         """Attention over the packed positions [pos_lo, seq_lens) and the first

@@ -246,14 +246,10 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
 // Split-K partials per (layer, sequence, KV head, head block): one wave of
 // resident decode CTAs over all such units (the CTAs of a unit share its
 // tiles round-robin), at most max_splits and one per 4 tiles of capacity.
-int auto_splits(bgtq_state* st, int units, int extra) {
+// Resident split CTAs the GPU holds at once (one wave).
+int split_slots(bgtq_state* st) {
   if (st->ctas_per_sm <= 0) st->ctas_per_sm = std::max(1, bgtq::decode_ctas_per_sm(st->shape));
-  const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
-  const int64_t slots = int64_t(st->ctas_per_sm) * st->num_sms;
-  int64_t n = slots / std::max(units, 1) - extra;  // extra CTAs per unit share the wave
-  n = std::min<int64_t>(n, max_splits_of(&st->cfg));
-  n = std::min<int64_t>(n, (tiles + 3) / 4);
-  return static_cast<int>(std::max<int64_t>(n, 1));
+  return st->ctas_per_sm * st->num_sms;
 }
 
 }  // namespace
@@ -516,14 +512,30 @@ int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, 
   return BGTQ_OK;
 }
 
-// Number of split-K partials per unit for a call (see auto_splits); a set
-// split size t gives ceil(capacity / t).  `extra` = CTAs per unit the split
-// pass launches beside the splits (the buffer CTA of a buffered call).
-int split_for(bgtq_state* st, int32_t layer_count, int32_t batch, int extra = 0) {
+// The split plan of a call (bgtq::SplitPlan).  A set split size t gives
+// ceil(tiles / (t / 64)) CTAs per unit.  Automatic: one wave of resident CTAs
+// (less `extra` per unit: the buffer CTA of a buffered call) spread over the
+// units in proportion to their tiles, at most twice a unit's even share, the
+// configured max_splits and the capacity's tile count.
+bgtq::SplitPlan split_for(bgtq_state* st, int32_t layer_count, int32_t batch, int extra = 0) {
   const int head_blocks = (st->shape.group + 7) / 8;
-  if (st->split_tokens > 0)
-    return static_cast<int>((st->cfg.capacity_tokens + st->split_tokens - 1) / st->split_tokens);
-  return auto_splits(st, batch * st->cfg.n_kv_heads * head_blocks * layer_count, extra);
+  bgtq::SplitPlan p{};
+  p.units_per_seq = layer_count * st->cfg.n_kv_heads * head_blocks;
+  const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
+  const int64_t max_sp = max_splits_of(&st->cfg);
+  if (st->split_tokens > 0) {
+    p.fixed_tiles = st->split_tokens / bgtq::kTile;
+    p.c_max = static_cast<int>(std::min<int64_t>(max_sp, (tiles + p.fixed_tiles - 1) / p.fixed_tiles));
+    p.budget = 0;
+    return p;
+  }
+  const int64_t units = int64_t(p.units_per_seq) * batch;
+  const int64_t budget = std::max<int64_t>(int64_t(split_slots(st)) - extra * units, units);
+  const int64_t share2 = std::max<int64_t>(1, 2 * budget / units);
+  p.budget = static_cast<int>(budget);
+  p.fixed_tiles = 0;
+  p.c_max = static_cast<int>(std::max<int64_t>(1, std::min({max_sp, share2, tiles})));
+  return p;
 }
 
 }  // namespace
@@ -559,7 +571,7 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  const int split = split_for(st, layer_count, batch);
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
@@ -584,7 +596,7 @@ int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
   if (n > 0 && (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)))
     return BGTQ_ERR_ALIGNMENT;
-  const int split = split_for(st, layer_count, batch);
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
   const __half* q = static_cast<const __half*>(d_q);
   const __half* k = static_cast<const __half*>(d_k);
@@ -621,7 +633,7 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_pos_lo) || !aligned16(d_buf_k) ||
       !aligned16(d_buf_v) || !aligned16(d_buf_count) || !aligned16(d_out))
     return BGTQ_ERR_ALIGNMENT;
-  const int split = split_for(st, layer_count, batch, 1);
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch, 1);
   cudaStream_t s = as_stream(stream);
   bgtq::BufferArgs buf;
   buf.q = static_cast<const __half*>(d_q);
@@ -696,8 +708,8 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  const int split = split_for(st, layer_count, batch);
-  const int64_t nspl = split;
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
+  const int64_t nspl = split.c_max;
   const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
   // the combine's arrival counters first, at a fixed place (they are 0
   // between calls, whatever the call's layout), then q~, its fragments, the

@@ -138,17 +138,32 @@ struct BufferArgs {
   const int32_t* pos_lo;
   int n_buf;
 };
+// How a decode call splits each unit (layer, sequence, KV head, block of 8
+// query heads) over CTAs.  The grid has c_max split CTAs per unit; a unit of
+// sequence b uses c_b of them (the rest exit at once), computed on the device
+// from the lengths by split_ctas: with fixed_tiles > 0, ceil(tiles_b /
+// fixed_tiles); else about `budget` CTAs over all units in proportion to their
+// tiles (budget * tiles_b / (units_per_seq * sum of tiles)), so that ragged
+// sequences finish together.  Always 1 <= c_b <= min(tiles_b, c_max) for a
+// unit with tiles, 0 without.
+struct SplitPlan {
+  int32_t c_max;
+  int32_t budget;
+  int32_t fixed_tiles;
+  int32_t units_per_seq;  // layer_count * Hkv * head blocks
+};
+
 // The split pass over the packed positions [pos_lo, seq_lens) (buf.pos_lo;
 // null = 0); with buf.k set, one more CTA per unit attends the buffered rows
 // and posts them as the row's extra combine intermediate.
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                                 int layer_count, const float* qrot, const int32_t* seq_lens, const BufferArgs& buf,
-                                int batch, int n_splits, cudaStream_t stream);
+                                int batch, const SplitPlan& plan, cudaStream_t stream);
 // Resident split-decode CTAs per SM for a config (0 on error).
 int decode_ctas_per_sm(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
-                           cudaStream_t stream);
+                           const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
+                           __half* out, cudaStream_t stream);
 // Per-layer logit MAE of the packed keys of sequence seq at cache positions
 // [w0, w0 + m) against the exact keys k (fp16 [layer_count][m][Hkv][128]),
 // for the queries q (fp16 [layer_count][m][Hq][128]) at the same positions

@@ -914,8 +914,8 @@ __global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace w
 // ---------------------------------------------------------------------------
 // a5: split-K decode straight from the packed tiles on the tensor cores.
 //
-// Grid (n_splits, batch * Hkv * head_blocks, layer_count), 128 threads.  The
-// CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
+// Grid (batch * Hkv * head_blocks, c_max, layer_count), 128 threads.  The
+// split CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
 // its 64-position tiles; each warp has its own 2-stage bulk-copy pipeline
 // (K tile, V tile, norms -> shared memory, completion on an mbarrier) and its
 // own online-softmax state.
@@ -1088,6 +1088,44 @@ __device__ __forceinline__ SeqRange seq_range(const Shape& sh, const int32_t* se
   return r;
 }
 
+// Packed tiles a call attends for one sequence: the tiles of [lo, len).
+__device__ __forceinline__ int64_t range_tiles(const SeqRange& r) {
+  return r.lo < r.len ? (r.len + kTile - 1) / kTile - r.lo / kTile : 0;
+}
+
+// Split CTAs of a unit with ntl tiles when the batch has `total` tiles per
+// unit summed over its sequences (see SplitPlan).  The split pass and the
+// combine evaluate it on the same inputs, so they agree.
+__device__ __forceinline__ int split_ctas(const SplitPlan& p, int64_t ntl, int64_t total) {
+  if (ntl <= 0) return 0;
+  int64_t c = p.fixed_tiles > 0 ? (ntl + p.fixed_tiles - 1) / p.fixed_tiles
+                                : static_cast<int64_t>(p.budget) * ntl / (total * p.units_per_seq);
+  c = c < 1 ? 1 : c;
+  c = c < ntl ? c : ntl;
+  c = c < p.c_max ? c : p.c_max;
+  return static_cast<int>(c);
+}
+
+// The batch's tiles summed over its sequences, by all NT threads of the CTA
+// (red: kNtWarps int64 of shared memory).  Needed only in budget mode.
+template <int NT>
+__device__ int64_t batch_tiles(const Shape& sh, const int32_t* seq_lens, const BufferArgs& buf, int batch,
+                               int64_t* red) {
+  const int tid = threadIdx.x;
+  long long t = 0;
+  for (int b = tid; b < batch; b += NT) t += range_tiles(seq_range(sh, seq_lens, buf, b));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if ((tid & 31) == 0) red[tid >> 5] = t;
+  __syncthreads();
+  int64_t sum = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) sum += red[w];
+  __syncthreads();
+  return sum;
+}
+
+
 // The fp16 buffered rows of one (layer, sequence, KV head, block of 8 query
 // heads), attended by one extra CTA of the split pass (128 threads): logits
 // q . k / sqrt(D) in log2 units (a thread per row), softmax per head, P v (a
@@ -1218,11 +1256,12 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
 }
 
-// Grid (ctas_per_unit [+ 1 buffer CTA], batch * Hkv * head_blocks,
-// layer_count), 128 threads.  A unit is one (layer, sequence, KV head, block
-// of up to 8 query heads); its tiles are dealt round-robin over the
-// W = 4 * ctas_per_unit warps of its CTAs, CTA-major within a round (warp w
-// of CTA c takes tiles w C + c, w C + c + W, ..., C = ctas_per_unit), so
+// Grid (batch * Hkv * head_blocks, [1 buffer CTA +] plan.c_max, layer_count),
+// 128 threads.  A unit is one (layer, sequence, KV head, block of up to 8
+// query heads); it uses C = split_ctas(...) of its c_max split CTAs (more for
+// longer sequences; the others exit at once).  Its tiles are dealt
+// round-robin over the W = 4 C warps of those CTAs, CTA-major within a round
+// (warp w of CTA c takes tiles w C + c, w C + c + W, ...), so
 // every warp gets the same number of tiles to within one and the last,
 // partial round lands on as many CTAs as it can.  Each CTA writes one
 // partial (m, l, acc) per query head -- an empty one (m = -inf, l = 0) when
@@ -1230,7 +1269,7 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
 template <int VB>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
-                      const int32_t* __restrict__ seq_lens, BufferArgs buf, int batch, int ctas_per_unit,
+                      const int32_t* __restrict__ seq_lens, BufferArgs buf, int batch, SplitPlan plan,
                       int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const DecodeLayout DL = decode_layout(sh.kbits, VB);
@@ -1245,10 +1284,13 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, t4 = lane & 3;
-  const int cu = blockIdx.x;
-  const int hb = blockIdx.y % head_blocks;
-  const int h = (blockIdx.y / head_blocks) % sh.n_kv_heads;
-  const int b = blockIdx.y / (head_blocks * sh.n_kv_heads);
+  // grid row 0 holds the buffer CTAs of a buffered call, so they are
+  // dispatched first; the split CTAs follow
+  const bool has_buf = buf.k != nullptr;
+  const int cu = has_buf ? static_cast<int>(blockIdx.y) - 1 : static_cast<int>(blockIdx.y);  // -1: buffer CTA
+  const int hb = blockIdx.x % head_blocks;
+  const int h = (blockIdx.x / head_blocks) % sh.n_kv_heads;
+  const int b = blockIdx.x / (head_blocks * sh.n_kv_heads);
   const int li = blockIdx.z;
   const int layer = layer0 + li;
   const int G = sh.group;
@@ -1272,12 +1314,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // input, read only after the wait).  A prefetch reads nothing into the
   // CTA and leaves memory as it is, so a stale or unused line costs only
   // bandwidth; the copies below still read after the wait.
-  if (lane == 0 && cu < ctas_per_unit) {
-    const int Wp = ctas_per_unit * kDecWarps;
-    const int wp = warp * ctas_per_unit + cu;
+  if (lane == 0 && batch == 1 && cu >= 0) {
+    // one sequence: its split count if it were full
+    const int cg = split_ctas(plan, sh.ntiles, sh.ntiles);
+    const int Wp = cg * kDecWarps;
+    const int wp = warp * cg + cu;
     const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
 #pragma unroll
-    for (int k = 0; k < kStages; ++k) {
+    for (int k = 0; k < (cu < cg ? kStages : 0); ++k) {
       const int64_t tile = wp + static_cast<int64_t>(k) * Wp;
       if (tile >= sh.ntiles) break;
       const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
@@ -1297,7 +1341,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // first positions unquantised (out-of-range values are flagged by the
   // combine kernel)
   const SeqRange sr = seq_range(sh, seq_lens, buf, b);
-  if (cu == ctas_per_unit) {
+  if (cu < 0) {
     // the extra CTA of a buffered call: the unit's fp16 buffered rows
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     buffer_attend(sh, ws, buf, sr, li, b, h, h0, nh, batch, smem_raw + DL.stage);
@@ -1305,30 +1349,26 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   }
   const int len = sr.len, lo = sr.lo;
   const int tlo = lo / kTile;
-  const int ntl = lo < len ? (len + kTile - 1) / kTile - tlo : 0;
-  // Tile t of the unit goes to warp (t mod W) / C of CTA (t mod W) mod C,
-  // C = ctas_per_unit: a partial last round of tiles is spread over all CTAs
-  // (and so over all SMs) before any CTA gets a second one.
-  const int W = ctas_per_unit * kDecWarps;
-  const int wu = warp * ctas_per_unit + cu;
+  const int ntl = static_cast<int>(range_tiles(sr));
+  // this unit's split CTAs (the same count the combine computes)
+  __shared__ int64_t s_red[kDecWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kDecThreads>(sh, seq_lens, buf, batch, s_red);
+  const int C = split_ctas(plan, ntl, total);
+  if (cu >= C) {
+    // not needed for this unit (its partials are slots 0 .. C-1)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  // Tile t of the unit goes to warp (t mod W) / C of CTA (t mod W) mod C:
+  // a partial last round of tiles is spread over all CTAs (and so over all
+  // SMs) before any CTA gets a second one.
+  const int W = C * kDecWarps;
+  const int wu = warp * C + cu;
   const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
   float* part_base = ws.partials +
                      (((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0) * sh.max_splits + cu) *
                          kPartialStride;
   const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
-  if (cu >= ntl) {
-    // no tile for this CTA: an empty partial per head
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    for (int hh = 0; hh < nh; ++hh) {
-      float* part = part_base + hh * part_head_stride;
-      part[4 + tid] = 0.f;
-      if (tid == 0) {
-        part[0] = -CUDART_INF_F;
-        part[1] = 0.f;
-      }
-    }
-    return;
-  }
   {
     const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
     if (qrot == nullptr) {
@@ -1621,7 +1661,7 @@ static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates fo
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
-                                                               int n_splits, BufferArgs buf, __half* __restrict__ out,
+                                                               SplitPlan plan, BufferArgs buf, __half* __restrict__ out,
                                                                bool early_rotation) {
   const int has_buf = buf.k != nullptr ? 1 : 0;
   const int slice = blockIdx.x % kCombSlices;
@@ -1665,6 +1705,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   // ---- one slice of the row's splits: warp w takes splits s0 + w + 8 j,
   // four at a time with all their loads in flight, merged online per warp
   // (lane = 4 rotated coordinates), then across the warps ----
+  __shared__ int64_t s_red[kCombWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kCombThreads>(sh, seq_lens, buf, batch, s_red);
+  const int n_splits = split_ctas(plan, range_tiles(sr), total);
   const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
   const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
   float m_w = -CUDART_INF_F, l_w = 0.f;
@@ -2025,14 +2068,15 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
                              const float* qrot, const int32_t* seq_lens, const BufferArgs& buf, int batch,
-                             int n_splits, cudaStream_t stream) {
+                             const SplitPlan& plan, cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
   static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
-  dim3 grid(n_splits + (buf.k != nullptr ? 1 : 0), batch * s.n_kv_heads * head_blocks, layer_count);
+  // units fastest, then split index: the CTAs every unit uses come first
+  dim3 grid(batch * s.n_kv_heads * head_blocks, (buf.k != nullptr ? 1 : 0) + plan.c_max, layer_count);
   return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, qrot, seq_lens, buf, batch, n_splits, head_blocks);
+                          ws, cache, layer0, qrot, seq_lens, buf, batch, plan, head_blocks);
 }
 
 template <int VB>
@@ -2102,22 +2146,22 @@ cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0,
 
 cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                                 int layer_count, const float* qrot, const int32_t* seq_lens, const BufferArgs& buf,
-                                int batch, int n_splits, cudaStream_t stream) {
+                                int batch, const SplitPlan& plan, cudaStream_t stream) {
   switch (s.vbits) {
-    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
-    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
-    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
-    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, n_splits, stream);
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
   }
 }
 
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
-                           const int32_t* seq_lens, int batch, int n_splits, const BufferArgs& buf, __half* out,
-                           cudaStream_t stream) {
+                           const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
+                           __half* out, cudaStream_t stream) {
   const int nsl = kCombSlices;  // the buffered rows, if any, come from the split pass
   const int rows = layer_count * batch * s.n_q_heads;
   return launch_dependent(combine_kernel, dim3(rows * nsl), dim3(kCombThreads), 0, stream, s, ws, layer0, seq_lens,
-                          batch, n_splits, buf, out, rows <= kEarlyRotationRows);
+                          batch, plan, buf, out, rows <= kEarlyRotationRows);
 }
 
 cudaError_t launch_logit_mae(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,

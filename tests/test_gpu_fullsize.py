@@ -1,6 +1,7 @@
 """Parity at the benchmark's full sizes and launch configuration.
 
-qwen3b (36 layers x 2 KV heads, 131072 tokens), batch (28 layers x 4 KV
+llama (1 layer x 8 KV heads, 32768 tokens, K2V2), qwen3b (36 layers x 2 KV
+heads, 131072 tokens), batch (28 layers x 4 KV
 heads, 16 ragged sequences of 16K-32K) and long (36 layers x 2 KV heads,
 524288 tokens): the cache is built and decoded exactly as bench.py does
 (same config, chunked prefill, per-layer and all-layers decode calls with the
@@ -31,6 +32,7 @@ pytestmark = pytest.mark.gpu
 
 SAMPLES = {
     # (layer, sequence) pairs checked against the oracle; all KV heads of each
+    "llama": [(0, 0)],
     "qwen3b": [(0, 0), (35, 0)],
     "batch": [(0, 0), (27, 15)],
     "long": [(35, 0)],
@@ -45,7 +47,7 @@ def dev():
     return torch.device("cuda:0")
 
 
-@pytest.mark.parametrize("name", ["qwen3b", "batch", "long"])
+@pytest.mark.parametrize("name", ["llama", "qwen3b", "batch", "long"])
 def test_full_size_parity(dev, name):
     w = wl.WORKLOADS[name]
     lens = wl.seq_lens(w)
@@ -110,8 +112,13 @@ def test_full_size_parity(dev, name):
         kv.decode_attn(l, q_all[l:l + 1], seq, out_layer[l:l + 1])
     out_all = torch.empty_like(out_layer)
     kv.decode_attn(0, q_all, seq, out_all, layer_count=w.n_layers)
+    # the benchmark's call (decode_step, here with no new row) is the same computation
+    out_step = torch.empty_like(out_layer)
+    for l in range(w.n_layers):
+        kv.decode_step(l, None, None, None, None, q_all[l:l + 1], seq, out_step[l:l + 1])
     torch.cuda.synchronize()
     assert kv.device_error() == 0
+    assert torch.equal(out_step, out_layer)
     assert torch.isfinite(out_layer.float()).all() and torch.isfinite(out_all.float()).all()
     a = out_layer.float().cpu().numpy()
     assert np.all(row_rel_err(out_all.float().cpu().numpy(), a) <= REL_TOL)

@@ -664,25 +664,13 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
 #pragma unroll 8
     for (int u = tid; u < kD * kD / 4; u += NT) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
   }
-  // Launched as a programmatic dependent of the previous kernel of the
-  // stream: the call's inputs and the cache are read after it has completed.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int start = start_v[b];
-  const int count = count_v[b];
-  if (start < 0 || count < 0 || count > n) {
-    if (tid == 0 && row == 0 && kind == 0) atomicOr(ws.err, kErrArg);
-    return;
-  }
-  if (row >= count) return;
-  const int64_t pos = static_cast<int64_t>(start) + row;
-  if (pos >= sh.capacity) {
-    if (tid == 0) atomicOr(ws.err, kErrCapacity);
-    return;
-  }
+  // the layout and the thresholds: library tables too
   __shared__ LayoutDev lay;
+  __shared__ float thr[5 * 16];
   __shared__ float xs[kD];
   __shared__ float fac[kNumGroupsMax];
   __shared__ __half nrm[kNumGroupsMax];
+  for (int u = tid; u < 5 * 16; u += NT) thr[u] = (&ws.codebook->threshold[0][0])[u];
   if (kind == 0) {
     if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
       reinterpret_cast<int32_t*>(&lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
@@ -699,14 +687,33 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
     }
   }
   __syncthreads();
+  // Launched as a programmatic dependent of the previous kernel of the
+  // stream: the call's inputs and the cache are read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // this row's values (row < n: inside the input whatever count is) and the
+  // sequence's start and count, all in flight together; record order:
+  // position i holds dim perm[i] (K), V keeps the dims
   const __half* x = (kind == 0 ? kx : vx) +
                     ((static_cast<size_t>(li) * batch + b) * n + row) * sh.n_kv_heads * kD + static_cast<size_t>(h) * kD;
-  // record order: position i holds dim perm[i] (K); V keeps the dims
+  float xv = 0.f;
   if (kind == 0) {
-    if (tid < lay.n_positions) xs[tid] = __half2float(x[lay.perm[tid]]);
+    if (tid < lay.n_positions) xv = __half2float(x[lay.perm[tid]]);
   } else if (tid < kD) {
-    xs[tid] = __half2float(x[tid]);
+    xv = __half2float(x[tid]);
   }
+  const int start = start_v[b];
+  const int count = count_v[b];
+  if (start < 0 || count < 0 || count > n) {
+    if (tid == 0 && row == 0 && kind == 0) atomicOr(ws.err, kErrArg);
+    return;
+  }
+  if (row >= count) return;
+  const int64_t pos = static_cast<int64_t>(start) + row;
+  if (pos >= sh.capacity) {
+    if (tid == 0) atomicOr(ws.err, kErrCapacity);
+    return;
+  }
+  if (tid < kD) xs[tid] = xv;
   __syncthreads();
   const int ng = lay.n_groups;
   if (tid < ng) {
@@ -739,7 +746,7 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
     const float u = y * fac[g];
     int code = 0;
     const int nt = (1 << w) - 1;
-    for (int t = 0; t < nt; ++t) code += (ws.codebook->threshold[w][t] <= u) ? 1 : 0;
+    for (int t = 0; t < nt; ++t) code += (thr[w * 16 + t] <= u) ? 1 : 0;
     // rewrite this code's bits, one atomic pair per touched word
     const int nwords = 256 * (kind == 0 ? sh.kbits : sh.vbits);
     uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;

@@ -1344,6 +1344,19 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // sequence lengths, rotated queries and cache are read after that kernel
   // has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the unit's q~ fragments (written by the query rotation): their loads go
+  // out with the length reads below and land in shared memory further down
+  const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+  constexpr int kFragPerThread = (kFragEntries + kDecThreads - 1) / kDecThreads;
+  uint4 fr[kFragPerThread];
+  if (qrot == nullptr && cu >= 0) {
+    const uint4* src = frag_block(sh, ws, li, b, h, hb);
+#pragma unroll
+    for (int i = 0; i < kFragPerThread; ++i) {
+      const int u = tid + i * kDecThreads;
+      if (u < 32 * nchunk) fr[i] = src[u];
+    }
+  }
   // the packed positions attended: [lo, len); lo > 0 when the caller keeps the
   // first positions unquantised (out-of-range values are flagged by the
   // combine kernel)
@@ -1377,11 +1390,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
                          kPartialStride;
   const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
   {
-    const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
     if (qrot == nullptr) {
-      // q~ fragments of this unit, written by the query rotation
-      const uint4* src = frag_block(sh, ws, li, b, h, hb);
-      for (int u = tid; u < 32 * nchunk; u += kDecThreads) bq[u] = src[u];
+#pragma unroll
+      for (int i = 0; i < kFragPerThread; ++i) {
+        const int u = tid + i * kDecThreads;
+        if (u < 32 * nchunk) bq[u] = fr[i];
+      }
     } else {
       // the split pass on its own: the fragments from the caller's q~
       // (fp32, record order): coordinates 16 j + 4 t .. + 3 of chunk c's

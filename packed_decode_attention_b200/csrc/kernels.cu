@@ -378,10 +378,20 @@ __device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kD], int tid, i
 // the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
+constexpr int kXtPitch = kTile + 4;  // row pitch of xt: 16-byte rows, transposed writes spread over banks
+
+// The Lloyd-Max code of u for width w >= 1: the number of the 2^w - 1
+// ascending thresholds t[] that are <= u (ties go up), by binary search.
+__device__ __forceinline__ int lloyd_code(const float* t, int w, float u) {
+  int c = 0;
+  for (int s = 1 << (w - 1); s > 0; s >>= 1)
+    if (t[c + s - 1] <= u) c += s;
+  return c;
+}
 
 struct EncodeSmem {
-  float xt[kD][kTile];           // new rows, transposed, record order (zero elsewhere)
-  float mt[kD][kD];              // mt[j][i] = R[i][j] (record order)
+  float xt[kD][kXtPitch];        // new rows, transposed, record order (zero elsewhere)
+  float mt[kD][kD];              // mt[j][c(i)] = R[i][j] (record order), c(8 o + 4 q + e) = 64 q + 4 o + e
   float fac[kTile][kNumGroupsMax];
   __half nrm[kTile][kNumGroupsMax];
   uint8_t codes[kTile][kD];
@@ -450,8 +460,13 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   }
   for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
   const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
-  for (int i = tid; i < kD * kD / 4; i += kEncThreads)
-      reinterpret_cast<float4*>(&S.mt[0][0])[i] = reinterpret_cast<const float4*>(mglob)[i];
+  // columns swizzled so that the 16 output groups of a warp read the first
+  // and the second half of their 8 columns as two contiguous 256-byte spans
+  for (int i = tid; i < kD * kD / 4; i += kEncThreads) {
+    const int j = i / (kD / 4), c4 = i % (kD / 4);  // float4 c4 of row j: columns 4 c4 .. 4 c4 + 3
+    const int o = c4 >> 1, q = c4 & 1;
+    reinterpret_cast<float4*>(&S.mt[j][0])[q * 16 + o] = reinterpret_cast<const float4*>(mglob)[i];
+  }
   __syncthreads();
   const int ng = S.lay.n_groups;
   const int npos = S.lay.n_positions;
@@ -530,10 +545,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
+#pragma unroll 4
       for (int j = jlo; j < jhi; ++j) {
         const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][rg * 4]);
-        const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][i0]);
-        const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][i0 + 4]);
+        const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][4 * og]);
+        const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][64 + 4 * og]);
         const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
         const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
@@ -551,10 +567,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
           if (g < 0) continue;
           const int w = S.lay.width[g];
           const float u = acc[a][q] * S.fac[r][g];
-          int code = 0;
-          const int nt = (1 << w) - 1;
-          for (int t = 0; t < nt; ++t) code += (S.thr[w][t] <= u) ? 1 : 0;
-          S.codes[r][i0 + q] = static_cast<uint8_t>(code);
+          S.codes[r][i0 + q] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
         }
       }
     }
@@ -744,9 +757,7 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
     for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
     const int w = lay.width[g];
     const float u = y * fac[g];
-    int code = 0;
-    const int nt = (1 << w) - 1;
-    for (int t = 0; t < nt; ++t) code += (thr[w * 16 + t] <= u) ? 1 : 0;
+    const int code = lloyd_code(thr + w * 16, w, u);
     // rewrite this code's bits, one atomic pair per touched word
     const int nwords = 256 * (kind == 0 ? sh.kbits : sh.vbits);
     uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;

@@ -239,8 +239,13 @@ __device__ __forceinline__ GroupGeo group_geo(const LayoutDev& lay, int g) {
 __device__ __forceinline__ int k_token(int mu, int lane, int n) { return 16 * mu + (lane >> 2) + 8 * (n >= 4); }
 __device__ __forceinline__ int k_coord(int j, int lane, int n) { return 16 * j + 4 * (lane & 3) + (n & 3); }
 
+// Row pitch (bytes) of a tile's code matrix [64 tokens][128 coordinates] in
+// shared memory: 132 puts the rows of consecutive tokens in different banks.
+constexpr int kCodePitch = kD + 4;
+
 template <int B>
-__device__ void unpack_k_group(const uint32_t* tw, const GroupGeo& q, uint8_t (*codes)[kD], int tid, int nthreads) {
+__device__ void unpack_k_group(const uint32_t* tw, const GroupGeo& q, uint8_t (*codes)[kCodePitch], int tid,
+                               int nthreads) {
   const uint32_t* gw = tw + q.word;
   for (int u = tid; u < q.nfull * 32; u += nthreads) {
     const int j = u >> 5, lane = u & 31;
@@ -280,7 +285,8 @@ __device__ void unpack_k_group(const uint32_t* tw, const GroupGeo& q, uint8_t (*
 }
 
 template <int B>
-__device__ void pack_k_group(uint32_t* tw, const GroupGeo& q, const uint8_t (*codes)[kD], int tid, int nthreads) {
+__device__ void pack_k_group(uint32_t* tw, const GroupGeo& q, const uint8_t (*codes)[kCodePitch], int tid,
+                             int nthreads) {
   uint32_t* gw = tw + q.word;
   for (int u = tid; u < q.nfull * 32; u += nthreads) {
     const int j = u >> 5, lane = u & 31;
@@ -335,7 +341,7 @@ __device__ __forceinline__ int v_token(int kappa, int lane, int n) {
 __device__ __forceinline__ int v_coord(int m, int lane, int n) { return 16 * m + (lane >> 2) + 8 * (n >= 4); }
 
 template <int B>
-__device__ void unpack_v_tile(const uint32_t* tw, uint8_t (*codes)[kD], int tid, int nthreads) {
+__device__ void unpack_v_tile(const uint32_t* tw, uint8_t (*codes)[kCodePitch], int tid, int nthreads) {
   for (int u = tid; u < 8 * 32; u += nthreads) {
     const int m = u >> 5, lane = u & 31;
     uint32_t w[B], s[4];
@@ -347,7 +353,7 @@ __device__ void unpack_v_tile(const uint32_t* tw, uint8_t (*codes)[kD], int tid,
 }
 
 template <int B>
-__device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kD], int tid, int nthreads) {
+__device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kCodePitch], int tid, int nthreads) {
   for (int u = tid; u < 8 * 32; u += nthreads) {
     const int m = u >> 5, lane = u & 31;
     uint32_t s[4], w[B];
@@ -378,7 +384,9 @@ __device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kD], int tid, i
 // the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
-constexpr int kXtPitch = kTile + 4;  // row pitch of xt: 16-byte rows, transposed writes spread over banks
+// Column of element (coordinate j, row r) in xt[j][]: float4 groups of 4 rows,
+// XOR-swizzled by j so that the transposed writes spread over the banks.
+__device__ __forceinline__ int xt_col(int j, int r) { return (((r >> 2) ^ ((j >> 3) & 15)) << 2) | (r & 3); }
 
 // The Lloyd-Max code of u for width w >= 1: the number of the 2^w - 1
 // ascending thresholds t[] that are <= u (ties go up), by binary search.
@@ -390,11 +398,11 @@ __device__ __forceinline__ int lloyd_code(const float* t, int w, float u) {
 }
 
 struct EncodeSmem {
-  float xt[kD][kXtPitch];        // new rows, transposed, record order (zero elsewhere)
+  float xt[kD][kTile];           // new rows, transposed, record order (zero elsewhere), columns xt_col
   float mt[kD][kD];              // mt[j][c(i)] = R[i][j] (record order), c(8 o + 4 q + e) = 64 q + 4 o + e
   float fac[kTile][kNumGroupsMax];
   __half nrm[kTile][kNumGroupsMax];
-  uint8_t codes[kTile][kD];
+  uint8_t codes[kTile][kCodePitch];
   uint32_t words[1024];
   float thr[5][16];
   int32_t inv[kD];
@@ -497,12 +505,19 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
   const __half* x = kind == 0 ? kx : vx;
   const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
                         static_cast<size_t>(h) * kD;
-  for (int e = tid; e < kTile * kD; e += kEncThreads) {
-    const int r = e / kD, dm = e % kD;
-    const int tr = r;
-    const bool valid = tr >= tr0 && tr < tr1;
-    const float v = valid ? __half2float(xbase[static_cast<size_t>(tr - tr0) * row_stride + dm]) : 0.f;
-    S.xt[S.inv[dm]][tr] = v;
+  for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
+    const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (r >= tr0 && r < tr1)
+      raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(h2[k]);
+      const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
+      S.xt[j0][xt_col(j0, r)] = f.x;
+      S.xt[j1][xt_col(j1, r)] = f.y;
+    }
   }
   __syncthreads();
   // norms: fp64 sum of squares of the exact fp16 inputs
@@ -514,7 +529,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
       const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
       double s2 = 0.0;
       for (int j = j0; j < j1; ++j) {
-        const double v = S.xt[j][r];
+        const double v = S.xt[j][xt_col(j, r)];
         s2 += v * v;
       }
       const double nr = sqrt(s2);
@@ -547,7 +562,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
         for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
 #pragma unroll 4
       for (int j = jlo; j < jhi; ++j) {
-        const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][rg * 4]);
+        const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][4 * (rg ^ ((j >> 3) & 15))]);
         const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][4 * og]);
         const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][64 + 4 * og]);
         const float xs[4] = {xv.x, xv.y, xv.z, xv.w};

@@ -11,6 +11,8 @@
 // chatpaper summary / arXiv 2606.24033 abstract, blockgtq README) on top of
 // TurboQuant-MSE (arXiv 2504.19874); split-K decoding after FlashAttention /
 // FlashAttention-2 (arXiv 2205.14135, 2307.08691), both cited by the pages.
+#include <algorithm>
+
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -376,12 +378,12 @@ __device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kCodePitch], in
   }
 
 // ---------------------------------------------------------------------------
-// a3: encode.  Grid (layer_count * batch * Hkv, ceil(n / 64) + 1, 2 kinds),
-// 256 threads.  A CTA owns one 64-position tile of one (layer, sequence, KV
-// head) and kind (K or V): it unpacks the tile's codes when the call writes
-// only part of it, encodes its new rows (y = R x in fp32, norms in fp64,
-// u = sqrt(d) y / n, code = #{thresholds <= u}) into the codes, and packs
-// the tile again.
+// a3: encode.  Grid (layer_count * batch * Hkv, per_unit, 2 kinds), 256
+// threads.  A CTA loads one (layer, KV head, kind)'s rotation and tables once
+// and then takes every per_unit-th 64-position tile that the call writes for
+// one sequence: it unpacks the tile's codes when the call writes only part of
+// it, encodes its new rows (y = R x in fp32, norms in fp64, u = sqrt(d) y /
+// n, code = #{thresholds <= u}) into the codes, and packs the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
 // Column of element (coordinate j, row r) in xt[j][]: float4 groups of 4 rows,
@@ -430,27 +432,16 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     return;
   }
   if (count == 0) return;
-  const int64_t tile = start / kTile + blockIdx.y;
-  const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
-  int64_t p1 = min(tile * kTile + kTile, static_cast<int64_t>(start) + count);
-  if (p0 >= p1) return;
-  if (p1 > sh.capacity) {
-    if (tid == 0) atomicOr(ws.err, kErrCapacity);
-    p1 = sh.capacity;
-    if (p0 >= p1) return;
+  int64_t p_end = static_cast<int64_t>(start) + count;  // rows land at [start, p_end)
+  if (p_end > sh.capacity) {
+    if (tid == 0 && blockIdx.y == 0) atomicOr(ws.err, kErrCapacity);
+    p_end = sh.capacity;
   }
-  const int tr0 = static_cast<int>(p0 - tile * kTile), tr1 = static_cast<int>(p1 - tile * kTile);
-  const bool whole = (tr0 == 0 && tr1 == kTile);
+  const int64_t t_first = start / kTile;
+  if (t_first + blockIdx.y >= (p_end + kTile - 1) / kTile) return;  // no tile for this CTA
   const int bits_avg = kind == 0 ? sh.kbits : sh.vbits;
   const int nwords = 256 * bits_avg;
   const int lh = layer * sh.n_kv_heads + h;
-  const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
-  if (slot < 0) {
-    if (tid == 0) atomicOr(ws.err, kErrPage);
-    return;
-  }
-  uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
-
   if (kind == 0) {
     if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
       reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
@@ -488,127 +479,144 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     }
     S.gof[tid] = g;
   }
-  // existing codes of a partly written tile
-  if (!whole) {
-    if (kind == 0) {
-      for (int g = 0; g < ng; ++g) {
-        const GroupGeo q = group_geo(S.lay, g);
-        BGTQ_WIDTH_SWITCH(q.width, unpack_k_group, gtile, q, S.codes, tid, kEncThreads)
+  __syncthreads();
+  // ---- this CTA's tiles: t_first + blockIdx.y, then every gridDim.y-th ----
+  for (int64_t tile = t_first + blockIdx.y; tile * kTile < p_end; tile += gridDim.y) {
+    const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
+    const int64_t p1 = min(tile * kTile + kTile, p_end);
+    const int tr0 = static_cast<int>(p0 - tile * kTile), tr1 = static_cast<int>(p1 - tile * kTile);
+    const bool whole = (tr0 == 0 && tr1 == kTile);
+    if (p0 >= p1) continue;  // the first rows are past the capacity
+    const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+    if (slot < 0) {  // uniform over the CTA
+      if (tid == 0) atomicOr(ws.err, kErrPage);
+      continue;
+    }
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
+    // existing codes of a partly written tile
+    if (!whole) {
+      if (kind == 0) {
+        for (int g = 0; g < ng; ++g) {
+          const GroupGeo q = group_geo(S.lay, g);
+          BGTQ_WIDTH_SWITCH(q.width, unpack_k_group, gtile, q, S.codes, tid, kEncThreads)
+        }
+      } else {
+        BGTQ_WIDTH_SWITCH(sh.vbits, unpack_v_tile, gtile, S.codes, tid, kEncThreads)
       }
-    } else {
-      BGTQ_WIDTH_SWITCH(sh.vbits, unpack_v_tile, gtile, S.codes, tid, kEncThreads)
     }
-  }
-  __syncthreads();
-  // new rows -> xt (record order)
-  const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
-  const __half* x = kind == 0 ? kx : vx;
-  const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
-                        static_cast<size_t>(h) * kD;
-  for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
-    const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
-    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-    if (r >= tr0 && r < tr1)
-      raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(h2[k]);
-      const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
-      S.xt[j0][xt_col(j0, r)] = f.x;
-      S.xt[j1][xt_col(j1, r)] = f.y;
-    }
-  }
-  __syncthreads();
-  // norms: fp64 sum of squares of the exact fp16 inputs
-  {
-    const int r = tid >> 2, g = tid & 3;
-    float f = 0.f;
-    __half nh = __float2half(0.f);
-    if (g < ng && r >= tr0 && r < tr1) {
-      const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
-      double s2 = 0.0;
-      for (int j = j0; j < j1; ++j) {
-        const double v = S.xt[j][xt_col(j, r)];
-        s2 += v * v;
+    __syncthreads();
+    // new rows -> xt (record order)
+    const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
+    const __half* x = kind == 0 ? kx : vx;
+    const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
+                          static_cast<size_t>(h) * kD;
+    for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
+      const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (r >= tr0 && r < tr1)
+        raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+  #pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(h2[k]);
+        const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
+        S.xt[j0][xt_col(j0, r)] = f.x;
+        S.xt[j1][xt_col(j1, r)] = f.y;
       }
-      const double nr = sqrt(s2);
-      nh = __double2half(nr);
-      f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;
     }
-    S.fac[r][g] = f;
-    S.nrm[r][g] = nh;
-  }
-  __syncthreads();
-  // y = R x per new row (fp32, coordinate order), then the codes
-  {
-    // register tile: 4 rows x 8 outputs per thread over all 64 rows
-    const int rg = tid >> 4, og = tid & 15;
-    const int i0 = og * 8;
-    if (i0 < npos && rg * 4 < tr1 && rg * 4 + 4 > tr0) {
-      int gi[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) gi[q] = S.gof[i0 + q];
-      int ghi = gi[0];
-#pragma unroll
-      for (int q = 1; q < 8; ++q)
-        if (gi[q] > ghi) ghi = gi[q];
-      const int jlo = S.lay.start[gi[0]];
-      const int jhi = S.lay.start[ghi] + S.lay.size[ghi];
-      float acc[4][8];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
-#pragma unroll 4
-      for (int j = jlo; j < jhi; ++j) {
-        const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][4 * (rg ^ ((j >> 3) & 15))]);
-        const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][4 * og]);
-        const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][64 + 4 * og]);
-        const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
-        const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-#pragma unroll
+    __syncthreads();
+    // norms: fp64 sum of squares of the exact fp16 inputs
+    {
+      const int r = tid >> 2, g = tid & 3;
+      float f = 0.f;
+      __half nh = __float2half(0.f);
+      if (g < ng && r >= tr0 && r < tr1) {
+        const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
+        double s2 = 0.0;
+        for (int j = j0; j < j1; ++j) {
+          const double v = S.xt[j][xt_col(j, r)];
+          s2 += v * v;
+        }
+        const double nr = sqrt(s2);
+        nh = __double2half(nr);
+        f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;
+      }
+      S.fac[r][g] = f;
+      S.nrm[r][g] = nh;
+    }
+    __syncthreads();
+    // y = R x per new row (fp32, coordinate order), then the codes
+    {
+      // register tile: 4 rows x 8 outputs per thread over all 64 rows
+      const int rg = tid >> 4, og = tid & 15;
+      const int i0 = og * 8;
+      if (i0 < npos && rg * 4 < tr1 && rg * 4 + 4 > tr0) {
+        int gi[8];
+  #pragma unroll
+        for (int q = 0; q < 8; ++q) gi[q] = S.gof[i0 + q];
+        int ghi = gi[0];
+  #pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (gi[q] > ghi) ghi = gi[q];
+        const int jlo = S.lay.start[gi[0]];
+        const int jhi = S.lay.start[ghi] + S.lay.size[ghi];
+        float acc[4][8];
+  #pragma unroll
         for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc[a][q] = fmaf(xs[a], ms[q], acc[a][q]);
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int r = rg * 4 + a;
-        if (r < tr0 || r >= tr1) continue;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int g = gi[q];
-          if (g < 0) continue;
-          const int w = S.lay.width[g];
-          const float u = acc[a][q] * S.fac[r][g];
-          S.codes[r][i0 + q] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
+  #pragma unroll 4
+        for (int j = jlo; j < jhi; ++j) {
+          const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][4 * (rg ^ ((j >> 3) & 15))]);
+          const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][4 * og]);
+          const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][64 + 4 * og]);
+          const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+          const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+  #pragma unroll
+          for (int a = 0; a < 4; ++a)
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) acc[a][q] = fmaf(xs[a], ms[q], acc[a][q]);
+        }
+  #pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int r = rg * 4 + a;
+          if (r < tr0 || r >= tr1) continue;
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int g = gi[q];
+            if (g < 0) continue;
+            const int w = S.lay.width[g];
+            const float u = acc[a][q] * S.fac[r][g];
+            S.codes[r][i0 + q] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
+          }
         }
       }
     }
-  }
-  __syncthreads();
-  // repack the tile and write it back
-  if (kind == 0) {
-    for (int g = 0; g < ng; ++g) {
-      const GroupGeo q = group_geo(S.lay, g);
-      BGTQ_WIDTH_SWITCH(q.width, pack_k_group, S.words, q, S.codes, tid, kEncThreads)
-    }
-  } else {
-    BGTQ_WIDTH_SWITCH(sh.vbits, pack_v_tile, S.words, S.codes, tid, kEncThreads)
-  }
-  __syncthreads();
-  for (int i = tid; i < nwords / 4; i += kEncThreads)
-    reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
-  if (tid >= tr0 && tid < tr1) {
-    const size_t pos = static_cast<size_t>(slot) * kTile + tid;
+    __syncthreads();
+    // repack the tile and write it back
     if (kind == 0) {
-      __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
-      dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
-      dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
+      for (int g = 0; g < ng; ++g) {
+        const GroupGeo q = group_geo(S.lay, g);
+        BGTQ_WIDTH_SWITCH(q.width, pack_k_group, S.words, q, S.codes, tid, kEncThreads)
+      }
     } else {
-      cache.vnorm[pos] = S.nrm[tid][0];
+      BGTQ_WIDTH_SWITCH(sh.vbits, pack_v_tile, S.words, S.codes, tid, kEncThreads)
     }
+    __syncthreads();
+    for (int i = tid; i < nwords / 4; i += kEncThreads)
+      reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
+    if (tid >= tr0 && tid < tr1) {
+      const size_t pos = static_cast<size_t>(slot) * kTile + tid;
+      if (kind == 0) {
+        __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
+        dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
+        dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
+      } else {
+        cache.vnorm[pos] = S.nrm[tid][0];
+      }
+    }
+
+    __syncthreads();  // the buffers are reused by the next tile
   }
 }
 
@@ -2169,7 +2177,18 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
     return launch_dependent(append_kernel, dim3(layer_count * batch * s.n_kv_heads, n, 2), dim3(kAppThreads),
                             kD * kD * sizeof(float), stream, s, ws, cache, layer0, k, v, start, count, batch, n);
   }
-  dim3 grid(layer_count * batch * s.n_kv_heads, (n + kTile - 1) / kTile + 1, 2);
+  // about two waves of CTAs (two fit an SM); each loops over its unit's tiles
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  const int units = layer_count * batch * s.n_kv_heads;
+  const int tiles = (n + kTile - 1) / kTile + 1;  // rows may start inside a tile
+  const int per_unit = std::max(1, std::min(tiles, (4 * sms) / (2 * units)));
+  dim3 grid(units, per_unit, 2);
   encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
   return cudaGetLastError();
 }

@@ -13,6 +13,10 @@
  *   bgtq_encode_append  rotate, normalise, Lloyd-Max quantise, bit-pack K/V
  *   bgtq_rotate_query   the query in each width group's rotated basis
  *   bgtq_decode_attn    one GQA decode step over the packed cache
+ *   bgtq_decode_step    encode_append of a step's rows + decode_attn in one call
+ *   bgtq_decode_attn_buffered  decode with fp16 sink / recent-window rows
+ *   bgtq_logit_mae      per-layer logit error of the packed keys (diagnostic)
+ *   bgtq_set_block_table  page table of a paged cache
  *
  * Conventions
  *  - Every function returns 0 (BGTQ_OK) or a negative BGTQ_ERR_* code and

@@ -217,6 +217,22 @@ def test_decode_other_widths_and_pairings(dev, over):
     _decode_identical(w, dev, [1500], **over)
 
 
+@pytest.mark.parametrize("n_kv,n_q", [(2, 2), (1, 16), (1, 5)])
+def test_decode_group_sizes(dev, n_kv, n_q):
+    """G = 1 (one query head per KV head), G = 16 (two blocks of 8 query
+    heads per KV head, the largest group) and G = 5 (a partial block)."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], n_kv_heads=n_kv, n_q_heads=n_q, seq_len=1300)
+    _decode_identical(w, dev, [1300])
+
+
+def test_decode_ragged_automatic_split_one_long_sequence(dev):
+    """Automatic split counts follow the lengths: one long sequence next to
+    short and empty ones (the long one gets most of the split CTAs, capped at
+    twice its even share)."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], batch=5, seq_len=4096)
+    _decode_identical(w, dev, [4096, 64, 0, 130, 1])
+
+
 def test_decode_single_token_is_v_hat(dev):
     w = wl.scaled(wl.WORKLOADS["tiny"], seq_len=64)
     cfg = library_config(w)
@@ -432,6 +448,7 @@ def test_small_appends_equal_one_encode(dev):
     ([100, 3000, 132, 500], 4, 128),     # short sequences: the packed range empties
     ([2000], 0, 64),
     ([700], 16, 0),
+    ([1500], 4, 1020),                   # the largest buffer, 1024 rows
 ])
 def test_decode_buffered_sink_and_window(dev, lens, n_sink, n_window):
     """fp16 sink + recent window next to the packed cache (the README's

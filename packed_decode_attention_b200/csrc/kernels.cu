@@ -204,20 +204,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void fill_bytetab(ByteTab& t, const float* centroids, int bits) {
-  uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
-  const int n = 1 << bits;
-  for (int e = 0; e < n; ++e) {
-    const uint32_t h = __half_as_ushort(__float2half_rn(centroids[e]));
-    lo[e >> 2] |= (h & 0xFFu) << (8 * (e & 3));
-    hi[e >> 2] |= (h >> 8) << (8 * (e & 3));
-  }
-  for (int i = 0; i < 4; ++i) {
-    t.lo[i] = lo[i];
-    t.hi[i] = hi[i];
-  }
-}
-
 // Group geometry of a K layout (record order, widest group first).
 struct GroupGeo {
   int width, d, nfull, r, word, chunk, start;

@@ -6,7 +6,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libbgtq.so")
-SOURCES = ["csrc/kernels.cu", "csrc/api.cu", "csrc/host_tables.cpp"]
+SOURCES = ["csrc/encode.cu", "csrc/decode.cu", "csrc/diag.cu", "csrc/api.cu", "csrc/host_tables.cpp"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
@@ -17,7 +17,7 @@ NVCC_FLAGS = [
 
 def sources():
     return [os.path.join(PKG, s) for s in SOURCES] + [
-        os.path.join(PKG, "csrc", h) for h in ("device_tables.h", "host_tables.h")] + [
+        os.path.join(PKG, "csrc", h) for h in ("device_tables.h", "host_tables.h", "common.cuh")] + [
         os.path.join(ROOT, "include", "bgtq.h")]
 
 

@@ -1,6 +1,6 @@
 // The C ABI declared in include/bgtq.h.  Host logic only: argument checks,
 // buffer carving, table construction and upload, kernel launches.  Every
-// step of the path itself runs in kernels.cu.
+// step of the path itself runs in the kernels (encode.cu, decode.cu, diag.cu).
 #include <cuda_runtime.h>
 
 #include <algorithm>

@@ -1,0 +1,936 @@
+// Decode kernels of the Block-GTQ path (B200, sm_100a):
+//
+//   decode_mma_kernel    split-K flash decoding from the packed tiles (mma.sync),
+//                        with the fp16 sink / window rows of a buffered call
+//   combine_kernel       log-sum-exp merge of the splits + inverse V rotation
+//
+// Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (Block-GTQ;
+// chatpaper summary / arXiv 2606.24033 abstract, blockgtq README) on top of
+// TurboQuant-MSE (arXiv 2504.19874); split-K decoding after FlashAttention /
+// FlashAttention-2 (arXiv 2205.14135, 2307.08691), both cited by the pages.
+#include "common.cuh"
+
+namespace bgtq {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// a5: split-K decode straight from the packed tiles on the tensor cores.
+//
+// Grid (batch * Hkv * head_blocks, c_max, layer_count), 128 threads.  The
+// split CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
+// its 64-position tiles; each warp has its own 2-stage bulk-copy pipeline
+// (K tile, V tile, norms -> shared memory, completion on an mbarrier) and its
+// own online-softmax state.
+//
+// Logits (per warp per tile): S^T[64 tokens x 8 heads] = K_hat q~^T as
+// mma.sync m16n8k16 tiles -- A = centroids C[codes] (exact in fp16), looked
+// up in registers with PRMT byte tables from the lane's selector words;
+// B = q~ * log2(e) split into fp16 hi + lo (two MMAs).  Each width group
+// accumulates separately and is scaled by its per-token norm.
+// P V: O^T[128 dims x 8 heads] += V_hat^T P'^T with P' = 2^(logit - max) *
+// n_V / sqrt(D) in fp16, moved from the logit accumulator layout into a B
+// operand with movmatrix.  Everything stays in V's rotated basis; the
+// combine kernel rotates back.
+// ---------------------------------------------------------------------------
+constexpr int kStages = 2;
+constexpr int kDecMinBlocks = 3;  // CTAs per SM the register budget is sized for
+constexpr int kWaitLimit = 1 << 20;  // polls of up to kPollSuspendNs each: about a second
+constexpr float kRescaleSlack = 8.f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// A hint to bring [p, p + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// One bounded poll: the thread may sleep up to kPollSuspendNs waiting for the phase.
+constexpr uint32_t kPollSuspendNs = 1000;
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kPollSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity; gives up after kWaitLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Shared memory of the buffer CTA: q of 8 heads, logits / weights [8][rows], (M, L) per head.
+constexpr int kBufSmemBytes = (8 * kD + 8 * kMaxBufferRows + 16) * 4;
+
+struct DecodeLayout {  // byte offsets inside the dynamic shared memory
+  int bars, bq, tabk, grp, pdesc, ms, ls, mres, wsc, stage, stage_bytes, total;
+};
+
+__host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
+  DecodeLayout L;
+  L.bars = 0;
+  L.bq = align128(kDecWarps * kStages * 8);
+  L.grp = L.bq + kMaxChunks * 32 * 16;    // a copy of DecodeTableDev: grp, tabk, pdesc, tabv
+  L.tabk = L.grp + kNumGroupsMax * 8 * 4;
+  L.pdesc = L.tabk + kNumGroupsMax * 8 * 4;
+  L.ms = L.grp + static_cast<int>(sizeof(DecodeTableDev));
+  L.ls = L.ms + kDecWarps * 8 * 4;
+  L.mres = L.ls + kDecWarps * 8 * 4;           // merged m, l per head [2][8]
+  L.wsc = L.mres + 2 * 8 * 4;                  // merge weights [warp][8]
+  L.stage = align128(L.wsc + kDecWarps * 8 * 4);
+  L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
+  const int stages = kDecWarps * kStages * L.stage_bytes;
+  const int merge = kDecWarps * 8 * kD * 4;  // reuses the stage buffers after the loop
+  int need = stages > merge ? stages : merge;
+  if (need < kBufSmemBytes) need = kBufSmemBytes;  // the buffer CTA of a buffered call
+  L.total = L.stage + need;
+  return L;
+}
+
+// The range of a decode call's sequence: the packed positions [lo, len) and
+// the buffered row count, clamped the same way by every kernel that reads
+// them (the combine raises the flag).
+struct SeqRange {
+  int len, lo, cnt;
+  bool bad;
+};
+
+__device__ __forceinline__ SeqRange seq_range(const Shape& sh, const int32_t* seq_lens, const BufferArgs& buf, int b) {
+  SeqRange r;
+  r.len = seq_lens[b];
+  r.lo = buf.pos_lo != nullptr ? buf.pos_lo[b] : 0;
+  r.cnt = buf.k != nullptr ? buf.count[b] : 0;
+  r.bad = r.len < 0 || r.len > sh.capacity || r.lo < 0 || r.lo > r.len || r.cnt < 0 || r.cnt > buf.n_buf;
+  if (r.len < 0 || r.len > sh.capacity) r.len = 0;
+  if (r.lo < 0 || r.lo > r.len) r.lo = r.len;
+  r.cnt = r.cnt < 0 ? 0 : (r.cnt > buf.n_buf ? buf.n_buf : r.cnt);
+  return r;
+}
+
+// Packed tiles a call attends for one sequence: the tiles of [lo, len).
+__device__ __forceinline__ int64_t range_tiles(const SeqRange& r) {
+  return r.lo < r.len ? (r.len + kTile - 1) / kTile - r.lo / kTile : 0;
+}
+
+// Split CTAs of a unit with ntl tiles when the batch has `total` tiles per
+// unit summed over its sequences (see SplitPlan).  The split pass and the
+// combine evaluate it on the same inputs, so they agree.
+__device__ __forceinline__ int split_ctas(const SplitPlan& p, int64_t ntl, int64_t total) {
+  if (ntl <= 0) return 0;
+  int64_t c = p.fixed_tiles > 0 ? (ntl + p.fixed_tiles - 1) / p.fixed_tiles
+                                : static_cast<int64_t>(p.budget) * ntl / (total * p.units_per_seq);
+  c = c < 1 ? 1 : c;
+  c = c < ntl ? c : ntl;
+  c = c < p.c_max ? c : p.c_max;
+  return static_cast<int>(c);
+}
+
+// The batch's tiles summed over its sequences, by all NT threads of the CTA
+// (red: kNtWarps int64 of shared memory).  Needed only in budget mode.
+template <int NT>
+__device__ int64_t batch_tiles(const Shape& sh, const int32_t* seq_lens, const BufferArgs& buf, int batch,
+                               int64_t* red) {
+  const int tid = threadIdx.x;
+  long long t = 0;
+  for (int b = tid; b < batch; b += NT) t += range_tiles(seq_range(sh, seq_lens, buf, b));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if ((tid & 31) == 0) red[tid >> 5] = t;
+  __syncthreads();
+  int64_t sum = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) sum += red[w];
+  __syncthreads();
+  return sum;
+}
+
+
+// The fp16 buffered rows of one (layer, sequence, KV head, block of 8 query
+// heads), attended by one extra CTA of the split pass (128 threads): logits
+// q . k / sqrt(D) in log2 units (a thread per row), softmax per head, P v (a
+// thread per dimension, unrotated).  Each head's (m, l, acc) goes to the
+// row's extra combine intermediate, which then counts as arrived.
+__device__ void buffer_attend(const Shape& sh, const Workspace& ws, const BufferArgs& buf, const SeqRange& sr, int li,
+                              int b, int h, int h0, int nh, int batch, unsigned char* smem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = sh.group;
+  float* qs = reinterpret_cast<float*>(smem);   // [128 dims][8 heads]
+  float* lg = qs + 8 * kD;                      // [8][kMaxBufferRows]
+  float* ml = lg + 8 * kMaxBufferRows;          // [8][2]
+  const int cnt = sr.cnt;
+  const size_t qrow = ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
+  for (int i = tid; i < 8 * kD; i += kDecThreads) {
+    const int hh = i / kD, dim = i % kD;
+    qs[dim * 8 + hh] = hh < nh ? __half2float(buf.q[qrow + i]) * (kInvSqrtD * kLog2e) : 0.f;
+  }
+  __syncthreads();
+  const size_t rstride = static_cast<size_t>(sh.n_kv_heads) * kD;
+  const size_t base = (static_cast<size_t>(li) * batch + b) * buf.n_buf * rstride + static_cast<size_t>(h) * kD;
+  for (int r = tid; r < cnt; r += kDecThreads) {
+    const uint4* kr = reinterpret_cast<const uint4*>(buf.k + base + r * rstride);
+    float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // half of the row's dimensions per pass: 8 loads of 8 values in flight
+#pragma unroll 1
+    for (int c8 = 0; c8 < 2; ++c8) {
+      uint4 kw[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) kw[c] = kr[8 * c8 + c];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const __half2* h2 = reinterpret_cast<const __half2*>(&kw[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float kv = e & 1 ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
+          const float4* qa = reinterpret_cast<const float4*>(qs + (8 * (8 * c8 + c) + e) * 8);
+          const float4 a0 = qa[0], a1 = qa[1];
+          d[0] = fmaf(a0.x, kv, d[0]);
+          d[1] = fmaf(a0.y, kv, d[1]);
+          d[2] = fmaf(a0.z, kv, d[2]);
+          d[3] = fmaf(a0.w, kv, d[3]);
+          d[4] = fmaf(a1.x, kv, d[4]);
+          d[5] = fmaf(a1.y, kv, d[5]);
+          d[6] = fmaf(a1.z, kv, d[6]);
+          d[7] = fmaf(a1.w, kv, d[7]);
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) lg[hh * kMaxBufferRows + r] = d[hh];
+  }
+  __syncthreads();
+  // per head: maximum, weights 2^(logit - M) in place, denominator
+  for (int hh = warp; hh < 8; hh += kDecWarps) {
+    float M = -CUDART_INF_F;
+    for (int r = lane; r < cnt; r += 32) M = fmaxf(M, lg[hh * kMaxBufferRows + r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int r = lane; r < cnt; r += 32) {
+      const float p = exp2f(lg[hh * kMaxBufferRows + r] - M);
+      lg[hh * kMaxBufferRows + r] = p;
+      L += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      ml[2 * hh] = M;
+      ml[2 * hh + 1] = L;
+    }
+  }
+  __syncthreads();
+  // P v: thread (8 dimensions dg, row phase rp of 8), 8 values per load; the
+  // phases are then summed through shared memory (over the weights)
+  const int dg = tid & 15, rp = tid >> 4;
+  float acc[8][8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+#pragma unroll 4
+  for (int r = rp; r < cnt; r += 8) {
+    const uint4 vw = *reinterpret_cast<const uint4*>(buf.v + base + r * rstride + 8 * dg);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&vw);
+    float vv[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      vv[2 * e] = f.x;
+      vv[2 * e + 1] = f.y;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      const float p = lg[hh * kMaxBufferRows + r];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vv[e], acc[hh][e]);
+    }
+  }
+  __syncthreads();
+  float* red = lg;  // [8 phases][8 heads][128 dims]
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    float4* dst = reinterpret_cast<float4*>(red + (rp * 8 + hh) * kD + 8 * dg);
+    dst[0] = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+    dst[1] = make_float4(acc[hh][4], acc[hh][5], acc[hh][6], acc[hh][7]);
+  }
+  __syncthreads();
+  const int d = tid;  // kDecThreads == kD: a thread per output dimension
+  const size_t wrow0 = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0;
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    if (hh >= nh) break;
+    float* mid = ws.comb_mid + ((wrow0 + hh) * (kCombSlices + 1) + kCombSlices) * kPartialStride;
+    float a = 0.f;
+#pragma unroll
+    for (int ph = 0; ph < 8; ++ph) a += red[(ph * 8 + hh) * kD + d];
+    mid[4 + d] = cnt > 0 ? a : 0.f;
+    if (d == 0) {
+      mid[0] = cnt > 0 ? ml[2 * hh] : -CUDART_INF_F;
+      mid[1] = cnt > 0 ? ml[2 * hh + 1] : 0.f;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  // the combine of a row with no packed position and no buffered row writes
+  // zeros without counting arrivals: do not count this one either
+  if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
+}
+
+// Grid (batch * Hkv * head_blocks, [1 buffer CTA +] plan.c_max, layer_count),
+// 128 threads.  A unit is one (layer, sequence, KV head, block of up to 8
+// query heads); it uses C = split_ctas(...) of its c_max split CTAs (more for
+// longer sequences; the others exit at once).  Its tiles are dealt
+// round-robin over the W = 4 C warps of those CTAs, CTA-major within a round
+// (warp w of CTA c takes tiles w C + c, w C + c + W, ...), so
+// every warp gets the same number of tiles to within one and the last,
+// partial round lands on as many CTAs as it can.  Each CTA writes one
+// partial (m, l, acc) per query head -- an empty one (m = -inf, l = 0) when
+// it has no tile.
+template <int VB>
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+    decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
+                      const int32_t* __restrict__ seq_lens, BufferArgs buf, int batch, SplitPlan plan,
+                      int head_blocks) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const DecodeLayout DL = decode_layout(sh.kbits, VB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
+  uint4* bq = reinterpret_cast<uint4*>(smem_raw + DL.bq);
+  uint32_t* tabk = reinterpret_cast<uint32_t*>(smem_raw + DL.tabk);
+  int32_t* grp = reinterpret_cast<int32_t*>(smem_raw + DL.grp);
+  uint32_t* pdesc = reinterpret_cast<uint32_t*>(smem_raw + DL.pdesc);
+  float* ms = reinterpret_cast<float*>(smem_raw + DL.ms);
+  float* ls = reinterpret_cast<float*>(smem_raw + DL.ls);
+  unsigned char* stage_base = smem_raw + DL.stage;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  // grid row 0 holds the buffer CTAs of a buffered call, so they are
+  // dispatched first; the split CTAs follow
+  const bool has_buf = buf.k != nullptr;
+  const int cu = has_buf ? static_cast<int>(blockIdx.y) - 1 : static_cast<int>(blockIdx.y);  // -1: buffer CTA
+  const int hb = blockIdx.x % head_blocks;
+  const int h = (blockIdx.x / head_blocks) % sh.n_kv_heads;
+  const int b = blockIdx.x / (head_blocks * sh.n_kv_heads);
+  const int li = blockIdx.z;
+  const int layer = layer0 + li;
+  const int G = sh.group;
+  const int h0 = 8 * hb;                       // first query head of this block within the group
+  const int nh = min(8, G - h0);
+  const int lh = layer * sh.n_kv_heads + h;
+  const LayoutDev& lay = ws.layouts[lh];
+
+  // ---- per-CTA set-up: the (layer, KV head) decode table (a library table) ----
+  const int ng = lay.n_groups;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(ws.dectab + lh);
+    uint4* dst = reinterpret_cast<uint4*>(grp);  // grp, tabk, pdesc, tabv are contiguous
+    for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += kDecThreads) dst[u] = src[u];
+  }
+  if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
+  __syncthreads();
+  if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  // While the previous kernel may still run: an L2 prefetch hint for this
+  // warp's first tiles, taken as if the sequence were full (the length is an
+  // input, read only after the wait).  A prefetch reads nothing into the
+  // CTA and leaves memory as it is, so a stale or unused line costs only
+  // bandwidth; the copies below still read after the wait.
+  if (lane == 0 && batch == 1 && cu >= 0) {
+    // one sequence: its split count if it were full
+    const int cg = split_ctas(plan, sh.ntiles, sh.ntiles);
+    const int Wp = cg * kDecWarps;
+    const int wp = warp * cg + cu;
+    const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
+#pragma unroll
+    for (int k = 0; k < (cu < cg ? kStages : 0); ++k) {
+      const int64_t tile = wp + static_cast<int64_t>(k) * Wp;
+      if (tile >= sh.ntiles) break;
+      const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+      if (slot < 0) break;
+      prefetch_l2(cache.ktile + slot * (kb / 4), kb);
+      prefetch_l2(cache.vtile + slot * (vb / 4), vb);
+      prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
+      prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
+    }
+  }
+  // Launched as a programmatic dependent of the previous kernel (the query
+  // rotation): everything above reads only the library's tables; the
+  // sequence lengths, rotated queries and cache are read after that kernel
+  // has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the unit's q~ fragments (written by the query rotation): their loads go
+  // out with the length reads below and land in shared memory further down
+  const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+  constexpr int kFragPerThread = (kFragEntries + kDecThreads - 1) / kDecThreads;
+  uint4 fr[kFragPerThread];
+  if (qrot == nullptr && cu >= 0) {
+    const uint4* src = frag_block(sh, ws, li, b, h, hb);
+#pragma unroll
+    for (int i = 0; i < kFragPerThread; ++i) {
+      const int u = tid + i * kDecThreads;
+      if (u < 32 * nchunk) fr[i] = src[u];
+    }
+  }
+  // the packed positions attended: [lo, len); lo > 0 when the caller keeps the
+  // first positions unquantised (out-of-range values are flagged by the
+  // combine kernel)
+  const SeqRange sr = seq_range(sh, seq_lens, buf, b);
+  if (cu < 0) {
+    // the extra CTA of a buffered call: the unit's fp16 buffered rows
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    buffer_attend(sh, ws, buf, sr, li, b, h, h0, nh, batch, smem_raw + DL.stage);
+    return;
+  }
+  const int len = sr.len, lo = sr.lo;
+  const int tlo = lo / kTile;
+  const int ntl = static_cast<int>(range_tiles(sr));
+  // this unit's split CTAs (the same count the combine computes)
+  __shared__ int64_t s_red[kDecWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kDecThreads>(sh, seq_lens, buf, batch, s_red);
+  const int C = split_ctas(plan, ntl, total);
+  if (cu >= C) {
+    // not needed for this unit (its partials are slots 0 .. C-1)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  // Tile t of the unit goes to warp (t mod W) / C of CTA (t mod W) mod C:
+  // a partial last round of tiles is spread over all CTAs (and so over all
+  // SMs) before any CTA gets a second one.
+  const int W = C * kDecWarps;
+  const int wu = warp * C + cu;
+  const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
+  float* part_base = ws.partials +
+                     (((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0) * sh.max_splits + cu) *
+                         kPartialStride;
+  const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
+  {
+    if (qrot == nullptr) {
+#pragma unroll
+      for (int i = 0; i < kFragPerThread; ++i) {
+        const int u = tid + i * kDecThreads;
+        if (u < 32 * nchunk) bq[u] = fr[i];
+      }
+    } else {
+      // the split pass on its own: the fragments from the caller's q~
+      // (fp32, record order): coordinates 16 j + 4 t .. + 3 of chunk c's
+      // group for head t / 4 ... see write_frags for the layout
+      const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
+      for (int u = tid; u < 32 * nchunk; u += kDecThreads) {
+        const int c = u >> 5, ln = u & 31;
+        int g = 0;
+        while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
+        const int j = c - lay.chunk_base[g];
+        const int d = lay.size[g], st = lay.start[g];
+        const int head = ln >> 2;
+        float v[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int coord = 16 * j + 4 * (ln & 3) + m;
+          v[m] = (head < nh && coord < d) ? qsrc[head * kD + st + coord] * kLog2e : 0.f;
+        }
+        const __half2 a = __floats2half2_rn(v[0], v[1]);
+        const __half2 c2 = __floats2half2_rn(v[2], v[3]);
+        const float2 af = __half22float2(a), cf = __half22float2(c2);
+        const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
+        const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
+        bq[u] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&c2),
+                           *reinterpret_cast<const uint32_t*>(&al), *reinterpret_cast<const uint32_t*>(&cl));
+      }
+    }
+  }
+  ByteTab tv;
+  {
+    const uint4 a0 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32);
+    const uint4 a1 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32 + 4);
+    tv.lo[0] = a0.x; tv.lo[1] = a0.y; tv.lo[2] = a0.z; tv.lo[3] = a0.w;
+    tv.hi[0] = a1.x; tv.hi[1] = a1.y; tv.hi[2] = a1.z; tv.hi[3] = a1.w;
+  }
+  __syncthreads();
+
+  // ---- per-warp pipeline over this warp's tiles ----
+  const int kwords = 256 * sh.kbits, vwords = 256 * VB;
+  const uint32_t kbytes = 4u * kwords, vbytes = 4u * vwords;
+  const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
+  unsigned char* my_stage = stage_base + static_cast<size_t>(warp) * kStages * DL.stage_bytes;
+  uint64_t* my_bars = bars + warp * kStages;
+
+  auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
+    const int tile = tlo + wu + k * W;
+    int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+    if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
+      atomicOr(ws.err, kErrPage);
+      slot = static_cast<int64_t>(layer * sh.n_kv_heads + h) * cache.n_pages;
+    }
+    unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
+    uint64_t* bar = &my_bars[k % kStages];
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(bar, stage_tx);
+    bulk_copy_g2s(dst, cache.ktile + slot * kwords, kbytes, bar);
+    bulk_copy_g2s(dst + kbytes, cache.vtile + slot * vwords, vbytes, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes, cache.knorm + slot * kTile * 4, kTile * 8, bar);
+    bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, cache.vnorm + slot * kTile, kTile * 2, bar);
+  };
+  if (lane == 0)
+    for (int k = 0; k < kStages && k < my_tiles; ++k) issue(k);
+
+  float O[8][4];
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) O[m][r] = 0.f;
+  float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
+  int failed_at = -1;
+
+  for (int k = 0; k < my_tiles; ++k) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&my_bars[k % kStages], (k / kStages) & 1))) {
+      failed_at = k;
+      break;
+    }
+    const unsigned char* st = my_stage + (k % kStages) * DL.stage_bytes;
+    const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
+    const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
+    const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
+    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
+    const int tpos = (tlo + wu + k * W) * kTile;
+    const int nvalid = min(kTile, len - tpos);       // positions [nlow, nvalid) of the tile are attended
+    const int nlow = max(0, lo - tpos);
+
+    // logits, one width group at a time, each scaled by its per-token norm
+    float L[4][4];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) L[mu][r] = 0.f;
+    for (int g = 0; g < ng; ++g) {
+      const int4 gp = *reinterpret_cast<const int4*>(grp + g * 8);  // width, nfull, r, word
+      const int chunk = grp[g * 8 + 4];
+      ByteTab t;
+      const uint4 tl = *reinterpret_cast<const uint4*>(tabk + 8 * g);
+      const uint4 th = *reinterpret_cast<const uint4*>(tabk + 8 * g + 4);
+      t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
+      t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+      const uint32_t pd = pdesc[g * 32 + lane];
+      const uint32_t* gw = kt + gp.w;
+      const uint4* bqg = bq + chunk * 32 + lane;
+      float S[4][4];
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) S[mu][r] = 0.f;
+      switch (gp.x) {
+        case 1: group_logits<1>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 2: group_logits<2>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 3: group_logits<3>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        default: group_logits<4>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+      }
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
+        const float nb = __half2float(kn[(16 * mu + g8 + 8) * 4 + g]);
+        L[mu][0] = fmaf(na, S[mu][0], L[mu][0]);
+        L[mu][1] = fmaf(na, S[mu][1], L[mu][1]);
+        L[mu][2] = fmaf(nb, S[mu][2], L[mu][2]);
+        L[mu][3] = fmaf(nb, S[mu][3], L[mu][3]);
+      }
+    }
+    // online softmax over the tile for heads 2*t4 and 2*t4+1; positions past
+    // the valid length carry no weight (their norms may be anything)
+    float wv[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      wv[mu][0] = __half2float(vn[16 * mu + g8]) * kInvSqrtD;
+      wv[mu][1] = __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD;
+    }
+    if (nvalid < kTile || nlow > 0) {
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        if (16 * mu + g8 >= nvalid || 16 * mu + g8 < nlow) {
+          L[mu][0] = L[mu][1] = -CUDART_INF_F;
+          wv[mu][0] = 0.f;
+        }
+        if (16 * mu + g8 + 8 >= nvalid || 16 * mu + g8 + 8 < nlow) {
+          L[mu][2] = L[mu][3] = -CUDART_INF_F;
+          wv[mu][1] = 0.f;
+        }
+      }
+    }
+    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
+      mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
+    }
+    // The reference maximum moves only when some logit of the tile exceeds it
+    // by more than kRescaleSlack (log2 units), so O is rescaled rarely;
+    // weights stay <= 2^kRescaleSlack and l and O always share the same
+    // reference.  l is kept per lane and summed over the warp at the end.
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kRescaleSlack || mx[1] > m_run[1] + kRescaleSlack)) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
+      }
+      float alpha[2] = {1.f, 1.f};
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (mx[c] > m_run[c] + kRescaleSlack) {
+          alpha[c] = fast_exp2(m_run[c] - mx[c]);
+          m_run[c] = mx[c];
+        }
+        l_run[c] *= alpha[c];
+      }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        O[m][0] *= alpha[0];
+        O[m][1] *= alpha[1];
+        O[m][2] *= alpha[0];
+        O[m][3] *= alpha[1];
+      }
+    }
+    uint32_t bp[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
+      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
+      l_run[0] += p0 + p2;
+      l_run[1] += p1 + p3;
+      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
+      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
+    }
+    // P V in V's rotated basis
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      uint32_t w[VB], sv[4];
+#pragma unroll
+      for (int kk = 0; kk < VB; ++kk) w[kk] = vt[m * 32 * VB + 32 * kk + lane];
+      quartet_decode<VB>(w, sv);
+#pragma unroll
+      for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
+    }
+    __syncwarp();
+    if (lane == 0 && k + kStages < my_tiles) issue(k + kStages);
+  }
+  // the combine kernel may be scheduled now; it waits for this grid before reading the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const bool timed_out = failed_at >= 0;
+  if (timed_out) {
+    if (lane == 0) atomicOr(ws.err, kErrTimeout);
+    // copies issued but not yet consumed: let them land (bounded) before the
+    // stage buffers are reused or the CTA exits
+    const int issued = min(my_tiles, failed_at + kStages);
+    for (int k = failed_at; k < issued; ++k) mbar_wait(&my_bars[k % kStages], (k / kStages) & 1);
+  }
+  __syncthreads();
+  // ---- merge the warps (the stage buffers are reused) ----
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
+  }
+  float* accs = reinterpret_cast<float*>(stage_base);  // [warp][8 heads][128]
+  if (g8 == 0) {
+    ms[warp * 8 + 2 * t4] = m_run[0];
+    ms[warp * 8 + 2 * t4 + 1] = m_run[1];
+    ls[warp * 8 + 2 * t4] = l_run[0];
+    ls[warp * 8 + 2 * t4 + 1] = l_run[1];
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    float* a = accs + warp * 8 * kD;
+    a[(2 * t4) * kD + 16 * m + g8] = O[m][0];
+    a[(2 * t4 + 1) * kD + 16 * m + g8] = O[m][1];
+    a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
+    a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
+  }
+  if (__syncthreads_or(timed_out)) return;
+  // per head: the common maximum, the warps' weights (warps without a tile
+  // hold m = -inf, l = 0, acc = 0) and the weighted denominator
+  float* wsc = reinterpret_cast<float*>(smem_raw + DL.wsc);
+  float* mres = reinterpret_cast<float*>(smem_raw + DL.mres);
+  if (tid < 8) {
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
+    float lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float mw = ms[w * 8 + tid];
+      const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
+      wsc[w * 8 + tid] = sc;
+      lsum = fmaf(sc, ls[w * 8 + tid], lsum);
+    }
+    mres[tid] = M;
+    mres[8 + tid] = lsum;
+  }
+  __syncthreads();
+  const int i = tid;
+  for (int hh = 0; hh < nh; ++hh) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) a = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a);
+    float* part = part_base + hh * part_head_stride;
+    part[4 + i] = a;
+    if (i == 0) {
+      part[0] = mres[hh];
+      part[1] = mres[8 + hh];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq *
+// kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
+// (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated coordinates) into
+// an intermediate (m, l, acc) in V's rotated basis.  In a buffered call the
+// split pass has already posted the row's fp16 buffered rows as one more
+// intermediate (acc unrotated).  The row's last CTA to finish (an arrival
+// counter, reset by that CTA) merges them:
+// o = (R_V^T sum_s w_s acc_s + w_buf acc_buf) / (sum_s w_s l_s + w_buf l_buf).
+// ---------------------------------------------------------------------------
+constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
+// Up to this many rows per launch, every combine CTA loads its rotation
+// column early (8 slices x 64 KB per row of L2 reads).
+constexpr int kEarlyRotationRows = 256;
+static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates four at a time");
+
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
+                                                               const int32_t* __restrict__ seq_lens, int batch,
+                                                               SplitPlan plan, BufferArgs buf, __half* __restrict__ out,
+                                                               bool early_rotation) {
+  const int has_buf = buf.k != nullptr ? 1 : 0;
+  const int slice = blockIdx.x % kCombSlices;
+  const int rowi = blockIdx.x / kCombSlices;
+  const int hq = rowi % sh.n_q_heads;
+  const int b = (rowi / sh.n_q_heads) % batch;
+  const int li = rowi / (sh.n_q_heads * batch);
+  const int layer = layer0 + li;
+  const int kvh = hq / sh.group;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dd = tid & (kD - 1), half = tid >> 7;
+  // A library table: this thread's half column of the inverse V rotation,
+  // used if this CTA merges the row.  For a small launch every CTA reads it
+  // before the split pass has finished, off the critical path; for a large
+  // one (many layers per call) only the merging CTAs do, later.
+  const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  float mvr[64];
+  if (early_rotation) {
+#pragma unroll
+    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+  }
+  // the next kernel of the stream may start its own table-only set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Launched as a programmatic dependent of the split pass: inputs, partials
+  // and the output are touched only after that kernel has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const SeqRange sr = seq_range(sh, seq_lens, buf, b);
+  if (sr.bad && tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
+  const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
+  if (sr.lo >= sr.len && sr.cnt == 0) {
+    if (slice == 0 && tid < kD) out[row * kD + tid] = __float2half(0.f);
+    return;
+  }
+  const size_t wrow = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + hq;  // workspace row
+  const float* part = ws.partials + wrow * sh.max_splits * kPartialStride;
+  __shared__ float accs[kCombWarps][kD];
+  __shared__ float msw[kCombWarps], lsw[kCombWarps];
+  __shared__ float a_s[kD];
+  __shared__ int last;
+  float* mid = ws.comb_mid + (wrow * (kCombSlices + 1) + slice) * kPartialStride;
+  // ---- one slice of the row's splits: warp w takes splits s0 + w + 8 j,
+  // four at a time with all their loads in flight, merged online per warp
+  // (lane = 4 rotated coordinates), then across the warps ----
+  __shared__ int64_t s_red[kCombWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kCombThreads>(sh, seq_lens, buf, batch, s_red);
+  const int n_splits = split_ctas(plan, range_tiles(sr), total);
+  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
+  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
+  float m_w = -CUDART_INF_F, l_w = 0.f;
+  float4 a_w = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int base = s0 + warp; base < s1; base += 4 * kCombWarps) {
+    float mm[4], ll[4];
+    float4 aa[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int sj = base + j * kCombWarps;
+      if (sj < s1) {
+        const float* p = part + static_cast<size_t>(sj) * kPartialStride;
+        mm[j] = p[0];
+        ll[j] = p[1];
+        aa[j] = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+      } else {
+        mm[j] = -CUDART_INF_F;
+        ll[j] = 0.f;
+        aa[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const float mb = fmaxf(fmaxf(m_w, fmaxf(mm[0], mm[1])), fmaxf(mm[2], mm[3]));
+    if (mb == -CUDART_INF_F) continue;  // only empty splits so far
+    const float f = m_w == -CUDART_INF_F ? 0.f : exp2f(m_w - mb);
+    l_w *= f;
+    a_w.x *= f; a_w.y *= f; a_w.z *= f; a_w.w *= f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float wgt = mm[j] == -CUDART_INF_F ? 0.f : exp2f(mm[j] - mb);
+      l_w = fmaf(wgt, ll[j], l_w);
+      a_w.x = fmaf(wgt, aa[j].x, a_w.x);
+      a_w.y = fmaf(wgt, aa[j].y, a_w.y);
+      a_w.z = fmaf(wgt, aa[j].z, a_w.z);
+      a_w.w = fmaf(wgt, aa[j].w, a_w.w);
+    }
+    m_w = mb;
+  }
+  *reinterpret_cast<float4*>(&accs[warp][4 * lane]) = a_w;
+  if (lane == 0) {
+    msw[warp] = m_w;
+    lsw[warp] = l_w;
+  }
+  __syncthreads();
+  {
+    float M = msw[0];
+#pragma unroll
+    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, msw[w]);
+    if (tid < kD) {
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) {
+        const float wgt = msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M);
+        a = fmaf(wgt, accs[w][tid], a);
+      }
+      mid[4 + tid] = a;
+    }
+    if (tid == 0) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) l = fmaf(msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M), lsw[w], l);
+      mid[0] = M;
+      mid[1] = l;
+    }
+  }
+  // ---- the row's last CTA merges the intermediates ----
+  const int nmid = kCombSlices + has_buf;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == static_cast<unsigned>(nmid - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* mids = ws.comb_mid + wrow * (kCombSlices + 1) * kPartialStride;
+  float mk[kCombSlices + 1], lk[kCombSlices + 1], ak[kCombSlices + 1];
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) {
+    if (k < nmid) {
+      mk[k] = __ldcg(mids + k * kPartialStride);
+      lk[k] = __ldcg(mids + k * kPartialStride + 1);
+      ak[k] = __ldcg(mids + k * kPartialStride + 4 + dd);
+    } else {
+      mk[k] = -CUDART_INF_F;
+      lk[k] = 0.f;
+      ak[k] = 0.f;
+    }
+  }
+  float Mt = -CUDART_INF_F;
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) Mt = fmaxf(Mt, mk[k]);
+  float Lt = 0.f, at = 0.f, ab = 0.f;
+#pragma unroll
+  for (int k = 0; k <= kCombSlices; ++k) {
+    const float w = mk[k] == -CUDART_INF_F ? 0.f : exp2f(mk[k] - Mt);
+    Lt = fmaf(w, lk[k], Lt);
+    if (k < kCombSlices) at = fmaf(w, ak[k], at);  // rotated basis
+    else ab = w * ak[k];                            // the buffer's rows, unrotated
+  }
+  if (tid < kD) a_s[tid] = at / Lt;
+  if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
+  if (!early_rotation) {
+#pragma unroll
+    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+  }
+  __syncthreads();
+  // inverse V rotation: two threads per output, half of the inputs each
+  float o = 0.f;
+#pragma unroll
+  for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
+  if (half == 1) accs[0][dd] = o;
+  __syncthreads();
+  if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
+}
+
+template <int VB>
+cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                             const float* qrot, const int32_t* seq_lens, const BufferArgs& buf, int batch,
+                             const SplitPlan& plan, cudaStream_t stream) {
+  // the largest layout over K widths, so one attribute value serves every call
+  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
+  if (attr != cudaSuccess) return attr;
+  const int head_blocks = (s.group + 7) / 8;
+  // units fastest, then split index: the CTAs every unit uses come first
+  dim3 grid(batch * s.n_kv_heads * head_blocks, (buf.k != nullptr ? 1 : 0) + plan.c_max, layer_count);
+  return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
+                          ws, cache, layer0, qrot, seq_lens, buf, batch, plan, head_blocks);
+}
+
+template <int VB>
+int ctas_per_sm_vb(const Shape& s) {
+  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
+  if (attr != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<VB>, kDecThreads,
+                                                    decode_layout(s.kbits, VB).total) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+}  // namespace
+
+int decode_ctas_per_sm(const Shape& s) {
+  switch (s.vbits) {
+    case 1: return ctas_per_sm_vb<1>(s);
+    case 2: return ctas_per_sm_vb<2>(s);
+    case 3: return ctas_per_sm_vb<3>(s);
+    default: return ctas_per_sm_vb<4>(s);
+  }
+}
+
+cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const float* qrot, const int32_t* seq_lens, const BufferArgs& buf,
+                                int batch, const SplitPlan& plan, cudaStream_t stream) {
+  switch (s.vbits) {
+    case 1: return launch_decode_vb<1>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    case 2: return launch_decode_vb<2>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    case 3: return launch_decode_vb<3>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+    default: return launch_decode_vb<4>(s, ws, cache, layer0, layer_count, qrot, seq_lens, buf, batch, plan, stream);
+  }
+}
+
+cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
+                           const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
+                           __half* out, cudaStream_t stream) {
+  const int nsl = kCombSlices;  // the buffered rows, if any, come from the split pass
+  const int rows = layer_count * batch * s.n_q_heads;
+  return launch_dependent(combine_kernel, dim3(rows * nsl), dim3(kCombThreads), 0, stream, s, ws, layer0, seq_lens,
+                          batch, plan, buf, out, rows <= kEarlyRotationRows);
+}
+
+}  // namespace bgtq

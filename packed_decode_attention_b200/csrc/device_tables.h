@@ -1,5 +1,5 @@
 // Device-side table formats and kernel launch parameters shared by the
-// kernels (kernels.cu) and the C ABI (api.cu).
+// kernels (encode.cu, decode.cu, diag.cu, common.cuh) and the C ABI (api.cu).
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -107,7 +107,7 @@ constexpr uint32_t kErrNonFinite = 8;
 constexpr uint32_t kErrTimeout = 16;
 constexpr uint32_t kErrPage = 32;
 
-// Launchers (kernels.cu).  Each returns the cudaError_t of its launch.
+// Launchers (encode.cu, decode.cu, diag.cu).  Each returns the cudaError_t of its launch.
 cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,
                           const __half* calib_k, int nk, int pairing, cudaStream_t stream);
 cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,

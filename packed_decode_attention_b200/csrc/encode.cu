@@ -1,0 +1,676 @@
+// Kernels of the Block-GTQ path that write the cache or prepare a query
+// (B200, sm_100a):
+//
+//   energy_kernel        label-free per-RoPE-block Q/K energy, exact 128-bit sums
+//   encode_kernel        TQ-MSE: rotate (fp32), normalise (fp64), quantise, pack tiles
+//   append_kernel        the same for a few rows: patch only their code bits
+//   rotate_query_kernel  q~ per width group (rotated basis, 1/sqrt(d_g), 1/sqrt(D))
+//   prep_kernel          a decode step's appends and query rotation in one launch
+//
+// Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (Block-GTQ;
+// chatpaper summary / arXiv 2606.24033 abstract, blockgtq README) on top of
+// TurboQuant-MSE (arXiv 2504.19874); split-K decoding after FlashAttention /
+// FlashAttention-2 (arXiv 2205.14135, 2307.08691), both cited by the pages.
+#include "common.cuh"
+
+namespace bgtq {
+
+namespace {
+
+__device__ __forceinline__ uint64_t fp16_fixed(uint16_t bits, uint32_t* nonfinite) {
+  // |x| * 2^24 for a binary16 x: subnormals are m * 2^-24, normals
+  // (1024 + m) * 2^(e - 25).
+  const uint32_t e = (bits >> 10) & 31u;
+  const uint32_t m = bits & 1023u;
+  if (e == 31u) {
+    *nonfinite = 1u;
+    return 0;
+  }
+  if (e == 0u) return m;
+  return static_cast<uint64_t>(1024u + m) << (e - 1u);
+}
+
+// ---------------------------------------------------------------------------
+// a1: energy.  Grid (L * Hkv, kEnergyChunks), 128 threads = one per dim.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ q, int nq,
+                                                     const __half* __restrict__ k, int nk, int Hq,
+                                                     int Hkv, int G, int L, int pairing,
+                                                     unsigned __int128* __restrict__ eq,
+                                                     unsigned __int128* __restrict__ ek,
+                                                     uint32_t* err) {
+  const int layer = blockIdx.x / Hkv;
+  const int h = blockIdx.x % Hkv;
+  const int c = blockIdx.y;
+  const int d = threadIdx.x;
+  const int rq = (nq + kEnergyChunks - 1) / kEnergyChunks;
+  const int rk = (nk + kEnergyChunks - 1) / kEnergyChunks;
+  uint32_t bad = 0;
+  unsigned __int128 sq = 0, sk = 0;
+  const unsigned short* qb = reinterpret_cast<const unsigned short*>(q);
+  const unsigned short* kb = reinterpret_cast<const unsigned short*>(k);
+  const int rq_end = min(nq, (c + 1) * rq);
+  for (int r = c * rq; r < rq_end; ++r) {
+    const size_t row = (static_cast<size_t>(layer) * nq + r) * Hq + static_cast<size_t>(h) * G;
+    for (int gh = 0; gh < G; ++gh) {
+      const uint64_t x = fp16_fixed(qb[(row + gh) * kD + d], &bad);
+      sq += static_cast<unsigned __int128>(x) * x;
+    }
+  }
+  const int rk_end = min(nk, (c + 1) * rk);
+  for (int r = c * rk; r < rk_end; ++r) {
+    const size_t row = (static_cast<size_t>(layer) * nk + r) * Hkv + h;
+    const uint64_t x = fp16_fixed(kb[row * kD + d], &bad);
+    sk += static_cast<unsigned __int128>(x) * x;
+  }
+  __shared__ unsigned __int128 s_q[kD], s_k[kD];
+  s_q[d] = sq;
+  s_k[d] = sk;
+  __syncthreads();
+  if (d < kD / 2) {
+    const int a = pairing == 0 ? d : 2 * d;
+    const int b = pairing == 0 ? d + kD / 2 : 2 * d + 1;
+    const size_t o = ((static_cast<size_t>(c) * L + layer) * Hkv + h) * (kD / 2) + d;
+    eq[o] = s_q[a] + s_q[b];
+    ek[o] = s_k[a] + s_k[b];
+  }
+  if (bad) atomicOr(err, kErrNonFinite);
+}
+
+
+// ---------------------------------------------------------------------------
+// a3: encode.  Grid (layer_count * batch * Hkv, per_unit, 2 kinds), 256
+// threads.  A CTA loads one (layer, KV head, kind)'s rotation and tables once
+// and then takes every per_unit-th 64-position tile that the call writes for
+// one sequence: it unpacks the tile's codes when the call writes only part of
+// it, encodes its new rows (y = R x in fp32, norms in fp64, u = sqrt(d) y /
+// n, code = #{thresholds <= u}) into the codes, and packs the tile again.
+// ---------------------------------------------------------------------------
+constexpr int kEncThreads = 256;
+// Column of element (coordinate j, row r) in xt[j][]: float4 groups of 4 rows,
+// XOR-swizzled by j so that the transposed writes spread over the banks.
+__device__ __forceinline__ int xt_col(int j, int r) { return (((r >> 2) ^ ((j >> 3) & 15)) << 2) | (r & 3); }
+
+// The Lloyd-Max code of u for width w >= 1: the number of the 2^w - 1
+// ascending thresholds t[] that are <= u (ties go up), by binary search.
+__device__ __forceinline__ int lloyd_code(const float* t, int w, float u) {
+  int c = 0;
+  for (int s = 1 << (w - 1); s > 0; s >>= 1)
+    if (t[c + s - 1] <= u) c += s;
+  return c;
+}
+
+struct EncodeSmem {
+  float xt[kD][kTile];           // new rows, transposed, record order (zero elsewhere), columns xt_col
+  float mt[kD][kD];              // mt[j][c(i)] = R[i][j] (record order), c(8 o + 4 q + e) = 64 q + 4 o + e
+  float fac[kTile][kNumGroupsMax];
+  __half nrm[kTile][kNumGroupsMax];
+  uint8_t codes[kTile][kCodePitch];
+  uint32_t words[1024];
+  float thr[5][16];
+  int32_t inv[kD];
+  int32_t gof[kD];               // group of each record position (-1: width 0)
+  LayoutDev lay;
+};
+
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                             const __half* __restrict__ kx,
+                                                             const __half* __restrict__ vx,
+                                                             const int32_t* __restrict__ start_v,
+                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  EncodeSmem& S = *reinterpret_cast<EncodeSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int kind = blockIdx.z;
+  const int h = blockIdx.x % sh.n_kv_heads;
+  const int b = (blockIdx.x / sh.n_kv_heads) % batch;
+  const int li = blockIdx.x / (sh.n_kv_heads * batch);
+  const int layer = layer0 + li;
+  const int start = start_v[b];
+  const int count = count_v[b];
+  if (start < 0 || count < 0 || count > n) {
+    if (tid == 0 && blockIdx.y == 0 && kind == 0) atomicOr(ws.err, kErrArg);
+    return;
+  }
+  if (count == 0) return;
+  int64_t p_end = static_cast<int64_t>(start) + count;  // rows land at [start, p_end)
+  if (p_end > sh.capacity) {
+    if (tid == 0 && blockIdx.y == 0) atomicOr(ws.err, kErrCapacity);
+    p_end = sh.capacity;
+  }
+  const int64_t t_first = start / kTile;
+  if (t_first + blockIdx.y >= (p_end + kTile - 1) / kTile) return;  // no tile for this CTA
+  const int bits_avg = kind == 0 ? sh.kbits : sh.vbits;
+  const int nwords = 256 * bits_avg;
+  const int lh = layer * sh.n_kv_heads + h;
+  if (kind == 0) {
+    if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
+      reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
+  } else if (tid == 0) {
+    S.lay.n_groups = 1;
+    S.lay.n_positions = kD;
+    for (int g = 0; g < kNumGroupsMax; ++g) {
+      S.lay.width[g] = g == 0 ? sh.vbits : 0;
+      S.lay.size[g] = g == 0 ? kD : 0;
+      S.lay.start[g] = g == 0 ? 0 : kD;
+      S.lay.bitoff[g] = 0;
+      S.lay.tile_word[g] = 0;
+      S.lay.chunk_base[g] = 0;
+    }
+  }
+  for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
+  const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
+  // columns swizzled so that the 16 output groups of a warp read the first
+  // and the second half of their 8 columns as two contiguous 256-byte spans
+  for (int i = tid; i < kD * kD / 4; i += kEncThreads) {
+    const int j = i / (kD / 4), c4 = i % (kD / 4);  // float4 c4 of row j: columns 4 c4 .. 4 c4 + 3
+    const int o = c4 >> 1, q = c4 & 1;
+    reinterpret_cast<float4*>(&S.mt[j][0])[q * 16 + o] = reinterpret_cast<const float4*>(mglob)[i];
+  }
+  __syncthreads();
+  const int ng = S.lay.n_groups;
+  const int npos = S.lay.n_positions;
+  if (tid < kD) {
+    S.inv[kind == 0 ? S.lay.perm[tid] : tid] = tid;
+    int g = -1;
+    if (tid < npos) {
+      g = 0;
+      for (int t = 1; t < ng; ++t)
+        if (tid >= S.lay.start[t]) g = t;
+    }
+    S.gof[tid] = g;
+  }
+  __syncthreads();
+  // ---- this CTA's tiles: t_first + blockIdx.y, then every gridDim.y-th ----
+  for (int64_t tile = t_first + blockIdx.y; tile * kTile < p_end; tile += gridDim.y) {
+    const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
+    const int64_t p1 = min(tile * kTile + kTile, p_end);
+    const int tr0 = static_cast<int>(p0 - tile * kTile), tr1 = static_cast<int>(p1 - tile * kTile);
+    const bool whole = (tr0 == 0 && tr1 == kTile);
+    if (p0 >= p1) continue;  // the first rows are past the capacity
+    const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+    if (slot < 0) {  // uniform over the CTA
+      if (tid == 0) atomicOr(ws.err, kErrPage);
+      continue;
+    }
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
+    // existing codes of a partly written tile
+    if (!whole) {
+      if (kind == 0) {
+        for (int g = 0; g < ng; ++g) {
+          const GroupGeo q = group_geo(S.lay, g);
+          BGTQ_WIDTH_SWITCH(q.width, unpack_k_group, gtile, q, S.codes, tid, kEncThreads)
+        }
+      } else {
+        BGTQ_WIDTH_SWITCH(sh.vbits, unpack_v_tile, gtile, S.codes, tid, kEncThreads)
+      }
+    }
+    __syncthreads();
+    // new rows -> xt (record order)
+    const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
+    const __half* x = kind == 0 ? kx : vx;
+    const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
+                          static_cast<size_t>(h) * kD;
+    for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
+      const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (r >= tr0 && r < tr1)
+        raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+  #pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(h2[k]);
+        const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
+        S.xt[j0][xt_col(j0, r)] = f.x;
+        S.xt[j1][xt_col(j1, r)] = f.y;
+      }
+    }
+    __syncthreads();
+    // norms: fp64 sum of squares of the exact fp16 inputs
+    {
+      const int r = tid >> 2, g = tid & 3;
+      float f = 0.f;
+      __half nh = __float2half(0.f);
+      if (g < ng && r >= tr0 && r < tr1) {
+        const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
+        double s2 = 0.0;
+        for (int j = j0; j < j1; ++j) {
+          const double v = S.xt[j][xt_col(j, r)];
+          s2 += v * v;
+        }
+        const double nr = sqrt(s2);
+        nh = __double2half(nr);
+        f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;
+      }
+      S.fac[r][g] = f;
+      S.nrm[r][g] = nh;
+    }
+    __syncthreads();
+    // y = R x per new row (fp32, coordinate order), then the codes
+    {
+      // register tile: 4 rows x 8 outputs per thread over all 64 rows
+      const int rg = tid >> 4, og = tid & 15;
+      const int i0 = og * 8;
+      if (i0 < npos && rg * 4 < tr1 && rg * 4 + 4 > tr0) {
+        int gi[8];
+  #pragma unroll
+        for (int q = 0; q < 8; ++q) gi[q] = S.gof[i0 + q];
+        int ghi = gi[0];
+  #pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (gi[q] > ghi) ghi = gi[q];
+        const int jlo = S.lay.start[gi[0]];
+        const int jhi = S.lay.start[ghi] + S.lay.size[ghi];
+        float acc[4][8];
+  #pragma unroll
+        for (int a = 0; a < 4; ++a)
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) acc[a][q] = 0.f;
+  #pragma unroll 4
+        for (int j = jlo; j < jhi; ++j) {
+          const float4 xv = *reinterpret_cast<const float4*>(&S.xt[j][4 * (rg ^ ((j >> 3) & 15))]);
+          const float4 m0 = *reinterpret_cast<const float4*>(&S.mt[j][4 * og]);
+          const float4 m1 = *reinterpret_cast<const float4*>(&S.mt[j][64 + 4 * og]);
+          const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+          const float ms[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+  #pragma unroll
+          for (int a = 0; a < 4; ++a)
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) acc[a][q] = fmaf(xs[a], ms[q], acc[a][q]);
+        }
+  #pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int r = rg * 4 + a;
+          if (r < tr0 || r >= tr1) continue;
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int g = gi[q];
+            if (g < 0) continue;
+            const int w = S.lay.width[g];
+            const float u = acc[a][q] * S.fac[r][g];
+            S.codes[r][i0 + q] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // repack the tile and write it back
+    if (kind == 0) {
+      for (int g = 0; g < ng; ++g) {
+        const GroupGeo q = group_geo(S.lay, g);
+        BGTQ_WIDTH_SWITCH(q.width, pack_k_group, S.words, q, S.codes, tid, kEncThreads)
+      }
+    } else {
+      BGTQ_WIDTH_SWITCH(sh.vbits, pack_v_tile, S.words, S.codes, tid, kEncThreads)
+    }
+    __syncthreads();
+    for (int i = tid; i < nwords / 4; i += kEncThreads)
+      reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
+    if (tid >= tr0 && tid < tr1) {
+      const size_t pos = static_cast<size_t>(slot) * kTile + tid;
+      if (kind == 0) {
+        __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
+        dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
+        dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
+      } else {
+        cache.vnorm[pos] = S.nrm[tid][0];
+      }
+    }
+
+    __syncthreads();  // the buffers are reused by the next tile
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3 for a few rows (decode-time appends): grid (layer_count * batch * Hkv,
+// n, 2 kinds), 128 threads.  A CTA encodes one new row of one (layer,
+// sequence, KV head) and kind with the same arithmetic as encode_kernel
+// (norms summed in fp64 in coordinate order, y = sum_j R[i][j] x_j in fp32
+// in coordinate order from the group's first coordinate, u = y * sqrt(d) /
+// ||x||, code = #{thresholds <= u}) and rewrites only that row's code bits
+// in the packed tile, with global atomics: bits of other positions are never
+// touched, so rows appended by different CTAs to the same tile do not race.
+// ---------------------------------------------------------------------------
+constexpr int kAppThreads = 128;
+
+// Plane word (0..b-1) and bit of code bit q of selector sel, nibble n, in a
+// quartet of width b (see the quartet formulas above).
+__device__ __forceinline__ void quartet_bit(int b, int sel, int n, int q, int& k, int& bit) {
+  if (b == 4) {
+    k = sel;
+    bit = 4 * n + q;
+  } else if (b == 1) {
+    k = 0;
+    bit = 4 * n + sel;
+  } else if (q < 2) {
+    k = sel >> 1;
+    bit = 4 * n + 2 * (sel & 1) + q;
+  } else {
+    k = 2;
+    bit = 4 * n + sel;
+  }
+}
+
+// Word (relative to the tile) of plane k for a K code, and the selector
+// and nibble it sits in: token p (0..63), coordinate c of group g.
+__device__ __forceinline__ int k_code_word(const LayoutDev& lay, int g, int c, int p, int k, int& sel, int& n) {
+  const int b = lay.width[g], d = lay.size[g];
+  const int nfull = d >> 4, r = d & 15, nf = r >> 2;
+  const int j = c >> 4, cc = c & 15, t = cc >> 2, m4 = cc & 3;
+  const int pr = p & 15, gg = pr & 7;
+  sel = p >> 4;
+  n = m4 + 4 * (pr >> 3);
+  const int base = lay.tile_word[g];
+  if (j < nfull) return base + j * 32 * b + 32 * k + 4 * gg + t;
+  const int pc = base + nfull * 32 * b;
+  if (t < nf) return pc + 8 * nf * k + gg * nf + t;
+  // half quad of the partial chunk: virtual lane gg / 2, upper half for odd gg
+  n = (n & 1) + 2 * (n >> 2) + 4 * (gg & 1);
+  return pc + 8 * nf * b + 4 * k + (gg >> 1);
+}
+
+// Same for a V code: token p, dimension i.
+__device__ __forceinline__ int v_code_word(int vb, int i, int p, int k, int& sel, int& n) {
+  const int m = i >> 4, cm = i & 15, gg = cm & 7;
+  const int pt = p & 15, t = (pt & 7) >> 1, member = (pt & 1) + 2 * (pt >> 3);
+  sel = p >> 4;
+  n = member + 4 * (cm >> 3);
+  return m * 32 * vb + 32 * k + 4 * gg + t;
+}
+
+// One appended row of one (layer, sequence, KV head) and kind, by a CTA of
+// NT >= 128 threads: bx = (layer, sequence, KV head) index, row < n, kind 0
+// = K, 1 = V; mts = 64 KB of shared memory for the rotation.
+template <int NT>
+__device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws, const CacheDev& cache, int layer0,
+                                            const __half* __restrict__ kx, const __half* __restrict__ vx,
+                                            const int32_t* __restrict__ start_v, const int32_t* __restrict__ count_v,
+                                            int batch, int n, int bx, int row, int kind, float* mts) {
+  const int tid = threadIdx.x;
+  const int h = bx % sh.n_kv_heads;
+  const int b = (bx / sh.n_kv_heads) % batch;
+  const int li = bx / (sh.n_kv_heads * batch);
+  const int layer = layer0 + li;
+  const int lh = layer * sh.n_kv_heads + h;
+  // the next kernel of the stream may start its own table-only set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the kind's rotation (transposed, [in][out]) in shared memory, all loads
+  // in flight; a library table, read before the inputs are ready
+  {
+    const uint4* src = reinterpret_cast<const uint4*>((kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD);
+#pragma unroll 8
+    for (int u = tid; u < kD * kD / 4; u += NT) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
+  }
+  // the layout and the thresholds: library tables too
+  __shared__ LayoutDev lay;
+  __shared__ float thr[5 * 16];
+  __shared__ float xs[kD];
+  __shared__ float fac[kNumGroupsMax];
+  __shared__ __half nrm[kNumGroupsMax];
+  for (int u = tid; u < 5 * 16; u += NT) thr[u] = (&ws.codebook->threshold[0][0])[u];
+  if (kind == 0) {
+    if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
+      reinterpret_cast<int32_t*>(&lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
+    for (int u = tid + NT; u < static_cast<int>(sizeof(LayoutDev) / 4); u += NT)
+      reinterpret_cast<int32_t*>(&lay)[u] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[u];
+  } else if (tid == 0) {
+    lay.n_groups = 1;
+    lay.n_positions = kD;
+    for (int g = 0; g < kNumGroupsMax; ++g) {
+      lay.width[g] = g == 0 ? sh.vbits : 0;
+      lay.size[g] = g == 0 ? kD : 0;
+      lay.start[g] = g == 0 ? 0 : kD;
+      lay.tile_word[g] = 0;
+    }
+  }
+  __syncthreads();
+  // Launched as a programmatic dependent of the previous kernel of the
+  // stream: the call's inputs and the cache are read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // this row's values (row < n: inside the input whatever count is) and the
+  // sequence's start and count, all in flight together; record order:
+  // position i holds dim perm[i] (K), V keeps the dims
+  const __half* x = (kind == 0 ? kx : vx) +
+                    ((static_cast<size_t>(li) * batch + b) * n + row) * sh.n_kv_heads * kD + static_cast<size_t>(h) * kD;
+  float xv = 0.f;
+  if (kind == 0) {
+    if (tid < lay.n_positions) xv = __half2float(x[lay.perm[tid]]);
+  } else if (tid < kD) {
+    xv = __half2float(x[tid]);
+  }
+  const int start = start_v[b];
+  const int count = count_v[b];
+  if (start < 0 || count < 0 || count > n) {
+    if (tid == 0 && row == 0 && kind == 0) atomicOr(ws.err, kErrArg);
+    return;
+  }
+  if (row >= count) return;
+  const int64_t pos = static_cast<int64_t>(start) + row;
+  if (pos >= sh.capacity) {
+    if (tid == 0) atomicOr(ws.err, kErrCapacity);
+    return;
+  }
+  if (tid < kD) xs[tid] = xv;
+  __syncthreads();
+  const int ng = lay.n_groups;
+  if (tid < ng) {
+    const int j0 = lay.start[tid], j1 = j0 + lay.size[tid];
+    double s2 = 0.0;
+    for (int j = j0; j < j1; ++j) {
+      const double v = xs[j];
+      s2 += v * v;
+    }
+    const double nr = sqrt(s2);
+    nrm[tid] = __double2half(nr);
+    fac[tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[tid])) / nr) : 0.f;
+  }
+  __syncthreads();
+  const int i = tid;
+  const int tile = static_cast<int>(pos / kTile), p = static_cast<int>(pos % kTile);
+  const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+  if (slot < 0) {  // uniform over the CTA; no barrier follows
+    if (tid == 0) atomicOr(ws.err, kErrPage);
+    return;
+  }
+  if (i < lay.n_positions) {
+    int g = 0;
+    for (int t = 1; t < ng; ++t)
+      if (i >= lay.start[t]) g = t;
+    const int j0 = lay.start[g], j1 = j0 + lay.size[g];
+    float y = 0.f;
+    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
+    const int w = lay.width[g];
+    const float u = y * fac[g];
+    const int code = lloyd_code(thr + w * 16, w, u);
+    // rewrite this code's bits, one atomic pair per touched word
+    const int nwords = 256 * (kind == 0 ? sh.kbits : sh.vbits);
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
+    int cur = -1;
+    uint32_t mask = 0, val = 0;
+    for (int q = 0; q < w; ++q) {
+      int k, bit, sel, nib;
+      if (kind == 0) k_code_word(lay, g, i - lay.start[g], p, 0, sel, nib);
+      else v_code_word(w, i, p, 0, sel, nib);
+      quartet_bit(w, sel, nib, q, k, bit);
+      const int wk = kind == 0 ? k_code_word(lay, g, i - lay.start[g], p, k, sel, nib) : v_code_word(w, i, p, k, sel, nib);
+      if (wk != cur) {
+        if (cur >= 0) {
+          atomicAnd(gtile + cur, ~mask);
+          atomicOr(gtile + cur, val);
+        }
+        cur = wk;
+        mask = 0;
+        val = 0;
+      }
+      mask |= 1u << bit;
+      val |= static_cast<uint32_t>((code >> q) & 1) << bit;
+    }
+    if (cur >= 0) {
+      atomicAnd(gtile + cur, ~mask);
+      atomicOr(gtile + cur, val);
+    }
+  }
+  if (tid == 0) {
+    const size_t tp = static_cast<size_t>(slot) * kTile + p;
+    if (kind == 0) {
+      __half2* dst = reinterpret_cast<__half2*>(cache.knorm + tp * 4);
+      const __half z = __float2half(0.f);
+      dst[0] = __halves2half2(nrm[0], ng > 1 ? nrm[1] : z);
+      dst[1] = __halves2half2(ng > 2 ? nrm[2] : z, ng > 3 ? nrm[3] : z);
+    } else {
+      cache.vnorm[tp] = nrm[0];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                             const __half* __restrict__ kx,
+                                                             const __half* __restrict__ vx,
+                                                             const int32_t* __restrict__ start_v,
+                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+  extern __shared__ __align__(16) float mts[];  // [kD][kD]
+  append_body<kAppThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, blockIdx.x, blockIdx.y,
+                           blockIdx.z, mts);
+}
+
+// One query row (layer, sequence, query head) = bx, by a CTA of kRotThreads.
+__device__ __forceinline__ void rotate_body(const Shape& sh, const Workspace& ws, int layer0,
+                                            const __half* __restrict__ q, int batch, float* __restrict__ qrot,
+                                            int bx) {
+  // the decode kernel that follows may start its own set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int hq = bx % sh.n_q_heads;
+  const int b = (bx / sh.n_q_heads) % batch;
+  const int li = bx / (sh.n_q_heads * batch);
+  const int layer = layer0 + li;
+  const int kvh = hq / sh.group;
+  const LayoutDev& lay = ws.layouts[layer * sh.n_kv_heads + kvh];
+  const int tid = threadIdx.x, i = tid & (kD - 1), half = tid >> 7;
+  // this thread's half column of the (block-diagonal) rotation, all loads in flight at once
+  const float* mt = ws.mkt + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
+  float m[64];
+#pragma unroll
+  for (int u = 0; u < 64; ++u) m[u] = __ldg(mt + (half * 64 + u) * kD + i);
+  __shared__ float qp[kD];
+  __shared__ float part[kD];
+  const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
+  // Launched as a programmatic dependent of the previous kernel of the
+  // stream: the query is read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid < kD) qp[tid] = __half2float(q[row * kD + lay.perm[tid]]);
+  __syncthreads();
+  float sacc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 64; ++u) sacc = fmaf(m[u], qp[half * 64 + u], sacc);
+  if (half == 1) part[i] = sacc;
+  __syncthreads();
+  if (half == 0) {
+    float out = 0.f;
+    if (i < lay.n_positions) {
+      int g = 0;
+      for (int t = 1; t < lay.n_groups; ++t)
+        if (i >= lay.start[t]) g = t;
+      out = (sacc + part[i]) * lay.inv_sqrt_d[g] * kInvSqrtD;
+    }
+    qrot[row * kD + i] = out;
+    qp[i] = out;
+  }
+  __syncthreads();
+  write_frags(lay, qp, hq % sh.group, sh.group, frag_block(sh, ws, li, b, kvh, (hq % sh.group) >> 3), tid, kRotThreads);
+}
+
+__global__ void __launch_bounds__(kRotThreads) rotate_query_kernel(Shape sh, Workspace ws, int layer0,
+                                                                   const __half* __restrict__ q, int batch,
+                                                                   float* __restrict__ qrot) {
+  rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
+}
+
+// A decode step's preparation in one launch: the first n_rot CTAs rotate the
+// query rows (as rotate_query_kernel), the others append the step's new K/V
+// rows (as append_kernel, CTA a - n_rot = ((kind * n + row) * n_units + unit),
+// n_units = layer_count * batch * Hkv).  The two parts are independent.
+__global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                           const __half* __restrict__ q, int batch,
+                                                           float* __restrict__ qrot, const __half* __restrict__ kx,
+                                                           const __half* __restrict__ vx,
+                                                           const int32_t* __restrict__ start_v,
+                                                           const int32_t* __restrict__ count_v, int n, int n_rot,
+                                                           int n_units) {
+  extern __shared__ __align__(16) float mts[];  // [kD][kD], the append part
+  if (static_cast<int>(blockIdx.x) < n_rot) {
+    rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
+  } else {
+    const int a = blockIdx.x - n_rot;
+    append_body<kRotThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, a % n_units,
+                             (a / n_units) % n, a / (n_units * n), mts);
+  }
+}
+
+cudaError_t encode_smem_once() {
+  static const cudaError_t status = set_smem(encode_kernel, sizeof(EncodeSmem));
+  return status;
+}
+
+// Launches a kernel as a programmatic dependent of the previous kernel in
+// the stream: it may start while that kernel finishes.  Every kernel
+// launched this way reads only library tables before griddepcontrol.wait and
+// everything produced by earlier work in the stream after it, so the chain
+// append -> rotate -> split -> combine (and the next call's kernels) keeps
+// stream order for all data while the table-only prologues overlap.
+}  // namespace
+
+cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* calib_q, int nq,
+                          const __half* calib_k, int nk, int pairing, cudaStream_t stream) {
+  dim3 grid(s.n_layers * s.n_kv_heads, kEnergyChunks);
+  energy_kernel<<<grid, kD, 0, stream>>>(calib_q, nq, calib_k, nk, s.n_q_heads, s.n_kv_heads, s.group, s.n_layers,
+                                         pairing, ws.energy_q, ws.energy_k, ws.err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                          int layer_count, const __half* k, const __half* v, const int32_t* start,
+                          const int32_t* count, int batch, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const cudaError_t e = encode_smem_once();
+  if (e != cudaSuccess) return e;
+  if (n <= kAppendMaxRows) {
+    // a few rows per sequence: rewrite only their code bits
+    static const cudaError_t attr = set_smem(append_kernel, kD * kD * sizeof(float));
+    if (attr != cudaSuccess) return attr;
+    return launch_dependent(append_kernel, dim3(layer_count * batch * s.n_kv_heads, n, 2), dim3(kAppThreads),
+                            kD * kD * sizeof(float), stream, s, ws, cache, layer0, k, v, start, count, batch, n);
+  }
+  // about two waves of CTAs (two fit an SM); each loops over its unit's tiles
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  const int units = layer_count * batch * s.n_kv_heads;
+  const int tiles = (n + kTile - 1) / kTile + 1;  // rows may start inside a tile
+  const int per_unit = std::max(1, std::min(tiles, (4 * sms) / (2 * units)));
+  dim3 grid(units, per_unit, 2);
+  encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                        const __half* q, int batch, float* qrot, const __half* k, const __half* v,
+                        const int32_t* start, const int32_t* count, int n, cudaStream_t stream) {
+  static const cudaError_t attr = set_smem(prep_kernel, kD * kD * sizeof(float));
+  if (attr != cudaSuccess) return attr;
+  const int n_rot = layer_count * batch * s.n_q_heads;
+  const int n_units = layer_count * batch * s.n_kv_heads;
+  return launch_dependent(prep_kernel, dim3(n_rot + n_units * n * 2), dim3(kRotThreads), kD * kD * sizeof(float),
+                          stream, s, ws, cache, layer0, q, batch, qrot, k, v, start, count, n, n_rot, n_units);
+}
+
+cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
+                                const __half* q, int batch, float* qrot, cudaStream_t stream) {
+  return launch_dependent(rotate_query_kernel, dim3(layer_count * batch * s.n_q_heads), dim3(kRotThreads), 0, stream, s,
+                          ws, layer0, q, batch, qrot);
+}
+
+}  // namespace bgtq

@@ -448,9 +448,8 @@ def main():
 
     def step_buffered():
         for l in range(L):
-            kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
-            kv.decode_attn_buffered(l, q_all[l:l + 1], seq_hi, seq_lo, buf_k[l:l + 1], buf_v[l:l + 1], buf_cnt,
-                                    out[l:l + 1])
+            kv.decode_step_buffered(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq_hi, seq_lo,
+                                    buf_k[l:l + 1], buf_v[l:l + 1], buf_cnt, out[l:l + 1])
 
     ms_buf, g_buf, _ = time_graph(step_buffered, args.steps, args.warmup)
     ms_buf = max_over_ranks(ms_buf, world, dev)

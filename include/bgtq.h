@@ -15,6 +15,7 @@
  *   bgtq_decode_attn    one GQA decode step over the packed cache
  *   bgtq_decode_step    encode_append of a step's rows + decode_attn in one call
  *   bgtq_decode_attn_buffered  decode with fp16 sink / recent-window rows
+ *   bgtq_decode_step_buffered  the same after a step's appends, in one call
  *   bgtq_logit_mae      per-layer logit error of the packed keys (diagnostic)
  *   bgtq_set_block_table  page table of a paged cache
  *
@@ -273,6 +274,18 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
  * scratch.  ASYNC. */
 int bgtq_logit_mae(bgtq_state* st, int32_t layer, int32_t layer_count, int32_t seq, int32_t w0, int32_t m,
                    const void* d_q, const void* d_k, double* d_mae, void* stream);
+
+/* bgtq_encode_append of a step's new rows followed by
+ * bgtq_decode_attn_buffered, as one call (the appends and the query rotation
+ * share a launch for 1..16 rows per sequence): same arguments, results and
+ * errors as those two calls in that order.  In the withbuffer setting the
+ * rows appended are typically those leaving the recent fp16 window.  n = 0
+ * appends nothing (d_k, d_v, d_start and d_count may then be NULL).  ASYNC. */
+int bgtq_decode_step_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                              const int32_t* d_start, const int32_t* d_count, int32_t n, const void* d_q,
+                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch,
+                              const void* d_buf_k, const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf,
+                              void* d_out, void* stream);
 
 /* The two stages of bgtq_decode_attn after bgtq_rotate_query, for callers
  * that time or schedule them separately (same arguments and results):

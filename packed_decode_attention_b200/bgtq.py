@@ -102,6 +102,8 @@ _SIGS = {
     "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_logit_mae": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
     "bgtq_decode_step": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "bgtq_decode_step_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP,
+                                                 _VP, _VP, _I32, _VP, _VP]),
     "bgtq_set_block_table": (ctypes.c_int, [_VP, _VP]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
@@ -265,6 +267,14 @@ def bgtq_decode_step(state, layer, layer_count, d_k, d_v, d_start, d_count, n, d
                                   _ptr(d_q), _ptr(d_seq_lens), batch, _ptr(d_out), _stream(stream)))
 
 
+def bgtq_decode_step_buffered(state, layer, layer_count, d_k, d_v, d_start, d_count, n, d_q, d_seq_lens, d_pos_lo,
+                              batch, d_buf_k, d_buf_v, d_buf_count, n_buf, d_out, stream=None):
+    _check(lib().bgtq_decode_step_buffered(state, layer, layer_count, _ptr(d_k), _ptr(d_v), _ptr(d_start),
+                                           _ptr(d_count), n, _ptr(d_q), _ptr(d_seq_lens), _ptr(d_pos_lo), batch,
+                                           _ptr(d_buf_k), _ptr(d_buf_v), _ptr(d_buf_count), n_buf, _ptr(d_out),
+                                           _stream(stream)))
+
+
 def bgtq_decode_split(state, layer, layer_count, d_qrot, d_seq_lens, batch, stream=None):
     _check(lib().bgtq_decode_split(state, layer, layer_count, _ptr(d_qrot), _ptr(d_seq_lens), batch, _stream(stream)))
 
@@ -388,6 +398,14 @@ class PackedKVCache:
         sequence seq: q fp16 [layer_count, m, Hq, 128], k (exact keys) fp16
         [layer_count, m, Hkv, 128], out float64 [layer_count, Hq]."""
         bgtq_logit_mae(self.state, layer, layer_count, seq, w0, q.shape[1], q, k, out)
+
+    def decode_step_buffered(self, layer, k, v, start, count, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out,
+                             layer_count=1):
+        """encode_append(k, v, start, count) then decode_attn_buffered(...), in one call; k = None
+        appends nothing."""
+        n = 0 if k is None else k.shape[2]
+        bgtq_decode_step_buffered(self.state, layer, layer_count, k, v, start, count, n, q, seq_lens, pos_lo,
+                                  q.shape[1], buf_k, buf_v, buf_count, buf_k.shape[2], out)
 
     def decode_split(self, layer, qrot, seq_lens, layer_count=1):
         """The split-K stage alone from rotated queries (fp32 [layer_count, batch, Hq, 128])."""

@@ -585,34 +585,54 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   return BGTQ_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Checks of a decode step's append arguments (n = 0: none).
+int check_step_appends(const void* d_k, const void* d_v, const int32_t* d_start, const int32_t* d_count, int32_t n) {
+  if (n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
+  if (n > 0 && (!d_k || !d_v || !d_start || !d_count)) return BGTQ_ERR_NULL;
+  if (n > 0 && (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)))
+    return BGTQ_ERR_ALIGNMENT;
+  return BGTQ_OK;
+}
+
+// A decode step's appends and query rotation: one launch for 1..16 rows per
+// sequence (they are independent), else the encode (if any) then the rotation.
+cudaError_t queue_step_prep(bgtq_state* st, int32_t layer, int32_t layer_count, const __half* q, int32_t batch,
+                            const void* d_k, const void* d_v, const int32_t* d_start, const int32_t* d_count,
+                            int32_t n, cudaStream_t s) {
+  const __half* k = static_cast<const __half*>(d_k);
+  const __half* v = static_cast<const __half*>(d_v);
+  if (n >= 1 && n <= bgtq::kAppendMaxRows)
+    return bgtq::launch_prep(st->shape, st->ws, st->cache, layer, layer_count, q, batch, st->ws.qrot, k, v, d_start,
+                             d_count, n, s);
+  const cudaError_t e =
+      n > 0 ? bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, k, v, d_start, d_count, batch, n, s)
+            : cudaSuccess;
+  if (e != cudaSuccess) return e;
+  return bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, q, batch, st->ws.qrot, s);
+}
+
+}  // namespace
+
+extern "C" {
+
 int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
                      const int32_t* d_start, const int32_t* d_count, int32_t n, const void* d_q,
                      const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream) {
   if (!st || !d_q || !d_seq_lens || !d_out) return BGTQ_ERR_NULL;
-  if (n > 0 && (!d_k || !d_v || !d_start || !d_count)) return BGTQ_ERR_NULL;
-  const int v = check_decode_args(st, layer, layer_count, batch);
+  int v = check_step_appends(d_k, d_v, d_start, d_count, n);
   if (v != BGTQ_OK) return v;
-  if (n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
+  v = check_decode_args(st, layer, layer_count, batch);
+  if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  if (n > 0 && (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)))
-    return BGTQ_ERR_ALIGNMENT;
   const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
-  const __half* q = static_cast<const __half*>(d_q);
-  const __half* k = static_cast<const __half*>(d_k);
-  const __half* vv = static_cast<const __half*>(d_v);
-  cudaError_t e;
-  if (n >= 1 && n <= bgtq::kAppendMaxRows) {
-    // the appends and the query rotation in one launch
-    e = bgtq::launch_prep(st->shape, st->ws, st->cache, layer, layer_count, q, batch, st->ws.qrot, k, vv, d_start,
-                          d_count, n, s);
-  } else {
-    e = n > 0 ? bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, k, vv, d_start, d_count, batch,
-                                    n, s)
-              : cudaSuccess;
-    if (e == cudaSuccess) e = bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, q, batch, st->ws.qrot, s);
-  }
-  if (e != cudaSuccess) return BGTQ_ERR_CUDA;
+  if (queue_step_prep(st, layer, layer_count, static_cast<const __half*>(d_q), batch, d_k, d_v, d_start, d_count, n,
+                      s) != cudaSuccess)
+    return BGTQ_ERR_CUDA;
   if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens,
                                 bgtq::BufferArgs{}, batch, split, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
@@ -622,12 +642,19 @@ int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   return BGTQ_OK;
 }
 
-int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
-                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
-                              const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,
-                              void* stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_buffered_impl(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                         const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
+                         const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out, void* stream,
+                         const void* d_k, const void* d_v, const int32_t* d_start, const int32_t* d_count,
+                         int32_t n) {
   if (!st || !d_q || !d_seq_lens || !d_pos_lo || !d_buf_k || !d_buf_v || !d_buf_count || !d_out) return BGTQ_ERR_NULL;
-  const int v = check_decode_args(st, layer, layer_count, batch);
+  int v = check_step_appends(d_k, d_v, d_start, d_count, n);
+  if (v != BGTQ_OK) return v;
+  v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (n_buf < 1 || n_buf > bgtq::kMaxBufferRows) return BGTQ_ERR_INVALID_ARG;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_pos_lo) || !aligned16(d_buf_k) ||
@@ -642,8 +669,7 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
   buf.count = d_buf_count;
   buf.pos_lo = d_pos_lo;
   buf.n_buf = n_buf;
-  if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
-                                st->ws.qrot, s) != cudaSuccess)
+  if (queue_step_prep(st, layer, layer_count, buf.q, batch, d_k, d_v, d_start, d_count, n, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   if (bgtq::launch_decode_split(st->shape, st->ws, st->cache, layer, layer_count, nullptr, d_seq_lens, buf, batch,
                                 split, s) != cudaSuccess)
@@ -652,6 +678,27 @@ int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
                            static_cast<__half*>(d_out), s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
   return BGTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bgtq_decode_attn_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
+                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch, const void* d_buf_k,
+                              const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf, void* d_out,
+                              void* stream) {
+  return decode_buffered_impl(st, layer, layer_count, d_q, d_seq_lens, d_pos_lo, batch, d_buf_k, d_buf_v, d_buf_count,
+                              n_buf, d_out, stream, nullptr, nullptr, nullptr, nullptr, 0);
+}
+
+int bgtq_decode_step_buffered(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                              const int32_t* d_start, const int32_t* d_count, int32_t n, const void* d_q,
+                              const int32_t* d_seq_lens, const int32_t* d_pos_lo, int32_t batch,
+                              const void* d_buf_k, const void* d_buf_v, const int32_t* d_buf_count, int32_t n_buf,
+                              void* d_out, void* stream) {
+  return decode_buffered_impl(st, layer, layer_count, d_q, d_seq_lens, d_pos_lo, batch, d_buf_k, d_buf_v, d_buf_count,
+                              n_buf, d_out, stream, d_k, d_v, d_start, d_count, n);
 }
 
 int bgtq_logit_mae(bgtq_state* st, int32_t layer, int32_t layer_count, int32_t seq, int32_t w0, int32_t m,

@@ -575,3 +575,50 @@ def test_decode_step_equals_append_then_decode(dev, n):
     assert torch.isfinite(ob.float()).all()
     for kv in kvs:
         kv.close()
+
+
+@pytest.mark.parametrize("n", [1, 0])
+def test_decode_step_buffered_equals_append_then_buffered_decode(dev, n):
+    """bgtq_decode_step_buffered gives the same cache bytes and output, bit for
+    bit, as bgtq_encode_append followed by bgtq_decode_attn_buffered."""
+    lens = [900, 300]
+    w = wl.scaled(wl.WORKLOADS["tiny"], n_kv_heads=2, n_q_heads=8, batch=2, seq_len=1024, n_calib=64)
+    cfg = library_config(w)
+    cq, ck = wl.calibration(w)
+    kvs = []
+    for _ in range(2):
+        kv = bgtq.PackedKVCache(cfg, dev)
+        kv.allocate(cq.to(dev), ck.to(dev))
+        for b, ln in enumerate(lens):
+            k = torch.zeros((1, 2, ln, 2, 128), dtype=torch.float16)
+            v = torch.zeros_like(k)
+            k[0, b] = wl.keys(w, 0, b, 0, ln)
+            v[0, b] = wl.values(w, 0, b, 0, ln)
+            count = torch.zeros(2, dtype=torch.int32, device=dev)
+            count[b] = ln
+            kv.encode_append(0, k.to(dev), v.to(dev), torch.zeros(2, dtype=torch.int32, device=dev), count)
+        kvs.append(kv)
+    kn = torch.stack([wl.keys(w, 0, b, lens[b], 1) for b in range(2)])[None].to(dev)
+    vn = torch.stack([wl.values(w, 0, b, lens[b], 1) for b in range(2)])[None].to(dev)
+    start = torch.tensor(lens, dtype=torch.int32, device=dev)
+    count = torch.full((2,), n, dtype=torch.int32, device=dev)
+    hi = torch.tensor([ln + n - 40 for ln in lens], dtype=torch.int32, device=dev)
+    lo = torch.full((2,), 4, dtype=torch.int32, device=dev)
+    bk = torch.randn((1, 2, 44, 2, 128), device=dev).half()
+    bv = torch.randn_like(bk)
+    bc = torch.full((2,), 44, dtype=torch.int32, device=dev)
+    q = wl.decode_query(w, 0, [ln + n for ln in lens])[None].to(dev)
+    a, bkv = kvs
+    oa = torch.empty((1, 2, 8, 128), dtype=torch.float16, device=dev)
+    if n:
+        a.encode_append(0, kn, vn, start, count)
+    a.decode_attn_buffered(0, q, hi, lo, bk, bv, bc, oa)
+    ob = torch.empty_like(oa)
+    bkv.decode_step_buffered(0, kn if n else None, vn if n else None, start if n else None, count if n else None, q,
+                             hi, lo, bk, bv, bc, ob)
+    torch.cuda.synchronize()
+    assert a.device_error() == 0 and bkv.device_error() == 0
+    assert torch.equal(a.cache, bkv.cache)
+    assert torch.equal(oa, ob)
+    for kv in kvs:
+        kv.close()

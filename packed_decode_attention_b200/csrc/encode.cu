@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
 // n, code = #{thresholds <= u}) into the codes, and packs the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
+constexpr int kEncTilesPerCta = 8;  // tiles a CTA encodes with one load of its rotation
 // Column of element (coordinate j, row r) in xt[j][]: float4 groups of 4 rows,
 // XOR-swizzled by j so that the transposed writes spread over the banks.
 __device__ __forceinline__ int xt_col(int j, int r) { return (((r >> 2) ^ ((j >> 3) & 15)) << 2) | (r & 3); }
@@ -640,7 +641,10 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
     return launch_dependent(append_kernel, dim3(layer_count * batch * s.n_kv_heads, n, 2), dim3(kAppThreads),
                             kD * kD * sizeof(float), stream, s, ws, cache, layer0, k, v, start, count, batch, n);
   }
-  // about two waves of CTAs (two fit an SM); each loops over its unit's tiles
+  // CTAs per unit: at least two waves if every unit has rows, and at most
+  // kEncTilesPerCta tiles per CTA (the counts are device data: a call may
+  // write one sequence of a large batch; the CTAs of units without rows exit
+  // at once)
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
@@ -650,7 +654,8 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
   }
   const int units = layer_count * batch * s.n_kv_heads;
   const int tiles = (n + kTile - 1) / kTile + 1;  // rows may start inside a tile
-  const int per_unit = std::max(1, std::min(tiles, (4 * sms) / (2 * units)));
+  const int per_unit = std::max((tiles + kEncTilesPerCta - 1) / kEncTilesPerCta,
+                                std::min(tiles, std::max(1, (4 * sms) / (2 * units))));
   dim3 grid(units, per_unit, 2);
   encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
   return cudaGetLastError();

@@ -454,19 +454,31 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   if (tid < kD) xs[tid] = xv;
   __syncthreads();
   const int ng = lay.n_groups;
-  if (tid < ng) {
-    const int j0 = lay.start[tid], j1 = j0 + lay.size[tid];
+  // The group norms (fp64, coordinate order) and y = R x (fp32, coordinate
+  // order) are independent: with 256 threads the norms run on threads
+  // 128.. beside the rotation on threads 0..127; with 128, first.
+  const int i = tid;
+  const int norm_tid = tid - (NT >= 2 * kD ? kD : 0);
+  if (norm_tid >= 0 && norm_tid < ng) {
+    const int j0 = lay.start[norm_tid], j1 = j0 + lay.size[norm_tid];
     double s2 = 0.0;
     for (int j = j0; j < j1; ++j) {
       const double v = xs[j];
       s2 += v * v;
     }
     const double nr = sqrt(s2);
-    nrm[tid] = __double2half(nr);
-    fac[tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[tid])) / nr) : 0.f;
+    nrm[norm_tid] = __double2half(nr);
+    fac[norm_tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[norm_tid])) / nr) : 0.f;
+  }
+  int g = 0;
+  float y = 0.f;
+  if (i < lay.n_positions) {
+    for (int t = 1; t < ng; ++t)
+      if (i >= lay.start[t]) g = t;
+    const int j0 = lay.start[g], j1 = j0 + lay.size[g];
+    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
   }
   __syncthreads();
-  const int i = tid;
   const int tile = static_cast<int>(pos / kTile), p = static_cast<int>(pos % kTile);
   const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
   if (slot < 0) {  // uniform over the CTA; no barrier follows
@@ -474,12 +486,6 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
     return;
   }
   if (i < lay.n_positions) {
-    int g = 0;
-    for (int t = 1; t < ng; ++t)
-      if (i >= lay.start[t]) g = t;
-    const int j0 = lay.start[g], j1 = j0 + lay.size[g];
-    float y = 0.f;
-    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
     const int w = lay.width[g];
     const float u = y * fac[g];
     const int code = lloyd_code(thr + w * 16, w, u);

@@ -349,6 +349,14 @@ int bgtq_set_block_table(bgtq_state* st, const int32_t* d_block_table);
  * floating-point reassociation. */
 int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens);
 
+/* Test hook for the bounded waits (no fault is involved): while tile >= 0,
+ * the split pass issues no copy for cache tile `tile` of any unit, so the
+ * warp that waits for it gives up after about a second of polls, raises
+ * BGTQ_DEVERR_TIMEOUT, lets its other copies land and posts empty partials
+ * for its CTA; the output then leaves that CTA's positions out.  -1 turns the
+ * hook off (the default).  SYNC (host only). */
+int bgtq_test_drop_tile_copies(bgtq_state* st, int32_t tile);
+
 /* Synchronises "stream", reads the device error flag into *h_flags
  * (BGTQ_DEVERR_* bits) and clears it.  SYNC. */
 int bgtq_get_device_error(bgtq_state* st, void* stream, int32_t* h_flags);

@@ -105,6 +105,7 @@ _SIGS = {
     "bgtq_decode_step_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP,
                                                  _VP, _VP, _I32, _VP, _VP]),
     "bgtq_set_block_table": (ctypes.c_int, [_VP, _VP]),
+    "bgtq_test_drop_tile_copies": (ctypes.c_int, [_VP, _I32]),
     "bgtq_decode_split": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP]),
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
@@ -419,6 +420,10 @@ class PackedKVCache:
         device (kept referenced here; its contents are read at kernel time)."""
         bgtq_set_block_table(self.state, table)
         self._block_table = table
+
+    def test_drop_tile_copies(self, tile):
+        """Test hook: the split pass skips the copies of cache tile `tile` (-1: off)."""
+        _check(lib().bgtq_test_drop_tile_copies(self.state, tile))
 
     def set_split_tokens(self, tokens):
         bgtq_set_split_tokens(self.state, tokens)

@@ -287,6 +287,7 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->shape.max_splits = max_splits_of(cfg);
   st->shape.capacity = cfg->capacity_tokens;
   st->shape.ntiles = tiles_of(cfg);
+  st->shape.drop_tile = -1;
   uint8_t* c8 = static_cast<uint8_t*>(d_cache);
   st->cache.ktile = reinterpret_cast<uint32_t*>(c8 + p.krec);
   st->cache.knorm = reinterpret_cast<__half*>(c8 + p.knorm);
@@ -802,6 +803,13 @@ int bgtq_set_block_table(bgtq_state* st, const int32_t* d_block_table) {
   if (st->cache.n_pages == 0) return BGTQ_ERR_INVALID_ARG;
   if (d_block_table && !aligned16(d_block_table)) return BGTQ_ERR_ALIGNMENT;
   st->cache.block_table = d_block_table;
+  return BGTQ_OK;
+}
+
+int bgtq_test_drop_tile_copies(bgtq_state* st, int32_t tile) {
+  if (!st) return BGTQ_ERR_NULL;
+  if (tile < -1) return BGTQ_ERR_INVALID_ARG;
+  st->shape.drop_tile = tile;
   return BGTQ_OK;
 }
 

@@ -477,6 +477,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 
   auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
     const int tile = tlo + wu + k * W;
+    if (tile == sh.drop_tile) {
+      // test hook: the copy is never issued, so the wait on it runs out
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&my_bars[k % kStages], stage_tx);
+      return;
+    }
     int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
     if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
       atomicOr(ws.err, kErrPage);
@@ -663,12 +669,17 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
     a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
   }
-  if (__syncthreads_or(timed_out)) return;
+  const bool cta_timed_out = __syncthreads_or(timed_out);
   // per head: the common maximum, the warps' weights (warps without a tile
-  // hold m = -inf, l = 0, acc = 0) and the weighted denominator
+  // hold m = -inf, l = 0, acc = 0) and the weighted denominator; a CTA that
+  // gave up on a copy posts empty partials (its error flag is raised)
   float* wsc = reinterpret_cast<float*>(smem_raw + DL.wsc);
   float* mres = reinterpret_cast<float*>(smem_raw + DL.mres);
-  if (tid < 8) {
+  if (tid < 8 && cta_timed_out) {
+    for (int w = 0; w < kDecWarps; ++w) wsc[w * 8 + tid] = 0.f;
+    mres[tid] = -CUDART_INF_F;
+    mres[8 + tid] = 0.f;
+  } else if (tid < 8) {
     float M = -CUDART_INF_F;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
@@ -690,7 +701,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) a = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a);
     float* part = part_base + hh * part_head_stride;
-    part[4 + i] = a;
+    part[4 + i] = cta_timed_out ? 0.f : a;
     if (i == 0) {
       part[0] = mres[hh];
       part[1] = mres[8 + hh];

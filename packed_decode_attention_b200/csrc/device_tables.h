@@ -97,6 +97,8 @@ struct Shape {
   int32_t kbits, vbits, max_splits;
   int64_t capacity;
   int64_t ntiles;                // tiles per (layer, sequence, KV head)
+  int32_t drop_tile;             // test hook: the split pass issues no copy for this tile (-1: off)
+  int32_t pad;
 };
 
 // Error flag bits (same values as BGTQ_DEVERR_* in bgtq.h).

@@ -17,7 +17,8 @@ from packed_decode_attention_b200 import bgtq
 from packed_decode_attention_b200 import workloads as wl
 
 from oracle import tiles as otiles
-from parity_helpers import (CODE_AGREEMENT, REL_TOL, compare_codes, fp16_ulp_apart, gpu_codes, library_config,
+from parity_helpers import (CODE_AGREEMENT, REL_TOL, compare_codes, encode_on_gpu, fp16_ulp_apart, gpu_codes,
+                            library_config,
                             oracle_config, oracle_u, row_rel_err, upload_oracle_rows)
 
 pytestmark = pytest.mark.gpu
@@ -622,3 +623,38 @@ def test_decode_step_buffered_equals_append_then_buffered_decode(dev, n):
     assert torch.equal(oa, ob)
     for kv in kvs:
         kv.close()
+
+
+def test_copy_timeout_raises_the_flag_and_recovers(dev):
+    """The split pass's waits are bounded.  With the copies of one tile never
+    issued (a host-side test hook; nothing faults), the warp waiting for it
+    gives up after about a second, raises BGTQ_DEVERR_TIMEOUT and its CTA
+    posts empty partials: the outputs stay finite.  With the hook off again
+    the same call gives the earlier output bit for bit: the context is still
+    usable."""
+    w = wl.scaled(wl.WORKLOADS["tiny"], seq_len=4096, n_calib=64)
+    cfg = library_config(w)
+    kv = bgtq.PackedKVCache(cfg, dev)
+    cq, ck = wl.calibration(w)
+    kv.allocate(cq.to(dev), ck.to(dev))
+    encode_on_gpu(kv, w, [0], [4096], dev)
+    q = wl.decode_query(w, 0, [4096])[None].to(dev)
+    seq = torch.tensor([4096], dtype=torch.int32, device=dev)
+    ref = torch.empty((1, 1, 4, 128), dtype=torch.float16, device=dev)
+    kv.decode_attn(0, q, seq, ref)
+    torch.cuda.synchronize()
+    assert kv.device_error() == 0
+    kv.test_drop_tile_copies(5)
+    got = torch.empty_like(ref)
+    kv.decode_attn(0, q, seq, got)
+    torch.cuda.synchronize()
+    assert kv.device_error() & 16                       # BGTQ_DEVERR_TIMEOUT
+    assert torch.isfinite(got.float()).all()
+    assert not torch.equal(got, ref)                     # that CTA's positions are left out
+    kv.test_drop_tile_copies(-1)
+    again = torch.empty_like(ref)
+    kv.decode_attn(0, q, seq, again)
+    torch.cuda.synchronize()
+    assert kv.device_error() == 0
+    assert torch.equal(again, ref)
+    kv.close()

@@ -6,6 +6,15 @@ owns the two device buffers (torch tensors) and one library state.
 
 The library must be built (``python -m packed_decode_attention_b200.build``
 or ``__graft_entry__.build()``); importing the binding without it raises.
+
+A decode step, per layer ``l`` (tensors on the GPU; shapes in include/bgtq.h)::
+
+    kv = PackedKVCache(Config(n_layers=36, n_kv_heads=2, n_q_heads=16,
+                              max_batch=1, capacity_tokens=131072), "cuda")
+    kv.allocate(calib_q, calib_k)                    # Block-GTQ widths + tables
+    kv.encode_append(l, k, v, start, count)          # prefill
+    kv.decode_step(l, k_new, v_new, start, count,    # append the new rows,
+                   q, seq_lens, out)                 # then attend
 """
 import ctypes
 import os
@@ -25,6 +34,7 @@ DEVERR_SEQ_LEN = 2
 DEVERR_ARG = 4
 DEVERR_NONFINITE = 8
 DEVERR_TIMEOUT = 16
+DEVERR_PAGE = 32
 
 
 class BgtqError(RuntimeError):

@@ -90,7 +90,7 @@ enum {
 };
 
 typedef struct {
-  int32_t n_layers;          /* >= 1 */
+  int32_t n_layers;          /* 1..65535 (a call's layers are a launch grid dimension) */
   int32_t n_kv_heads;        /* >= 1 */
   int32_t n_q_heads;         /* multiple of n_kv_heads; G = n_q_heads / n_kv_heads <= 16 */
   int32_t head_dim;          /* must be 128 */
@@ -113,7 +113,8 @@ typedef struct bgtq_state bgtq_state;
 /* Bytes of the two caller-owned device buffers for a config.
  * cache_bytes: the packed K/V cache (layout above).  workspace_bytes: the
  * device tables plus scratch (energy partial sums, rotated queries, split-K
- * partials, error flag).  SYNC (host only). */
+ * partials, error flag).  A config whose cache or workspace would reach
+ * 2^56 bytes is rejected with BGTQ_ERR_INVALID_ARG.  SYNC (host only). */
 int bgtq_required_bytes(const bgtq_config* cfg, size_t* cache_bytes, size_t* workspace_bytes);
 
 /* Creates a state over caller buffers of at least the required sizes (both

@@ -45,6 +45,24 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Allocation set, and for a paged cache a block table given.
 bool cache_ready(const bgtq_state* st) { return st->ready && (st->cache.n_pages == 0 || st->cache.block_table); }
 
+constexpr int kMaxLayers = 65535;
+
+int max_splits_of(const bgtq_config* c) { return c->max_splits == 0 ? 256 : c->max_splits; }
+
+// The cache and the workspace of a config, estimated in floating point (an
+// upper bound of the exact plan), each below 2^56 bytes.
+bool sizes_in_range(const bgtq_config* c) {
+  const double lh = double(c->n_layers) * c->n_kv_heads;
+  const double tiles = c->page_pool_tiles > 0 ? lh * c->page_pool_tiles
+                                              : lh * c->max_batch * ((c->capacity_tokens + 63) / 64);
+  const double cache = tiles * (1024.0 * (c->k_avg_bits + c->v_avg_bits) + 64.0 * 10) + 4096.0;
+  const double qrows = double(c->n_layers) * c->max_batch * c->n_q_heads;
+  const int splits = c->max_splits == 0 ? 256 : c->max_splits;
+  const double ws = lh * (4.0 * 128 * 128 * 4 + 16384.0) + qrows * (splits + 16.0) * 1024.0 + (1 << 20);
+  const double limit = 72057594037927936.0;  // 2^56
+  return cache < limit && ws < limit;
+}
+
 int validate_config(const bgtq_config* c) {
   if (!c) return BGTQ_ERR_NULL;
   if (c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->max_batch < 1) return BGTQ_ERR_INVALID_ARG;
@@ -56,10 +74,12 @@ int validate_config(const bgtq_config* c) {
   if (c->rope_pairing != 0 && c->rope_pairing != 1) return BGTQ_ERR_INVALID_ARG;
   if (c->max_splits < 0 || c->max_splits > 1024 || c->page_pool_tiles < 0) return BGTQ_ERR_INVALID_ARG;
   if (c->capacity_tokens < 1 || c->capacity_tokens > (int64_t(1) << 30)) return BGTQ_ERR_INVALID_ARG;
+  // a call's layers are a grid dimension of every launch (at most 65535)
+  if (c->n_layers > kMaxLayers) return BGTQ_ERR_INVALID_ARG;
+  // the buffer plan's byte counts, bounded before any size_t arithmetic
+  if (!sizes_in_range(c)) return BGTQ_ERR_INVALID_ARG;
   return BGTQ_OK;
 }
-
-int max_splits_of(const bgtq_config* c) { return c->max_splits == 0 ? 256 : c->max_splits; }
 
 struct Layout {
   size_t krec, knorm, vrec, vnorm, cache_total;
@@ -106,6 +126,11 @@ Layout plan(const bgtq_config* c) {
   p.comb_count = align_up(p.comb_mid + qrows * (bgtq::kCombSlices + 1) * bgtq::kPartialStride * sizeof(float));
   p.ws_total = align_up(p.comb_count + qrows * sizeof(uint32_t));
   return p;
+}
+
+// layers [layer, layer + layer_count) of the config (no overflow for any int32 inputs)
+bool layer_range_ok(const bgtq_config& c, int32_t layer, int32_t layer_count) {
+  return layer >= 0 && layer < c.n_layers && layer_count >= 1 && layer_count <= c.n_layers - layer;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -243,10 +268,9 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   return BGTQ_OK;
 }
 
-// Split-K partials per (layer, sequence, KV head, head block): one wave of
-// resident decode CTAs over all such units (the CTAs of a unit share its
-// tiles round-robin), at most max_splits and one per 4 tiles of capacity.
-// Resident split CTAs the GPU holds at once (one wave).
+// Resident split CTAs the GPU holds at once (one wave): the automatic split
+// plan spreads them over a call's (layer, sequence, KV head, head block)
+// units (see split_for).
 int split_slots(bgtq_state* st) {
   if (st->ctas_per_sm <= 0) st->ctas_per_sm = std::max(1, bgtq::decode_ctas_per_sm(st->shape));
   return st->ctas_per_sm * st->num_sms;
@@ -478,7 +502,7 @@ int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count, const
   if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
   if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
-  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
   if (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)) return BGTQ_ERR_ALIGNMENT;
   if (n == 0) return BGTQ_OK;
@@ -494,7 +518,7 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
   if (!st || !d_q || !d_qrot) return BGTQ_ERR_NULL;
   if (!st->ready) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
-  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
   if (!aligned16(d_q) || !aligned16(d_qrot)) return BGTQ_ERR_ALIGNMENT;
   return bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
@@ -508,7 +532,7 @@ namespace {
 int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, int32_t batch) {
   if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
   const bgtq_config& c = st->cfg;
-  if (layer < 0 || layer_count < 1 || layer + layer_count > c.n_layers) return BGTQ_ERR_INVALID_ARG;
+  if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
   return BGTQ_OK;
 }

@@ -45,12 +45,21 @@ def test_required_bytes_is_host_only_and_validates(lib):
     assert cache % 256 == 0 and ws % 256 == 0
     bad = [dict(head_dim=64), dict(n_q_heads=15), dict(k_avg_bits=5), dict(b_min=4, b_max=3),
            dict(k_avg_bits=1, b_min=2), dict(rope_pairing=2), dict(capacity_tokens=0), dict(max_splits=2000),
-           dict(page_pool_tiles=-1)]
+           dict(page_pool_tiles=-1), dict(n_layers=65536),
+           # sizes past 2^56 bytes (they would overflow the buffer plan's arithmetic)
+           dict(n_layers=65535, max_batch=2 ** 31 - 1, capacity_tokens=2 ** 30),
+           dict(n_layers=65535, n_kv_heads=2 ** 20, n_q_heads=2 ** 20, max_batch=2 ** 20)]
     for change in bad:
         c = bgtq.Config(**{**cfg.__dict__, **change})
         with pytest.raises(bgtq.BgtqError) as e:
             bgtq.bgtq_required_bytes(c)
         assert e.value.status == -1
+    # the largest layer count is accepted and sized exactly like a smaller one, per layer
+    one, _ = bgtq.bgtq_required_bytes(bgtq.Config(n_layers=1, n_kv_heads=1, n_q_heads=1, max_batch=1,
+                                                  capacity_tokens=64))
+    most, _ = bgtq.bgtq_required_bytes(bgtq.Config(n_layers=65535, n_kv_heads=1, n_q_heads=1, max_batch=1,
+                                                   capacity_tokens=64))
+    assert 65535 * (one - 1024) <= most <= 65535 * one
 
 
 def test_paged_cache_is_sized_by_its_pool(lib):

@@ -333,6 +333,11 @@ def test_host_side_argument_checks(dev):
     with pytest.raises(bgtq.BgtqError) as e:
         bgtq.bgtq_decode_attn(kv.state, 0, 1, q.data_ptr() + 2, seq, 1, q)
     assert e.value.status == -8
+    # layer ranges are checked without overflow (1 + (2^31 - 1) must not wrap)
+    for layer, count in [(1, 2 ** 31 - 1), (2 ** 31 - 1, 2 ** 31 - 1), (-1, 1), (0, 0), (0, 2)]:
+        with pytest.raises(bgtq.BgtqError) as e:
+            bgtq.bgtq_decode_attn(kv.state, layer, count, q, seq, 1, q.clone())
+        assert e.value.status == -1
     kv.close()
 
 

@@ -160,6 +160,28 @@ def _ptr(x):
     return x.data_ptr()
 
 
+ERR_INVALID_ARG = -1
+
+
+def _expect(t, name, shape, dtype, device):
+    """Raises BgtqError(ERR_INVALID_ARG) unless t is a contiguous torch tensor
+    of dtype on device with this shape (None: any extent).  PackedKVCache
+    checks its tensors this way before a pointer reaches the library, which
+    reads the layouts that include/bgtq.h states."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise BgtqError(ERR_INVALID_ARG, f"{name}: a torch tensor is expected")
+    if t.dtype != dtype:
+        raise BgtqError(ERR_INVALID_ARG, f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device.type != device.type or (device.index is not None and t.device.index != device.index):
+        raise BgtqError(ERR_INVALID_ARG, f"{name}: on {t.device}, expected {device}")
+    if t.dim() != len(shape) or any(e is not None and t.shape[i] != e for i, e in enumerate(shape)):
+        want = tuple("*" if e is None else e for e in shape)
+        raise BgtqError(ERR_INVALID_ARG, f"{name}: shape {tuple(t.shape)}, expected {want}")
+    if not t.is_contiguous():
+        raise BgtqError(ERR_INVALID_ARG, f"{name}: not contiguous")
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -370,64 +392,142 @@ class PackedKVCache:
         return self.cache[self.offsets[3]:self.offsets[3] + n].view(torch.float16).view(*t[:-1], t[-1] * TILE)
 
     # -- calls --
+    # Every tensor is checked against the layout its call reads (see _expect)
+    # before its pointer is passed on; counts and ranges are checked by the
+    # library itself.
+    def _q_like(self, t, name, layer_count, dtype):
+        _expect(t, name, (layer_count, None, self.cfg.n_q_heads, HEAD_DIM), dtype, self.device)
+        return t.shape[1]
+
+    def _per_seq(self, t, name, batch):
+        import torch
+        _expect(t, name, (batch,), torch.int32, self.device)
+
+    def _rows(self, k, v, start, count, layer_count, batch=None):
+        """Checks appended rows k, v [layer_count, batch, n, Hkv, 128] (batch None: any) and
+        start, count [batch]; returns (batch, n)."""
+        import torch
+        _expect(k, "k", (layer_count, batch, None, self.cfg.n_kv_heads, HEAD_DIM), torch.float16, self.device)
+        _expect(v, "v", tuple(k.shape), torch.float16, self.device)
+        self._per_seq(start, "start", k.shape[1])
+        self._per_seq(count, "count", k.shape[1])
+        return k.shape[1], k.shape[2]
+
     def allocate(self, calib_q, calib_k):
+        """calib_q fp16 [n_layers, Nq, Hq, 128], calib_k fp16 [n_layers, Nk, Hkv, 128] on the device."""
+        import torch
+        c = self.cfg
+        _expect(calib_q, "calib_q", (c.n_layers, None, c.n_q_heads, HEAD_DIM), torch.float16, self.device)
+        _expect(calib_k, "calib_k", (c.n_layers, None, c.n_kv_heads, HEAD_DIM), torch.float16, self.device)
         bgtq_allocate(self.state, calib_q, calib_q.shape[1], calib_k, calib_k.shape[1])
 
     def set_allocation(self, widths):
-        bgtq_set_allocation(self.state, widths)
+        """int8 widths [n_layers, n_kv_heads, 64] (host)."""
+        w = np.asarray(widths)
+        if w.shape != (self.cfg.n_layers, self.cfg.n_kv_heads, N_BLOCKS):
+            raise BgtqError(ERR_INVALID_ARG, f"widths: shape {w.shape}, expected "
+                                             f"{(self.cfg.n_layers, self.cfg.n_kv_heads, N_BLOCKS)}")
+        bgtq_set_allocation(self.state, w)
 
     def get_allocation(self):
         return bgtq_get_allocation(self.state, self.cfg.n_layers, self.cfg.n_kv_heads)
 
     def encode_append(self, layer, k, v, start, count, layer_count=1):
         """k, v fp16 [layer_count, batch, n, Hkv, 128]; start, count int32 [batch] on the device."""
-        bgtq_encode_append(self.state, layer, layer_count, k, v, start, count, k.shape[1], k.shape[2])
+        batch, n = self._rows(k, v, start, count, layer_count)
+        bgtq_encode_append(self.state, layer, layer_count, k, v, start, count, batch, n)
 
     def rotate_query(self, layer, q, out, layer_count=1):
-        bgtq_rotate_query(self.state, layer, layer_count, q, q.shape[1], out)
+        """q fp16 and out fp32 [layer_count, batch, Hq, 128] on the device."""
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float32, self.device)
+        bgtq_rotate_query(self.state, layer, layer_count, q, batch, out)
 
     def decode_attn(self, layer, q, seq_lens, out, layer_count=1):
         """q, out fp16 [layer_count, batch, Hq, 128]; seq_lens int32 [batch] on the device."""
-        bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, q.shape[1], out)
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float16, self.device)
+        self._per_seq(seq_lens, "seq_lens", batch)
+        bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, batch, out)
 
     def decode_step(self, layer, k, v, start, count, q, seq_lens, out, layer_count=1):
         """encode_append(k, v, start, count) then decode_attn(q, seq_lens, out), in one call (the appends
         and the query rotation share a launch when k holds at most 16 rows per sequence); k = None
         appends nothing."""
-        n = 0 if k is None else k.shape[2]
-        bgtq_decode_step(self.state, layer, layer_count, k, v, start, count, n, q, seq_lens, q.shape[1], out)
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float16, self.device)
+        self._per_seq(seq_lens, "seq_lens", batch)
+        n = 0 if k is None else self._rows(k, v, start, count, layer_count, batch)[1]
+        bgtq_decode_step(self.state, layer, layer_count, k, v, start, count, n, q, seq_lens, batch, out)
+
+    def _buffer(self, seq_lens, pos_lo, buf_k, buf_v, buf_count, layer_count, batch):
+        import torch
+        self._per_seq(seq_lens, "seq_lens", batch)
+        self._per_seq(pos_lo, "pos_lo", batch)
+        _expect(buf_k, "buf_k", (layer_count, batch, None, self.cfg.n_kv_heads, HEAD_DIM), torch.float16,
+                self.device)
+        _expect(buf_v, "buf_v", tuple(buf_k.shape), torch.float16, self.device)
+        self._per_seq(buf_count, "buf_count", batch)
+        return buf_k.shape[2]
 
     def decode_attn_buffered(self, layer, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out, layer_count=1):
         """Attention over the packed positions [pos_lo, seq_lens) and the first
         buf_count fp16 buffered rows (buf_k, buf_v fp16 [layer_count, batch,
         n_buf, Hkv, 128])."""
-        bgtq_decode_attn_buffered(self.state, layer, layer_count, q, seq_lens, pos_lo, q.shape[1], buf_k, buf_v,
-                                  buf_count, buf_k.shape[2], out)
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float16, self.device)
+        n_buf = self._buffer(seq_lens, pos_lo, buf_k, buf_v, buf_count, layer_count, batch)
+        bgtq_decode_attn_buffered(self.state, layer, layer_count, q, seq_lens, pos_lo, batch, buf_k, buf_v,
+                                  buf_count, n_buf, out)
 
     def logit_mae(self, layer, seq, w0, q, k, out, layer_count=1):
         """Per-head logit MAE of the packed keys at positions [w0, w0 + m) of
         sequence seq: q fp16 [layer_count, m, Hq, 128], k (exact keys) fp16
         [layer_count, m, Hkv, 128], out float64 [layer_count, Hq]."""
-        bgtq_logit_mae(self.state, layer, layer_count, seq, w0, q.shape[1], q, k, out)
+        import torch
+        m = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(k, "k", (layer_count, m, self.cfg.n_kv_heads, HEAD_DIM), torch.float16, self.device)
+        _expect(out, "out", (layer_count, self.cfg.n_q_heads), torch.float64, self.device)
+        bgtq_logit_mae(self.state, layer, layer_count, seq, w0, m, q, k, out)
 
     def decode_step_buffered(self, layer, k, v, start, count, q, seq_lens, pos_lo, buf_k, buf_v, buf_count, out,
                              layer_count=1):
         """encode_append(k, v, start, count) then decode_attn_buffered(...), in one call; k = None
         appends nothing."""
-        n = 0 if k is None else k.shape[2]
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float16, self.device)
+        n_buf = self._buffer(seq_lens, pos_lo, buf_k, buf_v, buf_count, layer_count, batch)
+        n = 0 if k is None else self._rows(k, v, start, count, layer_count, batch)[1]
         bgtq_decode_step_buffered(self.state, layer, layer_count, k, v, start, count, n, q, seq_lens, pos_lo,
-                                  q.shape[1], buf_k, buf_v, buf_count, buf_k.shape[2], out)
+                                  batch, buf_k, buf_v, buf_count, n_buf, out)
 
     def decode_split(self, layer, qrot, seq_lens, layer_count=1):
         """The split-K stage alone from rotated queries (fp32 [layer_count, batch, Hq, 128])."""
-        bgtq_decode_split(self.state, layer, layer_count, qrot, seq_lens, qrot.shape[1])
+        import torch
+        batch = self._q_like(qrot, "qrot", layer_count, torch.float32)
+        self._per_seq(seq_lens, "seq_lens", batch)
+        bgtq_decode_split(self.state, layer, layer_count, qrot, seq_lens, batch)
 
     def decode_combine(self, layer, seq_lens, out, layer_count=1):
-        bgtq_decode_combine(self.state, layer, layer_count, seq_lens, out.shape[1], out)
+        """The combine stage alone: out fp16 [layer_count, batch, Hq, 128]."""
+        import torch
+        batch = self._q_like(out, "out", layer_count, torch.float16)
+        self._per_seq(seq_lens, "seq_lens", batch)
+        bgtq_decode_combine(self.state, layer, layer_count, seq_lens, batch, out)
 
     def set_block_table(self, table):
         """Paged cache: int32 [max_batch, ceil(capacity / 64)] page ids on the
-        device (kept referenced here; its contents are read at kernel time)."""
+        device (kept referenced here; its contents are read at kernel time).
+        A contiguous cache rejects any table."""
+        import torch
+        c = self.cfg
+        if c.page_pool_tiles > 0 and table is not None:
+            _expect(table, "table", (c.max_batch, (c.capacity_tokens + TILE - 1) // TILE), torch.int32, self.device)
         bgtq_set_block_table(self.state, table)
         self._block_table = table
 

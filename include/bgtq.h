@@ -34,6 +34,10 @@
  *    Query head h reads KV head h / G, G = n_q_heads / n_kv_heads.
  *  - fp16 tensors are IEEE binary16, row-major, densely packed, 16-byte
  *    aligned.
+ *  - A state is not thread-safe: call it from one host thread at a time.
+ *    Its decode calls share the workspace's scratch (rotated queries, split
+ *    partials, the combine's counters), so two of its calls must not overlap
+ *    on the GPU: issue them on one stream, or order the streams.
  *
  * Cache layout inside d_cache (offsets from bgtq_cache_offsets, each
  * 256-byte aligned; L layers, B = max_batch, H = n_kv_heads, T =

@@ -8,10 +8,15 @@ packed cache (rotate the query, split-K pass, combine).  Steps run as one
 CUDA graph.  value = sequences * steps / time  (decode tokens/s).
 
 Printed as one JSON line on rank 0.  Also measured in the same run:
-  roofline      the split-K decode kernel alone, CUDA events around each launch
+  roofline      the split-K decode kernel: its per-layer launches back to back
+                in a captured graph (launch_ms) and with events around each
+                launch (launch_ms_isolated), against the measured HBM peak
   e2e           same step through the C ABI from pinned host buffers (H2D of
                 the queries and new K/V, D2H of the outputs inside the timing)
   multi_layer   all layers in one launch per kernel
+  buffered      the step with 4 fp16 sink rows and a 128-row fp16 window
+  paged         the step on a paged copy of the cache (shuffled pages)
+  logit_mae     per-layer logit MAE, Block-GTQ against uniform TQ-MSE
   fp16_baseline dense fp16 FlashAttention-2 decode over the unquantised K/V
   cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU)
 

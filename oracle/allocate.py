@@ -1,5 +1,7 @@
 """Greedy integer bit allocation by marginal gain, and the group layout.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: Block-GTQ abstract ("greedily allocates integer bit widths by marginal
 gain"; "high-energy RoPE blocks ... should receive more bits") and the
 blockgtq README ("shifting bits toward high-energy blocks under a fixed

@@ -1,5 +1,7 @@
 """Dense GQA decode attention from packed records (the plain definition).
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: Block-GTQ abstract ("packed-cache serving path") and the blockgtq
 README (fused decode over the packed K3V3 cache, compared with fp16
 FlashAttention-2).  What that path computes is ordinary decode attention

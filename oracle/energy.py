@@ -1,5 +1,7 @@
 """Label-free per-RoPE-block Q/K energy score.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: Block-GTQ abstract ("for each layer and KV head, Block-GTQ computes a
 label-free energy score for each RoPE block") and the blockgtq README ("a
 Q/K energy score per block", computed from saved calibration Q/K

@@ -1,5 +1,7 @@
 """Seeded Haar-random rotations (the TQ-MSE random rotation).
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: TurboQuant-MSE, which Block-GTQ builds on (Block-GTQ abstract; blockgtq
 README, method blurb), quantises a vector after a random rotation; the pages
 do not say how the rotation is drawn or grouped.  Reading used here: one Haar

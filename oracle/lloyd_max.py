@@ -1,5 +1,7 @@
 """Gaussian Lloyd-Max scalar quantiser (the TQ-MSE codebook).
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: the Block-GTQ abstract ("built on TurboQuant-MSE (TQ-MSE)") and the
 blockgtq README (TQ-MSE encoder); TurboQuant (arXiv 2504.19874) is the cited
 source of TQ-MSE: after a random rotation each coordinate of a normalised

@@ -1,5 +1,7 @@
 """Cache-level oracle calls: allocate, encode rows, rotate the query, decode.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 These mirror the library's three calls (allocate, encode-append, decode
 attention) on plain arrays for one layer at a time.  The per-(layer, KV head)
 tables are the group layout from the allocation, one fp32 Haar rotation per

@@ -1,5 +1,7 @@
 """The packed-cache tile format: where every code bit of a 64-token tile goes.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 The pages only say that the serving path decodes attention from a packed
 cache (Block-GTQ abstract, "packed-cache serving path"; blockgtq README);
 they give no format.  This module defines the one the library stores, bit by

@@ -1,5 +1,7 @@
 """TurboQuant-MSE encode of one row per bit-width group, and the record format.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
 Pages: Block-GTQ abstract / blockgtq README -- the widths chosen by the
 allocator go to the TQ-MSE encoder, and the serving path keeps a packed
 cache of the codes.  TQ-MSE (TurboQuant, arXiv 2504.19874, cited by the

@@ -132,9 +132,9 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes,
 /* Frees the host-side state (never the caller's device buffers). NULL is a no-op. */
 void bgtq_destroy(bgtq_state* st);
 
-/* Block-GTQ allocation ("for each layer and KV head, computes a label-free
- * energy score for each RoPE block and greedily allocates integer bit widths
- * by marginal gain", abstract).  Score of block j: s_j = EQ_j * EK_j with
+/* Block-GTQ allocation (abstract: per layer and KV head, a label-free energy
+ * score for every RoPE block, then integer widths handed out greedily by
+ * marginal gain).  Score of block j: s_j = EQ_j * EK_j with
  * EQ_j = sum over rows and the G query heads of the group of ||q_j||^2 and
  * EK_j = sum over rows of ||k_j||^2, accumulated exactly on the GPU (fp16 x
  * 2^24 is an integer; 128-bit sums).  Greedy: every block starts at b_min;

@@ -2,10 +2,10 @@
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-Pages: Block-GTQ abstract ("greedily allocates integer bit widths by marginal
-gain"; "high-energy RoPE blocks ... should receive more bits") and the
-blockgtq README ("shifting bits toward high-energy blocks under a fixed
-average budget").  Readings used here (the pages give no formula):
+Pages: the Block-GTQ abstract (integer widths handed out greedily by
+marginal gain, so that blocks with more energy get more bits) and the
+blockgtq README (bits move toward high-energy blocks while the average per
+dim stays fixed).  Readings used here (the pages give no formula):
 
 * budget: every block has two dims, so an average of A bits per dim over D
   dims is sum_j b_j = A * D / 2;
@@ -16,10 +16,10 @@ average budget").  Readings used here (the pages give no formula):
 * Dist(b) is the N(0,1) Lloyd-Max distortion, the fixed constants
   ``lloyd_max.DISTORTION``.
 
-Group layout (reading of "rotated once per bit-width group"): the dims of
-all blocks with the same width form one group; groups are ordered by width,
-largest first; inside a group the dims are in ascending order.  Width-0
-groups (possible only with b_min = 0) store nothing.
+Group layout (one TQ-MSE rotation per bit-width group, read as follows):
+the dims of all blocks with the same width form one group; groups are
+ordered by width, largest first; inside a group the dims are in ascending
+order.  Width-0 groups (possible only with b_min = 0) store nothing.
 """
 import numpy as np
 

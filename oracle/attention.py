@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-Pages: Block-GTQ abstract ("packed-cache serving path") and the blockgtq
-README (fused decode over the packed K3V3 cache, compared with fp16
+Pages: the Block-GTQ abstract (a serving path that attends straight from the
+packed cache) and the blockgtq README (fused decode over the packed K3V3 cache, compared with fp16
 FlashAttention-2).  What that path computes is ordinary decode attention
 over the dequantised cache:
 

@@ -2,9 +2,9 @@
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-Pages: the Block-GTQ abstract (Block-GTQ "better preserves RoPE query-key
-logits", per-layer MAE lowered against uniform TQ-MSE at 2 and 3 bits per
-dim, K-only quantisation) and the blockgtq README, bit allocation
+Pages: the Block-GTQ abstract (Block-GTQ keeps the RoPE query-key logits
+closer to exact: a lower per-layer MAE than uniform TQ-MSE at 2 and 3 bits
+per dim, with only K quantised) and the blockgtq README, bit allocation
 (`bench_perlayer_diag.py ... --avg-bits 3 --window-M 1024`, per-layer kernel
 MAE table).  The pages do not define the window or the averaging; the
 reading used here is the plain one:

@@ -2,10 +2,10 @@
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-Pages: Block-GTQ abstract ("for each layer and KV head, Block-GTQ computes a
-label-free energy score for each RoPE block") and the blockgtq README ("a
-Q/K energy score per block", computed from saved calibration Q/K
-activations).  The formula is not printed.  Reading used here:
+Pages: the Block-GTQ abstract (a label-free energy score for every RoPE
+block, computed separately per layer and KV head) and the blockgtq README
+(the score combines Q and K, taken from saved calibration activations).  The
+formula is not printed.  Reading used here:
 
   under RoPE, q . k = sum_j q_j^T R(theta_j (m - n)) k_j over the D/2
   two-dimensional blocks j; averaged over the relative phase,

@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
 The pages only say that the serving path decodes attention from a packed
-cache (Block-GTQ abstract, "packed-cache serving path"; blockgtq README);
+cache (Block-GTQ abstract, its serving path; blockgtq README);
 they give no format.  This module defines the one the library stores, bit by
 bit, so that both sides pack identically.  Codes are those of ``tqmse``
 (record order: width groups widest first, rotated coordinates in order).

@@ -4,8 +4,8 @@
 //    Block-GTQ pages build on;
 //  * Haar rotation: SplitMix64 (Steele et al. 2014) -> Box-Muller (1958) ->
 //    Householder QR with Mezzadri's (2007) sign fix;
-//  * greedy marginal-gain bit allocation, as the Block-GTQ abstract states
-//    ("greedily allocates integer bit widths by marginal gain").
+//  * greedy marginal-gain bit allocation: the Block-GTQ abstract assigns
+//    integer widths one greedy step at a time by their marginal gain.
 #include "host_tables.h"
 
 #include <algorithm>

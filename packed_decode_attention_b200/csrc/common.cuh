@@ -302,7 +302,7 @@ __device__ void pack_v_tile(uint32_t* tw, const uint8_t (*codes)[kCodePitch], in
   }
 
 // ---------------------------------------------------------------------------
-// a4: rotate the query.  Grid (layer_count * batch * Hq), 128 threads.
+// Query rotation.  Grid (layer_count * batch * Hq), 128 threads.
 // ---------------------------------------------------------------------------
 constexpr int kRotThreads = 256;
 

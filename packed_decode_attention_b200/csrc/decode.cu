@@ -15,7 +15,7 @@ namespace bgtq {
 namespace {
 
 // ---------------------------------------------------------------------------
-// a5: split-K decode straight from the packed tiles on the tensor cores.
+// Split-K decode straight from the packed tiles on the tensor cores.
 //
 // Grid (batch * Hkv * head_blocks, c_max, layer_count), 128 threads.  The
 // split CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// a6: combine the splits and rotate back.  Grid (layer_count*batch*Hq *
+// Combine the splits and rotate back.  Grid (layer_count*batch*Hq *
 // kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
 // (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated coordinates) into
 // an intermediate (m, l, acc) in V's rotated basis.  In a buffered call the

@@ -13,7 +13,7 @@ namespace bgtq {
 namespace {
 
 // ---------------------------------------------------------------------------
-// f2: per-layer logit MAE of the packed keys (K only).  For every causal pair
+// Per-layer logit MAE of the packed keys (K only).  For every causal pair
 // (query i, key j), 0 <= j <= i < m, of a window of m cached positions
 // w0 .. w0+m-1: |q_i . k_hat_j - q_i . k_j| / sqrt(D), where q_i . k_hat_j is
 // the logit exactly as the split decode computes it (group_logits on the

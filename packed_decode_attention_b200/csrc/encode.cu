@@ -31,7 +31,7 @@ __device__ __forceinline__ uint64_t fp16_fixed(uint16_t bits, uint32_t* nonfinit
 }
 
 // ---------------------------------------------------------------------------
-// a1: energy.  Grid (L * Hkv, kEnergyChunks), 128 threads = one per dim.
+// Energy score.  Grid (L * Hkv, kEnergyChunks), 128 threads = one per dim.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ q, int nq,
                                                      const __half* __restrict__ k, int nk, int Hq,
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
 
 
 // ---------------------------------------------------------------------------
-// a3: encode.  Grid (layer_count * batch * Hkv, per_unit, 2 kinds), 256
+// Encode.  Grid (layer_count * batch * Hkv, per_unit, 2 kinds), 256
 // threads.  A CTA loads one (layer, KV head, kind)'s rotation and tables once
 // and then takes every per_unit-th 64-position tile that the call writes for
 // one sequence: it unpacks the tile's codes when the call writes only part of

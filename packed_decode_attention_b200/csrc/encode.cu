@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
 }
 
 // ---------------------------------------------------------------------------
-// a3 for a few rows (decode-time appends): grid (layer_count * batch * Hkv,
+// Encode for a few rows (decode-time appends): grid (layer_count * batch * Hkv,
 // n, 2 kinds), 128 threads.  A CTA encodes one new row of one (layer,
 // sequence, KV head) and kind with the same arithmetic as encode_kernel
 // (norms summed in fp64 in coordinate order, y = sum_j R[i][j] x_j in fp32

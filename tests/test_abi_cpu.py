@@ -30,6 +30,50 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
     assert sorted(bgtq.declared_symbols()) == names
 
 
+def _header_prototypes():
+    """{name: (return type, [parameter declarations])} from include/bgtq.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for ret, name, args in re.findall(r"([A-Za-z_][\w\s\*]*?)\b(bgtq_[a-z_]+)\s*\(([^)]*)\)\s*;", text):
+        params = [a.strip() for a in args.split(",") if a.strip() and a.strip() != "void"]
+        out[name] = (" ".join(ret.split()), params)
+    return out
+
+
+def _ctype_of(decl):
+    """The ctypes type a C parameter declaration must be bound with (None: any
+    pointer type, c_void_p or a typed ctypes pointer)."""
+    import ctypes
+    if "*" in decl:
+        return None
+    base = decl.rsplit(" ", 1)[0]
+    return {"int32_t": ctypes.c_int32, "size_t": ctypes.c_size_t}[base]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes signature has the header's parameter count and, parameter
+    by parameter, the same kind (pointer, int32, size_t) and return type: a
+    mismatch would shift every later argument of the call."""
+    import ctypes
+    protos = _header_prototypes()
+    assert sorted(protos) == header_functions()
+    for name, (ret, params) in protos.items():
+        res, args = bgtq._SIGS[name]
+        assert len(args) == len(params), (name, len(args), len(params))
+        for decl, bound in zip(params, args):
+            want = _ctype_of(decl)
+            if want is None:
+                assert bound is ctypes.c_void_p or issubclass(bound, ctypes._Pointer), (name, decl)
+            else:
+                assert bound is want, (name, decl, bound)
+        if ret == "void":
+            assert res is None, name
+        elif ret == "int":
+            assert res is ctypes.c_int, name
+        else:
+            assert ret.startswith("const char") and res is ctypes.c_char_p, (name, ret)
+
+
 def test_error_strings(lib):
     assert bgtq.bgtq_error_string(0) == "ok"
     assert bgtq.bgtq_error_string(-1) == "invalid argument"

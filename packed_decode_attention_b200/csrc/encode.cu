@@ -287,7 +287,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
       }
     }
     __syncthreads();
-    // norms: fp64 sum of squares of the exact fp16 inputs
+    // norms: fp64 sum of squares of the exact fp16 inputs (of the turned
+    // fp32 values when K arrives before RoPE)
     {
       const int r = tid >> 2, g = tid & 3;
       float f = 0.f;

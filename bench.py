@@ -661,6 +661,26 @@ def main():
                 "note": "K-only logit MAE (q.k / sqrt(128)) over causal pairs, synthetic Q/K"}
         del qd, kd
 
+    # ---- the fused RoPE + encode (K before RoPE), timed after every decode
+    # measurement: it rewrites the first chunk of layer 0 ----
+    n_r = min(chunk, lens[0])
+    kk = torch.zeros((1, B, n_r, H, 128), dtype=torch.float16, device=dev)
+    kk[0, 0] = wl.keys(w, 0, 0, 0, n_r, device=dev)
+    st0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    c0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    c0[0] = n_r
+    rope_ms = []
+    for it in range(4):
+        e0.record()
+        kv.encode_append(0, kk, kk, st0, c0, rope_base=w.rope_base)
+        e1.record()
+        torch.cuda.synchronize()
+        if it:
+            rope_ms.append(e0.elapsed_time(e1))
+    assert kv.device_error() == 0, "device error in the fused RoPE + encode"
+    rope_rows_per_s = n_r * H / (statistics.mean(rope_ms) * 1e-3)
+    del kk
+
     # ---- CPU oracle on a bounded sample ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -700,6 +720,7 @@ def main():
         "allocate_ms": alloc_ms,
         "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),
         "prefill_encode_call_rows": chunk,
+        "prefill_encode_rope_rows_per_s": rope_rows_per_s,
         "compression_vs_fp16": 512.0 / (sum(lens[b] * tb[l, h] for l in range(L) for b in range(B) for h in range(H))
                                         / (sum(lens) * L * H)),
     }

@@ -11,6 +11,7 @@
  *
  *   bgtq_allocate       energy score per block + greedy allocation + tables
  *   bgtq_encode_append  rotate, normalise, Lloyd-Max quantise, bit-pack K/V
+ *   bgtq_encode_append_rope  the same from K before RoPE (RoPE fused in)
  *   bgtq_rotate_query   the query in each width group's rotated basis
  *   bgtq_decode_attn    one GQA decode step over the packed cache
  *   bgtq_decode_step    encode_append of a step's rows + decode_attn in one call
@@ -198,6 +199,23 @@ int bgtq_cache_offsets(const bgtq_state* st, size_t* out);
 int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count,
                        const void* d_k, const void* d_v, const int32_t* d_start,
                        const int32_t* d_count, int32_t batch, int32_t n, void* stream);
+
+/* The fused RoPE + encode: bgtq_encode_append with the K rows taken before
+ * RoPE (the key projection's output).  Row r of sequence b is turned by
+ * RoPE at its cache position p = start[b] + r before it is encoded: block j
+ * of the config's rope_pairing (dims (j, j+64) or (2j, 2j+1)) becomes
+ * (a cos t - b sin t, a sin t + b cos t) with t = p * rope_base^(-2j/128),
+ * the product in fp64 reduced to [-pi, pi], sin and cos in fp32.  The
+ * turned values are encoded in fp32 without rounding to fp16.  Groups hold
+ * whole RoPE blocks, so a group's norm is that of the row as given, up to
+ * the rounding of the turned values.
+ * V rows are encoded as in bgtq_encode_append.  rope_base: finite, > 1
+ * (BGTQ_ERR_INVALID_ARG otherwise).  Arguments, layouts and device errors
+ * otherwise as bgtq_encode_append.  ASYNC. */
+int bgtq_encode_append_rope(bgtq_state* st, int32_t layer, int32_t layer_count,
+                            const void* d_k, const void* d_v, const int32_t* d_start,
+                            const int32_t* d_count, int32_t batch, int32_t n, double rope_base,
+                            void* stream);
 
 /* q~ in record order: per K group g, (1/sqrt(128)) (1/sqrt(d_g)) R_g q[D_g].
  *   d_q     fp16 [layer_count][batch][n_q_heads][128]

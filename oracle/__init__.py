@@ -23,4 +23,5 @@ tqmse       rotate / normalise / quantise one row; bit-pack a record.
 attention   dense decode attention from packed records.
 model       the per-(layer, KV head) tables and the cache-level calls.
 diag        the per-layer logit MAE of a packed key cache (K only).
+rope        rotary position embedding of key rows (the fused RoPE + encode).
 """

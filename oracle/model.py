@@ -20,7 +20,7 @@ from dataclasses import dataclass
 import numpy as np
 
 from . import allocate as alloc
-from . import energy, haar, lloyd_max, tiles, tqmse
+from . import energy, haar, lloyd_max, rope, tiles, tqmse
 from .attention import attend, dequantise_keys, dequantise_values
 
 KIND_K = 0
@@ -90,9 +90,25 @@ def encode_rows(tables, layer, head, k_rows, v_rows):
     Returns a dict with the cache bytes (k_tiles, k_norms, v_tiles, v_norm;
     the tiles padded with code 0 past row n) and the codes in record order.
     """
-    cfg = tables.cfg
     k = np.asarray(k_rows, dtype=np.float16).astype(np.float64)
     v = np.asarray(v_rows, dtype=np.float16).astype(np.float64)
+    return _encode(tables, layer, head, k, v)
+
+
+def encode_rows_rope(tables, layer, head, k_rows, v_rows, positions, base):
+    """The fused RoPE + encode: fp16 keys [n, D] taken before RoPE, turned by
+    RoPE at their positions [n] with the given base (the configuration's
+    pairing) in float64 and encoded without rounding the turned values;
+    values as in encode_rows.  Same result layout as encode_rows."""
+    k = np.asarray(k_rows, dtype=np.float16).astype(np.float64)
+    k = rope.apply_rope(k, positions, base, tables.cfg.pairing)
+    v = np.asarray(v_rows, dtype=np.float16).astype(np.float64)
+    return _encode(tables, layer, head, k, v)
+
+
+def _encode(tables, layer, head, k, v):
+    """encode_rows on float64 rows k, v [n, D]."""
+    cfg = tables.cfg
     n = k.shape[0]
     groups = tables.groups[layer, head]
     k_codes = []

@@ -107,6 +107,8 @@ _SIGS = {
     "bgtq_get_rotation": (ctypes.c_int, [_VP, _I32, _I32, _I32, _I32, _VP, _VP]),
     "bgtq_cache_offsets": (ctypes.c_int, [_VP, _VP]),
     "bgtq_encode_append": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
+    "bgtq_encode_append_rope": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32, ctypes.c_double,
+                                               _VP]),
     "bgtq_rotate_query": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_buffered": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _VP, _I32, _VP, _VP, _VP, _I32, _VP, _VP]),
@@ -267,6 +269,12 @@ def bgtq_cache_offsets(state):
 def bgtq_encode_append(state, layer, layer_count, d_k, d_v, d_start, d_count, batch, n, stream=None):
     _check(lib().bgtq_encode_append(state, layer, layer_count, _ptr(d_k), _ptr(d_v), _ptr(d_start), _ptr(d_count),
                                     batch, n, _stream(stream)))
+
+
+def bgtq_encode_append_rope(state, layer, layer_count, d_k, d_v, d_start, d_count, batch, n, rope_base,
+                            stream=None):
+    _check(lib().bgtq_encode_append_rope(state, layer, layer_count, _ptr(d_k), _ptr(d_v), _ptr(d_start),
+                                         _ptr(d_count), batch, n, float(rope_base), _stream(stream)))
 
 
 def bgtq_rotate_query(state, layer, layer_count, d_q, batch, d_qrot, stream=None):
@@ -432,10 +440,15 @@ class PackedKVCache:
     def get_allocation(self):
         return bgtq_get_allocation(self.state, self.cfg.n_layers, self.cfg.n_kv_heads)
 
-    def encode_append(self, layer, k, v, start, count, layer_count=1):
-        """k, v fp16 [layer_count, batch, n, Hkv, 128]; start, count int32 [batch] on the device."""
+    def encode_append(self, layer, k, v, start, count, layer_count=1, rope_base=None):
+        """k, v fp16 [layer_count, batch, n, Hkv, 128]; start, count int32 [batch] on the device.
+        rope_base given: k is taken before RoPE and turned inside the encode
+        (bgtq_encode_append_rope)."""
         batch, n = self._rows(k, v, start, count, layer_count)
-        bgtq_encode_append(self.state, layer, layer_count, k, v, start, count, batch, n)
+        if rope_base is None:
+            bgtq_encode_append(self.state, layer, layer_count, k, v, start, count, batch, n)
+        else:
+            bgtq_encode_append_rope(self.state, layer, layer_count, k, v, start, count, batch, n, rope_base)
 
     def rotate_query(self, layer, q, out, layer_count=1):
         """q fp16 and out fp32 [layer_count, batch, Hq, 128] on the device."""

@@ -513,6 +513,25 @@ int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count, const
              : BGTQ_ERR_CUDA;
 }
 
+int bgtq_encode_append_rope(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_k, const void* d_v,
+                            const int32_t* d_start, const int32_t* d_count, int32_t batch, int32_t n, double rope_base,
+                            void* stream) {
+  if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
+  if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
+  const bgtq_config& c = st->cfg;
+  if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
+  if (!std::isfinite(rope_base) || !(rope_base > 1.0)) return BGTQ_ERR_INVALID_ARG;
+  if (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_start) || !aligned16(d_count)) return BGTQ_ERR_ALIGNMENT;
+  if (n == 0) return BGTQ_OK;
+  const bgtq::RopeArgs rope{rope_base, c.rope_pairing, 1};
+  return bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, static_cast<const __half*>(d_k),
+                             static_cast<const __half*>(d_v), d_start, d_count, batch, n, as_stream(stream), rope) ==
+                 cudaSuccess
+             ? BGTQ_OK
+             : BGTQ_ERR_CUDA;
+}
+
 int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q, int32_t batch, float* d_qrot,
                       void* stream) {
   if (!st || !d_q || !d_qrot) return BGTQ_ERR_NULL;

@@ -101,6 +101,15 @@ struct Shape {
   int32_t pad;
 };
 
+// RoPE applied inside the encode (K rows taken before RoPE): block j of the
+// pairing (0: dims (j, j+64); 1: (2j, 2j+1)) is turned by the angle
+// position * base^(-2j/128).  on = 0: the rows are taken as they are.
+struct RopeArgs {
+  double base;
+  int32_t pairing;
+  int32_t on;
+};
+
 // Error flag bits (same values as BGTQ_DEVERR_* in bgtq.h).
 constexpr uint32_t kErrCapacity = 1;
 constexpr uint32_t kErrSeqLen = 2;
@@ -114,7 +123,8 @@ cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* cal
                           const __half* calib_k, int nk, int pairing, cudaStream_t stream);
 cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                           int layer_count, const __half* k, const __half* v, const int32_t* start,
-                          const int32_t* count, int batch, int n, cudaStream_t stream);
+                          const int32_t* count, int batch, int n, cudaStream_t stream,
+                          RopeArgs rope = RopeArgs{0.0, 0, 0});
 cudaError_t launch_rotate_query(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                                 const __half* q, int batch, float* qrot, cudaStream_t stream);
 // Calls with at most this many rows per sequence append row by row (the

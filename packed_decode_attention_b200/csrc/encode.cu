@@ -101,8 +101,25 @@ __device__ __forceinline__ int lloyd_code(const float* t, int w, float u) {
   return c;
 }
 
+// RoPE inside the encode: sin and cos of the angle p * theta of one block
+// (theta = base^(-2j/D)), the product in fp64 reduced to [-pi, pi] with 2 pi
+// split into two doubles, then the hardware sin / cos of the remainder
+// (absolute error about 4e-7 on [-pi, pi]).
+__device__ __forceinline__ void rope_sincos(double theta, int64_t p, float* s, float* c) {
+  const double a = static_cast<double>(p) * theta;
+  const double k = rint(a * 0.15915494309189535);  // a / (2 pi), to the nearest integer
+  double r = fma(-k, 6.283185307179586, a);
+  r = fma(-k, 2.4492935982947064e-16, r);
+  __sincosf(static_cast<float>(r), s, c);
+}
+
+__device__ __forceinline__ double rope_theta(const RopeArgs& rope, int j) {
+  return pow(rope.base, -2.0 * j / kD);
+}
+
 struct EncodeSmem {
   float xt[kD][kTile];           // new rows, transposed, record order (zero elsewhere), columns xt_col
+  double theta[kD / 2];          // RoPE frequencies of the 64 blocks (rope.on only)
   float mt[kD][kD];              // mt[j][c(i)] = R[i][j] (record order), c(8 o + 4 q + e) = 64 q + 4 o + e
   float fac[kTile][kNumGroupsMax];
   __half nrm[kTile][kNumGroupsMax];
@@ -114,11 +131,14 @@ struct EncodeSmem {
   LayoutDev lay;
 };
 
+// TURN: K rows arrive before RoPE and are turned on load (see RopeArgs).
+template <bool TURN>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
                                                              const __half* __restrict__ kx,
                                                              const __half* __restrict__ vx,
                                                              const int32_t* __restrict__ start_v,
-                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+                                                             const int32_t* __restrict__ count_v, int batch, int n,
+                                                             RopeArgs rope) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   EncodeSmem& S = *reinterpret_cast<EncodeSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -160,6 +180,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     }
   }
   for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
+  const bool turn = TURN && kind == 0;  // K rows taken before RoPE
+  if (turn && tid < kD / 2) S.theta[tid] = rope_theta(rope, tid);
   const float* mglob = (kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD;
   // columns swizzled so that the 16 output groups of a warp read the first
   // and the second half of their 8 columns as two contiguous 256-byte spans
@@ -212,22 +234,61 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
     const __half* x = kind == 0 ? kx : vx;
     const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
                           static_cast<size_t>(h) * kD;
-    for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
-      const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (r >= tr0 && r < tr1)
-        raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
-      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+    if (!turn) {
+      for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
+        const int r = e >> 4, c8 = e & 15;  // row, 8 coordinates
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+        if (r >= tr0 && r < tr1)
+          raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
   #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = __half22float2(h2[k]);
-        const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
-        S.xt[j0][xt_col(j0, r)] = f.x;
-        S.xt[j1][xt_col(j1, r)] = f.y;
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __half22float2(h2[k]);
+          const int j0 = S.inv[8 * c8 + 2 * k], j1 = S.inv[8 * c8 + 2 * k + 1];
+          S.xt[j0][xt_col(j0, r)] = f.x;
+          S.xt[j1][xt_col(j1, r)] = f.y;
+        }
+      }
+    } else {
+      // K before RoPE: a thread takes 8 blocks (8 c .. 8 c + 7) of a row,
+      // both dims of each, and turns them by RoPE at the row's position
+      for (int e = tid; e < kTile * 8; e += kEncThreads) {
+        const int r = e >> 3, c = e & 7;
+        float xa[8], xb[8];
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) xa[i] = xb[i] = 0.f;
+        if (r >= tr0 && r < tr1) {
+          const __half* xr = xbase + static_cast<size_t>(r - tr0) * row_stride;
+          // pairing 0: dims 8 c + i and 64 + 8 c + i; pairing 1: dims 16 c + 2 i and 16 c + 2 i + 1
+          const uint4 u0 = *reinterpret_cast<const uint4*>(xr + (rope.pairing == 0 ? 8 * c : 16 * c));
+          const uint4 u1 = *reinterpret_cast<const uint4*>(xr + (rope.pairing == 0 ? kD / 2 + 8 * c : 16 * c + 8));
+          const __half* h0 = reinterpret_cast<const __half*>(&u0);
+          const __half* h1 = reinterpret_cast<const __half*>(&u1);
+          const int64_t p = tile * kTile + r;
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a = rope.pairing == 0 ? __half2float(h0[i]) : __half2float(i < 4 ? h0[2 * i] : h1[2 * i - 8]);
+            const float bv =
+                rope.pairing == 0 ? __half2float(h1[i]) : __half2float(i < 4 ? h0[2 * i + 1] : h1[2 * i - 7]);
+            float sn, cs;
+            rope_sincos(S.theta[8 * c + i], p, &sn, &cs);
+            xa[i] = fmaf(a, cs, -bv * sn);
+            xb[i] = fmaf(a, sn, bv * cs);
+          }
+        }
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = 8 * c + i;
+          const int da = rope.pairing == 0 ? j : 2 * j, db = rope.pairing == 0 ? j + kD / 2 : 2 * j + 1;
+          const int ja = S.inv[da], jb = S.inv[db];
+          S.xt[ja][xt_col(ja, r)] = xa[i];
+          S.xt[jb][xt_col(jb, r)] = xb[i];
+        }
       }
     }
     __syncthreads();
-    // norms: fp64 sum of squares of the exact fp16 inputs
+    // norms: fp64 sum of squares of the exact fp16 inputs (of the turned
+    // fp32 values when K arrives before RoPE)
     {
       const int r = tid >> 2, g = tid & 3;
       float f = 0.f;
@@ -382,11 +443,12 @@ __device__ __forceinline__ int v_code_word(int vb, int i, int p, int k, int& sel
 // One appended row of one (layer, sequence, KV head) and kind, by a CTA of
 // NT >= 128 threads: bx = (layer, sequence, KV head) index, row < n, kind 0
 // = K, 1 = V; mts = 64 KB of shared memory for the rotation.
-template <int NT>
+template <int NT, bool TURN>
 __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws, const CacheDev& cache, int layer0,
                                             const __half* __restrict__ kx, const __half* __restrict__ vx,
                                             const int32_t* __restrict__ start_v, const int32_t* __restrict__ count_v,
-                                            int batch, int n, int bx, int row, int kind, float* mts) {
+                                            int batch, int n, int bx, int row, int kind, float* mts,
+                                            RopeArgs rope) {
   const int tid = threadIdx.x;
   const int h = bx % sh.n_kv_heads;
   const int b = (bx / sh.n_kv_heads) % batch;
@@ -433,9 +495,16 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   // position i holds dim perm[i] (K), V keeps the dims
   const __half* x = (kind == 0 ? kx : vx) +
                     ((static_cast<size_t>(li) * batch + b) * n + row) * sh.n_kv_heads * kD + static_cast<size_t>(h) * kD;
-  float xv = 0.f;
+  float xv = 0.f, xpv = 0.f;
+  const bool turn = TURN && kind == 0;  // K before RoPE
+  int dim = 0;
   if (kind == 0) {
-    if (tid < lay.n_positions) xv = __half2float(x[lay.perm[tid]]);
+    if (tid < lay.n_positions) {
+      dim = lay.perm[tid];
+      xv = __half2float(x[dim]);
+      // the other dim of this dim's RoPE block
+      if (turn) xpv = __half2float(x[rope.pairing == 0 ? dim ^ (kD / 2) : dim ^ 1]);
+    }
   } else if (tid < kD) {
     xv = __half2float(x[tid]);
   }
@@ -450,6 +519,14 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   if (pos >= sh.capacity) {
     if (tid == 0) atomicOr(ws.err, kErrCapacity);
     return;
+  }
+  if (turn && tid < lay.n_positions) {
+    // block (a, b) turns to (a cos - b sin, a sin + b cos)
+    const bool first = rope.pairing == 0 ? dim < kD / 2 : (dim & 1) == 0;
+    const int j = rope.pairing == 0 ? dim & (kD / 2 - 1) : dim >> 1;
+    float sn, cs;
+    rope_sincos(rope_theta(rope, j), pos, &sn, &cs);
+    xv = first ? fmaf(xv, cs, -xpv * sn) : fmaf(xpv, sn, xv * cs);
   }
   if (tid < kD) xs[tid] = xv;
   __syncthreads();
@@ -530,14 +607,16 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   }
 }
 
+template <bool TURN>
 __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
                                                              const __half* __restrict__ kx,
                                                              const __half* __restrict__ vx,
                                                              const int32_t* __restrict__ start_v,
-                                                             const int32_t* __restrict__ count_v, int batch, int n) {
+                                                             const int32_t* __restrict__ count_v, int batch, int n,
+                                                             RopeArgs rope) {
   extern __shared__ __align__(16) float mts[];  // [kD][kD]
-  append_body<kAppThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, blockIdx.x, blockIdx.y,
-                           blockIdx.z, mts);
+  append_body<kAppThreads, TURN>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, blockIdx.x, blockIdx.y,
+                                 blockIdx.z, mts, rope);
 }
 
 // One query row (layer, sequence, query head) = bx, by a CTA of kRotThreads.
@@ -608,13 +687,24 @@ __global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace w
     rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
   } else {
     const int a = blockIdx.x - n_rot;
-    append_body<kRotThreads>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, a % n_units,
-                             (a / n_units) % n, a / (n_units * n), mts);
+    append_body<kRotThreads, false>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, a % n_units,
+                                    (a / n_units) % n, a / (n_units * n), mts, RopeArgs{0.0, 0, 0});
   }
 }
 
 cudaError_t encode_smem_once() {
-  static const cudaError_t status = set_smem(encode_kernel, sizeof(EncodeSmem));
+  static const cudaError_t status = set_smem(encode_kernel<false>, sizeof(EncodeSmem));
+  return status;
+}
+
+cudaError_t encode_rope_smem_once() {
+  static const cudaError_t status = set_smem(encode_kernel<true>, sizeof(EncodeSmem));
+  return status;
+}
+
+template <bool TURN>
+cudaError_t append_smem_once() {
+  static const cudaError_t status = set_smem(append_kernel<TURN>, kD * kD * sizeof(float));
   return status;
 }
 
@@ -636,16 +726,19 @@ cudaError_t launch_energy(const Shape& s, const Workspace& ws, const __half* cal
 
 cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                           int layer_count, const __half* k, const __half* v, const int32_t* start,
-                          const int32_t* count, int batch, int n, cudaStream_t stream) {
+                          const int32_t* count, int batch, int n, cudaStream_t stream, RopeArgs rope) {
   if (n <= 0) return cudaSuccess;
-  const cudaError_t e = encode_smem_once();
+  const cudaError_t e = rope.on ? encode_rope_smem_once() : encode_smem_once();
   if (e != cudaSuccess) return e;
   if (n <= kAppendMaxRows) {
     // a few rows per sequence: rewrite only their code bits
-    static const cudaError_t attr = set_smem(append_kernel, kD * kD * sizeof(float));
+    const cudaError_t attr = rope.on ? append_smem_once<true>() : append_smem_once<false>();
     if (attr != cudaSuccess) return attr;
-    return launch_dependent(append_kernel, dim3(layer_count * batch * s.n_kv_heads, n, 2), dim3(kAppThreads),
-                            kD * kD * sizeof(float), stream, s, ws, cache, layer0, k, v, start, count, batch, n);
+    const dim3 agrid(layer_count * batch * s.n_kv_heads, n, 2);
+    return rope.on ? launch_dependent(append_kernel<true>, agrid, dim3(kAppThreads), kD * kD * sizeof(float), stream,
+                                      s, ws, cache, layer0, k, v, start, count, batch, n, rope)
+                   : launch_dependent(append_kernel<false>, agrid, dim3(kAppThreads), kD * kD * sizeof(float), stream,
+                                      s, ws, cache, layer0, k, v, start, count, batch, n, rope);
   }
   // CTAs per unit: at least two waves if every unit has rows, and at most
   // kEncTilesPerCta tiles per CTA (the counts are device data: a call may
@@ -663,7 +756,12 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
   const int per_unit = std::max((tiles + kEncTilesPerCta - 1) / kEncTilesPerCta,
                                 std::min(tiles, std::max(1, (4 * sms) / (2 * units))));
   dim3 grid(units, per_unit, 2);
-  encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count, batch, n);
+  if (rope.on)
+    encode_kernel<true><<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count,
+                                                                          batch, n, rope);
+  else
+    encode_kernel<false><<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count,
+                                                                           batch, n, rope);
   return cudaGetLastError();
 }
 

@@ -47,7 +47,7 @@ def _ctype_of(decl):
     if "*" in decl:
         return None
     base = decl.rsplit(" ", 1)[0]
-    return {"int32_t": ctypes.c_int32, "size_t": ctypes.c_size_t}[base]
+    return {"int32_t": ctypes.c_int32, "size_t": ctypes.c_size_t, "double": ctypes.c_double}[base]
 
 
 def test_binding_signatures_match_the_header(lib):

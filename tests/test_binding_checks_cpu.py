@@ -51,6 +51,7 @@ def test_matching_tensors_reach_the_library(kv):
     assert status(kv.encode_append, 0, k, k.clone(), s, s, layer_count=L) == ERR_NULL
     kd = h(L, 40, 2, 128)
     assert status(kv.encode_append, 0, kd[:, None], kd[:, None], i32(1), i32(1), layer_count=L) == ERR_NULL
+    assert status(kv.encode_append, 0, k, k, s, s, layer_count=L, rope_base=1e6) == ERR_NULL
     assert status(kv.rotate_query, 0, q, torch.zeros(q.shape), layer_count=L) == ERR_NULL
     assert status(kv.decode_attn, 0, q, s, out, layer_count=L) == ERR_NULL
     assert status(kv.decode_attn, 1, q[1:2], s, out[1:2]) == ERR_NULL

@@ -35,6 +35,10 @@
  *    Query head h reads KV head h / G, G = n_q_heads / n_kv_heads.
  *  - fp16 tensors are IEEE binary16, row-major, densely packed, 16-byte
  *    aligned.
+ *  - A state belongs to the CUDA device that was current at bgtq_create
+ *    (its buffers live there).  Every call that launches work or copies
+ *    returns BGTQ_ERR_INVALID_ARG, launching nothing, when another device
+ *    is current.
  *  - A state is not thread-safe: call it from one host thread at a time.
  *    Its decode calls share the workspace's scratch (rotated queries, split
  *    partials, the combine's counters), so two of its calls must not overlap
@@ -185,7 +189,13 @@ int bgtq_get_rotation(const bgtq_state* st, int32_t layer, int32_t kv_head, int3
  * out[0] K tiles, out[1] K norms, out[2] V tiles, out[3] V norms. */
 int bgtq_cache_offsets(const bgtq_state* st, size_t* out);
 
-/* TQ-MSE encode + bit-pack of new rows into the cache.  For each layer
+/* TQ-MSE encode + bit-pack of new rows into the cache.  Source: the
+ * Block-GTQ abstract (the allocator's widths feed the TurboQuant-MSE
+ * encoder, and the serving path keeps a packed cache) and the blockgtq
+ * README's method blurb (integer widths on top of the TQ-MSE encoder) and
+ * packed-cache deployment path; TurboQuant (arXiv 2504.19874, cited on the
+ * mlsanity index page) for the encoder itself: a random rotation, then the
+ * Lloyd-Max scalar quantiser of each rotated coordinate.  For each layer
  * l in [layer, layer + layer_count), sequence b < batch, row r < count[b]:
  * the K and V rows at d_k/d_v[l - layer][b][r][h][:] go to cache position
  * start[b] + r of (l, b, h).  Per K width group g (dims D_g, d = |D_g|):
@@ -217,14 +227,25 @@ int bgtq_encode_append_rope(bgtq_state* st, int32_t layer, int32_t layer_count,
                             const int32_t* d_count, int32_t batch, int32_t n, double rope_base,
                             void* stream);
 
-/* q~ in record order: per K group g, (1/sqrt(128)) (1/sqrt(d_g)) R_g q[D_g].
+/* The query in each K width group's rotated basis.  Source: TurboQuant's
+ * encoder (arXiv 2504.19874, cited on the mlsanity index page) rotates each
+ * group of a key by R_g, and R_g is orthogonal, so q . R_g^T y = (R_g q) . y:
+ * the logits of the Block-GTQ abstract's packed-cache serving path can be
+ * taken from the codes once q is rotated, one rotation per width group.
+ * q~ in record order: per K group g, (1/sqrt(128)) (1/sqrt(d_g)) R_g q[D_g].
  *   d_q     fp16 [layer_count][batch][n_q_heads][128]
  *   d_qrot  fp32 [layer_count][batch][n_q_heads][128]
  * Also writes the tensor-core operand form of q~ into the workspace.  ASYNC. */
 int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                       int32_t batch, float* d_qrot, void* stream);
 
-/* One decode step: for each layer in [layer, layer + layer_count), sequence
+/* One decode step over the packed cache.  Source: the Block-GTQ abstract's
+ * packed-cache serving path (attention at 128K-512K context straight from
+ * the packed K3V3 cache) and the blockgtq README's decode benchmark and
+ * backend table (a fused decode kernel reading the packed cache); split-K
+ * decoding after FlashAttention / FlashAttention-2 (arXiv 2205.14135,
+ * 2307.08691, cited on the mlsanity index page).
+ * For each layer in [layer, layer + layer_count), sequence
  * b < batch and query head h,
  *   out = sum_t softmax_t(q . k_hat_t / sqrt(128)) v_hat_t over cache
  *   positions t < seq_lens[b],
@@ -238,7 +259,11 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
 int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const void* d_q,
                      const int32_t* d_seq_lens, int32_t batch, void* d_out, void* stream);
 
-/* One decode step of a layer range: bgtq_encode_append of the step's new
+/* One decode step of a layer range as a serving loop runs it: the step's
+ * new K/V rows go into the packed cache, then attention reads it (the
+ * Block-GTQ abstract's packed-cache serving path; the blockgtq README's
+ * decode benchmark, which times decode steps at a given context length).
+ * bgtq_encode_append of the step's new
  * rows followed by bgtq_decode_attn, with the same arguments, results and
  * errors as those two calls in that order (seq_lens should count the new
  * rows).  With 1 <= n <= 16 rows per sequence the appends and the query
@@ -342,7 +367,10 @@ int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, cons
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any
- * stream capture.  Every call on a device shares the one array and reads
+ * stream capture.  The address is kept for the life of the process: after
+ * cudaDeviceReset (a new primary context) it is stale, so no call may
+ * follow a reset of a device the library has used.  Every call on a device
+ * shares the one array and reads
  * only what the same call wrote: calls that overlap on the GPU (different
  * streams, or different states at once) race on it.  ASYNC after the first
  * call. */

@@ -1,4 +1,4 @@
-"""TurboQuant-MSE encode of one row per bit-width group, and the record format.
+"""TurboQuant-MSE encode of one row per bit-width group (codes and norms).
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
@@ -16,11 +16,13 @@ encode, group g of width b over dims D_g (d = |D_g|):
     code_i = #{fp32 thresholds <= u_i} (ties go up)
     stored norm = fp16(n), round-to-nearest-even; codes use the unrounded n.
 
-record: the codes of all groups (width-descending, rotated-coordinate order
-inside a group) as one LSB-first bitstream in little-endian 32-bit words;
-code k of width b occupies bits [o_k, o_k + b) with o_k the sum of the
-widths before it.  A record is A * D / 8 bytes for an average of A bits per
-dim -- 48 bytes for D = 128 at 3 bits.
+This module stops at the codes and norms.  The cache stores them in the
+64-position tile format of ``tiles`` (bit-plane selector words, one region
+per width group, widest group first): ``record_widths`` gives the width of
+each coordinate in record order (groups width-descending, rotated-coordinate
+order inside a group), the order ``tiles`` packs.  A position still costs
+exactly A * D bits of codes for an average of A bits per dim (48 bytes for
+D = 128 at 3 bits), plus its fp16 norms.
 """
 import numpy as np
 

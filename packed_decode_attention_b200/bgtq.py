@@ -465,6 +465,15 @@ class PackedKVCache:
         self._per_seq(seq_lens, "seq_lens", batch)
         bgtq_decode_attn(self.state, layer, layer_count, q, seq_lens, batch, out)
 
+    def decode_attn_static_scratch(self, layer, q, seq_lens, out, layer_count=1):
+        """decode_attn with its scratch in the library's static device array
+        (bgtq_decode_attn_static_scratch): same tensors, checked the same way."""
+        import torch
+        batch = self._q_like(q, "q", layer_count, torch.float16)
+        _expect(out, "out", tuple(q.shape), torch.float16, self.device)
+        self._per_seq(seq_lens, "seq_lens", batch)
+        bgtq_decode_attn_static_scratch(self.state, layer, layer_count, q, seq_lens, batch, out)
+
     def decode_step(self, layer, k, v, start, count, q, seq_lens, out, layer_count=1):
         """encode_append(k, v, start, count) then decode_attn(q, seq_lens, out), in one call (the appends
         and the query rotation share a launch when k holds at most 16 rows per sequence); k = None

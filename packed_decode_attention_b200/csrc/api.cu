@@ -27,6 +27,7 @@ struct bgtq_state {
   int split_tokens = 0;  // 0 = automatic
   int ctas_per_sm = 0;   // resident decode CTAs per SM (looked up on first use)
   int num_sms = 148;
+  int device = -1;       // the CUDA device current at bgtq_create: its buffers live there
   bool ready = false;
   bool have_energy = false;
   std::vector<int8_t> widths;                    // [L][Hkv][64]
@@ -44,6 +45,15 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Allocation set, and for a paged cache a block table given.
 bool cache_ready(const bgtq_state* st) { return st->ready && (st->cache.n_pages == 0 || st->cache.block_table); }
+
+// A call that launches or copies runs on the device the state was created
+// on: its cache, workspace and tables live there, and a launch on another
+// device would read them through the wrong context.
+int check_device(const bgtq_state* st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BGTQ_ERR_CUDA;
+  return dev == st->device ? BGTQ_OK : BGTQ_ERR_INVALID_ARG;
+}
 
 constexpr int kMaxLayers = 65535;
 
@@ -343,7 +353,12 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   const size_t comb_count_bytes = p.ws_total - p.comb_count;
   st->widths.assign(size_t(cfg->n_layers) * cfg->n_kv_heads * bgtq::kBlocks, 0);
   int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) {
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    delete st;
+    return BGTQ_ERR_CUDA;
+  }
+  st->device = dev;
+  {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) st->num_sms = sms;
   }
@@ -373,6 +388,8 @@ void bgtq_destroy(bgtq_state* st) { delete st; }
 int bgtq_allocate(bgtq_state* st, const void* d_calib_q, int32_t nq, const void* d_calib_k, int32_t nk, void* stream) {
   if (!st || !d_calib_q || !d_calib_k) return BGTQ_ERR_NULL;
   if (nq < 1 || nk < 1) return BGTQ_ERR_INVALID_ARG;
+  const int dv = check_device(st);
+  if (dv != BGTQ_OK) return dv;
   const bgtq_config& c = st->cfg;
   cudaStream_t s = as_stream(stream);
   if (bgtq::launch_energy(st->shape, st->ws, static_cast<const __half*>(d_calib_q), nq,
@@ -416,6 +433,8 @@ int bgtq_allocate(bgtq_state* st, const void* d_calib_q, int32_t nq, const void*
 
 int bgtq_set_allocation(bgtq_state* st, const int8_t* h_widths, void* stream) {
   if (!st || !h_widths) return BGTQ_ERR_NULL;
+  const int dv = check_device(st);
+  if (dv != BGTQ_OK) return dv;
   const bgtq_config& c = st->cfg;
   const size_t lh = size_t(c.n_layers) * c.n_kv_heads;
   for (size_t i = 0; i < lh; ++i) {
@@ -501,6 +520,7 @@ int bgtq_encode_append(bgtq_state* st, int32_t layer, int32_t layer_count, const
                        const int32_t* d_start, const int32_t* d_count, int32_t batch, int32_t n, void* stream) {
   if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
   if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
+  if (const int dv = check_device(st)) return dv;
   const bgtq_config& c = st->cfg;
   if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
@@ -518,6 +538,7 @@ int bgtq_encode_append_rope(bgtq_state* st, int32_t layer, int32_t layer_count, 
                             void* stream) {
   if (!st || !d_k || !d_v || !d_start || !d_count) return BGTQ_ERR_NULL;
   if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
+  if (const int dv = check_device(st)) return dv;
   const bgtq_config& c = st->cfg;
   if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch || n < 0 || n > (1 << 30) / 64) return BGTQ_ERR_INVALID_ARG;
@@ -536,6 +557,7 @@ int bgtq_rotate_query(bgtq_state* st, int32_t layer, int32_t layer_count, const 
                       void* stream) {
   if (!st || !d_q || !d_qrot) return BGTQ_ERR_NULL;
   if (!st->ready) return BGTQ_ERR_NOT_READY;
+  if (const int dv = check_device(st)) return dv;
   const bgtq_config& c = st->cfg;
   if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
@@ -550,6 +572,7 @@ namespace {
 
 int check_decode_args(const bgtq_state* st, int32_t layer, int32_t layer_count, int32_t batch) {
   if (!cache_ready(st)) return BGTQ_ERR_NOT_READY;
+  if (const int dv = check_device(st)) return dv;
   const bgtq_config& c = st->cfg;
   if (!layer_range_ok(c, layer, layer_count)) return BGTQ_ERR_INVALID_ARG;
   if (batch < 1 || batch > c.max_batch) return BGTQ_ERR_INVALID_ARG;
@@ -866,6 +889,7 @@ int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens) {
 
 int bgtq_get_device_error(bgtq_state* st, void* stream, int32_t* h_flags) {
   if (!st || !h_flags) return BGTQ_ERR_NULL;
+  if (const int dv = check_device(st)) return dv;
   cudaStream_t s = as_stream(stream);
   uint32_t flag = 0;
   cudaError_t e = cudaStreamSynchronize(s);

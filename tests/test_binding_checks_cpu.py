@@ -55,6 +55,7 @@ def test_matching_tensors_reach_the_library(kv):
     assert status(kv.rotate_query, 0, q, torch.zeros(q.shape), layer_count=L) == ERR_NULL
     assert status(kv.decode_attn, 0, q, s, out, layer_count=L) == ERR_NULL
     assert status(kv.decode_attn, 1, q[1:2], s, out[1:2]) == ERR_NULL
+    assert status(kv.decode_attn_static_scratch, 0, q, s, out, layer_count=L) == ERR_NULL
     assert status(kv.decode_step, 0, k, k, s, s, q, s, out, layer_count=L) == ERR_NULL
     assert status(kv.decode_step, 0, None, None, None, None, q, s, out, layer_count=L) == ERR_NULL
     assert status(kv.decode_attn_buffered, 0, q, s, s, bk, bk, s, out, layer_count=L) == ERR_NULL
@@ -90,6 +91,9 @@ def test_mismatched_tensors_are_refused_before_the_library(kv):
         (kv.decode_attn, (0, h(L, B, 4, 128), s, h(L, B, 4, 128)), {"layer_count": L}),  # query heads
         (kv.decode_attn, (0, q.transpose(2, 3).contiguous().transpose(2, 3), s, out), {"layer_count": L}),
         (kv.decode_attn, (0, q.numpy(), s, out), {"layer_count": L}),            # not a tensor
+        (kv.decode_attn_static_scratch, (0, q, s, h(L, B, 8, 64)), {"layer_count": L}),  # out shape
+        (kv.decode_attn_static_scratch, (0, q, i32(B + 1), out), {"layer_count": L}),    # seq_lens length
+        (kv.decode_attn_static_scratch, (0, q, s, out), {}),                              # layer_count 1 vs 2
         (kv.decode_step, (0, h(L, B + 1, 1, 2, 128), h(L, B + 1, 1, 2, 128), i32(B + 1), i32(B + 1), q, s, out),
          {"layer_count": L}),                                                    # rows of another batch
         (kv.decode_attn_buffered, (0, q, s, s, bk, h(L, B, 6, 2, 128), s, out), {"layer_count": L}),

@@ -87,3 +87,68 @@ def test_quantiser_is_nearest_centroid(bits):
     # ties go to the upper cell; zero maps to the first positive centroid
     assert np.array_equal(lm.quantise(tf.astype(np.float64), bits), np.arange(1, len(cf)))
     assert lm.quantise(np.array([0.0]), bits)[0] == 1 << (bits - 1)
+
+
+def _stored_quantiser_mse(bits):
+    """Exact E[(X - Q(X))^2] of the stored quantiser (binary16 levels, cells
+    at their midpoints) for X ~ N(0, 1), cell by cell:
+    int_a^b (x - c)^2 phi = P - (b phi(b) - a phi(a)) - 2 c (phi(a) - phi(b)) + c^2 P,
+    with P = Phi(b) - Phi(a)."""
+    def phi(x):
+        return 0.0 if math.isinf(x) else math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+
+    def xphi(x):
+        return 0.0 if math.isinf(x) else x * phi(x)
+
+    def Phi(x):
+        if math.isinf(x):
+            return 1.0 if x > 0 else 0.0
+        return 0.5 * (1.0 + math.erf(x / math.sqrt(2.0)))
+
+    cf, tf = lm.codebook_fp16(bits)
+    c = cf.astype(np.float64)
+    t = np.concatenate(([-math.inf], tf.astype(np.float64), [math.inf]))
+    total = 0.0
+    for k in range(len(c)):
+        a, b = t[k], t[k + 1]
+        p = Phi(b) - Phi(a)
+        total += p - (xphi(b) - xphi(a)) - 2.0 * c[k] * (phi(a) - phi(b)) + c[k] * c[k] * p
+    return total
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_stored_table_distortion(bits):
+    """The table both sides store (binary16 levels) keeps the Lloyd-Max
+    distortion: its exact MSE is within 1e-5 relative of the float64 optimum
+    and of the allocator's constant D(b), and never below the optimum."""
+    d = _stored_quantiser_mse(bits)
+    assert d >= lm.mse(bits) * (1 - 1e-12)
+    assert abs(d - lm.mse(bits)) <= 1e-5 * lm.mse(bits)
+    assert abs(d - lm.DISTORTION[bits]) <= 1e-5 + 5e-4 * lm.DISTORTION[bits]
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_stored_table_distortion_by_sampling(bits):
+    """Brute force: 2e6 N(0,1) samples coded with the stored thresholds and
+    reconstructed with the stored binary16 levels (not the float64 ones)
+    reproduce the closed form above within 5 standard errors."""
+    rng = np.random.default_rng(200 + bits)
+    x = rng.standard_normal(2_000_000)
+    cf, _ = lm.codebook_fp16(bits)
+    err = (x - cf.astype(np.float64)[lm.quantise(x, bits)]) ** 2
+    assert abs(err.mean() - _stored_quantiser_mse(bits)) < 5 * err.std() / math.sqrt(len(x))
+
+
+def test_stored_levels_match_max_1960_table(golden):
+    """Each stored binary16 level is within Max's printed precision (1.5 units
+    of his last digit) plus half a binary16 ulp of his Table I entry; the
+    largest gap over all 15 positive levels is 7.4e-4 (b = 2, 1.5107 vs 1.510)."""
+    worst = 0.0
+    for row in golden("lloyd_max_gaussian.txt"):
+        bits = int(row[0])
+        cf, _ = lm.codebook_fp16(bits)
+        for val, text in zip(cf[1 << (bits - 1):].astype(np.float64), row[2:]):
+            half_ulp = 2.0 ** (math.floor(math.log2(abs(val))) - 11)
+            assert abs(val - float(text)) <= _tol(text) + half_ulp, (bits, val, text)
+            worst = max(worst, abs(val - float(text)))
+    assert worst < 7.5e-4

@@ -4,26 +4,36 @@
 One step = one decode step of the whole model: for every layer, append the
 step's new token to the packed cache (TQ-MSE encode of its K and V rows at
 position len-1, so lengths stay fixed) and run GQA decode attention over the
-packed cache (rotate the query, split-K pass, combine).  Steps run as one
-CUDA graph.  value = sequences * steps / time  (decode tokens/s).
+packed cache (query rotation, split-K pass, split merge and inverse V
+rotation: one fused launch).  Steps run as one CUDA graph.
+value = sequences * steps / time (decode tokens/s).
 
 Printed as one JSON line on rank 0.  Also measured in the same run:
-  roofline      the split-K decode kernel: its per-layer launches back to back
+  roofline      the fused decode kernel: its per-layer launches back to back
                 in a captured graph (launch_ms) and with events around each
-                launch (launch_ms_isolated), against the measured HBM peak
-  e2e           same step through the C ABI from pinned host buffers (H2D of
-                the queries and new K/V, D2H of the outputs inside the timing)
+                launch inside a captured step (launch_ms_isolated), against
+                the measured HBM peak
+  e2e           the same step through the C ABI from pinned host buffers (H2D
+                of the queries and new K/V, D2H of the outputs inside the timing)
   multi_layer   all layers in one launch per kernel
   buffered      the step with 4 fp16 sink rows and a 128-row fp16 window
   paged         the step on a paged copy of the cache (shuffled pages)
   logit_mae     per-layer logit MAE, Block-GTQ against uniform TQ-MSE
-  fp16_baseline dense fp16 FlashAttention-2 decode over the unquantised K/V
-  cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU)
+  fp16_baseline dense fp16 decode over the unquantised K/V: FlashAttention-2's
+                decode with its split count swept, and torch SDPA; the best
+                one with its HBM fraction
+  cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU),
+                extrapolated to a step and labelled so
+  workloads     (one GPU) the other benchmark shapes -- tiny, llama, batch,
+                long -- each with its step, roofline, fp16 baseline, CPU
+                baseline and compression; long adds the 131072-row prefill
+                chunk's encode rate
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen3b]
   python bench.py --impl reference ...   (the CPU oracle as the reference arm)
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -37,12 +47,23 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 FALLBACK_HBM_GBS = 6650.0
+SIDE_WORKLOADS = ("tiny", "llama", "batch", "long")
 
-# DRAM bytes (read + write) per split-kernel launch from the ncu capture
-# summarised in profiles/decode_split_mma_qwen3b.md, for the workload it was
-# taken on (an 8-layer copy of it: the same per-layer launch).  Reported as
-# the roofline's "traffic"; None for other workloads.
-NCU_TRAFFIC_PER_LAUNCH = {"qwen3b": 27.8839e6}
+# DRAM bytes (read + write) per launch of the decode kernel from an ncu
+# capture, per workload, with the date of the capture and a digest of the
+# kernel sources it was taken on.  The roofline reports it only while the
+# sources still match that digest (null otherwise: the kernel has changed).
+NCU_TRAFFIC = {}
+KERNEL_SOURCES = ("packed_decode_attention_b200/csrc/decode.cu", "packed_decode_attention_b200/csrc/common.cuh",
+                  "packed_decode_attention_b200/csrc/device_tables.h")
+
+
+def kernel_digest():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def parse_args():
@@ -57,6 +78,9 @@ def parse_args():
     ap.add_argument("--no-fp16-baseline", action="store_true")
     ap.add_argument("--no-diag", action="store_true", help="skip the per-layer logit-MAE diagnostic")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache step")
+    ap.add_argument("--no-side", action="store_true", help="skip the other workloads (the workloads object)")
+    ap.add_argument("--decode-path", type=int, default=-1, choices=[-1, 0, 1],
+                    help="1: fused decode launch, 0: rotation + split + combine, -1: the library's default")
     return ap.parse_args()
 
 
@@ -100,6 +124,14 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def cpu_cores():
+    """Host cores this process may run on (its CPU affinity)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except Exception:
+        return max(1, os.cpu_count() or 1)
 
 
 class ClockSampler:
@@ -199,25 +231,18 @@ def token_bytes(kv, cfg):
     return out
 
 
-def cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        n = 1
-    return max(n, 1)
-
-
 class OracleSample:
     """A bounded sample of the workload for the CPU oracle: a few (layer, KV
-    head) pairs of sequence 0 at its full length, each with its own oracle
-    allocation, tables and packed cache (built once, untimed).  One timed unit
-    is the oracle's decode of the G query heads of a pair over its cache plus
-    the encode of one new K/V row; a full step is every (layer, KV head) of
-    every sequence, so the step time is the unit time scaled by
-    layers * KV heads * (total cached tokens / sample length)."""
+    head) pairs of sequence 0 over its first `t_len` cached tokens (at most
+    max_tokens), each with its own oracle allocation, tables and packed cache
+    (built once, untimed).  One timed unit is the oracle's decode of the G
+    query heads of a pair over that cache plus the encode of one new K/V row.
+    A full step is every (layer, KV head) of every sequence over all its
+    tokens, so the step time is extrapolated from the unit time by the factor
+    layers * KV heads * (total cached tokens / t_len); the decode's cost is
+    linear in the tokens."""
 
-    def __init__(self, w, lens, max_pairs=4):
+    def __init__(self, w, lens, max_pairs=4, max_tokens=None):
         import numpy as np
 
         from oracle import model
@@ -227,7 +252,7 @@ class OracleSample:
         pairs = [(l, h) for l in range(w.n_layers) for h in range(w.n_kv_heads)]
         self.n_pairs = len(pairs)
         pick = [pairs[i] for i in np.linspace(0, len(pairs) - 1, num=min(max_pairs, len(pairs))).astype(int)]
-        self.t_len = lens[0]
+        self.t_len = lens[0] if max_tokens is None else min(lens[0], max_tokens)
         cfg = model.Config(w.n_layers, w.n_kv_heads, w.n_q_heads, 128, w.k_bits, w.v_bits, 1, 4, 0, w.seed)
         self.units = []
         for (l, h) in pick:
@@ -243,6 +268,12 @@ class OracleSample:
             q = wl.queries(w, l, 0, [self.t_len], tag=2)[0, h * w.group:(h + 1) * w.group].numpy()
             self.units.append((tb, l, h, k[-1:], v[-1:], q, enc))
 
+    @property
+    def scale(self):
+        """Full step time / one unit's time."""
+        w = self.w
+        return w.n_layers * w.n_kv_heads * (sum(self.lens) / float(self.t_len))
+
     def time_unit(self, i):
         from oracle import model
         tb, l, h, k1, v1, q, enc = self.units[i % len(self.units)]
@@ -251,15 +282,33 @@ class OracleSample:
         model.decode(tb, l, h, q, enc["k_tiles"], enc["k_norms"], enc["v_tiles"], enc["v_norm"], enc["n"])
         return time.perf_counter() - t0
 
-    def step_seconds(self, unit_s):
-        return unit_s * self.w.n_layers * self.w.n_kv_heads * (sum(self.lens) / float(self.t_len))
-
-    def describe(self, n_timed):
+    def describe(self):
         w = self.w
-        return (f"oracle decode of the {w.group} query heads of one (layer, KV head) over {self.t_len} tokens "
-                f"+ encode of one K/V row; {n_timed} units over {len(self.units)} of {self.n_pairs} pairs "
-                f"(sequence 0 of {w.batch}); step time = unit time x {w.n_layers * w.n_kv_heads} pairs "
-                f"x total/sample tokens")
+        return (f"oracle decode of the {w.group} query heads of one (layer, KV head) over {self.t_len} cached "
+                f"tokens of sequence 0 + encode of one K/V row, on {len(self.units)} of {self.n_pairs} "
+                f"(layer, KV head) pairs; a full step (every pair of all {w.batch} sequences, "
+                f"{sum(self.lens)} cached tokens each) is extrapolated as the mean unit time x {self.scale:.6g}")
+
+
+def oracle_baseline(w, lens, n_units, max_pairs=3, max_tokens=None):
+    """The oracle on the host cores (BLAS threads = the process's cores):
+    n_units timed units, extrapolated to one step.  Returns (cpu_baseline
+    dict, unit seconds list)."""
+    import contextlib
+    cores = cpu_cores()
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=cores)
+    except Exception:
+        limiter = contextlib.nullcontext()
+    with limiter:
+        sample = OracleSample(w, lens, max_pairs=max_pairs, max_tokens=max_tokens)
+        units = [sample.time_unit(i) for i in range(n_units)]
+    unit_s = statistics.mean(units)
+    step_s = unit_s * sample.scale
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": sample.describe(), "extrapolated": True, "units_timed": len(units),
+            "unit_ms": unit_s * 1e3, "scale_to_step": sample.scale, "step_ms_extrapolated": step_s * 1e3}, units
 
 
 def run_reference(args):
@@ -269,22 +318,31 @@ def run_reference(args):
     from packed_decode_attention_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
     lens = wl.seq_lens(w)
-    sample = OracleSample(w, lens, max_pairs=2)
-    times = []
-    for i in range(args.warmup + args.steps):
-        dt = sample.time_unit(i)
-        if i >= args.warmup:
-            times.append(sample.step_seconds(dt))
-    step_s = statistics.mean(times)
-    value = w.batch / step_s
+    # warm-up units run untimed; each timed step is one unit of the sample
     cores = cpu_cores()
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=cores)
+    except Exception:
+        pass
+    sample = OracleSample(w, lens, max_pairs=2)
+    for i in range(args.warmup):
+        sample.time_unit(i)
+    units = [sample.time_unit(args.warmup + i) for i in range(args.steps)]
+    unit_s = statistics.mean(units)
+    step_s = unit_s * sample.scale
+    value = w.batch / step_s
     line = {
         "impl": "reference", "metric": "decode_tokens_per_s", "value": value, "unit": "tokens/s",
-        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": unit_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, lens),
+        "step_definition": "each step is one unit of the bounded sample (see cpu_baseline.sample); value is "
+                           "tokens/s of a full decode step extrapolated from the mean unit time",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample.describe(args.steps)},
+                         "sample": sample.describe(), "extrapolated": True, "units_timed": len(units),
+                         "unit_ms": unit_s * 1e3, "scale_to_step": sample.scale,
+                         "step_ms_extrapolated": step_s * 1e3},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -300,35 +358,126 @@ def workload_config(w, lens):
             "parallelism": "replicas"}
 
 
-def main():
-    args = parse_args()
-    if args.impl == "reference":
-        return run_reference(args)
+def time_graph(fn, steps, warmup, world=1):
+    """Average ms of one call of fn, captured as a CUDA graph and replayed
+    `steps` times after `warmup` replays, CUDA events around the timed region.
+    Returns (ms, graph, (wall t0, wall t1))."""
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    z.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    return a.elapsed_time(z) / steps, g, (t_wall0, t_wall1)
 
+
+def fp16_baseline(w, lens, q_all, kf, vf, seq, steps, warmup, world, dev, peak, ms_packed):
+    """Dense fp16 decode over the unquantised K/V: FlashAttention-2's decode
+    (flash_attn_with_kvcache) with its split count swept, and torch SDPA
+    (flash and cuDNN backends, per sequence); the best one is the baseline."""
+    import torch
+    import torch.nn.functional as F
+    L, B, HQ = w.n_layers, w.batch, w.n_q_heads
+    H = w.n_kv_heads
+    qf = q_all.view(L, B, 1, HQ, 128)
+    step_bytes = int(sum(lens) * H * L * 512 + L * B * HQ * 512)
+    cands = []
+    try:
+        from flash_attn import flash_attn_with_kvcache
+        for ns in (0, 2, 4, 8, 16, 32, 64, 128):
+            def fa2(ns=ns):
+                for l in range(L):
+                    flash_attn_with_kvcache(qf[l], kf[l], vf[l], cache_seqlens=seq, num_splits=ns)
+            cands.append((f"flash_attn_with_kvcache (FlashAttention-2 decode), num_splits={ns}", fa2))
+    except Exception:
+        pass
+    results = []
+    for name, fn in cands:
+        try:
+            ms, g, _ = time_graph(fn, max(3, steps // 2), max(2, warmup // 2), world)
+            del g
+            ms = max_over_ranks(ms, world, dev)
+            results.append({"impl": name, "ms_per_step": ms})
+        except Exception as e:  # report, do not fail the bench
+            results.append({"impl": name, "error": str(e)[:160]})
+            torch.cuda.synchronize()
+    # torch SDPA per sequence, timed eagerly (launched one call at a time)
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for backend, bname in ((SDPBackend.FLASH_ATTENTION, "flash"), (SDPBackend.CUDNN_ATTENTION, "cudnn")):
+        def sdpa(backend=backend):
+            with sdpa_kernel(backend):
+                for l in range(L):
+                    for b in range(B):
+                        qq = q_all[l, b][None, :, None, :]
+                        kk = kf[l][b, :lens[b]].transpose(0, 1)[None]
+                        vv = vf[l][b, :lens[b]].transpose(0, 1)[None]
+                        F.scaled_dot_product_attention(qq, kk, vv, enable_gqa=True)
+        name = f"torch scaled_dot_product_attention ({bname} backend, eager)"
+        try:
+            for _ in range(2):
+                sdpa()
+            torch.cuda.synchronize()
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(3, steps // 2)
+            a.record()
+            for _ in range(n):
+                sdpa()
+            z.record()
+            torch.cuda.synchronize()
+            results.append({"impl": name, "ms_per_step": max_over_ranks(a.elapsed_time(z) / n, world, dev)})
+        except Exception as e:
+            results.append({"impl": name, "error": str(e)[:160]})
+            torch.cuda.synchronize()
+    ok = [r for r in results if "ms_per_step" in r]
+    if not ok:
+        return {"error": "no fp16 decode ran", "candidates": results}
+    best = min(ok, key=lambda r: r["ms_per_step"])
+    gbs = step_bytes / (best["ms_per_step"] * 1e-3) / 1e9
+    fa2 = [r for r in ok if r["impl"].startswith("flash_attn_with_kvcache")]
+    fa2_default = next((r for r in fa2 if r["impl"].endswith("num_splits=0")), None)
+    return {"impl": best["impl"], "ms_per_step": best["ms_per_step"],
+            "tokens_per_s": world * B / (best["ms_per_step"] * 1e-3), "bytes_per_step": step_bytes,
+            "hbm_gbs": gbs, "hbm_frac": gbs / peak, "speedup_of_packed": best["ms_per_step"] / ms_packed,
+            "fa2_default_ms": fa2_default["ms_per_step"] if fa2_default else None,
+            "candidates": [{k: (round(v, 5) if isinstance(v, float) else v) for k, v in r.items()} for r in results]}
+
+
+def measure(w, args, dev, world, rank, full):
+    """Every figure of one workload.  full: the headline workload (all extras);
+    otherwise the step, roofline, fp16 and CPU baselines, compression and
+    (long context) the prefill chunk's encode rate."""
     import numpy as np
     import torch
 
     from packed_decode_attention_b200 import bgtq
     from packed_decode_attention_b200 import workloads as wl
 
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-
-    w = wl.WORKLOADS[args.workload]
-    if args.layers:
-        w = wl.scaled(w, n_layers=args.layers)
     lens = wl.seq_lens(w)
     L, H, HQ, B = w.n_layers, w.n_kv_heads, w.n_q_heads, w.batch
     cap = w.seq_len
     cfg = bgtq.Config(**wl.bench_config_fields(w))
     kv = bgtq.PackedKVCache(cfg, dev)
-    stream = torch.cuda.current_stream()
+    if args.decode_path >= 0:
+        kv.set_decode_path(args.decode_path)
+    fused = kv.decode_path_fused()
+    steps = args.steps if full else max(5, args.steps // 2)
+    warmup = args.warmup if full else max(3, args.warmup // 2)
+    peak, peak_kind = peaks()
 
     # ---- calibration + allocation (one-time) ----
     cq, ck = wl.calibration(w, device=dev)
@@ -368,6 +517,7 @@ def main():
                 torch.cuda.synchronize()
                 enc_ms += e0.elapsed_time(e1)
                 enc_rows += n * H
+                del kk, vv
     assert kv.device_error() == 0, "device error after prefill"
 
     # ---- step inputs ----
@@ -384,251 +534,230 @@ def main():
     out = torch.empty((L, B, HQ, 128), dtype=torch.float16, device=dev)
 
     def step():
-        # per layer: append the new K/V row, then attend (appends and query
-        # rotation share one launch, then the split pass and the combine)
+        # per layer: append the new K/V row, then attend
         for l in range(L):
             kv.decode_step(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq, out[l:l + 1])
 
-    def step_multi():
-        kv.encode_append(0, knew, vnew, start1, count1, layer_count=L)
-        kv.decode_attn(0, q_all, seq, out, layer_count=L)
-
-    def time_graph(fn, steps, warmup, sampler=None):
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        for _ in range(warmup):
-            g.replay()
-        torch.cuda.synchronize()
-        barrier(world)
-        torch.cuda.synchronize()
-        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t_wall0 = time.time()
-        a.record()
-        for _ in range(steps):
-            g.replay()
-        z.record()
-        torch.cuda.synchronize()
-        t_wall1 = time.time()
-        barrier(world)
-        return a.elapsed_time(z) / steps, g, (t_wall0, t_wall1)
-
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(uuid, local)
+    sampler = ClockSampler(uuid, dev.index or 0)
     sampler.start()
-    time.sleep(0.5)
-    ms_step, graph, (tw0, tw1) = time_graph(step, args.steps, args.warmup)
+    time.sleep(0.3)
+    ms_step, graph, (tw0, tw1) = time_graph(step, steps, warmup, world)
     sampler.stop()
     clocks = sampler.summary(tw0, tw1)
     ms_step = max_over_ranks(ms_step, world, dev)
     assert kv.device_error() == 0, "device error during the timed steps"
-    out_check = out.float()
-    assert torch.isfinite(out_check).all(), "non-finite decode output"
+    assert torch.isfinite(out.float()).all(), "non-finite decode output"
 
-    ms_multi, g_multi, _ = time_graph(step_multi, args.steps, args.warmup)
-    ms_multi = max_over_ranks(ms_multi, world, dev)
-    del g_multi
-
-    # ---- the same step with an fp16 sink + recent window (the README's
-    # "withbuffer" setting): packed positions [sink, len - window) plus the
-    # buffered rows ----
-    SINK, WINDOW = 4, 128
-    lo_b = [min(SINK, n) for n in lens]
-    hi_b = [max(lo_b[b], lens[b] - WINDOW) for b in range(B)]
-    n_buf = SINK + WINDOW
-    buf_k = torch.zeros((L, B, n_buf, H, 128), dtype=torch.float16, device=dev)
-    buf_v = torch.zeros_like(buf_k)
-    for l in range(L):
-        for b in range(B):
-            rows = list(range(lo_b[b])) + list(range(hi_b[b], lens[b]))
-            for j, r in enumerate(rows):
-                buf_k[l, b, j] = wl.keys(w, l, b, r, 1, device=dev)[0]
-                buf_v[l, b, j] = wl.values(w, l, b, r, 1, device=dev)[0]
-    buf_cnt = torch.tensor([lo_b[b] + lens[b] - hi_b[b] for b in range(B)], dtype=torch.int32, device=dev)
-    seq_hi = torch.tensor(hi_b, dtype=torch.int32, device=dev)
-    seq_lo = torch.tensor(lo_b, dtype=torch.int32, device=dev)
-
-    def step_buffered():
-        for l in range(L):
-            kv.decode_step_buffered(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq_hi, seq_lo,
-                                    buf_k[l:l + 1], buf_v[l:l + 1], buf_cnt, out[l:l + 1])
-
-    ms_buf, g_buf, _ = time_graph(step_buffered, args.steps, args.warmup)
-    ms_buf = max_over_ranks(ms_buf, world, dev)
-    del g_buf, buf_k, buf_v
-    assert kv.device_error() == 0, "device error in the buffered step"
-
-    # ---- the same step over a paged copy of the cache: a tight pool of
-    # 64-position pages, shuffled over the sequences' tiles ----
-    paged = None
-    if not args.no_paged:
-        T = (cap + 63) // 64
-        need = [(n + 63) // 64 for n in lens]
-        pool = sum(need)
-        ids = torch.randperm(pool, generator=torch.Generator().manual_seed(7)).to(torch.int32)
-        table = torch.full((B, T), -1, dtype=torch.int32)
-        k0 = 0
-        for b in range(B):
-            table[b, :need[b]] = ids[k0:k0 + need[b]]
-            k0 += need[b]
-        bt = table.to(dev)
-        kvp = bgtq.PackedKVCache(bgtq.Config(**dict(wl.bench_config_fields(w), page_pool_tiles=pool)), dev)
-        kvp.set_block_table(bt)
-        kvp.set_allocation(kv.get_allocation())
-        for l in range(L):
-            for b in range(B):
-                pg = bt[b, :need[b]].long()
-                for h in range(H):
-                    kvp.k_tiles()[l, h][pg] = kv.k_tiles()[l, b, h, :need[b]]
-                    kvp.v_tiles()[l, h][pg] = kv.v_tiles()[l, b, h, :need[b]]
-                    kvp.k_norms()[l, h].view(pool, 64, 4)[pg] = kv.k_norms()[l, b, h, :need[b] * 64].view(-1, 64, 4)
-                    kvp.v_norms()[l, h].view(pool, 64)[pg] = kv.v_norms()[l, b, h, :need[b] * 64].view(-1, 64)
-        out_p = torch.empty_like(out)
-
-        def step_paged():
-            for l in range(L):
-                kvp.decode_step(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq,
-                                out_p[l:l + 1])
-
-        ms_paged, g_p, _ = time_graph(step_paged, args.steps, args.warmup)
-        ms_paged = max_over_ranks(ms_paged, world, dev)
-        del g_p
-        step()
-        step_paged()
-        torch.cuda.synchronize()
-        assert kvp.device_error() == 0, "device error in the paged step"
-        paged = {"ms_per_step": ms_paged, "tokens_per_s": world * B / (ms_paged * 1e-3), "pages": pool,
-                 "cache_bytes": kvp.cache_bytes, "contiguous_cache_bytes": kv.cache_bytes,
-                 "output_equal_to_contiguous": bool(torch.equal(out, out_p)),
-                 "note": "block-table indirection, pages shuffled over the sequences"}
-        kvp.close()
-        del kvp, out_p
-
-    # ---- the split-K kernel in isolation: events around each per-layer
-    # launch, in a captured step (the event nodes keep the split kernel from
-    # overlapping its neighbours, so each interval is that kernel's whole
-    # duration, start-up included) ----
+    # ---- roofline: the decode kernel's average launch duration, its
+    # per-layer launches (same inputs, same launch configuration as in the
+    # step) back to back in one captured graph ----
     tb = token_bytes(kv, cfg)
-    qrot = torch.empty((1, B, HQ, 128), dtype=torch.float32, device=dev)
+    bytes_per_layer = [sum(lens[b] * tb[l, h] for b in range(B) for h in range(H)) + B * HQ * 512 for l in range(L)]
+    alg_bytes = statistics.mean(bytes_per_layer)
+
+    def decodes_back_to_back():
+        for l in range(L):
+            kv.decode_attn(l, q_all[l:l + 1], seq, out[l:l + 1])
+
+    ms_dec, g_d, _ = time_graph(decodes_back_to_back, steps, warmup, world)
+    del g_d
+    launch_ms = max_over_ranks(ms_dec / L, world, dev)
+    achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
+
+    # the same launches with events around each one inside a captured step
+    # (the event nodes keep it from overlapping its neighbours: start-up included)
     ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
           for _ in range(L)]
 
-    def step_timed_split():
+    def step_timed():
         for l in range(L):
             kv.encode_append(l, knew[l:l + 1], vnew[l:l + 1], start1, count1)
-            kv.rotate_query(l, q_all[l:l + 1], qrot)
             ev[l][0].record()
-            kv.decode_split(l, qrot, seq)
+            kv.decode_attn(l, q_all[l:l + 1], seq, out[l:l + 1])
             ev[l][1].record()
-            kv.decode_combine(l, seq, out[l:l + 1])
 
-    step_timed_split()
+    step_timed()
     torch.cuda.synchronize()
-    g_split = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_split):
-        step_timed_split()
-    split_ms = []
-    for it in range(args.warmup + args.steps):
-        g_split.replay()
+    g_t = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_t):
+        step_timed()
+    iso = []
+    for it in range(warmup + steps):
+        g_t.replay()
         torch.cuda.synchronize()
-        if it >= args.warmup:
-            split_ms.extend(a.elapsed_time(z) for a, z in ev)
-    del g_split
-    split_isolated_ms = statistics.mean(split_ms)
+        if it >= warmup:
+            iso.extend(a.elapsed_time(z) for a, z in ev)
+    del g_t
+    launch_ms_isolated = statistics.mean(iso)
 
-    # ---- the split kernel's average launch duration: the step's per-layer
-    # split launches (same inputs, same launch configuration) back to back in
-    # one captured graph, CUDA events around the whole timed region, divided
-    # by the launches; each launch's set-up overlaps the previous one's tail,
-    # as in the step ----
-    qrot_all = torch.empty((L, B, HQ, 128), dtype=torch.float32, device=dev)
-    for l in range(L):
-        kv.rotate_query(l, q_all[l:l + 1], qrot_all[l:l + 1])
+    digest = kernel_digest()
+    cap_rec = NCU_TRAFFIC.get(w.name)
+    traffic = cap_rec["bytes_per_launch"] if cap_rec and cap_rec.get("kernel_digest") == digest else None
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic,
+                "traffic_source": (f"ncu capture of {cap_rec['captured']} ({cap_rec['case']}), same kernel sources"
+                                   if traffic is not None else "no ncu capture of the current kernel sources"),
+                "kernel": "decode_fused_kernel" if fused else "decode_mma_kernel + combine_kernel",
+                "launch_ms": launch_ms, "launch_ms_isolated": launch_ms_isolated,
+                "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind, "kernel_digest": digest,
+                "timing": "launch_ms: the step's per-layer decode launches back to back in a captured graph, "
+                          "events around the region / launches; launch_ms_isolated: events around each launch "
+                          "inside a captured step (start-up not overlapped)"}
+    step_bytes = sum(bytes_per_layer)
+    res = {"ms_per_step": ms_step, "tokens_per_s": world * B / (ms_step * 1e-3),
+           "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9, "roofline": roofline, "clocks": clocks,
+           "decode_path": "fused (one launch per decode call)" if fused else "query rotation + split + combine",
+           "decode_wave_ctas": kv.decode_wave_ctas(),
+           "gpu_launches": (2 if fused else 3) * L * steps,
+           "allocate_ms": alloc_ms, "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),
+           "prefill_encode_call_rows": chunk,
+           "compression_vs_fp16": 512.0 / (sum(lens[b] * tb[l, h] for l in range(L) for b in range(B)
+                                                for h in range(H)) / (sum(lens) * L * H))}
 
-    def splits_back_to_back():
+    if full:
+        # ---- end to end from pinned host memory ----
+        q_h = q_all.cpu().pin_memory()
+        k_h = knew.cpu().pin_memory()
+        v_h = vnew.cpu().pin_memory()
+        o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
+        d2h = o_h.numel() * 2
+        for _ in range(warmup):
+            q_all.copy_(q_h, non_blocking=True)
+            knew.copy_(k_h, non_blocking=True)
+            vnew.copy_(v_h, non_blocking=True)
+            graph.replay()
+            o_h.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            q_all.copy_(q_h, non_blocking=True)
+            knew.copy_(k_h, non_blocking=True)
+            vnew.copy_(v_h, non_blocking=True)
+            graph.replay()
+            o_h.copy_(out, non_blocking=True)
+        z.record()
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(a.elapsed_time(z) / steps, world, dev)
+        res["e2e"] = {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+
+        # ---- all layers in one launch per kernel ----
+        def step_multi():
+            kv.encode_append(0, knew, vnew, start1, count1, layer_count=L)
+            kv.decode_attn(0, q_all, seq, out, layer_count=L)
+
+        ms_multi, g_m, _ = time_graph(step_multi, steps, warmup, world)
+        del g_m
+        ms_multi = max_over_ranks(ms_multi, world, dev)
+        res["multi_layer"] = {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
+                              "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9}
+
+        # ---- fp16 sink + recent window (the README's "withbuffer" setting) ----
+        SINK, WINDOW = 4, 128
+        lo_b = [min(SINK, n) for n in lens]
+        hi_b = [max(lo_b[b], lens[b] - WINDOW) for b in range(B)]
+        n_buf = SINK + WINDOW
+        buf_k = torch.zeros((L, B, n_buf, H, 128), dtype=torch.float16, device=dev)
+        buf_v = torch.zeros_like(buf_k)
         for l in range(L):
-            kv.decode_split(l, qrot_all[l:l + 1], seq)
+            for b in range(B):
+                rows = list(range(lo_b[b])) + list(range(hi_b[b], lens[b]))
+                for j, r in enumerate(rows):
+                    buf_k[l, b, j] = wl.keys(w, l, b, r, 1, device=dev)[0]
+                    buf_v[l, b, j] = wl.values(w, l, b, r, 1, device=dev)[0]
+        buf_cnt = torch.tensor([lo_b[b] + lens[b] - hi_b[b] for b in range(B)], dtype=torch.int32, device=dev)
+        seq_hi = torch.tensor(hi_b, dtype=torch.int32, device=dev)
+        seq_lo = torch.tensor(lo_b, dtype=torch.int32, device=dev)
 
-    ms_splits, g_sp, _ = time_graph(splits_back_to_back, args.steps, args.warmup)
-    del g_sp
-    split_avg_ms = max_over_ranks(ms_splits / L, world, dev)
-    bytes_per_layer = [sum(lens[b] * tb[l, h] for b in range(B) for h in range(H)) for l in range(L)]
-    alg_bytes = statistics.mean(bytes_per_layer)
-    achieved = alg_bytes / (split_avg_ms * 1e-3) / 1e9
-    peak, peak_kind = peaks()
+        def step_buffered():
+            for l in range(L):
+                kv.decode_step_buffered(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq_hi,
+                                        seq_lo, buf_k[l:l + 1], buf_v[l:l + 1], buf_cnt, out[l:l + 1])
 
-    # ---- end to end from pinned host memory ----
-    q_h = q_all.cpu().pin_memory()
-    k_h = knew.cpu().pin_memory()
-    v_h = vnew.cpu().pin_memory()
-    o_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
-    d2h = o_h.numel() * 2
-    for _ in range(args.warmup):
-        q_all.copy_(q_h, non_blocking=True)
-        knew.copy_(k_h, non_blocking=True)
-        vnew.copy_(v_h, non_blocking=True)
-        graph.replay()
-        o_h.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(args.steps):
-        q_all.copy_(q_h, non_blocking=True)
-        knew.copy_(k_h, non_blocking=True)
-        vnew.copy_(v_h, non_blocking=True)
-        graph.replay()
-        o_h.copy_(out, non_blocking=True)
-    z.record()
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(a.elapsed_time(z) / args.steps, world, dev)
-    del graph
+        ms_buf, g_buf, _ = time_graph(step_buffered, steps, warmup, world)
+        ms_buf = max_over_ranks(ms_buf, world, dev)
+        del g_buf, buf_k, buf_v
+        assert kv.device_error() == 0, "device error in the buffered step"
+        res["buffered"] = {"ms_per_step": ms_buf, "tokens_per_s": world * B / (ms_buf * 1e-3), "sink": SINK,
+                           "window": WINDOW, "note": "fp16 sink + recent window next to the packed cache "
+                                                     "(query rotation, split pass with buffer CTAs, combine)"}
 
-    # ---- dense fp16 baseline (FlashAttention-2 decode) ----
-    fp16 = None
-    if want_fp16:
-        import torch.nn.functional as F
-        qf = q_all.view(L, B, 1, HQ, 128)
+        # ---- the split pass alone (the three-launch path's dominant kernel) ----
+        qrot_all = torch.empty((L, B, HQ, 128), dtype=torch.float32, device=dev)
+        for l in range(L):
+            kv.rotate_query(l, q_all[l:l + 1], qrot_all[l:l + 1])
 
-        def fp16_step_sdpa():
+        def splits_back_to_back():
+            for l in range(L):
+                kv.decode_split(l, qrot_all[l:l + 1], seq)
+
+        ms_sp, g_sp, _ = time_graph(splits_back_to_back, steps, warmup, world)
+        del g_sp
+        sp_ms = max_over_ranks(ms_sp / L, world, dev)
+        sp_bytes = alg_bytes - B * HQ * 512
+        res["split_pass"] = {"launch_ms": sp_ms, "achieved_gbs": sp_bytes / (sp_ms * 1e-3) / 1e9,
+                             "frac": sp_bytes / (sp_ms * 1e-3) / 1e9 / peak,
+                             "note": "decode_mma_kernel (buffered and stage calls), per-layer launches back to back"}
+        del qrot_all
+
+        # ---- the same step over a paged copy of the cache ----
+        if not args.no_paged:
+            T = (cap + 63) // 64
+            need = [(n + 63) // 64 for n in lens]
+            pool = sum(need)
+            ids = torch.randperm(pool, generator=torch.Generator().manual_seed(7)).to(torch.int32)
+            table = torch.full((B, T), -1, dtype=torch.int32)
+            k0 = 0
+            for b in range(B):
+                table[b, :need[b]] = ids[k0:k0 + need[b]]
+                k0 += need[b]
+            bt = table.to(dev)
+            kvp = bgtq.PackedKVCache(bgtq.Config(**dict(wl.bench_config_fields(w), page_pool_tiles=pool)), dev)
+            kvp.set_block_table(bt)
+            kvp.set_allocation(kv.get_allocation())
             for l in range(L):
                 for b in range(B):
-                    qq = q_all[l, b][None, :, None, :]
-                    kk = kf[l][b, :lens[b]].transpose(0, 1)[None]
-                    vv = vf[l][b, :lens[b]].transpose(0, 1)[None]
-                    F.scaled_dot_product_attention(qq, kk, vv, enable_gqa=True)
+                    pg = bt[b, :need[b]].long()
+                    for h in range(H):
+                        kvp.k_tiles()[l, h][pg] = kv.k_tiles()[l, b, h, :need[b]]
+                        kvp.v_tiles()[l, h][pg] = kv.v_tiles()[l, b, h, :need[b]]
+                        kvp.k_norms()[l, h].view(pool, 64, 4)[pg] = kv.k_norms()[l, b, h, :need[b] * 64].view(-1, 64, 4)
+                        kvp.v_norms()[l, h].view(pool, 64)[pg] = kv.v_norms()[l, b, h, :need[b] * 64].view(-1, 64)
+            out_p = torch.empty_like(out)
 
-        try:
-            from flash_attn import flash_attn_with_kvcache
-
-            def fp16_step():
+            def step_paged():
                 for l in range(L):
-                    flash_attn_with_kvcache(qf[l], kf[l], vf[l], cache_seqlens=seq)
+                    kvp.decode_step(l, knew[l:l + 1], vnew[l:l + 1], start1, count1, q_all[l:l + 1], seq,
+                                    out_p[l:l + 1])
 
-            fp16_step()
+            ms_paged, g_p, _ = time_graph(step_paged, steps, warmup, world)
+            ms_paged = max_over_ranks(ms_paged, world, dev)
+            del g_p
+            step()
+            step_paged()
             torch.cuda.synchronize()
-            name = "flash_attn_with_kvcache (FlashAttention-2 decode)"
-        except Exception:
-            fp16_step = fp16_step_sdpa
-            name = "torch scaled_dot_product_attention"
-        try:
-            ms_fp16, g16, _ = time_graph(fp16_step, args.steps, args.warmup)
-            ms_fp16 = max_over_ranks(ms_fp16, world, dev)
-            del g16
-            fp16 = {"impl": name, "ms_per_step": ms_fp16, "tokens_per_s": world * B / (ms_fp16 * 1e-3),
-                    "bytes_per_step": int(sum(lens) * H * L * 512), "speedup_of_packed": ms_fp16 / ms_step}
-        except Exception as e:  # report, do not fail the bench
-            fp16 = {"impl": name, "error": str(e)[:200]}
-        del kf, vf
+            assert kvp.device_error() == 0, "device error in the paged step"
+            res["paged"] = {"ms_per_step": ms_paged, "tokens_per_s": world * B / (ms_paged * 1e-3), "pages": pool,
+                            "cache_bytes": kvp.cache_bytes, "contiguous_cache_bytes": kv.cache_bytes,
+                            "output_equal_to_contiguous": bool(torch.equal(out, out_p)),
+                            "note": "block-table indirection, pages shuffled over the sequences"}
+            kvp.close()
+            del kvp, out_p
+    del graph
 
-    # ---- per-layer logit MAE (K only): Block-GTQ against uniform TQ-MSE at
-    # the same average width, over a 1024-position window of sequence 0 ----
-    diag = None
-    if not args.no_diag:
+    # ---- dense fp16 baseline ----
+    if want_fp16:
+        res["fp16_baseline"] = fp16_baseline(w, lens, q_all, kf, vf, seq, steps, warmup, world, dev, peak, ms_step)
+        del kf, vf
+        torch.cuda.empty_cache()
+
+    if full and not args.no_diag:
+        # ---- per-layer logit MAE (K only): Block-GTQ against uniform TQ-MSE at
+        # the same average width, over a 1024-position window of sequence 0 ----
         M = min(1024, lens[0])
         qd = torch.stack([wl.queries(w, l, 0, torch.arange(M), tag=3, device=dev) for l in range(L)])
         kd = torch.stack([wl.keys(w, l, 0, 0, M, device=dev) for l in range(L)])
@@ -653,12 +782,12 @@ def main():
         kvu.close()
         g_l = mae_g.mean(dim=1).cpu().numpy()
         u_l = mae_u.mean(dim=1).cpu().numpy()
-        diag = {"window": M, "pairs_per_head": M * (M + 1) // 2, "block_gtq_mean": float(g_l.mean()),
-                "tq_mse_mean": float(u_l.mean()), "reduction": float(1 - g_l.mean() / u_l.mean()),
-                "wins": f"{int((g_l < u_l).sum())}/{L}", "ms_all_layers": diag_ms,
-                "per_layer_block_gtq": [round(float(x), 5) for x in g_l],
-                "per_layer_tq_mse": [round(float(x), 5) for x in u_l],
-                "note": "K-only logit MAE (q.k / sqrt(128)) over causal pairs, synthetic Q/K"}
+        res["logit_mae"] = {"window": M, "pairs_per_head": M * (M + 1) // 2, "block_gtq_mean": float(g_l.mean()),
+                            "tq_mse_mean": float(u_l.mean()), "reduction": float(1 - g_l.mean() / u_l.mean()),
+                            "wins": f"{int((g_l < u_l).sum())}/{L}", "ms_all_layers": diag_ms,
+                            "per_layer_block_gtq": [round(float(x), 5) for x in g_l],
+                            "per_layer_tq_mse": [round(float(x), 5) for x in u_l],
+                            "note": "K-only logit MAE (q.k / sqrt(128)) over causal pairs, synthetic Q/K"}
         del qd, kd
 
     # ---- the fused RoPE + encode (K before RoPE), timed after every decode
@@ -678,55 +807,75 @@ def main():
         if it:
             rope_ms.append(e0.elapsed_time(e1))
     assert kv.device_error() == 0, "device error in the fused RoPE + encode"
-    rope_rows_per_s = n_r * H / (statistics.mean(rope_ms) * 1e-3)
+    res["prefill_encode_rope_rows_per_s"] = n_r * H / (statistics.mean(rope_ms) * 1e-3)
     del kk
+    kv.close()
+    del kv, q_all, knew, vnew, out, seq
+    torch.cuda.empty_cache()
 
     # ---- CPU oracle on a bounded sample ----
-    cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = OracleSample(w, lens, max_pairs=3)
-        units = [sample.time_unit(i) for i in range(len(sample.units) * 2)]
-        st = sample.step_seconds(statistics.mean(units))
-        cpu = {"value": B / st, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": sample.describe(len(units))}
+        n_units = 6 if full else 2
+        max_tokens = None if full else 16384
+        res["cpu_baseline"], _ = oracle_baseline(w, lens, n_units, max_pairs=3 if full else 1,
+                                                 max_tokens=max_tokens)
+    return res
 
-    value = job_value(world, B, ms_step)
-    step_bytes = sum(bytes_per_layer) + L * B * HQ * 512
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    from packed_decode_attention_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    if args.layers:
+        w = wl.scaled(w, n_layers=args.layers)
+    lens = wl.seq_lens(w)
+    r = measure(w, args, dev, world, rank, full=True)
+
+    sides = None
+    if world == 1 and not args.no_side and not args.layers:
+        sides = {}
+        for name in SIDE_WORKLOADS:
+            if name == args.workload:
+                continue
+            sw = wl.WORKLOADS[name]
+            try:
+                s = measure(sw, args, dev, 1, rank, full=False)
+                s["config"] = workload_config(sw, wl.seq_lens(sw))
+                sides[name] = s
+            except Exception as e:  # keep the headline line even if a side workload fails
+                sides[name] = {"error": f"{type(e).__name__}: {str(e)[:200]}"}
+                torch.cuda.empty_cache()
+
     line = {
-        "metric": "decode_tokens_per_s", "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, lens),
-        "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": NCU_TRAFFIC_PER_LAUNCH.get(args.workload), "kernel": "decode_mma_kernel",
-                     "launch_ms": split_avg_ms, "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind,
-                     "launch_ms_isolated": split_isolated_ms,
-                     "timing": "launch_ms: the step's per-layer split launches back to back in a captured graph, "
-                               "events around the region / launches; launch_ms_isolated: events around each "
-                               "launch inside a captured step (start-up not overlapped)"},
-        "e2e": {"value": world * B / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * L * args.steps,
-        "clocks": clocks,
-        "buffered": {"ms_per_step": ms_buf, "tokens_per_s": world * B / (ms_buf * 1e-3), "sink": SINK,
-                     "window": WINDOW, "note": "fp16 sink + recent window next to the packed cache"},
-        "multi_layer": {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
-                        "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9},
-        "fp16_baseline": fp16,
-        "logit_mae": diag,
-        "paged": paged,
-        "cpu_baseline": cpu,
-        "allocate_ms": alloc_ms,
-        "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),
-        "prefill_encode_call_rows": chunk,
-        "prefill_encode_rope_rows_per_s": rope_rows_per_s,
-        "compression_vs_fp16": 512.0 / (sum(lens[b] * tb[l, h] for l in range(L) for b in range(B) for h in range(H))
-                                        / (sum(lens) * L * H)),
+        "metric": "decode_tokens_per_s", "value": r["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16*f16+f32 (mma.sync: fp16 operands, fp32 accumulate)",
+        "data": "synthetic", "config": workload_config(w, lens),
     }
+    for k in ("step_hbm_gbs", "roofline", "e2e", "gpu_launches", "clocks", "decode_path", "decode_wave_ctas", "buffered",
+              "multi_layer", "split_pass", "fp16_baseline", "logit_mae", "paged", "cpu_baseline", "allocate_ms",
+              "prefill_encode_rows_per_s", "prefill_encode_call_rows", "prefill_encode_rope_rows_per_s",
+              "compression_vs_fp16"):
+        if k in r:
+            line[k] = r[k]
+    line["workloads"] = sides
     if rank == 0:
         print(json.dumps(line), flush=True)
-    kv.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

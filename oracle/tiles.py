@@ -31,6 +31,15 @@ Quartet: four selectors s0..s3 of one lane at width b stored as b plane words
   b = 2: A = (s0&M3) | (s1&M3)<<2,  B = (s2&M3) | (s3&M3)<<2
   b = 3: A, B as for b = 2, and H = (s0&M4)>>2 | (s1&M4)>>1 | (s2&M4) | (s3&M4)<<1
   b = 4: s0, s1, s2, s3
+Stored symbol: widths 1..3 store the code c itself.  Width 4 stores it in
+sign-magnitude form,
+  sigma(c) = c - 8           for c >= 8   (the 8 positive levels, 0..7)
+  sigma(c) = 8 + (7 - c)     for c < 8    (their negatives, 8..15),
+so bit 3 of a symbol is the sign of its level and bits 0..2 index |level|
+among the positive levels: the Lloyd-Max codebook is symmetric
+(C[15 - c] = -C[c]), so symbol s stands for (-1)^[s >= 8] C[8 + s % 8].  The
+selectors below hold symbols; pack / unpack convert.
+
 A quartet region is b words x 32 lanes, word-major (word k of lane L at
 index 32 k + L).  K quartets: one per full chunk, s_mu for mu = 0..3.  V
 quartets: one per dim-tile m, s_kappa for kappa = 0..3.
@@ -173,6 +182,33 @@ def _unpack(tiles, bitmap, npos):
     return out
 
 
+def stored_symbol(codes, b):
+    """Codes -> the symbols a selector holds at width b (sigma at width 4)."""
+    c = np.asarray(codes, dtype=np.int64)
+    if b != 4:
+        return c
+    return np.where(c >= 8, c - 8, 15 - c)
+
+
+def code_of_symbol(symbols, b):
+    """Inverse of stored_symbol."""
+    s = np.asarray(symbols, dtype=np.int64)
+    if b != 4:
+        return s
+    return np.where(s >= 8, 15 - s, s + 8)
+
+
+def _k_symbols(codes, groups, inverse=False):
+    """Record-order K codes <-> symbols, group by group."""
+    out = np.array(codes, dtype=np.int64, copy=True)
+    start = 0
+    for b, d in groups:
+        cols = slice(start, start + len(d))
+        out[..., cols] = (code_of_symbol if inverse else stored_symbol)(out[..., cols], int(b))
+        start += len(d)
+    return out
+
+
 def group_spec(groups):
     """(width, size) tuple from oracle group layouts [(width, dims), ...]."""
     return tuple((int(b), len(d)) for b, d in groups)
@@ -180,21 +216,21 @@ def group_spec(groups):
 
 def pack_k_tiles(codes, groups, k_avg_bits):
     """Record-order K codes [n, P] -> uint8 [ceil(n/64), 1024*k_avg_bits]; rows past n are code 0."""
-    return _pack(_to_tiles(codes), k_tile_bitmap(group_spec(groups)), 1024 * k_avg_bits)
+    return _pack(_to_tiles(_k_symbols(codes, groups)), k_tile_bitmap(group_spec(groups)), 1024 * k_avg_bits)
 
 
 def unpack_k_tiles(tiles, groups, n=None):
-    codes = _unpack(tiles, k_tile_bitmap(group_spec(groups)), sum(len(d) for _, d in groups))
-    codes = codes.reshape(-1, codes.shape[-1])
+    sym = _unpack(tiles, k_tile_bitmap(group_spec(groups)), sum(len(d) for _, d in groups))
+    codes = _k_symbols(sym.reshape(-1, sym.shape[-1]), groups, inverse=True)
     return codes if n is None else codes[:n]
 
 
 def pack_v_tiles(codes, vb):
-    return _pack(_to_tiles(codes), v_tile_bitmap(vb), 1024 * vb)
+    return _pack(_to_tiles(stored_symbol(codes, vb)), v_tile_bitmap(vb), 1024 * vb)
 
 
 def unpack_v_tiles(tiles, vb, n=None):
-    codes = _unpack(tiles, v_tile_bitmap(vb), 128).reshape(-1, 128)
+    codes = code_of_symbol(_unpack(tiles, v_tile_bitmap(vb), 128).reshape(-1, 128), vb)
     return codes if n is None else codes[:n]
 
 

@@ -122,6 +122,8 @@ _SIGS = {
     "bgtq_decode_combine": (ctypes.c_int, [_VP, _I32, _I32, _VP, _I32, _VP, _VP]),
     "bgtq_decode_attn_static_scratch": (ctypes.c_int, [_VP, _I32, _I32, _VP, _VP, _I32, _VP, _VP]),
     "bgtq_set_split_tokens": (ctypes.c_int, [_VP, _I32]),
+    "bgtq_set_decode_path": (ctypes.c_int, [_VP, _I32]),
+    "bgtq_get_decode_path": (ctypes.c_int, [_VP, _VP, _VP]),
     "bgtq_get_device_error": (ctypes.c_int, [_VP, _VP, _VP]),
     "bgtq_error_string": (ctypes.c_char_p, [_I32]),
 }
@@ -333,6 +335,18 @@ def bgtq_decode_attn_static_scratch(state, layer, layer_count, d_q, d_seq_lens, 
 
 def bgtq_set_split_tokens(state, tokens):
     _check(lib().bgtq_set_split_tokens(state, tokens))
+
+
+def bgtq_set_decode_path(state, fused):
+    _check(lib().bgtq_set_decode_path(state, int(fused)))
+
+
+def bgtq_get_decode_path(state):
+    """(fused, ctas): fused 1 when the decode calls run as one fused launch (0: query
+    rotation, split pass and combine); ctas the CTAs one wave of that kernel holds."""
+    out, ctas = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().bgtq_get_decode_path(state, ctypes.byref(out), ctypes.byref(ctas)))
+    return out.value, ctas.value
 
 
 def bgtq_get_device_error(state, stream=None):
@@ -559,6 +573,18 @@ class PackedKVCache:
 
     def set_split_tokens(self, tokens):
         bgtq_set_split_tokens(self.state, tokens)
+
+    def set_decode_path(self, fused):
+        """1: decode_attn / decode_step run as one fused launch where the GPU can; 0: three launches."""
+        bgtq_set_decode_path(self.state, fused)
+
+    def decode_path_fused(self):
+        """True when decode_attn / decode_step run as one fused launch (bgtq_get_decode_path)."""
+        return bgtq_get_decode_path(self.state)[0] == 1
+
+    def decode_wave_ctas(self):
+        """CTAs one wave of the decode kernel holds (the automatic split plan's budget)."""
+        return bgtq_get_decode_path(self.state)[1]
 
     def device_error(self):
         return bgtq_get_device_error(self.state)

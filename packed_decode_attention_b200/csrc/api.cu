@@ -26,6 +26,8 @@ struct bgtq_state {
   size_t cache_bytes, ws_bytes;
   int split_tokens = 0;  // 0 = automatic
   int ctas_per_sm = 0;   // resident decode CTAs per SM (looked up on first use)
+  int fused_clusters = -1;  // co-resident clusters of the fused decode (looked up on first use; 0: not usable)
+  int decode_mode = 0;      // 1: the fused decode where the GPU can run it; 0: rotation + split + combine
   int num_sms = 148;
   int device = -1;       // the CUDA device current at bgtq_create: its buffers live there
   bool ready = false;
@@ -154,14 +156,18 @@ uint32_t half_bits(float x) {
   return v;
 }
 
-// PRMT byte tables of a width's fp16 codebook: words 0..3 hold the low
-// bytes of entries 4i..4i+3, words 4..7 the high bytes.
+// PRMT byte tables of a width's fp16 codebook, indexed by stored symbol:
+// words 0..3 hold the low bytes of entries 4i..4i+3, words 4..7 the high
+// bytes.  Widths 1..3: entry e = level e.  Width 4 (sign-magnitude
+// symbols): entry m = the positive level C[8 + m] for m = 0..7 (words 0, 1
+// and 4, 5); the sign is applied from the symbol's bit 3.
 void byte_table(int bits, uint32_t* out) {
   std::vector<float> cen, thr;
   bgtq::lloyd_max_codebook(bits, &cen, &thr);
   for (int i = 0; i < 8; ++i) out[i] = 0;
-  for (int e = 0; e < (1 << bits); ++e) {
-    const uint32_t h = half_bits(cen[e]);
+  const int entries = bits == 4 ? 8 : (1 << bits);
+  for (int e = 0; e < entries; ++e) {
+    const uint32_t h = half_bits(cen[bits == 4 ? 8 + e : e]);
     out[e >> 2] |= (h & 0xFFu) << (8 * (e & 3));
     out[4 + (e >> 2)] |= (h >> 8) << (8 * (e & 3));
   }
@@ -284,6 +290,47 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
 int split_slots(bgtq_state* st) {
   if (st->ctas_per_sm <= 0) st->ctas_per_sm = std::max(1, bgtq::decode_ctas_per_sm(st->shape));
   return st->ctas_per_sm * st->num_sms;
+}
+
+// CTAs of the fused decode the GPU holds at once (whole 8-CTA clusters); 0
+// when it cannot run, and the decode calls then use the split pass and the
+// combine.
+constexpr int kFusedCluster = 8;
+
+int fused_slots(bgtq_state* st) {
+  if (st->fused_clusters < 0) st->fused_clusters = std::max(0, bgtq::decode_fused_clusters(st->shape));
+  return st->fused_clusters * kFusedCluster;
+}
+
+// Whether the decode calls take the fused launch: requested and possible.
+bool use_fused(bgtq_state* st) { return st->decode_mode == 1 && fused_slots(st) > 0; }
+
+// The split plan of a fused decode call: as split_for, in whole clusters
+// (a set split size rounds each unit's count up to whole clusters; the
+// automatic plan spreads one wave of clusters over the units, at least one
+// each).
+bgtq::SplitPlan fused_plan(bgtq_state* st, int32_t layer_count, int32_t batch) {
+  const int cl = kFusedCluster;
+  auto up = [cl](int64_t x) { return (x + cl - 1) / cl * cl; };
+  const int head_blocks = (st->shape.group + 7) / 8;
+  bgtq::SplitPlan p{};
+  p.cluster = cl;
+  p.units_per_seq = layer_count * st->cfg.n_kv_heads * head_blocks;
+  const int64_t tiles = (st->cfg.capacity_tokens + bgtq::kTile - 1) / bgtq::kTile;
+  const int64_t max_sp = max_splits_of(&st->cfg);
+  if (st->split_tokens > 0) {
+    p.fixed_tiles = st->split_tokens / bgtq::kTile;
+    p.c_max = static_cast<int>(up(std::min<int64_t>(max_sp, (tiles + p.fixed_tiles - 1) / p.fixed_tiles)));
+    p.budget = 0;
+    return p;
+  }
+  const int64_t units = int64_t(p.units_per_seq) * batch;
+  const int64_t budget = std::max<int64_t>(fused_slots(st), cl * units);
+  const int64_t share2 = up(std::max<int64_t>(1, 2 * budget / units));
+  p.budget = static_cast<int>(std::min<int64_t>(budget, INT32_MAX));
+  p.fixed_tiles = 0;
+  p.c_max = static_cast<int>(std::max<int64_t>(cl, std::min({up(max_sp), share2, up(tiles)})));
+  return p;
 }
 
 }  // namespace
@@ -638,8 +685,14 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
+  if (use_fused(st))
+    return bgtq::launch_decode_fused(st->shape, st->ws, st->cache, layer, layer_count, static_cast<const __half*>(d_q),
+                                     d_seq_lens, batch, fused_plan(st, layer_count, batch),
+                                     static_cast<__half*>(d_out), s) == cudaSuccess
+               ? BGTQ_OK
+               : BGTQ_ERR_CUDA;
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
@@ -695,8 +748,19 @@ int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const v
   v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   cudaStream_t s = as_stream(stream);
+  if (use_fused(st)) {
+    // the appends, then the fused decode (which rotates the query itself)
+    if (n > 0 && bgtq::launch_encode(st->shape, st->ws, st->cache, layer, layer_count, static_cast<const __half*>(d_k),
+                                     static_cast<const __half*>(d_v), d_start, d_count, batch, n, s) != cudaSuccess)
+      return BGTQ_ERR_CUDA;
+    return bgtq::launch_decode_fused(st->shape, st->ws, st->cache, layer, layer_count, static_cast<const __half*>(d_q),
+                                     d_seq_lens, batch, fused_plan(st, layer_count, batch),
+                                     static_cast<__half*>(d_out), s) == cudaSuccess
+               ? BGTQ_OK
+               : BGTQ_ERR_CUDA;
+  }
+  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   if (queue_step_prep(st, layer, layer_count, static_cast<const __half*>(d_q), batch, d_k, d_v, d_start, d_count, n,
                       s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
@@ -822,9 +886,31 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   const int v = check_decode_args(st, layer, layer_count, batch);
   if (v != BGTQ_OK) return v;
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_out)) return BGTQ_ERR_ALIGNMENT;
+  const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
+  if (use_fused(st)) {
+    // the fused decode: the arrival counters, then one partial per cluster
+    const bgtq::SplitPlan plan = fused_plan(st, layer_count, batch);
+    const int64_t nclu = plan.c_max / kFusedCluster;
+    const size_t part_bytes = rows * size_t(nclu) * bgtq::kPartialStride * sizeof(float);
+    if (rows * sizeof(uint32_t) > kStaticCountBytes || kStaticCountBytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES)
+      return BGTQ_ERR_BUFFER_SIZE;
+    void* base = nullptr;
+    const int a = static_scratch_address(&base);
+    if (a != BGTQ_OK) return a;
+    bgtq::Workspace ws = st->ws;
+    unsigned char* b8 = static_cast<unsigned char*>(base);
+    ws.comb_count = reinterpret_cast<uint32_t*>(b8);
+    ws.partials = reinterpret_cast<float*>(b8 + kStaticCountBytes);
+    bgtq::Shape shape = st->shape;
+    shape.max_splits = static_cast<int32_t>(nclu);
+    return bgtq::launch_decode_fused(shape, ws, st->cache, layer, layer_count, static_cast<const __half*>(d_q),
+                                     d_seq_lens, batch, plan, static_cast<__half*>(d_out), as_stream(stream)) ==
+                   cudaSuccess
+               ? BGTQ_OK
+               : BGTQ_ERR_CUDA;
+  }
   const bgtq::SplitPlan split = split_for(st, layer_count, batch);
   const int64_t nspl = split.c_max;
-  const size_t rows = size_t(layer_count) * st->cfg.max_batch * st->cfg.n_q_heads;
   // the combine's arrival counters first, at a fixed place (they are 0
   // between calls, whatever the call's layout), then q~, its fragments, the
   // split partials and the combine's slice merges
@@ -884,6 +970,22 @@ int bgtq_set_split_tokens(bgtq_state* st, int32_t tokens) {
   if (tokens < 0 || tokens % bgtq::kSplitGranule != 0) return BGTQ_ERR_INVALID_ARG;
   if (tokens > 0 && (st->cfg.capacity_tokens + tokens - 1) / tokens > max_splits_of(&st->cfg)) return BGTQ_ERR_INVALID_ARG;
   st->split_tokens = tokens;
+  return BGTQ_OK;
+}
+
+int bgtq_set_decode_path(bgtq_state* st, int32_t fused) {
+  if (!st) return BGTQ_ERR_NULL;
+  if (fused != 0 && fused != 1) return BGTQ_ERR_INVALID_ARG;
+  st->decode_mode = fused;
+  return BGTQ_OK;
+}
+
+int bgtq_get_decode_path(bgtq_state* st, int32_t* h_fused, int32_t* h_ctas) {
+  if (!st || !h_fused || !h_ctas) return BGTQ_ERR_NULL;
+  if (const int dv = check_device(st)) return dv;
+  const bool f = use_fused(st);
+  *h_fused = f ? 1 : 0;
+  *h_ctas = f ? fused_slots(st) : split_slots(st);
   return BGTQ_OK;
 }
 

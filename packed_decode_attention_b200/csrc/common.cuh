@@ -92,10 +92,14 @@ struct ByteTab {
   uint32_t lo[4], hi[4];
 };
 
-// Four codes (selector nibbles 0..3) -> two fp16x2 registers: codes (0, 1)
-// and codes (2, 3).  PRMT picks bytes 0..7 of its two table words by the
-// nibble's low three bits; width-4 codes look up both halves of the table
-// and pick by their top bit.
+// Four symbols (selector nibbles 0..3) -> two fp16x2 registers: symbols
+// (0, 1) and (2, 3).  PRMT picks bytes 0..7 of its two table words by the
+// nibble's low three bits.  Width 4 holds sign-magnitude symbols: the low
+// three bits pick |level| from the 8-entry table.  For the sign, each
+// nibble of sel >> 1 has the symbol's sign bit as its bit 2, so it picks
+// 0x80 (sign set) or 0x00 from the words (0, 0x80808080); its bit 3 (the
+// next symbol's bit 0) may switch PRMT to replicating that byte's top bit,
+// which leaves the top bit as it is.  That top bit becomes the fp16 sign.
 template <int B>
 __device__ __forceinline__ void lookup4(const ByteTab& t, uint32_t sel, uint32_t& r01, uint32_t& r23) {
   uint32_t lo, hi;
@@ -104,9 +108,10 @@ __device__ __forceinline__ void lookup4(const ByteTab& t, uint32_t sel, uint32_t
     hi = prmt(t.hi[0], t.hi[1], sel);
   } else {
     const uint32_t s7 = sel & 0x7777u;
-    const uint32_t pick = 0x3210u | ((sel >> 1) & 0x4444u);
-    lo = prmt(prmt(t.lo[0], t.lo[1], s7), prmt(t.lo[2], t.lo[3], s7), pick);
-    hi = prmt(prmt(t.hi[0], t.hi[1], s7), prmt(t.hi[2], t.hi[3], s7), pick);
+    lo = prmt(t.lo[0], t.lo[1], s7);
+    hi = prmt(t.hi[0], t.hi[1], s7);
+    const uint32_t neg = prmt(0u, 0x80808080u, sel >> 1);
+    hi ^= neg & 0x80808080u;
   }
   r01 = prmt(lo, hi, 0x5140u);
   r23 = prmt(lo, hi, 0x7362u);
@@ -120,6 +125,16 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A * B for one m16n8k16 tile (the accumulator starts at zero).
+__device__ __forceinline__ void mma16816_zero(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
 // A-fragment from one selector word (rows g and g+8) times a B-fragment.
@@ -354,8 +369,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// S[mu] += A(selector s[mu]) * (q~ hi + q~ lo) for the four M-tiles of a chunk.
-template <bool WIDE>
+// S[mu] += A(selector s[mu]) * (q~ hi + q~ lo) for the four M-tiles of a
+// chunk; FIRST: S starts at zero (the group's first chunk).
+template <bool WIDE, bool FIRST>
 __device__ __forceinline__ void chunk_mma(const ByteTab& t, const uint32_t* s, uint4 bf, float (*S)[4]) {
   uint32_t a[4][4];
 #pragma unroll
@@ -364,7 +380,10 @@ __device__ __forceinline__ void chunk_mma(const ByteTab& t, const uint32_t* s, u
     lookup4<WIDE ? 4 : 3>(t, s[mu] >> 16, a[mu][1], a[mu][3]);
   }
 #pragma unroll
-  for (int mu = 0; mu < 4; ++mu) mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.x, bf.y);
+  for (int mu = 0; mu < 4; ++mu) {
+    if constexpr (FIRST) mma16816_zero(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.x, bf.y);
+    else mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.x, bf.y);
+  }
 #pragma unroll
   for (int mu = 0; mu < 4; ++mu) mma16816(S[mu], a[mu][0], a[mu][1], a[mu][2], a[mu][3], bf.z, bf.w);
 }
@@ -375,16 +394,25 @@ __device__ __forceinline__ void chunk_mma(const ByteTab& t, const uint32_t* s, u
 // stride per plane word (bits 12..19) inside the partial region, bit 20 set
 // for a half-quad lane, bit 21 for the upper half of its virtual lane.  Lanes
 // with no coordinates read any word of the region: their B rows are zero.
+// S need not be initialised: the group's first chunk overwrites it (a group
+// has at least one chunk).
 template <int B>
 __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool partial, uint32_t pd,
                                              const uint4* bqg, const ByteTab& t, int lane, float (*S)[4]) {
+  if (nfull > 0) {
+    uint32_t w[B], s[4];
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = gw[32 * k + lane];
+    quartet_decode<B>(w, s);
+    chunk_mma<B == 4, true>(t, s, bqg[0], S);
+  }
 #pragma unroll 1
-  for (int j = 0; j < nfull; ++j) {
+  for (int j = 1; j < nfull; ++j) {
     uint32_t w[B], s[4];
 #pragma unroll
     for (int k = 0; k < B; ++k) w[k] = gw[j * 32 * B + 32 * k + lane];
     quartet_decode<B>(w, s);
-    chunk_mma<B == 4>(t, s, bqg[j * 32], S);
+    chunk_mma<B == 4, false>(t, s, bqg[j * 32], S);
   }
   if (partial) {
     const uint32_t* pc = gw + nfull * 32 * B;
@@ -401,7 +429,8 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
         s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
       }
     }
-    chunk_mma<B == 4>(t, s, bqg[nfull * 32], S);
+    if (nfull > 0) chunk_mma<B == 4, false>(t, s, bqg[nfull * 32], S);
+    else chunk_mma<B == 4, true>(t, s, bqg[0], S);
   }
 }
 

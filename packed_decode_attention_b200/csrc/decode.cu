@@ -1,6 +1,9 @@
 // Decode kernels of the Block-GTQ path (B200, sm_100a):
 //
-//   decode_mma_kernel    split-K flash decoding from the packed tiles (mma.sync),
+//   decode_fused_kernel  query rotation, split-K flash decoding from the packed
+//                        tiles (mma.sync), split merge and inverse V rotation
+//                        in one launch (thread-block clusters)
+//   decode_mma_kernel    the split-K pass alone (caller's q~, stage calls),
 //                        with the fp16 sink / window rows of a buffered call
 //   combine_kernel       log-sum-exp merge of the splits + inverse V rotation
 //
@@ -145,6 +148,12 @@ __device__ __forceinline__ int split_ctas(const SplitPlan& p, int64_t ntl, int64
   c = c < 1 ? 1 : c;
   c = c < ntl ? c : ntl;
   c = c < p.c_max ? c : p.c_max;
+  // whole clusters (c_max is a multiple of the cluster size): a set split
+  // size rounds up; the one-wave budget rounds down, to stay one wave
+  if (p.cluster > 1) {
+    c = p.fixed_tiles > 0 ? (c + p.cluster - 1) / p.cluster * p.cluster : c / p.cluster * p.cluster;
+    c = c < p.cluster ? p.cluster : c;
+  }
   return static_cast<int>(c);
 }
 
@@ -298,6 +307,286 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
 }
 
+// ---------------------------------------------------------------------------
+// The per-warp tile loop shared by the split pass and the fused decode.
+//
+// A warp attends the tiles tlo + wu + k W (k < my_tiles) of one (layer,
+// sequence, KV head) unit for up to 8 query heads: its own 2-stage pipeline
+// of bulk copies (K tile, V tile, norms -> shared memory, completion on an
+// mbarrier, bounded waits) and its own online-softmax state (O in V's rotated
+// basis, the running maximum and denominator of heads 2 t4 and 2 t4 + 1).
+// ---------------------------------------------------------------------------
+struct TileSource {
+  Shape sh;
+  CacheDev cache;
+  uint32_t* err;
+  int layer, b, h;
+  int tlo, wu, W;        // the warp's first tile is tlo + wu, then every W-th
+  int kwords, vwords;    // 32-bit words of a K / V tile
+  unsigned char* stage;  // this warp's first stage buffer; stage k at stage + k * stage_stride
+  int stage_stride;
+  uint64_t* bars;        // the stages' mbarriers
+  int stage_bytes;
+};
+
+// Lane 0: copy the warp's k-th tile into stage k % kStages.
+__device__ __forceinline__ void issue_tile(const TileSource& src, int k) {
+  const uint32_t kbytes = 4u * src.kwords, vbytes = 4u * src.vwords;
+  const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
+  const int tile = src.tlo + src.wu + k * src.W;
+  uint64_t* bar = &src.bars[k % kStages];
+  if (tile == src.sh.drop_tile) {
+    // test hook: the copy is never issued, so the wait on it runs out
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(bar, stage_tx);
+    return;
+  }
+  int64_t slot = tile_slot(src.sh, src.cache, src.layer, src.b, src.h, tile);
+  if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
+    atomicOr(src.err, kErrPage);
+    slot = static_cast<int64_t>(src.layer * src.sh.n_kv_heads + src.h) * src.cache.n_pages;
+  }
+  unsigned char* dst = src.stage + (k % kStages) * src.stage_stride;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  mbar_expect_tx(bar, stage_tx);
+  bulk_copy_g2s(dst, src.cache.ktile + slot * src.kwords, kbytes, bar);
+  bulk_copy_g2s(dst + kbytes, src.cache.vtile + slot * src.vwords, vbytes, bar);
+  bulk_copy_g2s(dst + kbytes + vbytes, src.cache.knorm + slot * kTile * 4, kTile * 8, bar);
+  bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, src.cache.vnorm + slot * kTile, kTile * 2, bar);
+}
+
+// The decode tables a warp reads from shared memory (a copy of the
+// DecodeTableDev of its (layer, KV head)) and the query fragments.
+struct TileTables {
+  const int32_t* grp;
+  const uint32_t* tabk;
+  const uint32_t* pdesc;
+  const uint4* bq;
+  int ng;
+};
+
+// Attends the warp's my_tiles tiles over the positions [lo, len); the first
+// min(kStages, my_tiles) copies must already be issued.  Returns the index of
+// the tile whose copy wait gave up (-1: none).
+template <int VB>
+__device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTables& tt, const ByteTab& tv,
+                                            int my_tiles, int len, int lo, float (&O)[8][4], float (&m_run)[2],
+                                            float (&l_run)[2]) {
+  const int lane = threadIdx.x & 31;
+  const int g8 = lane >> 2;
+  const uint32_t kbytes = 4u * src.kwords, vbytes = 4u * src.vwords;
+#pragma unroll
+  for (int m = 0; m < 8; ++m)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) O[m][r] = 0.f;
+  m_run[0] = m_run[1] = -CUDART_INF_F;
+  l_run[0] = l_run[1] = 0.f;
+  int failed_at = -1;
+
+  for (int k = 0; k < my_tiles; ++k) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&src.bars[k % kStages], (k / kStages) & 1))) {
+      failed_at = k;
+      break;
+    }
+    const unsigned char* st = src.stage + (k % kStages) * src.stage_stride;
+    const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
+    const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
+    const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
+    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
+    const int tpos = (src.tlo + src.wu + k * src.W) * kTile;
+    const int nvalid = min(kTile, len - tpos);       // positions [nlow, nvalid) of the tile are attended
+    const int nlow = max(0, lo - tpos);
+
+    // logits, one width group at a time, each scaled by its per-token norm
+    float L[4][4];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) L[mu][r] = 0.f;
+    for (int g = 0; g < tt.ng; ++g) {
+      const int4 gp = *reinterpret_cast<const int4*>(tt.grp + g * 8);  // width, nfull, r, word
+      const int chunk = tt.grp[g * 8 + 4];
+      ByteTab t;
+      const uint4 tl = *reinterpret_cast<const uint4*>(tt.tabk + 8 * g);
+      const uint4 th = *reinterpret_cast<const uint4*>(tt.tabk + 8 * g + 4);
+      t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
+      t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+      const uint32_t pd = tt.pdesc[g * 32 + lane];
+      const uint32_t* gw = kt + gp.w;
+      const uint4* bqg = tt.bq + chunk * 32 + lane;
+      float S[4][4];
+      switch (gp.x) {
+        case 1: group_logits<1>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 2: group_logits<2>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        case 3: group_logits<3>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+        default: group_logits<4>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
+      }
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
+        const float nb = __half2float(kn[(16 * mu + g8 + 8) * 4 + g]);
+        L[mu][0] = fmaf(na, S[mu][0], L[mu][0]);
+        L[mu][1] = fmaf(na, S[mu][1], L[mu][1]);
+        L[mu][2] = fmaf(nb, S[mu][2], L[mu][2]);
+        L[mu][3] = fmaf(nb, S[mu][3], L[mu][3]);
+      }
+    }
+    // online softmax over the tile for heads 2*t4 and 2*t4+1; positions past
+    // the valid length carry no weight (their norms may be anything)
+    float wv[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      wv[mu][0] = __half2float(vn[16 * mu + g8]) * kInvSqrtD;
+      wv[mu][1] = __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD;
+    }
+    if (nvalid < kTile || nlow > 0) {
+#pragma unroll
+      for (int mu = 0; mu < 4; ++mu) {
+        if (16 * mu + g8 >= nvalid || 16 * mu + g8 < nlow) {
+          L[mu][0] = L[mu][1] = -CUDART_INF_F;
+          wv[mu][0] = 0.f;
+        }
+        if (16 * mu + g8 + 8 >= nvalid || 16 * mu + g8 + 8 < nlow) {
+          L[mu][2] = L[mu][3] = -CUDART_INF_F;
+          wv[mu][1] = 0.f;
+        }
+      }
+    }
+    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
+      mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
+    }
+    // The reference maximum moves only when some logit of the tile exceeds it
+    // by more than kRescaleSlack (log2 units), so O is rescaled rarely;
+    // weights stay <= 2^kRescaleSlack and l and O always share the same
+    // reference.  l is kept per lane and summed over the warp at the end.
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kRescaleSlack || mx[1] > m_run[1] + kRescaleSlack)) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
+      }
+      float alpha[2] = {1.f, 1.f};
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (mx[c] > m_run[c] + kRescaleSlack) {
+          alpha[c] = fast_exp2(m_run[c] - mx[c]);
+          m_run[c] = mx[c];
+        }
+        l_run[c] *= alpha[c];
+      }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        O[m][0] *= alpha[0];
+        O[m][1] *= alpha[1];
+        O[m][2] *= alpha[0];
+        O[m][3] *= alpha[1];
+      }
+    }
+    uint32_t bp[4][2];
+#pragma unroll
+    for (int mu = 0; mu < 4; ++mu) {
+      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
+      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
+      l_run[0] += p0 + p2;
+      l_run[1] += p1 + p3;
+      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
+      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
+    }
+    // P V in V's rotated basis
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      uint32_t w[VB], sv[4];
+#pragma unroll
+      for (int kk = 0; kk < VB; ++kk) w[kk] = vt[m * 32 * VB + 32 * kk + lane];
+      quartet_decode<VB>(w, sv);
+#pragma unroll
+      for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
+    }
+    __syncwarp();
+    if (lane == 0 && k + kStages < my_tiles) issue_tile(src, k + kStages);
+  }
+  if (failed_at >= 0) {
+    // copies issued but not yet consumed: let them land (bounded) before the
+    // stage buffers are reused or the CTA exits
+    if (lane == 0) atomicOr(src.err, kErrTimeout);
+    const int issued = min(my_tiles, failed_at + kStages);
+    for (int k = failed_at; k < issued; ++k) mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
+  }
+  return failed_at;
+}
+
+// Merges the CTA's warps (called by all threads after attend_tiles) into one
+// (m, l, acc[128]) per query head of the block: cm[8], clsum[8] and
+// cacc[8][128] (shared memory; cacc may alias the stage buffers, which are
+// free once every warp has left its loop).  accs: [kDecWarps][8][128] of
+// shared scratch (may alias the stage buffers too, not cacc); ms, ls:
+// [kDecWarps][8] each.  A CTA with a timed-out warp posts empty partials.
+__device__ __forceinline__ void merge_warps(const float (&O)[8][4], const float (&m_run)[2], float (&l_run)[2],
+                                            bool timed_out, float* accs, float* ms, float* ls, float* wsc, float* cm,
+                                            float* clsum, float* cacc, int nh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
+  }
+  __syncthreads();  // every warp has left its loop: the stage buffers are free
+  if (g8 == 0) {
+    ms[warp * 8 + 2 * t4] = m_run[0];
+    ms[warp * 8 + 2 * t4 + 1] = m_run[1];
+    ls[warp * 8 + 2 * t4] = l_run[0];
+    ls[warp * 8 + 2 * t4 + 1] = l_run[1];
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    float* a = accs + warp * 8 * kD;
+    a[(2 * t4) * kD + 16 * m + g8] = O[m][0];
+    a[(2 * t4 + 1) * kD + 16 * m + g8] = O[m][1];
+    a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
+    a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
+  }
+  const bool cta_timed_out = __syncthreads_or(timed_out);
+  // per head: the common maximum, the warps' weights (warps without a tile
+  // hold m = -inf, l = 0, acc = 0) and the weighted denominator
+  if (tid < 8 && cta_timed_out) {
+    for (int w = 0; w < kDecWarps; ++w) wsc[w * 8 + tid] = 0.f;
+    cm[tid] = -CUDART_INF_F;
+    clsum[tid] = 0.f;
+  } else if (tid < 8) {
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
+    float lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float mw = ms[w * 8 + tid];
+      const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
+      wsc[w * 8 + tid] = sc;
+      lsum = fmaf(sc, ls[w * 8 + tid], lsum);
+    }
+    cm[tid] = M;
+    clsum[tid] = lsum;
+  }
+  __syncthreads();
+  const int i = tid;  // kDecThreads == kD: a thread per dimension
+  float a[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    a[hh] = 0.f;
+    if (hh < nh) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) a[hh] = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a[hh]);
+    }
+  }
+  __syncthreads();  // cacc may alias accs
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) cacc[hh * kD + i] = a[hh];
+  __syncthreads();
+}
 // Grid (batch * Hkv * head_blocks, [1 buffer CTA +] plan.c_max, layer_count),
 // 128 threads.  A unit is one (layer, sequence, KV head, block of up to 8
 // query heads); it uses C = split_ctas(...) of its c_max split CTAs (more for
@@ -325,7 +614,6 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   unsigned char* stage_base = smem_raw + DL.stage;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g8 = lane >> 2, t4 = lane & 3;
   // grid row 0 holds the buffer CTAs of a buffered call, so they are
   // dispatched first; the split CTAs follow
   const bool has_buf = buf.k != nullptr;
@@ -469,242 +757,419 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   __syncthreads();
 
   // ---- per-warp pipeline over this warp's tiles ----
-  const int kwords = 256 * sh.kbits, vwords = 256 * VB;
-  const uint32_t kbytes = 4u * kwords, vbytes = 4u * vwords;
-  const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
-  unsigned char* my_stage = stage_base + static_cast<size_t>(warp) * kStages * DL.stage_bytes;
-  uint64_t* my_bars = bars + warp * kStages;
-
-  auto issue = [&](int k) {  // lane 0: copy this warp's k-th tile into stage k % kStages
-    const int tile = tlo + wu + k * W;
-    if (tile == sh.drop_tile) {
-      // test hook: the copy is never issued, so the wait on it runs out
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_expect_tx(&my_bars[k % kStages], stage_tx);
-      return;
-    }
-    int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
-    if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
-      atomicOr(ws.err, kErrPage);
-      slot = static_cast<int64_t>(layer * sh.n_kv_heads + h) * cache.n_pages;
-    }
-    unsigned char* dst = my_stage + (k % kStages) * DL.stage_bytes;
-    uint64_t* bar = &my_bars[k % kStages];
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(bar, stage_tx);
-    bulk_copy_g2s(dst, cache.ktile + slot * kwords, kbytes, bar);
-    bulk_copy_g2s(dst + kbytes, cache.vtile + slot * vwords, vbytes, bar);
-    bulk_copy_g2s(dst + kbytes + vbytes, cache.knorm + slot * kTile * 4, kTile * 8, bar);
-    bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, cache.vnorm + slot * kTile, kTile * 2, bar);
-  };
+  TileSource src;
+  src.sh = sh;
+  src.cache = cache;
+  src.err = ws.err;
+  src.layer = layer;
+  src.b = b;
+  src.h = h;
+  src.tlo = tlo;
+  src.wu = wu;
+  src.W = W;
+  src.kwords = 256 * sh.kbits;
+  src.vwords = 256 * VB;
+  src.stage = stage_base + static_cast<size_t>(warp) * kStages * DL.stage_bytes;
+  src.stage_stride = DL.stage_bytes;
+  src.bars = bars + warp * kStages;
+  src.stage_bytes = DL.stage_bytes;
   if (lane == 0)
-    for (int k = 0; k < kStages && k < my_tiles; ++k) issue(k);
-
-  float O[8][4];
-#pragma unroll
-  for (int m = 0; m < 8; ++m)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) O[m][r] = 0.f;
-  float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
-  int failed_at = -1;
-
-  for (int k = 0; k < my_tiles; ++k) {
-    if (!__all_sync(0xffffffffu, mbar_wait(&my_bars[k % kStages], (k / kStages) & 1))) {
-      failed_at = k;
-      break;
-    }
-    const unsigned char* st = my_stage + (k % kStages) * DL.stage_bytes;
-    const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
-    const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
-    const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
-    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
-    const int tpos = (tlo + wu + k * W) * kTile;
-    const int nvalid = min(kTile, len - tpos);       // positions [nlow, nvalid) of the tile are attended
-    const int nlow = max(0, lo - tpos);
-
-    // logits, one width group at a time, each scaled by its per-token norm
-    float L[4][4];
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) L[mu][r] = 0.f;
-    for (int g = 0; g < ng; ++g) {
-      const int4 gp = *reinterpret_cast<const int4*>(grp + g * 8);  // width, nfull, r, word
-      const int chunk = grp[g * 8 + 4];
-      ByteTab t;
-      const uint4 tl = *reinterpret_cast<const uint4*>(tabk + 8 * g);
-      const uint4 th = *reinterpret_cast<const uint4*>(tabk + 8 * g + 4);
-      t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
-      t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
-      const uint32_t pd = pdesc[g * 32 + lane];
-      const uint32_t* gw = kt + gp.w;
-      const uint4* bqg = bq + chunk * 32 + lane;
-      float S[4][4];
-#pragma unroll
-      for (int mu = 0; mu < 4; ++mu)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) S[mu][r] = 0.f;
-      switch (gp.x) {
-        case 1: group_logits<1>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
-        case 2: group_logits<2>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
-        case 3: group_logits<3>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
-        default: group_logits<4>(gw, gp.y, gp.z != 0, pd, bqg, t, lane, S); break;
-      }
-#pragma unroll
-      for (int mu = 0; mu < 4; ++mu) {
-        const float na = __half2float(kn[(16 * mu + g8) * 4 + g]);
-        const float nb = __half2float(kn[(16 * mu + g8 + 8) * 4 + g]);
-        L[mu][0] = fmaf(na, S[mu][0], L[mu][0]);
-        L[mu][1] = fmaf(na, S[mu][1], L[mu][1]);
-        L[mu][2] = fmaf(nb, S[mu][2], L[mu][2]);
-        L[mu][3] = fmaf(nb, S[mu][3], L[mu][3]);
-      }
-    }
-    // online softmax over the tile for heads 2*t4 and 2*t4+1; positions past
-    // the valid length carry no weight (their norms may be anything)
-    float wv[4][2];
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      wv[mu][0] = __half2float(vn[16 * mu + g8]) * kInvSqrtD;
-      wv[mu][1] = __half2float(vn[16 * mu + g8 + 8]) * kInvSqrtD;
-    }
-    if (nvalid < kTile || nlow > 0) {
-#pragma unroll
-      for (int mu = 0; mu < 4; ++mu) {
-        if (16 * mu + g8 >= nvalid || 16 * mu + g8 < nlow) {
-          L[mu][0] = L[mu][1] = -CUDART_INF_F;
-          wv[mu][0] = 0.f;
-        }
-        if (16 * mu + g8 + 8 >= nvalid || 16 * mu + g8 + 8 < nlow) {
-          L[mu][2] = L[mu][3] = -CUDART_INF_F;
-          wv[mu][1] = 0.f;
-        }
-      }
-    }
-    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      mx[0] = fmaxf(mx[0], fmaxf(L[mu][0], L[mu][2]));
-      mx[1] = fmaxf(mx[1], fmaxf(L[mu][1], L[mu][3]));
-    }
-    // The reference maximum moves only when some logit of the tile exceeds it
-    // by more than kRescaleSlack (log2 units), so O is rescaled rarely;
-    // weights stay <= 2^kRescaleSlack and l and O always share the same
-    // reference.  l is kept per lane and summed over the warp at the end.
-    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + kRescaleSlack || mx[1] > m_run[1] + kRescaleSlack)) {
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
-        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
-      }
-      float alpha[2] = {1.f, 1.f};
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (mx[c] > m_run[c] + kRescaleSlack) {
-          alpha[c] = fast_exp2(m_run[c] - mx[c]);
-          m_run[c] = mx[c];
-        }
-        l_run[c] *= alpha[c];
-      }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        O[m][0] *= alpha[0];
-        O[m][1] *= alpha[1];
-        O[m][2] *= alpha[0];
-        O[m][3] *= alpha[1];
-      }
-    }
-    uint32_t bp[4][2];
-#pragma unroll
-    for (int mu = 0; mu < 4; ++mu) {
-      const float p0 = fast_exp2(L[mu][0] - m_run[0]), p1 = fast_exp2(L[mu][1] - m_run[1]);
-      const float p2 = fast_exp2(L[mu][2] - m_run[0]), p3 = fast_exp2(L[mu][3] - m_run[1]);
-      l_run[0] += p0 + p2;
-      l_run[1] += p1 + p3;
-      bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
-      bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
-    }
-    // P V in V's rotated basis
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      uint32_t w[VB], sv[4];
-#pragma unroll
-      for (int kk = 0; kk < VB; ++kk) w[kk] = vt[m * 32 * VB + 32 * kk + lane];
-      quartet_decode<VB>(w, sv);
-#pragma unroll
-      for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
-    }
-    __syncwarp();
-    if (lane == 0 && k + kStages < my_tiles) issue(k + kStages);
-  }
+    for (int k = 0; k < kStages && k < my_tiles; ++k) issue_tile(src, k);
+  TileTables tt{grp, tabk, pdesc, bq, ng};
+  float O[8][4], m_run[2], l_run[2];
+  const int failed_at = attend_tiles<VB>(src, tt, tv, my_tiles, len, lo, O, m_run, l_run);
   // the combine kernel may be scheduled now; it waits for this grid before reading the partials
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const bool timed_out = failed_at >= 0;
-  if (timed_out) {
-    if (lane == 0) atomicOr(ws.err, kErrTimeout);
-    // copies issued but not yet consumed: let them land (bounded) before the
-    // stage buffers are reused or the CTA exits
-    const int issued = min(my_tiles, failed_at + kStages);
-    for (int k = failed_at; k < issued; ++k) mbar_wait(&my_bars[k % kStages], (k / kStages) & 1);
-  }
-  __syncthreads();
-  // ---- merge the warps (the stage buffers are reused) ----
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
-  }
-  float* accs = reinterpret_cast<float*>(stage_base);  // [warp][8 heads][128]
-  if (g8 == 0) {
-    ms[warp * 8 + 2 * t4] = m_run[0];
-    ms[warp * 8 + 2 * t4 + 1] = m_run[1];
-    ls[warp * 8 + 2 * t4] = l_run[0];
-    ls[warp * 8 + 2 * t4 + 1] = l_run[1];
-  }
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    float* a = accs + warp * 8 * kD;
-    a[(2 * t4) * kD + 16 * m + g8] = O[m][0];
-    a[(2 * t4 + 1) * kD + 16 * m + g8] = O[m][1];
-    a[(2 * t4) * kD + 16 * m + g8 + 8] = O[m][2];
-    a[(2 * t4 + 1) * kD + 16 * m + g8 + 8] = O[m][3];
-  }
-  const bool cta_timed_out = __syncthreads_or(timed_out);
-  // per head: the common maximum, the warps' weights (warps without a tile
-  // hold m = -inf, l = 0, acc = 0) and the weighted denominator; a CTA that
-  // gave up on a copy posts empty partials (its error flag is raised)
+  // ---- merge the warps (the stage buffers are reused) and post the partials ----
+  float* cacc = reinterpret_cast<float*>(stage_base);
   float* wsc = reinterpret_cast<float*>(smem_raw + DL.wsc);
   float* mres = reinterpret_cast<float*>(smem_raw + DL.mres);
-  if (tid < 8 && cta_timed_out) {
-    for (int w = 0; w < kDecWarps; ++w) wsc[w * 8 + tid] = 0.f;
-    mres[tid] = -CUDART_INF_F;
-    mres[8 + tid] = 0.f;
-  } else if (tid < 8) {
-    float M = -CUDART_INF_F;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
-    float lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-      const float mw = ms[w * 8 + tid];
-      const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
-      wsc[w * 8 + tid] = sc;
-      lsum = fmaf(sc, ls[w * 8 + tid], lsum);
-    }
-    mres[tid] = M;
-    mres[8 + tid] = lsum;
-  }
-  __syncthreads();
+  merge_warps(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, mres, mres + 8,
+              cacc, nh);
   const int i = tid;
   for (int hh = 0; hh < nh; ++hh) {
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) a = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a);
     float* part = part_base + hh * part_head_stride;
-    part[4 + i] = cta_timed_out ? 0.f : a;
+    part[4 + i] = cacc[hh * kD + i];
     if (i == 0) {
       part[0] = mres[hh];
       part[1] = mres[8 + hh];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused decode: the query rotation, the split-K pass and the split merge with
+// the inverse V rotation in one launch.
+//
+// Grid (batch * Hkv * head_blocks, plan.c_max, layer_count) in thread-block
+// clusters of kFusedCluster CTAs along y, 128 threads.  A unit (layer,
+// sequence, KV head, block of up to 8 query heads) uses C = split_ctas(...)
+// of its c_max CTAs, a multiple of the cluster size (whole clusters; unused
+// clusters exit at once).  Its tiles are dealt over the 4 C warps exactly as
+// in the split pass.
+//
+//  1. Before the dependency wait: the decode table, and rows
+//     [16 r, 16 r + 16) of the unit's K rotation (CTA rank r of the cluster).
+//  2. After it: the unit's query rows (gathered into record order); CTA r
+//     computes q~ for coordinates [16 r, 16 r + 16) of all heads and writes
+//     them into every CTA of its cluster (distributed shared memory); each
+//     CTA then builds its own mma B fragments.  The first tile copy of every
+//     warp is already in flight meanwhile.
+//  3. The tile loop (attend_tiles) and the merge of the CTA's warps.
+//  4. Cluster merge: CTA r merges head r over the cluster's CTAs (reading
+//     their shared memory) and posts one partial per cluster.
+//  5. The unit's last cluster to arrive (a counter it resets) merges the
+//     clusters' partials (CTA r: head r), shares the normalised accumulators
+//     through distributed shared memory, and CTA r writes output dims
+//     [16 r, 16 r + 16) of every head: o = R_V^T (sum_c w_c acc_c) /
+//     (sum_c w_c l_c), with w_c = 2^(m_c - max m).
+// No CTA waits on another outside its cluster's hardware barriers, so the
+// grid needs no co-residency beyond the cluster's.
+// ---------------------------------------------------------------------------
+constexpr int kFusedCluster = 8;
+constexpr int kRowPad = kD + 1;  // row pitch (floats) of the rotation scratch: consecutive rows in different banks
+static_assert(kFusedCluster * 16 == kD, "each CTA of a cluster rotates 16 coordinates");
+
+struct FusedLayout {  // byte offsets inside the dynamic shared memory
+  int bars, bq, tab, ms, ls, wsc, cm, flag, qt, stage, stage_bytes, rot, total;
+};
+
+__host__ __device__ inline FusedLayout fused_layout(int kbits, int vbits) {
+  FusedLayout L;
+  L.bars = 0;
+  L.bq = align128(kDecWarps * kStages * 8);
+  L.tab = L.bq + kMaxChunks * 32 * 16;
+  L.ms = L.tab + static_cast<int>(sizeof(DecodeTableDev));
+  L.ls = L.ms + kDecWarps * 8 * 4;
+  L.wsc = L.ls + kDecWarps * 8 * 4;
+  L.cm = L.wsc + kDecWarps * 8 * 4;           // the CTA's merged m[8], l[8]
+  L.flag = L.cm + 16 * 4;                      // "this cluster merges the unit" (written by rank 0)
+  L.qt = align128(L.flag + 16);                // q~ [8][kRowPad] fp32, later the merged accumulators
+  L.stage = align128(L.qt + 8 * kRowPad * 4);
+  L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
+  // stage k of warp w at stage + (k * kDecWarps + w) * stage_bytes: the
+  // second stages form one block, which holds the K rotation rows [16][kRowPad]
+  // and the query rows [8][kRowPad] until the first tiles are in flight, and
+  // the inverse V rotation slice [16][kRowPad] in the last cluster's merge
+  L.rot = L.stage + kDecWarps * L.stage_bytes;
+  const int rot_bytes = (16 + 8) * kRowPad * 4;
+  int need = kDecWarps * kStages * L.stage_bytes;
+  if (need < kDecWarps * L.stage_bytes + rot_bytes) need = kDecWarps * L.stage_bytes + rot_bytes;
+  const int merge = kDecWarps * 8 * kD * 4;  // the warp merge reuses the stage buffers
+  if (need < merge) need = merge;
+  L.total = L.stage + need;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+
+__device__ __forceinline__ void dsmem_st(uint32_t a, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void dsmem_st_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float dsmem_ld(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+
+// Every thread of every CTA of the cluster: shared-memory writes before it
+// (local or remote) are visible to every CTA after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int VB>
+__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+    decode_fused_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const __half* __restrict__ q,
+                        const int32_t* __restrict__ seq_lens, int batch, SplitPlan plan, int head_blocks,
+                        __half* __restrict__ out) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const FusedLayout FL = fused_layout(sh.kbits, VB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + FL.bars);
+  uint4* bq = reinterpret_cast<uint4*>(smem_raw + FL.bq);
+  int32_t* grp = reinterpret_cast<int32_t*>(smem_raw + FL.tab);  // grp, tabk, pdesc, tabv are contiguous
+  const uint32_t* tabk = reinterpret_cast<const uint32_t*>(smem_raw + FL.tab + offsetof(DecodeTableDev, tabk));
+  const uint32_t* pdesc = reinterpret_cast<const uint32_t*>(smem_raw + FL.tab + offsetof(DecodeTableDev, pdesc));
+  const uint32_t* tabv = reinterpret_cast<const uint32_t*>(smem_raw + FL.tab + offsetof(DecodeTableDev, tabv));
+  float* ms = reinterpret_cast<float*>(smem_raw + FL.ms);
+  float* ls = reinterpret_cast<float*>(smem_raw + FL.ls);
+  float* wsc = reinterpret_cast<float*>(smem_raw + FL.wsc);
+  float* cm = reinterpret_cast<float*>(smem_raw + FL.cm);
+  uint32_t* flag = reinterpret_cast<uint32_t*>(smem_raw + FL.flag);
+  float* qt = reinterpret_cast<float*>(smem_raw + FL.qt);
+  unsigned char* stage_base = smem_raw + FL.stage;
+  float* rk = reinterpret_cast<float*>(smem_raw + FL.rot);  // [16][kRowPad]
+  float* qr = rk + 16 * kRowPad;                              // [8][kRowPad]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cu = blockIdx.y;
+  const int rank = cu % kFusedCluster;  // the CTA's rank in its cluster (clusters run along y)
+  const int clu = cu / kFusedCluster;
+  const int hb = blockIdx.x % head_blocks;
+  const int h = (blockIdx.x / head_blocks) % sh.n_kv_heads;
+  const int b = blockIdx.x / (head_blocks * sh.n_kv_heads);
+  const int li = blockIdx.z;
+  const int layer = layer0 + li;
+  const int G = sh.group;
+  const int h0 = 8 * hb;
+  const int nh = min(8, G - h0);
+  const int lh = layer * sh.n_kv_heads + h;
+  const LayoutDev& lay = ws.layouts[lh];
+  const int ng = lay.n_groups;
+
+  // ---- 1. library tables only (the previous kernel may still run) ----
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(ws.dectab + lh);
+    uint4* dst = reinterpret_cast<uint4*>(grp);
+    for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += kDecThreads) dst[u] = src[u];
+  }
+  if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
+  // rows [16 rank, 16 rank + 16) of the block-diagonal K rotation (record
+  // order): R[i][j] = mkt[j][i]
+  {
+    const float* mk = ws.mkt + static_cast<size_t>(lh) * kD * kD;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int f = tid + k * kDecThreads;  // 512 float4 = 128 inputs x 16 outputs
+      const int j = f >> 2, q4 = f & 3;
+      const float4 v = *reinterpret_cast<const float4*>(mk + j * kD + 16 * rank + 4 * q4);
+      rk[(4 * q4 + 0) * kRowPad + j] = v.x;
+      rk[(4 * q4 + 1) * kRowPad + j] = v.y;
+      rk[(4 * q4 + 2) * kRowPad + j] = v.z;
+      rk[(4 * q4 + 3) * kRowPad + j] = v.w;
+    }
+  }
+  const int perm_j = lay.perm[tid] & (kD - 1);  // kDecThreads == kD: the original dim of record position tid
+  __syncthreads();
+  if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (lane == 0 && batch == 1) {
+    // L2 prefetch of this warp's first tile, as if the sequence were full
+    const int cg = split_ctas(plan, sh.ntiles, sh.ntiles);
+    const int64_t tile = warp * cg + cu;
+    if (cu < cg && tile < sh.ntiles) {
+      const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+      const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
+      if (slot >= 0) {
+        prefetch_l2(cache.ktile + slot * (kb / 4), kb);
+        prefetch_l2(cache.vtile + slot * (vb / 4), vb);
+        prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
+        prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
+      }
+    }
+  }
+  // Launched as a programmatic dependent of the previous kernel (the
+  // appends of a decode step, or the previous call): the query, the lengths
+  // and the cache are read after it has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- 2. the unit's range, split and tiles ----
+  const SeqRange sr = seq_range(sh, seq_lens, BufferArgs{}, b);
+  if (sr.bad && blockIdx.y == 0 && tid == 0 && h == 0 && hb == 0) atomicOr(ws.err, kErrSeqLen);
+  const int len = sr.len, lo = sr.lo;
+  const int tlo = lo / kTile;
+  const int ntl = static_cast<int>(range_tiles(sr));
+  __shared__ int64_t s_red[kDecWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kDecThreads>(sh, seq_lens, BufferArgs{}, batch, s_red);
+  const int C = split_ctas(plan, ntl, total);  // a multiple of the cluster size
+  const size_t qrow0 = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0;
+  const size_t wrow0 = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0;
+  if (C == 0) {
+    // no packed position: the first cluster writes zero outputs
+    if (clu == 0 && rank < nh) out[(qrow0 + rank) * kD + tid] = __float2half(0.f);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  if (cu >= C) {  // a whole cluster the unit does not use
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  const int nclu = C / kFusedCluster;
+  const int W = C * kDecWarps;
+  const int wu = warp * C + cu;
+  const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
+  TileSource src;
+  src.sh = sh;
+  src.cache = cache;
+  src.err = ws.err;
+  src.layer = layer;
+  src.b = b;
+  src.h = h;
+  src.tlo = tlo;
+  src.wu = wu;
+  src.W = W;
+  src.kwords = 256 * sh.kbits;
+  src.vwords = 256 * VB;
+  src.stage = stage_base + static_cast<size_t>(warp) * FL.stage_bytes;
+  src.stage_stride = kDecWarps * FL.stage_bytes;
+  src.bars = bars + warp * kStages;
+  src.stage_bytes = FL.stage_bytes;
+  // the first tile of each warp goes out now (its stage does not hold the
+  // rotation scratch); the second after the fragments are built
+  if (lane == 0 && my_tiles > 0) issue_tile(src, 0);
+
+  // ---- q~ for coordinates [16 rank, 16 rank + 16) of the block's heads ----
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh)
+    qr[hh * kRowPad + tid] = hh < nh ? __half2float(q[(qrow0 + hh) * kD + perm_j]) : 0.f;
+  __syncthreads();
+  {
+    const int hh = tid >> 4, o = tid & 15;
+    const int i = 16 * rank + o;
+    float v = 0.f;
+    if (i < lay.n_positions) {
+      int g = 0;
+      for (int t = 1; t < ng; ++t)
+        if (i >= lay.start[t]) g = t;
+      const int j0 = lay.start[g], j1 = j0 + lay.size[g];
+      const float* rrow = rk + o * kRowPad;
+      const float* qrow = qr + hh * kRowPad;
+      float a0 = 0.f, a1 = 0.f;
+      int j = j0;
+      for (; j + 1 < j1; j += 2) {
+        a0 = fmaf(rrow[j], qrow[j], a0);
+        a1 = fmaf(rrow[j + 1], qrow[j + 1], a1);
+      }
+      if (j < j1) a0 = fmaf(rrow[j], qrow[j], a0);
+      v = (a0 + a1) * (kInvSqrtD * lay.inv_sqrt_d[g]);
+    }
+#pragma unroll
+    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st(dsmem_addr(qt + hh * kRowPad + i, r2), v);
+  }
+  cluster_sync_all();
+  // the B fragments from q~ (see write_frags for the layout); heads past nh are zero
+  {
+    const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+    for (int u = tid; u < 32 * nchunk; u += kDecThreads) {
+      const int c = u >> 5, ln = u & 31;
+      int g = 0;
+      while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
+      const int j = c - lay.chunk_base[g];
+      const int d = lay.size[g], st = lay.start[g];
+      const int head = ln >> 2;
+      float v[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int coord = 16 * j + 4 * (ln & 3) + m;
+        v[m] = coord < d ? qt[head * kRowPad + st + coord] * kLog2e : 0.f;
+      }
+      const __half2 a = __floats2half2_rn(v[0], v[1]);
+      const __half2 c2 = __floats2half2_rn(v[2], v[3]);
+      const float2 af = __half22float2(a), cf = __half22float2(c2);
+      const __half2 al = __floats2half2_rn(v[0] - af.x, v[1] - af.y);
+      const __half2 cl = __floats2half2_rn(v[2] - cf.x, v[3] - cf.y);
+      bq[u] = make_uint4(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&c2),
+                         *reinterpret_cast<const uint32_t*>(&al), *reinterpret_cast<const uint32_t*>(&cl));
+    }
+  }
+  ByteTab tv;
+  {
+    const uint4 a0 = *reinterpret_cast<const uint4*>(tabv);
+    const uint4 a1 = *reinterpret_cast<const uint4*>(tabv + 4);
+    tv.lo[0] = a0.x; tv.lo[1] = a0.y; tv.lo[2] = a0.z; tv.lo[3] = a0.w;
+    tv.hi[0] = a1.x; tv.hi[1] = a1.y; tv.hi[2] = a1.z; tv.hi[3] = a1.w;
+  }
+  __syncthreads();  // fragments ready; the rotation scratch (second stages) is free
+  if (lane == 0 && my_tiles > 1) issue_tile(src, 1);
+
+  // ---- 3. the tiles, then the CTA's warps merged ----
+  TileTables tt{grp, tabk, pdesc, bq, ng};
+  float O[8][4], m_run[2], l_run[2];
+  const int failed_at = attend_tiles<VB>(src, tt, tv, my_tiles, len, lo, O, m_run, l_run);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  float* cacc = reinterpret_cast<float*>(stage_base);  // [8][kD]
+  merge_warps(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, cm, cm + 8, cacc,
+              nh);
+  cluster_sync_all();
+
+  // ---- 4. cluster merge: CTA rank r takes head r over the cluster's CTAs ----
+  if (rank < nh) {
+    float mr[kFusedCluster], wr[kFusedCluster];
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int c = 0; c < kFusedCluster; ++c) {
+      mr[c] = dsmem_ld(dsmem_addr(cm + rank, c));
+      M = fmaxf(M, mr[c]);
+    }
+    float Lsum = 0.f, a = 0.f;
+#pragma unroll
+    for (int c = 0; c < kFusedCluster; ++c) {
+      wr[c] = mr[c] == -CUDART_INF_F ? 0.f : fast_exp2(mr[c] - M);
+      Lsum = fmaf(wr[c], dsmem_ld(dsmem_addr(cm + 8 + rank, c)), Lsum);
+      a = fmaf(wr[c], dsmem_ld(dsmem_addr(cacc + rank * kD + tid, c)), a);
+    }
+    float* part = ws.partials + ((wrow0 + rank) * sh.max_splits + clu) * kPartialStride;
+    part[4 + tid] = a;
+    if (tid == 0) {
+      part[0] = M;
+      part[1] = Lsum;
+    }
+    __threadfence();
+  }
+  cluster_sync_all();  // remote reads done; the cluster's partials are written
+  if (tid == 0 && rank == 0) {
+    const uint32_t last = atomicAdd(ws.comb_count + wrow0, 1u) == static_cast<uint32_t>(nclu - 1) ? 1u : 0u;
+#pragma unroll
+    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st_u32(dsmem_addr(flag, r2), last);
+  }
+  cluster_sync_all();
+  if (*flag == 0u) return;  // the same for the whole cluster
+
+  // ---- 5. the unit's last cluster: merge the clusters, rotate back ----
+  __threadfence();
+  if (rank < nh) {
+    const float* part = ws.partials + (wrow0 + rank) * sh.max_splits * kPartialStride;
+    float M = -CUDART_INF_F;
+    for (int c = 0; c < nclu; ++c) M = fmaxf(M, __ldcg(part + c * kPartialStride));
+    float Lsum = 0.f, a = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < nclu; ++c) {
+      const float mc = __ldcg(part + c * kPartialStride);
+      const float w = mc == -CUDART_INF_F ? 0.f : exp2f(mc - M);
+      Lsum = fmaf(w, __ldcg(part + c * kPartialStride + 1), Lsum);
+      a = fmaf(w, __ldcg(part + c * kPartialStride + 4 + tid), a);
+    }
+    const float an = a / Lsum;
+#pragma unroll
+    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st(dsmem_addr(qt + rank * kRowPad + tid, r2), an);
+  }
+  // columns [16 rank, 16 rank + 16) of R_V (row-major [in][out]): rv[o][i] = R_V[i][16 rank + o]
+  float* rv = rk;
+  {
+    const float* mv = ws.mv + static_cast<size_t>(lh) * kD * kD;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int f = tid + k * kDecThreads;
+      const int i = f >> 2, q4 = f & 3;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(mv + i * kD + 16 * rank + 4 * q4));
+      rv[(4 * q4 + 0) * kRowPad + i] = v.x;
+      rv[(4 * q4 + 1) * kRowPad + i] = v.y;
+      rv[(4 * q4 + 2) * kRowPad + i] = v.z;
+      rv[(4 * q4 + 3) * kRowPad + i] = v.w;
+    }
+  }
+  if (tid == 0 && rank == 0) ws.comb_count[wrow0] = 0u;  // ready for the next call
+  cluster_sync_all();
+  {
+    const int hh = tid >> 4, o = tid & 15;
+    if (hh < nh) {
+      const float* rrow = rv + o * kRowPad;
+      const float* arow = qt + hh * kRowPad;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < kD; i += 2) {
+        s0 = fmaf(rrow[i], arow[i], s0);
+        s1 = fmaf(rrow[i + 1], arow[i + 1], s1);
+      }
+      out[(qrow0 + hh) * kD + 16 * rank + o] = __float2half(s0 + s1);
     }
   }
 }
@@ -913,7 +1378,80 @@ int ctas_per_sm_vb(const Shape& s) {
   return n;
 }
 
+template <int VB>
+cudaError_t fused_attr_once() {
+  static const cudaError_t attr = set_smem(decode_fused_kernel<VB>, fused_layout(4, VB).total);
+  return attr;
+}
+
+template <int VB>
+cudaError_t launch_fused_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                            const __half* q, const int32_t* seq_lens, int batch, const SplitPlan& plan, __half* out,
+                            cudaStream_t stream) {
+  const cudaError_t attr = fused_attr_once<VB>();
+  if (attr != cudaSuccess) return attr;
+  const int head_blocks = (s.group + 7) / 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch * s.n_kv_heads * head_blocks, plan.c_max, layer_count);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB).total;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = 1;
+  at[1].val.clusterDim.y = kFusedCluster;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<VB>, s, ws, cache, layer0, q, seq_lens, batch, plan,
+                            head_blocks, out);
+}
+
+template <int VB>
+int fused_clusters_vb(const Shape& s) {
+  if (fused_attr_once<VB>() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, kFusedCluster, 1);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB).total;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = kFusedCluster;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_fused_kernel<VB>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 }  // namespace
+
+int decode_fused_clusters(const Shape& s) {
+  switch (s.vbits) {
+    case 1: return fused_clusters_vb<1>(s);
+    case 2: return fused_clusters_vb<2>(s);
+    case 3: return fused_clusters_vb<3>(s);
+    default: return fused_clusters_vb<4>(s);
+  }
+}
+
+cudaError_t launch_decode_fused(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const __half* q, const int32_t* seq_lens, int batch,
+                                const SplitPlan& plan, __half* out, cudaStream_t stream) {
+  switch (s.vbits) {
+    case 1: return launch_fused_vb<1>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+    case 2: return launch_fused_vb<2>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+    case 3: return launch_fused_vb<3>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+    default: return launch_fused_vb<4>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+  }
+}
 
 int decode_ctas_per_sm(const Shape& s) {
   switch (s.vbits) {

@@ -163,6 +163,8 @@ struct SplitPlan {
   int32_t budget;
   int32_t fixed_tiles;
   int32_t units_per_seq;  // layer_count * Hkv * head blocks
+  int32_t cluster;        // > 1: counts rounded up to whole clusters of this size (the fused decode)
+  int32_t pad;
 };
 
 // The split pass over the packed positions [pos_lo, seq_lens) (buf.pos_lo;
@@ -173,6 +175,17 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
                                 int batch, const SplitPlan& plan, cudaStream_t stream);
 // Resident split-decode CTAs per SM for a config (0 on error).
 int decode_ctas_per_sm(const Shape& s);
+// The fused decode (query rotation, split-K pass, merge and inverse V
+// rotation in one launch, in clusters of 8 CTAs): q fp16
+// [layer_count][batch][Hq][128], out fp16 of the same shape; the plan's
+// c_max and cluster must be multiples of / equal to 8.  Partials, one per
+// cluster, and the per-unit arrival counters (zero between calls) are in
+// the workspace.
+cudaError_t launch_decode_fused(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
+                                int layer_count, const __half* q, const int32_t* seq_lens, int batch,
+                                const SplitPlan& plan, __half* out, cudaStream_t stream);
+// Co-resident 8-CTA clusters of the fused decode for a config (0: it cannot run).
+int decode_fused_clusters(const Shape& s);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
                            __half* out, cudaStream_t stream);

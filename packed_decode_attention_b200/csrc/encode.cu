@@ -92,12 +92,17 @@ constexpr int kEncTilesPerCta = 8;  // tiles a CTA encodes with one load of its 
 // XOR-swizzled by j so that the transposed writes spread over the banks.
 __device__ __forceinline__ int xt_col(int j, int r) { return (((r >> 2) ^ ((j >> 3) & 15)) << 2) | (r & 3); }
 
-// The Lloyd-Max code of u for width w >= 1: the number of the 2^w - 1
-// ascending thresholds t[] that are <= u (ties go up), by binary search.
+// The stored symbol of u's Lloyd-Max code for width w >= 1.  The code is
+// the number of the 2^w - 1 ascending thresholds t[] that are <= u (ties go
+// up), found by binary search.  Widths 1..3 store the code; width 4 stores
+// it in sign-magnitude form (bit 3 = the level's sign, bits 0..2 = the rank
+// of |level| among the positive levels: c - 8 for c >= 8, 15 - c below), so
+// that the decode looks |level| up in an 8-entry table.
 __device__ __forceinline__ int lloyd_code(const float* t, int w, float u) {
   int c = 0;
   for (int s = 1 << (w - 1); s > 0; s >>= 1)
     if (t[c + s - 1] <= u) c += s;
+  if (w == 4) c = (c & 8) ? (c ^ 8) : (c ^ 15);
   return c;
 }
 

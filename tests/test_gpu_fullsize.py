@@ -107,26 +107,29 @@ def test_full_size_parity(dev, name):
     del rows
 
     seq = torch.tensor(lens, dtype=torch.int32, device=dev)
-    out_layer = torch.empty((w.n_layers, w.batch, w.n_q_heads, 128), dtype=torch.float16, device=dev)
-    for l in range(w.n_layers):
-        kv.decode_attn(l, q_all[l:l + 1], seq, out_layer[l:l + 1])
-    out_all = torch.empty_like(out_layer)
-    kv.decode_attn(0, q_all, seq, out_all, layer_count=w.n_layers)
-    # the benchmark's call (decode_step, here with no new row) is the same computation
-    out_step = torch.empty_like(out_layer)
-    for l in range(w.n_layers):
-        kv.decode_step(l, None, None, None, None, q_all[l:l + 1], seq, out_step[l:l + 1])
-    torch.cuda.synchronize()
-    assert kv.device_error() == 0
-    assert torch.equal(out_step, out_layer)
-    assert torch.isfinite(out_layer.float()).all() and torch.isfinite(out_all.float()).all()
-    a = out_layer.float().cpu().numpy()
-    assert np.all(row_rel_err(out_all.float().cpu().numpy(), a) <= REL_TOL)
     g = w.group
     qh = q_all.cpu().numpy()
-    for (l, b, h), enc in encs.items():
-        ref = model.decode(tb, l, h, qh[l, b, h * g:(h + 1) * g], enc["k_tiles"], enc["k_norms"], enc["v_tiles"],
-                           enc["v_norm"], enc["n"])
-        err = row_rel_err(a[l, b, h * g:(h + 1) * g], ref)
-        assert np.all(err <= REL_TOL), (name, l, b, h, err.max())
+    refs = {(l, b, h): model.decode(tb, l, h, qh[l, b, h * g:(h + 1) * g], enc["k_tiles"], enc["k_norms"],
+                                    enc["v_tiles"], enc["v_norm"], enc["n"]) for (l, b, h), enc in encs.items()}
+    # both decode paths: three launches (rotation, split pass, combine) and the fused launch
+    for path in (0, 1):
+        kv.set_decode_path(path)
+        out_layer = torch.empty((w.n_layers, w.batch, w.n_q_heads, 128), dtype=torch.float16, device=dev)
+        for l in range(w.n_layers):
+            kv.decode_attn(l, q_all[l:l + 1], seq, out_layer[l:l + 1])
+        out_all = torch.empty_like(out_layer)
+        kv.decode_attn(0, q_all, seq, out_all, layer_count=w.n_layers)
+        # the benchmark's call (decode_step, here with no new row) is the same computation
+        out_step = torch.empty_like(out_layer)
+        for l in range(w.n_layers):
+            kv.decode_step(l, None, None, None, None, q_all[l:l + 1], seq, out_step[l:l + 1])
+        torch.cuda.synchronize()
+        assert kv.device_error() == 0
+        assert torch.equal(out_step, out_layer), path
+        assert torch.isfinite(out_layer.float()).all() and torch.isfinite(out_all.float()).all()
+        a = out_layer.float().cpu().numpy()
+        assert np.all(row_rel_err(out_all.float().cpu().numpy(), a) <= REL_TOL), path
+        for (l, b, h), ref in refs.items():
+            err = row_rel_err(a[l, b, h * g:(h + 1) * g], ref)
+            assert np.all(err <= REL_TOL), (name, path, l, b, h, err.max())
     kv.close()

@@ -106,17 +106,19 @@ def test_paged_equals_contiguous(dev, kbits, vbits):
     # decode, all layers per call and one layer per call
     seq = torch.tensor(cur, dtype=torch.int32, device=dev)
     q = torch.stack([wl.decode_query(w, l, cur, device=dev) for l in range(w.n_layers)])
-    outs = []
-    for kv in (cont, paged):
-        o = torch.empty_like(q)
-        kv.decode_attn(0, q, seq, o, layer_count=w.n_layers)
-        o1 = torch.empty_like(q)
-        for l in range(w.n_layers):
-            kv.decode_attn(l, q[l:l + 1], seq, o1[l:l + 1])
-        outs.append((o, o1))
-    torch.cuda.synchronize()
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
-    assert torch.isfinite(outs[0][0].float()).all()
+    for path in (0, 1):  # three launches, then the fused launch
+        outs = []
+        for kv in (cont, paged):
+            kv.set_decode_path(path)
+            o = torch.empty_like(q)
+            kv.decode_attn(0, q, seq, o, layer_count=w.n_layers)
+            o1 = torch.empty_like(q)
+            for l in range(w.n_layers):
+                kv.decode_attn(l, q[l:l + 1], seq, o1[l:l + 1])
+            outs.append((o, o1))
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1]), path
+        assert torch.isfinite(outs[0][0].float()).all()
     # buffered decode: 4 sink rows and the last 32 positions as fp16 rows
     lo = torch.full((len(cur),), 4, dtype=torch.int32, device=dev)
     hi = torch.tensor([max(4, n - 32) for n in cur], dtype=torch.int32, device=dev)
@@ -177,16 +179,18 @@ def test_paged_decode_matches_oracle(dev):
             kv.k_norms()[0, h].view(pool, 64, 4)[pages.to(dev)] = kn.view(nt, 64, 4).to(dev)
             kv.v_norms()[0, h].view(pool, 64)[pages.to(dev)] = vn.view(nt, 64).to(dev)
     q = wl.decode_query(w, 0, lens)
-    out = torch.empty((1, len(lens), w.n_q_heads, 128), dtype=torch.float16, device=dev)
-    kv.decode_attn(0, q[None].to(dev), torch.tensor(lens, dtype=torch.int32, device=dev), out)
-    torch.cuda.synchronize()
-    assert kv.device_error() == 0
-    got = out[0].float().cpu().numpy()
     g = w.group
-    for (b, h), enc in encs.items():
-        ref = model.decode(tb, 0, h, q[b, h * g:(h + 1) * g].numpy(), enc["k_tiles"], enc["k_norms"],
-                           enc["v_tiles"], enc["v_norm"], lens[b])
-        assert np.all(row_rel_err(got[b, h * g:(h + 1) * g], ref) <= REL_TOL), (b, h)
+    for path in (0, 1):  # three launches, then the fused launch
+        kv.set_decode_path(path)
+        out = torch.empty((1, len(lens), w.n_q_heads, 128), dtype=torch.float16, device=dev)
+        kv.decode_attn(0, q[None].to(dev), torch.tensor(lens, dtype=torch.int32, device=dev), out)
+        torch.cuda.synchronize()
+        assert kv.device_error() == 0
+        got = out[0].float().cpu().numpy()
+        for (b, h), enc in encs.items():
+            ref = model.decode(tb, 0, h, q[b, h * g:(h + 1) * g].numpy(), enc["k_tiles"], enc["k_norms"],
+                               enc["v_tiles"], enc["v_norm"], lens[b])
+            assert np.all(row_rel_err(got[b, h * g:(h + 1) * g], ref) <= REL_TOL), (path, b, h)
     kv.close()
 
 

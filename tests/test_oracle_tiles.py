@@ -14,7 +14,18 @@ def test_quartet_golden(golden):
         assert [f"{w:08X}" for w in tiles.quartet_pack(sel, b)] == row[5:]
 
 
-def _selectors_k(codes_tile, start, d, j, lane):
+def _symbol(c, b):
+    """The stored symbol of code c at width b, from its definition: widths 1..3
+    store c; width 4 stores the sign of the level in bit 3 and the rank of
+    |level| among the positive levels in bits 0..2."""
+    if b != 4:
+        return int(c)
+    negative = c < 8
+    rank = (7 - c) if negative else (c - 8)     # C[c] = -C[15 - c]: |C[c]| = C[8 + rank]
+    return (8 if negative else 0) | rank
+
+
+def _selectors_k(codes_tile, start, d, j, lane, b):
     """Lane's four selector words for chunk j from the plain definition
     (nibbles whose coordinate is past the group are 0)."""
     out = []
@@ -23,7 +34,7 @@ def _selectors_k(codes_tile, start, d, j, lane):
         for n in range(8):
             token, coord = tiles._k_selector_member(mu, j, lane, n)
             if coord < d:
-                w |= int(codes_tile[token, start + coord]) << (4 * n)
+                w |= _symbol(codes_tile[token, start + coord], b) << (4 * n)
         out.append(w)
     return out
 
@@ -50,7 +61,7 @@ def test_k_tile_quartets_match_the_plane_formulas(widths_seed):
         d = len(d)
         for j in range(d // 16):
             for lane in range(32):
-                expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, lane), b)
+                expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, lane, b), b)
                 got = [int(words[off + 32 * k + lane]) for k in range(b)]
                 assert got == expect, (b, d, j, lane)
             off += 32 * b
@@ -60,14 +71,14 @@ def test_k_tile_quartets_match_the_plane_formulas(widths_seed):
             nf = r // 4
             for g in range(8):
                 for t in range(nf):
-                    expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, 4 * g + t), b)
+                    expect = tiles.quartet_pack(_selectors_k(codes, start, d, j, 4 * g + t, b), b)
                     got = [int(words[off + 8 * nf * k + g * nf + t]) for k in range(b)]
                     assert got == expect, ("partial full lane", b, d, g, t)
             if r % 4:
                 for v in range(4):
                     halves = []
                     for g in (2 * v, 2 * v + 1):
-                        sel = _selectors_k(codes, start, d, j, 4 * g + nf)       # padding nibbles are 0
+                        sel = _selectors_k(codes, start, d, j, 4 * g + nf, b)       # padding nibbles are 0
                         halves.append([(w & 0xFF) | ((w >> 8) & 0xFF00) for w in sel])
                     virt = [halves[0][mu] | (halves[1][mu] << 16) for mu in range(4)]
                     got = [int(words[off + 8 * nf * b + 4 * k + v]) for k in range(b)]
@@ -125,3 +136,35 @@ def test_every_code_bit_stored_once():
     keys = set(zip(tok.tolist(), pos.tolist(), cb.tolist()))
     assert len(keys) == len(tok) == 64 * int(widths.sum())
     assert all(c < widths[p] for _, p, c in keys)
+
+
+def test_width4_symbols_stand_for_their_levels():
+    """Symbol s of a width-4 code is the level's sign (bit 3) and the rank of
+    |level| (bits 0..2): the stored symbol maps every code to a distinct
+    symbol, the inverse undoes it, and with the binary16 Lloyd-Max table the
+    level read back by sign and magnitude is the code's own level."""
+    from oracle import lloyd_max as lm
+    c16, _ = lm.codebook_fp16(4)
+    codes = np.arange(16)
+    sym = tiles.stored_symbol(codes, 4)
+    assert sorted(sym.tolist()) == list(range(16))
+    assert np.array_equal(tiles.code_of_symbol(sym, 4), codes)
+    for c, s in zip(codes, sym):
+        assert s == _symbol(c, 4)
+        level = (-1.0 if s >= 8 else 1.0) * c16[8 + (s & 7)]
+        assert level == c16[c]
+    for b in (1, 2, 3):
+        assert np.array_equal(tiles.stored_symbol(np.arange(1 << b), b), np.arange(1 << b))
+
+
+def test_v_tile_width4_holds_symbols():
+    rng = np.random.default_rng(11)
+    vc = rng.integers(0, 16, size=(64, 128))
+    words = tiles.pack_v_tiles(vc, 4)[0].view("<u4")
+    m, lane = 3, 17
+    for kappa in range(4):
+        w = 0
+        for n in range(8):
+            token, coord = tiles._v_selector_member(m, kappa, lane, n)
+            w |= _symbol(vc[token, coord], 4) << (4 * n)
+        assert int(words[m * 128 + 32 * kappa + lane]) == w

@@ -34,7 +34,10 @@ def _filled_cache(w, dev, lens):
     return cfg, kv
 
 
-def test_static_scratch_decode_matches_decode_attn_twice():
+@pytest.mark.parametrize("path", [0, 1])
+def test_static_scratch_decode_matches_decode_attn_twice(path):
+    """path 0: the three-launch decode; 1: the fused launch (both keep their
+    scratch in the static array)."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
     dev = torch.device("cuda:0")
@@ -42,6 +45,7 @@ def test_static_scratch_decode_matches_decode_attn_twice():
                   n_calib=128)
     lens = [3000, 1234]
     cfg, kv = _filled_cache(w, dev, lens)
+    kv.set_decode_path(path)
     seq = torch.tensor(lens, dtype=torch.int32, device=dev)
     for call, layer in enumerate((0, 1)):
         q = wl.decode_query(w, layer, lens)[None].to(dev)

@@ -27,6 +27,7 @@ struct bgtq_state {
   int split_tokens = 0;  // 0 = automatic
   int ctas_per_sm = 0;   // resident decode CTAs per SM (looked up on first use)
   int fused_clusters = -1;  // co-resident clusters of the fused decode (looked up on first use; 0: not usable)
+  int fused_cluster_size = 8;
   int decode_mode = 0;      // 1: the fused decode where the GPU can run it; 0: rotation + split + combine
   int num_sms = 148;
   int device = -1;       // the CUDA device current at bgtq_create: its buffers live there
@@ -295,11 +296,16 @@ int split_slots(bgtq_state* st) {
 // CTAs of the fused decode the GPU holds at once (whole 8-CTA clusters); 0
 // when it cannot run, and the decode calls then use the split pass and the
 // combine.
-constexpr int kFusedCluster = 8;
-
+// The cluster size (4 or 8 CTAs) whose one wave holds the most CTAs, the
+// larger on a tie; looked up once per state.
 int fused_slots(bgtq_state* st) {
-  if (st->fused_clusters < 0) st->fused_clusters = std::max(0, bgtq::decode_fused_clusters(st->shape));
-  return st->fused_clusters * kFusedCluster;
+  if (st->fused_clusters < 0) {
+    const int c8 = std::max(0, bgtq::decode_fused_clusters(st->shape, 8));
+    const int c4 = std::max(0, bgtq::decode_fused_clusters(st->shape, 4));
+    st->fused_cluster_size = 4 * c4 > 8 * c8 ? 4 : 8;
+    st->fused_clusters = st->fused_cluster_size == 4 ? c4 : c8;
+  }
+  return st->fused_clusters * st->fused_cluster_size;
 }
 
 // Whether the decode calls take the fused launch: requested and possible.
@@ -310,7 +316,8 @@ bool use_fused(bgtq_state* st) { return st->decode_mode == 1 && fused_slots(st) 
 // automatic plan spreads one wave of clusters over the units, at least one
 // each).
 bgtq::SplitPlan fused_plan(bgtq_state* st, int32_t layer_count, int32_t batch) {
-  const int cl = kFusedCluster;
+  fused_slots(st);
+  const int cl = st->fused_cluster_size;
   auto up = [cl](int64_t x) { return (x + cl - 1) / cl * cl; };
   const int head_blocks = (st->shape.group + 7) / 8;
   bgtq::SplitPlan p{};
@@ -409,6 +416,7 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) st->num_sms = sms;
   }
+  st->shape.n_sms = st->num_sms;
   bgtq::CodebookDev cb;
   std::memset(&cb, 0, sizeof(cb));
   for (int b = 1; b <= 4; ++b) {
@@ -890,7 +898,7 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   if (use_fused(st)) {
     // the fused decode: the arrival counters, then one partial per cluster
     const bgtq::SplitPlan plan = fused_plan(st, layer_count, batch);
-    const int64_t nclu = plan.c_max / kFusedCluster;
+    const int64_t nclu = plan.c_max / plan.cluster;
     const size_t part_bytes = rows * size_t(nclu) * bgtq::kPartialStride * sizeof(float);
     if (rows * sizeof(uint32_t) > kStaticCountBytes || kStaticCountBytes + part_bytes > BGTQ_STATIC_SCRATCH_BYTES)
       return BGTQ_ERR_BUFFER_SIZE;

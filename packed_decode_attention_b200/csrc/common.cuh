@@ -86,10 +86,11 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Byte tables of the fp16 codebook: lo[i] / hi[i] hold the low / high bytes
+// Byte tables of the fp16 codebook (8 entries: the levels of widths 1..3,
+// the positive levels of width 4): lo[i] / hi[i] hold the low / high bytes
 // of entries 4i .. 4i+3.
 struct ByteTab {
-  uint32_t lo[4], hi[4];
+  uint32_t lo[2], hi[2];
 };
 
 // Four symbols (selector nibbles 0..3) -> two fp16x2 registers: symbols

@@ -36,8 +36,12 @@ namespace {
 // operand with movmatrix.  Everything stays in V's rotated basis; the
 // combine kernel rotates back.
 // ---------------------------------------------------------------------------
+// Per warp: two stages for the K tile and the norms, one buffer for the V
+// tile (refilled as soon as the previous tile's P V is done: the next
+// tile's logits and softmax cover its copy).
 constexpr int kStages = 2;
-constexpr int kDecMinBlocks = 3;  // CTAs per SM the register budget is sized for
+constexpr int kBarsPerWarp = kStages + 1;
+constexpr int kDecMinBlocks = 4;  // CTAs per SM the register budget is sized for
 constexpr int kWaitLimit = 1 << 20;  // polls of up to kPollSuspendNs each: about a second
 constexpr float kRescaleSlack = 8.f;
 
@@ -65,6 +69,30 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// Before the dependency wait of a one-sequence call: an L2 prefetch hint for
+// the first kPrefetchTiles tiles the warp would get if the sequence were
+// full (lane k takes the warp's k-th tile), so that the cache streams into
+// L2 while the previous kernel finishes.  A prefetch reads nothing into the
+// CTA and leaves memory as it is: L2 is where global memory is coherent, so
+// a line a later kernel rewrites is read afresh by the copies after the
+// wait, and a line the sequence does not reach costs only bandwidth.
+constexpr int kPrefetchTiles = 4;
+
+__device__ __forceinline__ void prefetch_warp_tiles(const Shape& sh, const CacheDev& cache, int layer, int b, int h,
+                                                    int c_full, int warp, int nw, int cu, int kbits, int vbits) {
+  const int lane = threadIdx.x & 31;
+  if (cu >= c_full || lane >= kPrefetchTiles) return;
+  const int64_t tile = warp * c_full + cu + static_cast<int64_t>(lane) * c_full * nw;
+  if (tile >= sh.ntiles) return;
+  const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+  if (slot < 0) return;
+  const uint32_t kb = 1024u * kbits, vb = 1024u * vbits;
+  prefetch_l2(cache.ktile + slot * (kb / 4), kb);
+  prefetch_l2(cache.vtile + slot * (vb / 4), vb);
+  prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
+  prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
+}
+
 // One bounded poll: the thread may sleep up to kPollSuspendNs waiting for the phase.
 constexpr uint32_t kPollSuspendNs = 1000;
 
@@ -89,24 +117,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 constexpr int kBufSmemBytes = (8 * kD + 8 * kMaxBufferRows + 16) * 4;
 
 struct DecodeLayout {  // byte offsets inside the dynamic shared memory
-  int bars, bq, tabk, grp, pdesc, ms, ls, mres, wsc, stage, stage_bytes, total;
+  int bars, bq, tabk, grp, pdesc, ms, ls, mres, wsc, stage, kst_bytes, v_bytes, total;
 };
 
-__host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits) {
+// The stage region of a CTA of nw warps: K stage s of warp w at stage +
+// (s * nw + w) * kst_bytes (K tile, K norms, V norms), then warp w's V
+// buffer at stage + kStages * nw * kst_bytes + w * v_bytes.
+__host__ __device__ inline DecodeLayout decode_layout(int kbits, int vbits, int nw) {
   DecodeLayout L;
   L.bars = 0;
-  L.bq = align128(kDecWarps * kStages * 8);
+  L.bq = align128(nw * kBarsPerWarp * 8);
   L.grp = L.bq + kMaxChunks * 32 * 16;    // a copy of DecodeTableDev: grp, tabk, pdesc, tabv
   L.tabk = L.grp + kNumGroupsMax * 8 * 4;
   L.pdesc = L.tabk + kNumGroupsMax * 8 * 4;
   L.ms = L.grp + static_cast<int>(sizeof(DecodeTableDev));
-  L.ls = L.ms + kDecWarps * 8 * 4;
-  L.mres = L.ls + kDecWarps * 8 * 4;           // merged m, l per head [2][8]
-  L.wsc = L.mres + 2 * 8 * 4;                  // merge weights [warp][8]
-  L.stage = align128(L.wsc + kDecWarps * 8 * 4);
-  L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
-  const int stages = kDecWarps * kStages * L.stage_bytes;
-  const int merge = kDecWarps * 8 * kD * 4;  // reuses the stage buffers after the loop
+  L.ls = L.ms + nw * 8 * 4;
+  L.mres = L.ls + nw * 8 * 4;           // merged m, l per head [2][8]
+  L.wsc = L.mres + 2 * 8 * 4;           // merge weights [warp][8]
+  L.stage = align128(L.wsc + nw * 8 * 4);
+  L.kst_bytes = 1024 * kbits + kTile * 8 + kTile * 2;
+  L.v_bytes = 1024 * vbits;
+  const int stages = nw * (kStages * L.kst_bytes + L.v_bytes);
+  const int merge = nw * 8 * kD * 4;  // reuses the stage buffers after the loop
   int need = stages > merge ? stages : merge;
   if (need < kBufSmemBytes) need = kBufSmemBytes;  // the buffer CTA of a buffered call
   L.total = L.stage + need;
@@ -182,8 +214,11 @@ __device__ int64_t batch_tiles(const Shape& sh, const int32_t* seq_lens, const B
 // q . k / sqrt(D) in log2 units (a thread per row), softmax per head, P v (a
 // thread per dimension, unrotated).  Each head's (m, l, acc) goes to the
 // row's extra combine intermediate, which then counts as arrived.
+// NT threads (128 or more): the P v part runs on the first 128.
+template <int NT>
 __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const BufferArgs& buf, const SeqRange& sr, int li,
                               int b, int h, int h0, int nh, int batch, unsigned char* smem) {
+  static_assert(NT >= kD && NT % 32 == 0, "at least a thread per dimension");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = sh.group;
   float* qs = reinterpret_cast<float*>(smem);   // [128 dims][8 heads]
@@ -191,14 +226,14 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   float* ml = lg + 8 * kMaxBufferRows;          // [8][2]
   const int cnt = sr.cnt;
   const size_t qrow = ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
-  for (int i = tid; i < 8 * kD; i += kDecThreads) {
+  for (int i = tid; i < 8 * kD; i += NT) {
     const int hh = i / kD, dim = i % kD;
     qs[dim * 8 + hh] = hh < nh ? __half2float(buf.q[qrow + i]) * (kInvSqrtD * kLog2e) : 0.f;
   }
   __syncthreads();
   const size_t rstride = static_cast<size_t>(sh.n_kv_heads) * kD;
   const size_t base = (static_cast<size_t>(li) * batch + b) * buf.n_buf * rstride + static_cast<size_t>(h) * kD;
-  for (int r = tid; r < cnt; r += kDecThreads) {
+  for (int r = tid; r < cnt; r += NT) {
     const uint4* kr = reinterpret_cast<const uint4*>(buf.k + base + r * rstride);
     float d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     // half of the row's dimensions per pass: 8 loads of 8 values in flight
@@ -231,7 +266,7 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   }
   __syncthreads();
   // per head: maximum, weights 2^(logit - M) in place, denominator
-  for (int hh = warp; hh < 8; hh += kDecWarps) {
+  for (int hh = warp; hh < 8; hh += NT / 32) {
     float M = -CUDART_INF_F;
     for (int r = lane; r < cnt; r += 32) M = fmaxf(M, lg[hh * kMaxBufferRows + r]);
 #pragma unroll
@@ -253,13 +288,14 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   // P v: thread (8 dimensions dg, row phase rp of 8), 8 values per load; the
   // phases are then summed through shared memory (over the weights)
   const int dg = tid & 15, rp = tid >> 4;
+  const int rend = tid < kD ? cnt : 0;  // threads past the first 128 take no rows
   float acc[8][8];
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
 #pragma unroll 4
-  for (int r = rp; r < cnt; r += 8) {
+  for (int r = rp; r < rend; r += 8) {
     const uint4 vw = *reinterpret_cast<const uint4*>(buf.v + base + r * rstride + 8 * dg);
     const __half2* h2 = reinterpret_cast<const __half2*>(&vw);
     float vv[8];
@@ -278,18 +314,20 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
   }
   __syncthreads();
   float* red = lg;  // [8 phases][8 heads][128 dims]
+  if (tid < kD) {
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh) {
-    float4* dst = reinterpret_cast<float4*>(red + (rp * 8 + hh) * kD + 8 * dg);
-    dst[0] = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
-    dst[1] = make_float4(acc[hh][4], acc[hh][5], acc[hh][6], acc[hh][7]);
+    for (int hh = 0; hh < 8; ++hh) {
+      float4* dst = reinterpret_cast<float4*>(red + (rp * 8 + hh) * kD + 8 * dg);
+      dst[0] = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+      dst[1] = make_float4(acc[hh][4], acc[hh][5], acc[hh][6], acc[hh][7]);
+    }
   }
   __syncthreads();
-  const int d = tid;  // kDecThreads == kD: a thread per output dimension
+  const int d = tid;  // the first 128 threads: a thread per output dimension
   const size_t wrow0 = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0;
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) {
-    if (hh >= nh) break;
+    if (hh >= nh || d >= kD) break;
     float* mid = ws.comb_mid + ((wrow0 + hh) * (kCombSlices + 1) + kCombSlices) * kPartialStride;
     float a = 0.f;
 #pragma unroll
@@ -323,36 +361,56 @@ struct TileSource {
   int layer, b, h;
   int tlo, wu, W;        // the warp's first tile is tlo + wu, then every W-th
   int kwords, vwords;    // 32-bit words of a K / V tile
-  unsigned char* stage;  // this warp's first stage buffer; stage k at stage + k * stage_stride
-  int stage_stride;
-  uint64_t* bars;        // the stages' mbarriers
-  int stage_bytes;
+  unsigned char* kstage; // this warp's K stage 0; stage s at kstage + s * kstride
+  int kstride;
+  unsigned char* vbuf;   // this warp's V buffer
+  uint64_t* bars;        // the K stages' mbarriers, then the V buffer's
 };
 
-// Lane 0: copy the warp's k-th tile into stage k % kStages.
-__device__ __forceinline__ void issue_tile(const TileSource& src, int k) {
-  const uint32_t kbytes = 4u * src.kwords, vbytes = 4u * src.vwords;
-  const uint32_t stage_tx = kbytes + vbytes + kTile * 8 + kTile * 2;
-  const int tile = src.tlo + src.wu + k * src.W;
-  uint64_t* bar = &src.bars[k % kStages];
-  if (tile == src.sh.drop_tile) {
-    // test hook: the copy is never issued, so the wait on it runs out
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(bar, stage_tx);
-    return;
-  }
+__device__ __forceinline__ int64_t source_slot(const TileSource& src, int tile) {
   int64_t slot = tile_slot(src.sh, src.cache, src.layer, src.b, src.h, tile);
   if (slot < 0) {  // a page id outside the pool: flagged, page 0 read instead
     atomicOr(src.err, kErrPage);
     slot = static_cast<int64_t>(src.layer * src.sh.n_kv_heads + src.h) * src.cache.n_pages;
   }
-  unsigned char* dst = src.stage + (k % kStages) * src.stage_stride;
+  return slot;
+}
+
+// Lane 0: copy the K tile and the norms of the warp's k-th tile into K stage k % kStages.
+__device__ __forceinline__ void issue_k(const TileSource& src, int k) {
+  const uint32_t kbytes = 4u * src.kwords;
+  const uint32_t tx = kbytes + kTile * 8 + kTile * 2;
+  const int tile = src.tlo + src.wu + k * src.W;
+  uint64_t* bar = &src.bars[k % kStages];
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  mbar_expect_tx(bar, stage_tx);
+  mbar_expect_tx(bar, tx);
+  if (tile == src.sh.drop_tile) return;  // test hook: no copy, so the wait on it runs out
+  const int64_t slot = source_slot(src, tile);
+  unsigned char* dst = src.kstage + (k % kStages) * src.kstride;
   bulk_copy_g2s(dst, src.cache.ktile + slot * src.kwords, kbytes, bar);
-  bulk_copy_g2s(dst + kbytes, src.cache.vtile + slot * src.vwords, vbytes, bar);
-  bulk_copy_g2s(dst + kbytes + vbytes, src.cache.knorm + slot * kTile * 4, kTile * 8, bar);
-  bulk_copy_g2s(dst + kbytes + vbytes + kTile * 8, src.cache.vnorm + slot * kTile, kTile * 2, bar);
+  bulk_copy_g2s(dst + kbytes, src.cache.knorm + slot * kTile * 4, kTile * 8, bar);
+  bulk_copy_g2s(dst + kbytes + kTile * 8, src.cache.vnorm + slot * kTile, kTile * 2, bar);
+}
+
+// Lane 0: copy the V tile of the warp's k-th tile into its V buffer.
+__device__ __forceinline__ void issue_v(const TileSource& src, int k) {
+  const uint32_t vbytes = 4u * src.vwords;
+  const int tile = src.tlo + src.wu + k * src.W;
+  uint64_t* bar = &src.bars[kStages];
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  mbar_expect_tx(bar, vbytes);
+  if (tile == src.sh.drop_tile) return;
+  const int64_t slot = source_slot(src, tile);
+  bulk_copy_g2s(src.vbuf, src.cache.vtile + slot * src.vwords, vbytes, bar);
+}
+
+// Lane 0: the copies a warp starts with (K of its first two tiles, V of its first).
+__device__ __forceinline__ void issue_first(const TileSource& src, int my_tiles) {
+  if (my_tiles > 0) {
+    issue_k(src, 0);
+    issue_v(src, 0);
+  }
+  if (my_tiles > 1) issue_k(src, 1);
 }
 
 // The decode tables a warp reads from shared memory (a copy of the
@@ -365,16 +423,16 @@ struct TileTables {
   int ng;
 };
 
-// Attends the warp's my_tiles tiles over the positions [lo, len); the first
-// min(kStages, my_tiles) copies must already be issued.  Returns the index of
-// the tile whose copy wait gave up (-1: none).
+// Attends the warp's my_tiles tiles over the positions [lo, len); the copies
+// of issue_first must already be issued.  Returns the index of the tile
+// whose copy wait gave up (-1: none).
 template <int VB>
 __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTables& tt, const ByteTab& tv,
                                             int my_tiles, int len, int lo, float (&O)[8][4], float (&m_run)[2],
                                             float (&l_run)[2]) {
   const int lane = threadIdx.x & 31;
   const int g8 = lane >> 2;
-  const uint32_t kbytes = 4u * src.kwords, vbytes = 4u * src.vwords;
+  const uint32_t kbytes = 4u * src.kwords;
 #pragma unroll
   for (int m = 0; m < 8; ++m)
 #pragma unroll
@@ -382,17 +440,17 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
   m_run[0] = m_run[1] = -CUDART_INF_F;
   l_run[0] = l_run[1] = 0.f;
   int failed_at = -1;
+  bool k_consumed = false;  // at a failure: whether that tile's K stage had landed
 
   for (int k = 0; k < my_tiles; ++k) {
     if (!__all_sync(0xffffffffu, mbar_wait(&src.bars[k % kStages], (k / kStages) & 1))) {
       failed_at = k;
       break;
     }
-    const unsigned char* st = src.stage + (k % kStages) * src.stage_stride;
+    const unsigned char* st = src.kstage + (k % kStages) * src.kstride;
     const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
-    const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + kbytes);
-    const __half* kn = reinterpret_cast<const __half*>(st + kbytes + vbytes);
-    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + vbytes + kTile * 8);
+    const __half* kn = reinterpret_cast<const __half*>(st + kbytes);
+    const __half* vn = reinterpret_cast<const __half*>(st + kbytes + kTile * 8);
     const int tpos = (src.tlo + src.wu + k * src.W) * kTile;
     const int nvalid = min(kTile, len - tpos);       // positions [nlow, nvalid) of the tile are attended
     const int nlow = max(0, lo - tpos);
@@ -409,8 +467,8 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       ByteTab t;
       const uint4 tl = *reinterpret_cast<const uint4*>(tt.tabk + 8 * g);
       const uint4 th = *reinterpret_cast<const uint4*>(tt.tabk + 8 * g + 4);
-      t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
-      t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+      t.lo[0] = tl.x; t.lo[1] = tl.y;
+      t.hi[0] = th.x; t.hi[1] = th.y;
       const uint32_t pd = tt.pdesc[g * 32 + lane];
       const uint32_t* gw = kt + gp.w;
       const uint4* bqg = tt.bq + chunk * 32 + lane;
@@ -495,7 +553,13 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       bp[mu][0] = transpose8x8(pack_half2(p0 * wv[mu][0], p1 * wv[mu][0]));
       bp[mu][1] = transpose8x8(pack_half2(p2 * wv[mu][1], p3 * wv[mu][1]));
     }
-    // P V in V's rotated basis
+    // P V in V's rotated basis, from the V buffer
+    if (!__all_sync(0xffffffffu, mbar_wait(&src.bars[kStages], k & 1))) {
+      failed_at = k;
+      k_consumed = true;
+      break;
+    }
+    const uint32_t* vt = reinterpret_cast<const uint32_t*>(src.vbuf);
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       uint32_t w[VB], sv[4];
@@ -506,27 +570,35 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
     }
     __syncwarp();
-    if (lane == 0 && k + kStages < my_tiles) issue_tile(src, k + kStages);
+    if (lane == 0) {
+      if (k + 1 < my_tiles) issue_v(src, k + 1);
+      if (k + kStages < my_tiles) issue_k(src, k + kStages);
+    }
   }
   if (failed_at >= 0) {
     // copies issued but not yet consumed: let them land (bounded) before the
-    // stage buffers are reused or the CTA exits
+    // buffers are reused or the CTA exits.  At the failure at tile f the K
+    // stages of tiles up to f + 1 and the V buffer of tile f were issued.
     if (lane == 0) atomicOr(src.err, kErrTimeout);
-    const int issued = min(my_tiles, failed_at + kStages);
-    for (int k = failed_at; k < issued; ++k) mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
+    const int f = failed_at;
+    for (int k = k_consumed ? f + 1 : f; k < min(my_tiles, f + kStages); ++k)
+      mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
+    mbar_wait(&src.bars[kStages], f & 1);
   }
   return failed_at;
 }
 
-// Merges the CTA's warps (called by all threads after attend_tiles) into one
-// (m, l, acc[128]) per query head of the block: cm[8], clsum[8] and
+// Merges the CTA's NW warps (called by all threads after attend_tiles) into
+// one (m, l, acc[128]) per query head of the block: cm[8], clsum[8] and
 // cacc[8][128] (shared memory; cacc may alias the stage buffers, which are
-// free once every warp has left its loop).  accs: [kDecWarps][8][128] of
-// shared scratch (may alias the stage buffers too, not cacc); ms, ls:
-// [kDecWarps][8] each.  A CTA with a timed-out warp posts empty partials.
+// free once every warp has left its loop).  accs: [NW][8][128] of shared
+// scratch (may alias the stage buffers too, and cacc); ms, ls, wsc: [NW][8]
+// each.  A CTA with a timed-out warp posts empty partials.
+template <int NW>
 __device__ __forceinline__ void merge_warps(const float (&O)[8][4], const float (&m_run)[2], float (&l_run)[2],
                                             bool timed_out, float* accs, float* ms, float* ls, float* wsc, float* cm,
                                             float* clsum, float* cacc, int nh) {
+  constexpr int NT = NW * 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, t4 = lane & 3;
 #pragma unroll
@@ -553,16 +625,14 @@ __device__ __forceinline__ void merge_warps(const float (&O)[8][4], const float 
   // per head: the common maximum, the warps' weights (warps without a tile
   // hold m = -inf, l = 0, acc = 0) and the weighted denominator
   if (tid < 8 && cta_timed_out) {
-    for (int w = 0; w < kDecWarps; ++w) wsc[w * 8 + tid] = 0.f;
+    for (int w = 0; w < NW; ++w) wsc[w * 8 + tid] = 0.f;
     cm[tid] = -CUDART_INF_F;
     clsum[tid] = 0.f;
   } else if (tid < 8) {
     float M = -CUDART_INF_F;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, ms[w * 8 + tid]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, ms[w * 8 + tid]);
     float lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const float mw = ms[w * 8 + tid];
       const float sc = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
       wsc[w * 8 + tid] = sc;
@@ -572,21 +642,24 @@ __device__ __forceinline__ void merge_warps(const float (&O)[8][4], const float 
     clsum[tid] = lsum;
   }
   __syncthreads();
-  const int i = tid;  // kDecThreads == kD: a thread per dimension
-  float a[8];
+  // (head, dimension) pairs u = tid, tid + NT, ...
+  constexpr int kPer = 8 * kD / NT;
+  float a[kPer];
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh) {
-    a[hh] = 0.f;
+  for (int k = 0; k < kPer; ++k) {
+    const int u = tid + k * NT, hh = u / kD, i = u % kD;
+    a[k] = 0.f;
     if (hh < nh) {
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) a[hh] = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a[hh]);
+#pragma unroll 4
+      for (int w = 0; w < NW; ++w) a[k] = fmaf(wsc[w * 8 + hh], accs[(w * 8 + hh) * kD + i], a[k]);
     }
   }
   __syncthreads();  // cacc may alias accs
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh) cacc[hh * kD + i] = a[hh];
+  for (int k = 0; k < kPer; ++k) cacc[tid + k * NT] = a[k];
   __syncthreads();
 }
+
 // Grid (batch * Hkv * head_blocks, [1 buffer CTA +] plan.c_max, layer_count),
 // 128 threads.  A unit is one (layer, sequence, KV head, block of up to 8
 // query heads); it uses C = split_ctas(...) of its c_max split CTAs (more for
@@ -597,13 +670,14 @@ __device__ __forceinline__ void merge_warps(const float (&O)[8][4], const float 
 // partial round lands on as many CTAs as it can.  Each CTA writes one
 // partial (m, l, acc) per query head -- an empty one (m = -inf, l = 0) when
 // it has no tile.
-template <int VB>
-__global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
+template <int VB, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == kDecWarps ? kDecMinBlocks : 1)
     decode_mma_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const float* __restrict__ qrot,
                       const int32_t* __restrict__ seq_lens, BufferArgs buf, int batch, SplitPlan plan,
                       int head_blocks) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const DecodeLayout DL = decode_layout(sh.kbits, VB);
+  constexpr int NT = NW * 32;
+  const DecodeLayout DL = decode_layout(sh.kbits, VB, NW);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + DL.bars);
   uint4* bq = reinterpret_cast<uint4*>(smem_raw + DL.bq);
   uint32_t* tabk = reinterpret_cast<uint32_t*>(smem_raw + DL.tabk);
@@ -634,34 +708,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   {
     const uint4* src = reinterpret_cast<const uint4*>(ws.dectab + lh);
     uint4* dst = reinterpret_cast<uint4*>(grp);  // grp, tabk, pdesc, tabv are contiguous
-    for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += kDecThreads) dst[u] = src[u];
+    for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += NT) dst[u] = src[u];
   }
-  if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
+  if (tid < NW * kBarsPerWarp) mbar_init(&bars[tid], 1);
   __syncthreads();
   if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  // While the previous kernel may still run: an L2 prefetch hint for this
-  // warp's first tiles, taken as if the sequence were full (the length is an
-  // input, read only after the wait).  A prefetch reads nothing into the
-  // CTA and leaves memory as it is, so a stale or unused line costs only
-  // bandwidth; the copies below still read after the wait.
-  if (lane == 0 && batch == 1 && cu >= 0) {
-    // one sequence: its split count if it were full
-    const int cg = split_ctas(plan, sh.ntiles, sh.ntiles);
-    const int Wp = cg * kDecWarps;
-    const int wp = warp * cg + cu;
-    const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
-#pragma unroll
-    for (int k = 0; k < (cu < cg ? kStages : 0); ++k) {
-      const int64_t tile = wp + static_cast<int64_t>(k) * Wp;
-      if (tile >= sh.ntiles) break;
-      const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
-      if (slot < 0) break;
-      prefetch_l2(cache.ktile + slot * (kb / 4), kb);
-      prefetch_l2(cache.vtile + slot * (vb / 4), vb);
-      prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
-      prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
-    }
-  }
+  // While the previous kernel may still run: L2 prefetch hints for this
+  // warp's first tiles (the copies below still read after the wait)
+  if (batch == 1 && cu >= 0)
+    prefetch_warp_tiles(sh, cache, layer, b, h, split_ctas(plan, sh.ntiles, sh.ntiles), warp, NW, cu, sh.kbits, VB);
   // Launched as a programmatic dependent of the previous kernel (the query
   // rotation): everything above reads only the library's tables; the
   // sequence lengths, rotated queries and cache are read after that kernel
@@ -670,13 +725,13 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // the unit's q~ fragments (written by the query rotation): their loads go
   // out with the length reads below and land in shared memory further down
   const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
-  constexpr int kFragPerThread = (kFragEntries + kDecThreads - 1) / kDecThreads;
+  constexpr int kFragPerThread = (kFragEntries + NT - 1) / NT;
   uint4 fr[kFragPerThread];
   if (qrot == nullptr && cu >= 0) {
     const uint4* src = frag_block(sh, ws, li, b, h, hb);
 #pragma unroll
     for (int i = 0; i < kFragPerThread; ++i) {
-      const int u = tid + i * kDecThreads;
+      const int u = tid + i * NT;
       if (u < 32 * nchunk) fr[i] = src[u];
     }
   }
@@ -687,15 +742,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   if (cu < 0) {
     // the extra CTA of a buffered call: the unit's fp16 buffered rows
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    buffer_attend(sh, ws, buf, sr, li, b, h, h0, nh, batch, smem_raw + DL.stage);
+    buffer_attend<NT>(sh, ws, buf, sr, li, b, h, h0, nh, batch, smem_raw + DL.stage);
     return;
   }
   const int len = sr.len, lo = sr.lo;
   const int tlo = lo / kTile;
   const int ntl = static_cast<int>(range_tiles(sr));
   // this unit's split CTAs (the same count the combine computes)
-  __shared__ int64_t s_red[kDecWarps];
-  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kDecThreads>(sh, seq_lens, buf, batch, s_red);
+  __shared__ int64_t s_red[NW];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<NT>(sh, seq_lens, buf, batch, s_red);
   const int C = split_ctas(plan, ntl, total);
   if (cu >= C) {
     // not needed for this unit (its partials are slots 0 .. C-1)
@@ -705,7 +760,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   // Tile t of the unit goes to warp (t mod W) / C of CTA (t mod W) mod C:
   // a partial last round of tiles is spread over all CTAs (and so over all
   // SMs) before any CTA gets a second one.
-  const int W = C * kDecWarps;
+  const int W = C * NW;
   const int wu = warp * C + cu;
   const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
   float* part_base = ws.partials +
@@ -716,7 +771,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     if (qrot == nullptr) {
 #pragma unroll
       for (int i = 0; i < kFragPerThread; ++i) {
-        const int u = tid + i * kDecThreads;
+        const int u = tid + i * NT;
         if (u < 32 * nchunk) bq[u] = fr[i];
       }
     } else {
@@ -724,7 +779,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
       // (fp32, record order): coordinates 16 j + 4 t .. + 3 of chunk c's
       // group for head t / 4 ... see write_frags for the layout
       const float* qsrc = qrot + ((static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0) * kD;
-      for (int u = tid; u < 32 * nchunk; u += kDecThreads) {
+      for (int u = tid; u < 32 * nchunk; u += NT) {
         const int c = u >> 5, ln = u & 31;
         int g = 0;
         while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
@@ -751,8 +806,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   {
     const uint4 a0 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32);
     const uint4 a1 = *reinterpret_cast<const uint4*>(tabk + kNumGroupsMax * 8 + kNumGroupsMax * 32 + 4);
-    tv.lo[0] = a0.x; tv.lo[1] = a0.y; tv.lo[2] = a0.z; tv.lo[3] = a0.w;
-    tv.hi[0] = a1.x; tv.hi[1] = a1.y; tv.hi[2] = a1.z; tv.hi[3] = a1.w;
+    tv.lo[0] = a0.x; tv.lo[1] = a0.y;
+    tv.hi[0] = a1.x; tv.hi[1] = a1.y;
   }
   __syncthreads();
 
@@ -769,12 +824,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   src.W = W;
   src.kwords = 256 * sh.kbits;
   src.vwords = 256 * VB;
-  src.stage = stage_base + static_cast<size_t>(warp) * kStages * DL.stage_bytes;
-  src.stage_stride = DL.stage_bytes;
-  src.bars = bars + warp * kStages;
-  src.stage_bytes = DL.stage_bytes;
-  if (lane == 0)
-    for (int k = 0; k < kStages && k < my_tiles; ++k) issue_tile(src, k);
+  src.kstage = stage_base + static_cast<size_t>(warp) * DL.kst_bytes;
+  src.kstride = NW * DL.kst_bytes;
+  src.vbuf = stage_base + kStages * NW * DL.kst_bytes + static_cast<size_t>(warp) * DL.v_bytes;
+  src.bars = bars + warp * kBarsPerWarp;
+  if (lane == 0) issue_first(src, my_tiles);
   TileTables tt{grp, tabk, pdesc, bq, ng};
   float O[8][4], m_run[2], l_run[2];
   const int failed_at = attend_tiles<VB>(src, tt, tv, my_tiles, len, lo, O, m_run, l_run);
@@ -784,12 +838,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   float* cacc = reinterpret_cast<float*>(stage_base);
   float* wsc = reinterpret_cast<float*>(smem_raw + DL.wsc);
   float* mres = reinterpret_cast<float*>(smem_raw + DL.mres);
-  merge_warps(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, mres, mres + 8,
-              cacc, nh);
-  const int i = tid;
-  for (int hh = 0; hh < nh; ++hh) {
+  merge_warps<NW>(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, mres,
+                  mres + 8, cacc, nh);
+  for (int u = tid; u < nh * kD; u += NT) {
+    const int hh = u / kD, i = u % kD;
     float* part = part_base + hh * part_head_stride;
-    part[4 + i] = cacc[hh * kD + i];
+    part[4 + i] = cacc[u];
     if (i == 0) {
       part[0] = mres[hh];
       part[1] = mres[8 + hh];
@@ -802,7 +856,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // the inverse V rotation in one launch.
 //
 // Grid (batch * Hkv * head_blocks, plan.c_max, layer_count) in thread-block
-// clusters of kFusedCluster CTAs along y, 128 threads.  A unit (layer,
+// clusters of CL (4 or 8) CTAs along y, 128 threads.  A unit (layer,
 // sequence, KV head, block of up to 8 query heads) uses C = split_ctas(...)
 // of its c_max CTAs, a multiple of the cluster size (whole clusters; unused
 // clusters exit at once).  Its tiles are dealt over the 4 C warps exactly as
@@ -826,18 +880,18 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 // No CTA waits on another outside its cluster's hardware barriers, so the
 // grid needs no co-residency beyond the cluster's.
 // ---------------------------------------------------------------------------
-constexpr int kFusedCluster = 8;
 constexpr int kRowPad = kD + 1;  // row pitch (floats) of the rotation scratch: consecutive rows in different banks
-static_assert(kFusedCluster * 16 == kD, "each CTA of a cluster rotates 16 coordinates");
 
 struct FusedLayout {  // byte offsets inside the dynamic shared memory
-  int bars, bq, tab, ms, ls, wsc, cm, flag, qt, stage, stage_bytes, rot, total;
+  int bars, bq, tab, ms, ls, wsc, cm, flag, qt, stage, kst_bytes, v_bytes, rot, vbase, total;
 };
 
-__host__ __device__ inline FusedLayout fused_layout(int kbits, int vbits) {
+// CL = CTAs per cluster (4 or 8): CTA rank r rotates and writes back the
+// kD / CL coordinates [r kD / CL, (r + 1) kD / CL).
+__host__ __device__ inline FusedLayout fused_layout(int kbits, int vbits, int CL) {
   FusedLayout L;
   L.bars = 0;
-  L.bq = align128(kDecWarps * kStages * 8);
+  L.bq = align128(kDecWarps * kBarsPerWarp * 8);
   L.tab = L.bq + kMaxChunks * 32 * 16;
   L.ms = L.tab + static_cast<int>(sizeof(DecodeTableDev));
   L.ls = L.ms + kDecWarps * 8 * 4;
@@ -846,15 +900,20 @@ __host__ __device__ inline FusedLayout fused_layout(int kbits, int vbits) {
   L.flag = L.cm + 16 * 4;                      // "this cluster merges the unit" (written by rank 0)
   L.qt = align128(L.flag + 16);                // q~ [8][kRowPad] fp32, later the merged accumulators
   L.stage = align128(L.qt + 8 * kRowPad * 4);
-  L.stage_bytes = 1024 * (kbits + vbits) + kTile * 8 + kTile * 2;
-  // stage k of warp w at stage + (k * kDecWarps + w) * stage_bytes: the
-  // second stages form one block, which holds the K rotation rows [16][kRowPad]
-  // and the query rows [8][kRowPad] until the first tiles are in flight, and
-  // the inverse V rotation slice [16][kRowPad] in the last cluster's merge
-  L.rot = L.stage + kDecWarps * L.stage_bytes;
-  const int rot_bytes = (16 + 8) * kRowPad * 4;
-  int need = kDecWarps * kStages * L.stage_bytes;
-  if (need < kDecWarps * L.stage_bytes + rot_bytes) need = kDecWarps * L.stage_bytes + rot_bytes;
+  L.kst_bytes = 1024 * kbits + kTile * 8 + kTile * 2;
+  L.v_bytes = 1024 * vbits;
+  // K stage s of warp w at stage + (s * kDecWarps + w) * kst_bytes: the
+  // second K stages form one block, which holds the K rotation rows
+  // [kD / CL][kRowPad] and the query rows [8][kRowPad] until the first tiles
+  // are in flight, and the inverse V rotation slice [kD / CL][kRowPad] in
+  // the last cluster's merge; the V buffers follow (warp w at vbase + w *
+  // v_bytes)
+  L.rot = L.stage + kDecWarps * L.kst_bytes;
+  const int rot_bytes = (kD / CL + 8) * kRowPad * 4;
+  int kblock = kStages * kDecWarps * L.kst_bytes;
+  if (kblock < kDecWarps * L.kst_bytes + rot_bytes) kblock = kDecWarps * L.kst_bytes + rot_bytes;
+  L.vbase = L.stage + kblock;
+  int need = kblock + kDecWarps * L.v_bytes;
   const int merge = kDecWarps * 8 * kD * 4;  // the warp merge reuses the stage buffers
   if (need < merge) need = merge;
   L.total = L.stage + need;
@@ -887,13 +946,15 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int VB>
+template <int VB, int CL>
 __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     decode_fused_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0, const __half* __restrict__ q,
                         const int32_t* __restrict__ seq_lens, int batch, SplitPlan plan, int head_blocks,
                         __half* __restrict__ out) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const FusedLayout FL = fused_layout(sh.kbits, VB);
+  constexpr int CPR = kD / CL;  // coordinates (and output dims) per CTA rank
+  const FusedLayout FL = fused_layout(sh.kbits, VB, CL);
+  static_assert(kDecThreads == kD, "the fused decode's thread-per-dimension steps");
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + FL.bars);
   uint4* bq = reinterpret_cast<uint4*>(smem_raw + FL.bq);
   int32_t* grp = reinterpret_cast<int32_t*>(smem_raw + FL.tab);  // grp, tabk, pdesc, tabv are contiguous
@@ -907,13 +968,13 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   uint32_t* flag = reinterpret_cast<uint32_t*>(smem_raw + FL.flag);
   float* qt = reinterpret_cast<float*>(smem_raw + FL.qt);
   unsigned char* stage_base = smem_raw + FL.stage;
-  float* rk = reinterpret_cast<float*>(smem_raw + FL.rot);  // [16][kRowPad]
-  float* qr = rk + 16 * kRowPad;                              // [8][kRowPad]
+  float* rk = reinterpret_cast<float*>(smem_raw + FL.rot);  // [CPR][kRowPad]
+  float* qr = rk + CPR * kRowPad;                             // [8][kRowPad]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cu = blockIdx.y;
-  const int rank = cu % kFusedCluster;  // the CTA's rank in its cluster (clusters run along y)
-  const int clu = cu / kFusedCluster;
+  const int rank = cu % CL;  // the CTA's rank in its cluster (clusters run along y)
+  const int clu = cu / CL;
   const int hb = blockIdx.x % head_blocks;
   const int h = (blockIdx.x / head_blocks) % sh.n_kv_heads;
   const int b = blockIdx.x / (head_blocks * sh.n_kv_heads);
@@ -932,16 +993,17 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     uint4* dst = reinterpret_cast<uint4*>(grp);
     for (int u = tid; u < static_cast<int>(sizeof(DecodeTableDev) / 16); u += kDecThreads) dst[u] = src[u];
   }
-  if (tid < kDecWarps * kStages) mbar_init(&bars[tid], 1);
-  // rows [16 rank, 16 rank + 16) of the block-diagonal K rotation (record
-  // order): R[i][j] = mkt[j][i]
+  if (tid < kDecWarps * kBarsPerWarp) mbar_init(&bars[tid], 1);
+  // rows [CPR rank, CPR rank + CPR) of the block-diagonal K rotation
+  // (record order): R[i][j] = mkt[j][i]
   {
     const float* mk = ws.mkt + static_cast<size_t>(lh) * kD * kD;
+    constexpr int Q4 = CPR / 4;  // float4 per input row
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int f = tid + k * kDecThreads;  // 512 float4 = 128 inputs x 16 outputs
-      const int j = f >> 2, q4 = f & 3;
-      const float4 v = *reinterpret_cast<const float4*>(mk + j * kD + 16 * rank + 4 * q4);
+    for (int k = 0; k < CPR / 4; ++k) {
+      const int f = tid + k * kDecThreads;  // 128 inputs x CPR outputs
+      const int j = f / Q4, q4 = f % Q4;
+      const float4 v = *reinterpret_cast<const float4*>(mk + j * kD + CPR * rank + 4 * q4);
       rk[(4 * q4 + 0) * kRowPad + j] = v.x;
       rk[(4 * q4 + 1) * kRowPad + j] = v.y;
       rk[(4 * q4 + 2) * kRowPad + j] = v.z;
@@ -949,29 +1011,58 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     }
   }
   const int perm_j = lay.perm[tid] & (kD - 1);  // kDecThreads == kD: the original dim of record position tid
-  __syncthreads();
-  if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  if (lane == 0 && batch == 1) {
-    // L2 prefetch of this warp's first tile, as if the sequence were full
-    const int cg = split_ctas(plan, sh.ntiles, sh.ntiles);
-    const int64_t tile = warp * cg + cu;
-    if (cu < cg && tile < sh.ntiles) {
-      const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
-      const uint32_t kb = 1024u * sh.kbits, vb = 1024u * VB;
-      if (slot >= 0) {
-        prefetch_l2(cache.ktile + slot * (kb / 4), kb);
-        prefetch_l2(cache.vtile + slot * (vb / 4), vb);
-        prefetch_l2(cache.knorm + slot * kTile * 4, kTile * 8);
-        prefetch_l2(cache.vnorm + slot * kTile, kTile * 2);
-      }
+  // This thread's rotation output coordinate i = CPR rank + o (o = tid mod
+  // CPR; its heads are tid / CPR + 128 / CPR k): the group range [j0, j1)
+  // and scale, and its fragment entries' q~ offsets and valid counts -- all
+  // from the layout, a library table, before the wait.
+  static_assert(kDecThreads % CPR == 0, "one output coordinate per thread");
+  int rot_j0 = 0, rot_j1 = 0;
+  float rot_scale = 0.f;
+  {
+    const int i = CPR * rank + tid % CPR;
+    if (i < lay.n_positions) {
+      int g = 0;
+      for (int t = 1; t < ng; ++t)
+        if (i >= lay.start[t]) g = t;
+      rot_j0 = lay.start[g];
+      rot_j1 = rot_j0 + lay.size[g];
+      rot_scale = kInvSqrtD * lay.inv_sqrt_d[g] * kLog2e;
     }
   }
+  constexpr int kFragPerThread = (kFragEntries + kDecThreads - 1) / kDecThreads;
+  const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
+  int fr_off[kFragPerThread], fr_cnt[kFragPerThread];
+#pragma unroll
+  for (int k = 0; k < kFragPerThread; ++k) {
+    const int u = tid + k * kDecThreads;
+    fr_off[k] = 0;
+    fr_cnt[k] = 0;
+    if (u < 32 * nchunk) {
+      const int c = u >> 5, ln = u & 31;
+      int g = 0;
+      while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
+      const int c0 = 16 * (c - lay.chunk_base[g]) + 4 * (ln & 3);
+      fr_off[k] = (ln >> 2) * kRowPad + lay.start[g] + c0;
+      fr_cnt[k] = min(4, max(0, lay.size[g] - c0));
+    }
+  }
+  __syncthreads();
+  if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (batch == 1)
+    prefetch_warp_tiles(sh, cache, layer, b, h, split_ctas(plan, sh.ntiles, sh.ntiles), warp, kDecWarps, cu, sh.kbits,
+                        VB);
   // Launched as a programmatic dependent of the previous kernel (the
   // appends of a decode step, or the previous call): the query, the lengths
   // and the cache are read after it has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- 2. the unit's range, split and tiles ----
+  // ---- 2. the unit's query rows and range, then its split and tiles ----
+  // (the query loads go out before the tile copies, which fill the memory
+  // system; they land in qr further down)
+  const size_t qrow0 = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0;
+  __half qv[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) qv[hh] = hh < nh ? q[(qrow0 + hh) * kD + perm_j] : __float2half(0.f);
   const SeqRange sr = seq_range(sh, seq_lens, BufferArgs{}, b);
   if (sr.bad && blockIdx.y == 0 && tid == 0 && h == 0 && hb == 0) atomicOr(ws.err, kErrSeqLen);
   const int len = sr.len, lo = sr.lo;
@@ -980,11 +1071,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   __shared__ int64_t s_red[kDecWarps];
   const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kDecThreads>(sh, seq_lens, BufferArgs{}, batch, s_red);
   const int C = split_ctas(plan, ntl, total);  // a multiple of the cluster size
-  const size_t qrow0 = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + h * G + h0;
   const size_t wrow0 = (static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0;
   if (C == 0) {
     // no packed position: the first cluster writes zero outputs
-    if (clu == 0 && rank < nh) out[(qrow0 + rank) * kD + tid] = __float2half(0.f);
+    if (clu == 0)
+      for (int hh = rank; hh < nh; hh += CL) out[(qrow0 + hh) * kD + tid] = __float2half(0.f);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     return;
   }
@@ -992,7 +1083,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     return;
   }
-  const int nclu = C / kFusedCluster;
+  const int nclu = C / CL;
   const int W = C * kDecWarps;
   const int wu = warp * C + cu;
   const int my_tiles = wu < ntl ? (ntl - wu + W - 1) / W : 0;
@@ -1008,59 +1099,49 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   src.W = W;
   src.kwords = 256 * sh.kbits;
   src.vwords = 256 * VB;
-  src.stage = stage_base + static_cast<size_t>(warp) * FL.stage_bytes;
-  src.stage_stride = kDecWarps * FL.stage_bytes;
-  src.bars = bars + warp * kStages;
-  src.stage_bytes = FL.stage_bytes;
-  // the first tile of each warp goes out now (its stage does not hold the
-  // rotation scratch); the second after the fragments are built
-  if (lane == 0 && my_tiles > 0) issue_tile(src, 0);
+  src.kstage = stage_base + static_cast<size_t>(warp) * FL.kst_bytes;
+  src.kstride = kDecWarps * FL.kst_bytes;
+  src.vbuf = smem_raw + FL.vbase + static_cast<size_t>(warp) * FL.v_bytes;
+  src.bars = bars + warp * kBarsPerWarp;
+  // the first tile of each warp goes out now (its K stage and the V buffers
+  // do not hold the rotation scratch); the second K stage after the
+  // fragments are built
+  if (lane == 0 && my_tiles > 0) {
+    issue_k(src, 0);
+    issue_v(src, 0);
+  }
 
-  // ---- q~ for coordinates [16 rank, 16 rank + 16) of the block's heads ----
+  // ---- q~ for coordinates [CPR rank, CPR rank + CPR) of the block's heads ----
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh)
-    qr[hh * kRowPad + tid] = hh < nh ? __half2float(q[(qrow0 + hh) * kD + perm_j]) : 0.f;
+  for (int hh = 0; hh < 8; ++hh) qr[hh * kRowPad + tid] = __half2float(qv[hh]);
   __syncthreads();
   {
-    const int hh = tid >> 4, o = tid & 15;
-    const int i = 16 * rank + o;
-    float v = 0.f;
-    if (i < lay.n_positions) {
-      int g = 0;
-      for (int t = 1; t < ng; ++t)
-        if (i >= lay.start[t]) g = t;
-      const int j0 = lay.start[g], j1 = j0 + lay.size[g];
-      const float* rrow = rk + o * kRowPad;
+    const int o = tid % CPR;
+    const int i = CPR * rank + o;
+    const float* rrow = rk + o * kRowPad;
+#pragma unroll
+    for (int k = 0; k < 8 * CPR / kDecThreads; ++k) {
+      const int hh = tid / CPR + k * (kDecThreads / CPR);
       const float* qrow = qr + hh * kRowPad;
       float a0 = 0.f, a1 = 0.f;
-      int j = j0;
-      for (; j + 1 < j1; j += 2) {
+      for (int j = rot_j0; j < rot_j1; j += 2) {  // group sizes are even (whole RoPE blocks)
         a0 = fmaf(rrow[j], qrow[j], a0);
         a1 = fmaf(rrow[j + 1], qrow[j + 1], a1);
       }
-      if (j < j1) a0 = fmaf(rrow[j], qrow[j], a0);
-      v = (a0 + a1) * (kInvSqrtD * lay.inv_sqrt_d[g]);
-    }
+      const float v = (a0 + a1) * rot_scale;  // log2(e) q~
 #pragma unroll
-    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st(dsmem_addr(qt + hh * kRowPad + i, r2), v);
+      for (int r2 = 0; r2 < CL; ++r2) dsmem_st(dsmem_addr(qt + hh * kRowPad + i, r2), v);
+    }
   }
   cluster_sync_all();
-  // the B fragments from q~ (see write_frags for the layout); heads past nh are zero
-  {
-    const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
-    for (int u = tid; u < 32 * nchunk; u += kDecThreads) {
-      const int c = u >> 5, ln = u & 31;
-      int g = 0;
-      while (g + 1 < ng && c >= lay.chunk_base[g + 1]) ++g;
-      const int j = c - lay.chunk_base[g];
-      const int d = lay.size[g], st = lay.start[g];
-      const int head = ln >> 2;
+  // the B fragments from log2(e) q~ (see write_frags for the layout); heads past nh are zero
+#pragma unroll
+  for (int k = 0; k < kFragPerThread; ++k) {
+    const int u = tid + k * kDecThreads;
+    if (u < 32 * nchunk) {
       float v[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int coord = 16 * j + 4 * (ln & 3) + m;
-        v[m] = coord < d ? qt[head * kRowPad + st + coord] * kLog2e : 0.f;
-      }
+      for (int m = 0; m < 4; ++m) v[m] = m < fr_cnt[k] ? qt[fr_off[k] + m] : 0.f;
       const __half2 a = __floats2half2_rn(v[0], v[1]);
       const __half2 c2 = __floats2half2_rn(v[2], v[3]);
       const float2 af = __half22float2(a), cf = __half22float2(c2);
@@ -1074,11 +1155,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   {
     const uint4 a0 = *reinterpret_cast<const uint4*>(tabv);
     const uint4 a1 = *reinterpret_cast<const uint4*>(tabv + 4);
-    tv.lo[0] = a0.x; tv.lo[1] = a0.y; tv.lo[2] = a0.z; tv.lo[3] = a0.w;
-    tv.hi[0] = a1.x; tv.hi[1] = a1.y; tv.hi[2] = a1.z; tv.hi[3] = a1.w;
+    tv.lo[0] = a0.x; tv.lo[1] = a0.y;
+    tv.hi[0] = a1.x; tv.hi[1] = a1.y;
   }
   __syncthreads();  // fragments ready; the rotation scratch (second stages) is free
-  if (lane == 0 && my_tiles > 1) issue_tile(src, 1);
+  if (lane == 0 && my_tiles > 1) issue_k(src, 1);
 
   // ---- 3. the tiles, then the CTA's warps merged ----
   TileTables tt{grp, tabk, pdesc, bq, ng};
@@ -1086,91 +1167,150 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   const int failed_at = attend_tiles<VB>(src, tt, tv, my_tiles, len, lo, O, m_run, l_run);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   float* cacc = reinterpret_cast<float*>(stage_base);  // [8][kD]
-  merge_warps(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, cm, cm + 8, cacc,
-              nh);
+  merge_warps<kDecWarps>(O, m_run, l_run, failed_at >= 0, reinterpret_cast<float*>(stage_base), ms, ls, wsc, cm,
+                        cm + 8, cacc, nh);
   cluster_sync_all();
 
-  // ---- 4. cluster merge: CTA rank r takes head r over the cluster's CTAs ----
-  if (rank < nh) {
-    float mr[kFusedCluster], wr[kFusedCluster];
+  // ---- 4. cluster merge: CTA rank r takes heads r, r + CL, ... over the cluster's CTAs ----
+  for (int hh = rank; hh < nh; hh += CL) {
+    float mr[CL], wr[CL];
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int c = 0; c < kFusedCluster; ++c) {
-      mr[c] = dsmem_ld(dsmem_addr(cm + rank, c));
+    for (int c = 0; c < CL; ++c) {
+      mr[c] = dsmem_ld(dsmem_addr(cm + hh, c));
       M = fmaxf(M, mr[c]);
     }
     float Lsum = 0.f, a = 0.f;
 #pragma unroll
-    for (int c = 0; c < kFusedCluster; ++c) {
+    for (int c = 0; c < CL; ++c) {
       wr[c] = mr[c] == -CUDART_INF_F ? 0.f : fast_exp2(mr[c] - M);
-      Lsum = fmaf(wr[c], dsmem_ld(dsmem_addr(cm + 8 + rank, c)), Lsum);
-      a = fmaf(wr[c], dsmem_ld(dsmem_addr(cacc + rank * kD + tid, c)), a);
+      Lsum = fmaf(wr[c], dsmem_ld(dsmem_addr(cm + 8 + hh, c)), Lsum);
+      a = fmaf(wr[c], dsmem_ld(dsmem_addr(cacc + hh * kD + tid, c)), a);
     }
-    float* part = ws.partials + ((wrow0 + rank) * sh.max_splits + clu) * kPartialStride;
+    float* part = ws.partials + ((wrow0 + hh) * sh.max_splits + clu) * kPartialStride;
     part[4 + tid] = a;
     if (tid == 0) {
       part[0] = M;
       part[1] = Lsum;
     }
-    __threadfence();
   }
-  cluster_sync_all();  // remote reads done; the cluster's partials are written
+  // remote reads done; the cluster's partial writes happen before the
+  // barrier, and the fence of the thread that counts the arrival orders them
+  // (cumulatively) before its atomic
+  cluster_sync_all();
   if (tid == 0 && rank == 0) {
+    __threadfence();
     const uint32_t last = atomicAdd(ws.comb_count + wrow0, 1u) == static_cast<uint32_t>(nclu - 1) ? 1u : 0u;
+    __threadfence();  // the other clusters' partials, seen through the count, before the loads below
 #pragma unroll
-    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st_u32(dsmem_addr(flag, r2), last);
+    for (int r2 = 0; r2 < CL; ++r2) dsmem_st_u32(dsmem_addr(flag, r2), last);
   }
   cluster_sync_all();
   if (*flag == 0u) return;  // the same for the whole cluster
 
   // ---- 5. the unit's last cluster: merge the clusters, rotate back ----
-  __threadfence();
-  if (rank < nh) {
-    const float* part = ws.partials + (wrow0 + rank) * sh.max_splits * kPartialStride;
-    float M = -CUDART_INF_F;
-    for (int c = 0; c < nclu; ++c) M = fmaxf(M, __ldcg(part + c * kPartialStride));
-    float Lsum = 0.f, a = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < nclu; ++c) {
-      const float mc = __ldcg(part + c * kPartialStride);
-      const float w = mc == -CUDART_INF_F ? 0.f : exp2f(mc - M);
-      Lsum = fmaf(w, __ldcg(part + c * kPartialStride + 1), Lsum);
-      a = fmaf(w, __ldcg(part + c * kPartialStride + 4 + tid), a);
-    }
-    const float an = a / Lsum;
-#pragma unroll
-    for (int r2 = 0; r2 < kFusedCluster; ++r2) dsmem_st(dsmem_addr(qt + rank * kRowPad + tid, r2), an);
-  }
-  // columns [16 rank, 16 rank + 16) of R_V (row-major [in][out]): rv[o][i] = R_V[i][16 rank + o]
-  float* rv = rk;
+  // CTA rank r merges heads r, r + CL, ...: warp w takes the clusters
+  // w, w + 4, ... (eight at a time, all their loads in flight), a lane four
+  // dims; the warps' (m, l, acc) then meet in shared memory (the stage
+  // buffers are free: no CTA reads this CTA's shared memory any more).
+  // columns [CPR rank, CPR rank + CPR) of R_V (row-major [in][out]), a
+  // library table: loaded first, stored as rv[o][i] = R_V[i][CPR rank + o]
+  // after the merges
+  constexpr int kRvLoads = CPR / 4;
+  float4 rvv[kRvLoads];
   {
     const float* mv = ws.mv + static_cast<size_t>(lh) * kD * kD;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kRvLoads; ++k) {
       const int f = tid + k * kDecThreads;
-      const int i = f >> 2, q4 = f & 3;
-      const float4 v = __ldg(reinterpret_cast<const float4*>(mv + i * kD + 16 * rank + 4 * q4));
-      rv[(4 * q4 + 0) * kRowPad + i] = v.x;
-      rv[(4 * q4 + 1) * kRowPad + i] = v.y;
-      rv[(4 * q4 + 2) * kRowPad + i] = v.z;
-      rv[(4 * q4 + 3) * kRowPad + i] = v.w;
+      rvv[k] = __ldg(reinterpret_cast<const float4*>(mv + (f / (CPR / 4)) * kD + CPR * rank + 4 * (f % (CPR / 4))));
     }
+  }
+  float* wacc = reinterpret_cast<float*>(stage_base);  // [kDecWarps][kD]
+  float* wml = wacc + kDecWarps * kD;                  // [kDecWarps][2]
+  for (int hh = rank; hh < nh; hh += CL) {
+    const float* part = ws.partials + (wrow0 + hh) * sh.max_splits * kPartialStride;
+    float m_w = -CUDART_INF_F, l_w = 0.f;
+    float4 a_w = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = warp; c0 < nclu; c0 += 8 * kDecWarps) {
+      float mm[8], ll[8];
+      float4 aa[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + j * kDecWarps;
+        if (c < nclu) {
+          const float* p = part + static_cast<size_t>(c) * kPartialStride;
+          mm[j] = __ldcg(p);
+          ll[j] = __ldcg(p + 1);
+          aa[j] = __ldcg(reinterpret_cast<const float4*>(p + 4) + lane);
+        } else {
+          mm[j] = -CUDART_INF_F;
+          ll[j] = 0.f;
+          aa[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mb = m_w;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mb = fmaxf(mb, mm[j]);
+      if (mb == -CUDART_INF_F) continue;  // only empty clusters so far
+      const float f = m_w == -CUDART_INF_F ? 0.f : exp2f(m_w - mb);
+      l_w *= f;
+      a_w.x *= f; a_w.y *= f; a_w.z *= f; a_w.w *= f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float wgt = mm[j] == -CUDART_INF_F ? 0.f : exp2f(mm[j] - mb);
+        l_w = fmaf(wgt, ll[j], l_w);
+        a_w.x = fmaf(wgt, aa[j].x, a_w.x);
+        a_w.y = fmaf(wgt, aa[j].y, a_w.y);
+        a_w.z = fmaf(wgt, aa[j].z, a_w.z);
+        a_w.w = fmaf(wgt, aa[j].w, a_w.w);
+      }
+      m_w = mb;
+    }
+    *reinterpret_cast<float4*>(wacc + warp * kD + 4 * lane) = a_w;
+    if (lane == 0) {
+      wml[2 * warp] = m_w;
+      wml[2 * warp + 1] = l_w;
+    }
+    __syncthreads();
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wml[2 * w]);
+    float Lsum = 0.f, a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float wgt = wml[2 * w] == -CUDART_INF_F ? 0.f : exp2f(wml[2 * w] - M);
+      Lsum = fmaf(wgt, wml[2 * w + 1], Lsum);
+      a = fmaf(wgt, wacc[w * kD + tid], a);
+    }
+    const float an = a / Lsum;
+#pragma unroll
+    for (int r2 = 0; r2 < CL; ++r2) dsmem_st(dsmem_addr(qt + hh * kRowPad + tid, r2), an);
+    __syncthreads();  // wacc is reused by the next head
+  }
+  float* rv = rk;
+#pragma unroll
+  for (int k = 0; k < kRvLoads; ++k) {
+    const int f = tid + k * kDecThreads;
+    const int i = f / (CPR / 4), q4 = f % (CPR / 4);
+    rv[(4 * q4 + 0) * kRowPad + i] = rvv[k].x;
+    rv[(4 * q4 + 1) * kRowPad + i] = rvv[k].y;
+    rv[(4 * q4 + 2) * kRowPad + i] = rvv[k].z;
+    rv[(4 * q4 + 3) * kRowPad + i] = rvv[k].w;
   }
   if (tid == 0 && rank == 0) ws.comb_count[wrow0] = 0u;  // ready for the next call
   cluster_sync_all();
-  {
-    const int hh = tid >> 4, o = tid & 15;
-    if (hh < nh) {
-      const float* rrow = rv + o * kRowPad;
-      const float* arow = qt + hh * kRowPad;
-      float s0 = 0.f, s1 = 0.f;
+  for (int u = tid; u < nh * CPR; u += kDecThreads) {
+    const int hh = u / CPR, o = u % CPR;
+    const float* rrow = rv + o * kRowPad;
+    const float* arow = qt + hh * kRowPad;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll 8
-      for (int i = 0; i < kD; i += 2) {
-        s0 = fmaf(rrow[i], arow[i], s0);
-        s1 = fmaf(rrow[i + 1], arow[i + 1], s1);
-      }
-      out[(qrow0 + hh) * kD + 16 * rank + o] = __float2half(s0 + s1);
+    for (int i = 0; i < kD; i += 2) {
+      s0 = fmaf(rrow[i], arow[i], s0);
+      s1 = fmaf(rrow[i + 1], arow[i + 1], s1);
     }
+    out[(qrow0 + hh) * kD + CPR * rank + o] = __float2half(s0 + s1);
   }
 }
 
@@ -1353,92 +1493,117 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
 }
 
+// Warps per CTA of the split pass: one CTA of 16 warps per SM.  Its warp
+// w runs on sub-partition w mod 4, and a unit's tiles go to warps in slot
+// order (w C + cu), so the tiles a partial last round leaves spread over the
+// four sub-partitions of every SM.
+constexpr int kSplitWarps = 16;
+
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
                              const float* qrot, const int32_t* seq_lens, const BufferArgs& buf, int batch,
                              const SplitPlan& plan, cudaStream_t stream) {
   // the largest layout over K widths, so one attribute value serves every call
-  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
+  static const cudaError_t attr =
+      set_smem(decode_mma_kernel<VB, kSplitWarps>, decode_layout(4, VB, kSplitWarps).total);
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
   // units fastest, then split index: the CTAs every unit uses come first
   dim3 grid(batch * s.n_kv_heads * head_blocks, (buf.k != nullptr ? 1 : 0) + plan.c_max, layer_count);
-  return launch_dependent(decode_mma_kernel<VB>, grid, dim3(kDecThreads), decode_layout(s.kbits, VB).total, stream, s,
-                          ws, cache, layer0, qrot, seq_lens, buf, batch, plan, head_blocks);
+  return launch_dependent(decode_mma_kernel<VB, kSplitWarps>, grid, dim3(kSplitWarps * 32),
+                          decode_layout(s.kbits, VB, kSplitWarps).total, stream, s, ws, cache, layer0, qrot, seq_lens,
+                          buf, batch, plan, head_blocks);
 }
 
 template <int VB>
 int ctas_per_sm_vb(const Shape& s) {
-  static const cudaError_t attr = set_smem(decode_mma_kernel<VB>, decode_layout(4, VB).total);
+  static const cudaError_t attr =
+      set_smem(decode_mma_kernel<VB, kSplitWarps>, decode_layout(4, VB, kSplitWarps).total);
   if (attr != cudaSuccess) return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<VB>, kDecThreads,
-                                                    decode_layout(s.kbits, VB).total) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_mma_kernel<VB, kSplitWarps>, kSplitWarps * 32,
+                                                    decode_layout(s.kbits, VB, kSplitWarps).total) != cudaSuccess)
     return 0;
   return n;
 }
 
-template <int VB>
+template <int VB, int CL>
 cudaError_t fused_attr_once() {
-  static const cudaError_t attr = set_smem(decode_fused_kernel<VB>, fused_layout(4, VB).total);
+  static const cudaError_t attr = set_smem(decode_fused_kernel<VB, CL>, fused_layout(4, VB, CL).total);
   return attr;
 }
 
-template <int VB>
-cudaError_t launch_fused_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
-                            const __half* q, const int32_t* seq_lens, int batch, const SplitPlan& plan, __half* out,
-                            cudaStream_t stream) {
-  const cudaError_t attr = fused_attr_once<VB>();
+template <int VB, int CL>
+cudaError_t launch_fused_vcl(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                             const __half* q, const int32_t* seq_lens, int batch, const SplitPlan& plan, __half* out,
+                             cudaStream_t stream) {
+  const cudaError_t attr = fused_attr_once<VB, CL>();
   if (attr != cudaSuccess) return attr;
   const int head_blocks = (s.group + 7) / 8;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch * s.n_kv_heads * head_blocks, plan.c_max, layer_count);
   cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB).total;
+  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB, CL).total;
   cfg.stream = stream;
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   at[1].id = cudaLaunchAttributeClusterDimension;
   at[1].val.clusterDim.x = 1;
-  at[1].val.clusterDim.y = kFusedCluster;
+  at[1].val.clusterDim.y = CL;
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<VB>, s, ws, cache, layer0, q, seq_lens, batch, plan,
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel<VB, CL>, s, ws, cache, layer0, q, seq_lens, batch, plan,
                             head_blocks, out);
 }
 
 template <int VB>
-int fused_clusters_vb(const Shape& s) {
-  if (fused_attr_once<VB>() != cudaSuccess) return 0;
+cudaError_t launch_fused_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
+                            const __half* q, const int32_t* seq_lens, int batch, const SplitPlan& plan, __half* out,
+                            cudaStream_t stream) {
+  if (plan.cluster == 4)
+    return launch_fused_vcl<VB, 4>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+  if (plan.cluster == 8)
+    return launch_fused_vcl<VB, 8>(s, ws, cache, layer0, layer_count, q, seq_lens, batch, plan, out, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <int VB, int CL>
+int fused_clusters_vcl(const Shape& s) {
+  if (fused_attr_once<VB, CL>() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1, kFusedCluster, 1);
+  cfg.gridDim = dim3(1, CL, 1);
   cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB).total;
+  cfg.dynamicSmemBytes = fused_layout(s.kbits, VB, CL).total;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
-  at[0].val.clusterDim.y = kFusedCluster;
+  at[0].val.clusterDim.y = CL;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_fused_kernel<VB>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_fused_kernel<VB, CL>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
   return n;
 }
 
+template <int VB>
+int fused_clusters_vb(const Shape& s, int cl) {
+  return cl == 4 ? fused_clusters_vcl<VB, 4>(s) : cl == 8 ? fused_clusters_vcl<VB, 8>(s) : 0;
+}
+
 }  // namespace
 
-int decode_fused_clusters(const Shape& s) {
+int decode_fused_clusters(const Shape& s, int cluster) {
   switch (s.vbits) {
-    case 1: return fused_clusters_vb<1>(s);
-    case 2: return fused_clusters_vb<2>(s);
-    case 3: return fused_clusters_vb<3>(s);
-    default: return fused_clusters_vb<4>(s);
+    case 1: return fused_clusters_vb<1>(s, cluster);
+    case 2: return fused_clusters_vb<2>(s, cluster);
+    case 3: return fused_clusters_vb<3>(s, cluster);
+    default: return fused_clusters_vb<4>(s, cluster);
   }
 }
 

@@ -98,7 +98,7 @@ struct Shape {
   int64_t capacity;
   int64_t ntiles;                // tiles per (layer, sequence, KV head)
   int32_t drop_tile;             // test hook: the split pass issues no copy for this tile (-1: off)
-  int32_t pad;
+  int32_t n_sms;                 // SMs of the device (the decode's warp-to-tile rotation)
 };
 
 // RoPE applied inside the encode (K rows taken before RoPE): block j of the
@@ -176,16 +176,17 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
 // Resident split-decode CTAs per SM for a config (0 on error).
 int decode_ctas_per_sm(const Shape& s);
 // The fused decode (query rotation, split-K pass, merge and inverse V
-// rotation in one launch, in clusters of 8 CTAs): q fp16
+// rotation in one launch, in clusters of plan.cluster = 4 or 8 CTAs): q fp16
 // [layer_count][batch][Hq][128], out fp16 of the same shape; the plan's
-// c_max and cluster must be multiples of / equal to 8.  Partials, one per
-// cluster, and the per-unit arrival counters (zero between calls) are in
-// the workspace.
+// c_max must be a multiple of its cluster size.  Partials, one per cluster,
+// and the per-unit arrival counters (zero between calls) are in the
+// workspace.
 cudaError_t launch_decode_fused(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0,
                                 int layer_count, const __half* q, const int32_t* seq_lens, int batch,
                                 const SplitPlan& plan, __half* out, cudaStream_t stream);
-// Co-resident 8-CTA clusters of the fused decode for a config (0: it cannot run).
-int decode_fused_clusters(const Shape& s);
+// Co-resident clusters of `cluster` (4 or 8) CTAs of the fused decode for a
+// config (0: it cannot run).
+int decode_fused_clusters(const Shape& s, int cluster);
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
                            __half* out, cudaStream_t stream);

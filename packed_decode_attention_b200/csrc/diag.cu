@@ -148,8 +148,8 @@ __global__ void __launch_bounds__(kDecThreads) logit_mae_kernel(Shape sh, Worksp
         const int chunk = grp[g * 8 + 4];
         const uint4 tl = *reinterpret_cast<const uint4*>(tabk + 8 * g);
         const uint4 th = *reinterpret_cast<const uint4*>(tabk + 8 * g + 4);
-        t.lo[0] = tl.x; t.lo[1] = tl.y; t.lo[2] = tl.z; t.lo[3] = tl.w;
-        t.hi[0] = th.x; t.hi[1] = th.y; t.hi[2] = th.z; t.hi[3] = th.w;
+        t.lo[0] = tl.x; t.lo[1] = tl.y;
+        t.hi[0] = th.x; t.hi[1] = th.y;
         const uint32_t pd = pdesc[g * 32 + lane];
         const uint32_t* gw = kt + gp.w;
         const uint4* bqg = bq + chunk * 32 + lane;

@@ -404,13 +404,14 @@ __device__ __forceinline__ void issue_v(const TileSource& src, int k) {
   bulk_copy_g2s(src.vbuf, src.cache.vtile + slot * src.vwords, vbytes, bar);
 }
 
-// Lane 0: the copies a warp starts with (K of its first two tiles, V of its first).
+// Lane 0: the copies a warp starts with, its first tile (K and V).  The
+// second tile's K goes out once the first K has landed (attend_tiles), so
+// that every warp's first tile comes in before any warp's second.
 __device__ __forceinline__ void issue_first(const TileSource& src, int my_tiles) {
   if (my_tiles > 0) {
     issue_k(src, 0);
     issue_v(src, 0);
   }
-  if (my_tiles > 1) issue_k(src, 1);
 }
 
 // The decode tables a warp reads from shared memory (a copy of the
@@ -424,8 +425,8 @@ struct TileTables {
 };
 
 // Attends the warp's my_tiles tiles over the positions [lo, len); the copies
-// of issue_first must already be issued.  Returns the index of the tile
-// whose copy wait gave up (-1: none).
+// of issue_first must already be issued (this issues the rest).  Returns the
+// index of the tile whose copy wait gave up (-1: none).
 template <int VB>
 __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTables& tt, const ByteTab& tv,
                                             int my_tiles, int len, int lo, float (&O)[8][4], float (&m_run)[2],
@@ -447,6 +448,7 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       failed_at = k;
       break;
     }
+    if (k == 0 && lane == 0 && my_tiles > 1) issue_k(src, 1);
     const unsigned char* st = src.kstage + (k % kStages) * src.kstride;
     const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
     const __half* kn = reinterpret_cast<const __half*>(st + kbytes);
@@ -581,8 +583,8 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
     // stages of tiles up to f + 1 and the V buffer of tile f were issued.
     if (lane == 0) atomicOr(src.err, kErrTimeout);
     const int f = failed_at;
-    for (int k = k_consumed ? f + 1 : f; k < min(my_tiles, f + kStages); ++k)
-      mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
+    const int k_issued = (f == 0 && !k_consumed) ? 1 : min(my_tiles, f + kStages);  // K1 waits for K0
+    for (int k = k_consumed ? f + 1 : f; k < k_issued; ++k) mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
     mbar_wait(&src.bars[kStages], f & 1);
   }
   return failed_at;
@@ -1104,12 +1106,10 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
   src.vbuf = smem_raw + FL.vbase + static_cast<size_t>(warp) * FL.v_bytes;
   src.bars = bars + warp * kBarsPerWarp;
   // the first tile of each warp goes out now (its K stage and the V buffers
-  // do not hold the rotation scratch); the second K stage after the
-  // fragments are built
-  if (lane == 0 && my_tiles > 0) {
-    issue_k(src, 0);
-    issue_v(src, 0);
-  }
+  // do not hold the rotation scratch, which the second K stages do until
+  // the fragments are built; the tile loop issues the second K stage once
+  // the first has landed)
+  if (lane == 0) issue_first(src, my_tiles);
 
   // ---- q~ for coordinates [CPR rank, CPR rank + CPR) of the block's heads ----
 #pragma unroll
@@ -1159,7 +1159,6 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
     tv.hi[0] = a1.x; tv.hi[1] = a1.y;
   }
   __syncthreads();  // fragments ready; the rotation scratch (second stages) is free
-  if (lane == 0 && my_tiles > 1) issue_k(src, 1);
 
   // ---- 3. the tiles, then the CTA's warps merged ----
   TileTables tt{grp, tabk, pdesc, bq, ng};
@@ -1493,11 +1492,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
 }
 
-// Warps per CTA of the split pass: one CTA of 16 warps per SM.  Its warp
-// w runs on sub-partition w mod 4, and a unit's tiles go to warps in slot
-// order (w C + cu), so the tiles a partial last round leaves spread over the
-// four sub-partitions of every SM.
-constexpr int kSplitWarps = 16;
+// Warps per CTA of the split pass (several CTAs per SM: a CTA that finishes
+// frees its slot for the next launch's CTAs, which overlap their set-up
+// with this launch's tail).
+constexpr int kSplitWarps = kDecWarps;
 
 template <int VB>
 cudaError_t launch_decode_vb(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,

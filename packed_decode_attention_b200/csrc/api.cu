@@ -660,6 +660,21 @@ bgtq::SplitPlan split_for(bgtq_state* st, int32_t layer_count, int32_t batch, in
   return p;
 }
 
+// The plan of a split pass that directly follows the call's own query
+// rotation or decode-step preparation (bgtq::SplitPlan::early): the pass
+// may read the caller's arrays and copy its first tiles before its wait.
+// The preparation kernel appends 1..kAppendMaxRows rows per sequence itself;
+// more rows go through the encode, which has completed by then.
+bgtq::SplitPlan after_prep(bgtq::SplitPlan p, const int32_t* d_start = nullptr, const int32_t* d_count = nullptr,
+                           int32_t n = 0) {
+  p.early = 1;
+  if (n >= 1 && n <= bgtq::kAppendMaxRows) {
+    p.app_start = d_start;
+    p.app_count = d_count;
+  }
+  return p;
+}
+
 }  // namespace
 
 int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const float* d_qrot,
@@ -700,7 +715,7 @@ int bgtq_decode_attn(bgtq_state* st, int32_t layer, int32_t layer_count, const v
                                      static_cast<__half*>(d_out), s) == cudaSuccess
                ? BGTQ_OK
                : BGTQ_ERR_CUDA;
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
+  const bgtq::SplitPlan split = after_prep(split_for(st, layer_count, batch));
   if (bgtq::launch_rotate_query(st->shape, st->ws, layer, layer_count, static_cast<const __half*>(d_q), batch,
                                 st->ws.qrot, s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
@@ -768,7 +783,7 @@ int bgtq_decode_step(bgtq_state* st, int32_t layer, int32_t layer_count, const v
                ? BGTQ_OK
                : BGTQ_ERR_CUDA;
   }
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
+  const bgtq::SplitPlan split = after_prep(split_for(st, layer_count, batch), d_start, d_count, n);
   if (queue_step_prep(st, layer, layer_count, static_cast<const __half*>(d_q), batch, d_k, d_v, d_start, d_count, n,
                       s) != cudaSuccess)
     return BGTQ_ERR_CUDA;
@@ -799,7 +814,7 @@ int decode_buffered_impl(bgtq_state* st, int32_t layer, int32_t layer_count, con
   if (!aligned16(d_q) || !aligned16(d_seq_lens) || !aligned16(d_pos_lo) || !aligned16(d_buf_k) ||
       !aligned16(d_buf_v) || !aligned16(d_buf_count) || !aligned16(d_out))
     return BGTQ_ERR_ALIGNMENT;
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch, 1);
+  const bgtq::SplitPlan split = after_prep(split_for(st, layer_count, batch, 1), d_start, d_count, n);
   cudaStream_t s = as_stream(stream);
   bgtq::BufferArgs buf;
   buf.q = static_cast<const __half*>(d_q);
@@ -917,7 +932,7 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
                ? BGTQ_OK
                : BGTQ_ERR_CUDA;
   }
-  const bgtq::SplitPlan split = split_for(st, layer_count, batch);
+  const bgtq::SplitPlan split = after_prep(split_for(st, layer_count, batch));
   const int64_t nspl = split.c_max;
   // the combine's arrival counters first, at a fixed place (they are 0
   // between calls, whatever the call's layout), then q~, its fragments, the

@@ -33,7 +33,7 @@ __host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
 // pool (the caller raises kErrPage).
 __device__ __forceinline__ int64_t tile_slot(const Shape& sh, const CacheDev& c, int layer, int b, int h, int64_t t) {
   if (c.n_pages == 0) return ((static_cast<int64_t>(layer) * sh.max_batch + b) * sh.n_kv_heads + h) * sh.ntiles + t;
-  const int32_t page = c.block_table[static_cast<int64_t>(b) * sh.ntiles + t];
+  const int32_t page = __ldcg(c.block_table + static_cast<int64_t>(b) * sh.ntiles + t);  // through L2: see seq_range
   if (page < 0 || page >= c.n_pages) return -1;
   return (static_cast<int64_t>(layer) * sh.n_kv_heads + h) * c.n_pages + page;
 }
@@ -422,13 +422,12 @@ __device__ __forceinline__ void group_logits(const uint32_t* gw, int nfull, bool
 #pragma unroll
     for (int k = 0; k < B; ++k) w[k] = pc[base + stride * k];
     quartet_decode<B>(w, s);
-    if (pd & (1u << 20)) {
-      const int sh = (pd >> 21) & 1 ? 16 : 0;
+    {
+      // a half-quad lane keeps the two nibble bytes of its half, each
+      // followed by a zero byte (a PRMT from the word and zero); others keep s
+      const uint32_t hsel = !(pd & (1u << 20)) ? 0x3210u : ((pd >> 21) & 1) ? 0x4342u : 0x4140u;
 #pragma unroll
-      for (int mu = 0; mu < 4; ++mu) {
-        const uint32_t x = (s[mu] >> sh) & 0xFFFFu;
-        s[mu] = (x & 0xFFu) | ((x & 0xFF00u) << 8);
-      }
+      for (int mu = 0; mu < 4; ++mu) s[mu] = prmt(s[mu], 0u, hsel);
     }
     if (nfull > 0) chunk_mma<B == 4, false>(t, s, bqg[nfull * 32], S);
     else chunk_mma<B == 4, true>(t, s, bqg[0], S);

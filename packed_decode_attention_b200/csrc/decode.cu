@@ -153,11 +153,14 @@ struct SeqRange {
   bool bad;
 };
 
+// The caller's arrays are read through L2 (ld.global.cg): the split pass may
+// read them before its dependency wait, and no copy in this SM's L1 may be
+// older than the stream's last write.
 __device__ __forceinline__ SeqRange seq_range(const Shape& sh, const int32_t* seq_lens, const BufferArgs& buf, int b) {
   SeqRange r;
-  r.len = seq_lens[b];
-  r.lo = buf.pos_lo != nullptr ? buf.pos_lo[b] : 0;
-  r.cnt = buf.k != nullptr ? buf.count[b] : 0;
+  r.len = __ldcg(seq_lens + b);
+  r.lo = buf.pos_lo != nullptr ? __ldcg(buf.pos_lo + b) : 0;
+  r.cnt = buf.k != nullptr ? __ldcg(buf.count + b) : 0;
   r.bad = r.len < 0 || r.len > sh.capacity || r.lo < 0 || r.lo > r.len || r.cnt < 0 || r.cnt > buf.n_buf;
   if (r.len < 0 || r.len > sh.capacity) r.len = 0;
   if (r.lo < 0 || r.lo > r.len) r.lo = r.len;
@@ -404,9 +407,22 @@ __device__ __forceinline__ void issue_v(const TileSource& src, int k) {
   bulk_copy_g2s(src.vbuf, src.cache.vtile + slot * src.vwords, vbytes, bar);
 }
 
-// Lane 0: the copies a warp starts with, its first tile (K and V).  The
-// second tile's K goes out once the first K has landed (attend_tiles), so
-// that every warp's first tile comes in before any warp's second.
+// Lanes 1 .. kPrefetchTiles - 1: L2 prefetch hints for the warp's tiles 1, 2, ...
+__device__ __forceinline__ void prefetch_next_tiles(const TileSource& src, int my_tiles) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0 || lane >= kPrefetchTiles || lane >= my_tiles) return;
+  const int64_t slot = tile_slot(src.sh, src.cache, src.layer, src.b, src.h, src.tlo + src.wu + lane * src.W);
+  if (slot < 0) return;
+  prefetch_l2(src.cache.ktile + slot * src.kwords, 4u * src.kwords);
+  prefetch_l2(src.cache.vtile + slot * src.vwords, 4u * src.vwords);
+  prefetch_l2(src.cache.knorm + slot * kTile * 4, kTile * 8);
+  prefetch_l2(src.cache.vnorm + slot * kTile, kTile * 2);
+}
+
+// Lane 0: the copies a warp starts with, its first tile (K and V).  Each
+// later tile's K goes out once the previous tile's K has landed, its V once
+// the previous tile is done (attend_tiles), so every warp's first tile
+// comes in before any warp's second.
 __device__ __forceinline__ void issue_first(const TileSource& src, int my_tiles) {
   if (my_tiles > 0) {
     issue_k(src, 0);
@@ -448,7 +464,8 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       failed_at = k;
       break;
     }
-    if (k == 0 && lane == 0 && my_tiles > 1) issue_k(src, 1);
+    // the other K stage held tile k - 1, which is done: tile k + 1's K goes there
+    if (lane == 0 && k + 1 < my_tiles) issue_k(src, k + 1);
     const unsigned char* st = src.kstage + (k % kStages) * src.kstride;
     const uint32_t* kt = reinterpret_cast<const uint32_t*>(st);
     const __half* kn = reinterpret_cast<const __half*>(st + kbytes);
@@ -572,18 +589,16 @@ __device__ __forceinline__ int attend_tiles(const TileSource& src, const TileTab
       for (int kappa = 0; kappa < 4; ++kappa) mma_selector<VB>(O[m], tv, sv[kappa], bp[kappa][0], bp[kappa][1]);
     }
     __syncwarp();
-    if (lane == 0) {
-      if (k + 1 < my_tiles) issue_v(src, k + 1);
-      if (k + kStages < my_tiles) issue_k(src, k + kStages);
-    }
+    if (lane == 0 && k + 1 < my_tiles) issue_v(src, k + 1);
   }
   if (failed_at >= 0) {
     // copies issued but not yet consumed: let them land (bounded) before the
     // buffers are reused or the CTA exits.  At the failure at tile f the K
-    // stages of tiles up to f + 1 and the V buffer of tile f were issued.
+    // stage of tile f + 1 (once tile f's K had landed) and the V buffer of
+    // tile f were issued.
     if (lane == 0) atomicOr(src.err, kErrTimeout);
     const int f = failed_at;
-    const int k_issued = (f == 0 && !k_consumed) ? 1 : min(my_tiles, f + kStages);  // K1 waits for K0
+    const int k_issued = k_consumed ? min(my_tiles, f + 2) : f + 1;
     for (int k = k_consumed ? f + 1 : f; k < k_issued; ++k) mbar_wait(&src.bars[k % kStages], (k / kStages) & 1);
     mbar_wait(&src.bars[kStages], f & 1);
   }
@@ -715,28 +730,25 @@ __global__ void __launch_bounds__(NW * 32, NW == kDecWarps ? kDecMinBlocks : 1)
   if (tid < NW * kBarsPerWarp) mbar_init(&bars[tid], 1);
   __syncthreads();
   if (tid == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  // While the previous kernel may still run: L2 prefetch hints for this
-  // warp's first tiles (the copies below still read after the wait)
-  if (batch == 1 && cu >= 0)
-    prefetch_warp_tiles(sh, cache, layer, b, h, split_ctas(plan, sh.ntiles, sh.ntiles), warp, NW, cu, sh.kbits, VB);
-  // Launched as a programmatic dependent of the previous kernel (the query
-  // rotation): everything above reads only the library's tables; the
-  // sequence lengths, rotated queries and cache are read after that kernel
-  // has completed.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // the unit's q~ fragments (written by the query rotation): their loads go
-  // out with the length reads below and land in shared memory further down
+  // Launched as a programmatic dependent of the previous kernel.  Without
+  // plan.early everything before griddepcontrol.wait reads only the library's
+  // tables.  With it, the previous kernel is this call's query rotation (or
+  // decode-step preparation), whose CTAs let this grid start only after
+  // their own wait, so all earlier work of the stream has completed: the
+  // caller's lengths, block table and cache are read before the wait too,
+  // and each warp's first tile is copied then, unless it holds a row that
+  // the preparation appends in the same launch.  The rotated queries are
+  // always read after the wait.
+  const bool early = plan.early != 0 && cu >= 0;
+  if (!early) {
+    // L2 prefetch hints for this warp's first tiles while the previous
+    // kernel may still run (the copies below still read after the wait)
+    if (batch == 1 && cu >= 0)
+      prefetch_warp_tiles(sh, cache, layer, b, h, split_ctas(plan, sh.ntiles, sh.ntiles), warp, NW, cu, sh.kbits, VB);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
   const int nchunk = lay.chunk_base[ng - 1] + ((lay.size[ng - 1] + 15) >> 4);
   constexpr int kFragPerThread = (kFragEntries + NT - 1) / NT;
-  uint4 fr[kFragPerThread];
-  if (qrot == nullptr && cu >= 0) {
-    const uint4* src = frag_block(sh, ws, li, b, h, hb);
-#pragma unroll
-    for (int i = 0; i < kFragPerThread; ++i) {
-      const int u = tid + i * NT;
-      if (u < 32 * nchunk) fr[i] = src[u];
-    }
-  }
   // the packed positions attended: [lo, len); lo > 0 when the caller keeps the
   // first positions unquantised (out-of-range values are flagged by the
   // combine kernel)
@@ -768,6 +780,45 @@ __global__ void __launch_bounds__(NW * 32, NW == kDecWarps ? kDecMinBlocks : 1)
   float* part_base = ws.partials +
                      (((static_cast<size_t>(li) * sh.max_batch + b) * sh.n_q_heads + h * G + h0) * sh.max_splits + cu) *
                          kPartialStride;
+  TileSource src;
+  src.sh = sh;
+  src.cache = cache;
+  src.err = ws.err;
+  src.layer = layer;
+  src.b = b;
+  src.h = h;
+  src.tlo = tlo;
+  src.wu = wu;
+  src.W = W;
+  src.kwords = 256 * sh.kbits;
+  src.vwords = 256 * VB;
+  src.kstage = stage_base + static_cast<size_t>(warp) * DL.kst_bytes;
+  src.kstride = NW * DL.kst_bytes;
+  src.vbuf = stage_base + kStages * NW * DL.kst_bytes + static_cast<size_t>(warp) * DL.v_bytes;
+  src.bars = bars + warp * kBarsPerWarp;
+  bool first_issued = false;
+  if (early) {
+    const int64_t p0 = static_cast<int64_t>(tlo + wu) * kTile;
+    bool appended = false;  // the first tile holds a row the preparation appends
+    if (plan.app_start != nullptr) {
+      const int as = __ldcg(plan.app_start + b), ac = __ldcg(plan.app_count + b);
+      appended = ac > 0 && p0 < static_cast<int64_t>(as) + ac && static_cast<int64_t>(as) < p0 + kTile;
+    }
+    first_issued = my_tiles > 0 && !appended;
+    if (lane == 0 && first_issued) issue_first(src, my_tiles);
+    prefetch_next_tiles(src, my_tiles);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
+  // the unit's q~ fragments (written by the query rotation)
+  uint4 fr[kFragPerThread];
+  if (qrot == nullptr) {
+    const uint4* fsrc = frag_block(sh, ws, li, b, h, hb);
+#pragma unroll
+    for (int i = 0; i < kFragPerThread; ++i) {
+      const int u = tid + i * NT;
+      if (u < 32 * nchunk) fr[i] = fsrc[u];
+    }
+  }
   const size_t part_head_stride = static_cast<size_t>(sh.max_splits) * kPartialStride;
   {
     if (qrot == nullptr) {
@@ -814,23 +865,7 @@ __global__ void __launch_bounds__(NW * 32, NW == kDecWarps ? kDecMinBlocks : 1)
   __syncthreads();
 
   // ---- per-warp pipeline over this warp's tiles ----
-  TileSource src;
-  src.sh = sh;
-  src.cache = cache;
-  src.err = ws.err;
-  src.layer = layer;
-  src.b = b;
-  src.h = h;
-  src.tlo = tlo;
-  src.wu = wu;
-  src.W = W;
-  src.kwords = 256 * sh.kbits;
-  src.vwords = 256 * VB;
-  src.kstage = stage_base + static_cast<size_t>(warp) * DL.kst_bytes;
-  src.kstride = NW * DL.kst_bytes;
-  src.vbuf = stage_base + kStages * NW * DL.kst_bytes + static_cast<size_t>(warp) * DL.v_bytes;
-  src.bars = bars + warp * kBarsPerWarp;
-  if (lane == 0) issue_first(src, my_tiles);
+  if (lane == 0 && !first_issued) issue_first(src, my_tiles);
   TileTables tt{grp, tabk, pdesc, bq, ng};
   float O[8][4], m_run[2], l_run[2];
   const int failed_at = attend_tiles<VB>(src, tt, tv, my_tiles, len, lo, O, m_run, l_run);

@@ -164,7 +164,16 @@ struct SplitPlan {
   int32_t fixed_tiles;
   int32_t units_per_seq;  // layer_count * Hkv * head blocks
   int32_t cluster;        // > 1: counts rounded up to whole clusters of this size (the fused decode)
-  int32_t pad;
+  // 1: the split pass follows the call's own query rotation (or decode-step
+  // preparation), which lets it start only once everything earlier in the
+  // stream has completed; it then reads the caller's lengths and issues its
+  // first tiles' copies before its dependency wait.
+  int32_t early;
+  // the rows the preparation kernel appends in the same launch as the
+  // rotation ([start, start + count) per sequence; null: none): a first
+  // tile holding one of them is copied only after the wait
+  const int32_t* app_start;
+  const int32_t* app_count;
 };
 
 // The split pass over the packed positions [pos_lo, seq_lens) (buf.pos_lo;

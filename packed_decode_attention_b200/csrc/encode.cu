@@ -460,8 +460,6 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   const int li = bx / (sh.n_kv_heads * batch);
   const int layer = layer0 + li;
   const int lh = layer * sh.n_kv_heads + h;
-  // the next kernel of the stream may start its own table-only set-up now
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the kind's rotation (transposed, [in][out]) in shared memory, all loads
   // in flight; a library table, read before the inputs are ready
   {
@@ -495,6 +493,9 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   // Launched as a programmatic dependent of the previous kernel of the
   // stream: the call's inputs and the cache are read after it has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Only now may the next kernel start: it then relies on all earlier work
+  // of the stream having completed (see SplitPlan::early).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // this row's values (row < n: inside the input whatever count is) and the
   // sequence's start and count, all in flight together; record order:
   // position i holds dim perm[i] (K), V keeps the dims
@@ -628,8 +629,6 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
 __device__ __forceinline__ void rotate_body(const Shape& sh, const Workspace& ws, int layer0,
                                             const __half* __restrict__ q, int batch, float* __restrict__ qrot,
                                             int bx) {
-  // the decode kernel that follows may start its own set-up now
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int hq = bx % sh.n_q_heads;
   const int b = (bx / sh.n_q_heads) % batch;
   const int li = bx / (sh.n_q_heads * batch);
@@ -648,6 +647,9 @@ __device__ __forceinline__ void rotate_body(const Shape& sh, const Workspace& ws
   // Launched as a programmatic dependent of the previous kernel of the
   // stream: the query is read after it has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Only now may the decode kernel that follows start: it then relies on all
+  // earlier work of the stream having completed (see SplitPlan::early).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid < kD) qp[tid] = __half2float(q[row * kD + lay.perm[tid]]);
   __syncthreads();
   float sacc = 0.f;

@@ -33,8 +33,10 @@ pytestmark = pytest.mark.gpu
 SAMPLES = {
     # (layer, sequence) pairs checked against the oracle; all KV heads of each
     "llama": [(0, 0)],
-    "qwen3b": [(0, 0), (35, 0)],
-    "batch": [(0, 0), (27, 15)],
+    "qwen3b": [(0, 0), (17, 0), (35, 0)],
+    # the ragged batch: its first and last sequences, the shortest (1), the
+    # longest (10) and two of middle length (4, 7)
+    "batch": [(0, 0), (20, 1), (9, 4), (13, 7), (5, 10), (27, 15)],
     "long": [(35, 0)],
 }
 

@@ -41,7 +41,7 @@
  *    is current.
  *  - A state is not thread-safe: call it from one host thread at a time.
  *    Its decode calls share the workspace's scratch (rotated queries, split
- *    partials, the combine's counters), so two of its calls must not overlap
+ *    partials, arrival counters), so two of its calls must not overlap
  *    on the GPU: issue them on one stream, or order the streams.
  *
  * Cache layout inside d_cache (offsets from bgtq_cache_offsets, each
@@ -341,7 +341,10 @@ int bgtq_decode_step_buffered(bgtq_state* st, int32_t layer, int32_t layer_count
  * rotated queries d_qrot (fp32 [layer_count][batch][n_q_heads][128], as
  * written by bgtq_rotate_query) into the workspace's partials, and
  * bgtq_decode_combine merges them into d_out.  Both must see the same
- * layer, layer_count, batch and split setting.  ASYNC. */
+ * layer, layer_count, batch, split setting and length values.  The combine
+ * reads d_seq_lens as soon as the work queued before it on the stream lets
+ * it start, so it must follow its bgtq_decode_split on the stream with no
+ * kernel of the caller's in between.  ASYNC. */
 int bgtq_decode_split(bgtq_state* st, int32_t layer, int32_t layer_count, const float* d_qrot,
                       const int32_t* d_seq_lens, int32_t batch, void* stream);
 int bgtq_decode_combine(bgtq_state* st, int32_t layer, int32_t layer_count, const int32_t* d_seq_lens,

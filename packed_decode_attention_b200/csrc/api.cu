@@ -96,8 +96,8 @@ int validate_config(const bgtq_config* c) {
 
 struct Layout {
   size_t krec, knorm, vrec, vnorm, cache_total;
-  size_t err, codebook, layouts, dectab, mkt, mvt, mv, energy_q, energy_k, qrot, qfrag, partials, comb_mid, comb_count,
-      ws_total;
+  size_t err, codebook, layouts, dectab, mkt, mvt, mv, rb, energy_q, energy_k, qrot, qfrag, partials, comb_mid,
+      comb_count, ws_total;
 };
 
 int64_t tiles_of(const bgtq_config* c) { return (c->capacity_tokens + bgtq::kTile - 1) / bgtq::kTile; }
@@ -129,7 +129,8 @@ Layout plan(const bgtq_config* c) {
   p.mkt = align_up(p.dectab + lh * sizeof(bgtq::DecodeTableDev));
   p.mvt = align_up(p.mkt + lh * kD * kD * sizeof(float));
   p.mv = align_up(p.mvt + lh * kD * kD * sizeof(float));
-  p.energy_q = align_up(p.mv + lh * kD * kD * sizeof(float));
+  p.rb = align_up(p.mv + lh * kD * kD * sizeof(float));
+  p.energy_q = align_up(p.rb + lh * 2 * 2 * kD * kD * sizeof(uint16_t));
   p.energy_k = align_up(p.energy_q + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
   p.qrot = align_up(p.energy_k + size_t(bgtq::kEnergyChunks) * lh * 64 * 16);
   const size_t qrows = size_t(c->n_layers) * c->max_batch * c->n_q_heads;
@@ -216,6 +217,7 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   std::vector<bgtq::LayoutDev> ldev(size_t(L) * H);
   std::vector<bgtq::DecodeTableDev> dtab(size_t(L) * H);
   std::vector<float> mkt(size_t(L) * H * kD * kD, 0.f), mvt(size_t(L) * H * kD * kD), mv(size_t(L) * H * kD * kD);
+  std::vector<__half> rb(size_t(L) * H * 2 * 2 * kD * kD);
   for (int l = 0; l < L; ++l) {
     for (int h = 0; h < H; ++h) {
       const size_t lh = size_t(l) * H + h;
@@ -268,6 +270,22 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
           vv[i * kD + j] = v;
           vt[j * kD + i] = v;
         }
+      // the tensor-core encode's operands: per kind, element (out i, in d) =
+      // R[i][inv(d)] (inputs in the rows' dimension order), as fp16 hi and
+      // lo = fp16(value - hi)
+      for (int kind = 0; kind < 2; ++kind) {
+        __half* hi = rb.data() + (lh * 2 + kind) * 2 * kD * kD;
+        __half* lo = hi + kD * kD;
+        for (int j = 0; j < kD; ++j) {
+          const int d = kind == 0 ? lay.perm[j] : j;
+          for (int i = 0; i < kD; ++i) {
+            const float v = kind == 0 ? mk[size_t(j) * kD + i] : vt[size_t(j) * kD + i];
+            const __half h16 = __float2half_rn(v);
+            hi[size_t(i) * kD + d] = h16;
+            lo[size_t(i) * kD + d] = __float2half_rn(v - __half2float(h16));
+          }
+        }
+      }
     }
   }
   for (size_t i = 0; i < ldev.size(); ++i) dtab[i] = decode_table(ldev[i], c.v_avg_bits);
@@ -279,6 +297,7 @@ int build_and_upload(bgtq_state* st, cudaStream_t stream) {
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mkt, mkt.data(), mkt.size() * 4, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mvt, mvt.data(), mvt.size() * 4, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.mv, mv.data(), mv.size() * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(st->ws.rb, rb.data(), rb.size() * 2, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return BGTQ_ERR_CUDA;
   st->ready = true;
@@ -396,6 +415,7 @@ int bgtq_create(const bgtq_config* cfg, void* d_cache, size_t cache_bytes, void*
   st->ws.mkt = reinterpret_cast<float*>(w8 + p.mkt);
   st->ws.mvt = reinterpret_cast<float*>(w8 + p.mvt);
   st->ws.mv = reinterpret_cast<float*>(w8 + p.mv);
+  st->ws.rb = reinterpret_cast<__half*>(w8 + p.rb);
   st->ws.energy_q = reinterpret_cast<unsigned __int128*>(w8 + p.energy_q);
   st->ws.energy_k = reinterpret_cast<unsigned __int128*>(w8 + p.energy_k);
   st->ws.dectab = reinterpret_cast<bgtq::DecodeTableDev*>(w8 + p.dectab);
@@ -876,7 +896,8 @@ int bgtq_logit_mae(bgtq_state* st, int32_t layer, int32_t layer_count, int32_t s
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_static_scratch[BGTQ_STATIC_SCRATCH_BYTES];
 
-// Bytes at the start of the static array for the combine's arrival counters.
+// Bytes at the start of the static array for the arrival counters (the
+// fused decode's; the split pass and combine leave them unused).
 constexpr size_t kStaticCountBytes = 64 << 10;
 
 namespace {
@@ -934,9 +955,8 @@ int bgtq_decode_attn_static_scratch(bgtq_state* st, int32_t layer, int32_t layer
   }
   const bgtq::SplitPlan split = after_prep(split_for(st, layer_count, batch));
   const int64_t nspl = split.c_max;
-  // the combine's arrival counters first, at a fixed place (they are 0
-  // between calls, whatever the call's layout), then q~, its fragments, the
-  // split partials and the combine's slice merges
+  // the arrival counters' place first (as for the fused decode), then q~,
+  // its fragments, the split partials and the combine's intermediates
   const size_t count_bytes = kStaticCountBytes;
   const size_t qrot_bytes = rows * kD * sizeof(float);
   const size_t fbytes = frag_bytes(&st->cfg, layer_count);

@@ -45,9 +45,6 @@ constexpr int kDecMinBlocks = 4;  // CTAs per SM the register budget is sized fo
 constexpr int kWaitLimit = 1 << 20;  // polls of up to kPollSuspendNs each: about a second
 constexpr float kRescaleSlack = 8.f;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -216,7 +213,7 @@ __device__ int64_t batch_tiles(const Shape& sh, const int32_t* seq_lens, const B
 // heads), attended by one extra CTA of the split pass (128 threads): logits
 // q . k / sqrt(D) in log2 units (a thread per row), softmax per head, P v (a
 // thread per dimension, unrotated).  Each head's (m, l, acc) goes to the
-// row's extra combine intermediate, which then counts as arrived.
+// row's extra combine intermediate, read by the combine after this grid.
 // NT threads (128 or more): the P v part runs on the first 128.
 template <int NT>
 __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const BufferArgs& buf, const SeqRange& sr, int li,
@@ -341,11 +338,6 @@ __device__ void buffer_attend(const Shape& sh, const Workspace& ws, const Buffer
       mid[1] = cnt > 0 ? ml[2 * hh + 1] : 0.f;
     }
   }
-  __threadfence();
-  __syncthreads();
-  // the combine of a row with no packed position and no buffered row writes
-  // zeros without counting arrivals: do not count this one either
-  if (tid < nh && !(sr.lo >= sr.len && cnt == 0)) atomicAdd(ws.comb_count + wrow0 + tid, 1u);
 }
 
 // ---------------------------------------------------------------------------
@@ -1350,27 +1342,29 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 
 // ---------------------------------------------------------------------------
 // Combine the splits and rotate back.  Grid (layer_count*batch*Hq *
-// kCombSlices), 256 threads.  Each CTA merges one slice of a row's splits
-// (w_s = 2^(m_s - M), 0 for empty splits; lane = 4 rotated coordinates) into
-// an intermediate (m, l, acc) in V's rotated basis.  In a buffered call the
-// split pass has already posted the row's fp16 buffered rows as one more
-// intermediate (acc unrotated).  The row's last CTA to finish (an arrival
-// counter, reset by that CTA) merges them:
+// kCombSlices), 256 threads, in clusters of kCombSlices CTAs: one cluster
+// per row.  CTA (slice) r merges slice r of the row's splits (w_s = 2^(m_s -
+// M), 0 for empty splits; lane = 4 rotated coordinates) into an
+// intermediate (m, l, acc) in V's rotated basis in its shared memory.  CTA 0
+// then reads the cluster's intermediates through distributed shared memory
+// (and, in a buffered call, the row's fp16 buffered rows, which the split
+// pass posted to global memory with acc unrotated) and computes
 // o = (R_V^T sum_s w_s acc_s + w_buf acc_buf) / (sum_s w_s l_s + w_buf l_buf).
 // ---------------------------------------------------------------------------
 constexpr int kCombThreads = 256;
 constexpr int kCombWarps = kCombThreads / 32;
-// Up to this many rows per launch, every combine CTA loads its rotation
-// column early (8 slices x 64 KB per row of L2 reads).
+// Up to this many rows per launch, CTA 0 of every row loads its rotation
+// column before the dependency wait (64 KB per row of L2 reads).
 constexpr int kEarlyRotationRows = 256;
 static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates four at a time");
+static_assert(kCombSlices <= 8, "a row's slices form one portable cluster");
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
                                                                SplitPlan plan, BufferArgs buf, __half* __restrict__ out,
                                                                bool early_rotation) {
   const int has_buf = buf.k != nullptr ? 1 : 0;
-  const int slice = blockIdx.x % kCombSlices;
+  const int slice = blockIdx.x % kCombSlices;  // the CTA's rank in its cluster
   const int rowi = blockIdx.x / kCombSlices;
   const int hq = rowi % sh.n_q_heads;
   const int b = (rowi / sh.n_q_heads) % batch;
@@ -1380,24 +1374,27 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int dd = tid & (kD - 1), half = tid >> 7;
   // A library table: this thread's half column of the inverse V rotation,
-  // used if this CTA merges the row.  For a small launch every CTA reads it
-  // before the split pass has finished, off the critical path; for a large
-  // one (many layers per call) only the merging CTAs do, later.
+  // used by the row's CTA 0.  For a small launch it is read before the
+  // split pass has finished, off the critical path.
   const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
   float mvr[64];
-  if (early_rotation) {
+  if (early_rotation && slice == 0) {
 #pragma unroll
     for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
   }
   // the next kernel of the stream may start its own table-only set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // Launched as a programmatic dependent of the split pass: inputs, partials
-  // and the output are touched only after that kernel has completed.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The split pass lets this grid start only after its own dependency wait,
+  // so the caller's lengths are complete: they are read before this grid's
+  // wait.  The partials and the output are touched only after it.
   const SeqRange sr = seq_range(sh, seq_lens, buf, b);
-  if (sr.bad && tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;
-  if (sr.lo >= sr.len && sr.cnt == 0) {
+  __shared__ int64_t s_red[kCombWarps];
+  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kCombThreads>(sh, seq_lens, buf, batch, s_red);
+  const int n_splits = split_ctas(plan, range_tiles(sr), total);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (sr.bad && tid == 0 && hq == 0 && slice == 0) atomicOr(ws.err, kErrSeqLen);
+  if (sr.lo >= sr.len && sr.cnt == 0) {  // the whole cluster: an empty row
     if (slice == 0 && tid < kD) out[row * kD + tid] = __float2half(0.f);
     return;
   }
@@ -1405,15 +1402,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   const float* part = ws.partials + wrow * sh.max_splits * kPartialStride;
   __shared__ float accs[kCombWarps][kD];
   __shared__ float msw[kCombWarps], lsw[kCombWarps];
+  __shared__ __align__(16) float cmid[4 + kD];  // this slice's (m, l, -, -, acc[128])
   __shared__ float a_s[kD];
-  __shared__ int last;
-  float* mid = ws.comb_mid + (wrow * (kCombSlices + 1) + slice) * kPartialStride;
   // ---- one slice of the row's splits: warp w takes splits s0 + w + 8 j,
   // four at a time with all their loads in flight, merged online per warp
   // (lane = 4 rotated coordinates), then across the warps ----
-  __shared__ int64_t s_red[kCombWarps];
-  const int64_t total = plan.fixed_tiles > 0 ? 0 : batch_tiles<kCombThreads>(sh, seq_lens, buf, batch, s_red);
-  const int n_splits = split_ctas(plan, range_tiles(sr), total);
   const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
   const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
   float m_w = -CUDART_INF_F, l_w = 0.f;
@@ -1468,63 +1461,64 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
         const float wgt = msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M);
         a = fmaf(wgt, accs[w][tid], a);
       }
-      mid[4 + tid] = a;
+      cmid[4 + tid] = a;
     }
     if (tid == 0) {
       float l = 0.f;
 #pragma unroll
       for (int w = 0; w < kCombWarps; ++w) l = fmaf(msw[w] == -CUDART_INF_F ? 0.f : exp2f(msw[w] - M), lsw[w], l);
-      mid[0] = M;
-      mid[1] = l;
+      cmid[0] = M;
+      cmid[1] = l;
     }
   }
-  // ---- the row's last CTA merges the intermediates ----
-  const int nmid = kCombSlices + has_buf;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last = atomicAdd(ws.comb_count + wrow, 1u) == static_cast<unsigned>(nmid - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  const float* mids = ws.comb_mid + wrow * (kCombSlices + 1) * kPartialStride;
-  float mk[kCombSlices + 1], lk[kCombSlices + 1], ak[kCombSlices + 1];
+  // every slice's intermediate is visible to the cluster's CTA 0
+  cluster_sync_all();
+  if (slice == 0) {
+    // ---- CTA 0 merges the cluster's intermediates (and the buffer's) ----
+    float mk[kCombSlices + 1], lk[kCombSlices + 1], ak[kCombSlices + 1];
 #pragma unroll
-  for (int k = 0; k <= kCombSlices; ++k) {
-    if (k < nmid) {
-      mk[k] = __ldcg(mids + k * kPartialStride);
-      lk[k] = __ldcg(mids + k * kPartialStride + 1);
-      ak[k] = __ldcg(mids + k * kPartialStride + 4 + dd);
+    for (int k = 0; k < kCombSlices; ++k) {
+      mk[k] = dsmem_ld(dsmem_addr(&cmid[0], k));
+      lk[k] = dsmem_ld(dsmem_addr(&cmid[1], k));
+      ak[k] = dsmem_ld(dsmem_addr(&cmid[4 + dd], k));
+    }
+    if (has_buf) {
+      const float* bm = ws.comb_mid + (wrow * (kCombSlices + 1) + kCombSlices) * kPartialStride;
+      mk[kCombSlices] = __ldcg(bm);
+      lk[kCombSlices] = __ldcg(bm + 1);
+      ak[kCombSlices] = __ldcg(bm + 4 + dd);
     } else {
-      mk[k] = -CUDART_INF_F;
-      lk[k] = 0.f;
-      ak[k] = 0.f;
+      mk[kCombSlices] = -CUDART_INF_F;
+      lk[kCombSlices] = 0.f;
+      ak[kCombSlices] = 0.f;
     }
+    float Mt = -CUDART_INF_F;
+#pragma unroll
+    for (int k = 0; k <= kCombSlices; ++k) Mt = fmaxf(Mt, mk[k]);
+    float Lt = 0.f, at = 0.f, ab = 0.f;
+#pragma unroll
+    for (int k = 0; k <= kCombSlices; ++k) {
+      const float w = mk[k] == -CUDART_INF_F ? 0.f : exp2f(mk[k] - Mt);
+      Lt = fmaf(w, lk[k], Lt);
+      if (k < kCombSlices) at = fmaf(w, ak[k], at);  // rotated basis
+      else ab = w * ak[k];                            // the buffer's rows, unrotated
+    }
+    if (tid < kD) a_s[tid] = at / Lt;
+    if (!early_rotation) {
+#pragma unroll
+      for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+    }
+    __syncthreads();
+    // inverse V rotation: two threads per output, half of the inputs each
+    float o = 0.f;
+#pragma unroll
+    for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
+    if (half == 1) accs[0][dd] = o;
+    __syncthreads();
+    if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
   }
-  float Mt = -CUDART_INF_F;
-#pragma unroll
-  for (int k = 0; k <= kCombSlices; ++k) Mt = fmaxf(Mt, mk[k]);
-  float Lt = 0.f, at = 0.f, ab = 0.f;
-#pragma unroll
-  for (int k = 0; k <= kCombSlices; ++k) {
-    const float w = mk[k] == -CUDART_INF_F ? 0.f : exp2f(mk[k] - Mt);
-    Lt = fmaf(w, lk[k], Lt);
-    if (k < kCombSlices) at = fmaf(w, ak[k], at);  // rotated basis
-    else ab = w * ak[k];                            // the buffer's rows, unrotated
-  }
-  if (tid < kD) a_s[tid] = at / Lt;
-  if (tid == 0) ws.comb_count[wrow] = 0u;  // ready for the next call
-  if (!early_rotation) {
-#pragma unroll
-    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
-  }
-  __syncthreads();
-  // inverse V rotation: two threads per output, half of the inputs each
-  float o = 0.f;
-#pragma unroll
-  for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
-  if (half == 1) accs[0][dd] = o;
-  __syncthreads();
-  if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
+  // the other CTAs keep their shared memory until CTA 0 has read it
+  cluster_sync_all();
 }
 
 // Warps per CTA of the split pass (several CTAs per SM: a CTA that finishes
@@ -1674,10 +1668,23 @@ cudaError_t launch_decode_split(const Shape& s, const Workspace& ws, const Cache
 cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int layer_count,
                            const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
                            __half* out, cudaStream_t stream) {
-  const int nsl = kCombSlices;  // the buffered rows, if any, come from the split pass
   const int rows = layer_count * batch * s.n_q_heads;
-  return launch_dependent(combine_kernel, dim3(rows * nsl), dim3(kCombThreads), 0, stream, s, ws, layer0, seq_lens,
-                          batch, plan, buf, out, rows <= kEarlyRotationRows);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows * kCombSlices);
+  cfg.blockDim = dim3(kCombThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;  // a row's slices
+  at[1].val.clusterDim.x = kCombSlices;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, s, ws, layer0, seq_lens, batch, plan, buf, out,
+                            rows <= kEarlyRotationRows);
 }
 
 }  // namespace bgtq

@@ -65,14 +65,17 @@ struct Workspace {
   float* mkt;                    // [L][Hkv][128 in][128 out]: K rotation, block diagonal in record order, transposed
   float* mvt;                    // [L][Hkv][128 in][128 out]: V rotation transposed
   float* mv;                     // [L][Hkv][128 out][128 in]: V rotation (for the inverse rotation)
+  __half* rb;                    // [L][Hkv][K, V][hi, lo][128 out][128 in, the rows' dimension order]: the
+                                 // rotations as fp16 hi + lo operands of the tensor-core encode
   unsigned __int128* energy_q;   // [kEnergyChunks][L][Hkv][64]
   unsigned __int128* energy_k;   // [kEnergyChunks][L][Hkv][64]
   DecodeTableDev* dectab;        // [L][Hkv]
   float* qrot;                   // [L][B][Hq][128]
   uint4* qfrag;                  // [L][B][Hkv][head blocks][kFragEntries]
   float* partials;               // [L][B][Hq][max_splits][kPartialStride]
-  float* comb_mid;               // [L][B][Hq][kCombSlices + 1][kPartialStride]: slice merges of the combine
-  uint32_t* comb_count;          // [L][B][Hq]: slices merged so far (0 between calls)
+  float* comb_mid;               // [L][B][Hq][kCombSlices + 1][kPartialStride]: slot kCombSlices holds a
+                                 // buffered call's fp16-row intermediate
+  uint32_t* comb_count;          // [L][B][Hq]: the fused decode's clusters merged so far (0 between calls)
 };
 
 // Cache arrays; T = ceil(capacity / 64) tiles per (layer, sequence, KV head).

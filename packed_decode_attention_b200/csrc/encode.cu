@@ -2,7 +2,10 @@
 // (B200, sm_100a):
 //
 //   energy_kernel        label-free per-RoPE-block Q/K energy, exact 128-bit sums
-//   encode_kernel        TQ-MSE: rotate (fp32), normalise (fp64), quantise, pack tiles
+//   encode_tc_kernel     TQ-MSE: rotate (tensor cores, fp16 rows x fp16 hi + lo
+//                        rotation, fp32 accumulation), normalise (fp64),
+//                        quantise, pack tiles
+//   encode_kernel<true>  the same for K rows turned by RoPE on load (fp32 rotation)
 //   append_kernel        the same for a few rows: patch only their code bits
 //   rotate_query_kernel  q~ per width group (rotated basis, 1/sqrt(d_g), 1/sqrt(D))
 //   prep_kernel          a decode step's appends and query rotation in one launch
@@ -87,6 +90,21 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
 // n, code = #{thresholds <= u}) into the codes, and packs the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
+// fp16 per shared row of the tensor-core encode's operands: 272 bytes, so
+// the 8 rows of an ldmatrix hit distinct banks
+constexpr int kTcPitch = kD + 8;
+// Dynamic shared memory of an append CTA: the rotation as fp16 hi + lo
+// operand rows, or in fp32 for rows turned by RoPE
+constexpr size_t append_smem_bytes(bool turn) {
+  return turn ? kD * kD * sizeof(float) : 2 * kD * kTcPitch * sizeof(__half);
+}
+
+__device__ __forceinline__ void ldmatrix_x4(const void* row_addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                            uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(row_addr)));
+}
 constexpr int kEncTilesPerCta = 8;  // tiles a CTA encodes with one load of its rotation
 // Column of element (coordinate j, row r) in xt[j][]: float4 groups of 4 rows,
 // XOR-swizzled by j so that the transposed writes spread over the banks.
@@ -389,6 +407,234 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(Shape sh, Workspace
 }
 
 // ---------------------------------------------------------------------------
+// Encode with the rotation on the tensor cores, for rows taken as they are
+// (no RoPE turn; encode_kernel<true> keeps that path): the same tiles, norms
+// and codes as encode_kernel.  Per tile, Y = X B with X[64 rows][128 dims]
+// and B[d][i] = R[i][inv(d)] (R in record order, its inputs taken back to
+// the dimension order of the rows), as mma.sync m16n8k16: X in fp16 (the
+// inputs are fp16, so exact) and B split into fp16 hi + lo, two MMAs per
+// product, fp32 accumulation.  Warp w computes rows 16 (w & 3) .. + 15 and
+// record positions 64 (w >> 2) .. + 63; the codes follow from u = y sqrt(d)
+// / n as before.
+// ---------------------------------------------------------------------------
+// The (layer, KV head, kind)'s fp16 hi / lo rotation operands (a library
+// table, [out][in] rows of 256 bytes) into shared rows of kTcPitch: bh at
+// dst, bl right after it.
+__device__ __forceinline__ void stage_rotation_operands(const Workspace& ws, int lh, int kind, __half* dst, int tid,
+                                                        int nthreads) {
+  const uint4* src = reinterpret_cast<const uint4*>(ws.rb + (static_cast<size_t>(lh) * 2 + kind) * 2 * kD * kD);
+#pragma unroll 4
+  for (int u = tid; u < 2 * kD * kD / 8; u += nthreads) {
+    const int row = u >> 4, c = u & 15;  // row of hi (0..127) then lo (128..255), 8 inputs
+    *reinterpret_cast<uint4*>(dst + row * kTcPitch + 8 * c) = __ldg(src + u);
+  }
+}
+
+struct EncodeTcSmem {
+  __half x[kTile][kTcPitch];   // the tile's new rows in dimension order (zero elsewhere)
+  __half bh[kD][kTcPitch];     // bh[i][d] = fp16(R[i][inv(d)])
+  __half bl[kD][kTcPitch];     // bl[i][d] = fp16(R[i][inv(d)] - bh[i][d])
+  float fac[kTile][kNumGroupsMax];
+  __half nrm[kTile][kNumGroupsMax];
+  uint8_t codes[kTile][kCodePitch];
+  uint32_t words[1024];
+  float thr[5][16];
+  int32_t perm[kD];            // record position -> dimension
+  int32_t gof[kD];             // group of each record position (-1: width 0)
+  LayoutDev lay;
+};
+
+__global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Workspace ws, CacheDev cache, int layer0,
+                                                                   const __half* __restrict__ kx,
+                                                                   const __half* __restrict__ vx,
+                                                                   const int32_t* __restrict__ start_v,
+                                                                   const int32_t* __restrict__ count_v, int batch,
+                                                                   int n) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  EncodeTcSmem& S = *reinterpret_cast<EncodeTcSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kind = blockIdx.z;
+  const int h = blockIdx.x % sh.n_kv_heads;
+  const int b = (blockIdx.x / sh.n_kv_heads) % batch;
+  const int li = blockIdx.x / (sh.n_kv_heads * batch);
+  const int layer = layer0 + li;
+  const int start = start_v[b];
+  const int count = count_v[b];
+  if (start < 0 || count < 0 || count > n) {
+    if (tid == 0 && blockIdx.y == 0 && kind == 0) atomicOr(ws.err, kErrArg);
+    return;
+  }
+  if (count == 0) return;
+  int64_t p_end = static_cast<int64_t>(start) + count;  // rows land at [start, p_end)
+  if (p_end > sh.capacity) {
+    if (tid == 0 && blockIdx.y == 0) atomicOr(ws.err, kErrCapacity);
+    p_end = sh.capacity;
+  }
+  const int64_t t_first = start / kTile;
+  if (t_first + blockIdx.y >= (p_end + kTile - 1) / kTile) return;  // no tile for this CTA
+  const int bits_avg = kind == 0 ? sh.kbits : sh.vbits;
+  const int nwords = 256 * bits_avg;
+  const int lh = layer * sh.n_kv_heads + h;
+  if (kind == 0) {
+    if (tid < static_cast<int>(sizeof(LayoutDev) / 4))
+      reinterpret_cast<int32_t*>(&S.lay)[tid] = reinterpret_cast<const int32_t*>(ws.layouts + lh)[tid];
+  } else if (tid == 0) {
+    S.lay.n_groups = 1;
+    S.lay.n_positions = kD;
+    for (int g = 0; g < kNumGroupsMax; ++g) {
+      S.lay.width[g] = g == 0 ? sh.vbits : 0;
+      S.lay.size[g] = g == 0 ? kD : 0;
+      S.lay.start[g] = g == 0 ? 0 : kD;
+      S.lay.bitoff[g] = 0;
+      S.lay.tile_word[g] = 0;
+      S.lay.chunk_base[g] = 0;
+    }
+  }
+  for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
+  __syncthreads();
+  const int ng = S.lay.n_groups;
+  const int npos = S.lay.n_positions;
+  if (tid < kD) {
+    S.perm[tid] = kind == 0 ? S.lay.perm[tid] : tid;
+    int g = -1;
+    if (tid < npos) {
+      g = 0;
+      for (int t = 1; t < ng; ++t)
+        if (tid >= S.lay.start[t]) g = t;
+    }
+    S.gof[tid] = g;
+  }
+  __syncthreads();
+  stage_rotation_operands(ws, lh, kind, &S.bh[0][0], tid, kEncThreads);
+  __syncthreads();
+  const int mt = warp & 3, nh = warp >> 2;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const int lrow = lane & 7, lmat = lane >> 3;  // ldmatrix: this lane's row and matrix
+  // ---- this CTA's tiles: t_first + blockIdx.y, then every gridDim.y-th ----
+  for (int64_t tile = t_first + blockIdx.y; tile * kTile < p_end; tile += gridDim.y) {
+    const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
+    const int64_t p1 = min(tile * kTile + kTile, p_end);
+    const int tr0 = static_cast<int>(p0 - tile * kTile), tr1 = static_cast<int>(p1 - tile * kTile);
+    const bool whole = (tr0 == 0 && tr1 == kTile);
+    if (p0 >= p1) continue;  // the first rows are past the capacity
+    const int64_t slot = tile_slot(sh, cache, layer, b, h, tile);
+    if (slot < 0) {  // uniform over the CTA
+      if (tid == 0) atomicOr(ws.err, kErrPage);
+      continue;
+    }
+    uint32_t* gtile = (kind == 0 ? cache.ktile : cache.vtile) + slot * nwords;
+    // existing codes of a partly written tile
+    if (!whole) {
+      if (kind == 0) {
+        for (int g = 0; g < ng; ++g) {
+          const GroupGeo q = group_geo(S.lay, g);
+          BGTQ_WIDTH_SWITCH(q.width, unpack_k_group, gtile, q, S.codes, tid, kEncThreads)
+        }
+      } else {
+        BGTQ_WIDTH_SWITCH(sh.vbits, unpack_v_tile, gtile, S.codes, tid, kEncThreads)
+      }
+    }
+    // new rows -> x (dimension order, 16-byte copies)
+    const size_t row_stride = static_cast<size_t>(sh.n_kv_heads) * kD;
+    const __half* x = kind == 0 ? kx : vx;
+    const __half* xbase = x + ((static_cast<size_t>(li) * batch + b) * n + (p0 - start)) * row_stride +
+                          static_cast<size_t>(h) * kD;
+    for (int e = tid; e < kTile * (kD / 8); e += kEncThreads) {
+      const int r = e >> 4, c8 = e & 15;  // row, 8 dims
+      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+      if (r >= tr0 && r < tr1) raw = *reinterpret_cast<const uint4*>(xbase + static_cast<size_t>(r - tr0) * row_stride + 8 * c8);
+      *reinterpret_cast<uint4*>(&S.x[r][8 * c8]) = raw;
+    }
+    __syncthreads();
+    // norms: fp64 sum of squares of the exact fp16 inputs of each group
+    {
+      const int r = tid >> 2, g = tid & 3;
+      float f = 0.f;
+      __half nh16 = __float2half(0.f);
+      if (g < ng && r >= tr0 && r < tr1) {
+        const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
+        double s2 = 0.0;
+        for (int j = j0; j < j1; ++j) {
+          const double v = __half2float(S.x[r][S.perm[j]]);
+          s2 += v * v;
+        }
+        const double nr = sqrt(s2);
+        nh16 = __double2half(nr);
+        f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;
+      }
+      S.fac[r][g] = f;
+      S.nrm[r][g] = nh16;
+    }
+    // y = X B for this warp's 16 rows and 64 record positions
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    const bool rows_touched = 16 * mt < tr1 && 16 * mt + 16 > tr0 && 64 * nh < npos;
+    if (rows_touched) {
+#pragma unroll 2
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        // matrices: rows +0 / +8 (lmat & 1), dims +0 / +8 (lmat >> 1)
+        ldmatrix_x4(&S.x[16 * mt + 8 * (lmat & 1) + lrow][16 * ks + 8 * (lmat >> 1)], a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          uint32_t h0, h1, l0, l1;
+          // matrices: hi dims +0, hi dims +8, lo dims +0, lo dims +8 (outputs n0 .. n0 + 7)
+          const int n0 = 64 * nh + 8 * nt;
+          const __half* brow = (lmat < 2 ? &S.bh[0][0] : &S.bl[0][0]) + (n0 + lrow) * kTcPitch + 16 * ks +
+                               8 * (lmat & 1);
+          ldmatrix_x4(brow, h0, h1, l0, l1);
+          mma16816(acc[nt], a0, a1, a2, a3, h0, h1);
+          mma16816(acc[nt], a0, a1, a2, a3, l0, l1);
+        }
+      }
+    }
+    __syncthreads();  // fac, nrm and the unpacked codes are in place
+    if (rows_touched) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = 16 * mt + g8 + 8 * (e >> 1);
+          const int i = 64 * nh + 8 * nt + 2 * t4 + (e & 1);
+          const int g = S.gof[i];
+          if (r < tr0 || r >= tr1 || g < 0) continue;
+          const int w = S.lay.width[g];
+          const float u = acc[nt][e] * S.fac[r][g];
+          S.codes[r][i] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
+        }
+      }
+    }
+    __syncthreads();
+    // repack the tile and write it back
+    if (kind == 0) {
+      for (int g = 0; g < ng; ++g) {
+        const GroupGeo q = group_geo(S.lay, g);
+        BGTQ_WIDTH_SWITCH(q.width, pack_k_group, S.words, q, S.codes, tid, kEncThreads)
+      }
+    } else {
+      BGTQ_WIDTH_SWITCH(sh.vbits, pack_v_tile, S.words, S.codes, tid, kEncThreads)
+    }
+    __syncthreads();
+    for (int i = tid; i < nwords / 4; i += kEncThreads)
+      reinterpret_cast<uint4*>(gtile)[i] = reinterpret_cast<const uint4*>(S.words)[i];
+    if (tid >= tr0 && tid < tr1) {
+      const size_t pos = static_cast<size_t>(slot) * kTile + tid;
+      if (kind == 0) {
+        __half2* dst = reinterpret_cast<__half2*>(cache.knorm + pos * 4);
+        dst[0] = __halves2half2(S.nrm[tid][0], S.nrm[tid][1]);
+        dst[1] = __halves2half2(S.nrm[tid][2], S.nrm[tid][3]);
+      } else {
+        cache.vnorm[pos] = S.nrm[tid][0];
+      }
+    }
+    __syncthreads();  // the buffers are reused by the next tile
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Encode for a few rows (decode-time appends): grid (layer_count * batch * Hkv,
 // n, 2 kinds), 128 threads.  A CTA encodes one new row of one (layer,
 // sequence, KV head) and kind with the same arithmetic as encode_kernel
@@ -460,9 +706,13 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   const int li = bx / (sh.n_kv_heads * batch);
   const int layer = layer0 + li;
   const int lh = layer * sh.n_kv_heads + h;
-  // the kind's rotation (transposed, [in][out]) in shared memory, all loads
-  // in flight; a library table, read before the inputs are ready
-  {
+  // the kind's rotation in shared memory, a library table read before the
+  // inputs are ready: as the tensor-core encode's fp16 hi / lo operands
+  // (rows as they come), or transposed in fp32 ([in][out]) for rows turned
+  // by RoPE here
+  if constexpr (!TURN) {
+    stage_rotation_operands(ws, lh, kind, reinterpret_cast<__half*>(mts), tid, NT);
+  } else {
     const uint4* src = reinterpret_cast<const uint4*>((kind == 0 ? ws.mkt : ws.mvt) + static_cast<size_t>(lh) * kD * kD);
 #pragma unroll 8
     for (int u = tid; u < kD * kD / 4; u += NT) reinterpret_cast<uint4*>(mts)[u] = __ldg(src + u);
@@ -555,11 +805,55 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   }
   int g = 0;
   float y = 0.f;
-  if (i < lay.n_positions) {
+  if (i < lay.n_positions)
     for (int t = 1; t < ng; ++t)
       if (i >= lay.start[t]) g = t;
-    const int j0 = lay.start[g], j1 = j0 + lay.size[g];
-    for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
+  if constexpr (!TURN) {
+    // y = R x on the tensor cores, exactly as the tile encode computes a
+    // row (the same operands and the same order of MMAs per output): the
+    // row is row 0 of the A tile (the others zero), warp w takes outputs
+    // 8 (w NTL) .. 8 (w NTL + NTL) - 1
+    __shared__ float ys[kD];
+    constexpr int NTL = kD / 8 / (NT / 32);
+    const int lane = tid & 31, warp = tid >> 5;
+    const int lrow = lane & 7, lmat = lane >> 3;
+    const __half* bh = reinterpret_cast<const __half*>(mts);
+    uint32_t xa[kD / 16][2];
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      xa[ks][0] = lane < 4 ? *reinterpret_cast<const uint32_t*>(x + 16 * ks + 2 * lane) : 0u;
+      xa[ks][1] = lane < 4 ? *reinterpret_cast<const uint32_t*>(x + 16 * ks + 8 + 2 * lane) : 0u;
+    }
+    float acc[NTL][4];
+#pragma unroll
+    for (int t = 0; t < NTL; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+#pragma unroll
+      for (int t = 0; t < NTL; ++t) {
+        const int n0 = 8 * (warp * NTL + t);
+        uint32_t h0, h1, l0, l1;
+        ldmatrix_x4(bh + ((lmat >> 1) * kD + n0 + lrow) * kTcPitch + 16 * ks + 8 * (lmat & 1), h0, h1, l0, l1);
+        mma16816(acc[t], xa[ks][0], 0u, xa[ks][1], 0u, h0, h1);
+        mma16816(acc[t], xa[ks][0], 0u, xa[ks][1], 0u, l0, l1);
+      }
+    }
+    if (lane < 4) {
+#pragma unroll
+      for (int t = 0; t < NTL; ++t) {
+        ys[8 * (warp * NTL + t) + 2 * lane] = acc[t][0];
+        ys[8 * (warp * NTL + t) + 2 * lane + 1] = acc[t][1];
+      }
+    }
+    __syncthreads();
+    if (i < lay.n_positions) y = ys[i];
+  } else {
+    if (i < lay.n_positions) {
+      const int j0 = lay.start[g], j1 = j0 + lay.size[g];
+      for (int j = j0; j < j1; ++j) y = fmaf(xs[j], mts[j * kD + i], y);
+    }
   }
   __syncthreads();
   const int tile = static_cast<int>(pos / kTile), p = static_cast<int>(pos % kTile);
@@ -620,7 +914,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(Shape sh, Workspace
                                                              const int32_t* __restrict__ start_v,
                                                              const int32_t* __restrict__ count_v, int batch, int n,
                                                              RopeArgs rope) {
-  extern __shared__ __align__(16) float mts[];  // [kD][kD]
+  extern __shared__ __align__(16) float mts[];  // the rotation (append_smem_bytes)
   append_body<kAppThreads, TURN>(sh, ws, cache, layer0, kx, vx, start_v, count_v, batch, n, blockIdx.x, blockIdx.y,
                                  blockIdx.z, mts, rope);
 }
@@ -689,7 +983,7 @@ __global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace w
                                                            const int32_t* __restrict__ start_v,
                                                            const int32_t* __restrict__ count_v, int n, int n_rot,
                                                            int n_units) {
-  extern __shared__ __align__(16) float mts[];  // [kD][kD], the append part
+  extern __shared__ __align__(16) float mts[];  // the append part's rotation (append_smem_bytes)
   if (static_cast<int>(blockIdx.x) < n_rot) {
     rotate_body(sh, ws, layer0, q, batch, qrot, blockIdx.x);
   } else {
@@ -700,7 +994,7 @@ __global__ void __launch_bounds__(kRotThreads) prep_kernel(Shape sh, Workspace w
 }
 
 cudaError_t encode_smem_once() {
-  static const cudaError_t status = set_smem(encode_kernel<false>, sizeof(EncodeSmem));
+  static const cudaError_t status = set_smem(encode_tc_kernel, sizeof(EncodeTcSmem));
   return status;
 }
 
@@ -711,7 +1005,7 @@ cudaError_t encode_rope_smem_once() {
 
 template <bool TURN>
 cudaError_t append_smem_once() {
-  static const cudaError_t status = set_smem(append_kernel<TURN>, kD * kD * sizeof(float));
+  static const cudaError_t status = set_smem(append_kernel<TURN>, append_smem_bytes(TURN));
   return status;
 }
 
@@ -742,9 +1036,9 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
     const cudaError_t attr = rope.on ? append_smem_once<true>() : append_smem_once<false>();
     if (attr != cudaSuccess) return attr;
     const dim3 agrid(layer_count * batch * s.n_kv_heads, n, 2);
-    return rope.on ? launch_dependent(append_kernel<true>, agrid, dim3(kAppThreads), kD * kD * sizeof(float), stream,
+    return rope.on ? launch_dependent(append_kernel<true>, agrid, dim3(kAppThreads), append_smem_bytes(true), stream,
                                       s, ws, cache, layer0, k, v, start, count, batch, n, rope)
-                   : launch_dependent(append_kernel<false>, agrid, dim3(kAppThreads), kD * kD * sizeof(float), stream,
+                   : launch_dependent(append_kernel<false>, agrid, dim3(kAppThreads), append_smem_bytes(false), stream,
                                       s, ws, cache, layer0, k, v, start, count, batch, n, rope);
   }
   // CTAs per unit: at least two waves if every unit has rows, and at most
@@ -767,19 +1061,19 @@ cudaError_t launch_encode(const Shape& s, const Workspace& ws, const CacheDev& c
     encode_kernel<true><<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count,
                                                                           batch, n, rope);
   else
-    encode_kernel<false><<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(s, ws, cache, layer0, k, v, start, count,
-                                                                           batch, n, rope);
+    encode_tc_kernel<<<grid, kEncThreads, sizeof(EncodeTcSmem), stream>>>(s, ws, cache, layer0, k, v, start, count,
+                                                                         batch, n);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const Shape& s, const Workspace& ws, const CacheDev& cache, int layer0, int layer_count,
                         const __half* q, int batch, float* qrot, const __half* k, const __half* v,
                         const int32_t* start, const int32_t* count, int n, cudaStream_t stream) {
-  static const cudaError_t attr = set_smem(prep_kernel, kD * kD * sizeof(float));
+  static const cudaError_t attr = set_smem(prep_kernel, append_smem_bytes(false));
   if (attr != cudaSuccess) return attr;
   const int n_rot = layer_count * batch * s.n_q_heads;
   const int n_units = layer_count * batch * s.n_kv_heads;
-  return launch_dependent(prep_kernel, dim3(n_rot + n_units * n * 2), dim3(kRotThreads), kD * kD * sizeof(float),
+  return launch_dependent(prep_kernel, dim3(n_rot + n_units * n * 2), dim3(kRotThreads), append_smem_bytes(false),
                           stream, s, ws, cache, layer0, q, batch, qrot, k, v, start, count, n, n_rot, n_units);
 }
 

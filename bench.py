@@ -358,6 +358,14 @@ def workload_config(w, lens):
             "parallelism": "replicas"}
 
 
+def host_overhead_hidden():
+    """Keeps the GPU busy (a ~1 ms spin) while the host issues the call timed
+    next, so that events around one eager call measure its kernels and not the
+    host-side argument checks in front of them."""
+    import torch
+    torch.cuda._sleep(2_000_000)
+
+
 def time_graph(fn, steps, warmup, world=1):
     """Average ms of one call of fn, captured as a CUDA graph and replayed
     `steps` times after `warmup` replays, CUDA events around the timed region.
@@ -494,8 +502,6 @@ def measure(w, args, dev, world, rank, full):
     kf = [torch.empty((B, cap, H, 128), dtype=torch.float16, device=dev) for _ in range(L)] if want_fp16 else None
     vf = [torch.empty((B, cap, H, 128), dtype=torch.float16, device=dev) for _ in range(L)] if want_fp16 else None
     chunk = w.encode_chunk or 32768  # rows per encode call: the long workload's 131072-row prefill chunk
-    enc_ms = 0.0
-    enc_rows = 0
     for l in range(L):
         for b in range(B):
             for s0 in range(0, lens[b], chunk):
@@ -511,14 +517,25 @@ def measure(w, args, dev, world, rank, full):
                 count = torch.zeros(B, dtype=torch.int32, device=dev)
                 start[b] = s0
                 count[b] = n
-                e0.record()
                 kv.encode_append(l, kk, vv, start, count)
-                e1.record()
-                torch.cuda.synchronize()
-                enc_ms += e0.elapsed_time(e1)
-                enc_rows += n * H
                 del kk, vv
+    torch.cuda.synchronize()
     assert kv.device_error() == 0, "device error after prefill"
+    # prefill rate: one prefill call (the first chunk of layer 0, sequence 0)
+    # encoded again -- the same rows, so the same bytes -- as a captured
+    # graph replayed back to back (the kernels only, without the host's
+    # argument checks)
+    n_p = min(chunk, lens[0])
+    kk = torch.zeros((1, B, n_p, H, 128), dtype=torch.float16, device=dev)
+    vv = torch.zeros_like(kk)
+    kk[0, 0] = wl.keys(w, 0, 0, 0, n_p, device=dev)
+    vv[0, 0] = wl.values(w, 0, 0, 0, n_p, device=dev)
+    st_p = torch.zeros(B, dtype=torch.int32, device=dev)
+    cnt_p = torch.zeros(B, dtype=torch.int32, device=dev)
+    cnt_p[0] = n_p
+    enc_call_ms, g_e, _ = time_graph(lambda: kv.encode_append(0, kk, vv, st_p, cnt_p), 5, 3)
+    del g_e, kk, vv
+    assert kv.device_error() == 0, "device error in the prefill re-encode"
 
     # ---- step inputs ----
     seq = torch.tensor(lens, dtype=torch.int32, device=dev)
@@ -610,8 +627,8 @@ def measure(w, args, dev, world, rank, full):
            "decode_path": "fused (one launch per decode call)" if fused else "query rotation + split + combine",
            "decode_wave_ctas": kv.decode_wave_ctas(),
            "gpu_launches": (2 if fused else 3) * L * steps,
-           "allocate_ms": alloc_ms, "prefill_encode_rows_per_s": enc_rows / (enc_ms * 1e-3),
-           "prefill_encode_call_rows": chunk,
+           "allocate_ms": alloc_ms, "prefill_encode_rows_per_s": n_p * H / (enc_call_ms * 1e-3),
+           "prefill_encode_call_rows": n_p, "prefill_encode_call_ms": enc_call_ms,
            "compression_vs_fp16": 512.0 / (sum(lens[b] * tb[l, h] for l in range(L) for b in range(B)
                                                 for h in range(H)) / (sum(lens) * L * H))}
 
@@ -653,8 +670,12 @@ def measure(w, args, dev, world, rank, full):
         ms_multi, g_m, _ = time_graph(step_multi, steps, warmup, world)
         del g_m
         ms_multi = max_over_ranks(ms_multi, world, dev)
+        ml_gbs = step_bytes / (ms_multi * 1e-3) / 1e9
         res["multi_layer"] = {"ms_per_step": ms_multi, "tokens_per_s": world * B / (ms_multi * 1e-3),
-                              "hbm_gbs": step_bytes / (ms_multi * 1e-3) / 1e9}
+                              "hbm_gbs": ml_gbs, "frac": ml_gbs / peak,
+                              "note": "the same step with all layers in one launch per kernel (appends, then "
+                                      "rotation + split + combine): the kernels without per-layer launch "
+                                      "granularity; a model cannot batch its layers like this"}
 
         # ---- fp16 sink + recent window (the README's "withbuffer" setting) ----
         SINK, WINDOW = 4, 128
@@ -764,6 +785,7 @@ def measure(w, args, dev, world, rank, full):
         mae_g = torch.zeros((L, HQ), dtype=torch.float64, device=dev)
         kv.logit_mae(0, 0, 0, qd, kd, mae_g, layer_count=L)
         torch.cuda.synchronize()
+        host_overhead_hidden()
         e0.record()
         kv.logit_mae(0, 0, 0, qd, kd, mae_g, layer_count=L)
         e1.record()
@@ -798,16 +820,10 @@ def measure(w, args, dev, world, rank, full):
     st0 = torch.zeros(B, dtype=torch.int32, device=dev)
     c0 = torch.zeros(B, dtype=torch.int32, device=dev)
     c0[0] = n_r
-    rope_ms = []
-    for it in range(4):
-        e0.record()
-        kv.encode_append(0, kk, kk, st0, c0, rope_base=w.rope_base)
-        e1.record()
-        torch.cuda.synchronize()
-        if it:
-            rope_ms.append(e0.elapsed_time(e1))
+    rope_ms, g_r, _ = time_graph(lambda: kv.encode_append(0, kk, kk, st0, c0, rope_base=w.rope_base), 5, 3)
+    del g_r
     assert kv.device_error() == 0, "device error in the fused RoPE + encode"
-    res["prefill_encode_rope_rows_per_s"] = n_r * H / (statistics.mean(rope_ms) * 1e-3)
+    res["prefill_encode_rope_rows_per_s"] = n_r * H / (rope_ms * 1e-3)
     del kk
     kv.close()
     del kv, q_all, knew, vnew, out, seq

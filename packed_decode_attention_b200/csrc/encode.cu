@@ -90,6 +90,28 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
 // n, code = #{thresholds <= u}) into the codes, and packs the tile again.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
+
+// Sum of squares of one (row, group) in fp64, in one fixed order shared by
+// the tile encode and the appends (rows as they come): eight partial sums
+// s_k over the positions j0 + k, j0 + k + 8, ... below j1, then
+// ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)).  The eight chains keep
+// the latency of the dependent adds off a thread's critical path; the
+// squares of fp16 inputs are exact in fp64.
+template <typename F>
+__device__ __forceinline__ double sum_squares(int j0, int j1, F value) {
+  double s[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
+  for (int j = j0; j < j1; j += 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (j + k < j1) {
+        const double v = value(j + k);
+        s[k] = fma(v, v, s[k]);
+      }
+    }
+  }
+  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+}
 // fp16 per shared row of the tensor-core encode's operands: 272 bytes, so
 // the 8 rows of an ldmatrix hit distinct banks
 constexpr int kTcPitch = kD + 8;
@@ -430,6 +452,31 @@ __device__ __forceinline__ void stage_rotation_operands(const Workspace& ws, int
   }
 }
 
+// The thresholds of width w spread over 15 ascending entries: the first
+// 2^(4-w) - 1 are -inf, then each threshold appears 2^(4-w) times.  Then
+// c = #{entries <= u} = 2^(4-w) (code + 1) - 1, so a branch-free 4-step
+// search serves every width: code16 returns #{thresholds <= u} (ties go up)
+// as lloyd_code does, and the width-4 sign-magnitude symbol.
+__device__ __forceinline__ void spread_thresholds(const float* thr, float (*thr16)[16], int tid, int nthreads) {
+  for (int u = tid; u < 5 * 16; u += nthreads) {
+    const int w = u >> 4, k = u & 15;
+    const int m = w > 0 ? 1 << (4 - w) : 1;
+    float t = CUDART_INF_F;  // entry 15 and width 0: never read
+    if (w > 0 && k < 15) t = k < m - 1 ? -CUDART_INF_F : thr[w * 16 + (k - (m - 1)) / m];
+    thr16[w][k] = t;
+  }
+}
+
+__device__ __forceinline__ int code16(const float* t16, int w, float u) {
+  int c = 0;
+#pragma unroll
+  for (int s = 8; s > 0; s >>= 1)
+    if (t16[c + s - 1] <= u) c += s;
+  int code = ((c + 1) >> (4 - w)) - 1;
+  if (w == 4) code = (code & 8) ? (code ^ 8) : (code ^ 15);
+  return code;
+}
+
 struct EncodeTcSmem {
   __half x[kTile][kTcPitch];   // the tile's new rows in dimension order (zero elsewhere)
   __half bh[kD][kTcPitch];     // bh[i][d] = fp16(R[i][inv(d)])
@@ -438,7 +485,7 @@ struct EncodeTcSmem {
   __half nrm[kTile][kNumGroupsMax];
   uint8_t codes[kTile][kCodePitch];
   uint32_t words[1024];
-  float thr[5][16];
+  float thr16[5][16];           // width w's thresholds spread to 15 entries (see code16)
   int32_t perm[kD];            // record position -> dimension
   int32_t gof[kD];             // group of each record position (-1: width 0)
   LayoutDev lay;
@@ -490,7 +537,7 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
       S.lay.chunk_base[g] = 0;
     }
   }
-  for (int i = tid; i < 5 * 16; i += kEncThreads) (&S.thr[0][0])[i] = (&ws.codebook->threshold[0][0])[i];
+  spread_thresholds(&ws.codebook->threshold[0][0], S.thr16, tid, kEncThreads);
   __syncthreads();
   const int ng = S.lay.n_groups;
   const int npos = S.lay.n_positions;
@@ -510,6 +557,17 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
   const int mt = warp & 3, nh = warp >> 2;
   const int g8 = lane >> 2, t4 = lane & 3;
   const int lrow = lane & 7, lmat = lane >> 3;  // ldmatrix: this lane's row and matrix
+  // this thread's 16 output positions i = 64 nh + 8 nt + 2 t4 + c (col =
+  // 2 nt + c): a byte each of group (bits 0..1) and width (bits 2..4), 0xFF
+  // for a position that holds no code
+  uint32_t colinfo[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int col = 0; col < 16; ++col) {
+    const int i = 64 * nh + 8 * (col >> 1) + 2 * t4 + (col & 1);
+    const int g = S.gof[i];
+    const uint32_t byte = g < 0 ? 0xFFu : static_cast<uint32_t>(g | (S.lay.width[g] << 2));
+    colinfo[col >> 2] |= byte << (8 * (col & 3));
+  }
   // ---- this CTA's tiles: t_first + blockIdx.y, then every gridDim.y-th ----
   for (int64_t tile = t_first + blockIdx.y; tile * kTile < p_end; tile += gridDim.y) {
     const int64_t p0 = max(tile * kTile, static_cast<int64_t>(start));
@@ -546,18 +604,16 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
       *reinterpret_cast<uint4*>(&S.x[r][8 * c8]) = raw;
     }
     __syncthreads();
-    // norms: fp64 sum of squares of the exact fp16 inputs of each group
+    // norms: fp64 sums of squares of the exact fp16 inputs of each group, a
+    // thread per (row, group)
     {
       const int r = tid >> 2, g = tid & 3;
       float f = 0.f;
       __half nh16 = __float2half(0.f);
       if (g < ng && r >= tr0 && r < tr1) {
-        const int j0 = S.lay.start[g], j1 = j0 + S.lay.size[g];
-        double s2 = 0.0;
-        for (int j = j0; j < j1; ++j) {
-          const double v = __half2float(S.x[r][S.perm[j]]);
-          s2 += v * v;
-        }
+        const int j0 = S.lay.start[g];
+        const double s2 = sum_squares(j0, j0 + S.lay.size[g],
+                                      [&](int j) { return static_cast<double>(__half2float(S.x[r][S.perm[j]])); });
         const double nr = sqrt(s2);
         nh16 = __double2half(nr);
         f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;
@@ -593,17 +649,20 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
     }
     __syncthreads();  // fac, nrm and the unpacked codes are in place
     if (rows_touched) {
+      const int ra = 16 * mt + g8, rb = ra + 8;
+      const bool oka = ra >= tr0 && ra < tr1, okb = rb >= tr0 && rb < tr1;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int r = 16 * mt + g8 + 8 * (e >> 1);
+          const int col = 2 * nt + (e & 1);
+          const uint32_t info = (colinfo[col >> 2] >> (8 * (col & 3))) & 0xFFu;
+          const bool row_ok = (e >> 1) ? okb : oka;
+          if (!row_ok || info == 0xFFu) continue;
+          const int g = info & 3, w = info >> 2;
+          const float fac = S.fac[(e >> 1) ? rb : ra][g];
           const int i = 64 * nh + 8 * nt + 2 * t4 + (e & 1);
-          const int g = S.gof[i];
-          if (r < tr0 || r >= tr1 || g < 0) continue;
-          const int w = S.lay.width[g];
-          const float u = acc[nt][e] * S.fac[r][g];
-          S.codes[r][i] = static_cast<uint8_t>(lloyd_code(S.thr[w], w, u));
+          S.codes[(e >> 1) ? rb : ra][i] = static_cast<uint8_t>(code16(S.thr16[w], w, acc[nt][e] * fac));
         }
       }
     }
@@ -787,21 +846,35 @@ __device__ __forceinline__ void append_body(const Shape& sh, const Workspace& ws
   if (tid < kD) xs[tid] = xv;
   __syncthreads();
   const int ng = lay.n_groups;
-  // The group norms (fp64, coordinate order) and y = R x (fp32, coordinate
-  // order) are independent: with 256 threads the norms run on threads
-  // 128.. beside the rotation on threads 0..127; with 128, first.
+  // The group norms (fp64) and y = R x are independent: a thread per group
+  // sums the squares, on threads 128.. beside the rotation with 256 threads,
+  // else first.  Rows as they come: in the tile encode's eight-chain order,
+  // with the tensor cores rotating (below).  Rows turned here by RoPE: in
+  // coordinate order, as the fp32 tile encode does.
   const int i = tid;
-  const int norm_tid = tid - (NT >= 2 * kD ? kD : 0);
-  if (norm_tid >= 0 && norm_tid < ng) {
-    const int j0 = lay.start[norm_tid], j1 = j0 + lay.size[norm_tid];
-    double s2 = 0.0;
-    for (int j = j0; j < j1; ++j) {
-      const double v = xs[j];
-      s2 += v * v;
+  if constexpr (!TURN) {
+    // a thread per group, in the tile encode's order (threads 128.. with 256)
+    const int norm_tid = tid - (NT >= 2 * kD ? kD : 0);
+    if (norm_tid >= 0 && norm_tid < ng) {
+      const int j0 = lay.start[norm_tid];
+      const double s2 = sum_squares(j0, j0 + lay.size[norm_tid], [&](int j) { return static_cast<double>(xs[j]); });
+      const double nr = sqrt(s2);
+      nrm[norm_tid] = __double2half(nr);
+      fac[norm_tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[norm_tid])) / nr) : 0.f;
     }
-    const double nr = sqrt(s2);
-    nrm[norm_tid] = __double2half(nr);
-    fac[norm_tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[norm_tid])) / nr) : 0.f;
+  } else {
+    const int norm_tid = tid - (NT >= 2 * kD ? kD : 0);
+    if (norm_tid >= 0 && norm_tid < ng) {
+      const int j0 = lay.start[norm_tid], j1 = j0 + lay.size[norm_tid];
+      double s2 = 0.0;
+      for (int j = j0; j < j1; ++j) {
+        const double v = xs[j];
+        s2 += v * v;
+      }
+      const double nr = sqrt(s2);
+      nrm[norm_tid] = __double2half(nr);
+      fac[norm_tid] = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(lay.size[norm_tid])) / nr) : 0.f;
+    }
   }
   int g = 0;
   float y = 0.f;

@@ -611,19 +611,45 @@ def measure(w, args, dev, world, rank, full):
     digest = kernel_digest()
     cap_rec = NCU_TRAFFIC.get(w.name)
     traffic = cap_rec["bytes_per_launch"] if cap_rec and cap_rec.get("kernel_digest") == digest else None
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": traffic,
-                "traffic_source": (f"ncu capture of {cap_rec['captured']} ({cap_rec['case']}), same kernel sources"
-                                   if traffic is not None else "no ncu capture of the current kernel sources"),
-                "kernel": "decode_fused_kernel" if fused else "decode_mma_kernel + combine_kernel",
-                "launch_ms": launch_ms, "launch_ms_isolated": launch_ms_isolated,
-                "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind, "kernel_digest": digest,
-                "timing": "launch_ms: the step's per-layer decode launches back to back in a captured graph, "
-                          "events around the region / launches; launch_ms_isolated: events around each launch "
-                          "inside a captured step (start-up not overlapped)"}
+    traffic_source = (f"ncu capture of {cap_rec['captured']} ({cap_rec['case']}), same kernel sources"
+                      if traffic is not None else "no ncu capture of the current kernel sources")
+    decode_call = {"launch_ms": launch_ms, "launch_ms_isolated": launch_ms_isolated, "achieved_gbs": achieved,
+                   "frac": achieved / peak,
+                   "kernels": "decode_fused_kernel" if fused else "rotate_query_kernel + decode_mma_kernel + combine_kernel",
+                   "timing": "launch_ms: the step's per-layer bgtq_decode_attn calls back to back in a captured "
+                             "graph, events around the region / calls; launch_ms_isolated: events around each call "
+                             "inside a captured step (start-up not overlapped)"}
+    if fused:
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": traffic, "traffic_source": traffic_source, "kernel": "decode_fused_kernel",
+                    "launch_ms": launch_ms, "alg_bytes_per_launch": alg_bytes, "peak_kind": peak_kind,
+                    "kernel_digest": digest, "timing": decode_call["timing"]}
+    else:
+        # the dominant kernel alone: the split pass's per-layer launches
+        # (bgtq_decode_split on the step's rotated queries) back to back
+        qrot_all = torch.empty((L, B, HQ, 128), dtype=torch.float32, device=dev)
+        for l in range(L):
+            kv.rotate_query(l, q_all[l:l + 1], qrot_all[l:l + 1])
+
+        def splits_back_to_back():
+            for l in range(L):
+                kv.decode_split(l, qrot_all[l:l + 1], seq)
+
+        ms_sp, g_sp, _ = time_graph(splits_back_to_back, steps, warmup, world)
+        del g_sp, qrot_all
+        sp_ms = max_over_ranks(ms_sp / L, world, dev)
+        sp_bytes = alg_bytes - B * HQ * 512  # the packed cache only (q and o are the other kernels')
+        sp_gbs = sp_bytes / (sp_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": sp_gbs, "peak": peak, "unit": "GB/s", "frac": sp_gbs / peak,
+                    "traffic": traffic, "traffic_source": traffic_source, "kernel": "decode_mma_kernel",
+                    "launch_ms": sp_ms, "alg_bytes_per_launch": sp_bytes, "peak_kind": peak_kind,
+                    "kernel_digest": digest,
+                    "timing": "launch_ms: the split pass's per-layer launches (bgtq_decode_split) back to back "
+                              "in a captured graph, events around the region / launches"}
     step_bytes = sum(bytes_per_layer)
     res = {"ms_per_step": ms_step, "tokens_per_s": world * B / (ms_step * 1e-3),
-           "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9, "roofline": roofline, "clocks": clocks,
+           "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9, "roofline": roofline, "decode_call": decode_call,
+           "clocks": clocks,
            "decode_path": "fused (one launch per decode call)" if fused else "query rotation + split + combine",
            "decode_wave_ctas": kv.decode_wave_ctas(),
            "gpu_launches": (2 if fused else 3) * L * steps,
@@ -706,24 +732,6 @@ def measure(w, args, dev, world, rank, full):
         res["buffered"] = {"ms_per_step": ms_buf, "tokens_per_s": world * B / (ms_buf * 1e-3), "sink": SINK,
                            "window": WINDOW, "note": "fp16 sink + recent window next to the packed cache "
                                                      "(query rotation, split pass with buffer CTAs, combine)"}
-
-        # ---- the split pass alone (the three-launch path's dominant kernel) ----
-        qrot_all = torch.empty((L, B, HQ, 128), dtype=torch.float32, device=dev)
-        for l in range(L):
-            kv.rotate_query(l, q_all[l:l + 1], qrot_all[l:l + 1])
-
-        def splits_back_to_back():
-            for l in range(L):
-                kv.decode_split(l, qrot_all[l:l + 1], seq)
-
-        ms_sp, g_sp, _ = time_graph(splits_back_to_back, steps, warmup, world)
-        del g_sp
-        sp_ms = max_over_ranks(ms_sp / L, world, dev)
-        sp_bytes = alg_bytes - B * HQ * 512
-        res["split_pass"] = {"launch_ms": sp_ms, "achieved_gbs": sp_bytes / (sp_ms * 1e-3) / 1e9,
-                             "frac": sp_bytes / (sp_ms * 1e-3) / 1e9 / peak,
-                             "note": "decode_mma_kernel (buffered and stage calls), per-layer launches back to back"}
-        del qrot_all
 
         # ---- the same step over a paged copy of the cache ----
         if not args.no_paged:
@@ -884,8 +892,9 @@ def main():
         "data": "synthetic", "config": workload_config(w, lens),
     }
     for k in ("step_hbm_gbs", "roofline", "e2e", "gpu_launches", "clocks", "decode_path", "decode_wave_ctas", "buffered",
-              "multi_layer", "split_pass", "fp16_baseline", "logit_mae", "paged", "cpu_baseline", "allocate_ms",
-              "prefill_encode_rows_per_s", "prefill_encode_call_rows", "prefill_encode_rope_rows_per_s",
+              "multi_layer", "decode_call", "fp16_baseline", "logit_mae", "paged", "cpu_baseline", "allocate_ms",
+              "prefill_encode_rows_per_s", "prefill_encode_call_rows", "prefill_encode_call_ms",
+              "prefill_encode_rope_rows_per_s",
               "compression_vs_fp16"):
         if k in r:
             line[k] = r[k]

@@ -604,16 +604,38 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
       *reinterpret_cast<uint4*>(&S.x[r][8 * c8]) = raw;
     }
     __syncthreads();
-    // norms: fp64 sums of squares of the exact fp16 inputs of each group, a
-    // thread per (row, group)
+    // norms: fp64 sums of squares of the exact fp16 inputs of each group in
+    // sum_squares' order.  K: a thread per (row, group).  V (one group of
+    // 128): the row's four threads q take chains 2q and 2q + 1 each and meet
+    // in the same tree through two shuffles.
     {
       const int r = tid >> 2, g = tid & 3;
+      const bool row_in = r >= tr0 && r < tr1;
+      double s2 = 0.0;
+      bool mine = false;
+      if (kind == 0) {
+        mine = g < ng && row_in;
+        if (mine) {
+          const int j0 = S.lay.start[g];
+          s2 = sum_squares(j0, j0 + S.lay.size[g],
+                           [&](int j) { return static_cast<double>(__half2float(S.x[r][S.perm[j]])); });
+        }
+      } else {
+        double c0 = 0.0, c1 = 0.0;
+#pragma unroll 4
+        for (int j = 2 * g; j < kD; j += 8) {
+          const double v0 = __half2float(S.x[r][j]), v1 = __half2float(S.x[r][j + 1]);
+          c0 = fma(v0, v0, c0);
+          c1 = fma(v1, v1, c1);
+        }
+        double p = c0 + c1;                         // s_2q + s_2q+1
+        p += __shfl_xor_sync(0xffffffffu, p, 1);    // (s0 + s1) + (s2 + s3), or the upper four
+        s2 = p + __shfl_xor_sync(0xffffffffu, p, 2);
+        mine = g == 0 && row_in;
+      }
       float f = 0.f;
       __half nh16 = __float2half(0.f);
-      if (g < ng && r >= tr0 && r < tr1) {
-        const int j0 = S.lay.start[g];
-        const double s2 = sum_squares(j0, j0 + S.lay.size[g],
-                                      [&](int j) { return static_cast<double>(__half2float(S.x[r][S.perm[j]])); });
+      if (mine) {
         const double nr = sqrt(s2);
         nh16 = __double2half(nr);
         f = nr > 0.0 ? static_cast<float>(sqrt(static_cast<double>(S.lay.size[g])) / nr) : 0.f;

@@ -1025,11 +1025,24 @@ __device__ __forceinline__ void rotate_body(const Shape& sh, const Workspace& ws
   const int kvh = hq / sh.group;
   const LayoutDev& lay = ws.layouts[layer * sh.n_kv_heads + kvh];
   const int tid = threadIdx.x, i = tid & (kD - 1), half = tid >> 7;
-  // this thread's half column of the (block-diagonal) rotation, all loads in flight at once
+  // this thread's half column of the (block-diagonal) rotation, all loads in
+  // flight at once; only the inputs of output i's group are loaded (the
+  // column's other entries are zero)
   const float* mt = ws.mkt + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
   float m[64];
+  int jlo = 0, jhi = 0;
+  if (i < lay.n_positions) {
+    int g = 0;
+    for (int t = 1; t < lay.n_groups; ++t)
+      if (i >= lay.start[t]) g = t;
+    jlo = lay.start[g];
+    jhi = jlo + lay.size[g];
+  }
 #pragma unroll
-  for (int u = 0; u < 64; ++u) m[u] = __ldg(mt + (half * 64 + u) * kD + i);
+  for (int u = 0; u < 64; ++u) {
+    const int j = half * 64 + u;
+    m[u] = j >= jlo && j < jhi ? __ldg(mt + j * kD + i) : 0.f;
+  }
   __shared__ float qp[kD];
   __shared__ float part[kD];
   const size_t row = (static_cast<size_t>(li) * batch + b) * sh.n_q_heads + hq;

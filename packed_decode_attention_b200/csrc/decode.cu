@@ -1359,10 +1359,14 @@ constexpr int kEarlyRotationRows = 256;
 static_assert(kCombWarps * 4 <= kD, "a warp's lanes cover the 128 coordinates four at a time");
 static_assert(kCombSlices <= 8, "a row's slices form one portable cluster");
 
+// EARLY: CTA 0 holds its rotation column in registers, loaded before the
+// dependency wait (small launches); otherwise it reads the column inside the
+// product, so that the kernel needs fewer registers and more clusters fit
+// an SM at once (large launches).
+template <bool EARLY>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
-                                                               SplitPlan plan, BufferArgs buf, __half* __restrict__ out,
-                                                               bool early_rotation) {
+                                                               SplitPlan plan, BufferArgs buf, __half* __restrict__ out) {
   const int has_buf = buf.k != nullptr ? 1 : 0;
   const int slice = blockIdx.x % kCombSlices;  // the CTA's rank in its cluster
   const int rowi = blockIdx.x / kCombSlices;
@@ -1377,10 +1381,12 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   // used by the row's CTA 0.  For a small launch it is read before the
   // split pass has finished, off the critical path.
   const float* mv = ws.mv + static_cast<size_t>(layer * sh.n_kv_heads + kvh) * kD * kD;
-  float mvr[64];
-  if (early_rotation && slice == 0) {
+  float mvr[EARLY ? 64 : 1];
+  if constexpr (EARLY) {
+    if (slice == 0) {
 #pragma unroll
-    for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+      for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
+    }
   }
   // the next kernel of the stream may start its own table-only set-up now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -1482,6 +1488,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
       lk[k] = dsmem_ld(dsmem_addr(&cmid[1], k));
       ak[k] = dsmem_ld(dsmem_addr(&cmid[4 + dd], k));
     }
+    // the other CTAs may leave once CTA 0 has read their shared memory
+    cluster_sync_all();
     if (has_buf) {
       const float* bm = ws.comb_mid + (wrow * (kCombSlices + 1) + kCombSlices) * kPartialStride;
       mk[kCombSlices] = __ldcg(bm);
@@ -1504,21 +1512,21 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
       else ab = w * ak[k];                            // the buffer's rows, unrotated
     }
     if (tid < kD) a_s[tid] = at / Lt;
-    if (!early_rotation) {
-#pragma unroll
-      for (int r = 0; r < 64; ++r) mvr[r] = __ldg(mv + (half * 64 + r) * kD + dd);
-    }
     __syncthreads();
     // inverse V rotation: two threads per output, half of the inputs each
     float o = 0.f;
 #pragma unroll
-    for (int r = 0; r < 64; ++r) o = fmaf(mvr[r], a_s[half * 64 + r], o);
+    for (int r = 0; r < 64; ++r) {
+      const float m = EARLY ? mvr[r] : __ldg(mv + (half * 64 + r) * kD + dd);
+      o = fmaf(m, a_s[half * 64 + r], o);
+    }
     if (half == 1) accs[0][dd] = o;
     __syncthreads();
     if (half == 0) out[row * kD + dd] = __float2half(o + accs[0][dd] + ab / Lt);
+  } else {
+    // keep this CTA's shared memory until CTA 0 has read it
+    cluster_sync_all();
   }
-  // the other CTAs keep their shared memory until CTA 0 has read it
-  cluster_sync_all();
 }
 
 // Warps per CTA of the split pass (several CTAs per SM: a CTA that finishes
@@ -1683,8 +1691,9 @@ cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int 
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, s, ws, layer0, seq_lens, batch, plan, buf, out,
-                            rows <= kEarlyRotationRows);
+  return rows <= kEarlyRotationRows
+             ? cudaLaunchKernelEx(&cfg, combine_kernel<true>, s, ws, layer0, seq_lens, batch, plan, buf, out)
+             : cudaLaunchKernelEx(&cfg, combine_kernel<false>, s, ws, layer0, seq_lens, batch, plan, buf, out);
 }
 
 }  // namespace bgtq

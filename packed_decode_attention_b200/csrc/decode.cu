@@ -1341,9 +1341,9 @@ __global__ void __launch_bounds__(kDecThreads, kDecMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// Combine the splits and rotate back.  Grid (layer_count*batch*Hq *
-// kCombSlices), 256 threads, in clusters of kCombSlices CTAs: one cluster
-// per row.  CTA (slice) r merges slice r of the row's splits (w_s = 2^(m_s -
+// Combine the splits and rotate back.  Grid (layer_count*batch*Hq * S),
+// 256 threads, in clusters of S = kCombSlices CTAs (1 when every unit has
+// few splits): one cluster per row.  CTA (slice) r merges slice r of the row's splits (w_s = 2^(m_s -
 // M), 0 for empty splits; lane = 4 rotated coordinates) into an
 // intermediate (m, l, acc) in V's rotated basis in its shared memory.  CTA 0
 // then reads the cluster's intermediates through distributed shared memory
@@ -1363,13 +1363,15 @@ static_assert(kCombSlices <= 8, "a row's slices form one portable cluster");
 // dependency wait (small launches); otherwise it reads the column inside the
 // product, so that the kernel needs fewer registers and more clusters fit
 // an SM at once (large launches).
-template <bool EARLY>
+// S: CTAs (slices) per row, the cluster size: kCombSlices, or 1 when no
+// unit has more splits than one CTA merges in one round of loads.
+template <bool EARLY, int S>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspace ws, int layer0,
                                                                const int32_t* __restrict__ seq_lens, int batch,
                                                                SplitPlan plan, BufferArgs buf, __half* __restrict__ out) {
   const int has_buf = buf.k != nullptr ? 1 : 0;
-  const int slice = blockIdx.x % kCombSlices;  // the CTA's rank in its cluster
-  const int rowi = blockIdx.x / kCombSlices;
+  const int slice = blockIdx.x % S;  // the CTA's rank in its cluster
+  const int rowi = blockIdx.x / S;
   const int hq = rowi % sh.n_q_heads;
   const int b = (rowi / sh.n_q_heads) % batch;
   const int li = rowi / (sh.n_q_heads * batch);
@@ -1413,8 +1415,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   // ---- one slice of the row's splits: warp w takes splits s0 + w + 8 j,
   // four at a time with all their loads in flight, merged online per warp
   // (lane = 4 rotated coordinates), then across the warps ----
-  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / kCombSlices);
-  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / kCombSlices);
+  const int s0 = static_cast<int>((static_cast<int64_t>(slice) * n_splits) / S);
+  const int s1 = static_cast<int>((static_cast<int64_t>(slice + 1) * n_splits) / S);
   float m_w = -CUDART_INF_F, l_w = 0.f;
   float4 a_w = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int base = s0 + warp; base < s1; base += 4 * kCombWarps) {
@@ -1481,9 +1483,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
   cluster_sync_all();
   if (slice == 0) {
     // ---- CTA 0 merges the cluster's intermediates (and the buffer's) ----
-    float mk[kCombSlices + 1], lk[kCombSlices + 1], ak[kCombSlices + 1];
+    float mk[S + 1], lk[S + 1], ak[S + 1];
 #pragma unroll
-    for (int k = 0; k < kCombSlices; ++k) {
+    for (int k = 0; k < S; ++k) {
       mk[k] = dsmem_ld(dsmem_addr(&cmid[0], k));
       lk[k] = dsmem_ld(dsmem_addr(&cmid[1], k));
       ak[k] = dsmem_ld(dsmem_addr(&cmid[4 + dd], k));
@@ -1492,23 +1494,23 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(Shape sh, Workspa
     cluster_sync_all();
     if (has_buf) {
       const float* bm = ws.comb_mid + (wrow * (kCombSlices + 1) + kCombSlices) * kPartialStride;
-      mk[kCombSlices] = __ldcg(bm);
-      lk[kCombSlices] = __ldcg(bm + 1);
-      ak[kCombSlices] = __ldcg(bm + 4 + dd);
+      mk[S] = __ldcg(bm);
+      lk[S] = __ldcg(bm + 1);
+      ak[S] = __ldcg(bm + 4 + dd);
     } else {
-      mk[kCombSlices] = -CUDART_INF_F;
-      lk[kCombSlices] = 0.f;
-      ak[kCombSlices] = 0.f;
+      mk[S] = -CUDART_INF_F;
+      lk[S] = 0.f;
+      ak[S] = 0.f;
     }
     float Mt = -CUDART_INF_F;
 #pragma unroll
-    for (int k = 0; k <= kCombSlices; ++k) Mt = fmaxf(Mt, mk[k]);
+    for (int k = 0; k <= S; ++k) Mt = fmaxf(Mt, mk[k]);
     float Lt = 0.f, at = 0.f, ab = 0.f;
 #pragma unroll
-    for (int k = 0; k <= kCombSlices; ++k) {
+    for (int k = 0; k <= S; ++k) {
       const float w = mk[k] == -CUDART_INF_F ? 0.f : exp2f(mk[k] - Mt);
       Lt = fmaf(w, lk[k], Lt);
-      if (k < kCombSlices) at = fmaf(w, ak[k], at);  // rotated basis
+      if (k < S) at = fmaf(w, ak[k], at);  // rotated basis
       else ab = w * ak[k];                            // the buffer's rows, unrotated
     }
     if (tid < kD) a_s[tid] = at / Lt;
@@ -1677,8 +1679,11 @@ cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int 
                            const int32_t* seq_lens, int batch, const SplitPlan& plan, const BufferArgs& buf,
                            __half* out, cudaStream_t stream) {
   const int rows = layer_count * batch * s.n_q_heads;
+  // one CTA per row when no unit has more splits than its 8 warps load in
+  // one round (4 each); else a cluster of kCombSlices slices per row
+  const int S = plan.c_max <= 4 * (kCombThreads / 32) ? 1 : kCombSlices;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(rows * kCombSlices);
+  cfg.gridDim = dim3(rows * S);
   cfg.blockDim = dim3(kCombThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -1686,14 +1691,19 @@ cudaError_t launch_combine(const Shape& s, const Workspace& ws, int layer0, int 
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   at[1].id = cudaLaunchAttributeClusterDimension;  // a row's slices
-  at[1].val.clusterDim.x = kCombSlices;
+  at[1].val.clusterDim.x = S;
   at[1].val.clusterDim.y = 1;
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return rows <= kEarlyRotationRows
-             ? cudaLaunchKernelEx(&cfg, combine_kernel<true>, s, ws, layer0, seq_lens, batch, plan, buf, out)
-             : cudaLaunchKernelEx(&cfg, combine_kernel<false>, s, ws, layer0, seq_lens, batch, plan, buf, out);
+  const bool early = rows <= kEarlyRotationRows;
+  if (S == 1)
+    return early ? cudaLaunchKernelEx(&cfg, combine_kernel<true, 1>, s, ws, layer0, seq_lens, batch, plan, buf, out)
+                 : cudaLaunchKernelEx(&cfg, combine_kernel<false, 1>, s, ws, layer0, seq_lens, batch, plan, buf, out);
+  return early
+             ? cudaLaunchKernelEx(&cfg, combine_kernel<true, kCombSlices>, s, ws, layer0, seq_lens, batch, plan, buf, out)
+             : cudaLaunchKernelEx(&cfg, combine_kernel<false, kCombSlices>, s, ws, layer0, seq_lens, batch, plan, buf,
+                                  out);
 }
 
 }  // namespace bgtq

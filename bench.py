@@ -53,7 +53,12 @@ SIDE_WORKLOADS = ("tiny", "llama", "batch", "long")
 # capture, per workload, with the date of the capture and a digest of the
 # kernel sources it was taken on.  The roofline reports it only while the
 # sources still match that digest (null otherwise: the kernel has changed).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "qwen3b": {"bytes_per_launch": 27901184, "captured": "2026-12-02",
+               "case": "8 of the 36 layers, the same per-layer split launch; dram__bytes_read.sum 27.90 MB, "
+                       "dram__bytes_write.sum 0",
+               "kernel_digest": "235ce497d49dad9f"},
+}
 KERNEL_SOURCES = ("packed_decode_attention_b200/csrc/decode.cu", "packed_decode_attention_b200/csrc/common.cuh",
                   "packed_decode_attention_b200/csrc/device_tables.h")
 

@@ -41,7 +41,7 @@ namespace {
 // tile's logits and softmax cover its copy).
 constexpr int kStages = 2;
 constexpr int kBarsPerWarp = kStages + 1;
-constexpr int kDecMinBlocks = 4;  // CTAs per SM the register budget is sized for
+constexpr int kDecMinBlocks = 3;  // CTAs per SM the register budget is sized for
 constexpr int kWaitLimit = 1 << 20;  // polls of up to kPollSuspendNs each: about a second
 constexpr float kRescaleSlack = 8.f;
 

@@ -413,9 +413,10 @@ int bgtq_test_drop_tile_copies(bgtq_state* st, int32_t tile);
 
 /* Selects the decode calls' kernels: fused = 1 asks for the fused launch
  * (query rotation, split-K pass, split merge and inverse V rotation in one
- * kernel of 8-CTA clusters), taken where the GPU can co-schedule such a
- * cluster for the config; fused = 0 (the default) runs the query rotation,
- * the split pass and the combine as three launches.  Both compute the same
+ * kernel of 4- or 8-CTA clusters, whichever holds more CTAs at once), taken
+ * where the GPU can co-schedule such a cluster for the config; fused = 0 (the
+ * default) runs the query rotation, the split pass and the combine as three
+ * launches.  Both compute the same
  * attention up to the order of the split merge.  Other values:
  * BGTQ_ERR_INVALID_ARG.  SYNC (host only). */
 int bgtq_set_decode_path(bgtq_state* st, int32_t fused);
@@ -425,12 +426,12 @@ int bgtq_set_decode_path(bgtq_state* st, int32_t fused);
  * holds at once for that kernel).  *h_fused = 1 when
  * bgtq_decode_attn, bgtq_decode_step and bgtq_decode_attn_static_scratch run
  * as one fused launch per call (query rotation, split-K pass, split merge and
- * inverse V rotation in thread-block clusters of 8 CTAs; bgtq_decode_step
+ * inverse V rotation in thread-block clusters of 4 or 8 CTAs; bgtq_decode_step
  * launches the appends before it); 0 when they run the query rotation, the
  * split pass and the combine as three launches (as the buffered and stage
  * calls always do): the fused path was not selected, or this GPU cannot
- * co-schedule its cluster for the config.  Both compute the same attention.  SYNC (host only; the first call
- * may query the GPU's occupancy). */
+ * co-schedule its cluster for the config.  Both compute the same attention.
+ * SYNC (host only; the first call may query the GPU's occupancy). */
 int bgtq_get_decode_path(bgtq_state* st, int32_t* h_fused, int32_t* h_ctas);
 
 /* Synchronises "stream", reads the device error flag into *h_flags

@@ -455,8 +455,8 @@ __device__ __forceinline__ void stage_rotation_operands(const Workspace& ws, int
 // The thresholds of width w spread over 15 ascending entries: the first
 // 2^(4-w) - 1 are -inf, then each threshold appears 2^(4-w) times.  Then
 // c = #{entries <= u} = 2^(4-w) (code + 1) - 1, so a branch-free 4-step
-// search serves every width: code16 returns #{thresholds <= u} (ties go up)
-// as lloyd_code does, and the width-4 sign-magnitude symbol.
+// search serves every width and gives #{thresholds <= u} (ties go up) as
+// lloyd_code does.
 __device__ __forceinline__ void spread_thresholds(const float* thr, float (*thr16)[16], int tid, int nthreads) {
   for (int u = tid; u < 5 * 16; u += nthreads) {
     const int w = u >> 4, k = u & 15;
@@ -467,11 +467,8 @@ __device__ __forceinline__ void spread_thresholds(const float* thr, float (*thr1
   }
 }
 
-__device__ __forceinline__ int code16(const float* t16, int w, float u) {
-  int c = 0;
-#pragma unroll
-  for (int s = 8; s > 0; s >>= 1)
-    if (t16[c + s - 1] <= u) c += s;
+// The code (width-4: its sign-magnitude symbol) from c = #{spread entries <= u}.
+__device__ __forceinline__ int code_of_spread_count(int c, int w) {
   int code = ((c + 1) >> (4 - w)) - 1;
   if (w == 4) code = (code & 8) ? (code ^ 8) : (code ^ 15);
   return code;
@@ -485,7 +482,7 @@ struct EncodeTcSmem {
   __half nrm[kTile][kNumGroupsMax];
   uint8_t codes[kTile][kCodePitch];
   uint32_t words[1024];
-  float thr16[5][16];           // width w's thresholds spread to 15 entries (see code16)
+  float thr16[5][16];           // width w's thresholds spread to 15 entries (see spread_thresholds)
   int32_t perm[kD];            // record position -> dimension
   int32_t gof[kD];             // group of each record position (-1: width 0)
   LayoutDev lay;
@@ -671,20 +668,36 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_tc_kernel(Shape sh, Wor
     }
     __syncthreads();  // fac, nrm and the unpacked codes are in place
     if (rows_touched) {
+      // the codes of 8 outputs at a time, their four search steps in
+      // lockstep (8 independent shared loads per step, no branch per output)
       const int ra = 16 * mt + g8, rb = ra + 8;
       const bool oka = ra >= tr0 && ra < tr1, okb = rb >= tr0 && rb < tr1;
+      const float* thr = &S.thr16[0][0];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt0 = 0; nt0 < 8; nt0 += 2) {
+        float u8[8];
+        int w8[8], c8[8];
+        bool st8[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int q = 0; q < 8; ++q) {
+          const int nt = nt0 + (q >> 2), e = q & 3;
           const int col = 2 * nt + (e & 1);
           const uint32_t info = (colinfo[col >> 2] >> (8 * (col & 3))) & 0xFFu;
-          const bool row_ok = (e >> 1) ? okb : oka;
-          if (!row_ok || info == 0xFFu) continue;
-          const int g = info & 3, w = info >> 2;
-          const float fac = S.fac[(e >> 1) ? rb : ra][g];
-          const int i = 64 * nh + 8 * nt + 2 * t4 + (e & 1);
-          S.codes[(e >> 1) ? rb : ra][i] = static_cast<uint8_t>(code16(S.thr16[w], w, acc[nt][e] * fac));
+          st8[q] = info != 0xFFu && ((e >> 1) ? okb : oka);
+          w8[q] = st8[q] ? static_cast<int>(info >> 2) : 4;  // a position with no code: any width
+          u8[q] = acc[nt][e] * S.fac[(e >> 1) ? rb : ra][info & 3];
+          c8[q] = 0;
+        }
+#pragma unroll
+        for (int step = 8; step > 0; step >>= 1)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) c8[q] += thr[16 * w8[q] + c8[q] + step - 1] <= u8[q] ? step : 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (!st8[q]) continue;
+          const int nt = nt0 + (q >> 2), e = q & 3;
+          S.codes[(e >> 1) ? rb : ra][64 * nh + 8 * nt + 2 * t4 + (e & 1)] =
+              static_cast<uint8_t>(code_of_spread_count(c8[q], w8[q]));
         }
       }
     }

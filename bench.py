@@ -56,8 +56,9 @@ SIDE_WORKLOADS = ("tiny", "llama", "batch", "long")
 NCU_TRAFFIC = {
     "qwen3b": {"bytes_per_launch": 27897344, "captured": "2026-12-02",
                "case": "8 of the 36 layers, the same per-layer split launch; dram__bytes_read.sum 27.90 MB, "
-                       "dram__bytes_write.sum 0",
-               "kernel_digest": "2944aa7cf6d47af1"},
+                       "dram__bytes_write.sum 0; decode.cu's header comments edited since (sources digest "
+                       "2944aa7cf6d47af1 at the capture), no code change",
+               "kernel_digest": "69fdba149f4e04c1"},
 }
 KERNEL_SOURCES = ("packed_decode_attention_b200/csrc/decode.cu", "packed_decode_attention_b200/csrc/common.cuh",
                   "packed_decode_attention_b200/csrc/device_tables.h")

@@ -3,9 +3,12 @@
 //   decode_fused_kernel  query rotation, split-K flash decoding from the packed
 //                        tiles (mma.sync), split merge and inverse V rotation
 //                        in one launch (thread-block clusters)
-//   decode_mma_kernel    the split-K pass alone (caller's q~, stage calls),
-//                        with the fp16 sink / window rows of a buffered call
-//   combine_kernel       log-sum-exp merge of the splits + inverse V rotation
+//   decode_mma_kernel    the split-K pass of the three-launch decode (after
+//                        the query rotation or the decode step's prep) and
+//                        of the stage calls, with the fp16 sink / window rows
+//                        of a buffered call
+//   combine_kernel       log-sum-exp merge of the splits (a cluster of up to
+//                        8 CTAs per row) + inverse V rotation
 //
 // Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (Block-GTQ;
 // chatpaper summary / arXiv 2606.24033 abstract, blockgtq README) on top of
@@ -22,9 +25,9 @@ namespace {
 //
 // Grid (batch * Hkv * head_blocks, c_max, layer_count), 128 threads.  The
 // split CTAs of a (layer, sequence, KV head, block of up to 8 query heads) share
-// its 64-position tiles; each warp has its own 2-stage bulk-copy pipeline
-// (K tile, V tile, norms -> shared memory, completion on an mbarrier) and its
-// own online-softmax state.
+// its 64-position tiles; each warp has its own bulk-copy pipeline (two
+// stages of K tile + norms, one V buffer -> shared memory, completion on
+// mbarriers) and its own online-softmax state.
 //
 // Logits (per warp per tile): S^T[64 tokens x 8 heads] = K_hat q~^T as
 // mma.sync m16n8k16 tiles -- A = centroids C[codes] (exact in fp16), looked

@@ -86,8 +86,11 @@ __global__ void __launch_bounds__(128) energy_kernel(const __half* __restrict__ 
 // threads.  A CTA loads one (layer, KV head, kind)'s rotation and tables once
 // and then takes every per_unit-th 64-position tile that the call writes for
 // one sequence: it unpacks the tile's codes when the call writes only part of
-// it, encodes its new rows (y = R x in fp32, norms in fp64, u = sqrt(d) y /
-// n, code = #{thresholds <= u}) into the codes, and packs the tile again.
+// it, encodes its new rows (y = R x, norms in fp64, u = sqrt(d) y / n, code =
+// #{thresholds <= u}) into the codes, and packs the tile again.
+// encode_kernel<true> does this for K rows turned by RoPE on load, with the
+// rotation in fp32 FMAs; encode_tc_kernel (below) for rows as they come, with
+// the rotation on the tensor cores.
 // ---------------------------------------------------------------------------
 constexpr int kEncThreads = 256;
 
